@@ -1,0 +1,218 @@
+"""ctypes binding of libgdn.so (include/gdn.h).
+
+Argument marshalling only: shapes and dtypes of torch tensors are turned into a
+``gdn_dims`` struct and raw device pointers, and the call is enqueued on the
+current torch CUDA stream.  Every step of the computation runs in the library's
+CUDA kernels.  There is no fallback: if the library is missing the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libgdn.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "gdn.h")
+
+GDN_OK, GDN_ERR_INVALID, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
+    GDN_ERR_DEVICE_INPUT = range(6)
+GDN_BF16, GDN_FP32 = 0, 1
+GDN_DECAY_SCALAR, GDN_DECAY_CHANNEL = 0, 1
+GDN_FLAG_CUDA_CORES = 1
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in
+                ("B", "T", "H", "d_k", "d_v", "n_seqs", "dtype", "decay", "flags")]
+
+
+_lib = None
+
+
+def lib():
+    """Load libgdn.so (built in-tree by ``python -m gated_delta_rule_140_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m gated_delta_rule_140_b200.build` (needs nvcc)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, fp, sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t
+    D = ctypes.POINTER(Dims)
+    L.gdn_chunk_fwd_workspace_size.argtypes = [D]
+    L.gdn_chunk_fwd_workspace_size.restype = sz
+    L.gdn_chunk_fwd.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
+    L.gdn_chunk_fwd.restype = ctypes.c_int
+    L.gdn_recurrent_step.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp]
+    L.gdn_recurrent_step.restype = ctypes.c_int
+    L.gdn_workspace_init.argtypes = [vp, sz, vp]
+    L.gdn_workspace_init.restype = ctypes.c_int
+    L.gdn_workspace_status.argtypes = [vp, vp]
+    L.gdn_workspace_status.restype = ctypes.c_int
+    L.gdn_chunk_fwd_path.argtypes = [D]
+    L.gdn_chunk_fwd_path.restype = ctypes.c_char_p
+    L.gdn_status_string.argtypes = [ctypes.c_int]
+    L.gdn_status_string.restype = ctypes.c_char_p
+    L.gdn_launch_count.argtypes = []
+    L.gdn_launch_count.restype = ctypes.c_uint64
+    _lib = L
+    return L
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/gdn.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(int(status)).decode()
+
+
+def launch_count() -> int:
+    return int(lib().gdn_launch_count())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt):
+    import torch
+    if dt == torch.bfloat16:
+        return GDN_BF16
+    if dt == torch.float32:
+        return GDN_FP32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {dt}")
+
+
+def _check_dev(name, t, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False) -> Dims:
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    return Dims(B, T, H, dk, dv, (len(cu_seqlens) - 1) if cu_seqlens is not None else B,
+                _dtype_code(q.dtype),
+                GDN_DECAY_CHANNEL if log_alpha.dim() == 4 else GDN_DECAY_SCALAR,
+                GDN_FLAG_CUDA_CORES if cuda_cores else 0)
+
+
+def chunk_fwd_path(dims: Dims) -> str:
+    """"tensor_core" or "cuda_core": the prefill kernel gdn_chunk_fwd selects."""
+    r = lib().gdn_chunk_fwd_path(ctypes.byref(dims))
+    if r is None:
+        raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd_path")
+    return r.decode()
+
+
+def workspace_size(dims: Dims) -> int:
+    n = int(lib().gdn_chunk_fwd_workspace_size(ctypes.byref(dims)))
+    if n == 0:
+        raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd_workspace_size")
+    return n
+
+
+class Workspace:
+    """A zeroed device workspace that grows on demand (one per stream)."""
+
+    def __init__(self, device=None):
+        self.buf = None
+        self.device = device
+
+    def get(self, nbytes: int, stream=None):
+        import torch
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+    def status(self, stream=None) -> int:
+        if self.buf is None:
+            return GDN_OK
+        return int(lib().gdn_workspace_status(_ptr(self.buf), _stream(stream)))
+
+
+_default_ws = {}
+
+
+def _workspace_for(device, stream) -> Workspace:
+    key = (str(device), None if stream is None else stream.cuda_stream)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
+              output_final_state=True, o=None, final_state=None, workspace: Workspace = None,
+              cuda_cores=False, stream=None):
+    """Chunkwise prefill (gdn_chunk_fwd).  Returns (o, final_state or None)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_dev(name, t, q.dtype)
+    _check_dev("log_alpha", log_alpha, torch.float32)
+    _check_dev("beta", beta, torch.float32)
+    _check_dev("initial_state", initial_state, torch.float32)
+    _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores)
+    if o is None:
+        o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(dims.n_seqs, dims.H, dims.d_v, dims.d_k, dtype=torch.float32,
+                                  device=q.device)
+    ws = workspace if workspace is not None else _workspace_for(q.device, stream)
+    nbytes = workspace_size(dims)
+    buf = ws.get(nbytes, stream)
+    st = lib().gdn_chunk_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                             _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(o),
+                             _ptr(final_state), _ptr(buf), ctypes.c_size_t(buf.numel()),
+                             _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd")
+    return o, final_state
+
+
+def recurrent_step(q, k, v, log_alpha, beta, state, *, o=None, stream=None):
+    """One decode step (gdn_recurrent_step); ``state`` [N,H,dv,dk] fp32 is updated
+    in place.  q, k [N,H,dk]; v [N,H,dv]; log_alpha [N,H] or [N,H,dk]; beta [N,H].
+    Returns o [N,H,dv]."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_dev(name, t, q.dtype)
+    _check_dev("log_alpha", log_alpha, torch.float32)
+    _check_dev("beta", beta, torch.float32)
+    _check_dev("state", state, torch.float32)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dims = Dims(N, 1, H, dk, dv, N, _dtype_code(q.dtype),
+                GDN_DECAY_CHANNEL if log_alpha.dim() == 3 else GDN_DECAY_SCALAR, 0)
+    if o is None:
+        o = torch.empty(N, H, dv, dtype=q.dtype, device=q.device)
+    st = lib().gdn_recurrent_step(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(o),
+                                  _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_recurrent_step")
+    return o

@@ -1,0 +1,161 @@
+// gdn_api.cu -- the extern "C" entry points of libgdn.so (declared in
+// include/gdn.h): host-side argument validation, workspace bookkeeping and
+// kernel selection.  Every step of the computation runs in the kernels of the
+// other translation units; this file only checks and launches.
+#include <atomic>
+
+#include "gdn_internal.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Host validation of the dims shared by both calls.
+gdn_status check_dims(const gdn_dims *d, bool prefill) {
+    if (!d) return GDN_ERR_INVALID;
+    if (d->B < 0 || d->H <= 0 || d->T < 0) return GDN_ERR_INVALID;
+    if (d->dtype != GDN_BF16 && d->dtype != GDN_FP32) return GDN_ERR_INVALID;
+    if (d->decay != GDN_DECAY_SCALAR && d->decay != GDN_DECAY_CHANNEL) return GDN_ERR_INVALID;
+    if (d->d_k <= 0 || d->d_v <= 0) return GDN_ERR_INVALID;
+    if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
+        return GDN_ERR_UNSUPPORTED;
+    if ((d->flags & ~GDN_FLAG_CUDA_CORES) != 0) return GDN_ERR_INVALID;
+    if (prefill && d->n_seqs < 0) return GDN_ERR_INVALID;
+    // every index the kernels form must fit in 63 bits; keep the token axis sane
+    if ((long long)d->B * d->T * d->H * (d->d_k > d->d_v ? d->d_k : d->d_v) > (1LL << 40))
+        return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+bool use_tensor_cores(const gdn_dims &d) {
+    return !(d.flags & GDN_FLAG_CUDA_CORES) && gdn::chunk_tc_supported(d);
+}
+
+int prefill_seqs(const gdn_dims &d, const int32_t *cu_seqlens) {
+    return cu_seqlens ? d.n_seqs : d.B;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims) {
+    if (check_dims(dims, true) != GDN_OK) return 0;
+    size_t extra = use_tensor_cores(*dims) ? gdn::chunk_tc_scratch_bytes(*dims) : 0;
+    return gdn::kWorkspaceHeader + ((extra + 255) & ~size_t(255));
+}
+
+gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         const float *initial_state, const int32_t *cu_seqlens,
+                         void *o, float *final_state,
+                         void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    gdn_status st = check_dims(dims, true);
+    if (st != GDN_OK) return st;
+    const gdn_dims &d = *dims;
+    if (cu_seqlens) {
+        if (d.B != 1 || d.n_seqs < 1) return GDN_ERR_INVALID;
+    } else if (d.n_seqs != 0 && d.n_seqs != d.B) {
+        return GDN_ERR_INVALID;
+    }
+    const int n_seqs = prefill_seqs(d, cu_seqlens);
+    const bool any_tokens = (long long)d.B * d.T > 0;
+    if (any_tokens && (!q || !k || !v || !log_alpha || !beta || !o)) return GDN_ERR_INVALID;
+    if (!workspace || workspace_bytes < gdn_chunk_fwd_workspace_size(dims)) return GDN_ERR_INVALID;
+    for (const void *p : {q, k, v, (const void *)o, (const void *)initial_state,
+                          (const void *)final_state, (const void *)workspace})
+        if (p && !aligned16(p)) return GDN_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(log_alpha) | reinterpret_cast<uintptr_t>(beta) |
+         reinterpret_cast<uintptr_t>(cu_seqlens)) & 3u)
+        return GDN_ERR_INVALID;
+
+    gdn::PrefillArgs a{};
+    a.q = q; a.k = k; a.v = v;
+    a.log_alpha = log_alpha; a.beta = beta;
+    a.s0 = initial_state; a.cu_seqlens = cu_seqlens;
+    a.o = o; a.s_final = final_state;
+    a.err = reinterpret_cast<uint32_t *>(workspace);
+    a.scratch = reinterpret_cast<char *>(workspace) + gdn::kWorkspaceHeader;
+    a.B = d.B; a.T = d.T; a.H = d.H; a.dk = d.d_k; a.dv = d.d_v; a.n_seqs = n_seqs;
+    a.channel = d.decay == GDN_DECAY_CHANNEL;
+    a.bf16 = d.dtype == GDN_BF16;
+
+    // Nothing to compute and nothing to write: an empty batch is a no-op.
+    if (n_seqs == 0) return GDN_OK;
+    int launches = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = use_tensor_cores(d) ? gdn::launch_chunk_tc(a, s, &launches)
+                                        : gdn::launch_chunk_simt(a, s, &launches);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta,
+                              float *state_inout, void *o, gdn_stream_t stream) {
+    gdn_status st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    const gdn_dims &d = *dims;
+    if (d.B == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state_inout || !o) return GDN_ERR_INVALID;
+    // 16-byte state rows; 8-byte (bf16 x4) or 16-byte (fp32 x4) token vectors
+    if (!aligned16(state_inout)) return GDN_ERR_INVALID;
+    for (const void *p : {q, k, v, (const void *)o})
+        if (reinterpret_cast<uintptr_t>(p) & (d.dtype == GDN_BF16 ? 7u : 15u)) return GDN_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(log_alpha) | reinterpret_cast<uintptr_t>(beta)) & 3u)
+        return GDN_ERR_INVALID;
+    gdn::DecodeArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.state = state_inout; a.o = o;
+    a.N = d.B; a.H = d.H; a.dk = d.d_k; a.dv = d.d_v;
+    a.channel = d.decay == GDN_DECAY_CHANNEL;
+    a.bf16 = d.dtype == GDN_BF16;
+    int launches = 0;
+    cudaError_t e = gdn::launch_decode(a, reinterpret_cast<cudaStream_t>(stream), &launches);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (!workspace || workspace_bytes < gdn::kWorkspaceHeader || !aligned16(workspace))
+        return GDN_ERR_INVALID;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWorkspaceHeader,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_workspace_status(void *workspace, gdn_stream_t stream) {
+    if (!workspace || !aligned16(workspace)) return GDN_ERR_INVALID;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (word == 0) return GDN_OK;
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    return (word & gdn::kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_ERR_DEVICE_INPUT;
+}
+
+const char *gdn_chunk_fwd_path(const gdn_dims *dims) {
+    if (check_dims(dims, true) != GDN_OK) return nullptr;
+    return use_tensor_cores(*dims) ? "tensor_core" : "cuda_core";
+}
+
+const char *gdn_status_string(gdn_status status) {
+    switch (status) {
+        case GDN_OK: return "GDN_OK";
+        case GDN_ERR_INVALID: return "GDN_ERR_INVALID: invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: unsupported shape or dtype";
+        case GDN_ERR_CUDA: return "GDN_ERR_CUDA: CUDA runtime or launch failure";
+        case GDN_ERR_TIMEOUT: return "GDN_ERR_TIMEOUT: a device-side bounded wait expired";
+        case GDN_ERR_DEVICE_INPUT: return "GDN_ERR_DEVICE_INPUT: bad cu_seqlens contents";
+    }
+    return "unknown gdn_status";
+}
+
+uint64_t gdn_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+}  // extern "C"

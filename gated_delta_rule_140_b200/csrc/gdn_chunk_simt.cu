@@ -1,0 +1,243 @@
+// gdn_chunk_simt.cu -- chunkwise gated delta rule prefill on the fp32 CUDA
+// cores.  This is the fp32 path of gdn_chunk_fwd (fp32 inputs need 1e-4
+// agreement, which bf16 tensor-core operands cannot give) and the reference
+// device path the tensor-core kernel is tested against.
+//
+// One CTA per (sequence, head, 32-wide slice of d_v); the state slice
+// S[v0:v0+32, :] stays in shared memory and the CTA walks the sequence's
+// chunks of C = 64 tokens in order (FG2-GDN paper, section 3.6: WY
+// representation + UT transform inside a chunk, inter-chunk state
+// propagation, intra-chunk causal product).  Per chunk, in fp32:
+//   g_r   = sum_{s<=r} log alpha_s                        (per key channel for KDA)
+//   A_rs  = beta_r sum_c k_rc k_sc e^{g_rc - g_sc}, s < r  (strictly lower)
+//   T     = (I + A)^{-1}                                  (forward substitution)
+//   W     = T diag(beta) (K . e^{G}),  U = T diag(beta) V
+//   V'    = U - W S^T
+//   O     = (Q . e^{G}) S^T + (Q K^T . e^{g_r - g_s}, s <= r) V'
+//   S    <- S Diag(e^{g_C}) + V'^T (K . e^{g_C - G})
+// A partial last chunk is padded with zero tokens (k = q = v = beta = log
+// alpha = 0), which leave the state and the valid rows' outputs unchanged.
+#include "gdn_internal.cuh"
+
+namespace gdn {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kDvs = 32;  // d_v slice per CTA
+
+template <int DK, bool CH>
+struct SimtSmem {
+    static constexpr int C = kChunk;
+    static constexpr int LDK = DK + 1;    // odd strides: no bank conflicts
+    static constexpr int LDV = kDvs + 1;
+    static constexpr int LC = C + 1;
+    static constexpr int kK = 0;
+    static constexpr int kQ = kK + C * LDK;
+    static constexpr int kW = kQ + C * LDK;
+    static constexpr int kG = kW + C * LDK;
+    static constexpr int kA = kG + (CH ? C * LDK : C);
+    static constexpr int kT = kA + C * LC;
+    static constexpr int kV = kT + C * LC;
+    static constexpr int kS = kV + C * LDV;
+    static constexpr int kB = kS + kDvs * LDK;
+    static constexpr int kFloats = kB + C;
+    static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+template <int DK, bool CH>
+__global__ void __launch_bounds__(kThreads)
+chunk_simt_kernel(PrefillArgs a) {
+    using L_ = SimtSmem<DK, CH>;
+    constexpr int C = kChunk, LDK = L_::LDK, LDV = L_::LDV, LC = L_::LC;
+    extern __shared__ float sm[];
+    float *K = sm + L_::kK, *Q = sm + L_::kQ, *W = sm + L_::kW, *G = sm + L_::kG;
+    float *A = sm + L_::kA, *Tm = sm + L_::kT, *V = sm + L_::kV, *S = sm + L_::kS;
+    float *bt = sm + L_::kB;
+    const int tid = threadIdx.x;
+
+    const int nslices = a.dv / kDvs;
+    const int item = blockIdx.x;
+    const int slice = item % nslices;
+    const int h = (item / nslices) % a.H;
+    const int n = item / (nslices * a.H);
+    const int v0 = slice * kDvs;
+    const int H = a.H, dv = a.dv;
+
+    long long t_begin, t_end;
+    seq_range(a, n, &t_begin, &t_end);
+
+    // chunk-start state slice
+    const size_t sbase = ((size_t)n * H + h) * dv * DK;
+    for (int idx = tid; idx < kDvs * DK; idx += kThreads) {
+        const int i = idx / DK, c = idx % DK;
+        S[i * LDK + c] = a.s0 ? a.s0[sbase + (size_t)(v0 + i) * DK + c] : 0.f;
+    }
+
+    auto g_at = [&](int r, int c) -> float { return CH ? G[r * LDK + c] : G[r]; };
+
+    for (long long t0 = t_begin; t0 < t_end; t0 += C) {
+        const int L = (t_end - t0) < C ? (int)(t_end - t0) : C;
+        __syncthreads();
+        // ---- load the chunk (fp32), zero-pad rows >= L -------------------
+        for (int idx = tid; idx < C * DK; idx += kThreads) {
+            const int r = idx / DK, c = idx % DK;
+            const long long off = ((t0 + r) * H + h) * (long long)DK + c;
+            const bool ok = r < L;
+            K[r * LDK + c] = ok ? load_elem(a.k, off, a.bf16) : 0.f;
+            Q[r * LDK + c] = ok ? load_elem(a.q, off, a.bf16) : 0.f;
+            if (CH) G[r * LDK + c] = ok ? a.log_alpha[off] : 0.f;
+        }
+        for (int idx = tid; idx < C * kDvs; idx += kThreads) {
+            const int r = idx / kDvs, i = idx % kDvs;
+            V[r * LDV + i] = r < L ? load_elem(a.v, ((t0 + r) * H + h) * (long long)dv + v0 + i,
+                                               a.bf16)
+                                   : 0.f;
+        }
+        for (int r = tid; r < C; r += kThreads) {
+            const bool ok = r < L;
+            bt[r] = ok ? a.beta[(t0 + r) * H + h] : 0.f;
+            if (!CH) G[r] = ok ? a.log_alpha[(t0 + r) * H + h] : 0.f;
+        }
+        __syncthreads();
+        // ---- step 1: cumulative log decay --------------------------------
+        if (CH) {
+            for (int c = tid; c < DK; c += kThreads) {
+                float acc = 0.f;
+                for (int r = 0; r < C; ++r) { acc += G[r * LDK + c]; G[r * LDK + c] = acc; }
+            }
+        } else if (tid == 0) {
+            float acc = 0.f;
+            for (int r = 0; r < C; ++r) { acc += G[r]; G[r] = acc; }
+        }
+        __syncthreads();
+        // ---- step 2: A (strictly lower), T initialised to I ---------------
+        for (int idx = tid; idx < C * C; idx += kThreads) {
+            const int r = idx / C, s = idx % C;
+            float acc = 0.f;
+            if (s < r) {
+                if (CH) {
+                    for (int c = 0; c < DK; ++c)
+                        acc += K[r * LDK + c] * K[s * LDK + c] * expf(g_at(r, c) - g_at(s, c));
+                } else {
+                    for (int c = 0; c < DK; ++c) acc += K[r * LDK + c] * K[s * LDK + c];
+                    acc *= expf(G[r] - G[s]);
+                }
+                acc *= bt[r];
+            }
+            A[r * LC + s] = acc;
+            Tm[r * LC + s] = (r == s) ? 1.f : 0.f;
+        }
+        __syncthreads();
+        // ---- step 3: T = (I + A)^{-1} by forward substitution -------------
+        // T_ij = -sum_{j <= m < i} A_im T_mj  (row i from the rows above it)
+        for (int i = 1; i < C; ++i) {
+            if (tid < i) {
+                const int j = tid;
+                float acc = 0.f;
+                for (int m = j; m < i; ++m) acc += A[i * LC + m] * Tm[m * LC + j];
+                Tm[i * LC + j] = -acc;
+            }
+            __syncthreads();
+        }
+        // ---- step 4: W = T diag(b)(K . e^G), U = T diag(b) V --------------
+        // Column c of W (and i of U) only involves column c (i), so one thread
+        // owns a column and updates it in place from the bottom row up.
+        if (tid < DK) {
+            const int c = tid;
+            for (int s = 0; s < C; ++s) W[s * LDK + c] = bt[s] * K[s * LDK + c] * expf(g_at(s, c));
+            for (int r = C - 1; r >= 0; --r) {
+                float acc = 0.f;
+                for (int s = 0; s <= r; ++s) acc += Tm[r * LC + s] * W[s * LDK + c];
+                W[r * LDK + c] = acc;
+            }
+        } else if (tid < DK + kDvs) {
+            const int i = tid - DK;
+            for (int s = 0; s < C; ++s) V[s * LDV + i] *= bt[s];
+            for (int r = C - 1; r >= 0; --r) {
+                float acc = 0.f;
+                for (int s = 0; s <= r; ++s) acc += Tm[r * LC + s] * V[s * LDV + i];
+                V[r * LDV + i] = acc;
+            }
+        }
+        __syncthreads();
+        // ---- step 5a: V' = U - W S^T (in place in V) ----------------------
+        for (int idx = tid; idx < C * kDvs; idx += kThreads) {
+            const int r = idx / kDvs, i = idx % kDvs;
+            float acc = 0.f;
+            for (int c = 0; c < DK; ++c) acc += W[r * LDK + c] * S[i * LDK + c];
+            V[r * LDV + i] -= acc;
+        }
+        // ---- step 6a: P = causal decayed Q K^T (into A) --------------------
+        for (int idx = tid; idx < C * C; idx += kThreads) {
+            const int r = idx / C, s = idx % C;
+            float acc = 0.f;
+            if (s <= r) {
+                if (CH) {
+                    for (int c = 0; c < DK; ++c)
+                        acc += Q[r * LDK + c] * K[s * LDK + c] * expf(g_at(r, c) - g_at(s, c));
+                } else {
+                    for (int c = 0; c < DK; ++c) acc += Q[r * LDK + c] * K[s * LDK + c];
+                    acc *= expf(G[r] - G[s]);
+                }
+            }
+            A[r * LC + s] = acc;
+        }
+        __syncthreads();
+        // ---- decayed Q and K^ = K . e^{g_C - G} (in place) ----------------
+        for (int idx = tid; idx < C * DK; idx += kThreads) {
+            const int r = idx / DK, c = idx % DK;
+            const float gr = g_at(r, c);
+            Q[r * LDK + c] *= expf(gr);
+            K[r * LDK + c] *= expf(g_at(C - 1, c) - gr);
+        }
+        __syncthreads();
+        // ---- step 6b: O = (Q . e^G) S^T + P V' ----------------------------
+        for (int idx = tid; idx < C * kDvs; idx += kThreads) {
+            const int r = idx / kDvs, i = idx % kDvs;
+            if (r >= L) continue;
+            float acc = 0.f;
+            for (int c = 0; c < DK; ++c) acc += Q[r * LDK + c] * S[i * LDK + c];
+            for (int s = 0; s <= r; ++s) acc += A[r * LC + s] * V[s * LDV + i];
+            store_elem(a.o, ((t0 + r) * H + h) * (long long)dv + v0 + i, acc, a.bf16);
+        }
+        __syncthreads();
+        // ---- step 5b: S <- S Diag(e^{g_C}) + V'^T K^ ----------------------
+        for (int idx = tid; idx < kDvs * DK; idx += kThreads) {
+            const int i = idx / DK, c = idx % DK;
+            float acc = S[i * LDK + c] * expf(g_at(C - 1, c));
+            for (int s = 0; s < C; ++s) acc += V[s * LDV + i] * K[s * LDK + c];
+            S[i * LDK + c] = acc;
+        }
+    }
+    __syncthreads();
+    if (a.s_final) {
+        for (int idx = tid; idx < kDvs * DK; idx += kThreads) {
+            const int i = idx / DK, c = idx % DK;
+            a.s_final[sbase + (size_t)(v0 + i) * DK + c] = S[i * LDK + c];
+        }
+    }
+}
+
+template <int DK, bool CH>
+cudaError_t launch_t(const PrefillArgs &a, cudaStream_t s) {
+    using L_ = SimtSmem<DK, CH>;
+    auto kern = chunk_simt_kernel<DK, CH>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)L_::kBytes);
+    if (e != cudaSuccess) return e;
+    const long long items = (long long)a.n_seqs * a.H * (a.dv / kDvs);
+    if (items == 0) return cudaSuccess;
+    kern<<<(unsigned)items, kThreads, L_::kBytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t s, int *launches) {
+    const long long items = (long long)a.n_seqs * a.H * (a.dv / kDvs);
+    if (items > 0 && launches) ++*launches;
+    if (a.dk == 128) return a.channel ? launch_t<128, true>(a, s) : launch_t<128, false>(a, s);
+    return a.channel ? launch_t<64, true>(a, s) : launch_t<64, false>(a, s);
+}
+
+}  // namespace gdn

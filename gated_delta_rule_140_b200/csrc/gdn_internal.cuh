@@ -1,0 +1,81 @@
+// gdn_internal.cuh -- definitions shared by the kernels of libgdn.so (not part
+// of the public ABI, which is include/gdn.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+constexpr int kChunk = 64;  // chunk size C of the chunkwise form
+
+// Sticky error bits kept in the first word of the workspace.
+enum : uint32_t { kErrBadSeqlens = 1u, kErrTimeout = 2u };
+constexpr size_t kWorkspaceHeader = 256;
+
+// Everything a prefill kernel needs, in device pointers.  Token-major layouts
+// (see gdn.h).  `seq_start` is null for fixed-length rows of T tokens.
+struct PrefillArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    const float *s0;          // [N,H,dv,dk] or null
+    const int32_t *cu_seqlens;  // [N+1] or null
+    void *o;
+    float *s_final;           // [N,H,dv,dk] or null
+    uint32_t *err;            // sticky error word (workspace)
+    void *scratch;            // workspace after the header
+    int B, T, H, dk, dv, n_seqs;
+    int channel;              // 1 = KDA channel-wise decay
+    int bf16;                 // 1 = bf16 q/k/v/o, 0 = fp32
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    float *state;
+    void *o;
+    int N, H, dk, dv;
+    int channel, bf16;
+};
+
+// Host launchers (each returns cudaGetLastError() of its launches).
+cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t s, int *launches);
+size_t chunk_tc_scratch_bytes(const gdn_dims &d);
+bool chunk_tc_supported(const gdn_dims &d);
+
+// Token range of sequence n for fixed rows or packed sequences, validated on
+// the device: a bad range records kErrBadSeqlens and yields an empty range.
+__device__ __forceinline__ void seq_range(const PrefillArgs &a, int n, long long *t0,
+                                          long long *t1) {
+    if (a.cu_seqlens == nullptr) {
+        *t0 = (long long)n * a.T;
+        *t1 = *t0 + a.T;
+        return;
+    }
+    long long s = a.cu_seqlens[n], e = a.cu_seqlens[n + 1];
+    if (s < 0 || e < s || e > (long long)a.T || (n == 0 && s != 0)) {
+        atomicOr(a.err, kErrBadSeqlens);
+        s = e = 0;
+    }
+    *t0 = s;
+    *t1 = e;
+}
+
+__device__ __forceinline__ float load_elem(const void *p, long long i, int bf16) {
+    return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(p)[i])
+                : reinterpret_cast<const float *>(p)[i];
+}
+
+__device__ __forceinline__ void store_elem(void *p, long long i, float x, int bf16) {
+    if (bf16)
+        reinterpret_cast<__nv_bfloat16 *>(p)[i] = __float2bfloat16_rn(x);
+    else
+        reinterpret_cast<float *>(p)[i] = x;
+}
+
+}  // namespace gdn

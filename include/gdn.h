@@ -1,0 +1,148 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) gated delta rule library, libgdn.so.
+ *
+ * The operation (state S in R^{d_v x d_k} per sequence and head, o_t = S_t q_t):
+ *   Gated DeltaNet (scalar decay alpha_t in (0,1), one beta_t for erase and
+ *   write):   S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   KDA (channel-wise decay Diag(alpha_t), alpha_t in R^{d_k}):
+ *             S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ * Sources: "FG2-GDN: Enhancing Long-Context Gated Delta Networks with Doubly
+ * Fine-Grained Control", section 1 (GDN, then KDA's Diag(alpha_t) as a tied
+ * diagonal-plus-rank-1 transition), section 3.6 (the chunkwise WY / UT
+ * algorithm), section 5 (the unified view S_t = A_t S_{t-1} + k_t v_t^T,
+ * o_t = S_t^T q_t, i.e. this map transposed); "Gated Delta Networks: Improving
+ * Mamba2 with Delta Rule", section 3.1 (one beta_t in both terms) and 3.3
+ * (scalar cumulative decay inside a chunk).
+ *
+ * Conventions for every call
+ *   - All tensor pointers are DEVICE pointers to contiguous row-major memory,
+ *     owned by the caller; the library keeps no pointer after a call returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns after launch.  Nothing is allocated.
+ *   - Layouts are token-major: q, k [B, T, H, d_k]; v, o [B, T, H, d_v];
+ *     log_alpha [B, T, H] (scalar decay) or [B, T, H, d_k] (channel decay),
+ *     fp32, natural log of alpha (so <= 0 for a decay); beta [B, T, H] fp32.
+ *     For a packed variable-length batch B = 1, T = total tokens and
+ *     cu_seqlens holds the N+1 int32 sequence offsets.
+ *   - States are fp32 [N, H, d_v, d_k] (row i = output channel i, d_k
+ *     contiguous), N = number of sequences.
+ *   - q, k, v and o share one dtype (gdn_dtype).  No scale is applied to q:
+ *     a caller that wants 1/sqrt(d_k) scales q first.
+ *   - Supported head sizes: d_k, d_v in {64, 128}.
+ *   - Errors: argument errors are detected on the host before any launch and
+ *     return a status without touching the device.  A failed launch returns
+ *     GDN_ERR_CUDA.  Errors only the device can see (inconsistent cu_seqlens
+ *     contents, an expired bounded wait) set a sticky error word in the
+ *     workspace, read and cleared by gdn_workspace_status().  No call traps.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque stream handle; pass a cudaStream_t (the same pointer type). */
+typedef struct CUstream_st *gdn_stream_t;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID = 1,      /* bad argument (null, shape, alignment, size)    */
+    GDN_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d_k = 96)       */
+    GDN_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed           */
+    GDN_ERR_TIMEOUT = 4,      /* a device-side bounded wait expired             */
+    GDN_ERR_DEVICE_INPUT = 5  /* the device found bad cu_seqlens contents       */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
+typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
+
+/* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: the
+ * tensor-core kernel for bf16 with d_k = d_v = 128, the fp32 CUDA-core kernel
+ * otherwise.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel (used by the
+ * tests to compare the two device paths). */
+enum { GDN_FLAG_CUDA_CORES = 1 };
+
+typedef struct {
+    int32_t B;       /* batch (1 for a packed batch)                           */
+    int32_t T;       /* tokens per batch row (total tokens when packed)         */
+    int32_t H;       /* heads                                                   */
+    int32_t d_k;     /* key / query head size                                   */
+    int32_t d_v;     /* value head size                                         */
+    int32_t n_seqs;  /* sequences: B, or len(cu_seqlens) - 1 when packed         */
+    int32_t dtype;   /* gdn_dtype of q, k, v, o                                 */
+    int32_t decay;   /* gdn_decay                                               */
+    int32_t flags;   /* GDN_FLAG_* (0 = default)                                */
+} gdn_dims;
+
+/* Bytes of device workspace gdn_chunk_fwd needs for `dims` (always >= 256).
+ * The first 256 bytes hold the sticky error word; zero the whole workspace
+ * once before its first use (gdn_workspace_init).  Returns 0 for invalid dims. */
+size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims);
+
+/* Chunkwise (WY / UT-transform) prefill, chunk size C = 64
+ * (FG2-GDN section 3.6).  Per sequence and head, over chunks of 64 tokens:
+ * cumulative log decay; the strictly lower beta- and decay-scaled K K^T (A);
+ * T = (I + A)^{-1}; W = T diag(beta)(decayed K), U = T diag(beta) V; the
+ * sequential inter-chunk state pass V' = U - W S^T, S <- decayed S + V'^T K^;
+ * and the output (decayed Q) S^T + (causal decayed Q K^T) V'.
+ *   q, k, v          inputs, layouts above, dtype dims->dtype
+ *   log_alpha, beta  fp32 gates
+ *   initial_state    fp32 [N,H,d_v,d_k], or NULL for zeros
+ *   cu_seqlens       device int32 [N+1] offsets (0, ..., T, non-decreasing),
+ *                    or NULL for B fixed-length rows of T tokens; chunks never
+ *                    cross a sequence boundary
+ *   o                output [B,T,H,d_v], dtype dims->dtype (rounded once,
+ *                    to nearest even, from fp32)
+ *   final_state      fp32 [N,H,d_v,d_k] or NULL; may alias initial_state
+ *   workspace        device scratch of >= gdn_chunk_fwd_workspace_size bytes,
+ *                    16-byte aligned, zeroed before first use; one call at a
+ *                    time may use a given workspace
+ * q, k, v, o and the states must be 16-byte aligned. */
+gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         const float *initial_state, const int32_t *cu_seqlens,
+                         void *o, float *final_state,
+                         void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* One recurrent decode step for N = dims->B sequences (dims->T is ignored,
+ * one token each): for every (sequence, head), with the state updated in place,
+ *   S <- S Diag(alpha) (I - beta k k^T) + beta v k^T   (scalar alpha for GDN)
+ *   o  = S q   (read with the updated state)
+ * The state's constant size is what makes decoding constant-memory (FG2-GDN
+ * abstract and "Inference Challenges"; Gated DeltaNet-2 abstract).
+ *   q, k [N,H,d_k], v [N,H,d_v] (dtype dims->dtype); log_alpha [N,H] or
+ *   [N,H,d_k]; beta [N,H]; state_inout fp32 [N,H,d_v,d_k]; o [N,H,d_v].
+ * No workspace; touches no memory other than these. */
+gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta,
+                              float *state_inout, void *o, gdn_stream_t stream);
+
+/* Zero the workspace header (the sticky error word) on `stream`. */
+gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
+/* Synchronise `stream`, read and clear the workspace's sticky error word.
+ * GDN_OK if no device-side error was recorded since the last read;
+ * GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_INPUT otherwise. */
+gdn_status gdn_workspace_status(void *workspace, gdn_stream_t stream);
+
+/* Name of the prefill kernel gdn_chunk_fwd selects for `dims` (static
+ * storage): "tensor_core" (tcgen05, bf16, d_k = d_v = 128) or "cuda_core"
+ * (fp32 CUDA cores); NULL for invalid dims. */
+const char *gdn_chunk_fwd_path(const gdn_dims *dims);
+
+/* Human-readable name of a status code (static storage). */
+const char *gdn_status_string(gdn_status status);
+
+/* Number of kernels this library has launched in this process (all calls,
+ * all threads); used to count device work in benchmarks. */
+uint64_t gdn_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,138 @@
+"""The C ABI of libgdn.so on the host, without a GPU: the library loads, exports
+every function include/gdn.h declares, and rejects bad arguments with a status
+code before touching the device."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from gated_delta_rule_140_b200 import _native as nat
+from gated_delta_rule_140_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return nat.lib()
+
+
+def test_library_exports_every_declared_symbol(L):
+    names = nat.header_functions()
+    assert {"gdn_chunk_fwd", "gdn_recurrent_step", "gdn_chunk_fwd_workspace_size",
+            "gdn_workspace_status", "gdn_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"libgdn.so does not export {n}"
+    out = subprocess.run(["nm", "-D", "--defined-only", nat.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+
+
+def test_library_links_no_oracle_and_no_torch(L):
+    out = subprocess.run(["ldd", nat.LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in out and "torch" not in out and "libc10" not in out
+    syms = subprocess.run(["nm", "-D", nat.LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle_" not in syms
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert nat.status_string(s).startswith("GDN_")
+    assert "unknown" in nat.status_string(99)
+
+
+def _dims(**kw):
+    d = dict(B=2, T=128, H=4, d_k=128, d_v=128, n_seqs=2, dtype=nat.GDN_BF16,
+             decay=nat.GDN_DECAY_SCALAR, flags=0)
+    d.update(kw)
+    return nat.Dims(*(d[f] for f, _ in nat.Dims._fields_))
+
+
+def test_workspace_size(L):
+    n = L.gdn_chunk_fwd_workspace_size(ctypes.byref(_dims()))
+    assert n >= 256 and n % 256 == 0
+    assert L.gdn_chunk_fwd_workspace_size(ctypes.byref(_dims(d_k=96))) == 0
+    assert L.gdn_chunk_fwd_workspace_size(None) == 0
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
+
+
+def _call_fwd(L, dims, **kw):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, cu=None, o=FAKE, sf=None,
+             ws=FAKE, wsb=1 << 20)
+    p.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    return L.gdn_chunk_fwd(ctypes.byref(dims), v(p["q"]), v(p["k"]), v(p["v"]), v(p["la"]),
+                           v(p["beta"]), v(p["s0"]), v(p["cu"]), v(p["o"]), v(p["sf"]),
+                           v(p["ws"]), ctypes.c_size_t(p["wsb"]), None)
+
+
+@pytest.mark.parametrize("case,kw,dims_kw,expect", [
+    ("null q", dict(q=None), {}, nat.GDN_ERR_INVALID),
+    ("null o", dict(o=None), {}, nat.GDN_ERR_INVALID),
+    ("null workspace", dict(ws=None), {}, nat.GDN_ERR_INVALID),
+    ("workspace too small", dict(wsb=16), {}, nat.GDN_ERR_INVALID),
+    ("misaligned k", dict(k=FAKE + 2), {}, nat.GDN_ERR_INVALID),
+    ("misaligned state", dict(s0=FAKE + 4), {}, nat.GDN_ERR_INVALID),
+    ("misaligned beta", dict(beta=FAKE + 2), {}, nat.GDN_ERR_INVALID),
+    ("d_k = 96", {}, dict(d_k=96), nat.GDN_ERR_UNSUPPORTED),
+    ("d_v = 0", {}, dict(d_v=0), nat.GDN_ERR_INVALID),
+    ("negative T", {}, dict(T=-1), nat.GDN_ERR_INVALID),
+    ("H = 0", {}, dict(H=0), nat.GDN_ERR_INVALID),
+    ("bad dtype", {}, dict(dtype=7), nat.GDN_ERR_INVALID),
+    ("bad decay", {}, dict(decay=3), nat.GDN_ERR_INVALID),
+    ("bad flags", {}, dict(flags=8), nat.GDN_ERR_INVALID),
+    ("n_seqs != B", {}, dict(n_seqs=3), nat.GDN_ERR_INVALID),
+    ("cu_seqlens with B > 1", dict(cu=FAKE), dict(n_seqs=2), nat.GDN_ERR_INVALID),
+    ("cu_seqlens with no sequences", dict(cu=FAKE), dict(B=1, n_seqs=0), nat.GDN_ERR_INVALID),
+])
+def test_chunk_fwd_rejects_bad_arguments(L, case, kw, dims_kw, expect):
+    assert _call_fwd(L, _dims(**dims_kw), **kw) == expect, case
+
+
+def test_null_dims(L):
+    assert L.gdn_chunk_fwd(None, *([None] * 10), ctypes.c_size_t(0), None) == nat.GDN_ERR_INVALID
+    assert L.gdn_recurrent_step(None, *([None] * 8)) == nat.GDN_ERR_INVALID
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=None), nat.GDN_ERR_INVALID),
+    (dict(state=FAKE + 8), nat.GDN_ERR_INVALID),
+    (dict(v=FAKE + 2), nat.GDN_ERR_INVALID),
+    (dict(la=FAKE + 1), nat.GDN_ERR_INVALID),
+])
+def test_recurrent_step_rejects_bad_arguments(L, kw, expect):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, state=FAKE, o=FAKE)
+    p.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    d = _dims(B=8, T=1, n_seqs=8)
+    assert L.gdn_recurrent_step(ctypes.byref(d), v(p["q"]), v(p["k"]), v(p["v"]), v(p["la"]),
+                                v(p["beta"]), v(p["state"]), v(p["o"]), None) == expect
+
+
+def test_empty_batch_is_a_noop_without_device(L):
+    # B = 0: nothing to launch, nothing touched -- succeeds even without a GPU
+    d = _dims(B=0, n_seqs=0)
+    assert _call_fwd(L, d, q=None, k=None, v=None, la=None, beta=None, o=None) == nat.GDN_OK
+    d = _dims(B=0, T=1, n_seqs=0)
+    assert L.gdn_recurrent_step(ctypes.byref(d), *([None] * 8)) == nat.GDN_OK
+
+
+def test_workspace_init_rejects_bad_arguments(L):
+    assert L.gdn_workspace_init(None, 256, None) == nat.GDN_ERR_INVALID
+    assert L.gdn_workspace_init(ctypes.c_void_p(FAKE), 16, None) == nat.GDN_ERR_INVALID
+    assert L.gdn_workspace_status(None, None) == nat.GDN_ERR_INVALID
+
+
+def test_python_api_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(nat, "_lib", None)
+    monkeypatch.setattr(nat, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        nat.lib()
+
+
+def test_build_uses_sm100a_flags():
+    assert "arch=compute_100a,code=sm_100a" in " ".join(B.NVCC_FLAGS)
+    assert os.path.exists(B.LIB)

@@ -1,0 +1,212 @@
+"""GPU parity: gdn_chunk_fwd and gdn_recurrent_step (through the C ABI) against
+the fp64 oracle on the same seeded inputs.
+
+Reduced cases span several 64-token chunks and a ragged tail and are compared
+element by element over every head; the full-size workloads run on the GPU in
+the launch configuration the benchmark times and are compared on sampled
+(sequence, head) chains, which the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_140_b200 import _native as nat
+from gated_delta_rule_140_b200 import chunk_fwd, recurrent_step
+from gated_delta_rule_140_b200.inputs import (WORKLOADS, decode_inputs, prefill_inputs,
+                                              workload_inputs)
+from tests.parity_util import TOL, gpu_head, oracle_heads, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, **kw):
+    d = to_dev(x)
+    o, sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                      d["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    return o, sf
+
+
+def _full_compare(x, o, sf, dtype):
+    ro, rs = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
+                              x["initial_state"], x["cu_seqlens"])
+    to, ts = TOL[dtype]
+    eo, es = rel_err(o, ro), rel_err(sf, rs)
+    assert eo <= to, f"o error {eo:.3g} > {to}"
+    assert es <= ts, f"final-state error {es:.3g} > {ts}"
+    return eo, es
+
+
+# --------------------------------------------------------------------------- #
+# reduced cases, every element                                                #
+# --------------------------------------------------------------------------- #
+def test_tiny_fp32_workload(cuda_ok):
+    """B=1, H=2, T=256, d=64, fp32, chunk 64, zero initial state, seed 0."""
+    x = workload_inputs("gdn_tiny_fp32")
+    o, sf = _run(x)
+    _full_compare(x, o, sf, torch.float32)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("decay", ["scalar", "channel"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("cuda_cores", [False, True])
+def test_reduced_ragged(cuda_ok, dtype, decay, d, cuda_cores):
+    """Several chunks and a ragged tail (T = 3*64 + 37), with an initial state."""
+    x = prefill_inputs(2, 229, 3, d, d, dtype=dtype, decay=decay, seed=21,
+                       alpha_shift=2.0 if decay == "scalar" else 3.0, init_std=0.05)
+    o, sf = _run(x, cuda_cores=cuda_cores)
+    _full_compare(x, o, sf, dtype)
+
+
+@pytest.mark.parametrize("decay", ["scalar", "channel"])
+def test_varlen_with_empty_and_short_sequences(cuda_ok, decay):
+    lens = [0, 1, 63, 64, 65, 200, 0, 130]
+    g = torch.Generator().manual_seed(22)
+    x = prefill_inputs(1, 0, 4, 128, 128, dtype=torch.bfloat16, decay=decay,
+                       alpha_shift=2.0 if decay == "scalar" else 3.0, init_std=0.02,
+                       lengths=lens, gen=g)
+    o, sf = _run(x)
+    _full_compare(x, o, sf, torch.bfloat16)
+    # empty sequences: the final state is the initial state, bit for bit
+    for n, L in enumerate(lens):
+        if L == 0:
+            assert torch.equal(sf[n].cpu(), x["initial_state"][n])
+
+
+def test_final_state_may_alias_initial_state(cuda_ok):
+    x = prefill_inputs(2, 150, 2, 128, 128, dtype=torch.bfloat16, seed=23, init_std=0.05)
+    d = to_dev(x)
+    o_ref, sf_ref = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                              d["initial_state"].clone())
+    s = d["initial_state"].clone()
+    o, sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], s, final_state=s)
+    torch.cuda.synchronize()
+    assert sf.data_ptr() == s.data_ptr()
+    assert torch.equal(o, o_ref) and torch.equal(s, sf_ref)
+
+
+def test_no_final_state_and_deterministic(cuda_ok):
+    x = prefill_inputs(1, 300, 2, 128, 128, dtype=torch.bfloat16, seed=24)
+    d = to_dev(x)
+    o1, sf1 = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                        output_final_state=False)
+    o2, _ = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"])
+    torch.cuda.synchronize()
+    assert sf1 is None
+    assert torch.equal(o1, o2), "two runs differ"
+
+
+def test_segment_chaining_on_device(cuda_ok):
+    """prefill(T1) then prefill(T2, S0 = final) agrees with prefill(T1 + T2)."""
+    x = prefill_inputs(1, 320, 2, 128, 128, dtype=torch.bfloat16, seed=25, init_std=0.02)
+    d = to_dev(x)
+    o, sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"])
+    a, b = slice(0, 128), slice(128, 320)
+    cut = lambda t, s: t[:, s].contiguous()
+    oa, sa = chunk_fwd(*(cut(d[n], a) for n in ("q", "k", "v", "log_alpha", "beta")),
+                       d["initial_state"])
+    ob, sb = chunk_fwd(*(cut(d[n], b) for n in ("q", "k", "v", "log_alpha", "beta")), sa)
+    torch.cuda.synchronize()
+    assert rel_err(torch.cat([oa, ob], 1).float(), o.float().cpu().numpy()) < 1e-2
+    assert rel_err(sb, sf.cpu().numpy()) < 1e-2
+
+
+def test_bad_cu_seqlens_reported_by_workspace_status(cuda_ok):
+    x = prefill_inputs(1, 256, 2, 128, 128, dtype=torch.bfloat16, seed=26)
+    d = to_dev(x)
+    cu = torch.tensor([0, 200, 100, 256], dtype=torch.int32, device="cuda")  # not monotone
+    ws = nat.Workspace()
+    chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, cu, workspace=ws)
+    assert ws.status() == nat.GDN_ERR_DEVICE_INPUT
+    assert ws.status() == nat.GDN_OK  # the word is cleared by the read
+    cu = torch.tensor([0, 100, 200, 256], dtype=torch.int32, device="cuda")
+    chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, cu, workspace=ws)
+    assert ws.status() == nat.GDN_OK
+
+
+def test_tensor_core_and_cuda_core_paths_agree(cuda_ok):
+    x = prefill_inputs(2, 512, 4, 128, 128, dtype=torch.bfloat16, seed=27, init_std=0.02)
+    o1, s1 = _run(x)
+    o2, s2 = _run(x, cuda_cores=True)
+    assert rel_err(o1, o2.float().cpu().numpy()) < 2e-2
+    assert rel_err(s1, s2.cpu().numpy()) < 1e-2
+
+
+# --------------------------------------------------------------------------- #
+# full-size workloads, sampled chains                                         #
+# --------------------------------------------------------------------------- #
+FULL = {
+    "gdn_prefill_bf16": [(0, 0), (3, 15), (1, 7)],
+    "gdn_varlen_bf16": [(0, 0), (31, 15), (17, 5)],
+    "kda_prefill_bf16": [(0, 0), (1, 31)],
+    "gdn_long_prefill_bf16": [(0, 0), (0, 31)],
+}
+
+
+@pytest.mark.parametrize("name", list(FULL))
+def test_full_workload_sampled(cuda_ok, name):
+    x = workload_inputs(name)
+    o, sf = _run(x)
+    assert torch.isfinite(o).all() and torch.isfinite(sf).all()
+    to, ts = TOL[WORKLOADS[name].dtype]
+    for n, h, ro, rs in oracle_heads(x, FULL[name]):
+        go, gs = gpu_head(x, o, sf, n, h)
+        eo, es = rel_err(go, ro), rel_err(gs, rs)
+        assert eo <= to, f"{name} (n={n}, h={h}) o error {eo:.3g}"
+        assert es <= ts, f"{name} (n={n}, h={h}) final-state error {es:.3g}"
+
+
+# --------------------------------------------------------------------------- #
+# decode                                                                      #
+# --------------------------------------------------------------------------- #
+def _decode_check(x, picks, dtype):
+    steps = x["q"].shape[0]
+    d = to_dev(x)
+    state = d["state"].clone()
+    outs = []
+    for t in range(steps):
+        outs.append(recurrent_step(d["q"][t], d["k"][t], d["v"][t], d["log_alpha"][t],
+                                   d["beta"][t], state))
+    torch.cuda.synchronize()
+    o = torch.stack(outs)  # [S,N,H,dv]
+    to, ts = TOL[dtype]
+    for n, h in picks:
+        # the oracle sees the same tokens as one sequence of `steps` tokens
+        seq = lambda t: t[:, n:n + 1, h:h + 1].transpose(0, 1)  # [1,S,1,...]
+        ro, rs = oracle.recurrent(seq(x["q"]), seq(x["k"]), seq(x["v"]),
+                                  seq(x["log_alpha"]), seq(x["beta"]),
+                                  x["state"][n:n + 1, h:h + 1])
+        assert rel_err(o[:, n, h], ro[0, :, 0]) <= to
+        assert rel_err(state[n, h], rs[0, 0]) <= ts
+
+
+@pytest.mark.parametrize("decay", ["scalar", "channel"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_reduced(cuda_ok, decay, d, dtype):
+    x = decode_inputs(5, 3, d, d, 20, dtype=dtype, decay=decay, seed=31,
+                      alpha_shift=2.0 if decay == "scalar" else 3.0)
+    _decode_check(x, [(n, h) for n in range(5) for h in range(3)], dtype)
+
+
+def test_decode_full_workload_sampled(cuda_ok):
+    """N=256, H=32, d=128, fp32 state in place, 64 steps."""
+    x = workload_inputs("gdn_decode")
+    _decode_check(x, [(0, 0), (255, 31), (100, 17)], torch.bfloat16)
+
+
+def test_decode_matches_prefill(cuda_ok):
+    """64 decode steps from S0 equal one 64-token prefill from S0 (same tokens)."""
+    x = decode_inputs(4, 2, 128, 128, 64, seed=32)
+    d = to_dev(x)
+    state = d["state"].clone()
+    outs = [recurrent_step(d["q"][t], d["k"][t], d["v"][t], d["log_alpha"][t], d["beta"][t],
+                           state) for t in range(64)]
+    seq = lambda t: t.transpose(0, 1).contiguous()  # [N,64,H,...]
+    o, sf = chunk_fwd(seq(d["q"]), seq(d["k"]), seq(d["v"]), seq(d["log_alpha"]),
+                      seq(d["beta"]), d["state"])
+    torch.cuda.synchronize()
+    assert rel_err(torch.stack(outs).transpose(0, 1), o.float().cpu().numpy()) < 2e-2
+    assert rel_err(state, sf.cpu().numpy()) < 1e-2
