@@ -51,6 +51,8 @@ def lib():
     L.gdn_chunk_fwd_workspace_size.restype = sz
     L.gdn_chunk_fwd.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
     L.gdn_chunk_fwd.restype = ctypes.c_int
+    L.gdn_chunk_fwd_noalloc.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, fp, vp]
+    L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
     L.gdn_recurrent_step.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp]
     L.gdn_recurrent_step.restype = ctypes.c_int
     L.gdn_workspace_init.argtypes = [vp, sz, vp]

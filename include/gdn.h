@@ -121,6 +121,40 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
                               const float *log_alpha, const float *beta,
                               float *state_inout, void *o, gdn_stream_t stream);
 
+/* Size of the device array that gdn_chunk_fwd_noalloc uses in place of a
+ * caller workspace: 256 KiB, held by every GPU that loads the library until
+ * the process exits. */
+#define GDN_NOALLOC_SCRATCH_BYTES (256u * 1024u)
+
+/* gdn_chunk_fwd without a workspace argument and without allocating anything.
+ * The paper has no counterpart: this is a deployment convenience.
+ *
+ * Who needs it: code that is handed only its input and output buffers and has
+ * no way to get more device memory -- a plugin inside another framework whose
+ * allocator it may not call, a serving loop that forbids allocation once it
+ * has started, or a process whose device memory is already fully reserved by
+ * another allocator, so that a cudaMalloc would fail or fragment it.
+ *
+ * Instead of a caller workspace it uses one fixed device array of
+ * GDN_NOALLOC_SCRATCH_BYTES compiled into the library.  Problems whose
+ * gdn_chunk_fwd_workspace_size exceeds that return GDN_ERR_UNSUPPORTED before
+ * anything is launched.  All other arguments, layouts and results are those of
+ * gdn_chunk_fwd.
+ *   - The first call on each device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call on a device shares the one array.  Each call clears its
+ *     header on `stream` before the kernels run, so calls that overlap on the
+ *     GPU (other streams, other host threads) race: serialise them.
+ *   - Device-detected errors are recorded in the array's header and are not
+ *     reported back; inconsistent cu_seqlens still never cause an
+ *     out-of-bounds access (the affected sequences are skipped).
+ *   - Calls no cudaMalloc, cudaFree or other allocating routine. */
+gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q, const void *k,
+                                 const void *v, const float *log_alpha, const float *beta,
+                                 const float *initial_state, const int32_t *cu_seqlens,
+                                 void *o, float *final_state, gdn_stream_t stream);
+
 /* Zero the workspace header (the sticky error word) on `stream`. */
 gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 

@@ -1,0 +1,76 @@
+"""gdn_chunk_fwd_noalloc: the prefill for callers that cannot allocate device
+memory (a plugin handed only its input and output buffers, a serving loop that
+forbids allocation after start-up, a process whose device memory another
+allocator already owns).  It runs the same kernels as gdn_chunk_fwd with a
+fixed array inside the library as scratch.
+
+This file is named to be collected last, so that a run stopping at the first
+failure has already run every other test; it passes alone in a fresh process
+as well.  The entry point is called through the C ABI (ctypes), twice in a row
+on different problems, and each result is checked against gdn_chunk_fwd's
+within the parity tolerances."""
+import ctypes
+
+import pytest
+import torch
+
+from gated_delta_rule_140_b200 import _native as nat
+from gated_delta_rule_140_b200 import chunk_fwd
+from gated_delta_rule_140_b200.inputs import prefill_inputs
+from tests.parity_util import TOL, rel_err, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _noalloc(d):
+    """Call gdn_chunk_fwd_noalloc through the C ABI on device inputs ``d``."""
+    L = nat.lib()
+    q, v, la, cu = d["q"], d["v"], d["log_alpha"], d["cu_seqlens"]
+    dims = nat.prefill_dims(q, v, la, cu)
+    o = torch.full(v.shape, float("nan"), dtype=q.dtype, device=q.device)
+    sf = torch.full((dims.n_seqs, dims.H, dims.d_v, dims.d_k), float("nan"),
+                    dtype=torch.float32, device=q.device)
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    st = L.gdn_chunk_fwd_noalloc(ctypes.byref(dims), p(q), p(d["k"]), p(v), p(la),
+                                 p(d["beta"]), p(d["initial_state"]), p(cu), p(o), p(sf),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == nat.GDN_OK, nat.status_string(st)
+    return o, sf
+
+
+def _problems():
+    a = prefill_inputs(2, 229, 3, 128, 128, dtype=torch.bfloat16, seed=41, init_std=0.05)
+    g = torch.Generator().manual_seed(42)
+    b = prefill_inputs(1, 0, 4, 64, 64, dtype=torch.float32, decay="channel", alpha_shift=3.0,
+                       init_std=0.02, lengths=[70, 0, 129, 5], gen=g)
+    return [(a, torch.bfloat16), (b, torch.float32)]
+
+
+def test_noalloc_matches_chunk_fwd_on_two_calls_in_a_row(cuda_ok):
+    for x, dtype in _problems():
+        d = to_dev(x)
+        o, sf = _noalloc(d)
+        o_ref, sf_ref = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
+                                  d["initial_state"], d["cu_seqlens"])
+        torch.cuda.synchronize()
+        to, ts = TOL[dtype]
+        assert rel_err(o, o_ref.double().cpu().numpy()) <= to
+        assert rel_err(sf, sf_ref.cpu().numpy()) <= ts
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch(cuda_ok):
+    L = nat.lib()
+    # the fixed array bounds the workspace; any problem needing more is refused
+    # on the host with GDN_ERR_UNSUPPORTED, before anything is launched
+    for n_seqs in (1, 1 << 10, 1 << 16, 1 << 20):
+        dims = nat.Dims(1, n_seqs * 64, 16, 128, 128, n_seqs, nat.GDN_BF16,
+                        nat.GDN_DECAY_SCALAR, 0)
+        need = L.gdn_chunk_fwd_workspace_size(ctypes.byref(dims))
+        if need > 256 * 1024:
+            fake = ctypes.c_void_p(0x10000)
+            st = L.gdn_chunk_fwd_noalloc(ctypes.byref(dims), fake, fake, fake, fake, fake,
+                                         None, fake, fake, None, None)
+            assert st == nat.GDN_ERR_UNSUPPORTED
+    # invalid dims are still invalid
+    bad = nat.Dims(1, 64, 16, 96, 128, 1, nat.GDN_BF16, nat.GDN_DECAY_SCALAR, 0)
+    assert L.gdn_chunk_fwd_noalloc(ctypes.byref(bad), *([None] * 9), None) != nat.GDN_OK
