@@ -10,26 +10,27 @@
 //
 //   D_kq  = [Q; K] K^T                  rows 0-63: Q K^T, rows 64-127: K K^T
 //   A_rs  = beta_r e^{g_r-g_s} (K K^T)_rs, s < r;  P_rs = e^{g_r-g_s} (Q K^T)_rs, s <= r
-//   T     = (I + A)^{-1}                 blocked forward substitution, fp32
+//   T     = (I + A)^{-1}                 blocked forward substitution (fp32, tf32 MMAs)
 //   T_b   = T diag(beta),  T_bg = T diag(beta gamma)       (bf16)
-//   D_w   = K^T T_bg^T                   = W^T,  W = T diag(beta)(gamma . K)
+//   D_w   = T_bg K                       rows 0-63: W = T diag(beta)(gamma . K)
 //   D_vp  = [T_b; 0] V                   rows 0-63: U = T diag(beta) V
-//   D_vp += [-W; gamma Q] S^T            rows 0-63: V' = U - W S^T; rows 64-127: gamma Q S^T
-//   D_ds  = K^^T V',  K^_s = e^{g_C-g_s} k_s
-//   D_vp += [0; P] V'                    rows 64-127: O = gamma Q S^T + P V'
-//   S    <- e^{g_C} S + D_ds^T
+//   D_vp += [-W; Q] S^T                  rows 0-63: V' = U - W S^T; rows 64-127: Q S^T
+//   D_ds  = K^T (kh . V'),  kh_s = e^{g_C-g_s}            (the decayed-key write)
+//   D_o   = [0; P] V'
+//   o_r   = gamma_r (Q S^T)_r + (P V')_r,   S <- e^{g_C} S + D_ds^T
 //
 // Warp roles (384 threads):
-//   warps 0-7  "local": everything that depends only on the chunk's own tokens
-//              (the first four and the "W/U" MMAs, A, T, W, P, K^, gamma Q),
-//              one chunk ahead of the state warps;
-//   warps 8-11 "state": the sequential inter-chunk pass (the [-W; gamma Q] S^T,
-//              K^^T V' and [0; P] V' MMAs, the fp32 state in registers --
-//              thread c holds column c of the state slice -- and the output).
-// The groups hand chunks over through mbarriers; tiles arrive by TMA into a
-// two-stage ring.  Every wait is bounded: on expiry the kernel records
-// kErrTimeout, both groups leave their loops at the next barrier, in-flight
-// copies and MMAs are drained (again with a bound) and TMEM is freed.
+//   warps 0-7  "local": the work that depends only on the chunk's own tokens
+//              (D_kq, A, T, W, U), one chunk ahead of the state warps;
+//   warps 8-11 "state": the sequential pass (the three S-dependent MMAs, P,
+//              the fp32 state in registers -- thread c holds column c of the
+//              state slice -- the output, and the next tile loads).
+// Tiles arrive by TMA into a two-stage ring; stage layout per 64-column atom:
+// [-W rows 0-63 | Q rows | K rows], so [Q; K] and [-W; Q] are both contiguous
+// M = 128 operands and the raw K tile also serves as an MN-major operand.
+// Every wait is bounded: on expiry the kernel records kErrTimeout, both groups
+// leave their loops at the next barrier, in-flight copies and MMAs are drained
+// (again with a bound) and TMEM is freed.
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
 
@@ -49,38 +50,41 @@ constexpr long long kWaitLimit = 1LL << 31;   // SM cycles (~1 s)
 constexpr int LDA = 68;         // fp32 row stride of A and T in smem
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_RAW = 0;          // 2 stages x 40 KB: [Q|K atom col 0][Q|K atom col 1][V]
-constexpr uint32_t RAW_STAGE = 40960;
-constexpr uint32_t RAW_K = 8192;         //   K rows follow Q rows inside an atom column
-constexpr uint32_t RAW_AC = 16384;       //   atom column stride
-constexpr uint32_t RAW_V = 32768;
-constexpr uint32_t OFF_WQ = 81920;       // [-W; gamma Q]: [atom col][128 rows][128 B]
-constexpr uint32_t OFF_KH = 114688;      // K^: 2 MN blocks x [64 rows][128 B]
-constexpr uint32_t OFF_TB = 131072;      // T diag(beta)  [64 rows][128 B]
-constexpr uint32_t OFF_Z = 139264;       // zeros         [64 rows][128 B]
-constexpr uint32_t OFF_P = 147456;       // P             [64 rows][128 B]
-constexpr uint32_t OFF_TG = 155648;      // T diag(beta gamma)
-constexpr uint32_t OFF_VP = 163840;      // V' MN-major   [64 rows r][64 i]
-constexpr uint32_t OFF_SB = 172032;      // S bf16 MN-major [128 rows c][64 i]
-constexpr uint32_t OFF_AF = 188416;      // A fp32 [64][LDA]
+constexpr uint32_t RAW_STAGE = 57344;    // one stage: 2 atom columns + V
+constexpr uint32_t RAW_AC = 24576;       //   atom column: [-W 64 rows][Q 64 rows][K 64 rows]
+constexpr uint32_t RAW_Q = 8192;
+constexpr uint32_t RAW_K = 16384;
+constexpr uint32_t RAW_V = 49152;        //   V slice tile [64 rows][128 B]
+constexpr uint32_t STAGE_LOAD_BYTES = 40960;  // Q, K (2 boxes each) and V per stage
+constexpr uint32_t OFF_RAW = 0;          // stages 0 and 1
+constexpr uint32_t OFF_TG = 114688;      // T diag(beta gamma) [64 rows][128 B]
+constexpr uint32_t OFF_TB = 122880;      // T diag(beta)       (also the 2nd half of [T_bg; T_b])
+constexpr uint32_t OFF_Z = 131072;       // zeros
+constexpr uint32_t OFF_P = 139264;       // P
+constexpr uint32_t OFF_VP = 147456;      // V'        MN-major [64 rows r][64 i]
+constexpr uint32_t OFF_VH = 155648;      // kh . V'   MN-major
+constexpr uint32_t OFF_SB = 163840;      // S (bf16)  MN-major [128 rows c][64 i]
+constexpr uint32_t OFF_AF = 180224;      // A fp32 [64][LDA]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * LDA * 4;   // T fp32 [64][LDA]
-constexpr uint32_t OFF_ROW = OFF_TF + 64 * LDA * 4;  // per-row scalars, 5 x 64 fp32
-constexpr uint32_t OFF_HAND = OFF_ROW + 5 * 64 * 4;  // g_C of the two chunks in flight
-constexpr uint32_t OFF_BAR = OFF_HAND + 64;
+constexpr uint32_t OFF_ROW = OFF_TF + 64 * LDA * 4;  // local per-row scalars: g, beta, beta e^g
+constexpr uint32_t OFF_HAND = OFF_ROW + 3 * 64 * 4;  // per chunk parity: g, e^g, e^{gC-g}, e^{gC}
+constexpr uint32_t HAND_STRIDE = 1024;
+constexpr uint32_t OFF_BAR = OFF_HAND + 2 * HAND_STRIDE;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;    // + alignment slack
 
 // TMEM columns (fp32 accumulators, 128 lanes each)
 constexpr uint32_t COL_KQ = 0;    // 2 buffers x 64
-constexpr uint32_t COL_W = 128;
-constexpr uint32_t COL_VP = 192;  // 2 buffers x 64
-constexpr uint32_t COL_DS = 320;
+constexpr uint32_t COL_W = 128;   // 128 columns
+constexpr uint32_t COL_VP = 256;  // 2 buffers x 64
+constexpr uint32_t COL_DS = 384;
+constexpr uint32_t COL_O = 448;
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);  // [Q;K] K^T
-constexpr uint32_t ID_MK = idesc_bf16(128, 64, true, false);   // K^T T_bg^T
-constexpr uint32_t ID_KM = idesc_bf16(128, 64, false, true);   // [T_b;0] V, [-W;gQ] S^T, [0;P] V'
-constexpr uint32_t ID_MM = idesc_bf16(128, 64, true, true);    // K^^T V'
+constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);   // [Q;K] K^T
+constexpr uint32_t ID_W = idesc_bf16(128, 128, false, true);    // [T_bg; T_b] K
+constexpr uint32_t ID_KM = idesc_bf16(128, 64, false, true);    // [T_b;0] V, [-W;Q] S^T, [0;P] V'
+constexpr uint32_t ID_MM = idesc_bf16(128, 64, true, true);     // K^T (kh . V')
 
 __device__ __forceinline__ uint4 pack8(const float *x) {
     uint4 u;
@@ -93,18 +97,6 @@ __device__ __forceinline__ uint4 pack8(const float *x) {
     u.z = *reinterpret_cast<uint32_t *>(&h2);
     u.w = *reinterpret_cast<uint32_t *>(&h3);
     return u;
-}
-
-__device__ __forceinline__ uint4 scale8(uint4 u, float s) {
-    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&u);
-    float x[8];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        float2 f = __bfloat1622float2(h[j]);
-        x[2 * j] = f.x * s;
-        x[2 * j + 1] = f.y * s;
-    }
-    return pack8(x);
 }
 
 // Wait with a bound; gives up early when the other group has aborted.
@@ -133,19 +125,16 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
     float *g_s = reinterpret_cast<float *>(sm + OFF_ROW);  // cumulative log decay g_r
     float *b_s = g_s + 64;                                 // beta_r
     float *bg_s = g_s + 128;                               // beta_r e^{g_r}
-    float *kh_s = g_s + 192;                               // e^{g_C - g_r}
-    float *gq_s = g_s + 256;                               // e^{g_r}
-    float *hand_gc = reinterpret_cast<float *>(sm + OFF_HAND);  // e^{g_C}, by chunk parity
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *bar_tma = bars + 0;     // [2] tiles of a stage landed
     uint64_t *bar_l = bars + 2;       // local MMAs done
     uint64_t *bar_s = bars + 3;       // state MMAs done
-    uint64_t *bar_wqfree = bars + 4;  // [-W; gamma Q] consumed by the state MMA
-    uint64_t *bar_pfree = bars + 5;   // P and K^ consumed by the state MMAs
-    uint64_t *bar_vpfree = bars + 6;  // [2] output accumulator of a stage read out
-    uint64_t *bar_ready = bars + 8;   // a chunk's operands are ready for the state pass
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 80);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 84);
+    uint64_t *bar_vpfree = bars + 4;  // [2] a chunk's state pass is over (its buffers are free)
+    uint64_t *bar_ready = bars + 6;   // a chunk's operands are ready for the state pass
+    uint64_t *bar_kqfree = bars + 7;  // the state pass has read Q K^T (D_kq) of a chunk
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 64);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 68);
+    int *tma_issued = reinterpret_cast<int *>(sm + OFF_BAR + 72);  // [2] loads issued per stage
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nsl = a.dv / DVS;
@@ -163,9 +152,10 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
     if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 9; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
         fence_mbar_init();
         *abort_flag = 0;
+        tma_issued[0] = tma_issued[1] = 0;
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
@@ -195,31 +185,40 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         const long long rem = t_end - (t_begin + (long long)m * C);
         return rem < C ? (int)rem : C;
     };
+    // Q, K and V tiles of chunk m into stage m % 2 (one thread).
+    auto issue_tma = [&](int m) {
+        const int st = m & 1;
+        const long long t0 = t_begin + (long long)m * C;
+        uint8_t *raw = sm + OFF_RAW + st * RAW_STAGE;
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bar_tma[st], STAGE_LOAD_BYTES);
+        tma_load_3d(raw + RAW_Q, &tm_q, 0, h, (int)t0, &bar_tma[st]);
+        tma_load_3d(raw + RAW_AC + RAW_Q, &tm_q, 64, h, (int)t0, &bar_tma[st]);
+        tma_load_3d(raw + RAW_K, &tm_k, 0, h, (int)t0, &bar_tma[st]);
+        tma_load_3d(raw + RAW_AC + RAW_K, &tm_k, 64, h, (int)t0, &bar_tma[st]);
+        tma_load_3d(raw + RAW_V, &tm_v, v0, h, (int)t0, &bar_tma[st]);
+        ++tma_issued[st];
+    };
 
     if (tid < kLocal) {
         // ============================ local group ============================
         const int lq = warp & 3, lhalf = warp >> 2;  // TMEM lane quadrant, column half
         const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
         uint32_t bl_wait = 0, bl_commit = 0;  // completions waited on / committed to bar_l
-        int tma_issued[2] = {0, 0}, tma_seen[2] = {0, 0};
+        int tma_seen0 = 0, tma_seen1 = 0;
+        // matrix descriptors: base per buffer, then + (byte offset >> 4) per K step;
+        // stage 1 is stage 0 + RAW_STAGE bytes
+        const uint64_t d_qk0 = desc_sw128(sbase + OFF_RAW + RAW_Q, 16, 1024);
+        const uint64_t d_kmn0 = desc_sw128(sbase + OFF_RAW + RAW_K, RAW_AC, 1024);
+        const uint64_t d_vmn0 = desc_sw128(sbase + OFF_RAW + RAW_V, 8192, 1024);
+        const uint64_t d_tg = desc_sw128(sbase + OFF_TG, 16, 1024);
+        const uint64_t d_tb = desc_sw128(sbase + OFF_TB, 16, 1024);
 
-        auto issue_tma = [&](int m) {  // leader only
-            const int st = m & 1;
-            const long long t0 = t_begin + (long long)m * C;
-            uint8_t *raw = sm + OFF_RAW + st * RAW_STAGE;
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&bar_tma[st], RAW_STAGE);
-            tma_load_3d(raw, &tm_q, 0, h, (int)t0, &bar_tma[st]);
-            tma_load_3d(raw + RAW_AC, &tm_q, 64, h, (int)t0, &bar_tma[st]);
-            tma_load_3d(raw + RAW_K, &tm_k, 0, h, (int)t0, &bar_tma[st]);
-            tma_load_3d(raw + RAW_AC + RAW_K, &tm_k, 64, h, (int)t0, &bar_tma[st]);
-            tma_load_3d(raw + RAW_V, &tm_v, v0, h, (int)t0, &bar_tma[st]);
-        };
         // wait for chunk m's tiles, zero rows past the sequence end, issue D_kq
         auto start_chunk = [&](int m) -> bool {
             const int st = m & 1;
-            bool ok = wait_bar(&bar_tma[st], (uint32_t)(tma_seen[st] & 1), abort_flag);
-            ++tma_seen[st];
+            bool ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag);
+            if (st) ++tma_seen1; else ++tma_seen0;
             const int L = chunk_len(m);
             if (L < C) {
                 uint8_t *raw = sm + OFF_RAW + st * RAW_STAGE;
@@ -227,24 +226,23 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const int r = L + (idx >> 3), pj = idx & 7;
                     const uint4 z = make_uint4(0, 0, 0, 0);
                     const uint32_t o = r * 128 + pj * 16;
-                    *reinterpret_cast<uint4 *>(raw + o) = z;                   // Q ac0
-                    *reinterpret_cast<uint4 *>(raw + RAW_AC + o) = z;          // Q ac1
-                    *reinterpret_cast<uint4 *>(raw + RAW_K + o) = z;           // K ac0
-                    *reinterpret_cast<uint4 *>(raw + RAW_AC + RAW_K + o) = z;  // K ac1
-                    *reinterpret_cast<uint4 *>(raw + RAW_V + o) = z;           // V
+                    *reinterpret_cast<uint4 *>(raw + RAW_Q + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + RAW_AC + RAW_Q + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + RAW_K + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + RAW_AC + RAW_K + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + RAW_V + o) = z;
                 }
                 fence_proxy_async_smem();
             }
-            const bool ab = named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag);
-            if (ab) return false;
+            if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) return false;
             if (tid == 0) {
                 tc_fence_after();
-                const uint32_t raw = sbase + OFF_RAW + st * RAW_STAGE;
+                const uint64_t da = d_qk0 + st * (RAW_STAGE >> 4);
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k) {
-                    const uint32_t off = (k >> 2) * RAW_AC + (k & 3) * 32;
-                    mma_bf16(tmem + COL_KQ + 64 * st, desc_sw128(raw + off, 16, 1024),
-                             desc_sw128(raw + RAW_K + off, 16, 1024), ID_KK, k > 0);
+                    const uint32_t off = ((k >> 2) * RAW_AC + (k & 3) * 32) >> 4;
+                    mma_bf16(tmem + COL_KQ + 64 * st, da + off, da + off + (RAW_K - RAW_Q) / 16,
+                             ID_KK, k > 0);
                 }
                 mma_commit(bar_l);
             }
@@ -252,30 +250,35 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             return true;
         };
 
+        // gates of the next chunk, prefetched into warp 0's registers
+        float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
+        auto load_gates = [&](int m) {
+            const long long t0 = t_begin + (long long)m * C;
+            const int L = chunk_len(m), r0 = 2 * lane, r1 = 2 * lane + 1;
+            nla0 = r0 < L ? a.log_alpha[(t0 + r0) * H + h] : 0.f;
+            nla1 = r1 < L ? a.log_alpha[(t0 + r1) * H + h] : 0.f;
+            nbe0 = r0 < L ? a.beta[(t0 + r0) * H + h] : 0.f;
+            nbe1 = r1 < L ? a.beta[(t0 + r1) * H + h] : 0.f;
+        };
         if (tid == 0) {
-            if (nchunks > 0) { issue_tma(0); ++tma_issued[0]; }
-            if (nchunks > 1) { issue_tma(1); ++tma_issued[1]; }
-        } else {
-            if (nchunks > 0) ++tma_issued[0];
-            if (nchunks > 1) ++tma_issued[1];
+            if (nchunks > 0) issue_tma(0);
+            if (nchunks > 1) issue_tma(1);
         }
+        if (warp == 0 && nchunks > 0) load_gates(0);
         bool alive = nchunks > 0 ? start_chunk(0) : true;
 
         for (int m = 0; alive && m < nchunks; ++m) {
             const int st = m & 1;
-            const long long t0 = t_begin + (long long)m * C;
-            const int L = chunk_len(m);
             uint8_t *raw = sm + OFF_RAW + st * RAW_STAGE;
-            const uint32_t raw_a = sbase + OFF_RAW + st * RAW_STAGE;
+            float *hand = reinterpret_cast<float *>(sm + OFF_HAND + st * HAND_STRIDE);
             bool ok = true;
 
-            // ---- gates: beta and the cumulative log decay (warp 0) ------------
+            // ---- gates (warp 0), once the state pass of chunk m-2 is over ------
             if (warp == 0) {
+                if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag);
                 const int r0 = 2 * lane, r1 = 2 * lane + 1;
-                const float la0 = r0 < L ? a.log_alpha[(t0 + r0) * H + h] : 0.f;
-                const float la1 = r1 < L ? a.log_alpha[(t0 + r1) * H + h] : 0.f;
-                const float be0 = r0 < L ? a.beta[(t0 + r0) * H + h] : 0.f;
-                const float be1 = r1 < L ? a.beta[(t0 + r1) * H + h] : 0.f;
+                const float la0 = nla0, la1 = nla1, be0 = nbe0, be1 = nbe1;
+                if (m + 1 < nchunks) load_gates(m + 1);
                 float incl = la0 + la1;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
@@ -284,12 +287,14 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 }
                 const float gC = __shfl_sync(0xffffffffu, incl, 31);
                 const float g1 = incl, g0 = incl - la1;
+                const float e0 = __expf(g0), e1 = __expf(g1);
                 g_s[r0] = g0; g_s[r1] = g1;
                 b_s[r0] = be0; b_s[r1] = be1;
-                bg_s[r0] = be0 * __expf(g0); bg_s[r1] = be1 * __expf(g1);
-                kh_s[r0] = __expf(gC - g0); kh_s[r1] = __expf(gC - g1);
-                gq_s[r0] = __expf(g0); gq_s[r1] = __expf(g1);
-                if (lane == 0) hand_gc[st] = __expf(gC);
+                bg_s[r0] = be0 * e0; bg_s[r1] = be1 * e1;
+                hand[r0] = g0; hand[r1] = g1;                               // g
+                hand[64 + r0] = e0; hand[64 + r1] = e1;                     // e^{g}
+                hand[128 + r0] = __expf(gC - g0); hand[128 + r1] = __expf(gC - g1);  // e^{gC-g}
+                if (lane == 0) hand[192] = __expf(gC);
             }
             // ---- D_kq of this chunk ----------------------------------------------
             ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
@@ -315,228 +320,268 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             }
             named_bar_sync(BAR_LOCAL, kLocal);
             // ---- T = (I + A)^{-1} ------------------------------------------------
-            // 16x16 diagonal blocks: warp w < 4 inverts block w, lane j < 16
-            // owns column j (forward substitution down the column).
+            // (1) 16x16 diagonal blocks: warp w < 4 inverts block w; lane j < 16
+            //     owns column j and runs the forward substitution in registers.
             if (warp < 4 && lane < 16) {
                 const int o = 16 * warp, j = lane;
                 float t[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
+                    float arow[16];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<float4 *>(arow + 4 * q4) =
+                            *reinterpret_cast<const float4 *>(AF + (o + i) * LDA + o + 4 * q4);
                     float acc = (i == j) ? 1.f : 0.f;
 #pragma unroll
-                    for (int mm = 0; mm < i; ++mm) acc -= AF[(o + i) * LDA + o + mm] * t[mm];
+                    for (int mm = 0; mm < i; ++mm) acc -= arow[mm] * t[mm];
                     t[i] = acc;
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) TF[(o + i) * LDA + o + j] = t[i];
             }
             named_bar_sync(BAR_LOCAL, kLocal);
-            // 32x32 halves: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22).
-            // X goes to the unused upper-right 16x16 block of each half.
-            {
-                const int hf = tid >> 7, e = tid & 127, ii = e >> 3, jj = 2 * (e & 7);
-                const int o = 32 * hf;  // half origin
-                float x0 = 0.f, x1 = 0.f;
+            const int fg = lane >> 2, ft = lane & 3;  // mma.sync fragment coordinates
+            // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
+            //     warp w < 4: half w/2, 8 output columns (w%2).  X goes to the
+            //     unused upper-right 16x16 block of the half.
+            if (warp < 4) {
+                const int o = 32 * (warp >> 1), n0 = 8 * (warp & 1);
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int mm = 0; mm < 16; ++mm) {
-                    const float av = AF[(o + 16 + ii) * LDA + o + mm];
-                    x0 += av * TF[(o + mm) * LDA + o + jj];
-                    x1 += av * TF[(o + mm) * LDA + o + jj + 1];
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int ar = o + 16 + fg, ac = o + 8 * ks + ft;
+                    af[0] = to_tf32(AF[ar * LDA + ac]);
+                    af[1] = to_tf32(AF[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AF[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AF[(ar + 8) * LDA + ac + 4]);
+                    bf[0] = to_tf32(TF[(o + 8 * ks + ft) * LDA + o + n0 + fg]);
+                    bf[1] = to_tf32(TF[(o + 8 * ks + ft + 4) * LDA + o + n0 + fg]);
+                    mma_tf32_16x8x8(x, af, bf);
                 }
-                TF[(o + ii) * LDA + o + 16 + jj] = x0;
-                TF[(o + ii) * LDA + o + 16 + jj + 1] = x1;
-                named_bar_sync(BAR_LOCAL, kLocal);
-                float y0 = 0.f, y1 = 0.f;
+                TF[(o + fg) * LDA + o + 16 + n0 + 2 * ft] = x[0];
+                TF[(o + fg) * LDA + o + 16 + n0 + 2 * ft + 1] = x[1];
+                TF[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft] = x[2];
+                TF[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft + 1] = x[3];
+                __syncwarp();
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int mm = 0; mm < 16; ++mm) {
-                    const float tv = TF[(o + 16 + ii) * LDA + o + 16 + mm];
-                    y0 += tv * TF[(o + mm) * LDA + o + 16 + jj];
-                    y1 += tv * TF[(o + mm) * LDA + o + 16 + jj + 1];
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int ar = o + 16 + fg, ac = o + 16 + 8 * ks + ft;
+                    af[0] = to_tf32(TF[ar * LDA + ac]);
+                    af[1] = to_tf32(TF[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(TF[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(TF[(ar + 8) * LDA + ac + 4]);
+                    bf[0] = to_tf32(TF[(o + 8 * ks + ft) * LDA + o + 16 + n0 + fg]);
+                    bf[1] = to_tf32(TF[(o + 8 * ks + ft + 4) * LDA + o + 16 + n0 + fg]);
+                    mma_tf32_16x8x8(y, af, bf);
                 }
-                TF[(o + 16 + ii) * LDA + o + jj] = -y0;
-                TF[(o + 16 + ii) * LDA + o + jj + 1] = -y1;
+                TF[(o + 16 + fg) * LDA + o + n0 + 2 * ft] = -y[0];
+                TF[(o + 16 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[1];
+                TF[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
+                TF[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
             }
             named_bar_sync(BAR_LOCAL, kLocal);
-            // full: T_{H1,H0} = -T_{H1} (A_{H1,H0} T_{H0}); X in the upper-right
-            // 32x32 block.  Thread: row i, four columns j4..j4+3.
+            // (3) T_{H1,H0} = -T_{H1} (A_{H1,H0} T_{H0}), 32x32 blocks; warp w owns
+            //     output rows 16(w/4).., columns 8(w%4)..  X goes to the unused
+            //     upper-right 32x32 block.  The upper triangles of T_{H0} and
+            //     T_{H1} hold scratch, so their fragments are masked.
             {
-                const int i = tid >> 3, j4 = 4 * (tid & 7);
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int k = 0; k < 32; ++k) {
-                    const float av = AF[(32 + i) * LDA + k];
-                    const float4 tv = *reinterpret_cast<const float4 *>(TF + k * LDA + j4);
-                    // T_{H0} is lower triangular: entries with k < j are zero, but
-                    // the upper part of TF holds scratch, so mask by column.
-                    x.x += (k >= j4 + 0) ? av * tv.x : 0.f;
-                    x.y += (k >= j4 + 1) ? av * tv.y : 0.f;
-                    x.z += (k >= j4 + 2) ? av * tv.z : 0.f;
-                    x.w += (k >= j4 + 3) ? av * tv.w : 0.f;
+                const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int ar = 32 + m0 + fg, ac = 8 * ks + ft;
+                    af[0] = to_tf32(AF[ar * LDA + ac]);
+                    af[1] = to_tf32(AF[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AF[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AF[(ar + 8) * LDA + ac + 4]);
+                    const int br = 8 * ks + ft, bc = n0 + fg;
+                    bf[0] = to_tf32(br >= bc ? TF[br * LDA + bc] : 0.f);
+                    bf[1] = to_tf32(br + 4 >= bc ? TF[(br + 4) * LDA + bc] : 0.f);
+                    mma_tf32_16x8x8(x, af, bf);
                 }
-                *reinterpret_cast<float4 *>(TF + i * LDA + 32 + j4) = x;
+                TF[(m0 + fg) * LDA + 32 + n0 + 2 * ft] = x[0];
+                TF[(m0 + fg) * LDA + 32 + n0 + 2 * ft + 1] = x[1];
+                TF[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft] = x[2];
+                TF[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft + 1] = x[3];
                 named_bar_sync(BAR_LOCAL, kLocal);
-                float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int k = 0; k <= i; ++k) {
-                    const float tv = TF[(32 + i) * LDA + 32 + k];
-                    const float4 xv = *reinterpret_cast<const float4 *>(TF + k * LDA + 32 + j4);
-                    y.x += tv * xv.x; y.y += tv * xv.y; y.z += tv * xv.z; y.w += tv * xv.w;
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int r = m0 + fg, kc = 8 * ks + ft;  // within H1
+                    af[0] = to_tf32(kc <= r ? TF[(32 + r) * LDA + 32 + kc] : 0.f);
+                    af[1] = to_tf32(kc <= r + 8 ? TF[(40 + r) * LDA + 32 + kc] : 0.f);
+                    af[2] = to_tf32(kc + 4 <= r ? TF[(32 + r) * LDA + 36 + kc] : 0.f);
+                    af[3] = to_tf32(kc + 4 <= r + 8 ? TF[(40 + r) * LDA + 36 + kc] : 0.f);
+                    bf[0] = to_tf32(TF[(8 * ks + ft) * LDA + 32 + n0 + fg]);
+                    bf[1] = to_tf32(TF[(8 * ks + ft + 4) * LDA + 32 + n0 + fg]);
+                    mma_tf32_16x8x8(y, af, bf);
                 }
-                *reinterpret_cast<float4 *>(TF + (32 + i) * LDA + j4) =
-                    make_float4(-y.x, -y.y, -y.z, -y.w);
+                TF[(32 + m0 + fg) * LDA + n0 + 2 * ft] = -y[0];
+                TF[(32 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[1];
+                TF[(40 + m0 + fg) * LDA + n0 + 2 * ft] = -y[2];
+                TF[(40 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[3];
             }
             named_bar_sync(BAR_LOCAL, kLocal);
             // ---- T diag(beta) and T diag(beta gamma) in bf16 (K-major, s cols) ---
-            for (int idx = tid; idx < 64 * 8; idx += kLocal) {
-                const int r = idx >> 3, j = idx & 7;
-                float tb[8], tg[8];
+#pragma unroll
+            for (int it = 0; it < 2; ++it) {
+                const int idx = tid + kLocal * it, r = idx >> 3, j = idx & 7;
+                float tv[8], bv[8], gv[8], tb[8], tg[8];
+                *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j);
+                *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j + 4);
+                *reinterpret_cast<float4 *>(bv) = *reinterpret_cast<const float4 *>(b_s + 8 * j);
+                *reinterpret_cast<float4 *>(bv + 4) = *reinterpret_cast<const float4 *>(b_s + 8 * j + 4);
+                *reinterpret_cast<float4 *>(gv) = *reinterpret_cast<const float4 *>(bg_s + 8 * j);
+                *reinterpret_cast<float4 *>(gv + 4) = *reinterpret_cast<const float4 *>(bg_s + 8 * j + 4);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int s = 8 * j + e;
-                    const float tv = s < r ? TF[r * LDA + s] : (s == r ? 1.f : 0.f);
-                    tb[e] = tv * b_s[s];
-                    tg[e] = tv * bg_s[s];
+                    const int s2 = 8 * j + e;
+                    const float t2 = s2 < r ? tv[e] : (s2 == r ? 1.f : 0.f);
+                    tb[e] = t2 * bv[e];
+                    tg[e] = t2 * gv[e];
                 }
                 *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128(r, j)) = pack8(tb);
                 *reinterpret_cast<uint4 *>(sm + OFF_TG + sw128(r, j)) = pack8(tg);
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_LOCAL, kLocal);
-            // ---- W^T = K^T T_bg^T;  D_vp = [T_b; 0] V ------------------------------
+            // ---- D_w = [T_bg; T_b] K (rows 0-63: W);  D_vp = [T_b; 0] V ----------
             if (tid == 0) {
-                if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag);
+                if (m >= 1) ok &= wait_bar(bar_kqfree, (uint32_t)((m - 1) & 1), abort_flag);
                 tc_fence_after();
+                const uint64_t dk = d_kmn0 + st * (RAW_STAGE >> 4);
+                const uint64_t dv = d_vmn0 + st * (RAW_STAGE >> 4);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tmem + COL_W, desc_sw128(raw_a + RAW_K + k * 2048, RAW_AC, 1024),
-                             desc_sw128(sbase + OFF_TG + k * 32, 16, 1024), ID_MK, k > 0);
+                    mma_bf16(tmem + COL_W, d_tg + k * 2, dk + k * 128, ID_W, k > 0);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tmem + COL_VP + 64 * st, desc_sw128(sbase + OFF_TB + k * 32, 16, 1024),
-                             desc_sw128(raw_a + RAW_V + k * 2048, 8192, 1024), ID_KM, k > 0);
+                    mma_bf16(tmem + COL_VP + 64 * st, d_tb + k * 2, dv + k * 128, ID_KM, k > 0);
                 mma_commit(bar_l);
             }
             ++bl_commit;
-            // ---- while those run: P, K^ and gamma Q (once the state group has
-            // consumed the previous chunk's copies) --------------------------------
-            if (m >= 1) {
-                ok &= wait_bar(bar_pfree, (uint32_t)((m - 1) & 1), abort_flag);
-                ok &= wait_bar(bar_wqfree, (uint32_t)((m - 1) & 1), abort_flag);
-            }
-            if (lq < 2) {  // P rows from Q K^T (TMEM lanes 0-63)
-                float x[32];
-                tmem_load<32>(tmem + lane_off + COL_KQ + 64 * st + 32 * lhalf, x);
-                const int r = 32 * lq + lane;
-                const float gr = g_s[r];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int s = 32 * lhalf + j;
-                    x[j] = s <= r ? __expf(gr - g_s[s]) * x[j] : 0.f;
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw128(r, 4 * lhalf + j)) = pack8(x + 8 * j);
-            }
-            for (int idx = tid; idx < 1024; idx += kLocal) {
-                const int b = idx >> 9, rem = idx & 511, r = rem >> 3, pj = rem & 7;
-                const uint32_t o = r * 128 + pj * 16;
-                const uint4 kv = *reinterpret_cast<const uint4 *>(raw + b * RAW_AC + RAW_K + o);
-                *reinterpret_cast<uint4 *>(sm + OFF_KH + b * 8192 + o) = scale8(kv, kh_s[r]);
-                const uint4 qv = *reinterpret_cast<const uint4 *>(raw + b * RAW_AC + o);
-                *reinterpret_cast<uint4 *>(sm + OFF_WQ + b * 16384 + 8192 + o) = scale8(qv, gq_s[r]);
-            }
-            // ---- -W into rows 0-63 of [-W; gamma Q] --------------------------------
             ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
             ++bl_wait;
             tc_fence_after();
-            {
-                float w[32];
-                tmem_load<32>(tmem + lane_off + COL_W + 32 * lhalf, w);  // lane c: W[r][c]
-                const int c = 32 * lq + lane, ac = c >> 6, cc = c & 63;
+            // ---- -W into rows 0-63 of the stage (K-major, atom column lhalf) ------
+            if (lq < 2) {
+                float w[64];
+                tmem_load<64>(tmem + lane_off + COL_W + 64 * lhalf, w);  // lane r: W[r][c]
+                const int r = 32 * lq + lane;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int r = 32 * lhalf + j;
-                    const uint32_t off = OFF_WQ + ac * 16384 + r * 128 +
-                                         (((cc >> 3) ^ (r & 7)) << 4) + (cc & 7) * 2;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + off) = __float2bfloat16_rn(-w[j]);
-                }
+                for (int j = 0; j < 64; ++j) w[j] = -w[j];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4 *>(raw + lhalf * RAW_AC + sw128(r, j)) = pack8(w + 8 * j);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
-            if (tid == 0) {
-                // stage st is free (its MMAs are done, copies read): prefetch m+2
-                if (m + 2 < nchunks) issue_tma(m + 2);
-                mbar_arrive(bar_ready);
-            }
-            if (m + 2 < nchunks) ++tma_issued[st];
+            if (tid == 0) mbar_arrive(bar_ready);
             // ---- start the next chunk's D_kq ------------------------------------
             if (m + 1 < nchunks && !start_chunk(m + 1)) break;
         }
-        // drain what this group launched, then report
-        if (*abort_flag && tid == 0) {
-            for (int s2 = 0; s2 < 2; ++s2)
-                for (int i = tma_seen[s2]; i < tma_issued[s2]; ++i)
-                    mbar_wait(&bar_tma[s2], (uint32_t)(i & 1), kWaitLimit);
+        // drain what this group launched
+        if (*abort_flag && tid == 0)
             for (uint32_t i = bl_wait; i < bl_commit; ++i) mbar_wait(bar_l, i & 1, kWaitLimit);
-        }
     } else {
         // ============================ state group ============================
         const int sq = warp & 3;  // TMEM lane quadrant = warp - 8
         const uint32_t lane_off = (uint32_t)(32 * sq) << 16;
         uint32_t bs_wait = 0, bs_commit = 0;
+        const uint64_t d_wq0 = desc_sw128(sbase + OFF_RAW, 16, 1024);
+        const uint64_t d_kmn0 = desc_sw128(sbase + OFF_RAW + RAW_K, RAW_AC, 1024);
+        const uint64_t d_sb = desc_sw128(sbase + OFF_SB, 16384, 1024);
+        const uint64_t d_vp = desc_sw128(sbase + OFF_VP, 8192, 1024);
+        const uint64_t d_vh = desc_sw128(sbase + OFF_VH, 8192, 1024);
+        const uint64_t d_z = desc_sw128(sbase + OFF_Z, 16, 1024);
         for (int m = 0; m < nchunks; ++m) {
             const int st = m & 1;
             const long long t0 = t_begin + (long long)m * C;
             const int L = chunk_len(m);
+            const float *hand = reinterpret_cast<const float *>(sm + OFF_HAND + st * HAND_STRIDE);
             bool ok = wait_bar(bar_ready, (uint32_t)(m & 1), abort_flag);
-            const float dec = hand_gc[st];  // read before the barrier: the slot is reused two chunks on
             tc_fence_after();
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
-            // ---- D_vp += [-W; gamma Q] S^T ----------------------------------------
+            const float dec = hand[192];
+            // ---- D_vp += [-W; Q] S^T ----------------------------------------------
             if (tid == kLocal) {
                 tc_fence_after();
+                const uint64_t da = d_wq0 + st * (RAW_STAGE >> 4);
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k)
-                    mma_bf16(tmem + COL_VP + 64 * st,
-                             desc_sw128(sbase + OFF_WQ + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                             desc_sw128(sbase + OFF_SB + k * 2048, 16384, 1024), ID_KM, 1);
+                    mma_bf16(tmem + COL_VP + 64 * st, da + (((k >> 2) * RAW_AC + (k & 3) * 32) >> 4),
+                             d_sb + k * 128, ID_KM, 1);
                 mma_commit(bar_s);
-                mma_commit(bar_wqfree);
             }
             ++bs_commit;
+            // ---- meanwhile: P from Q K^T (TMEM lanes 0-63) -------------------------
+            if (sq < 2) {
+                const int r = 32 * sq + lane;
+                const float gr = hand[r];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[32];
+                    tmem_load<32>(tmem + lane_off + COL_KQ + 64 * st + 32 * hh, x);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int s = 32 * hh + j;
+                        x[j] = s <= r ? __expf(gr - hand[s]) * x[j] : 0.f;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<uint4 *>(sm + OFF_P + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
+                }
+            }
+            tc_fence_before();
+            named_bar_sync(BAR_STATE, kState);
+            if (tid == kLocal) mbar_arrive(bar_kqfree);
             ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
             ++bs_wait;
             tc_fence_after();
-            // ---- V' = rows 0-63 as the MN-major operand --------------------------
+            // ---- V' (rows 0-63) and kh . V' as MN-major operands ------------------
             if (sq < 2) {
                 float vp[64];
                 tmem_load<64>(tmem + lane_off + COL_VP + 64 * st, vp);
                 const int r = 32 * sq + lane;
+                const float khr = hand[128 + r];
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<uint4 *>(sm + OFF_VP + sw128(r, j)) = pack8(vp + 8 * j);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) vp[j] *= khr;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    *reinterpret_cast<uint4 *>(sm + OFF_VH + sw128(r, j)) = pack8(vp + 8 * j);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
-            // ---- D_ds = K^^T V';  D_vp += [0; P] V' --------------------------------
+            // ---- D_ds = K^T (kh . V');  D_o = [0; P] V' ----------------------------
             if (tid == kLocal) {
                 tc_fence_after();
+                const uint64_t dk = d_kmn0 + st * (RAW_STAGE >> 4);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tmem + COL_DS, desc_sw128(sbase + OFF_KH + k * 2048, 8192, 1024),
-                             desc_sw128(sbase + OFF_VP + k * 2048, 8192, 1024), ID_MM, k > 0);
+                    mma_bf16(tmem + COL_DS, dk + k * 128, d_vh + k * 128, ID_MM, k > 0);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tmem + COL_VP + 64 * st, desc_sw128(sbase + OFF_Z + k * 32, 16, 1024),
-                             desc_sw128(sbase + OFF_VP + k * 2048, 8192, 1024), ID_KM, 1);
+                    mma_bf16(tmem + COL_O, d_z + k * 2, d_vp + k * 128, ID_KM, k > 0);
                 mma_commit(bar_s);
-                mma_commit(bar_pfree);
             }
             ++bs_commit;
             ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
             ++bs_wait;
             tc_fence_after();
-            // ---- S <- e^{g_C} S + dS;  output rows -------------------------------
+            // the stage is free: load chunk m+2 into it
+            if (tid == kLocal && ok && m + 2 < nchunks) issue_tma(m + 2);
+            // ---- S <- e^{g_C} S + dS;  o_r = e^{g_r} (Q S^T)_r + (P V')_r ----------
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float ds[32];
@@ -548,14 +593,22 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4 *>(sm + OFF_SB + sw128(c_st, j)) = pack8(s_reg + 8 * j);
             if (sq >= 2) {
-                float o[64];
-                tmem_load<64>(tmem + lane_off + COL_VP + 64 * st, o);
                 const int r = 32 * (sq - 2) + lane;
-                if (r < L) {
-                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.o) +
-                                         ((t0 + r) * H + h) * (long long)a.dv + v0;
+                const float er = hand[64 + r];
+                __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.o) +
+                                     ((t0 + r) * H + h) * (long long)a.dv + v0;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) reinterpret_cast<uint4 *>(dst)[j] = pack8(o + 8 * j);
+                for (int hh = 0; hh < 2; ++hh) {
+                    float qs[32], pv[32];
+                    tmem_load<32>(tmem + lane_off + COL_VP + 64 * st + 32 * hh, qs);
+                    tmem_load<32>(tmem + lane_off + COL_O + 32 * hh, pv);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) qs[j] = er * qs[j] + pv[j];
+                    if (r < L) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            reinterpret_cast<uint4 *>(dst)[4 * hh + j] = pack8(qs + 8 * j);
+                    }
                 }
             }
             fence_proxy_async_smem();
@@ -574,7 +627,14 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *abort_flag) atomicOr(a.err, kErrTimeout);
+    if (tid == 0 && *abort_flag) {
+        atomicOr(a.err, kErrTimeout);
+        // let every tile load already issued land before the CTA exits: loads of
+        // a stage complete in issue order, so the last one's phase suffices
+        for (int st = 0; st < 2; ++st)
+            if (tma_issued[st] > 0)
+                mbar_wait(&bar_tma[st], (uint32_t)((tma_issued[st] - 1) & 1), kWaitLimit);
+    }
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 

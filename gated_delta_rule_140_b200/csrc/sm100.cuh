@@ -198,6 +198,25 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
         : "memory");
 }
 
+// ------------------------------------------------- warp-level tf32 MMA --
+// mma.sync m16n8k8, tf32 inputs, fp32 accumulate (used for small 16x16 and
+// 32x32 block products on the CUDA-core side of the kernel).  Fragments:
+// g = lane / 4, t = lane % 4;  A (16x8): a0 (g, t), a1 (g+8, t), a2 (g, t+4),
+// a3 (g+8, t+4);  B (8x8): b0 (t, g), b1 (t+4, g);  C (16x8): c0 (g, 2t),
+// c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1).
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float *d, const uint32_t *a, const uint32_t *b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+        "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a
 // 128-byte-swizzled region whose base is 1024-byte aligned.
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
