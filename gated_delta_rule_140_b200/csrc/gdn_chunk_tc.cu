@@ -8,25 +8,25 @@
 // causal product; the Gated Delta Networks page, section 3.3, for the scalar
 // cumulative decay g_r, gamma_r = e^{g_r}).  Per chunk:
 //
-//   D_kq  = [Q; K] K^T                  rows 0-63: Q K^T, rows 64-127: K K^T
+//   D_kq  = [K; Q] K^T                  rows 0-63: K K^T, rows 64-127: Q K^T
 //   A_rs  = beta_r e^{g_r-g_s} (K K^T)_rs, s < r;  P_rs = e^{g_r-g_s} (Q K^T)_rs, s <= r
 //   T     = (I + A)^{-1}                 blocked forward substitution (fp32, tf32 MMAs)
 //   T_b   = T diag(beta),  T_bg = T diag(beta gamma)       (bf16)
-//   D_w   = T_bg K                       rows 0-63: W = T diag(beta)(gamma . K)
-//   D_vp  = [T_b; 0] V                   rows 0-63: U = T diag(beta) V
-//   D_vp += [-W; Q] S^T                  rows 0-63: V' = U - W S^T; rows 64-127: Q S^T
+//   D_w   = [T_bg; 0] K                  rows 0-63: W = T diag(beta)(gamma . K)
+//   D_vp  = [0; T_b] V                   rows 64-127: U = T diag(beta) V
+//   D_vp += [Q; -W] S^T                  rows 0-63: Q S^T; rows 64-127: V' = U - W S^T
 //   D_ds  = K^T (kh . V'),  kh_s = e^{g_C-g_s}            (the decayed-key write)
-//   D_o   = [0; P] V'
+//   D_o   = [P; 0] V'
 //   o_r   = gamma_r (Q S^T)_r + (P V')_r,   S <- e^{g_C} S + D_ds^T
 //
 // Warp roles (384 threads):
 //   warps 0-7  "local": the work that depends only on the chunk's own tokens
-//              (D_kq, A, T, W, U), one chunk ahead of the state warps;
-//   warps 8-11 "state": the sequential pass (the three S-dependent MMAs, P,
-//              the fp32 state in registers -- thread c holds column c of the
+//              (D_kq, A, T, W, U, P), one chunk ahead of the state warps;
+//   warps 8-11 "state": the sequential pass (the three S-dependent MMAs, the
+//              fp32 state in registers -- thread c holds column c of the
 //              state slice -- the output, and the next tile loads).
 // Tiles arrive by TMA into a two-stage ring; stage layout per 64-column atom:
-// [-W rows 0-63 | Q rows | K rows], so [Q; K] and [-W; Q] are both contiguous
+// [K rows 0-63 | Q rows | -W rows], so [K; Q] and [Q; -W] are both contiguous
 // M = 128 operands and the raw K tile also serves as an MN-major operand.
 // Every wait is bounded: on expiry the kernel records kErrTimeout, both groups
 // leave their loops at the next barrier, in-flight copies and MMAs are drained
@@ -45,29 +45,32 @@ constexpr int DVS = 64;         // d_v slice per CTA
 constexpr int kLocal = 256;     // threads of the local group
 constexpr int kState = 128;     // threads of the state group
 constexpr int kThreads = kLocal + kState;
-constexpr int BAR_LOCAL = 1, BAR_STATE = 2;  // named barrier ids
+constexpr int BAR_LOCAL = 1, BAR_STATE = 2, BAR_INV = 3;  // named barrier ids
 constexpr long long kWaitLimit = 1LL << 31;   // SM cycles (~1 s)
 constexpr int LDA = 68;         // fp32 row stride of A and T in smem
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t RAW_STAGE = 57344;    // one stage: 2 atom columns + V
-constexpr uint32_t RAW_AC = 24576;       //   atom column: [-W 64 rows][Q 64 rows][K 64 rows]
+constexpr uint32_t RAW_AC = 24576;       //   atom column: [K 64 rows][Q 64 rows][-W 64 rows]
+constexpr uint32_t RAW_K = 0;
 constexpr uint32_t RAW_Q = 8192;
-constexpr uint32_t RAW_K = 16384;
+constexpr uint32_t RAW_W = 16384;
 constexpr uint32_t RAW_V = 49152;        //   V slice tile [64 rows][128 B]
 constexpr uint32_t STAGE_LOAD_BYTES = 40960;  // Q, K (2 boxes each) and V per stage
 constexpr uint32_t OFF_RAW = 0;          // stages 0 and 1
-constexpr uint32_t OFF_TG = 114688;      // T diag(beta gamma) [64 rows][128 B]
-constexpr uint32_t OFF_TB = 122880;      // T diag(beta)       (also the 2nd half of [T_bg; T_b])
-constexpr uint32_t OFF_Z = 131072;       // zeros
-constexpr uint32_t OFF_P = 139264;       // P
-constexpr uint32_t OFF_VP = 147456;      // V'        MN-major [64 rows r][64 i]
-constexpr uint32_t OFF_VH = 155648;      // kh . V'   MN-major
-constexpr uint32_t OFF_SB = 163840;      // S (bf16)  MN-major [128 rows c][64 i]
-constexpr uint32_t OFF_AF = 180224;      // A fp32 [64][LDA]
+constexpr uint32_t OFF_TG = 114688;      // T diag(beta gamma) [64 rows][128 B]  } [T_bg; 0]
+constexpr uint32_t OFF_Z = 122880;       // zeros                                } [0; T_b]
+constexpr uint32_t OFF_TB = 131072;      // T diag(beta)
+constexpr uint32_t OFF_P = 139264;       // P                                    } [P; 0]
+constexpr uint32_t OFF_Z2 = 147456;      // zeros
+constexpr uint32_t OFF_VP = 155648;      // V'        MN-major [64 rows r][64 i]
+constexpr uint32_t OFF_VH = 163840;      // kh . V'   MN-major
+constexpr uint32_t OFF_SB = 172032;      // S (bf16)  MN-major [128 rows c][64 i]
+constexpr uint32_t OFF_AF = 188416;      // A fp32 [64][LDA]
 constexpr uint32_t OFF_TF = OFF_AF + 64 * LDA * 4;   // T fp32 [64][LDA]
-constexpr uint32_t OFF_ROW = OFF_TF + 64 * LDA * 4;  // local per-row scalars: g, beta, beta e^g
-constexpr uint32_t OFF_HAND = OFF_ROW + 3 * 64 * 4;  // per chunk parity: g, e^g, e^{gC-g}, e^{gC}
+constexpr uint32_t OFF_ROW = OFF_TF + 64 * LDA * 4;  // per chunk parity: g, beta, beta e^g,
+constexpr uint32_t ROW_STRIDE = 8 * 64 * 4;          // colf[64], rowf[64][4]
+constexpr uint32_t OFF_HAND = OFF_ROW + 2 * ROW_STRIDE;  // per chunk parity: g[64], g_C
 constexpr uint32_t HAND_STRIDE = 1024;
 constexpr uint32_t OFF_BAR = OFF_HAND + 2 * HAND_STRIDE;
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
@@ -81,9 +84,9 @@ constexpr uint32_t COL_DS = 384;
 constexpr uint32_t COL_O = 448;
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);   // [Q;K] K^T
-constexpr uint32_t ID_W = idesc_bf16(128, 128, false, true);    // [T_bg; T_b] K
-constexpr uint32_t ID_KM = idesc_bf16(128, 64, false, true);    // [T_b;0] V, [-W;Q] S^T, [0;P] V'
+constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);   // [K;Q] K^T
+constexpr uint32_t ID_W = idesc_bf16(128, 128, false, true);    // [T_bg; 0] K
+constexpr uint32_t ID_KM = idesc_bf16(128, 64, false, true);    // [0;T_b] V, [Q;-W] S^T, [P;0] V'
 constexpr uint32_t ID_MM = idesc_bf16(128, 64, true, true);     // K^T (kh . V')
 
 __device__ __forceinline__ uint4 pack8(const float *x) {
@@ -99,7 +102,33 @@ __device__ __forceinline__ uint4 pack8(const float *x) {
     return u;
 }
 
-// Wait with a bound; gives up early when the other group has aborted.
+// Scale one thread's 32 entries (columns 32*half ..) of row r of a C x C
+// product by the decay e^{g_r - g_s}, keeping s < r (strict) or s <= r.  Off
+// the diagonal 16-blocks the decay is the product of the two block-boundary
+// factors; only the row's own diagonal block takes exponentials.  Written
+// without lane-dependent branches (rows of one warp span two blocks) so the
+// independent load -> exp -> multiply chains overlap.
+__device__ __forceinline__ void decay_row(float *x, int r, int rb, int half, const float *g,
+                                          const float *colf, const float *rowf, bool incl) {
+    const float gr = g[r];
+    float d[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) d[e] = __expf(gr - g[16 * rb + e]);
+    const float f0 = rowf[4 * r + 2 * half], f1 = rowf[4 * r + 2 * half + 1];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        const int cb = 2 * half + (j >> 4);
+        const int s = 32 * half + j;
+        const float foff = (j < 16 ? f0 : f1) * colf[s];
+        const bool keep = incl ? (s <= r) : (s < r);
+        const float fd = (cb == rb && keep) ? d[j & 15] : 0.f;
+        x[j] *= cb < rb ? foff : fd;
+    }
+}
+
+// Called by one thread per group; the others sleep on a named barrier, so the
+// polling does not compete with the busy warps for issue slots or the shared
+// memory pipe.
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
@@ -109,6 +138,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
             *abort = 1;
             return false;
         }
+        __nanosleep(64);
     }
     return true;
 }
@@ -117,21 +147,27 @@ __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1024-byte aligned base by pointer arithmetic on the shared array (an
+    // integer round trip would lose the address space and turn every access
+    // below into a generic one)
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     float *AF = reinterpret_cast<float *>(sm + OFF_AF);
     float *TF = reinterpret_cast<float *>(sm + OFF_TF);
-    float *g_s = reinterpret_cast<float *>(sm + OFF_ROW);  // cumulative log decay g_r
-    float *b_s = g_s + 64;                                 // beta_r
-    float *bg_s = g_s + 128;                               // beta_r e^{g_r}
+    // Per-chunk gate rows (two buffers, by chunk parity):
+    //   g (cumulative log decay), beta, beta e^{g}; and the decay between tokens
+    //   r > s of different 16-token blocks, factored at the last token e of s's
+    //   block: e^{g_r - g_s} = e^{g_r - g_e} e^{g_e - g_s}, both factors <= 1
+    //   (no overflow, only the underflow the product has too):
+    //   colf[s] = e^{g_e(s) - g_s},  rowf[r][b] = e^{g_r - g_{16b+15}}, b < r/16.
+    auto gate_rows = [&](int st) { return reinterpret_cast<float *>(sm + OFF_ROW + st * ROW_STRIDE); };
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *bar_tma = bars + 0;     // [2] tiles of a stage landed
     uint64_t *bar_l = bars + 2;       // local MMAs done
     uint64_t *bar_s = bars + 3;       // state MMAs done
     uint64_t *bar_vpfree = bars + 4;  // [2] a chunk's state pass is over (its buffers are free)
     uint64_t *bar_ready = bars + 6;   // a chunk's operands are ready for the state pass
-    uint64_t *bar_kqfree = bars + 7;  // the state pass has read Q K^T (D_kq) of a chunk
+    uint64_t *bar_pfree = bars + 7;   // the state pass has consumed P of a chunk
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 64);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 68);
     int *tma_issued = reinterpret_cast<int *>(sm + OFF_BAR + 72);  // [2] loads issued per stage
@@ -160,8 +196,10 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
     }
-    for (int i = tid; i < 512; i += kThreads)
+    for (int i = tid; i < 512; i += kThreads) {
         reinterpret_cast<uint4 *>(sm + OFF_Z)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4 *>(sm + OFF_Z2)[i] = make_uint4(0, 0, 0, 0);
+    }
     fence_proxy_async_smem();
 
     // the state group's registers: thread c holds S[v0 + i][c], i in [0, 64)
@@ -208,19 +246,21 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         int tma_seen0 = 0, tma_seen1 = 0;
         // matrix descriptors: base per buffer, then + (byte offset >> 4) per K step;
         // stage 1 is stage 0 + RAW_STAGE bytes
-        const uint64_t d_qk0 = desc_sw128(sbase + OFF_RAW + RAW_Q, 16, 1024);
+        const uint64_t d_kq0 = desc_sw128(sbase + OFF_RAW + RAW_K, 16, 1024);
         const uint64_t d_kmn0 = desc_sw128(sbase + OFF_RAW + RAW_K, RAW_AC, 1024);
         const uint64_t d_vmn0 = desc_sw128(sbase + OFF_RAW + RAW_V, 8192, 1024);
         const uint64_t d_tg = desc_sw128(sbase + OFF_TG, 16, 1024);
-        const uint64_t d_tb = desc_sw128(sbase + OFF_TB, 16, 1024);
+        const uint64_t d_ztb = desc_sw128(sbase + OFF_Z, 16, 1024);
 
         // wait for chunk m's tiles, zero rows past the sequence end, issue D_kq
         auto start_chunk = [&](int m) -> bool {
             const int st = m & 1;
-            bool ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag);
+            bool ok = true;
+            if (tid == 0) ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag);
             if (st) ++tma_seen1; else ++tma_seen0;
             const int L = chunk_len(m);
             if (L < C) {
+                if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) return false;
                 uint8_t *raw = sm + OFF_RAW + st * RAW_STAGE;
                 for (int idx = tid; idx < (C - L) * 8; idx += kLocal) {
                     const int r = L + (idx >> 3), pj = idx & 7;
@@ -237,12 +277,11 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) return false;
             if (tid == 0) {
                 tc_fence_after();
-                const uint64_t da = d_qk0 + st * (RAW_STAGE >> 4);
+                const uint64_t da = d_kq0 + st * (RAW_STAGE >> 4);
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k) {
                     const uint32_t off = ((k >> 2) * RAW_AC + (k & 3) * 32) >> 4;
-                    mma_bf16(tmem + COL_KQ + 64 * st, da + off, da + off + (RAW_K - RAW_Q) / 16,
-                             ID_KK, k > 0);
+                    mma_bf16(tmem + COL_KQ + 64 * st, da + off, da + off, ID_KK, k > 0);
                 }
                 mma_commit(bar_l);
             }
@@ -250,7 +289,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             return true;
         };
 
-        // gates of the next chunk, prefetched into warp 0's registers
+        // gates of a chunk, prefetched into warp 4's registers one chunk ahead
         float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
         auto load_gates = [&](int m) {
             const long long t0 = t_begin + (long long)m * C;
@@ -260,87 +299,113 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             nbe0 = r0 < L ? a.beta[(t0 + r0) * H + h] : 0.f;
             nbe1 = r1 < L ? a.beta[(t0 + r1) * H + h] : 0.f;
         };
+        // gates of chunk mm (one warp): cumulative log decay, beta and the
+        // factored block decays, into the gate rows of mm's parity
+        auto compute_gates = [&](int mm) {
+            const int st = mm & 1;
+            float *g_s = gate_rows(st), *b_s = g_s + 64, *bg_s = g_s + 128;
+            float *colf_s = g_s + 192, *rowf_s = g_s + 256;
+            const int r0 = 2 * lane, r1 = 2 * lane + 1;
+            const float la0 = nla0, la1 = nla1, be0 = nbe0, be1 = nbe1;
+            if (mm + 1 < nchunks) load_gates(mm + 1);
+            float incl = la0 + la1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const float g1 = incl, g0 = incl - la1;
+            float gend[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) gend[b] = __shfl_sync(0xffffffffu, incl, 8 * b + 7);
+            const int blk = r0 >> 4;
+            const float e0 = __expf(g0), e1 = __expf(g1);
+            const float c0 = __expf(gend[blk] - g0), c1 = __expf(gend[blk] - g1);
+            float f0[3], f1[3];
+#pragma unroll
+            for (int b = 0; b < 3; ++b) {  // unconditional: no divergent exps
+                f0[b] = __expf(fminf(g0 - gend[b], 0.f));
+                f1[b] = __expf(fminf(g1 - gend[b], 0.f));
+            }
+            g_s[r0] = g0; g_s[r1] = g1;
+            b_s[r0] = be0; b_s[r1] = be1;
+            bg_s[r0] = be0 * e0; bg_s[r1] = be1 * e1;
+            colf_s[r0] = c0; colf_s[r1] = c1;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                rowf_s[4 * r0 + b] = b < blk ? f0[b < 3 ? b : 0] : 0.f;
+                rowf_s[4 * r1 + b] = b < blk ? f1[b < 3 ? b : 0] : 0.f;
+            }
+        };
         if (tid == 0) {
             if (nchunks > 0) issue_tma(0);
             if (nchunks > 1) issue_tma(1);
         }
-        if (warp == 0 && nchunks > 0) load_gates(0);
+        if (warp == 4 && nchunks > 0) {
+            load_gates(0);
+            compute_gates(0);
+        }
         bool alive = nchunks > 0 ? start_chunk(0) : true;
 
         for (int m = 0; alive && m < nchunks; ++m) {
             const int st = m & 1;
             uint8_t *raw = sm + OFF_RAW + st * RAW_STAGE;
-            float *hand = reinterpret_cast<float *>(sm + OFF_HAND + st * HAND_STRIDE);
+            const float *g_s = gate_rows(st), *b_s = g_s + 64, *bg_s = g_s + 128;
+            const float *colf_s = g_s + 192, *rowf_s = g_s + 256;
             bool ok = true;
 
-            // ---- gates (warp 0), once the state pass of chunk m-2 is over ------
-            if (warp == 0) {
-                if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag);
-                const int r0 = 2 * lane, r1 = 2 * lane + 1;
-                const float la0 = nla0, la1 = nla1, be0 = nbe0, be1 = nbe1;
-                if (m + 1 < nchunks) load_gates(m + 1);
-                float incl = la0 + la1;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (lane >= off) incl += y;
-                }
-                const float gC = __shfl_sync(0xffffffffu, incl, 31);
-                const float g1 = incl, g0 = incl - la1;
-                const float e0 = __expf(g0), e1 = __expf(g1);
-                g_s[r0] = g0; g_s[r1] = g1;
-                b_s[r0] = be0; b_s[r1] = be1;
-                bg_s[r0] = be0 * e0; bg_s[r1] = be1 * e1;
-                hand[r0] = g0; hand[r1] = g1;                               // g
-                hand[64 + r0] = e0; hand[64 + r1] = e1;                     // e^{g}
-                hand[128 + r0] = __expf(gC - g0); hand[128 + r1] = __expf(gC - g1);  // e^{gC-g}
-                if (lane == 0) hand[192] = __expf(gC);
-            }
             // ---- D_kq of this chunk ----------------------------------------------
-            ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
+            if (tid == 0) ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
             ++bl_wait;
-            tc_fence_after();
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
-            // A rows (K K^T: TMEM lanes 64-127), this thread's half of the columns
+            tc_fence_after();
+            // A rows (K K^T: TMEM lanes 0-63, sub-partitions 0-1) and, at the same
+            // time on sub-partitions 2-3, P rows (Q K^T: lanes 64-127), kept in
+            // registers as bf16 until the state pass frees the P slot.
+            uint4 p_hold[4];
             if (lq >= 2) {
                 float x[32];
                 tmem_load<32>(tmem + lane_off + COL_KQ + 64 * st + 32 * lhalf, x);
                 const int r = 32 * (lq - 2) + lane;
-                const float gr = g_s[r], br = b_s[r];
+                decay_row(x, r, r >> 4, lhalf, g_s, colf_s, rowf_s, true);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) p_hold[j] = pack8(x + 8 * j);
+            }
+            if (lq < 2) {
+                float x[32];
+                tmem_load<32>(tmem + lane_off + COL_KQ + 64 * st + 32 * lhalf, x);
+                const int r = 32 * lq + lane, br_blk = r >> 4;
+                decay_row(x, r, br_blk, lhalf, g_s, colf_s, rowf_s, false);
+                const float br = b_s[r];
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    float4 y;
-                    const int s = 32 * lhalf + j;
-                    y.x = s + 0 < r ? br * __expf(gr - g_s[s + 0]) * x[j + 0] : 0.f;
-                    y.y = s + 1 < r ? br * __expf(gr - g_s[s + 1]) * x[j + 1] : 0.f;
-                    y.z = s + 2 < r ? br * __expf(gr - g_s[s + 2]) * x[j + 2] : 0.f;
-                    y.w = s + 3 < r ? br * __expf(gr - g_s[s + 3]) * x[j + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(AF + r * LDA + s) = y;
+                    const float4 y = make_float4(br * x[j], br * x[j + 1], br * x[j + 2], br * x[j + 3]);
+                    *reinterpret_cast<float4 *>(AF + r * LDA + 32 * lhalf + j) = y;
                 }
             }
             named_bar_sync(BAR_LOCAL, kLocal);
             // ---- T = (I + A)^{-1} ------------------------------------------------
+            // meanwhile warp 4 prepares the next chunk's gates (during the
+            // diagonal blocks and the 32x32 level, which need warps 0-3 only)
+            if (warp == 4 && m + 1 < nchunks) compute_gates(m + 1);
             // (1) 16x16 diagonal blocks: warp w < 4 inverts block w; lane j < 16
-            //     owns column j and runs the forward substitution in registers.
+            //     owns column j.  Right-looking forward substitution: once t_m
+            //     is final it is eliminated from every later row, so the chain
+            //     of dependent operations is one FMA per row.
             if (warp < 4 && lane < 16) {
                 const int o = 16 * warp, j = lane;
                 float t[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    float arow[16];
+                for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4)
-                        *reinterpret_cast<float4 *>(arow + 4 * q4) =
-                            *reinterpret_cast<const float4 *>(AF + (o + i) * LDA + o + 4 * q4);
-                    float acc = (i == j) ? 1.f : 0.f;
+                for (int mm = 0; mm < 15; ++mm) {
 #pragma unroll
-                    for (int mm = 0; mm < i; ++mm) acc -= arow[mm] * t[mm];
-                    t[i] = acc;
+                    for (int i = mm + 1; i < 16; ++i) t[i] -= AF[(o + i) * LDA + o + mm] * t[mm];
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) TF[(o + i) * LDA + o + j] = t[i];
             }
-            named_bar_sync(BAR_LOCAL, kLocal);
+            if (warp < 4) named_bar_sync(BAR_INV, 128);
             const int fg = lane >> 2, ft = lane & 3;  // mma.sync fragment coordinates
             // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00) and T_32 = -T_33 (A_32 T_22);
             //     warp w < 4: half w/2, 8 output columns (w%2).  X goes to the
@@ -451,9 +516,11 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_LOCAL, kLocal);
-            // ---- D_w = [T_bg; T_b] K (rows 0-63: W);  D_vp = [T_b; 0] V ----------
+            // ---- D_w = [T_bg; 0] K (rows 0-63: W);  D_vp = [0; T_b] V --------------
+            // (D_vp of this parity and its handoff slot are free once the state
+            // pass of chunk m-2 is over)
             if (tid == 0) {
-                if (m >= 1) ok &= wait_bar(bar_kqfree, (uint32_t)((m - 1) & 1), abort_flag);
+                if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag);
                 tc_fence_after();
                 const uint64_t dk = d_kmn0 + st * (RAW_STAGE >> 4);
                 const uint64_t dv = d_vmn0 + st * (RAW_STAGE >> 4);
@@ -462,14 +529,32 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     mma_bf16(tmem + COL_W, d_tg + k * 2, dk + k * 128, ID_W, k > 0);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tmem + COL_VP + 64 * st, d_tb + k * 2, dv + k * 128, ID_KM, k > 0);
+                    mma_bf16(tmem + COL_VP + 64 * st, d_ztb + k * 2, dv + k * 128, ID_KM, k > 0);
                 mma_commit(bar_l);
             }
             ++bl_commit;
-            ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
+            // ---- while those run: store P once the state pass has consumed the
+            //      previous chunk's P ------------------------------------------------
+            if (tid == 0 && m >= 1) ok &= wait_bar(bar_pfree, (uint32_t)((m - 1) & 1), abort_flag);
+            if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
+            if (lq >= 2) {
+                const int r = 32 * (lq - 2) + lane;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    *reinterpret_cast<uint4 *>(sm + OFF_P + sw128(r, 4 * lhalf + j)) = p_hold[j];
+            } else if (warp == 5) {  // g and g_C for the state pass of this chunk
+                float *hand = reinterpret_cast<float *>(sm + OFF_HAND + st * HAND_STRIDE);
+                hand[2 * lane] = g_s[2 * lane];
+                hand[2 * lane + 1] = g_s[2 * lane + 1];
+                if (lane == 0) hand[64] = g_s[63];
+            }
+            if (tid == 0) ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
             ++bl_wait;
+            if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
             tc_fence_after();
-            // ---- -W into rows 0-63 of the stage (K-major, atom column lhalf) ------
+            // ---- the next chunk's D_kq, so that it overlaps the rest of this one
+            if (m + 1 < nchunks && !start_chunk(m + 1)) break;
+            // ---- -W into its rows of the stage (K-major, atom column lhalf) ------
             if (lq < 2) {
                 float w[64];
                 tmem_load<64>(tmem + lane_off + COL_W + 64 * lhalf, w);  // lane r: W[r][c]
@@ -478,14 +563,12 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 for (int j = 0; j < 64; ++j) w[j] = -w[j];
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    *reinterpret_cast<uint4 *>(raw + lhalf * RAW_AC + sw128(r, j)) = pack8(w + 8 * j);
+                    *reinterpret_cast<uint4 *>(raw + lhalf * RAW_AC + RAW_W + sw128(r, j)) = pack8(w + 8 * j);
             }
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
             if (tid == 0) mbar_arrive(bar_ready);
-            // ---- start the next chunk's D_kq ------------------------------------
-            if (m + 1 < nchunks && !start_chunk(m + 1)) break;
         }
         // drain what this group launched
         if (*abort_flag && tid == 0)
@@ -495,25 +578,27 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         const int sq = warp & 3;  // TMEM lane quadrant = warp - 8
         const uint32_t lane_off = (uint32_t)(32 * sq) << 16;
         uint32_t bs_wait = 0, bs_commit = 0;
-        const uint64_t d_wq0 = desc_sw128(sbase + OFF_RAW, 16, 1024);
+        const uint64_t d_qw0 = desc_sw128(sbase + OFF_RAW + RAW_Q, 16, 1024);
         const uint64_t d_kmn0 = desc_sw128(sbase + OFF_RAW + RAW_K, RAW_AC, 1024);
         const uint64_t d_sb = desc_sw128(sbase + OFF_SB, 16384, 1024);
         const uint64_t d_vp = desc_sw128(sbase + OFF_VP, 8192, 1024);
         const uint64_t d_vh = desc_sw128(sbase + OFF_VH, 8192, 1024);
-        const uint64_t d_z = desc_sw128(sbase + OFF_Z, 16, 1024);
+        const uint64_t d_pz = desc_sw128(sbase + OFF_P, 16, 1024);
         for (int m = 0; m < nchunks; ++m) {
             const int st = m & 1;
             const long long t0 = t_begin + (long long)m * C;
             const int L = chunk_len(m);
             const float *hand = reinterpret_cast<const float *>(sm + OFF_HAND + st * HAND_STRIDE);
-            bool ok = wait_bar(bar_ready, (uint32_t)(m & 1), abort_flag);
-            tc_fence_after();
+            bool ok = true;
+            if (tid == kLocal) ok = wait_bar(bar_ready, (uint32_t)(m & 1), abort_flag);
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
-            const float dec = hand[192];
-            // ---- D_vp += [-W; Q] S^T ----------------------------------------------
+            tc_fence_after();
+            const float gC = hand[64];
+            const float dec = __expf(gC);
+            // ---- D_vp += [Q; -W] S^T ----------------------------------------------
             if (tid == kLocal) {
                 tc_fence_after();
-                const uint64_t da = d_wq0 + st * (RAW_STAGE >> 4);
+                const uint64_t da = d_qw0 + st * (RAW_STAGE >> 4);
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k)
                     mma_bf16(tmem + COL_VP + 64 * st, da + (((k >> 2) * RAW_AC + (k & 3) * 32) >> 4),
@@ -521,36 +606,16 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 mma_commit(bar_s);
             }
             ++bs_commit;
-            // ---- meanwhile: P from Q K^T (TMEM lanes 0-63) -------------------------
-            if (sq < 2) {
-                const int r = 32 * sq + lane;
-                const float gr = hand[r];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float x[32];
-                    tmem_load<32>(tmem + lane_off + COL_KQ + 64 * st + 32 * hh, x);
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int s = 32 * hh + j;
-                        x[j] = s <= r ? __expf(gr - hand[s]) * x[j] : 0.f;
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4 *>(sm + OFF_P + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
-                }
-            }
-            tc_fence_before();
-            named_bar_sync(BAR_STATE, kState);
-            if (tid == kLocal) mbar_arrive(bar_kqfree);
-            ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
+            if (tid == kLocal) ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
             ++bs_wait;
+            if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
             tc_fence_after();
-            // ---- V' (rows 0-63) and kh . V' as MN-major operands ------------------
-            if (sq < 2) {
+            // ---- V' (rows 64-127) and kh . V' as MN-major operands ----------------
+            if (sq >= 2) {
                 float vp[64];
                 tmem_load<64>(tmem + lane_off + COL_VP + 64 * st, vp);
-                const int r = 32 * sq + lane;
-                const float khr = hand[128 + r];
+                const int r = 32 * (sq - 2) + lane;
+                const float khr = __expf(gC - hand[r]);
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
                     *reinterpret_cast<uint4 *>(sm + OFF_VP + sw128(r, j)) = pack8(vp + 8 * j);
@@ -563,7 +628,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
-            // ---- D_ds = K^T (kh . V');  D_o = [0; P] V' ----------------------------
+            // ---- D_ds = K^T (kh . V');  D_o = [P; 0] V' ----------------------------
             if (tid == kLocal) {
                 tc_fence_after();
                 const uint64_t dk = d_kmn0 + st * (RAW_STAGE >> 4);
@@ -572,12 +637,14 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     mma_bf16(tmem + COL_DS, dk + k * 128, d_vh + k * 128, ID_MM, k > 0);
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tmem + COL_O, d_z + k * 2, d_vp + k * 128, ID_KM, k > 0);
+                    mma_bf16(tmem + COL_O, d_pz + k * 2, d_vp + k * 128, ID_KM, k > 0);
                 mma_commit(bar_s);
+                mma_commit(bar_pfree);
             }
             ++bs_commit;
-            ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
+            if (tid == kLocal) ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
             ++bs_wait;
+            if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
             tc_fence_after();
             // the stage is free: load chunk m+2 into it
             if (tid == kLocal && ok && m + 2 < nchunks) issue_tma(m + 2);
@@ -592,9 +659,9 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4 *>(sm + OFF_SB + sw128(c_st, j)) = pack8(s_reg + 8 * j);
-            if (sq >= 2) {
-                const int r = 32 * (sq - 2) + lane;
-                const float er = hand[64 + r];
+            if (sq < 2) {
+                const int r = 32 * sq + lane;
+                const float er = __expf(hand[r]);
                 __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.o) +
                                      ((t0 + r) * H + h) * (long long)a.dv + v0;
 #pragma unroll

@@ -204,11 +204,10 @@ __device__ __forceinline__ void mma_commit(uint64_t *bar) {
 // g = lane / 4, t = lane % 4;  A (16x8): a0 (g, t), a1 (g+8, t), a2 (g, t+4),
 // a3 (g+8, t+4);  B (8x8): b0 (t, g), b1 (t+4, g);  C (16x8): c0 (g, 2t),
 // c1 (g, 2t+1), c2 (g+8, 2t), c3 (g+8, 2t+1).
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
+// fp32 bits used directly as a tf32 operand: the MMA reads the sign, exponent
+// and the top 10 mantissa bits (truncation, relative error < 2^-10), which
+// keeps the conversion off the special-function pipe.
+__device__ __forceinline__ uint32_t to_tf32(float x) { return __float_as_uint(x); }
 __device__ __forceinline__ void mma_tf32_16x8x8(float *d, const uint32_t *a, const uint32_t *b) {
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
