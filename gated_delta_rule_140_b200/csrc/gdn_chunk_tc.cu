@@ -112,8 +112,13 @@ __device__ __forceinline__ void decay_row(float *x, int r, int rb, int half, con
                                           const float *colf, const float *rowf, bool incl) {
     const float gr = g[r];
     float d[16];
+    if ((rb >> 1) == half) {  // uniform per warp: a warp's rows share rb >> 1
 #pragma unroll
-    for (int e = 0; e < 16; ++e) d[e] = __expf(gr - g[16 * rb + e]);
+        for (int e = 0; e < 16; ++e) d[e] = __expf(gr - g[16 * rb + e]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) d[e] = 0.f;
+    }
     const float f0 = rowf[4 * r + 2 * half], f1 = rowf[4 * r + 2 * half + 1];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
@@ -252,11 +257,14 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         const uint64_t d_tg = desc_sw128(sbase + OFF_TG, 16, 1024);
         const uint64_t d_ztb = desc_sw128(sbase + OFF_Z, 16, 1024);
 
-        // wait for chunk m's tiles, zero rows past the sequence end, issue D_kq
-        auto start_chunk = [&](int m) -> bool {
+        // wait for chunk m's tiles, zero rows past the sequence end, issue D_kq.
+        // The tile wait and the MMA issue (which blocks its thread for a few
+        // hundred cycles) are done by `issuer`, a thread whose warp has nothing
+        // else to do at that point.
+        auto start_chunk = [&](int m, int issuer) -> bool {
             const int st = m & 1;
             bool ok = true;
-            if (tid == 0) ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag);
+            if (tid == issuer) ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag);
             if (st) ++tma_seen1; else ++tma_seen0;
             const int L = chunk_len(m);
             if (L < C) {
@@ -275,7 +283,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 fence_proxy_async_smem();
             }
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) return false;
-            if (tid == 0) {
+            if (tid == issuer) {
                 tc_fence_after();
                 const uint64_t da = d_kq0 + st * (RAW_STAGE >> 4);
 #pragma unroll
@@ -345,7 +353,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             load_gates(0);
             compute_gates(0);
         }
-        bool alive = nchunks > 0 ? start_chunk(0) : true;
+        bool alive = nchunks > 0 ? start_chunk(0, 0) : true;
 
         for (int m = 0; alive && m < nchunks; ++m) {
             const int st = m & 1;
@@ -519,7 +527,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             // ---- D_w = [T_bg; 0] K (rows 0-63: W);  D_vp = [0; T_b] V --------------
             // (D_vp of this parity and its handoff slot are free once the state
             // pass of chunk m-2 is over)
-            if (tid == 0) {
+            if (tid == 4 * 32) {  // warp 4 is idle during the P stores below
                 if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag);
                 tc_fence_after();
                 const uint64_t dk = d_kmn0 + st * (RAW_STAGE >> 4);
@@ -553,7 +561,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
             tc_fence_after();
             // ---- the next chunk's D_kq, so that it overlaps the rest of this one
-            if (m + 1 < nchunks && !start_chunk(m + 1)) break;
+            if (m + 1 < nchunks && !start_chunk(m + 1, 6 * 32)) break;
             // ---- -W into its rows of the stage (K-major, atom column lhalf) ------
             if (lq < 2) {
                 float w[64];
