@@ -364,9 +364,11 @@ def run_ours(args, rank, world, local):
         pre_s, dec_s = pre_ms / K / 1e3, dec_ms / K / 1e3
         path = nat.chunk_fwd_path(nat.prefill_dims(xp["q"], xp["v"], xp["log_alpha"],
                                                    xp["cu_seqlens"]))
-        pre_kernel = "chunk_tc_kernel" if path == "tensor_core" else "chunk_simt_kernel"
-        pre_src = ("gated_delta_rule_140_b200/csrc/gdn_chunk_tc.cu" if pre_kernel == "chunk_tc_kernel"
-                   else "gated_delta_rule_140_b200/csrc/gdn_chunk_simt.cu")
+        pre_kernel, pre_src = {
+            "tensor_core_pair": ("chunk_pair_kernel", "gdn_chunk_pair.cu"),
+            "tensor_core": ("chunk_tc_kernel", "gdn_chunk_tc.cu"),
+        }.get(path, ("chunk_simt_kernel", "gdn_chunk_simt.cu"))
+        pre_src = "gated_delta_rule_140_b200/csrc/" + pre_src
         roof_pre = {"bound": "hbm", "achieved": pbytes / pre_s / 1e9, "peak": hbm,
                     "unit": "GB/s", "frac": pbytes / pre_s / 1e9 / hbm,
                     "traffic": traffic_for(pre_kernel, pre_src), "kernel": pre_kernel,

@@ -21,7 +21,7 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     if (d->d_k <= 0 || d->d_v <= 0) return GDN_ERR_INVALID;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
         return GDN_ERR_UNSUPPORTED;
-    if ((d->flags & ~GDN_FLAG_CUDA_CORES) != 0) return GDN_ERR_INVALID;
+    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR)) != 0) return GDN_ERR_INVALID;
     if (prefill && d->n_seqs < 0) return GDN_ERR_INVALID;
     // every index the kernels form must fit in 63 bits; keep the token axis sane
     if ((long long)d->B * d->T * d->H * (d->d_k > d->d_v ? d->d_k : d->d_v) > (1LL << 40))
@@ -29,8 +29,14 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     return GDN_OK;
 }
 
-bool use_tensor_cores(const gdn_dims &d) {
-    return !(d.flags & GDN_FLAG_CUDA_CORES) && gdn::chunk_tc_supported(d);
+enum class Path { kPair, kOneCta, kCudaCores };
+
+// The prefill kernel a call runs: the single-CTA tensor-core kernel by
+// default, the two-CTA one with GDN_FLAG_PAIR, the fp32 CUDA-core kernel for
+// every other shape or with GDN_FLAG_CUDA_CORES.
+Path select_path(const gdn_dims &d) {
+    if ((d.flags & GDN_FLAG_CUDA_CORES) || !gdn::chunk_tc_supported(d)) return Path::kCudaCores;
+    return (d.flags & GDN_FLAG_PAIR) ? Path::kPair : Path::kOneCta;
 }
 
 int prefill_seqs(const gdn_dims &d, const int32_t *cu_seqlens) {
@@ -43,7 +49,10 @@ extern "C" {
 
 size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims) {
     if (check_dims(dims, true) != GDN_OK) return 0;
-    size_t extra = use_tensor_cores(*dims) ? gdn::chunk_tc_scratch_bytes(*dims) : 0;
+    const Path p = select_path(*dims);
+    size_t extra = p == Path::kPair     ? gdn::chunk_pair_scratch_bytes(*dims)
+                   : p == Path::kOneCta ? gdn::chunk_tc_scratch_bytes(*dims)
+                                        : 0;
     return gdn::kWorkspaceHeader + ((extra + 255) & ~size_t(255));
 }
 
@@ -86,8 +95,10 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
     if (n_seqs == 0) return GDN_OK;
     int launches = 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = use_tensor_cores(d) ? gdn::launch_chunk_tc(a, s, &launches)
-                                        : gdn::launch_chunk_simt(a, s, &launches);
+    const Path p = select_path(d);
+    cudaError_t e = p == Path::kPair     ? gdn::launch_chunk_pair(a, s, &launches)
+                    : p == Path::kOneCta ? gdn::launch_chunk_tc(a, s, &launches)
+                                         : gdn::launch_chunk_simt(a, s, &launches);
     g_launches.fetch_add(launches, std::memory_order_relaxed);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
@@ -136,12 +147,17 @@ gdn_status gdn_workspace_status(void *workspace, gdn_stream_t stream) {
     if (word == 0) return GDN_OK;
     if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return GDN_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return GDN_ERR_CUDA;
+    if (word & gdn::kErrInternal) return GDN_ERR_CUDA;
     return (word & gdn::kErrTimeout) ? GDN_ERR_TIMEOUT : GDN_ERR_DEVICE_INPUT;
 }
 
 const char *gdn_chunk_fwd_path(const gdn_dims *dims) {
     if (check_dims(dims, true) != GDN_OK) return nullptr;
-    return use_tensor_cores(*dims) ? "tensor_core" : "cuda_core";
+    switch (select_path(*dims)) {
+        case Path::kPair: return "tensor_core_pair";
+        case Path::kOneCta: return "tensor_core";
+        default: return "cuda_core";
+    }
 }
 
 const char *gdn_status_string(gdn_status status) {

@@ -1,0 +1,938 @@
+// gdn_chunk_pair.cu -- chunkwise gated delta rule prefill on the tensor cores
+// with the chunk-local work and the sequential state pass on two different
+// SMs: one 2-CTA cluster per (sequence, head), bf16 inputs, d_k = d_v = 128,
+// scalar (GDN) decay.
+//
+// Chunkwise form (FG2-GDN paper, section 3.6: WY representation, UT transform,
+// inter-chunk state propagation; Gated Delta Networks page, section 3.3, for
+// the cumulative decay g_r within a chunk, gamma_r = e^{g_r}), C = 64 tokens:
+//
+//   A_rs = beta_r e^{g_r-g_s} k_r.k_s (s < r),  T = (I + A)^{-1}
+//   P_rs = e^{g_r-g_s} q_r.k_s (s <= r)
+//   T_b = T diag(beta),  T_bg = T diag(beta gamma),  W = T_bg K,  U = T_b V
+//   V'  = U - W S^T,     o = gamma Q S^T + P V',
+//   S  <- e^{g_C} S + V'^T (kh . K),  kh_s = e^{g_C - g_s}.
+//
+// The output is regrouped so that it needs nothing after the state product:
+//   o = (gamma Q - P W) S^T + (P T_b) V = Qh S^T + R V
+// and one accumulator per chunk (M = 128) holds both halves of the pass:
+//   D = [Qh; -W] S^T + [R; T_b] V  ->  rows 0-63: o,  rows 64-127: V'.
+// The state update needs V' only through  dS = (kh . K)^T V' = Kt^T V'.
+//
+// Rank 0 ("local" CTA) computes, per chunk, everything that depends only on
+// the chunk's tokens: A, T (fp32, tf32 MMAs for the off-diagonal blocks), P,
+// T_b, T_bg, P T_bg and R = P T_b (one MMA), [W; P W] = [T_bg; P T_bg] K (one
+// MMA), and writes Kt, Qh, -W, R, T_b as bf16 tiles in the swizzled layout the
+// state CTA's MMAs read, into a 2-slot ring in global memory (L2-resident: it
+// is rewritten every other chunk).  Two groups of 8 warps work on two chunks at
+// once (even / odd chunks, ring slot = chunk parity).
+// Rank 1 ("state" CTA) holds S (fp32, registers) for all 128 value channels as
+// two independent halves of 64, each with its own chain of warps, loads each
+// chunk's ring slot and V tile (bulk copy + TMA), and per chunk and half
+// issues D = [R;T_b] V_h + [Qh;-W] S_h^T, writes o, converts V' to bf16 and
+// issues dS = Kt^T V'.
+// The CTAs signal each other with mbarriers (ring slot written / ring slot
+// read).  Every wait is bounded: on expiry the CTA records kErrTimeout, raises
+// the abort flag of both CTAs, drains what it issued and leaves through the
+// final cluster barrier.
+#include "gdn_internal.cuh"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int C = kChunk;  // 64
+constexpr int DK = 128, DV = 128;
+constexpr int kThreads = 512;
+constexpr long long kWaitLimit = 1LL << 31;  // SM cycles (~1 s)
+constexpr int LDA = 68;                      // fp32 row stride of A and T
+
+// ---- ring slot / state-CTA stage layout (bytes, 1024-aligned tiles) --------
+// per atom column a (d_k 64a .. 64a+63):  [Kt rows 0-63 | Qh rows | -W rows]
+constexpr uint32_t SG_KT = 0, SG_QH = 8192, SG_MW = 16384, SG_AC = 24576;
+constexpr uint32_t SG_R = 49152, SG_TB = 57344;  // [R; T_b]  (A of the V product)
+constexpr uint32_t RING_SLOT = 65536;            // ring slot = stage bytes [0, 64K)
+constexpr uint32_t SG_V = 65536;                 // V tiles, d_v halves at +8K
+constexpr uint32_t S_STAGE = 81920;
+constexpr uint32_t S_STAGE_TX = RING_SLOT + 2 * 8192;
+constexpr uint32_t S_OFF_SB = 2 * S_STAGE;       // S_h^T bf16, MN-major [c][i], 16 KB per half
+constexpr uint32_t S_OFF_VP = S_OFF_SB + 2 * 16384;  // V'_h bf16, MN-major [r][i], 8 KB per half
+
+// ---- local-CTA group layout ---------------------------------------------------
+constexpr uint32_t L_RAW = 0;          // [K0 | Q0 | K1 | Q1], 8 KB each (TMA)
+constexpr uint32_t L_RAW_AC = 16384;   //   atom column stride: [K_a; Q_a] is an M=128 tile
+constexpr uint32_t L_PZT = 32768;      // [P | 0 | T_bg | P T_bg | T_b], 8 KB each
+constexpr uint32_t PZ_P = 0, PZ_Z = 8192, PZ_TG = 16384, PZ_PTG = 24576, PZ_TB = 32768;
+constexpr uint32_t L_AF = 73728;                   // A fp32 [64][LDA]
+constexpr uint32_t L_TF = L_AF + 64 * LDA * 4;     // T fp32 [64][LDA]
+constexpr uint32_t L_GATES = L_TF + 64 * LDA * 4;  // two gate-row buffers
+constexpr uint32_t GATES_STRIDE = 3072;
+constexpr uint32_t L_GROUP = 114688;
+static_assert(L_GATES + 2 * GATES_STRIDE <= L_GROUP, "local group layout");
+// gate rows (floats): g[64] beta[64] beta*gamma[64] colf[64] rowf[64][4] kh[64] gamma[64] dec
+constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
+              GR_GAM = 576, GR_DEC = 640;
+
+// ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
+constexpr uint32_t OFF_COMMON = 2 * L_GROUP;  // 229376
+static_assert(S_OFF_VP + 2 * 8192 <= OFF_COMMON, "state layout");
+constexpr uint32_t CM_ABORT = 0, CM_SLOT = 4, CM_TMEM = 8, CM_MDEC = 16, CM_SDEC = 24,
+                   CM_ISSUED = 32, CM_CDEC = 40, CM_BARS = 64;
+constexpr uint32_t SMEM_USED = OFF_COMMON + CM_BARS + 16 * 8;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+// state-CTA mbarriers
+constexpr int SB_FULL = 0, SB_READY = 2, SB_VO = 4, SB_DS = 6, SB_OFREE = 8, SB_CONS = 12,
+              SB_DRAIN = 14;
+// local-CTA mbarriers
+constexpr int LB_TMA = 0, LB_L = 2, LB_SLOTFREE = 4, LB_DRAIN = 6;
+
+// TMEM columns
+constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_GROUP = 192;  // local: per group
+constexpr uint32_t TM_DS = 256;                            // state: D_vo[st][h] at 64 (2st+h)
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);   // [K;Q] K^T
+constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, true); // [P;0][T_bg|T_b], [T_bg;PT_bg] K
+constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, true);   // [R;T_b] V_h, [Qh;-W] S_h^T
+constexpr uint32_t ID_MM = idesc_bf16(128, 64, true, true);     // Kt^T V'_h
+
+__device__ __forceinline__ uint4 pack8(const float *x) {
+    uint4 u;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(x[0], x[1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(x[2], x[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(x[4], x[5]);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(x[6], x[7]);
+    u.x = *reinterpret_cast<uint32_t *>(&h0);
+    u.y = *reinterpret_cast<uint32_t *>(&h1);
+    u.z = *reinterpret_cast<uint32_t *>(&h2);
+    u.w = *reinterpret_cast<uint32_t *>(&h3);
+    return u;
+}
+__device__ __forceinline__ void unpack8(uint4 u, float *x) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Decay of 32 entries (columns 32*half ..) of row r of a C x C product,
+// e^{g_r - g_s} for s < r (strict) or s <= r.  rq = r / 32 is uniform per warp,
+// so each warp takes one of three branches: the diagonal 32x32 block (exact
+// exponentials, g_r - g_s <= 0 wherever kept, masked elsewhere), a block
+// strictly below it (factored at the 16-block boundary: e^{g_r - g_e} e^{g_e - g_s},
+// both factors <= 1), or a block above it (not called: nothing to keep).
+__device__ __forceinline__ void decay_row(float *x, int r, int rq, int half, const float *gr,
+                                          bool incl) {
+    const float *g = gr + GR_G;
+    if (rq == half) {
+        const float g_r = g[r];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 gs = *reinterpret_cast<const float4 *>(g + 32 * half + 4 * j4);
+            const float gv[4] = {gs.x, gs.y, gs.z, gs.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int j = 4 * j4 + e, s = 32 * half + j;
+                const bool keep = incl ? (s <= r) : (s < r);
+                const float d = __expf(g_r - gv[e]);
+                x[j] = keep ? x[j] * d : 0.f;
+            }
+        }
+    } else {
+        const float *colf = gr + GR_COLF + 32 * half;
+        const float f0 = gr[GR_ROWF + 4 * r + 2 * half], f1 = gr[GR_ROWF + 4 * r + 2 * half + 1];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 c = *reinterpret_cast<const float4 *>(colf + 4 * j4);
+            const float f = j4 < 4 ? f0 : f1;
+            const float2 lo = __fmul2_rn(make_float2(x[4 * j4], x[4 * j4 + 1]), make_float2(f * c.x, f * c.y));
+            const float2 hi = __fmul2_rn(make_float2(x[4 * j4 + 2], x[4 * j4 + 3]), make_float2(f * c.z, f * c.w));
+            x[4 * j4] = lo.x; x[4 * j4 + 1] = lo.y; x[4 * j4 + 2] = hi.x; x[4 * j4 + 3] = hi.y;
+        }
+    }
+}
+
+struct Waiter {
+    volatile int *abort;
+    uint32_t peer_abort;  // shared::cluster address of the peer's abort flag
+    __device__ __forceinline__ void raise() const {
+        *abort = 1;
+        st_peer_u32(peer_abort, 1u);
+    }
+    // Bounded wait for a phase completed inside this CTA (MMA commits, TMA).
+    __device__ __forceinline__ bool wait(uint64_t *bar, uint32_t parity) const {
+        if (mbar_try_wait(bar, parity)) return true;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(bar, parity)) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitLimit) {
+                raise();
+                return false;
+            }
+            __nanosleep(32);
+        }
+        return true;
+    }
+    // Bounded wait for a phase completed by the peer CTA (acquire at cluster scope).
+    __device__ __forceinline__ bool wait_peer(uint64_t *bar, uint32_t parity) const {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        const long long t0 = clock64();
+        while (!mbar_try_wait_cluster(bar, parity)) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitLimit) {
+                raise();
+                return false;
+            }
+            __nanosleep(32);
+        }
+        return true;
+    }
+    // One lane waits, the warp gets the answer.
+    __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int lane) const {
+        bool ok = true;
+        if (lane == 0) ok = wait(bar, parity);
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  uint8_t *ring, int ring_slots) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    uint8_t *cm = sm + OFF_COMMON;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(cm + CM_ABORT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(cm + CM_BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cm + CM_TMEM);
+    int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // [2] loads issued per stage / group
+
+    const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int item = blockIdx.x >> 1;
+    const int h = item % a.H;
+    const int n = item / a.H;
+    const int H = a.H;
+    long long t_begin, t_end;
+    seq_range(a, n, &t_begin, &t_end);
+    const int nchunks = (int)((t_end - t_begin + C - 1) / C);
+    const size_t st_base = ((size_t)n * H + h) * DV * DK;
+    auto chunk_len = [&](int m) -> int {
+        const long long rem = t_end - (t_begin + (long long)m * C);
+        return rem < C ? (int)rem : C;
+    };
+
+    if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
+    if (tid == 0) {
+        for (int i = 0; i < 16; ++i) mbar_init(bars + i, (rank == 1 && (i == SB_CONS || i == SB_CONS + 1)) ? 2 : 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+        issued[0] = issued[1] = 0;
+        if (rank == 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+        } else {
+            tma_prefetch_desc(&tm_v);
+        }
+    }
+    cluster_sync();  // both CTAs' barriers and flags are initialised
+    if (rank == 1 && tid == 0) {
+        // the ring slot pair of this cluster: indexed by the state CTA's SM,
+        // which no other running cluster shares
+        const int slot = (int)sm_id();
+        const int v = slot < ring_slots ? slot : -1;
+        *reinterpret_cast<volatile int *>(cm + CM_SLOT) = v;
+        st_peer_u32(map_peer(sbase + OFF_COMMON + CM_SLOT, peer), (uint32_t)v);
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int slot = *reinterpret_cast<volatile int *>(cm + CM_SLOT);
+    const Waiter wt{abort_flag, map_peer(sbase + OFF_COMMON + CM_ABORT, peer)};
+    if (slot < 0) {
+        if (tid == 0) {
+            atomicOr(a.err, kErrInternal);
+            *abort_flag = 1;
+        }
+    }
+    uint8_t *ring_pair = slot >= 0 ? ring + (size_t)slot * 2 * RING_SLOT : ring;
+
+    if (slot >= 0 && rank == 0) {
+        // ============================ local CTA ============================
+        const int g = warp >> 3, lw = warp & 7, lq = warp & 3, lhalf = lw >> 2;
+        const int gtid = tid & 255;
+        const int BAR_G = 1 + g, BAR_INV = 3 + g;
+        uint8_t *grp = sm + g * L_GROUP;
+        const uint32_t gbase = sbase + g * L_GROUP;
+        uint8_t *raw = grp + L_RAW;
+        uint8_t *pzt = grp + L_PZT;
+        float *AF = reinterpret_cast<float *>(grp + L_AF);
+        float *TF = reinterpret_cast<float *>(grp + L_TF);
+        uint64_t *bar_tma = bars + LB_TMA + g, *bar_l = bars + LB_L + g;
+        uint64_t *bar_slotfree = bars + LB_SLOTFREE + g;
+        uint8_t *ring_slot = ring_pair + (size_t)g * RING_SLOT;
+        const uint32_t peer_ready = map_peer(smem_u32(bars + SB_READY + g), peer);
+        const uint32_t peer_mdec = map_peer(sbase + OFF_COMMON + CM_MDEC + 4 * g, peer);
+        const uint32_t tm_kq = tmem + g * TM_GROUP + TM_KQ, tm_ab = tmem + g * TM_GROUP + TM_AB;
+        const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
+        const uint64_t d_kq = desc_sw128(gbase + L_RAW, 16, 1024);
+        const uint64_t d_kmn = desc_sw128(gbase + L_RAW, L_RAW_AC, 1024);
+        const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);
+        const uint64_t d_tgtb = desc_sw128(gbase + L_PZT + PZ_TG, PZ_TB - PZ_TG, 1024);
+        const uint64_t d_tgptg = desc_sw128(gbase + L_PZT + PZ_TG, 16, 1024);
+        uint32_t bl_wait = 0;
+        const bool issuer = gtid == 0;      // tile loads and MMAs
+        const bool storer = gtid == 7 * 32;  // ring stores and the hand-off
+        bool pend = false;                   // storer: a chunk's ring stores are in flight
+        float pend_dec = 0.f;
+        // storer: once the pending chunk's ring stores are complete, hand it over
+        auto hand_over = [&]() {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            st_peer_u32(peer_mdec, __float_as_uint(pend_dec));
+            mbar_arrive_peer(peer_ready);
+            pend = false;
+        };
+
+        for (int i = gtid; i < 512; i += 256)
+            reinterpret_cast<uint4 *>(pzt + PZ_Z)[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+
+        auto issue_tma = [&](int m) {
+            const long long t0 = t_begin + (long long)m * C;
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(bar_tma, 4 * 8192);
+            tma_load_3d(raw + 0, &tm_k, 0, h, (int)t0, bar_tma);
+            tma_load_3d(raw + 8192, &tm_q, 0, h, (int)t0, bar_tma);
+            tma_load_3d(raw + L_RAW_AC, &tm_k, 64, h, (int)t0, bar_tma);
+            tma_load_3d(raw + L_RAW_AC + 8192, &tm_q, 64, h, (int)t0, bar_tma);
+            ++issued[g];
+        };
+        // gates, prefetched one group chunk ahead in the registers of warp lw 4
+        float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
+        auto load_gates = [&](int m) {
+            const long long t0 = t_begin + (long long)m * C;
+            const int L = chunk_len(m), r0 = 2 * lane, r1 = 2 * lane + 1;
+            nla0 = r0 < L ? a.log_alpha[(t0 + r0) * H + h] : 0.f;
+            nla1 = r1 < L ? a.log_alpha[(t0 + r1) * H + h] : 0.f;
+            nbe0 = r0 < L ? a.beta[(t0 + r0) * H + h] : 0.f;
+            nbe1 = r1 < L ? a.beta[(t0 + r1) * H + h] : 0.f;
+        };
+        auto gate_rows = [&](int m) { return reinterpret_cast<float *>(grp + L_GATES + ((m >> 1) & 1) * GATES_STRIDE); };
+        auto compute_gates = [&](int mm) {
+            float *gr = gate_rows(mm);
+            const int r0 = 2 * lane, r1 = 2 * lane + 1;
+            const float la0 = nla0, la1 = nla1, be0 = nbe0, be1 = nbe1;
+            if (mm + 2 < nchunks) load_gates(mm + 2);
+            float incl = la0 + la1;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += y;
+            }
+            const float g1 = incl, g0 = incl - la1;
+            float gend[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) gend[b] = __shfl_sync(0xffffffffu, incl, 8 * b + 7);
+            const float gC = gend[3];
+            const int blk = r0 >> 4;
+            const float e0 = __expf(g0), e1 = __expf(g1);
+            const float c0 = __expf(gend[blk] - g0), c1 = __expf(gend[blk] - g1);
+            const float k0 = __expf(gC - g0), k1 = __expf(gC - g1);
+            float f0[3], f1[3];
+#pragma unroll
+            for (int b = 0; b < 3; ++b) {
+                f0[b] = __expf(fminf(g0 - gend[b], 0.f));
+                f1[b] = __expf(fminf(g1 - gend[b], 0.f));
+            }
+            gr[GR_G + r0] = g0; gr[GR_G + r1] = g1;
+            gr[GR_B + r0] = be0; gr[GR_B + r1] = be1;
+            gr[GR_BG + r0] = be0 * e0; gr[GR_BG + r1] = be1 * e1;
+            gr[GR_COLF + r0] = c0; gr[GR_COLF + r1] = c1;
+            gr[GR_KH + r0] = k0; gr[GR_KH + r1] = k1;
+            gr[GR_GAM + r0] = e0; gr[GR_GAM + r1] = e1;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                gr[GR_ROWF + 4 * r0 + b] = b < blk ? f0[b < 3 ? b : 0] : 0.f;
+                gr[GR_ROWF + 4 * r1 + b] = b < blk ? f1[b < 3 ? b : 0] : 0.f;
+            }
+            if (lane == 31) gr[GR_DEC] = __expf(gC);
+        };
+
+        if (issuer && g < nchunks) issue_tma(g);
+        if (lw == 4 && g < nchunks) {
+            load_gates(g);
+            compute_gates(g);
+        }
+        named_bar_sync(BAR_G, 256);
+
+        for (int m = g; m < nchunks; m += 2) {
+            const int it = m >> 1;
+            const float *gr = gate_rows(m);
+            bool ok = true;
+            // ---- tiles of this chunk; rows past the sequence end read as zero.  The
+            //      group's next chunk is fetched into L2 now, its tile load issued
+            //      only at the end of this one (the raw tiles are in use until then)
+            if (issuer && m + 2 < nchunks) {
+                const int t2 = (int)(t_begin + (long long)(m + 2) * C);
+                tma_prefetch_l2_3d(&tm_k, 0, h, t2);
+                tma_prefetch_l2_3d(&tm_k, 64, h, t2);
+                tma_prefetch_l2_3d(&tm_q, 0, h, t2);
+                tma_prefetch_l2_3d(&tm_q, 64, h, t2);
+            }
+            if (issuer) ok = wt.wait(bar_tma, (uint32_t)(it & 1));
+            const int L = chunk_len(m);
+            if (L < C) {
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
+                    const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(raw + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + 8192 + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + L_RAW_AC + o) = z;
+                    *reinterpret_cast<uint4 *>(raw + L_RAW_AC + 8192 + o) = z;
+                }
+                fence_proxy_async_smem();
+            }
+            if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            // ---- D_kq = [K; Q] K^T --------------------------------------------------
+            if (issuer) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < DK / 16; ++k) {
+                    const uint32_t off = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
+                    mma_bf16(tm_kq, d_kq + off, d_kq + off, ID_KK, k > 0);
+                }
+                mma_commit(bar_l);
+                ok = wt.wait(bar_l, bl_wait & 1);
+            }
+            ++bl_wait;
+            if (storer && pend) bulk_wait_read();  // the staging tiles are rewritten below
+            if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            tc_fence_after();
+            // ---- A rows (lanes 0-63) -> fp32;  P rows (lanes 64-127) -> bf16 -------
+            if ((lq & 1) >= lhalf) {
+                float x[32];
+                tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
+                if (lq < 2) {
+                    const int r = 32 * lq + lane;
+                    decay_row(x, r, lq, lhalf, gr, false);
+                    const float br = gr[GR_B + r];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 y = make_float4(br * x[j], br * x[j + 1], br * x[j + 2], br * x[j + 3]);
+                        *reinterpret_cast<float4 *>(AF + r * LDA + 32 * lhalf + j) = y;
+                    }
+                } else {
+                    const int r = 32 * (lq - 2) + lane;
+                    decay_row(x, r, lq - 2, lhalf, gr, true);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<uint4 *>(pzt + PZ_P + sw128(r, 4 * lhalf + j)) = pack8(x + 8 * j);
+                }
+            } else if (lq >= 2) {
+                // P rows 0-31, columns 32-63 (above the diagonal): zero; the tile
+                // held R since the last chunk
+#pragma unroll
+                for (int j = 4; j < 8; ++j)
+                    *reinterpret_cast<uint4 *>(pzt + PZ_P + sw128(lane, j)) = make_uint4(0, 0, 0, 0);
+            }
+            named_bar_sync(BAR_G, 256);
+            // ---- T = (I + A)^{-1}: lw 0-3 (diagonal blocks, 32-level); meanwhile
+            //      lw 4 prepares the group's next gates ----------------------------------
+            if (lw >= 4) {
+                if (lw == 4 && m + 2 < nchunks) compute_gates(m + 2);
+                if (storer && pend) hand_over();  // the previous chunk of this group
+            } else {
+                // (1) 16x16 diagonal blocks: warp lw inverts block lw; lane j < 16
+                //     owns column j (right-looking forward substitution).
+                if (lane < 16) {
+                    const int o = 16 * lw, j = lane;
+                    float t[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                    for (int mm = 0; mm < 15; ++mm) {
+#pragma unroll
+                        for (int i = mm + 1; i < 16; ++i) t[i] -= AF[(o + i) * LDA + o + mm] * t[mm];
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) TF[(o + i) * LDA + o + j] = t[i];
+                }
+                named_bar_sync(BAR_INV, 128);
+                // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
+                const int fg = lane >> 2, ft = lane & 3;
+                const int o = 32 * (lw >> 1), n0 = 8 * (lw & 1);
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int ar = o + 16 + fg, ac = o + 8 * ks + ft;
+                    af[0] = to_tf32(AF[ar * LDA + ac]);
+                    af[1] = to_tf32(AF[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AF[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AF[(ar + 8) * LDA + ac + 4]);
+                    bf[0] = to_tf32(TF[(o + 8 * ks + ft) * LDA + o + n0 + fg]);
+                    bf[1] = to_tf32(TF[(o + 8 * ks + ft + 4) * LDA + o + n0 + fg]);
+                    mma_tf32_16x8x8(x, af, bf);
+                }
+                TF[(o + fg) * LDA + o + 16 + n0 + 2 * ft] = x[0];
+                TF[(o + fg) * LDA + o + 16 + n0 + 2 * ft + 1] = x[1];
+                TF[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft] = x[2];
+                TF[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft + 1] = x[3];
+                __syncwarp();
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 2; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int ar = o + 16 + fg, ac = o + 16 + 8 * ks + ft;
+                    af[0] = to_tf32(TF[ar * LDA + ac]);
+                    af[1] = to_tf32(TF[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(TF[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(TF[(ar + 8) * LDA + ac + 4]);
+                    bf[0] = to_tf32(TF[(o + 8 * ks + ft) * LDA + o + 16 + n0 + fg]);
+                    bf[1] = to_tf32(TF[(o + 8 * ks + ft + 4) * LDA + o + 16 + n0 + fg]);
+                    mma_tf32_16x8x8(y, af, bf);
+                }
+                TF[(o + 16 + fg) * LDA + o + n0 + 2 * ft] = -y[0];
+                TF[(o + 16 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[1];
+                TF[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
+                TF[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
+            }
+            if (named_bar_or(BAR_G, 256, *abort_flag)) break;
+            // (3) T_{H1,H0} = -T_{H1} (A_{H1,H0} T_{H0}), 32x32 blocks; warp lw owns
+            //     output rows 16(lw/4).., columns 8(lw%4)..; X goes to the unused
+            //     upper-right block, the masked upper triangles hold scratch.
+            {
+                const int fg = lane >> 2, ft = lane & 3;
+                const int m0 = 16 * (lw >> 2), n0 = 8 * (lw & 3);
+                float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int ar = 32 + m0 + fg, ac = 8 * ks + ft;
+                    af[0] = to_tf32(AF[ar * LDA + ac]);
+                    af[1] = to_tf32(AF[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AF[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AF[(ar + 8) * LDA + ac + 4]);
+                    const int br = 8 * ks + ft, bc = n0 + fg;
+                    bf[0] = to_tf32(br >= bc ? TF[br * LDA + bc] : 0.f);
+                    bf[1] = to_tf32(br + 4 >= bc ? TF[(br + 4) * LDA + bc] : 0.f);
+                    mma_tf32_16x8x8(x, af, bf);
+                }
+                TF[(m0 + fg) * LDA + 32 + n0 + 2 * ft] = x[0];
+                TF[(m0 + fg) * LDA + 32 + n0 + 2 * ft + 1] = x[1];
+                TF[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft] = x[2];
+                TF[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft + 1] = x[3];
+                named_bar_sync(BAR_G, 256);
+                float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t af[4], bf[2];
+                    const int r = m0 + fg, kc = 8 * ks + ft;
+                    af[0] = to_tf32(kc <= r ? TF[(32 + r) * LDA + 32 + kc] : 0.f);
+                    af[1] = to_tf32(kc <= r + 8 ? TF[(40 + r) * LDA + 32 + kc] : 0.f);
+                    af[2] = to_tf32(kc + 4 <= r ? TF[(32 + r) * LDA + 36 + kc] : 0.f);
+                    af[3] = to_tf32(kc + 4 <= r + 8 ? TF[(40 + r) * LDA + 36 + kc] : 0.f);
+                    bf[0] = to_tf32(TF[(8 * ks + ft) * LDA + 32 + n0 + fg]);
+                    bf[1] = to_tf32(TF[(8 * ks + ft + 4) * LDA + 32 + n0 + fg]);
+                    mma_tf32_16x8x8(y, af, bf);
+                }
+                TF[(32 + m0 + fg) * LDA + n0 + 2 * ft] = -y[0];
+                TF[(32 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[1];
+                TF[(40 + m0 + fg) * LDA + n0 + 2 * ft] = -y[2];
+                TF[(40 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[3];
+            }
+            named_bar_sync(BAR_G, 256);
+            // ---- T_b, T_bg in bf16 (K-major rows r, columns s) -------------------------
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
+                const int idx = gtid + 256 * q2, r = idx >> 3, j = idx & 7;
+                float tv[8], bv[8], gv[8], tb[8], tg[8];
+                *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j);
+                *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j + 4);
+                *reinterpret_cast<float4 *>(bv) = *reinterpret_cast<const float4 *>(gr + GR_B + 8 * j);
+                *reinterpret_cast<float4 *>(bv + 4) = *reinterpret_cast<const float4 *>(gr + GR_B + 8 * j + 4);
+                *reinterpret_cast<float4 *>(gv) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j);
+                *reinterpret_cast<float4 *>(gv + 4) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j + 4);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int s2 = 8 * j + e;
+                    const float t2 = s2 < r ? tv[e] : (s2 == r ? 1.f : 0.f);
+                    tb[e] = t2 * bv[e];
+                    tg[e] = t2 * gv[e];
+                }
+                *reinterpret_cast<uint4 *>(pzt + PZ_TB + sw128(r, j)) = pack8(tb);
+                *reinterpret_cast<uint4 *>(pzt + PZ_TG + sw128(r, j)) = pack8(tg);
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(BAR_G, 256);
+            // ---- D_ab = [P; 0] [T_bg | T_b]:  rows 0-63 = [P T_bg | R] -------------
+            if (issuer) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_bf16(tm_ab, d_pz + 2 * k, d_tgtb + 128 * k, ID_N128, k > 0);
+                mma_commit(bar_l);
+                ok = wt.wait(bar_l, bl_wait & 1);
+            }
+            ++bl_wait;
+            if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            tc_fence_after();
+            if (lq < 2) {  // lw 0,1: P T_bg;  lw 4,5: R, staged in P's tile (P is consumed)
+                const int r = 32 * lq + lane;
+                uint8_t *dst = pzt + (lhalf == 0 ? PZ_PTG : PZ_P);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[32];
+                    tmem_load<32>(tm_ab + lane_off + 64 * lhalf + 32 * hh, x);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        *reinterpret_cast<uint4 *>(dst + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(BAR_G, 256);
+            // ---- D_ab = [T_bg; P T_bg] K:  rows 0-63 = W, rows 64-127 = P W ---------
+            if (issuer) {
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_bf16(tm_ab, d_tgptg + 2 * k, d_kmn + 128 * k, ID_N128, k > 0);
+                mma_commit(bar_l);
+                ok = wt.wait(bar_l, bl_wait & 1);
+            }
+            ++bl_wait;
+            if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            tc_fence_after();
+            // ---- -W (lanes 0-63) and Qh = gamma Q - P W (lanes 64-127) staged in the
+            //      A / T tiles, Kt = kh . K in the T_bg / P T_bg tiles: the raw tiles are
+            //      free for the next chunk once this phase is over ----------------------
+            {
+                const int r = 32 * (lq & 1) + lane;
+                const float gam = gr[GR_GAM + r];
+                uint8_t *wst = grp + L_AF + lhalf * 8192;
+                uint8_t *qst = grp + L_AF + 16384 + lhalf * 8192;
+                const uint8_t *qt = raw + lhalf * L_RAW_AC + 8192;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[32];
+                    tmem_load<32>(tm_ab + lane_off + 64 * lhalf + 32 * hh, x);
+                    if (lq < 2) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            float w[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) w[e] = -x[8 * j + e];
+                            *reinterpret_cast<uint4 *>(wst + sw128(r, 4 * hh + j)) = pack8(w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t o = sw128(r, 4 * hh + j);
+                            float qv[8];
+                            unpack8(*reinterpret_cast<const uint4 *>(qt + o), qv);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) qv[e] = gam * qv[e] - x[8 * j + e];
+                            *reinterpret_cast<uint4 *>(qst + o) = pack8(qv);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const int idx = gtid + 256 * q2;
+                    const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
+                    float kv[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(raw + ac * L_RAW_AC + sw128(rr, j)), kv);
+                    const float sc = gr[GR_KH + rr];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) kv[e] *= sc;
+                    *reinterpret_cast<uint4 *>(pzt + PZ_TG + ac * 8192 + sw128(rr, j)) = pack8(kv);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (named_bar_or(BAR_G, 256, *abort_flag)) break;
+            // the raw tiles take the group's next chunk
+            if (issuer && m + 2 < nchunks) issue_tma(m + 2);
+            if (storer) {
+                // once the state CTA has read the slot's previous chunk, the eight
+                // tiles go to the ring by bulk copy; the hand-off follows during
+                // the next chunk (or after the loop)
+                if (m < 2 || wt.wait_peer(bar_slotfree, (uint32_t)((it - 1) & 1))) {
+                    bulk_store(ring_slot + SG_KT, pzt + PZ_TG, 8192);
+                    bulk_store(ring_slot + SG_QH, grp + L_AF + 16384, 8192);
+                    bulk_store(ring_slot + SG_MW, grp + L_AF, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_KT, pzt + PZ_PTG, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_QH, grp + L_AF + 24576, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_MW, grp + L_AF + 8192, 8192);
+                    bulk_store(ring_slot + SG_R, pzt + PZ_P, 8192);
+                    bulk_store(ring_slot + SG_TB, pzt + PZ_TB, 8192);
+                    bulk_commit();
+                    pend = true;
+                    pend_dec = gr[GR_DEC];
+                }
+            }
+        }
+        if (storer && pend && !*abort_flag) hand_over();
+        // drain: every MMA this issuer launched, every tile load not yet landed
+        if (storer) bulk_wait_all();
+        if (*abort_flag && issuer) {
+            mma_commit(bars + LB_DRAIN + g);
+            mbar_wait(bars + LB_DRAIN + g, 0, kWaitLimit);
+            if (issued[g] > 0) mbar_wait(bar_tma, (uint32_t)((issued[g] - 1) & 1), kWaitLimit);
+        }
+    } else if (slot >= 0) {
+        // ============================ state CTA ============================
+        float *sdec = reinterpret_cast<float *>(cm + CM_SDEC);
+        const float *mdec = reinterpret_cast<const float *>(cm + CM_MDEC);
+        if (warp < 8) {
+            // ---- chain of value half hv: warps 4hv..4hv+3, thread = key channel c
+            const int hv = warp >> 2, q = warp & 3, c = 32 * q + lane;
+            const int BAR_H = 1 + hv;
+            const bool leader = (tid & 127) == 0;
+            const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+            uint8_t *sb = sm + S_OFF_SB + hv * 16384;
+            uint8_t *vp = sm + S_OFF_VP + hv * 8192;
+            const uint64_t d_rtb = desc_sw128(sbase + SG_R, 16, 1024);
+            const uint64_t d_v = desc_sw128(sbase + SG_V + 8192 * hv, 8192, 1024);
+            const uint64_t d_qw = desc_sw128(sbase + SG_QH, 16, 1024);
+            const uint64_t d_sb = desc_sw128(sbase + S_OFF_SB + hv * 16384, 16384, 1024);
+            const uint64_t d_kt = desc_sw128(sbase + SG_KT, SG_AC, 1024);
+            const uint64_t d_vp = desc_sw128(sbase + S_OFF_VP + hv * 8192, 8192, 1024);
+            const uint32_t tm_ds = tmem + TM_DS + 64 * hv;
+            float s_reg[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+                s_reg[i] = a.s0 ? a.s0[st_base + (size_t)(64 * hv + i) * DK + c] : 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<uint4 *>(sb + sw128(c, j)) = pack8(s_reg + 8 * j);
+            fence_proxy_async_smem();
+            float *cdec = reinterpret_cast<float *>(cm + CM_CDEC) + hv;  // this chunk's e^{g_C}
+            // D_vo[st] = [R; T_b] V_h  (needs the chunk's stage and D_vo free)
+            auto issue_v = [&](int m) {
+                const uint32_t so = (m & 1) * (S_STAGE >> 4);
+                const uint32_t tm_vo = tmem + 64 * (2 * (m & 1) + hv);
+#pragma unroll
+                for (int k = 0; k < C / 16; ++k)
+                    mma_bf16(tm_vo, d_rtb + so + 2 * k, d_v + so + 128 * k, ID_N64, k > 0);
+            };
+            bool v_issued = false;
+            named_bar_sync(BAR_H, 128);
+            for (int m = 0; m < nchunks; ++m) {
+                const int st = m & 1, it = m >> 1;
+                const uint32_t so = st * (S_STAGE >> 4);
+                const uint32_t tm_vo = tmem + 64 * (2 * st + hv);
+                bool ok = true;
+                if (leader) {
+                    if (!v_issued) {
+                        ok = wt.wait(bars + SB_FULL + st, (uint32_t)(it & 1));
+                        if (ok && m >= 2) ok = wt.wait(bars + SB_OFREE + 2 * st + hv, (uint32_t)((it - 1) & 1));
+                        if (ok) {
+                            tc_fence_after();
+                            issue_v(m);
+                        }
+                    }
+                    // the stage has landed (waited here or before the early V
+                    // product): publish its decay to the chain
+                    *cdec = sdec[st];
+                    // D_vo += [Qh; -W] S_h^T
+                    if (ok) {
+#pragma unroll
+                        for (int k = 0; k < DK / 16; ++k) {
+                            const uint32_t off = ((k >> 2) * SG_AC + (k & 3) * 32) >> 4;
+                            mma_bf16(tm_vo, d_qw + so + off, d_sb + 128 * k, ID_N64, 1);
+                        }
+                        mma_commit(bars + SB_VO + hv);
+                    }
+                }
+                v_issued = false;
+                // V' rows (lanes 64-127) -> bf16, MN-major [r][i]
+                if (q >= 2) {
+                    const bool okv = wt.warp_wait(bars + SB_VO + hv, (uint32_t)(m & 1), lane);
+                    if (okv) {
+                        tc_fence_after();
+                        const int r = 32 * (q - 2) + lane;
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float x[32];
+                            tmem_load<32>(tm_vo + lane_off + 32 * hh, x);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                *reinterpret_cast<uint4 *>(vp + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
+                        }
+                    } else {
+                        ok = false;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (named_bar_or(BAR_H, 128, !ok || *abort_flag)) break;
+                const float dec = *cdec;
+                if (leader) {
+                    tc_fence_after();
+                    // dS_h = Kt^T V'_h
+#pragma unroll
+                    for (int k = 0; k < C / 16; ++k)
+                        mma_bf16(tm_ds, d_kt + so + 128 * k, d_vp + 128 * k, ID_MM, k > 0);
+                    mma_commit(bars + SB_DS + hv);
+                    mma_commit(bars + SB_CONS + st);
+                    // the next chunk's V product, if its stage is already there
+                    if (m + 1 < nchunks) {
+                        const int st1 = (m + 1) & 1, it1 = (m + 1) >> 1;
+                        if (mbar_try_wait(bars + SB_FULL + st1, (uint32_t)(it1 & 1)) &&
+                            (m + 1 < 2 ||
+                             mbar_try_wait(bars + SB_OFREE + 2 * st1 + hv, (uint32_t)((it1 - 1) & 1)))) {
+                            tc_fence_after();
+                            issue_v(m + 1);
+                            v_issued = true;
+                        }
+                    }
+                }
+                // S_h <- e^{g_C} S_h + dS_h
+                const bool okd = wt.warp_wait(bars + SB_DS + hv, (uint32_t)(m & 1), lane);
+                if (okd) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float ds[32];
+                        tmem_load<32>(tm_ds + lane_off + 32 * hh, ds);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) s_reg[32 * hh + i] = dec * s_reg[32 * hh + i] + ds[i];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<uint4 *>(sb + sw128(c, j)) = pack8(s_reg + 8 * j);
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (named_bar_or(BAR_H, 128, !okd || *abort_flag)) break;
+            }
+            if (*abort_flag) {
+                if (leader) {  // every MMA this leader launched
+                    mma_commit(bars + SB_DRAIN + hv);
+                    mbar_wait(bars + SB_DRAIN + hv, 0, kWaitLimit);
+                }
+            } else if (a.s_final) {
+#pragma unroll
+                for (int i = 0; i < 64; ++i) a.s_final[st_base + (size_t)(64 * hv + i) * DK + c] = s_reg[i];
+            }
+        } else if (warp == 8 || warp == 9 || warp == 12 || warp == 13) {
+            // ---- output rows of value half hv (lanes 0-63 of D_vo) ----------------
+            const int hv = (warp >> 2) & 1, q = warp & 1;
+            const int BAR_O = 3 + hv;
+            const uint32_t lane_off = (uint32_t)(32 * q) << 16;
+            const int r = 32 * q + lane;
+            for (int m = 0; m < nchunks; ++m) {
+                const int st = m & 1;
+                const bool ok = wt.warp_wait(bars + SB_VO + hv, (uint32_t)(m & 1), lane);
+                if (ok) {
+                    tc_fence_after();
+                    const long long t0 = t_begin + (long long)m * C;
+                    const int L = chunk_len(m);
+                    __nv_bfloat16 *dst = reinterpret_cast<__nv_bfloat16 *>(a.o) +
+                                         ((t0 + r) * H + h) * (long long)DV + 64 * hv;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float x[32];
+                        tmem_load<32>(tmem + 64 * (2 * st + hv) + lane_off + 32 * hh, x);
+                        if (r < L) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                reinterpret_cast<uint4 *>(dst)[4 * hh + j] = pack8(x + 8 * j);
+                        }
+                    }
+                }
+                tc_fence_before();
+                if (named_bar_or(BAR_O, 64, !ok || *abort_flag)) break;
+                if (q == 0 && lane == 0) mbar_arrive(bars + SB_OFREE + 2 * st + hv);
+            }
+        } else if (warp == 10 && lane == 0) {
+            // ---- loader: ring slot + V tiles of each chunk into its stage ----------
+            const uint32_t peer_slotfree = map_peer(smem_u32(bars), peer);  // + 8 * (LB_SLOTFREE + st)
+            for (int m = 0; m < nchunks; ++m) {
+                const int st = m & 1, it = m >> 1;
+                uint8_t *stage = sm + st * S_STAGE;
+                bool ok = true;
+                if (m >= 2) ok = wt.wait(bars + SB_CONS + st, (uint32_t)((it - 1) & 1));
+                if (ok) ok = wt.wait_peer(bars + SB_READY + st, (uint32_t)(it & 1));
+                if (!ok) break;
+                fence_proxy_async_global();
+                sdec[st] = mdec[st];
+                const uint8_t *src = ring_pair + (size_t)st * RING_SLOT;
+                const long long t0 = t_begin + (long long)m * C;
+                mbar_arrive_expect_tx(bars + SB_FULL + st, S_STAGE_TX);
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    bulk_load(stage + p * 16384, src + p * 16384, 16384, bars + SB_FULL + st);
+                tma_load_3d(stage + SG_V, &tm_v, 0, h, (int)t0, bars + SB_FULL + st);
+                tma_load_3d(stage + SG_V + 8192, &tm_v, 64, h, (int)t0, bars + SB_FULL + st);
+                ++issued[st];
+                // the slot is read once the stage has landed: give it back
+                if (!wt.wait(bars + SB_FULL + st, (uint32_t)(it & 1))) break;
+                mbar_arrive_peer(peer_slotfree + 8 * (LB_SLOTFREE + st));
+            }
+            if (*abort_flag)
+                for (int st = 0; st < 2; ++st)
+                    if (issued[st] > 0)
+                        mbar_wait(bars + SB_FULL + st, (uint32_t)((issued[st] - 1) & 1), kWaitLimit);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag && slot >= 0) atomicOr(a.err, kErrTimeout);
+    cluster_sync();  // no CTA leaves while its peer may still address its memory
+    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------- host --
+int ring_slots_for_device() {
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return 2 * nsm;  // SM ids are below this on every part this kernel runs on
+}
+
+}  // namespace
+
+size_t chunk_pair_scratch_bytes(const gdn_dims &) {
+    return (size_t)ring_slots_for_device() * 2 * RING_SLOT;
+}
+
+cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches) {
+    const long long items = (long long)a.n_seqs * a.H;
+    const long long ntok = (long long)a.B * a.T;
+    if (items == 0) return cudaSuccess;
+    if (ntok == 0) {
+        if (a.s_final && a.s_final != a.s0) {
+            const size_t bytes = (size_t)a.n_seqs * a.H * a.dv * a.dk * sizeof(float);
+            return a.s0 ? cudaMemcpyAsync(a.s_final, a.s0, bytes, cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(a.s_final, 0, bytes, s);
+        }
+        return cudaSuccess;
+    }
+    CUtensorMap mq, mk, mv;
+    if (!make_tile_map(&mq, a.q, a.dk, a.H, ntok) || !make_tile_map(&mk, a.k, a.dk, a.H, ntok) ||
+        !make_tile_map(&mv, a.v, a.dv, a.H, ntok))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(chunk_pair_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const int slots = ring_slots_for_device();
+    if (slots <= 0) return cudaErrorInvalidValue;
+    chunk_pair_kernel<<<(unsigned)(2 * items), kThreads, SMEM_BYTES, s>>>(
+        a, mq, mk, mv, reinterpret_cast<uint8_t *>(a.scratch), slots);
+    if (launches) ++*launches;
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

@@ -713,6 +713,8 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
 
+}  // namespace
+
 // ------------------------------------------------------------------- host --
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                    const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -733,7 +735,7 @@ EncodeTiledFn encode_fn() {
 }
 
 // [tokens, H, d] bf16 viewed as a 3-D tensor (d, H, tokens); box 64 x 1 x 64.
-bool make_map(CUtensorMap *m, const void *base, int d, int H, long long ntok) {
+bool make_tile_map(CUtensorMap *m, const void *base, int d, int H, long long ntok) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)ntok};
@@ -745,8 +747,6 @@ bool make_map(CUtensorMap *m, const void *base, int d, int H, long long ntok) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
            CUDA_SUCCESS;
 }
-
-}  // namespace
 
 bool chunk_tc_supported(const gdn_dims &d) {
     return d.dtype == GDN_BF16 && d.d_k == DK && d.d_v == 128 && d.decay == GDN_DECAY_SCALAR &&
@@ -769,8 +769,8 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t s, int *launches)
         return cudaSuccess;
     }
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, a.q, a.dk, a.H, ntok) || !make_map(&mk, a.k, a.dk, a.H, ntok) ||
-        !make_map(&mv, a.v, a.dv, a.H, ntok))
+    if (!make_tile_map(&mq, a.q, a.dk, a.H, ntok) || !make_tile_map(&mk, a.k, a.dk, a.H, ntok) ||
+        !make_tile_map(&mv, a.v, a.dv, a.H, ntok))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);

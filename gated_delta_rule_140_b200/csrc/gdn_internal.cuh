@@ -2,6 +2,7 @@
 // of the public ABI, which is include/gdn.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -13,7 +14,7 @@ namespace gdn {
 constexpr int kChunk = 64;  // chunk size C of the chunkwise form
 
 // Sticky error bits kept in the first word of the workspace.
-enum : uint32_t { kErrBadSeqlens = 1u, kErrTimeout = 2u };
+enum : uint32_t { kErrBadSeqlens = 1u, kErrTimeout = 2u, kErrInternal = 4u };
 constexpr size_t kWorkspaceHeader = 256;
 
 // Everything a prefill kernel needs, in device pointers.  Token-major layouts
@@ -45,8 +46,14 @@ struct DecodeArgs {
 cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches);
 size_t chunk_tc_scratch_bytes(const gdn_dims &d);
+size_t chunk_pair_scratch_bytes(const gdn_dims &d);
+// bf16 d_k = d_v = 128 scalar-decay shapes the tensor-core kernels take
 bool chunk_tc_supported(const gdn_dims &d);
+// [tokens, H, d] bf16 as a 3-D TMA tensor map (d, H, tokens), box 64 x 1 x 64,
+// 128-byte swizzle (defined with the single-CTA tensor-core kernel).
+bool make_tile_map(CUtensorMap *m, const void *base, int d, int H, long long ntok);
 
 // Token range of sequence n for fixed rows or packed sequences, validated on
 // the device: a bad range records kErrBadSeqlens and yields an empty range.

@@ -38,8 +38,14 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
                                             const float *beta, const float *initial_state,
                                             const int32_t *cu_seqlens, void *o,
                                             float *final_state, gdn_stream_t stream) {
-    const size_t need = gdn_chunk_fwd_workspace_size(dims);
+    size_t need = gdn_chunk_fwd_workspace_size(dims);
     if (need == 0) return GDN_ERR_INVALID;
+    gdn_dims d = *dims;
+    if (need > GDN_NOALLOC_SCRATCH_BYTES && (d.flags & GDN_FLAG_PAIR)) {
+        // the two-CTA kernel's ring does not fit: the default kernel
+        d.flags &= ~GDN_FLAG_PAIR;
+        need = gdn_chunk_fwd_workspace_size(&d);
+    }
     if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_UNSUPPORTED;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
@@ -51,6 +57,6 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
     if (cudaMemsetAsync(scratch, 0, gdn::kWorkspaceHeader,
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return GDN_ERR_CUDA;
-    return gdn_chunk_fwd(dims, q, k, v, log_alpha, beta, initial_state, cu_seqlens, o,
+    return gdn_chunk_fwd(&d, q, k, v, log_alpha, beta, initial_state, cu_seqlens, o,
                          final_state, scratch, GDN_NOALLOC_SCRATCH_BYTES, stream);
 }

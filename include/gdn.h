@@ -60,11 +60,15 @@ typedef enum {
 typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
 
-/* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: the
- * tensor-core kernel for bf16 with d_k = d_v = 128, the fp32 CUDA-core kernel
- * otherwise.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel (used by the
- * tests to compare the two device paths). */
-enum { GDN_FLAG_CUDA_CORES = 1 };
+/* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: for bf16
+ * with d_k = d_v = 128 and scalar decay the single-CTA tensor-core kernel, the
+ * fp32 CUDA-core kernel otherwise.  GDN_FLAG_PAIR selects, for the same shapes,
+ * the two-CTA tensor-core kernel (one thread-block cluster per sequence and
+ * head: one SM computes the chunk-local matrices, the other runs the
+ * sequential state pass; it needs a larger workspace, see below).
+ * GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use the
+ * flags to compare the device paths. */
+enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2 };
 
 typedef struct {
     int32_t B;       /* batch (1 for a packed batch)                           */
@@ -78,9 +82,14 @@ typedef struct {
     int32_t flags;   /* GDN_FLAG_* (0 = default)                                */
 } gdn_dims;
 
-/* Bytes of device workspace gdn_chunk_fwd needs for `dims` (always >= 256).
- * The first 256 bytes hold the sticky error word; zero the whole workspace
- * once before its first use (gdn_workspace_init).  Returns 0 for invalid dims. */
+/* Bytes of device workspace gdn_chunk_fwd needs for `dims` (always >= 256),
+ * on the current device.  The first 256 bytes hold the sticky error word;
+ * zero them once before the workspace's first use (gdn_workspace_init).  The
+ * two-CTA tensor-core kernel adds a ring of two 64 KiB slots for each SM index
+ * of the device (2 x its SM count), through which the chunk-local SM hands each
+ * chunk's matrices to the state SM; it is written before it is read and needs
+ * no initialisation.  The other kernels need only the header.  Returns 0 for
+ * invalid dims. */
 size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims);
 
 /* Chunkwise (WY / UT-transform) prefill, chunk size C = 64
@@ -136,10 +145,13 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
  * another allocator, so that a cudaMalloc would fail or fragment it.
  *
  * Instead of a caller workspace it uses one fixed device array of
- * GDN_NOALLOC_SCRATCH_BYTES compiled into the library.  Problems whose
- * gdn_chunk_fwd_workspace_size exceeds that return GDN_ERR_UNSUPPORTED before
- * anything is launched.  All other arguments, layouts and results are those of
- * gdn_chunk_fwd.
+ * GDN_NOALLOC_SCRATCH_BYTES compiled into the library.  Where the selected
+ * kernel's workspace (gdn_chunk_fwd_workspace_size) does not fit in it -- the
+ * two-CTA tensor-core kernel's ring never does -- the call runs the default
+ * kernel instead (GDN_FLAG_PAIR cleared), whose workspace is the header alone.
+ * Problems whose workspace exceeds the array even then return
+ * GDN_ERR_UNSUPPORTED before anything is launched.  All other arguments,
+ * layouts and results are those of gdn_chunk_fwd.
  *   - The first call on each device looks up the array's device address (with
  *     that device current) and caches it; make that first call before any
  *     stream capture.
@@ -160,12 +172,14 @@ gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_strea
 
 /* Synchronise `stream`, read and clear the workspace's sticky error word.
  * GDN_OK if no device-side error was recorded since the last read;
- * GDN_ERR_TIMEOUT or GDN_ERR_DEVICE_INPUT otherwise. */
+ * GDN_ERR_TIMEOUT, GDN_ERR_DEVICE_INPUT, or GDN_ERR_CUDA (a kernel found no
+ * ring slot for the SM it ran on) otherwise. */
 gdn_status gdn_workspace_status(void *workspace, gdn_stream_t stream);
 
 /* Name of the prefill kernel gdn_chunk_fwd selects for `dims` (static
- * storage): "tensor_core" (tcgen05, bf16, d_k = d_v = 128) or "cuda_core"
- * (fp32 CUDA cores); NULL for invalid dims. */
+ * storage): "tensor_core_pair" (two-CTA tcgen05 kernel), "tensor_core"
+ * (single-CTA tcgen05 kernel) or "cuda_core" (fp32 CUDA cores); NULL for
+ * invalid dims. */
 const char *gdn_chunk_fwd_path(const gdn_dims *dims);
 
 /* Human-readable name of a status code (static storage). */

@@ -51,12 +51,13 @@ def test_tiny_fp32_workload(cuda_ok):
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("decay", ["scalar", "channel"])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("cuda_cores", [False, True])
-def test_reduced_ragged(cuda_ok, dtype, decay, d, cuda_cores):
-    """Several chunks and a ragged tail (T = 3*64 + 37), with an initial state."""
+@pytest.mark.parametrize("path", ["default", "pair", "cuda_cores"])
+def test_reduced_ragged(cuda_ok, dtype, decay, d, path):
+    """Several chunks and a ragged tail (T = 3*64 + 37), with an initial state,
+    on each prefill kernel that takes the shape."""
     x = prefill_inputs(2, 229, 3, d, d, dtype=dtype, decay=decay, seed=21,
                        alpha_shift=2.0 if decay == "scalar" else 3.0, init_std=0.05)
-    o, sf = _run(x, cuda_cores=cuda_cores)
+    o, sf = _run(x, cuda_cores=path == "cuda_cores", pair=path == "pair")
     _full_compare(x, o, sf, dtype)
 
 
@@ -128,10 +129,36 @@ def test_bad_cu_seqlens_reported_by_workspace_status(cuda_ok):
 
 def test_tensor_core_and_cuda_core_paths_agree(cuda_ok):
     x = prefill_inputs(2, 512, 4, 128, 128, dtype=torch.bfloat16, seed=27, init_std=0.02)
+    d = to_dev(x)
+    assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"])) == "tensor_core"
+    assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"], pair=True)) == \
+        "tensor_core_pair"
     o1, s1 = _run(x)
-    o2, s2 = _run(x, cuda_cores=True)
-    assert rel_err(o1, o2.float().cpu().numpy()) < 2e-2
-    assert rel_err(s1, s2.cpu().numpy()) < 1e-2
+    for kw in ({"cuda_cores": True}, {"pair": True}):
+        o2, s2 = _run(x, **kw)
+        assert rel_err(o1, o2.float().cpu().numpy()) < 2e-2
+        assert rel_err(s1, s2.cpu().numpy()) < 1e-2
+
+
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 129, 640])
+def test_pair_kernel_chunk_counts(cuda_ok, T):
+    """The two-CTA kernel with 1..10 chunks per sequence: both local groups,
+    odd and even chunk counts, a one-token sequence."""
+    x = prefill_inputs(2, T, 2, 128, 128, dtype=torch.bfloat16, seed=28 + T, init_std=0.05)
+    o, sf = _run(x, pair=True)
+    _full_compare(x, o, sf, torch.bfloat16)
+
+
+def test_pair_kernel_strong_and_zero_decay(cuda_ok):
+    """log alpha from -20 to 0 per token: block decays that underflow, chunks
+    with no decay at all."""
+    x = prefill_inputs(1, 256, 2, 128, 128, dtype=torch.bfloat16, seed=29, init_std=0.05)
+    la = x["log_alpha"]
+    la[:, :64] = -20.0
+    la[:, 64:128] = 0.0
+    for pair in (False, True):
+        o, sf = _run(x, pair=pair)
+        _full_compare(x, o, sf, torch.bfloat16)
 
 
 # --------------------------------------------------------------------------- #
