@@ -31,12 +31,13 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
 
 enum class Path { kPair, kOneCta, kCudaCores };
 
-// The prefill kernel a call runs: the single-CTA tensor-core kernel by
-// default, the two-CTA one with GDN_FLAG_PAIR, the fp32 CUDA-core kernel for
-// every other shape or with GDN_FLAG_CUDA_CORES.
+// The prefill kernel a call runs.  bf16, d_k = d_v = 128: GDN the single-CTA
+// tensor-core kernel, or either decay the two-CTA kernel with GDN_FLAG_PAIR;
+// every other case, or GDN_FLAG_CUDA_CORES, the fp32 CUDA-core kernel.
 Path select_path(const gdn_dims &d) {
-    if ((d.flags & GDN_FLAG_CUDA_CORES) || !gdn::chunk_tc_supported(d)) return Path::kCudaCores;
-    return (d.flags & GDN_FLAG_PAIR) ? Path::kPair : Path::kOneCta;
+    if ((d.flags & GDN_FLAG_CUDA_CORES) || !gdn::chunk_pair_supported(d)) return Path::kCudaCores;
+    if (d.flags & GDN_FLAG_PAIR) return Path::kPair;
+    return gdn::chunk_tc_supported(d) ? Path::kOneCta : Path::kCudaCores;
 }
 
 int prefill_seqs(const gdn_dims &d, const int32_t *cu_seqlens) {

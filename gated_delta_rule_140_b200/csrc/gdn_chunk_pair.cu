@@ -1,36 +1,52 @@
 // gdn_chunk_pair.cu -- chunkwise gated delta rule prefill on the tensor cores
 // with the chunk-local work and the sequential state pass on two different
 // SMs: one 2-CTA cluster per (sequence, head), bf16 inputs, d_k = d_v = 128,
-// scalar (GDN) decay.
+// scalar (GDN) or channel-wise (KDA) decay.
 //
 // Chunkwise form (FG2-GDN paper, section 3.6: WY representation, UT transform,
 // inter-chunk state propagation; Gated Delta Networks page, section 3.3, for
-// the cumulative decay g_r within a chunk, gamma_r = e^{g_r}), C = 64 tokens:
+// the cumulative decay g_r within a chunk), C = 64 tokens.  With the decay
+// written per key channel (KDA; GDN has one value for all channels),
+// G_rc = sum_{t<=r} log alpha_tc and Kg = K . e^{G}, Qg = Q . e^{G}:
 //
-//   A_rs = beta_r e^{g_r-g_s} k_r.k_s (s < r),  T = (I + A)^{-1}
-//   P_rs = e^{g_r-g_s} q_r.k_s (s <= r)
-//   T_b = T diag(beta),  T_bg = T diag(beta gamma),  W = T_bg K,  U = T_b V
-//   V'  = U - W S^T,     o = gamma Q S^T + P V',
-//   S  <- e^{g_C} S + V'^T (kh . K),  kh_s = e^{g_C - g_s}.
+//   A_rs = beta_r sum_c k_rc k_sc e^{G_rc-G_sc} (s < r),  T = (I + A)^{-1}
+//   P_rs = sum_c q_rc k_sc e^{G_rc-G_sc} (s <= r)
+//   T_b = T diag(beta),  W = T_b Kg,  U = T_b V
+//   V'  = U - W S^T,     o = Qg S^T + P V',
+//   S  <- S Diag(e^{G_C}) + V'^T Kt,  Kt_sc = k_sc e^{G_Cc - G_sc}.
 //
 // The output is regrouped so that it needs nothing after the state product:
-//   o = (gamma Q - P W) S^T + (P T_b) V = Qh S^T + R V
+//   o = (Qg - P W) S^T + (P T_b) V = Qh S^T + R V
 // and one accumulator per chunk (M = 128) holds both halves of the pass:
 //   D = [Qh; -W] S^T + [R; T_b] V  ->  rows 0-63: o,  rows 64-127: V'.
-// The state update needs V' only through  dS = (kh . K)^T V' = Kt^T V'.
 //
 // Rank 0 ("local" CTA) computes, per chunk, everything that depends only on
-// the chunk's tokens: A, T (fp32, tf32 MMAs for the off-diagonal blocks), P,
-// T_b, T_bg, P T_bg and R = P T_b (one MMA), [W; P W] = [T_bg; P T_bg] K (one
-// MMA), and writes Kt, Qh, -W, R, T_b as bf16 tiles in the swizzled layout the
-// state CTA's MMAs read, into a 2-slot ring in global memory (L2-resident: it
-// is rewritten every other chunk).  Two groups of 8 warps work on two chunks at
-// once (even / odd chunks, ring slot = chunk parity).
+// the chunk's tokens and writes Kt, Qh, -W, R, T_b (bf16 tiles in the
+// swizzled layout the state CTA's MMAs read) and e^{G_C} into a 2-slot ring in
+// global memory, L2-resident since it is rewritten every other chunk.  Two
+// groups of 8 warps work on two chunks at once (even / odd chunks, ring slot =
+// chunk parity); per group and chunk:
+//   GDN: D = [K; Q] K^T, then A and P take the decay e^{g_r-g_s} (block
+//        factored, exact inside the diagonal 32x32 blocks); T_bg = T_b
+//        diag(e^{g}) so that W = T_bg K; [P T_bg | R] = P [T_bg | T_b];
+//        [W; P W] = [T_bg; P T_bg] K.
+//   KDA: K and Q are scaled in place to Kg, Qg and Ki = K . e^{-G} is formed,
+//        so that D = [Kg; Qg] Ki^T is the decayed product directly (A and P
+//        only take masks); R = P T_b; [W; P W] = [T_b; R] Kg.
+// T comes from blocked forward substitution in fp32 (tf32 MMAs for the
+// off-diagonal blocks), computed in place of A.
 // Rank 1 ("state" CTA) holds S (fp32, registers) for all 128 value channels as
 // two independent halves of 64, each with its own chain of warps, loads each
 // chunk's ring slot and V tile (bulk copy + TMA), and per chunk and half
 // issues D = [R;T_b] V_h + [Qh;-W] S_h^T, writes o, converts V' to bf16 and
 // issues dS = Kt^T V'.
+//
+// KDA range: Ki = K . e^{-G} is finite while a chunk's total decay on every
+// channel is above e^{-kMaxNegLogDecay}.  A chunk past that is computed with the
+// factor clamped, and its (sequence, head) is flagged in the workspace; the
+// host re-runs the flagged items exactly on the CUDA-core kernel, and this
+// kernel leaves their final state to it.
+//
 // The CTAs signal each other with mbarriers (ring slot written / ring slot
 // read).  Every wait is bounded: on expiry the CTA records kErrTimeout, raises
 // the abort flag of both CTAs, drains what it issued and leaves through the
@@ -47,55 +63,63 @@ constexpr int C = kChunk;  // 64
 constexpr int DK = 128, DV = 128;
 constexpr int kThreads = 512;
 constexpr long long kWaitLimit = 1LL << 31;  // SM cycles (~1 s)
-constexpr int LDA = 68;                      // fp32 row stride of A and T
+constexpr int LDA = 68;                      // fp32 row stride of A / T
+constexpr float kMaxNegLogDecay = 80.f;      // e^{80} < bf16 and fp32 max
 
 // ---- ring slot / state-CTA stage layout (bytes, 1024-aligned tiles) --------
 // per atom column a (d_k 64a .. 64a+63):  [Kt rows 0-63 | Qh rows | -W rows]
 constexpr uint32_t SG_KT = 0, SG_QH = 8192, SG_MW = 16384, SG_AC = 24576;
 constexpr uint32_t SG_R = 49152, SG_TB = 57344;  // [R; T_b]  (A of the V product)
-constexpr uint32_t RING_SLOT = 65536;            // ring slot = stage bytes [0, 64K)
-constexpr uint32_t SG_V = 65536;                 // V tiles, d_v halves at +8K
-constexpr uint32_t S_STAGE = 81920;
-constexpr uint32_t S_STAGE_TX = RING_SLOT + 2 * 8192;
+constexpr uint32_t SG_TILES = 65536;             // ring slot: the tiles, then
+constexpr uint32_t SG_DECB = 512;                //   e^{G_C} per key channel
+constexpr uint32_t RING_STRIDE = SG_TILES + 1024;
+constexpr uint32_t SG_V = 65536;                 // stage: V tiles, d_v halves at +8K
+constexpr uint32_t SG_DEC = 81920;               //        e^{G_C}
+constexpr uint32_t S_STAGE = 82944;
+constexpr uint32_t S_STAGE_TX = SG_TILES + SG_DECB + 2 * 8192;
 constexpr uint32_t S_OFF_SB = 2 * S_STAGE;       // S_h^T bf16, MN-major [c][i], 16 KB per half
 constexpr uint32_t S_OFF_VP = S_OFF_SB + 2 * 16384;  // V'_h bf16, MN-major [r][i], 8 KB per half
 
 // ---- local-CTA group layout ---------------------------------------------------
 constexpr uint32_t L_RAW = 0;          // [K0 | Q0 | K1 | Q1], 8 KB each (TMA)
 constexpr uint32_t L_RAW_AC = 16384;   //   atom column stride: [K_a; Q_a] is an M=128 tile
-constexpr uint32_t L_PZT = 32768;      // [P | 0 | T_bg | P T_bg | T_b], 8 KB each
-constexpr uint32_t PZ_P = 0, PZ_Z = 8192, PZ_TG = 16384, PZ_PTG = 24576, PZ_TB = 32768;
-constexpr uint32_t L_AF = 73728;                   // A fp32 [64][LDA]
-constexpr uint32_t L_TF = L_AF + 64 * LDA * 4;     // T fp32 [64][LDA]
-constexpr uint32_t L_GATES = L_TF + 64 * LDA * 4;  // two gate-row buffers
+constexpr uint32_t L_KX = 32768;       // 2 x 8 KB: KDA Ki (MMA operand), then Kt; GDN Kt
+constexpr uint32_t L_PZT = 49152;      // [P | 0 | X1 | X2 | X3], 8 KB each
+constexpr uint32_t PZ_P = 0, PZ_Z = 8192, PZ_X1 = 16384, PZ_X2 = 24576, PZ_X3 = 32768;
+//   GDN: X1 = T_bg, X2 = P T_bg, X3 = T_b;  KDA: X1 = T_b, X2 = R, X3 = Qh staging
+constexpr uint32_t L_AT = 90112;                   // A, then T in place: fp32 [64][LDA]
+constexpr uint32_t L_GATES = L_AT + 64 * LDA * 4;  // two gate-row buffers
 constexpr uint32_t GATES_STRIDE = 3072;
-constexpr uint32_t L_GROUP = 114688;
-static_assert(L_GATES + 2 * GATES_STRIDE <= L_GROUP, "local group layout");
-// gate rows (floats): g[64] beta[64] beta*gamma[64] colf[64] rowf[64][4] kh[64] gamma[64] dec
+constexpr uint32_t L_GROUP = 113664;
+static_assert(L_GATES % 1024 == 0 && L_GATES + 2 * GATES_STRIDE <= L_GROUP && L_GROUP % 1024 == 0,
+              "local group layout");
+// gate rows (floats).  GDN: g beta beta*gamma colf rowf[4] kh gamma, and dec;
+// KDA: beta and dec (the first 512 floats are the prefix-sum scratch)
 constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
               GR_GAM = 576, GR_DEC = 640;
+constexpr int GR_KB = 512;  // KDA beta (after the scratch)
 
 // ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
-constexpr uint32_t OFF_COMMON = 2 * L_GROUP;  // 229376
+constexpr uint32_t OFF_COMMON = 2 * L_GROUP;
 static_assert(S_OFF_VP + 2 * 8192 <= OFF_COMMON, "state layout");
-constexpr uint32_t CM_ABORT = 0, CM_SLOT = 4, CM_TMEM = 8, CM_MDEC = 16, CM_SDEC = 24,
-                   CM_ISSUED = 32, CM_CDEC = 40, CM_BARS = 64;
+constexpr uint32_t CM_ABORT = 0, CM_SLOT = 4, CM_TMEM = 8, CM_ISSUED = 32, CM_BARS = 64;
 constexpr uint32_t SMEM_USED = OFF_COMMON + CM_BARS + 16 * 8;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 // state-CTA mbarriers
 constexpr int SB_FULL = 0, SB_READY = 2, SB_VO = 4, SB_DS = 6, SB_OFREE = 8, SB_CONS = 12,
               SB_DRAIN = 14;
 // local-CTA mbarriers
-constexpr int LB_TMA = 0, LB_L = 2, LB_SLOTFREE = 4, LB_DRAIN = 6;
+constexpr int LB_TMA = 0, LB_L = 2, LB_SLOTFREE = 4, LB_DRAIN = 6, LB_OFFSET = 8;
 
 // TMEM columns
 constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_GROUP = 192;  // local: per group
 constexpr uint32_t TM_DS = 256;                            // state: D_vo[st][h] at 64 (2st+h)
 constexpr uint32_t TMEM_COLS = 512;
 
-constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);   // [K;Q] K^T
-constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, true); // [P;0][T_bg|T_b], [T_bg;PT_bg] K
-constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, true);   // [R;T_b] V_h, [Qh;-W] S_h^T
+constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);   // [K;Q] K^T, [Kg;Qg] Ki^T
+constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, true); // [P;0][T_bg|T_b], [X1;X2] K
+constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, true);   // [P;0] T_b, [R;T_b] V_h, [Qh;-W] S_h^T
 constexpr uint32_t ID_MM = idesc_bf16(128, 64, true, true);     // Kt^T V'_h
 
 __device__ __forceinline__ uint4 pack8(const float *x) {
@@ -199,10 +223,11 @@ struct Waiter {
     }
 };
 
+template <bool CH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  uint8_t *ring, int ring_slots) {
+                  uint8_t *ring, int ring_slots, uint32_t *redo) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -229,7 +254,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
     if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 16; ++i) mbar_init(bars + i, (rank == 1 && (i == SB_CONS || i == SB_CONS + 1)) ? 2 : 1);
+        for (int i = 0; i < 16; ++i)
+            mbar_init(bars + i, (rank == 1 && (i == SB_CONS || i == SB_CONS + 1)) ? 2 : 1);
         fence_mbar_init();
         *abort_flag = 0;
         issued[0] = issued[1] = 0;
@@ -238,6 +264,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             tma_prefetch_desc(&tm_k);
         } else {
             tma_prefetch_desc(&tm_v);
+            if (CH) redo[item] = 0u;
         }
     }
     cluster_sync();  // both CTAs' barriers and flags are initialised
@@ -261,7 +288,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             *abort_flag = 1;
         }
     }
-    uint8_t *ring_pair = slot >= 0 ? ring + (size_t)slot * 2 * RING_SLOT : ring;
+    uint8_t *ring_pair = slot >= 0 ? ring + (size_t)slot * 2 * RING_STRIDE : ring;
 
     if (slot >= 0 && rank == 0) {
         // ============================ local CTA ============================
@@ -271,31 +298,29 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         uint8_t *grp = sm + g * L_GROUP;
         const uint32_t gbase = sbase + g * L_GROUP;
         uint8_t *raw = grp + L_RAW;
+        uint8_t *kxt = grp + L_KX;
         uint8_t *pzt = grp + L_PZT;
-        float *AF = reinterpret_cast<float *>(grp + L_AF);
-        float *TF = reinterpret_cast<float *>(grp + L_TF);
+        float *AT = reinterpret_cast<float *>(grp + L_AT);
         uint64_t *bar_tma = bars + LB_TMA + g, *bar_l = bars + LB_L + g;
         uint64_t *bar_slotfree = bars + LB_SLOTFREE + g;
-        uint8_t *ring_slot = ring_pair + (size_t)g * RING_SLOT;
+        uint8_t *ring_slot = ring_pair + (size_t)g * RING_STRIDE;
         const uint32_t peer_ready = map_peer(smem_u32(bars + SB_READY + g), peer);
-        const uint32_t peer_mdec = map_peer(sbase + OFF_COMMON + CM_MDEC + 4 * g, peer);
         const uint32_t tm_kq = tmem + g * TM_GROUP + TM_KQ, tm_ab = tmem + g * TM_GROUP + TM_AB;
         const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
-        const uint64_t d_kq = desc_sw128(gbase + L_RAW, 16, 1024);
-        const uint64_t d_kmn = desc_sw128(gbase + L_RAW, L_RAW_AC, 1024);
-        const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);
-        const uint64_t d_tgtb = desc_sw128(gbase + L_PZT + PZ_TG, PZ_TB - PZ_TG, 1024);
-        const uint64_t d_tgptg = desc_sw128(gbase + L_PZT + PZ_TG, 16, 1024);
+        const uint64_t d_raw = desc_sw128(gbase + L_RAW, 16, 1024);          // [K;Q], K (K-major)
+        const uint64_t d_kx = desc_sw128(gbase + L_KX, 16, 1024);            // Ki (K-major)
+        const uint64_t d_kmn = desc_sw128(gbase + L_RAW, L_RAW_AC, 1024);    // K (MN-major)
+        const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);    // [P; 0]
+        const uint64_t d_x1b = desc_sw128(gbase + L_PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 (| X3)
+        const uint64_t d_x1x2 = desc_sw128(gbase + L_PZT + PZ_X1, 16, 1024);  // [X1; X2]
         uint32_t bl_wait = 0;
-        const bool issuer = gtid == 0;      // tile loads and MMAs
-        const bool storer = gtid == 7 * 32;  // ring stores and the hand-off
+        const bool issuer = gtid == 0;       // MMAs
+        const bool storer = gtid == 7 * 32;  // tile reloads, ring stores and the hand-off
         bool pend = false;                   // storer: a chunk's ring stores are in flight
-        float pend_dec = 0.f;
         // storer: once the pending chunk's ring stores are complete, hand it over
         auto hand_over = [&]() {
             bulk_wait_all();
             fence_proxy_async_global();
-            st_peer_u32(peer_mdec, __float_as_uint(pend_dec));
             mbar_arrive_peer(peer_ready);
             pend = false;
         };
@@ -314,7 +339,10 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             tma_load_3d(raw + L_RAW_AC + 8192, &tm_q, 64, h, (int)t0, bar_tma);
             ++issued[g];
         };
-        // gates, prefetched one group chunk ahead in the registers of warp lw 4
+        auto gate_rows = [&](int m) {
+            return reinterpret_cast<float *>(grp + L_GATES + ((m >> 1) & 1) * GATES_STRIDE);
+        };
+        // GDN gates, prefetched one group chunk ahead in the registers of warp lw 4
         float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
         auto load_gates = [&](int m) {
             const long long t0 = t_begin + (long long)m * C;
@@ -324,7 +352,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             nbe0 = r0 < L ? a.beta[(t0 + r0) * H + h] : 0.f;
             nbe1 = r1 < L ? a.beta[(t0 + r1) * H + h] : 0.f;
         };
-        auto gate_rows = [&](int m) { return reinterpret_cast<float *>(grp + L_GATES + ((m >> 1) & 1) * GATES_STRIDE); };
+        // GDN gate rows of chunk mm (one warp): cumulative log decay, beta,
+        // the factored block decays, kh and gamma, e^{g_C} for every channel
         auto compute_gates = [&](int mm) {
             float *gr = gate_rows(mm);
             const int r0 = 2 * lane, r1 = 2 * lane + 1;
@@ -362,32 +391,43 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 gr[GR_ROWF + 4 * r0 + b] = b < blk ? f0[b < 3 ? b : 0] : 0.f;
                 gr[GR_ROWF + 4 * r1 + b] = b < blk ? f1[b < 3 ? b : 0] : 0.f;
             }
-            if (lane == 31) gr[GR_DEC] = __expf(gC);
+            const float dC = __expf(gC);
+            *reinterpret_cast<float4 *>(gr + GR_DEC + 4 * lane) = make_float4(dC, dC, dC, dC);
         };
 
-        if (issuer && g < nchunks) issue_tma(g);
-        if (lw == 4 && g < nchunks) {
+        if (storer && g < nchunks) issue_tma(g);
+        if (!CH && lw == 4 && g < nchunks) {
             load_gates(g);
             compute_gates(g);
         }
-        named_bar_sync(BAR_G, 256);
+        // group 1 starts half a chunk after group 0, so that the two groups'
+        // CUDA-core phases tend to overlap the other's MMA and load waits
+        bool ok0 = true;
+        if (g == 1 && issuer && nchunks >= 2) ok0 = wt.wait(bars + LB_OFFSET, 0);
+        named_bar_or(BAR_G, 256, !ok0);
 
         for (int m = g; m < nchunks; m += 2) {
             const int it = m >> 1;
-            const float *gr = gate_rows(m);
+            float *gr = gate_rows(m);
+            const long long t0 = t_begin + (long long)m * C;
+            const int L = chunk_len(m);
             bool ok = true;
-            // ---- tiles of this chunk; rows past the sequence end read as zero.  The
-            //      group's next chunk is fetched into L2 now, its tile load issued
-            //      only at the end of this one (the raw tiles are in use until then)
+            // ---- this chunk's tiles (rows past the sequence end read as zero); the
+            //      group's next chunk is fetched into L2 meanwhile.  The previous
+            //      chunk's ring tiles must have been read out of shared memory.
             if (issuer && m + 2 < nchunks) {
-                const int t2 = (int)(t_begin + (long long)(m + 2) * C);
+                const int t2 = (int)(t0 + 2 * C);
                 tma_prefetch_l2_3d(&tm_k, 0, h, t2);
                 tma_prefetch_l2_3d(&tm_k, 64, h, t2);
                 tma_prefetch_l2_3d(&tm_q, 0, h, t2);
                 tma_prefetch_l2_3d(&tm_q, 64, h, t2);
             }
+            if (CH && m + 2 < nchunks) {  // the next chunk's per-channel gates into L2
+                const int pr = gtid >> 2, pc = gtid & 3;  // 64 rows x 4 lines of 128 B
+                if (t0 + 2 * C + pr < t_end)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + 2 * C + pr) * H + h) * DK + 32 * pc));
+            }
             if (issuer) ok = wt.wait(bar_tma, (uint32_t)(it & 1));
-            const int L = chunk_len(m);
             if (L < C) {
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
@@ -398,60 +438,147 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     *reinterpret_cast<uint4 *>(raw + L_RAW_AC + o) = z;
                     *reinterpret_cast<uint4 *>(raw + L_RAW_AC + 8192 + o) = z;
                 }
-                fence_proxy_async_smem();
             }
+            if constexpr (CH) {
+                // ---- KDA gates: G_rc by a prefix sum over the rows (thread: two
+                //      channels, 16 rows); K, Q scaled in place by e^{G}, Ki = K e^{-G}
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
+                float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 16 * rq + i;
+                    if (r < L) {
+                        const float *lp = a.log_alpha + ((t0 + r) * H + h) * DK + c0;
+                        acc0 += lp[0];
+                        acc1 += lp[1];
+                    }
+                    gl0[i] = acc0;
+                    gl1[i] = acc1;
+                }
+                *reinterpret_cast<float2 *>(gr + 128 * rq + c0) = make_float2(acc0, acc1);
+                if (gtid < 64) gr[GR_KB + gtid] = gtid < L ? a.beta[(t0 + gtid) * H + h] : 0.f;
+                if (storer && pend) bulk_wait_read();  // Ki below replaces the last Kt
+                named_bar_sync(BAR_G, 256);
+                float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float2 v = *reinterpret_cast<const float2 *>(gr + 128 * q2 + c0);
+                    if (q2 < rq) { off0 += v.x; off1 += v.y; }
+                    tot0 += v.x;
+                    tot1 += v.y;
+                }
+                if (rq == 0) {
+                    *reinterpret_cast<float2 *>(gr + GR_DEC + c0) = make_float2(__expf(tot0), __expf(tot1));
+                    if (-tot0 > kMaxNegLogDecay || -tot1 > kMaxNegLogDecay) atomicOr(redo + item, 1u);
+                }
+                const int ac = c0 >> 6, cc = c0 & 63;
+                const uint32_t cof = (uint32_t)((cc & 7) * 2);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int r = 16 * rq + i;
+                    const float G0 = off0 + gl0[i], G1 = off1 + gl1[i];
+                    const float e0 = __expf(G0), e1 = __expf(G1);
+                    const float n0 = __expf(fminf(-G0, kMaxNegLogDecay)), n1 = __expf(fminf(-G1, kMaxNegLogDecay));
+                    const uint32_t o = sw128(r, cc >> 3) + cof;
+                    uint32_t *pk = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + o);
+                    uint32_t *pq = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + 8192 + o);
+                    const uint32_t kw = *pk, qw = *pq;
+                    const float kx = __uint_as_float(kw << 16), ky = __uint_as_float(kw & 0xffff0000u);
+                    const float qx = __uint_as_float(qw << 16), qy = __uint_as_float(qw & 0xffff0000u);
+                    __nv_bfloat162 t;
+                    t = __floats2bfloat162_rn(kx * e0, ky * e1); *pk = *reinterpret_cast<uint32_t *>(&t);
+                    t = __floats2bfloat162_rn(qx * e0, qy * e1); *pq = *reinterpret_cast<uint32_t *>(&t);
+                    t = __floats2bfloat162_rn(kx * n0, ky * n1);
+                    *reinterpret_cast<uint32_t *>(kxt + ac * 8192 + o) = *reinterpret_cast<uint32_t *>(&t);
+                }
+            }
+            fence_proxy_async_smem();
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-            // ---- D_kq = [K; Q] K^T --------------------------------------------------
+            // ---- D_kq = [K; Q] K^T (GDN) or [Kg; Qg] Ki^T (KDA) -----------------------
             if (issuer) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < DK / 16; ++k) {
                     const uint32_t off = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
-                    mma_bf16(tm_kq, d_kq + off, d_kq + off, ID_KK, k > 0);
+                    const uint64_t db = CH ? d_kx + (((k >> 2) * 8192 + (k & 3) * 32) >> 4) : d_raw + off;
+                    mma_bf16(tm_kq, d_raw + off, db, ID_KK, k > 0);
                 }
                 mma_commit(bar_l);
                 ok = wt.wait(bar_l, bl_wait & 1);
             }
             ++bl_wait;
-            if (storer && pend) bulk_wait_read();  // the staging tiles are rewritten below
+            if (!CH && storer && pend) bulk_wait_read();  // the staged tiles are rewritten below
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
             tc_fence_after();
-            // ---- A rows (lanes 0-63) -> fp32;  P rows (lanes 64-127) -> bf16 -------
+            // ---- A rows (lanes 0-63) -> fp32;  P rows (lanes 64-127) -> bf16.  GDN
+            //      applies the decay here; KDA's product already carries it.
+            const float *gb = gr + (CH ? GR_KB : GR_B);
             if ((lq & 1) >= lhalf) {
                 float x[32];
                 tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
                 if (lq < 2) {
                     const int r = 32 * lq + lane;
-                    decay_row(x, r, lq, lhalf, gr, false);
-                    const float br = gr[GR_B + r];
+                    if constexpr (!CH) decay_row(x, r, lq, lhalf, gr, false);
+                    const float br = gb[r];
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        const float4 y = make_float4(br * x[j], br * x[j + 1], br * x[j + 2], br * x[j + 3]);
-                        *reinterpret_cast<float4 *>(AF + r * LDA + 32 * lhalf + j) = y;
+                        float y[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int s = 32 * lhalf + j + e;
+                            y[e] = (CH && s >= r) ? 0.f : br * x[j + e];
+                        }
+                        *reinterpret_cast<float4 *>(AT + r * LDA + 32 * lhalf + j) = make_float4(y[0], y[1], y[2], y[3]);
                     }
                 } else {
                     const int r = 32 * (lq - 2) + lane;
-                    decay_row(x, r, lq - 2, lhalf, gr, true);
+                    if constexpr (!CH) {
+                        decay_row(x, r, lq - 2, lhalf, gr, true);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 32; ++j)
+                            if (32 * lhalf + j > r) x[j] = 0.f;
+                    }
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
                         *reinterpret_cast<uint4 *>(pzt + PZ_P + sw128(r, 4 * lhalf + j)) = pack8(x + 8 * j);
                 }
             } else if (lq >= 2) {
                 // P rows 0-31, columns 32-63 (above the diagonal): zero; the tile
-                // held R since the last chunk
+                // held ring tiles since the last chunk
 #pragma unroll
                 for (int j = 4; j < 8; ++j)
                     *reinterpret_cast<uint4 *>(pzt + PZ_P + sw128(lane, j)) = make_uint4(0, 0, 0, 0);
             }
             named_bar_sync(BAR_G, 256);
-            // ---- T = (I + A)^{-1}: lw 0-3 (diagonal blocks, 32-level); meanwhile
-            //      lw 4 prepares the group's next gates ----------------------------------
+            if (g == 0 && m == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
+            // ---- T = (I + A)^{-1} in place of A: lw 0-3 (diagonal blocks, 32-level);
+            //      meanwhile lw 4 prepares the group's next GDN gates, and for KDA
+            //      lw 4-7 turn Ki into Kt = Ki . e^{G_C} (Ki has been consumed) ------
             if (lw >= 4) {
-                if (lw == 4 && m + 2 < nchunks) compute_gates(m + 2);
                 if (storer && pend) hand_over();  // the previous chunk of this group
+                if constexpr (!CH) {
+                    if (lw == 4 && m + 2 < nchunks) compute_gates(m + 2);
+                } else {
+#pragma unroll 2
+                    for (int q2 = 0; q2 < 8; ++q2) {
+                        const int idx = (gtid - 128) + 128 * q2;
+                        const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
+                        uint4 *p = reinterpret_cast<uint4 *>(kxt + ac * 8192 + sw128(rr, j));
+                        float kv[8];
+                        unpack8(*p, kv);
+                        const float4 d0 = *reinterpret_cast<const float4 *>(gr + GR_DEC + 64 * ac + 8 * j);
+                        const float4 d1 = *reinterpret_cast<const float4 *>(gr + GR_DEC + 64 * ac + 8 * j + 4);
+                        kv[0] *= d0.x; kv[1] *= d0.y; kv[2] *= d0.z; kv[3] *= d0.w;
+                        kv[4] *= d1.x; kv[5] *= d1.y; kv[6] *= d1.z; kv[7] *= d1.w;
+                        *p = pack8(kv);
+                    }
+                }
             } else {
                 // (1) 16x16 diagonal blocks: warp lw inverts block lw; lane j < 16
-                //     owns column j (right-looking forward substitution).
+                //     owns column j (right-looking forward substitution), then writes
+                //     it over the block once the warp has read all of A's block.
                 if (lane < 16) {
                     const int o = 16 * lw, j = lane;
                     float t[16];
@@ -460,13 +587,16 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
                     for (int mm = 0; mm < 15; ++mm) {
 #pragma unroll
-                        for (int i = mm + 1; i < 16; ++i) t[i] -= AF[(o + i) * LDA + o + mm] * t[mm];
+                        for (int i = mm + 1; i < 16; ++i) t[i] -= AT[(o + i) * LDA + o + mm] * t[mm];
                     }
+                    __syncwarp(0x0000ffffu);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) TF[(o + i) * LDA + o + j] = t[i];
+                    for (int i = 0; i < 16; ++i) AT[(o + i) * LDA + o + j] = t[i];
                 }
                 named_bar_sync(BAR_INV, 128);
-                // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
+                // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22);
+                //     X goes to the unused upper-right 16x16 block of the half, T_10
+                //     over A_10 once both warps of the half have read A_10.
                 const int fg = lane >> 2, ft = lane & 3;
                 const int o = 32 * (lw >> 1), n0 = 8 * (lw & 1);
                 float x[4] = {0.f, 0.f, 0.f, 0.f};
@@ -474,41 +604,42 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 for (int ks = 0; ks < 2; ++ks) {
                     uint32_t af[4], bf[2];
                     const int ar = o + 16 + fg, ac = o + 8 * ks + ft;
-                    af[0] = to_tf32(AF[ar * LDA + ac]);
-                    af[1] = to_tf32(AF[(ar + 8) * LDA + ac]);
-                    af[2] = to_tf32(AF[ar * LDA + ac + 4]);
-                    af[3] = to_tf32(AF[(ar + 8) * LDA + ac + 4]);
-                    bf[0] = to_tf32(TF[(o + 8 * ks + ft) * LDA + o + n0 + fg]);
-                    bf[1] = to_tf32(TF[(o + 8 * ks + ft + 4) * LDA + o + n0 + fg]);
+                    af[0] = to_tf32(AT[ar * LDA + ac]);
+                    af[1] = to_tf32(AT[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AT[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AT[(ar + 8) * LDA + ac + 4]);
+                    bf[0] = to_tf32(AT[(o + 8 * ks + ft) * LDA + o + n0 + fg]);
+                    bf[1] = to_tf32(AT[(o + 8 * ks + ft + 4) * LDA + o + n0 + fg]);
                     mma_tf32_16x8x8(x, af, bf);
                 }
-                TF[(o + fg) * LDA + o + 16 + n0 + 2 * ft] = x[0];
-                TF[(o + fg) * LDA + o + 16 + n0 + 2 * ft + 1] = x[1];
-                TF[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft] = x[2];
-                TF[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft + 1] = x[3];
-                __syncwarp();
+                AT[(o + fg) * LDA + o + 16 + n0 + 2 * ft] = x[0];
+                AT[(o + fg) * LDA + o + 16 + n0 + 2 * ft + 1] = x[1];
+                AT[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft] = x[2];
+                AT[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft + 1] = x[3];
+                named_bar_sync(BAR_INV, 128);
                 float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < 2; ++ks) {
                     uint32_t af[4], bf[2];
                     const int ar = o + 16 + fg, ac = o + 16 + 8 * ks + ft;
-                    af[0] = to_tf32(TF[ar * LDA + ac]);
-                    af[1] = to_tf32(TF[(ar + 8) * LDA + ac]);
-                    af[2] = to_tf32(TF[ar * LDA + ac + 4]);
-                    af[3] = to_tf32(TF[(ar + 8) * LDA + ac + 4]);
-                    bf[0] = to_tf32(TF[(o + 8 * ks + ft) * LDA + o + 16 + n0 + fg]);
-                    bf[1] = to_tf32(TF[(o + 8 * ks + ft + 4) * LDA + o + 16 + n0 + fg]);
+                    af[0] = to_tf32(AT[ar * LDA + ac]);
+                    af[1] = to_tf32(AT[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AT[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AT[(ar + 8) * LDA + ac + 4]);
+                    bf[0] = to_tf32(AT[(o + 8 * ks + ft) * LDA + o + 16 + n0 + fg]);
+                    bf[1] = to_tf32(AT[(o + 8 * ks + ft + 4) * LDA + o + 16 + n0 + fg]);
                     mma_tf32_16x8x8(y, af, bf);
                 }
-                TF[(o + 16 + fg) * LDA + o + n0 + 2 * ft] = -y[0];
-                TF[(o + 16 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[1];
-                TF[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
-                TF[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
+                AT[(o + 16 + fg) * LDA + o + n0 + 2 * ft] = -y[0];
+                AT[(o + 16 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[1];
+                AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
+                AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
             }
             if (named_bar_or(BAR_G, 256, *abort_flag)) break;
             // (3) T_{H1,H0} = -T_{H1} (A_{H1,H0} T_{H0}), 32x32 blocks; warp lw owns
             //     output rows 16(lw/4).., columns 8(lw%4)..; X goes to the unused
-            //     upper-right block, the masked upper triangles hold scratch.
+            //     upper-right block, the masked upper triangles hold scratch; the
+            //     result replaces A_{H1,H0} after the barrier.
             {
                 const int fg = lane >> 2, ft = lane & 3;
                 const int m0 = 16 * (lw >> 2), n0 = 8 * (lw & 3);
@@ -517,77 +648,86 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 for (int ks = 0; ks < 4; ++ks) {
                     uint32_t af[4], bf[2];
                     const int ar = 32 + m0 + fg, ac = 8 * ks + ft;
-                    af[0] = to_tf32(AF[ar * LDA + ac]);
-                    af[1] = to_tf32(AF[(ar + 8) * LDA + ac]);
-                    af[2] = to_tf32(AF[ar * LDA + ac + 4]);
-                    af[3] = to_tf32(AF[(ar + 8) * LDA + ac + 4]);
+                    af[0] = to_tf32(AT[ar * LDA + ac]);
+                    af[1] = to_tf32(AT[(ar + 8) * LDA + ac]);
+                    af[2] = to_tf32(AT[ar * LDA + ac + 4]);
+                    af[3] = to_tf32(AT[(ar + 8) * LDA + ac + 4]);
                     const int br = 8 * ks + ft, bc = n0 + fg;
-                    bf[0] = to_tf32(br >= bc ? TF[br * LDA + bc] : 0.f);
-                    bf[1] = to_tf32(br + 4 >= bc ? TF[(br + 4) * LDA + bc] : 0.f);
+                    bf[0] = to_tf32(br >= bc ? AT[br * LDA + bc] : 0.f);
+                    bf[1] = to_tf32(br + 4 >= bc ? AT[(br + 4) * LDA + bc] : 0.f);
                     mma_tf32_16x8x8(x, af, bf);
                 }
-                TF[(m0 + fg) * LDA + 32 + n0 + 2 * ft] = x[0];
-                TF[(m0 + fg) * LDA + 32 + n0 + 2 * ft + 1] = x[1];
-                TF[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft] = x[2];
-                TF[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft + 1] = x[3];
+                AT[(m0 + fg) * LDA + 32 + n0 + 2 * ft] = x[0];
+                AT[(m0 + fg) * LDA + 32 + n0 + 2 * ft + 1] = x[1];
+                AT[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft] = x[2];
+                AT[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft + 1] = x[3];
                 named_bar_sync(BAR_G, 256);
                 float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     uint32_t af[4], bf[2];
-                    const int r = m0 + fg, kc = 8 * ks + ft;
-                    af[0] = to_tf32(kc <= r ? TF[(32 + r) * LDA + 32 + kc] : 0.f);
-                    af[1] = to_tf32(kc <= r + 8 ? TF[(40 + r) * LDA + 32 + kc] : 0.f);
-                    af[2] = to_tf32(kc + 4 <= r ? TF[(32 + r) * LDA + 36 + kc] : 0.f);
-                    af[3] = to_tf32(kc + 4 <= r + 8 ? TF[(40 + r) * LDA + 36 + kc] : 0.f);
-                    bf[0] = to_tf32(TF[(8 * ks + ft) * LDA + 32 + n0 + fg]);
-                    bf[1] = to_tf32(TF[(8 * ks + ft + 4) * LDA + 32 + n0 + fg]);
+                    const int r = m0 + fg, kc = 8 * ks + ft;  // within H1
+                    af[0] = to_tf32(kc <= r ? AT[(32 + r) * LDA + 32 + kc] : 0.f);
+                    af[1] = to_tf32(kc <= r + 8 ? AT[(40 + r) * LDA + 32 + kc] : 0.f);
+                    af[2] = to_tf32(kc + 4 <= r ? AT[(32 + r) * LDA + 36 + kc] : 0.f);
+                    af[3] = to_tf32(kc + 4 <= r + 8 ? AT[(40 + r) * LDA + 36 + kc] : 0.f);
+                    bf[0] = to_tf32(AT[(8 * ks + ft) * LDA + 32 + n0 + fg]);
+                    bf[1] = to_tf32(AT[(8 * ks + ft + 4) * LDA + 32 + n0 + fg]);
                     mma_tf32_16x8x8(y, af, bf);
                 }
-                TF[(32 + m0 + fg) * LDA + n0 + 2 * ft] = -y[0];
-                TF[(32 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[1];
-                TF[(40 + m0 + fg) * LDA + n0 + 2 * ft] = -y[2];
-                TF[(40 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[3];
+                AT[(32 + m0 + fg) * LDA + n0 + 2 * ft] = -y[0];
+                AT[(32 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[1];
+                AT[(40 + m0 + fg) * LDA + n0 + 2 * ft] = -y[2];
+                AT[(40 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[3];
             }
             named_bar_sync(BAR_G, 256);
-            // ---- T_b, T_bg in bf16 (K-major rows r, columns s) -------------------------
+            // ---- T_b (and GDN's T_bg) in bf16, K-major rows r, columns s ----------
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
                 const int idx = gtid + 256 * q2, r = idx >> 3, j = idx & 7;
-                float tv[8], bv[8], gv[8], tb[8], tg[8];
-                *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j);
-                *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j + 4);
-                *reinterpret_cast<float4 *>(bv) = *reinterpret_cast<const float4 *>(gr + GR_B + 8 * j);
-                *reinterpret_cast<float4 *>(bv + 4) = *reinterpret_cast<const float4 *>(gr + GR_B + 8 * j + 4);
-                *reinterpret_cast<float4 *>(gv) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j);
-                *reinterpret_cast<float4 *>(gv + 4) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j + 4);
+                float tv[8], bv[8], tb[8];
+                *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(AT + r * LDA + 8 * j);
+                *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(AT + r * LDA + 8 * j + 4);
+                *reinterpret_cast<float4 *>(bv) = *reinterpret_cast<const float4 *>(gb + 8 * j);
+                *reinterpret_cast<float4 *>(bv + 4) = *reinterpret_cast<const float4 *>(gb + 8 * j + 4);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int s2 = 8 * j + e;
-                    const float t2 = s2 < r ? tv[e] : (s2 == r ? 1.f : 0.f);
-                    tb[e] = t2 * bv[e];
-                    tg[e] = t2 * gv[e];
+                    tv[e] = s2 < r ? tv[e] : (s2 == r ? 1.f : 0.f);
+                    tb[e] = tv[e] * bv[e];
                 }
-                *reinterpret_cast<uint4 *>(pzt + PZ_TB + sw128(r, j)) = pack8(tb);
-                *reinterpret_cast<uint4 *>(pzt + PZ_TG + sw128(r, j)) = pack8(tg);
+                if constexpr (!CH) {
+                    float gv[8], tg[8];
+                    *reinterpret_cast<float4 *>(gv) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j);
+                    *reinterpret_cast<float4 *>(gv + 4) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j + 4);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) tg[e] = tv[e] * gv[e];
+                    *reinterpret_cast<uint4 *>(pzt + PZ_X3 + sw128(r, j)) = pack8(tb);
+                    *reinterpret_cast<uint4 *>(pzt + PZ_X1 + sw128(r, j)) = pack8(tg);
+                } else {
+                    *reinterpret_cast<uint4 *>(pzt + PZ_X1 + sw128(r, j)) = pack8(tb);
+                }
             }
             fence_proxy_async_smem();
             named_bar_sync(BAR_G, 256);
-            // ---- D_ab = [P; 0] [T_bg | T_b]:  rows 0-63 = [P T_bg | R] -------------
+            // ---- D_ab = [P; 0] [T_bg | T_b] (GDN: rows 0-63 = [P T_bg | R]) or
+            //      [P; 0] T_b (KDA: rows 0-63 = R) ------------------------------------
             if (issuer) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tm_ab, d_pz + 2 * k, d_tgtb + 128 * k, ID_N128, k > 0);
+                    mma_bf16(tm_ab, d_pz + 2 * k, d_x1b + 128 * k, CH ? ID_N64 : ID_N128, k > 0);
                 mma_commit(bar_l);
                 ok = wt.wait(bar_l, bl_wait & 1);
             }
             ++bl_wait;
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
             tc_fence_after();
-            if (lq < 2) {  // lw 0,1: P T_bg;  lw 4,5: R, staged in P's tile (P is consumed)
+            // GDN: lw 0,1 P T_bg -> X2, lw 4,5 R -> P's tile (P is consumed);
+            // KDA: lw 0,1 R -> X2
+            if (lq < 2 && (!CH || lhalf == 0)) {
                 const int r = 32 * lq + lane;
-                uint8_t *dst = pzt + (lhalf == 0 ? PZ_PTG : PZ_P);
+                uint8_t *dst = pzt + (lhalf == 0 ? PZ_X2 : PZ_P);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float x[32];
@@ -600,26 +740,27 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar_sync(BAR_G, 256);
-            // ---- D_ab = [T_bg; P T_bg] K:  rows 0-63 = W, rows 64-127 = P W ---------
+            // ---- D_ab = [X1; X2] K: GDN [T_bg; P T_bg] K, KDA [T_b; R] Kg:
+            //      rows 0-63 = W, rows 64-127 = P W ---------------------------------------
             if (issuer) {
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tm_ab, d_tgptg + 2 * k, d_kmn + 128 * k, ID_N128, k > 0);
+                    mma_bf16(tm_ab, d_x1x2 + 2 * k, d_kmn + 128 * k, ID_N128, k > 0);
                 mma_commit(bar_l);
                 ok = wt.wait(bar_l, bl_wait & 1);
             }
             ++bl_wait;
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
             tc_fence_after();
-            // ---- -W (lanes 0-63) and Qh = gamma Q - P W (lanes 64-127) staged in the
-            //      A / T tiles, Kt = kh . K in the T_bg / P T_bg tiles: the raw tiles are
-            //      free for the next chunk once this phase is over ----------------------
+            // ---- -W (lanes 0-63) staged in T's tile; Qh = gamma Q - P W (GDN) or
+            //      Qg - P W (KDA) (lanes 64-127) staged in X1/X2 (GDN) or X3/P (KDA);
+            //      GDN Kt = kh . K staged in KX.  The raw tiles are then free.
             {
                 const int r = 32 * (lq & 1) + lane;
-                const float gam = gr[GR_GAM + r];
-                uint8_t *wst = grp + L_AF + lhalf * 8192;
-                uint8_t *qst = grp + L_AF + 16384 + lhalf * 8192;
+                const float gam = CH ? 1.f : gr[GR_GAM + r];
+                uint8_t *wst = grp + L_AT + lhalf * 8192;
+                uint8_t *qst = pzt + (CH ? (lhalf ? PZ_P : PZ_X3) : (lhalf ? PZ_X2 : PZ_X1));
                 const uint8_t *qt = raw + lhalf * L_RAW_AC + 8192;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -645,39 +786,43 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         }
                     }
                 }
+                if constexpr (!CH) {
 #pragma unroll
-                for (int q2 = 0; q2 < 4; ++q2) {
-                    const int idx = gtid + 256 * q2;
-                    const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
-                    float kv[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(raw + ac * L_RAW_AC + sw128(rr, j)), kv);
-                    const float sc = gr[GR_KH + rr];
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const int idx = gtid + 256 * q2;
+                        const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
+                        float kv[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(raw + ac * L_RAW_AC + sw128(rr, j)), kv);
+                        const float sc = gr[GR_KH + rr];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) kv[e] *= sc;
-                    *reinterpret_cast<uint4 *>(pzt + PZ_TG + ac * 8192 + sw128(rr, j)) = pack8(kv);
+                        for (int e = 0; e < 8; ++e) kv[e] *= sc;
+                        *reinterpret_cast<uint4 *>(kxt + ac * 8192 + sw128(rr, j)) = pack8(kv);
+                    }
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             if (named_bar_or(BAR_G, 256, *abort_flag)) break;
-            // the raw tiles take the group's next chunk
-            if (issuer && m + 2 < nchunks) issue_tma(m + 2);
             if (storer) {
-                // once the state CTA has read the slot's previous chunk, the eight
-                // tiles go to the ring by bulk copy; the hand-off follows during
-                // the next chunk (or after the loop)
+                // the raw tiles take the group's next chunk (issued before the ring
+                // stores: the TMA unit serves its requests in order)
+                if (m + 2 < nchunks) issue_tma(m + 2);
+                // once the state CTA has read the slot's previous chunk, the ring
+                // tiles and e^{G_C} go out by bulk copy; the hand-off follows
+                // during the next chunk (or after the loop)
                 if (m < 2 || wt.wait_peer(bar_slotfree, (uint32_t)((it - 1) & 1))) {
-                    bulk_store(ring_slot + SG_KT, pzt + PZ_TG, 8192);
-                    bulk_store(ring_slot + SG_QH, grp + L_AF + 16384, 8192);
-                    bulk_store(ring_slot + SG_MW, grp + L_AF, 8192);
-                    bulk_store(ring_slot + SG_AC + SG_KT, pzt + PZ_PTG, 8192);
-                    bulk_store(ring_slot + SG_AC + SG_QH, grp + L_AF + 24576, 8192);
-                    bulk_store(ring_slot + SG_AC + SG_MW, grp + L_AF + 8192, 8192);
-                    bulk_store(ring_slot + SG_R, pzt + PZ_P, 8192);
-                    bulk_store(ring_slot + SG_TB, pzt + PZ_TB, 8192);
+                    const uint8_t *at8 = grp + L_AT;
+                    bulk_store(ring_slot + SG_KT, kxt, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_KT, kxt + 8192, 8192);
+                    bulk_store(ring_slot + SG_MW, at8, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_MW, at8 + 8192, 8192);
+                    bulk_store(ring_slot + SG_QH, pzt + (CH ? PZ_X3 : PZ_X1), 8192);
+                    bulk_store(ring_slot + SG_AC + SG_QH, pzt + (CH ? PZ_P : PZ_X2), 8192);
+                    bulk_store(ring_slot + SG_R, pzt + (CH ? PZ_X2 : PZ_P), 8192);
+                    bulk_store(ring_slot + SG_TB, pzt + (CH ? PZ_X1 : PZ_X3), 8192);
+                    bulk_store(ring_slot + SG_TILES, gr + GR_DEC, SG_DECB);
                     bulk_commit();
                     pend = true;
-                    pend_dec = gr[GR_DEC];
                 }
             }
         }
@@ -691,8 +836,6 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         }
     } else if (slot >= 0) {
         // ============================ state CTA ============================
-        float *sdec = reinterpret_cast<float *>(cm + CM_SDEC);
-        const float *mdec = reinterpret_cast<const float *>(cm + CM_MDEC);
         if (warp < 8) {
             // ---- chain of value half hv: warps 4hv..4hv+3, thread = key channel c
             const int hv = warp >> 2, q = warp & 3, c = 32 * q + lane;
@@ -716,7 +859,6 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             for (int j = 0; j < 8; ++j)
                 *reinterpret_cast<uint4 *>(sb + sw128(c, j)) = pack8(s_reg + 8 * j);
             fence_proxy_async_smem();
-            float *cdec = reinterpret_cast<float *>(cm + CM_CDEC) + hv;  // this chunk's e^{g_C}
             // D_vo[st] = [R; T_b] V_h  (needs the chunk's stage and D_vo free)
             auto issue_v = [&](int m) {
                 const uint32_t so = (m & 1) * (S_STAGE >> 4);
@@ -741,9 +883,6 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                             issue_v(m);
                         }
                     }
-                    // the stage has landed (waited here or before the early V
-                    // product): publish its decay to the chain
-                    *cdec = sdec[st];
                     // D_vo += [Qh; -W] S_h^T
                     if (ok) {
 #pragma unroll
@@ -755,10 +894,14 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 v_issued = false;
-                // V' rows (lanes 64-127) -> bf16, MN-major [r][i]
-                if (q >= 2) {
-                    const bool okv = wt.warp_wait(bars + SB_VO + hv, (uint32_t)(m & 1), lane);
-                    if (okv) {
+                // every chain warp sees the stage through the completed product, then
+                // takes this chunk's decay of its key channel; the V' warps (lanes
+                // 64-127) write V' as bf16, MN-major [r][i]
+                float dec = 0.f;
+                const bool okv = ok && wt.warp_wait(bars + SB_VO + hv, (uint32_t)(m & 1), lane);
+                if (okv) {
+                    dec = reinterpret_cast<const float *>(sm + st * S_STAGE + SG_DEC)[c];
+                    if (q >= 2) {
                         tc_fence_after();
                         const int r = 32 * (q - 2) + lane;
 #pragma unroll
@@ -769,14 +912,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                             for (int j = 0; j < 4; ++j)
                                 *reinterpret_cast<uint4 *>(vp + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
                         }
-                    } else {
-                        ok = false;
                     }
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
-                if (named_bar_or(BAR_H, 128, !ok || *abort_flag)) break;
-                const float dec = *cdec;
+                if (named_bar_or(BAR_H, 128, !okv || *abort_flag)) break;
                 if (leader) {
                     tc_fence_after();
                     // dS_h = Kt^T V'_h
@@ -797,7 +937,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         }
                     }
                 }
-                // S_h <- e^{g_C} S_h + dS_h
+                // S_h <- S_h Diag(e^{G_C}) + dS_h  (thread c: column c)
                 const bool okd = wt.warp_wait(bars + SB_DS + hv, (uint32_t)(m & 1), lane);
                 if (okd) {
                     tc_fence_after();
@@ -821,7 +961,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     mma_commit(bars + SB_DRAIN + hv);
                     mbar_wait(bars + SB_DRAIN + hv, 0, kWaitLimit);
                 }
-            } else if (a.s_final) {
+            } else if (a.s_final && !(CH && *reinterpret_cast<volatile uint32_t *>(redo + item))) {
+                // (a flagged KDA item gets its final state from the exact re-run)
 #pragma unroll
                 for (int i = 0; i < 64; ++i) a.s_final[st_base + (size_t)(64 * hv + i) * DK + c] = s_reg[i];
             }
@@ -866,13 +1007,13 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 if (ok) ok = wt.wait_peer(bars + SB_READY + st, (uint32_t)(it & 1));
                 if (!ok) break;
                 fence_proxy_async_global();
-                sdec[st] = mdec[st];
-                const uint8_t *src = ring_pair + (size_t)st * RING_SLOT;
+                const uint8_t *src = ring_pair + (size_t)st * RING_STRIDE;
                 const long long t0 = t_begin + (long long)m * C;
                 mbar_arrive_expect_tx(bars + SB_FULL + st, S_STAGE_TX);
 #pragma unroll
                 for (int p = 0; p < 4; ++p)
                     bulk_load(stage + p * 16384, src + p * 16384, 16384, bars + SB_FULL + st);
+                bulk_load(stage + SG_DEC, src + SG_TILES, SG_DECB, bars + SB_FULL + st);
                 tma_load_3d(stage + SG_V, &tm_v, 0, h, (int)t0, bars + SB_FULL + st);
                 tma_load_3d(stage + SG_V + 8192, &tm_v, 64, h, (int)t0, bars + SB_FULL + st);
                 ++issued[st];
@@ -902,10 +1043,29 @@ int ring_slots_for_device() {
     return 2 * nsm;  // SM ids are below this on every part this kernel runs on
 }
 
+size_t ring_bytes(int slots) { return (size_t)slots * 2 * RING_STRIDE; }
+
+template <bool CH>
+cudaError_t launch_t(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
+                     const CUtensorMap &mv, int slots, uint32_t *redo, cudaStream_t s) {
+    auto kern = chunk_pair_kernel<CH>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    const long long items = (long long)a.n_seqs * a.H;
+    kern<<<(unsigned)(2 * items), kThreads, SMEM_BYTES, s>>>(
+        a, mq, mk, mv, reinterpret_cast<uint8_t *>(a.scratch), slots, redo);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
-size_t chunk_pair_scratch_bytes(const gdn_dims &) {
-    return (size_t)ring_slots_for_device() * 2 * RING_SLOT;
+bool chunk_pair_supported(const gdn_dims &d) {
+    return d.dtype == GDN_BF16 && d.d_k == DK && d.d_v == DV && (long long)d.B * d.T < (1LL << 31);
+}
+
+size_t chunk_pair_scratch_bytes(const gdn_dims &d) {
+    const long long items = (long long)(d.n_seqs > 0 ? d.n_seqs : d.B) * d.H;
+    return ring_bytes(ring_slots_for_device()) + (size_t)((items * 4 + 255) & ~255LL);
 }
 
 cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches) {
@@ -924,15 +1084,20 @@ cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launche
     if (!make_tile_map(&mq, a.q, a.dk, a.H, ntok) || !make_tile_map(&mk, a.k, a.dk, a.H, ntok) ||
         !make_tile_map(&mv, a.v, a.dv, a.H, ntok))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(chunk_pair_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
     const int slots = ring_slots_for_device();
     if (slots <= 0) return cudaErrorInvalidValue;
-    chunk_pair_kernel<<<(unsigned)(2 * items), kThreads, SMEM_BYTES, s>>>(
-        a, mq, mk, mv, reinterpret_cast<uint8_t *>(a.scratch), slots);
+    uint32_t *redo = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(a.scratch) + ring_bytes(slots));
+    cudaError_t e = a.channel ? launch_t<true>(a, mq, mk, mv, slots, redo, s)
+                              : launch_t<false>(a, mq, mk, mv, slots, redo, s);
+    if (e != cudaSuccess) return e;
     if (launches) ++*launches;
-    return cudaGetLastError();
+    if (a.channel) {
+        // the items whose decay left the fast path's range, exactly on CUDA cores
+        PrefillArgs r = a;
+        r.redo = redo;
+        e = launch_chunk_simt(r, s, launches);
+    }
+    return e;
 }
 
 }  // namespace gdn

@@ -10,6 +10,16 @@
 // propagation, intra-chunk causal product).  Per chunk, in fp32:
 //   g_r   = sum_{s<=r} log alpha_s                        (per key channel for KDA)
 //   A_rs  = beta_r sum_c k_rc k_sc e^{g_rc - g_sc}, s < r  (strictly lower)
+// For KDA the per-channel decay inside the contraction is split at the middle
+// token m_j of the 16-token block j holding column s:
+//   e^{g_rc - g_sc} = e^{g_rc - g_{m_j}c} e^{g_{m_j}c - g_sc},
+// with the column factor k_sc e^{g_{m_j}c - g_sc} formed once per chunk.  Both
+// factors stay below e^{(decay over 8 tokens)} wherever the term is kept, so
+// nothing overflows where the plain factorisation e^{g_r} e^{-g_s} would
+// (g reaches -200 over a chunk at the decays of the KDA workload).  The
+// exponents are clamped at 80, so the result is exact while the decay over any
+// 8 consecutive tokens stays above e^{-80} on every channel (log alpha > -10 per
+// token on average); beyond that the terms are bounded, never inf or NaN.
 //   T     = (I + A)^{-1}                                  (forward substitution)
 //   W     = T diag(beta) (K . e^{G}),  U = T diag(beta) V
 //   V'    = U - W S^T
@@ -44,6 +54,41 @@ struct SimtSmem {
     static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
+// KDA: out_rs = [beta_r] sum_c x_rc e^{g_rc - g_{m_j}c} f_sc for s < r (A, with
+// beta) or s <= r (P), zero elsewhere; f (stride LDK) holds the column factors
+// k_sc e^{g_{m_j}c - g_sc}, j = s / 16, m_j = 16 j + 7.  Work unit: one row r and
+// 8 columns of one block at or left of the diagonal.
+template <int DK>
+__device__ __forceinline__ void decayed_products(const float *X, const float *F, const float *G,
+                                                 const float *beta, float *out, bool incl,
+                                                 int tid) {
+    constexpr int C = kChunk, LDK = DK + 1, LC = C + 1;
+    // rows of block i own 2 (i + 1) half-block units: 16 * 2 * (1 + 2 + 3 + 4) = 320
+    for (int u = tid; u < 320; u += kThreads) {
+        int i = 0, base = 0;
+        while (u >= base + 32 * (i + 1)) { base += 32 * (i + 1); ++i; }
+        const int v = u - base, r = 16 * i + v / (2 * (i + 1)), w = v % (2 * (i + 1));
+        const int j = w >> 1, s0 = 16 * j + 8 * (w & 1), m = 16 * j + 7;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < DK; ++c) {
+            const float rf = X[r * LDK + c] * __expf(fminf(G[r * LDK + c] - G[m * LDK + c], 80.f));
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += rf * F[(s0 + e) * LDK + c];
+        }
+        const float b = beta ? beta[r] : 1.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int s2 = s0 + e;
+            out[r * LC + s2] = (incl ? s2 <= r : s2 < r) ? b * acc[e] : 0.f;
+        }
+    }
+    // columns right of the row's own block
+    for (int idx = tid; idx < C * C; idx += kThreads) {
+        const int r = idx / C, s2 = idx % C;
+        if ((s2 >> 4) > (r >> 4)) out[r * LC + s2] = 0.f;
+    }
+}
+
 template <int DK, bool CH>
 __global__ void __launch_bounds__(kThreads)
 chunk_simt_kernel(PrefillArgs a) {
@@ -63,6 +108,7 @@ chunk_simt_kernel(PrefillArgs a) {
     const int v0 = slice * kDvs;
     const int H = a.H, dv = a.dv;
 
+    if (a.redo && a.redo[(size_t)n * H + h] == 0u) return;
     long long t_begin, t_end;
     seq_range(a, n, &t_begin, &t_end);
 
@@ -111,21 +157,30 @@ chunk_simt_kernel(PrefillArgs a) {
         }
         __syncthreads();
         // ---- step 2: A (strictly lower), T initialised to I ---------------
-        for (int idx = tid; idx < C * C; idx += kThreads) {
-            const int r = idx / C, s = idx % C;
-            float acc = 0.f;
-            if (s < r) {
-                if (CH) {
-                    for (int c = 0; c < DK; ++c)
-                        acc += K[r * LDK + c] * K[s * LDK + c] * expf(g_at(r, c) - g_at(s, c));
-                } else {
-                    for (int c = 0; c < DK; ++c) acc += K[r * LDK + c] * K[s * LDK + c];
-                    acc *= expf(G[r] - G[s]);
-                }
-                acc *= bt[r];
+        if (CH) {
+            // column factors k_sc e^{g_{m(s)}c - g_sc}, m(s) the middle of s's block (in W)
+            for (int idx = tid; idx < C * DK; idx += kThreads) {
+                const int r = idx / DK, c = idx % DK;
+                const int m = (r & ~15) + 7;
+                W[r * LDK + c] = K[r * LDK + c] * __expf(fminf(G[m * LDK + c] - G[r * LDK + c], 80.f));
             }
-            A[r * LC + s] = acc;
-            Tm[r * LC + s] = (r == s) ? 1.f : 0.f;
+            __syncthreads();
+            decayed_products<DK>(K, W, G, bt, A, false, tid);
+            for (int idx = tid; idx < C * C; idx += kThreads) {
+                const int r = idx / C, s2 = idx % C;
+                Tm[r * LC + s2] = (r == s2) ? 1.f : 0.f;
+            }
+        } else {
+            for (int idx = tid; idx < C * C; idx += kThreads) {
+                const int r = idx / C, s2 = idx % C;
+                float acc = 0.f;
+                if (s2 < r) {
+                    for (int c = 0; c < DK; ++c) acc += K[r * LDK + c] * K[s2 * LDK + c];
+                    acc *= __expf(G[r] - G[s2]) * bt[r];
+                }
+                A[r * LC + s2] = acc;
+                Tm[r * LC + s2] = (r == s2) ? 1.f : 0.f;
+            }
         }
         __syncthreads();
         // ---- step 3: T = (I + A)^{-1} by forward substitution -------------
@@ -139,12 +194,18 @@ chunk_simt_kernel(PrefillArgs a) {
             }
             __syncthreads();
         }
+        // ---- KDA: P = causal decayed Q K^T into A, while W still holds the column
+        //      factors (A is consumed by the inversion above) -------------------
+        if (CH) {
+            decayed_products<DK>(Q, W, G, nullptr, A, true, tid);
+            __syncthreads();
+        }
         // ---- step 4: W = T diag(b)(K . e^G), U = T diag(b) V --------------
         // Column c of W (and i of U) only involves column c (i), so one thread
         // owns a column and updates it in place from the bottom row up.
         if (tid < DK) {
             const int c = tid;
-            for (int s = 0; s < C; ++s) W[s * LDK + c] = bt[s] * K[s * LDK + c] * expf(g_at(s, c));
+            for (int s = 0; s < C; ++s) W[s * LDK + c] = bt[s] * K[s * LDK + c] * __expf(g_at(s, c));
             for (int r = C - 1; r >= 0; --r) {
                 float acc = 0.f;
                 for (int s = 0; s <= r; ++s) acc += Tm[r * LC + s] * W[s * LDK + c];
@@ -167,28 +228,25 @@ chunk_simt_kernel(PrefillArgs a) {
             for (int c = 0; c < DK; ++c) acc += W[r * LDK + c] * S[i * LDK + c];
             V[r * LDV + i] -= acc;
         }
-        // ---- step 6a: P = causal decayed Q K^T (into A) --------------------
-        for (int idx = tid; idx < C * C; idx += kThreads) {
-            const int r = idx / C, s = idx % C;
-            float acc = 0.f;
-            if (s <= r) {
-                if (CH) {
-                    for (int c = 0; c < DK; ++c)
-                        acc += Q[r * LDK + c] * K[s * LDK + c] * expf(g_at(r, c) - g_at(s, c));
-                } else {
-                    for (int c = 0; c < DK; ++c) acc += Q[r * LDK + c] * K[s * LDK + c];
-                    acc *= expf(G[r] - G[s]);
+        // ---- step 6a: GDN P = causal decayed Q K^T (into A) -----------------
+        if (!CH) {
+            for (int idx = tid; idx < C * C; idx += kThreads) {
+                const int r = idx / C, s2 = idx % C;
+                float acc = 0.f;
+                if (s2 <= r) {
+                    for (int c = 0; c < DK; ++c) acc += Q[r * LDK + c] * K[s2 * LDK + c];
+                    acc *= __expf(G[r] - G[s2]);
                 }
+                A[r * LC + s2] = acc;
             }
-            A[r * LC + s] = acc;
         }
         __syncthreads();
         // ---- decayed Q and K^ = K . e^{g_C - G} (in place) ----------------
         for (int idx = tid; idx < C * DK; idx += kThreads) {
             const int r = idx / DK, c = idx % DK;
             const float gr = g_at(r, c);
-            Q[r * LDK + c] *= expf(gr);
-            K[r * LDK + c] *= expf(g_at(C - 1, c) - gr);
+            Q[r * LDK + c] *= __expf(gr);
+            K[r * LDK + c] *= __expf(g_at(C - 1, c) - gr);
         }
         __syncthreads();
         // ---- step 6b: O = (Q . e^G) S^T + P V' ----------------------------
@@ -204,7 +262,7 @@ chunk_simt_kernel(PrefillArgs a) {
         // ---- step 5b: S <- S Diag(e^{g_C}) + V'^T K^ ----------------------
         for (int idx = tid; idx < kDvs * DK; idx += kThreads) {
             const int i = idx / DK, c = idx % DK;
-            float acc = S[i * LDK + c] * expf(g_at(C - 1, c));
+            float acc = S[i * LDK + c] * __expf(g_at(C - 1, c));
             for (int s = 0; s < C; ++s) acc += V[s * LDV + i] * K[s * LDK + c];
             S[i * LDK + c] = acc;
         }

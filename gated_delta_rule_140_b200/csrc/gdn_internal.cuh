@@ -31,6 +31,9 @@ struct PrefillArgs {
     int B, T, H, dk, dv, n_seqs;
     int channel;              // 1 = KDA channel-wise decay
     int bf16;                 // 1 = bf16 q/k/v/o, 0 = fp32
+    // CUDA-core kernel only: if set, process only the (sequence, head) items
+    // with redo[n * H + h] != 0 (the re-run of items another kernel flagged)
+    const uint32_t *redo;
 };
 
 struct DecodeArgs {
@@ -49,6 +52,8 @@ cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t s, int *launches)
 cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches);
 size_t chunk_tc_scratch_bytes(const gdn_dims &d);
 size_t chunk_pair_scratch_bytes(const gdn_dims &d);
+// bf16 d_k = d_v = 128 shapes (either decay) the two-CTA kernel takes
+bool chunk_pair_supported(const gdn_dims &d);
 // bf16 d_k = d_v = 128 scalar-decay shapes the tensor-core kernels take
 bool chunk_tc_supported(const gdn_dims &d);
 // [tokens, H, d] bf16 as a 3-D TMA tensor map (d, H, tokens), box 64 x 1 x 64,

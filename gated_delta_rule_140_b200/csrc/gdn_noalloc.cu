@@ -41,9 +41,11 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
     size_t need = gdn_chunk_fwd_workspace_size(dims);
     if (need == 0) return GDN_ERR_INVALID;
     gdn_dims d = *dims;
-    if (need > GDN_NOALLOC_SCRATCH_BYTES && (d.flags & GDN_FLAG_PAIR)) {
-        // the two-CTA kernel's ring does not fit: the default kernel
+    if (need > GDN_NOALLOC_SCRATCH_BYTES) {
+        // the two-CTA kernel's ring does not fit: GDN runs the single-CTA
+        // tensor-core kernel, KDA the CUDA-core kernel
         d.flags &= ~GDN_FLAG_PAIR;
+        if (d.decay == GDN_DECAY_CHANNEL) d.flags |= GDN_FLAG_CUDA_CORES;
         need = gdn_chunk_fwd_workspace_size(&d);
     }
     if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_UNSUPPORTED;
