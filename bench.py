@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--decode-workload NAME]
+                    [--prefill-kernel default|pair|cuda_cores]
 
 A step is one pass of the whole hot path on one GPU:
   * prefill leg: gdn_chunk_fwd over one batch of the prefill workload
@@ -277,9 +278,12 @@ def run_ours(args, rank, world, local):
     steps_d = xd["q"].shape[0]
     stream = torch.cuda.current_stream()
 
+    kflags = {"pair": args.prefill_kernel == "pair",
+              "cuda_cores": args.prefill_kernel == "cuda_cores"}
+
     def prefill():
         chunk_fwd(xp["q"], xp["k"], xp["v"], xp["log_alpha"], xp["beta"], xp["initial_state"],
-                  xp["cu_seqlens"], o=o, final_state=sf, workspace=ws)
+                  xp["cu_seqlens"], o=o, final_state=sf, workspace=ws, **kflags)
 
     def decode(t):
         i = t % steps_d
@@ -335,7 +339,8 @@ def run_ours(args, rank, world, local):
             if v is not None:
                 dbuf[k2].copy_(v, non_blocking=True)
         chunk_fwd(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"],
-                  dbuf["initial_state"], dbuf["cu_seqlens"], o=o, final_state=sf, workspace=ws)
+                  dbuf["initial_state"], dbuf["cu_seqlens"], o=o, final_state=sf, workspace=ws,
+                  **kflags)
         o_h.copy_(o, non_blocking=True)
         sf_h.copy_(sf, non_blocking=True)
 
@@ -363,7 +368,7 @@ def run_ours(args, rank, world, local):
                               wd.decay == "channel")
         pre_s, dec_s = pre_ms / K / 1e3, dec_ms / K / 1e3
         path = nat.chunk_fwd_path(nat.prefill_dims(xp["q"], xp["v"], xp["log_alpha"],
-                                                   xp["cu_seqlens"]))
+                                                   xp["cu_seqlens"], **kflags))
         pre_kernel, pre_src = {
             "tensor_core_pair": ("chunk_pair_kernel", "gdn_chunk_pair.cu"),
             "tensor_core": ("chunk_tc_kernel", "gdn_chunk_tc.cu"),
@@ -380,7 +385,7 @@ def run_ours(args, rank, world, local):
                     "kernel": "decode_kernel", "alg_bytes": dbytes, "peak_source": pk_kind}
         dominant = roof_pre if pre_s >= dec_s else roof_dec
         cfg = {"workload": args.workload, "B": B, "T": T, "H": H, "d_k": dk, "d_v": dv,
-               "decay": wp.decay, "chunk": 64, "parallelism": f"dp{world} (independent batches)",
+               "decay": wp.decay, "chunk": 64, "prefill_kernel": pre_kernel, "parallelism": f"dp{world} (independent batches)",
                "l2": "inputs larger than L2 (no flush)",
                "decode_workload": f"{args.decode_workload}: N={wd.B}, H={wd.H}, d={wd.d}, "
                                   "fp32 state in place"}
@@ -419,6 +424,10 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill_bf16")
     ap.add_argument("--decode-workload", default="gdn_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-kernel", choices=["default", "pair", "cuda_cores"],
+                    default="default",
+                    help="prefill kernel: the library's choice, the two-CTA tensor-core "
+                         "kernel (GDN_FLAG_PAIR) or the fp32 CUDA-core kernel")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
