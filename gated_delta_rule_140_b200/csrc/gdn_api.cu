@@ -32,11 +32,11 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
 enum class Path { kPair, kOneCta, kCudaCores };
 
 // The prefill kernel a call runs.  bf16, d_k = d_v = 128: GDN the single-CTA
-// tensor-core kernel, or either decay the two-CTA kernel with GDN_FLAG_PAIR;
-// every other case, or GDN_FLAG_CUDA_CORES, the fp32 CUDA-core kernel.
+// tensor-core kernel (the two-CTA one with GDN_FLAG_PAIR), KDA the two-CTA
+// kernel; every other case, or GDN_FLAG_CUDA_CORES, the fp32 CUDA-core kernel.
 Path select_path(const gdn_dims &d) {
     if ((d.flags & GDN_FLAG_CUDA_CORES) || !gdn::chunk_pair_supported(d)) return Path::kCudaCores;
-    if (d.flags & GDN_FLAG_PAIR) return Path::kPair;
+    if (d.decay == GDN_DECAY_CHANNEL || (d.flags & GDN_FLAG_PAIR)) return Path::kPair;
     return gdn::chunk_tc_supported(d) ? Path::kOneCta : Path::kCudaCores;
 }
 

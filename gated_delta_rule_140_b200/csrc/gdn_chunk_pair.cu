@@ -30,9 +30,14 @@
 //        factored, exact inside the diagonal 32x32 blocks); T_bg = T_b
 //        diag(e^{g}) so that W = T_bg K; [P T_bg | R] = P [T_bg | T_b];
 //        [W; P W] = [T_bg; P T_bg] K.
-//   KDA: K and Q are scaled in place to Kg, Qg and Ki = K . e^{-G} is formed,
-//        so that D = [Kg; Qg] Ki^T is the decayed product directly (A and P
-//        only take masks); R = P T_b; [W; P W] = [T_b; R] Kg.
+//   KDA (one group, the other's shared memory holding its extra operands):
+//        each 16-token row block i takes the reference m_i = 16 i + 7 (its
+//        middle token): K and Q become KD, QD = . e^{G - G_{m(r)}} in place, and
+//        B_i = K[0, 16(i+1)) . e^{G_{m_i} - G}, so that D_i = [KD; QD] B_i^T
+//        (four MMAs, N = 16, 32, 48, 64) holds the decayed A and P of block i
+//        (masks only); every factor is within 8 tokens' decay of 1.  Then
+//        R = P T_b, Kg = KD . e^{G_{m(r)}}, [W; P W] = [T_b; R] Kg, and
+//        Qh = QD . e^{G_{m(r)}} - P W.
 // T comes from blocked forward substitution in fp32 (tf32 MMAs for the
 // off-diagonal blocks), computed in place of A.
 // Rank 1 ("state" CTA) holds S (fp32, registers) for all 128 value channels as
@@ -41,11 +46,12 @@
 // issues D = [R;T_b] V_h + [Qh;-W] S_h^T, writes o, converts V' to bf16 and
 // issues dS = Kt^T V'.
 //
-// KDA range: Ki = K . e^{-G} is finite while a chunk's total decay on every
-// channel is above e^{-kMaxNegLogDecay}.  A chunk past that is computed with the
-// factor clamped, and its (sequence, head) is flagged in the workspace; the
-// host re-runs the flagged items exactly on the CUDA-core kernel, and this
-// kernel leaves their final state to it.
+// KDA range: the factors are finite while the decay over any 8 consecutive
+// tokens stays above e^{-kMaxNegLogDecay} on every channel (log alpha > -10 per
+// token on average; the KDA workload's -3 is far inside).  A chunk past that is
+// computed with the exponents clamped and its (sequence, head) is flagged in the
+// workspace; the host re-runs the flagged items on the CUDA-core kernel, which
+// is exact for any decay, and this kernel leaves their final state to it.
 //
 // The CTAs signal each other with mbarriers (ring slot written / ring slot
 // read).  Every wait is bounded: on expiry the CTA records kErrTimeout, raises
@@ -98,6 +104,15 @@ static_assert(L_GATES % 1024 == 0 && L_GATES + 2 * GATES_STRIDE <= L_GROUP && L_
 constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
               GR_GAM = 576, GR_DEC = 640;
 constexpr int GR_KB = 512;  // KDA beta (after the scratch)
+// KDA (one local group): B operands of the decayed [K; Q] products, one per
+// 16-token row block i, B_i = K[0, 16(i+1)) . e^{G_{m_i} - G} (m_i = 16 i + 7);
+// afterwards Kg = K . e^{G} (W's operand).  Then the per-block tables.
+constexpr uint32_t L_BREG = L_GROUP;  // (group 1's space)
+__host__ __device__ constexpr uint32_t bi_off(int i) { return 2048u * i * (i + 1); }  // B_i: 2 atoms of 16(i+1) rows
+constexpr uint32_t L_KTAB = L_BREG + 40960;  // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
+constexpr uint32_t TM_KD = 192;              // D_i at 192 + 0, 16, 48, 96 (160 columns)
+__host__ __device__ constexpr uint32_t di_col(int i) { return 8u * i * (i + 1); }  // 0, 16, 48, 96
+static_assert(L_KTAB + 3 * 2048 <= 2 * L_GROUP, "KDA layout");
 
 // ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
 constexpr uint32_t OFF_COMMON = 2 * L_GROUP;
@@ -302,13 +317,14 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         uint8_t *pzt = grp + L_PZT;
         float *AT = reinterpret_cast<float *>(grp + L_AT);
         uint64_t *bar_tma = bars + LB_TMA + g, *bar_l = bars + LB_L + g;
-        uint64_t *bar_slotfree = bars + LB_SLOTFREE + g;
-        uint8_t *ring_slot = ring_pair + (size_t)g * RING_STRIDE;
-        const uint32_t peer_ready = map_peer(smem_u32(bars + SB_READY + g), peer);
+        // ring slot = chunk parity: GDN's two groups own one slot each, KDA's one
+        // group alternates between them
+        const uint32_t peer_ready0 = map_peer(smem_u32(bars + SB_READY), peer);
         const uint32_t tm_kq = tmem + g * TM_GROUP + TM_KQ, tm_ab = tmem + g * TM_GROUP + TM_AB;
+        const int mstep = CH ? 1 : 2;  // chunks of this group: g, g + mstep, ...
+        const bool active = !CH || g == 0;
         const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
         const uint64_t d_raw = desc_sw128(gbase + L_RAW, 16, 1024);          // [K;Q], K (K-major)
-        const uint64_t d_kx = desc_sw128(gbase + L_KX, 16, 1024);            // Ki (K-major)
         const uint64_t d_kmn = desc_sw128(gbase + L_RAW, L_RAW_AC, 1024);    // K (MN-major)
         const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);    // [P; 0]
         const uint64_t d_x1b = desc_sw128(gbase + L_PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 (| X3)
@@ -317,11 +333,12 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         const bool issuer = gtid == 0;       // MMAs
         const bool storer = gtid == 7 * 32;  // tile reloads, ring stores and the hand-off
         bool pend = false;                   // storer: a chunk's ring stores are in flight
+        int pend_slot = 0;
         // storer: once the pending chunk's ring stores are complete, hand it over
         auto hand_over = [&]() {
             bulk_wait_all();
             fence_proxy_async_global();
-            mbar_arrive_peer(peer_ready);
+            mbar_arrive_peer(peer_ready0 + 8 * pend_slot);
             pend = false;
         };
 
@@ -339,8 +356,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             tma_load_3d(raw + L_RAW_AC + 8192, &tm_q, 64, h, (int)t0, bar_tma);
             ++issued[g];
         };
+        // gate rows of a chunk: two buffers, by the chunk's index within the group
         auto gate_rows = [&](int m) {
-            return reinterpret_cast<float *>(grp + L_GATES + ((m >> 1) & 1) * GATES_STRIDE);
+            return reinterpret_cast<float *>(grp + L_GATES + (((CH ? m : m >> 1)) & 1) * GATES_STRIDE);
         };
         // GDN gates, prefetched one group chunk ahead in the registers of warp lw 4
         float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
@@ -395,7 +413,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             *reinterpret_cast<float4 *>(gr + GR_DEC + 4 * lane) = make_float4(dC, dC, dC, dC);
         };
 
-        if (storer && g < nchunks) issue_tma(g);
+        if (active && storer && g < nchunks) issue_tma(g);
         if (!CH && lw == 4 && g < nchunks) {
             load_gates(g);
             compute_gates(g);
@@ -403,11 +421,13 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         // group 1 starts half a chunk after group 0, so that the two groups'
         // CUDA-core phases tend to overlap the other's MMA and load waits
         bool ok0 = true;
-        if (g == 1 && issuer && nchunks >= 2) ok0 = wt.wait(bars + LB_OFFSET, 0);
+        if (!CH && g == 1 && issuer && nchunks >= 2) ok0 = wt.wait(bars + LB_OFFSET, 0);
         named_bar_or(BAR_G, 256, !ok0);
 
-        for (int m = g; m < nchunks; m += 2) {
-            const int it = m >> 1;
+        for (int m = g; active && m < nchunks; m += mstep) {
+            const int gi = CH ? m : m >> 1;  // index of the chunk within the group
+            const int rs = m & 1;            // its ring slot
+            uint8_t *ring_slot = ring_pair + (size_t)rs * RING_STRIDE;
             float *gr = gate_rows(m);
             const long long t0 = t_begin + (long long)m * C;
             const int L = chunk_len(m);
@@ -415,19 +435,19 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             // ---- this chunk's tiles (rows past the sequence end read as zero); the
             //      group's next chunk is fetched into L2 meanwhile.  The previous
             //      chunk's ring tiles must have been read out of shared memory.
-            if (issuer && m + 2 < nchunks) {
-                const int t2 = (int)(t0 + 2 * C);
+            if (issuer && m + mstep < nchunks) {
+                const int t2 = (int)(t0 + mstep * C);
                 tma_prefetch_l2_3d(&tm_k, 0, h, t2);
                 tma_prefetch_l2_3d(&tm_k, 64, h, t2);
                 tma_prefetch_l2_3d(&tm_q, 0, h, t2);
                 tma_prefetch_l2_3d(&tm_q, 64, h, t2);
             }
-            if (CH && m + 2 < nchunks) {  // the next chunk's per-channel gates into L2
+            if (CH && m + 1 < nchunks) {  // the next chunk's per-channel gates into L2
                 const int pr = gtid >> 2, pc = gtid & 3;  // 64 rows x 4 lines of 128 B
-                if (t0 + 2 * C + pr < t_end)
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + 2 * C + pr) * H + h) * DK + 32 * pc));
+                if (t0 + C + pr < t_end)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + C + pr) * H + h) * DK + 32 * pc));
             }
-            if (issuer) ok = wt.wait(bar_tma, (uint32_t)(it & 1));
+            if (issuer) ok = wt.wait(bar_tma, (uint32_t)(gi & 1));
             if (L < C) {
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
@@ -441,10 +461,14 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             }
             if constexpr (CH) {
                 // ---- KDA gates: G_rc by a prefix sum over the rows (thread: two
-                //      channels, 16 rows); K, Q scaled in place by e^{G}, Ki = K e^{-G}
+                //      channels, the 16 rows of block rq) and the block references
+                //      G at m_i = 16 i + 7; then, with every exponent within 8 tokens'
+                //      decay of zero: KD = K e^{G - G_{m(r)}} and QD likewise in place,
+                //      Kt = K e^{G_C - G} (ring tile), B_i = K[0,16(i+1)) e^{G_{m_i} - G}
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
-                float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f;
+                float *ktab = reinterpret_cast<float *>(sm + L_KTAB);
+                float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f, p70 = 0.f, p71 = 0.f;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int r = 16 * rq + i;
@@ -455,54 +479,90 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     }
                     gl0[i] = acc0;
                     gl1[i] = acc1;
+                    if (i == 7) { p70 = acc0; p71 = acc1; }
                 }
-                *reinterpret_cast<float2 *>(gr + 128 * rq + c0) = make_float2(acc0, acc1);
+                *reinterpret_cast<float2 *>(ktab + 128 * rq + c0) = make_float2(acc0, acc1);
+                *reinterpret_cast<float2 *>(ktab + 512 + 128 * rq + c0) = make_float2(p70, p71);
                 if (gtid < 64) gr[GR_KB + gtid] = gtid < L ? a.beta[(t0 + gtid) * H + h] : 0.f;
-                if (storer && pend) bulk_wait_read();  // Ki below replaces the last Kt
+                if (storer && pend) bulk_wait_read();  // the tiles below replace the last ones
                 named_bar_sync(BAR_G, 256);
-                float off0 = 0.f, off1 = 0.f, tot0 = 0.f, tot1 = 0.f;
+                float gm0[4], gm1[4], off0 = 0.f, off1 = 0.f, run0 = 0.f, run1 = 0.f;
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
-                    const float2 v = *reinterpret_cast<const float2 *>(gr + 128 * q2 + c0);
-                    if (q2 < rq) { off0 += v.x; off1 += v.y; }
-                    tot0 += v.x;
-                    tot1 += v.y;
+                    const float2 tt = *reinterpret_cast<const float2 *>(ktab + 128 * q2 + c0);
+                    const float2 pp = *reinterpret_cast<const float2 *>(ktab + 512 + 128 * q2 + c0);
+                    gm0[q2] = run0 + pp.x;
+                    gm1[q2] = run1 + pp.y;
+                    if (q2 == rq) { off0 = run0; off1 = run1; }
+                    run0 += tt.x;
+                    run1 += tt.y;
                 }
                 if (rq == 0) {
-                    *reinterpret_cast<float2 *>(gr + GR_DEC + c0) = make_float2(__expf(tot0), __expf(tot1));
-                    if (-tot0 > kMaxNegLogDecay || -tot1 > kMaxNegLogDecay) atomicOr(redo + item, 1u);
+                    *reinterpret_cast<float2 *>(gr + GR_DEC + c0) = make_float2(__expf(run0), __expf(run1));
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2)
+                        *reinterpret_cast<float2 *>(ktab + 1024 + 128 * q2 + c0) =
+                            make_float2(__expf(gm0[q2]), __expf(gm1[q2]));
                 }
                 const int ac = c0 >> 6, cc = c0 & 63;
                 const uint32_t cof = (uint32_t)((cc & 7) * 2);
+                float big = 0.f;  // largest exponent met (range check)
+                auto bf2 = [](float x, float y) {
+                    __nv_bfloat162 t = __floats2bfloat162_rn(x, y);
+                    return *reinterpret_cast<uint32_t *>(&t);
+                };
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int r = 16 * rq + i;
                     const float G0 = off0 + gl0[i], G1 = off1 + gl1[i];
-                    const float e0 = __expf(G0), e1 = __expf(G1);
-                    const float n0 = __expf(fminf(-G0, kMaxNegLogDecay)), n1 = __expf(fminf(-G1, kMaxNegLogDecay));
+                    const float x0 = G0 - gm0[rq], x1 = G1 - gm1[rq];
+                    big = fmaxf(big, fmaxf(fabsf(x0), fabsf(x1)));
+                    const float f0 = __expf(fminf(x0, kMaxNegLogDecay)), f1 = __expf(fminf(x1, kMaxNegLogDecay));
                     const uint32_t o = sw128(r, cc >> 3) + cof;
                     uint32_t *pk = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + o);
                     uint32_t *pq = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + 8192 + o);
                     const uint32_t kw = *pk, qw = *pq;
                     const float kx = __uint_as_float(kw << 16), ky = __uint_as_float(kw & 0xffff0000u);
                     const float qx = __uint_as_float(qw << 16), qy = __uint_as_float(qw & 0xffff0000u);
-                    __nv_bfloat162 t;
-                    t = __floats2bfloat162_rn(kx * e0, ky * e1); *pk = *reinterpret_cast<uint32_t *>(&t);
-                    t = __floats2bfloat162_rn(qx * e0, qy * e1); *pq = *reinterpret_cast<uint32_t *>(&t);
-                    t = __floats2bfloat162_rn(kx * n0, ky * n1);
-                    *reinterpret_cast<uint32_t *>(kxt + ac * 8192 + o) = *reinterpret_cast<uint32_t *>(&t);
+                    *pk = bf2(kx * f0, ky * f1);
+                    *pq = bf2(qx * f0, qy * f1);
+                    *reinterpret_cast<uint32_t *>(kxt + ac * 8192 + o) =
+                        bf2(kx * __expf(run0 - G0), ky * __expf(run1 - G1));
+#pragma unroll
+                    for (int bi = 0; bi < 4; ++bi) {
+                        if (bi < rq) continue;  // rq is uniform per warp
+                        const float e0 = __expf(fminf(gm0[bi] - G0, kMaxNegLogDecay));
+                        const float e1 = __expf(fminf(gm1[bi] - G1, kMaxNegLogDecay));
+                        *reinterpret_cast<uint32_t *>(sm + L_BREG + bi_off(bi) + ac * (2048u * (bi + 1)) + o) =
+                            bf2(kx * e0, ky * e1);
+                    }
                 }
+                if (big > kMaxNegLogDecay) atomicOr(redo + item, 1u);
             }
             fence_proxy_async_smem();
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-            // ---- D_kq = [K; Q] K^T (GDN) or [Kg; Qg] Ki^T (KDA) -----------------------
+            // ---- D_kq = [K; Q] K^T (GDN) or D_i = [KD; QD] B_i^T, i = 0..3 (KDA) -------
             if (issuer) {
                 tc_fence_after();
+                if constexpr (CH) {
 #pragma unroll
-                for (int k = 0; k < DK / 16; ++k) {
-                    const uint32_t off = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
-                    const uint64_t db = CH ? d_kx + (((k >> 2) * 8192 + (k & 3) * 32) >> 4) : d_raw + off;
-                    mma_bf16(tm_kq, d_raw + off, db, ID_KK, k > 0);
+                    for (int bi = 0; bi < 4; ++bi) {
+                        const uint32_t asz = 2048u * (bi + 1);
+                        const uint64_t db = desc_sw128(sbase + L_BREG + bi_off(bi), 16, 1024);
+                        const uint32_t idn = idesc_bf16(128, 16 * (bi + 1), false, false);
+#pragma unroll
+                        for (int k = 0; k < DK / 16; ++k) {
+                            const uint32_t offa = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
+                            const uint32_t offb = ((k >> 2) * asz + (k & 3) * 32) >> 4;
+                            mma_bf16(tmem + TM_KD + di_col(bi), d_raw + offa, db + offb, idn, k > 0);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int k = 0; k < DK / 16; ++k) {
+                        const uint32_t off = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
+                        mma_bf16(tm_kq, d_raw + off, d_raw + off, ID_KK, k > 0);
+                    }
                 }
                 mma_commit(bar_l);
                 ok = wt.wait(bar_l, bl_wait & 1);
@@ -516,7 +576,23 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             const float *gb = gr + (CH ? GR_KB : GR_B);
             if ((lq & 1) >= lhalf) {
                 float x[32];
-                tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
+                if constexpr (CH) {
+                    // rows of block b0 (lanes 0-15) / b1 (lanes 16-31) from D_b0 / D_b1,
+                    // whose first 16 (b + 1) columns are the decayed products
+                    const int b0 = 2 * (lq & 1), b1 = b0 + 1;
+                    float x1[32];
+                    tmem_load<32>(tmem + TM_KD + di_col(b0) + lane_off + 32 * lhalf, x);
+                    tmem_load<32>(tmem + TM_KD + di_col(b1) + lane_off + 32 * lhalf, x1);
+                    const bool hi = lane >= 16;
+                    const int nb = 16 * ((hi ? b1 : b0) + 1);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int s2 = 32 * lhalf + j;
+                        x[j] = s2 < nb ? (hi ? x1[j] : x[j]) : 0.f;
+                    }
+                } else {
+                    tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
+                }
                 if (lq < 2) {
                     const int r = 32 * lq + lane;
                     if constexpr (!CH) decay_row(x, r, lq, lhalf, gr, false);
@@ -555,24 +631,26 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (g == 0 && m == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
             // ---- T = (I + A)^{-1} in place of A: lw 0-3 (diagonal blocks, 32-level);
             //      meanwhile lw 4 prepares the group's next GDN gates, and for KDA
-            //      lw 4-7 turn Ki into Kt = Ki . e^{G_C} (Ki has been consumed) ------
+            //      lw 4-7 form W's operand Kg from KD ----------------------------------
             if (lw >= 4) {
                 if (storer && pend) hand_over();  // the previous chunk of this group
                 if constexpr (!CH) {
                     if (lw == 4 && m + 2 < nchunks) compute_gates(m + 2);
                 } else {
+                    // Kg = K e^{G} = KD e^{G_{m(r)}} into the B region (its products are done)
+                    const float *fm = reinterpret_cast<const float *>(sm + L_KTAB) + 1024;
 #pragma unroll 2
                     for (int q2 = 0; q2 < 8; ++q2) {
                         const int idx = (gtid - 128) + 128 * q2;
                         const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
-                        uint4 *p = reinterpret_cast<uint4 *>(kxt + ac * 8192 + sw128(rr, j));
                         float kv[8];
-                        unpack8(*p, kv);
-                        const float4 d0 = *reinterpret_cast<const float4 *>(gr + GR_DEC + 64 * ac + 8 * j);
-                        const float4 d1 = *reinterpret_cast<const float4 *>(gr + GR_DEC + 64 * ac + 8 * j + 4);
+                        unpack8(*reinterpret_cast<const uint4 *>(raw + ac * L_RAW_AC + sw128(rr, j)), kv);
+                        const float *f = fm + 128 * (rr >> 4) + 64 * ac + 8 * j;
+                        const float4 d0 = *reinterpret_cast<const float4 *>(f);
+                        const float4 d1 = *reinterpret_cast<const float4 *>(f + 4);
                         kv[0] *= d0.x; kv[1] *= d0.y; kv[2] *= d0.z; kv[3] *= d0.w;
                         kv[4] *= d1.x; kv[5] *= d1.y; kv[6] *= d1.z; kv[7] *= d1.w;
-                        *p = pack8(kv);
+                        *reinterpret_cast<uint4 *>(sm + L_BREG + ac * 8192 + sw128(rr, j)) = pack8(kv);
                     }
                 }
             } else {
@@ -744,9 +822,10 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             //      rows 0-63 = W, rows 64-127 = P W ---------------------------------------
             if (issuer) {
                 tc_fence_after();
+                const uint64_t dkb = CH ? desc_sw128(sbase + L_BREG, 8192, 1024) : d_kmn;  // Kg : K
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
-                    mma_bf16(tm_ab, d_x1x2 + 2 * k, d_kmn + 128 * k, ID_N128, k > 0);
+                    mma_bf16(tm_ab, d_x1x2 + 2 * k, dkb + 128 * k, ID_N128, k > 0);
                 mma_commit(bar_l);
                 ok = wt.wait(bar_l, bl_wait & 1);
             }
@@ -780,6 +859,14 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                             const uint32_t o = sw128(r, 4 * hh + j);
                             float qv[8];
                             unpack8(*reinterpret_cast<const uint4 *>(qt + o), qv);
+                            if constexpr (CH) {  // QD e^{G_{m(r)}}
+                                const float *f = reinterpret_cast<const float *>(sm + L_KTAB) + 1024 +
+                                                 128 * (r >> 4) + 64 * lhalf + 8 * (4 * hh + j);
+                                const float4 d0 = *reinterpret_cast<const float4 *>(f);
+                                const float4 d1 = *reinterpret_cast<const float4 *>(f + 4);
+                                qv[0] *= d0.x; qv[1] *= d0.y; qv[2] *= d0.z; qv[3] *= d0.w;
+                                qv[4] *= d1.x; qv[5] *= d1.y; qv[6] *= d1.z; qv[7] *= d1.w;
+                            }
 #pragma unroll
                             for (int e = 0; e < 8; ++e) qv[e] = gam * qv[e] - x[8 * j + e];
                             *reinterpret_cast<uint4 *>(qst + o) = pack8(qv);
@@ -806,11 +893,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (storer) {
                 // the raw tiles take the group's next chunk (issued before the ring
                 // stores: the TMA unit serves its requests in order)
-                if (m + 2 < nchunks) issue_tma(m + 2);
+                if (m + mstep < nchunks) issue_tma(m + mstep);
                 // once the state CTA has read the slot's previous chunk, the ring
                 // tiles and e^{G_C} go out by bulk copy; the hand-off follows
                 // during the next chunk (or after the loop)
-                if (m < 2 || wt.wait_peer(bar_slotfree, (uint32_t)((it - 1) & 1))) {
+                if (m < 2 || wt.wait_peer(bars + LB_SLOTFREE + rs, (uint32_t)(((m >> 1) - 1) & 1))) {
                     const uint8_t *at8 = grp + L_AT;
                     bulk_store(ring_slot + SG_KT, kxt, 8192);
                     bulk_store(ring_slot + SG_AC + SG_KT, kxt + 8192, 8192);
@@ -823,10 +910,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     bulk_store(ring_slot + SG_TILES, gr + GR_DEC, SG_DECB);
                     bulk_commit();
                     pend = true;
+                    pend_slot = rs;
                 }
             }
         }
-        if (storer && pend && !*abort_flag) hand_over();
+        if (active && storer && pend && !*abort_flag) hand_over();
         // drain: every MMA this issuer launched, every tile load not yet landed
         if (storer) bulk_wait_all();
         if (*abort_flag && issuer) {

@@ -10,16 +10,14 @@
 // propagation, intra-chunk causal product).  Per chunk, in fp32:
 //   g_r   = sum_{s<=r} log alpha_s                        (per key channel for KDA)
 //   A_rs  = beta_r sum_c k_rc k_sc e^{g_rc - g_sc}, s < r  (strictly lower)
-// For KDA the per-channel decay inside the contraction is split at the middle
-// token m_j of the 16-token block j holding column s:
-//   e^{g_rc - g_sc} = e^{g_rc - g_{m_j}c} e^{g_{m_j}c - g_sc},
-// with the column factor k_sc e^{g_{m_j}c - g_sc} formed once per chunk.  Both
-// factors stay below e^{(decay over 8 tokens)} wherever the term is kept, so
-// nothing overflows where the plain factorisation e^{g_r} e^{-g_s} would
-// (g reaches -200 over a chunk at the decays of the KDA workload).  The
-// exponents are clamped at 80, so the result is exact while the decay over any
-// 8 consecutive tokens stays above e^{-80} on every channel (log alpha > -10 per
-// token on average); beyond that the terms are bounded, never inf or NaN.
+// For KDA the per-channel decay inside the contraction is taken in two ways
+// (g reaches -200 over a chunk at the decays of the KDA workload, so the plain
+// factorisation e^{g_r} e^{-g_s} overflows):
+//   - s in an earlier 16-token block j than r: split at the block's last token
+//     e_j, e^{g_rc - g_sc} = e^{g_rc - g_{e_j}c} e^{g_{e_j}c - g_sc}, both factors
+//     <= 1, the column factor k_sc e^{g_{e_j}c - g_sc} formed once per chunk;
+//   - s in r's own block: e^{g_rc - g_sc} directly (<= 1 for s <= r).
+// Exact for any decay.
 //   T     = (I + A)^{-1}                                  (forward substitution)
 //   W     = T diag(beta) (K . e^{G}),  U = T diag(beta) V
 //   V'    = U - W S^T
@@ -54,32 +52,41 @@ struct SimtSmem {
     static constexpr size_t kBytes = sizeof(float) * kFloats;
 };
 
-// KDA: out_rs = [beta_r] sum_c x_rc e^{g_rc - g_{m_j}c} f_sc for s < r (A, with
-// beta) or s <= r (P), zero elsewhere; f (stride LDK) holds the column factors
-// k_sc e^{g_{m_j}c - g_sc}, j = s / 16, m_j = 16 j + 7.  Work unit: one row r and
+// KDA: out_rs = [beta_r] sum_c x_rc k_sc e^{g_rc - g_sc} for s < r (A, with
+// beta) or s <= r (P), zero elsewhere.  F (stride LDK) holds the column factors
+// k_sc e^{g_{e_j}c - g_sc}, j = s / 16, e_j = 16 j + 15.  Work unit: one row r and
 // 8 columns of one block at or left of the diagonal.
 template <int DK>
-__device__ __forceinline__ void decayed_products(const float *X, const float *F, const float *G,
-                                                 const float *beta, float *out, bool incl,
-                                                 int tid) {
+__device__ __forceinline__ void decayed_products(const float *X, const float *Kr, const float *F,
+                                                 const float *G, const float *beta, float *out,
+                                                 bool incl, int tid) {
     constexpr int C = kChunk, LDK = DK + 1, LC = C + 1;
     // rows of block i own 2 (i + 1) half-block units: 16 * 2 * (1 + 2 + 3 + 4) = 320
     for (int u = tid; u < 320; u += kThreads) {
         int i = 0, base = 0;
         while (u >= base + 32 * (i + 1)) { base += 32 * (i + 1); ++i; }
         const int v = u - base, r = 16 * i + v / (2 * (i + 1)), w = v % (2 * (i + 1));
-        const int j = w >> 1, s0 = 16 * j + 8 * (w & 1), m = 16 * j + 7;
+        const int j = w >> 1, s0 = 16 * j + 8 * (w & 1), e = 16 * j + 15;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int c = 0; c < DK; ++c) {
-            const float rf = X[r * LDK + c] * __expf(fminf(G[r * LDK + c] - G[m * LDK + c], 80.f));
+        if (j < i) {
+            for (int c = 0; c < DK; ++c) {
+                const float rf = X[r * LDK + c] * __expf(G[r * LDK + c] - G[e * LDK + c]);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] += rf * F[(s0 + e) * LDK + c];
+                for (int q = 0; q < 8; ++q) acc[q] += rf * F[(s0 + q) * LDK + c];
+            }
+        } else {
+            for (int c = 0; c < DK; ++c) {
+                const float xr = X[r * LDK + c], gr = G[r * LDK + c];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    acc[q] += xr * Kr[(s0 + q) * LDK + c] * __expf(fminf(gr - G[(s0 + q) * LDK + c], 0.f));
+            }
         }
         const float b = beta ? beta[r] : 1.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int s2 = s0 + e;
-            out[r * LC + s2] = (incl ? s2 <= r : s2 < r) ? b * acc[e] : 0.f;
+        for (int q = 0; q < 8; ++q) {
+            const int s2 = s0 + q;
+            out[r * LC + s2] = (incl ? s2 <= r : s2 < r) ? b * acc[q] : 0.f;
         }
     }
     // columns right of the row's own block
@@ -158,14 +165,13 @@ chunk_simt_kernel(PrefillArgs a) {
         __syncthreads();
         // ---- step 2: A (strictly lower), T initialised to I ---------------
         if (CH) {
-            // column factors k_sc e^{g_{m(s)}c - g_sc}, m(s) the middle of s's block (in W)
+            // column factors k_sc e^{g_{e(s)}c - g_sc}, e(s) the last token of s's block (in W)
             for (int idx = tid; idx < C * DK; idx += kThreads) {
                 const int r = idx / DK, c = idx % DK;
-                const int m = (r & ~15) + 7;
-                W[r * LDK + c] = K[r * LDK + c] * __expf(fminf(G[m * LDK + c] - G[r * LDK + c], 80.f));
+                W[r * LDK + c] = K[r * LDK + c] * __expf(G[(r | 15) * LDK + c] - G[r * LDK + c]);
             }
             __syncthreads();
-            decayed_products<DK>(K, W, G, bt, A, false, tid);
+            decayed_products<DK>(K, K, W, G, bt, A, false, tid);
             for (int idx = tid; idx < C * C; idx += kThreads) {
                 const int r = idx / C, s2 = idx % C;
                 Tm[r * LC + s2] = (r == s2) ? 1.f : 0.f;
@@ -197,7 +203,7 @@ chunk_simt_kernel(PrefillArgs a) {
         // ---- KDA: P = causal decayed Q K^T into A, while W still holds the column
         //      factors (A is consumed by the inversion above) -------------------
         if (CH) {
-            decayed_products<DK>(Q, W, G, nullptr, A, true, tid);
+            decayed_products<DK>(Q, K, W, G, nullptr, A, true, tid);
             __syncthreads();
         }
         // ---- step 4: W = T diag(b)(K . e^G), U = T diag(b) V --------------

@@ -61,16 +61,17 @@ typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
 
 /* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: for bf16
- * with d_k = d_v = 128 and scalar decay the single-CTA tensor-core kernel, the
- * fp32 CUDA-core kernel otherwise.  GDN_FLAG_PAIR selects, for bf16 with
- * d_k = d_v = 128 and either decay, the two-CTA tensor-core kernel (one
- * thread-block cluster per sequence and head: one SM computes the chunk-local
- * matrices, the other runs the sequential state pass; it needs a larger
- * workspace, see below).  For KDA that kernel covers chunks whose decay on
- * every key channel stays above e^-80; the (sequence, head) pairs with a chunk
- * beyond it are recomputed by the CUDA-core kernel within the same call.
- * GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use the
- * flags to compare the device paths. */
+ * with d_k = d_v = 128 the single-CTA tensor-core kernel (scalar decay) or the
+ * two-CTA tensor-core kernel (channel decay), the fp32 CUDA-core kernel
+ * otherwise.  GDN_FLAG_PAIR selects the two-CTA kernel for scalar decay too.
+ * The two-CTA kernel runs one thread-block cluster per sequence and head: one
+ * SM computes the chunk-local matrices, the other runs the sequential state
+ * pass; it needs a larger workspace (see below).  For channel decay it covers
+ * chunks whose decay over any 8 consecutive tokens stays above e^-80 on every
+ * key channel; the (sequence, head) pairs with a chunk beyond that are
+ * recomputed by the CUDA-core kernel (exact for any decay) within the same
+ * call.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use
+ * the flags to compare the device paths. */
 enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2 };
 
 typedef struct {
@@ -150,9 +151,9 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
  * Instead of a caller workspace it uses one fixed device array of
  * GDN_NOALLOC_SCRATCH_BYTES compiled into the library.  Where the selected
  * kernel's workspace (gdn_chunk_fwd_workspace_size) does not fit in it -- the
- * two-CTA tensor-core kernel's ring never does -- the call runs the default
- * kernel instead (GDN_FLAG_PAIR cleared: the single-CTA tensor-core kernel for
- * GDN, the CUDA-core kernel for KDA), whose workspace is the header alone.
+ * two-CTA tensor-core kernel's ring never does -- the call runs the single-CTA
+ * tensor-core kernel (scalar decay) or the CUDA-core kernel (channel decay)
+ * instead, whose workspace is the header alone.
  * Problems whose workspace exceeds the array even then return
  * GDN_ERR_UNSUPPORTED before anything is launched.  All other arguments,
  * layouts and results are those of gdn_chunk_fwd.

@@ -140,33 +140,29 @@ def test_tensor_core_and_cuda_core_paths_agree(cuda_ok):
         assert rel_err(s1, s2.cpu().numpy()) < 1e-2
 
 
-def test_kda_pair_kernel_and_strong_decay_is_redone_exactly(cuda_ok):
-    """KDA on the two-CTA kernel.  A chunk whose decay on some channel falls
-    below e^-80 (log alpha = -3 per token on 8 channels of head 0, both
-    sequences; the KDA workload's decays do so everywhere) is out of that
-    kernel's range: its (sequence, head) is recomputed exactly on CUDA cores."""
-    # mild decays (log alpha ~ -0.13 per token): the two-CTA kernel's own path
-    x = prefill_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
-                       alpha_shift=-2.0, seed=31, init_std=0.05)
-    o, sf = _run(x, pair=True)
-    _full_compare(x, o, sf, torch.bfloat16)
-    x = prefill_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
-                       alpha_shift=3.0, seed=30, init_std=0.05)
-    d = to_dev(x)
-    assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"], pair=True)) == \
-        "tensor_core_pair"
-    o, sf = _run(x, pair=True)
-    _full_compare(x, o, sf, torch.bfloat16)
-    x["log_alpha"][:, :, 0, :8] = -3.0
-    o, sf = _run(x, pair=True)
+def test_kda_pair_kernel_and_out_of_range_decay_is_redone_exactly(cuda_ok):
+    """KDA's default path is the two-CTA kernel (16-token block references).
+    Decays inside its range: mild, and the KDA workload's (log alpha ~ -3).
+    Out of range (log alpha = -30 per token on 8 channels of head 0: e^-240 over
+    8 tokens): that (sequence, head) is recomputed by the CUDA-core kernel,
+    which is exact for any decay; head 1 stays on the fast path."""
+    for shift, seed in ((-2.0, 31), (3.0, 30)):
+        x = prefill_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                           alpha_shift=shift, seed=seed, init_std=0.05)
+        d = to_dev(x)
+        assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"])) == \
+            "tensor_core_pair"
+        o, sf = _run(x)
+        _full_compare(x, o, sf, torch.bfloat16)
+    x["log_alpha"][:, :, 0, :8] = -30.0
+    o, sf = _run(x)
     _full_compare(x, o, sf, torch.bfloat16)
     # final state aliasing the initial state: the re-run must see the original S0
     d = to_dev(x)
     ref_o, ref_s = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
                              d["initial_state"].clone(), cuda_cores=True)
     s = d["initial_state"].clone()
-    o2, _ = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], s, final_state=s,
-                      pair=True)
+    o2, _ = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], s, final_state=s)
     torch.cuda.synchronize()
     assert rel_err(o2, ref_o.float().cpu().numpy()) < 2e-2
     assert rel_err(s, ref_s.cpu().numpy()) < 1e-2
