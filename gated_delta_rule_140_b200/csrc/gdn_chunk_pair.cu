@@ -104,15 +104,19 @@ static_assert(L_GATES % 1024 == 0 && L_GATES + 2 * GATES_STRIDE <= L_GROUP && L_
 constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
               GR_GAM = 576, GR_DEC = 640;
 constexpr int GR_KB = 512;  // KDA beta (after the scratch)
-// KDA (one local group): B operands of the decayed [K; Q] products, one per
-// 16-token row block i, B_i = K[0, 16(i+1)) . e^{G_{m_i} - G} (m_i = 16 i + 7);
-// afterwards Kg = K . e^{G} (W's operand).  Then the per-block tables.
+// KDA (one local group; the other group's space holds these): the B operand of
+// the decayed [K; Q] products, rows di_col(i) .. of it being, for 16-token row
+// block i, B_i = K[0, 16(i+1)) . e^{G_{m_i} - G} (m_i = 16 i + 7), 160 rows per
+// atom column; afterwards Kg = K . e^{G} (W's operand).  Then the per-block
+// tables and a second Kt buffer.
 constexpr uint32_t L_BREG = L_GROUP;  // (group 1's space)
-__host__ __device__ constexpr uint32_t bi_off(int i) { return 2048u * i * (i + 1); }  // B_i: 2 atoms of 16(i+1) rows
-constexpr uint32_t L_KTAB = L_BREG + 40960;  // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
-constexpr uint32_t TM_KD = 192;              // D_i at 192 + 0, 16, 48, 96 (160 columns)
+constexpr uint32_t BREG_AC = 160 * 128;      // atom column stride of the stacked B
 __host__ __device__ constexpr uint32_t di_col(int i) { return 8u * i * (i + 1); }  // 0, 16, 48, 96
-static_assert(L_KTAB + 3 * 2048 <= 2 * L_GROUP, "KDA layout");
+constexpr uint32_t L_KTAB = L_BREG + 2 * BREG_AC;  // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
+constexpr uint32_t L_KX2 = L_KTAB + 6144;          // KDA's second Kt buffer
+constexpr uint32_t TM_KD = 192;                    // D = [D_0 | D_1 | D_2 | D_3], 160 columns
+constexpr uint32_t ID_KD = idesc_bf16(128, 160, false, false);
+static_assert(L_KX2 % 1024 == 0 && L_KX2 + 16384 <= 2 * L_GROUP, "KDA layout");
 
 // ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
 constexpr uint32_t OFF_COMMON = 2 * L_GROUP;
@@ -429,6 +433,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             const int rs = m & 1;            // its ring slot
             uint8_t *ring_slot = ring_pair + (size_t)rs * RING_STRIDE;
             float *gr = gate_rows(m);
+            uint8_t *kxc = (CH && (gi & 1)) ? sm + L_KX2 : kxt;  // this chunk's Kt
             const long long t0 = t_begin + (long long)m * C;
             const int L = chunk_len(m);
             bool ok = true;
@@ -469,14 +474,17 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
                 float *ktab = reinterpret_cast<float *>(sm + L_KTAB);
                 float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f, p70 = 0.f, p71 = 0.f;
+                const float *lp0 = a.log_alpha + ((t0 + 16 * rq) * H + h) * DK + c0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {  // all loads first, then the sums
+                    const bool in = 16 * rq + i < L;
+                    gl0[i] = in ? lp0[(size_t)i * H * DK] : 0.f;
+                    gl1[i] = in ? lp0[(size_t)i * H * DK + 1] : 0.f;
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int r = 16 * rq + i;
-                    if (r < L) {
-                        const float *lp = a.log_alpha + ((t0 + r) * H + h) * DK + c0;
-                        acc0 += lp[0];
-                        acc1 += lp[1];
-                    }
+                    acc0 += gl0[i];
+                    acc1 += gl1[i];
                     gl0[i] = acc0;
                     gl1[i] = acc1;
                     if (i == 7) { p70 = acc0; p71 = acc1; }
@@ -484,7 +492,6 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 *reinterpret_cast<float2 *>(ktab + 128 * rq + c0) = make_float2(acc0, acc1);
                 *reinterpret_cast<float2 *>(ktab + 512 + 128 * rq + c0) = make_float2(p70, p71);
                 if (gtid < 64) gr[GR_KB + gtid] = gtid < L ? a.beta[(t0 + gtid) * H + h] : 0.f;
-                if (storer && pend) bulk_wait_read();  // the tiles below replace the last ones
                 named_bar_sync(BAR_G, 256);
                 float gm0[4], gm1[4], off0 = 0.f, off1 = 0.f, run0 = 0.f, run1 = 0.f;
 #pragma unroll
@@ -511,13 +518,27 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     __nv_bfloat162 t = __floats2bfloat162_rn(x, y);
                     return *reinterpret_cast<uint32_t *>(&t);
                 };
+                // this block's reference, and the factors from it to the later blocks'
+                // references and to the chunk end (all <= 1)
+                float gr0 = gm0[0], gr1 = gm1[0];
+#pragma unroll
+                for (int q2 = 1; q2 < 4; ++q2)
+                    if (q2 == rq) { gr0 = gm0[q2]; gr1 = gm1[q2]; }
+                float tb0[4], tb1[4];
+#pragma unroll
+                for (int bi = 0; bi < 4; ++bi) {
+                    tb0[bi] = bi > rq ? __expf(gm0[bi] - gr0) : 1.f;
+                    tb1[bi] = bi > rq ? __expf(gm1[bi] - gr1) : 1.f;
+                }
+                const float tc0 = __expf(run0 - gr0), tc1 = __expf(run1 - gr1);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int r = 16 * rq + i;
-                    const float G0 = off0 + gl0[i], G1 = off1 + gl1[i];
-                    const float x0 = G0 - gm0[rq], x1 = G1 - gm1[rq];
+                    const float x0 = off0 + gl0[i] - gr0, x1 = off1 + gl1[i] - gr1;
                     big = fmaxf(big, fmaxf(fabsf(x0), fabsf(x1)));
+                    // KD, QD = . e^{G - G_m};  KC = K e^{G_m - G} (B_rq's row)
                     const float f0 = __expf(fminf(x0, kMaxNegLogDecay)), f1 = __expf(fminf(x1, kMaxNegLogDecay));
+                    const float h0 = __expf(fminf(-x0, kMaxNegLogDecay)), h1 = __expf(fminf(-x1, kMaxNegLogDecay));
                     const uint32_t o = sw128(r, cc >> 3) + cof;
                     uint32_t *pk = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + o);
                     uint32_t *pq = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + 8192 + o);
@@ -526,36 +547,31 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const float qx = __uint_as_float(qw << 16), qy = __uint_as_float(qw & 0xffff0000u);
                     *pk = bf2(kx * f0, ky * f1);
                     *pq = bf2(qx * f0, qy * f1);
-                    *reinterpret_cast<uint32_t *>(kxt + ac * 8192 + o) =
-                        bf2(kx * __expf(run0 - G0), ky * __expf(run1 - G1));
+                    const float kc0 = kx * h0, kc1 = ky * h1;
+                    // Kt = K e^{G_C - G} = KC e^{G_C - G_m}
+                    *reinterpret_cast<uint32_t *>(kxc + ac * 8192 + o) = bf2(kc0 * tc0, kc1 * tc1);
+                    // B_i = K e^{G_{m_i} - G} = KC e^{G_{m_i} - G_m}, i >= rq
 #pragma unroll
                     for (int bi = 0; bi < 4; ++bi) {
                         if (bi < rq) continue;  // rq is uniform per warp
-                        const float e0 = __expf(fminf(gm0[bi] - G0, kMaxNegLogDecay));
-                        const float e1 = __expf(fminf(gm1[bi] - G1, kMaxNegLogDecay));
-                        *reinterpret_cast<uint32_t *>(sm + L_BREG + bi_off(bi) + ac * (2048u * (bi + 1)) + o) =
-                            bf2(kx * e0, ky * e1);
+                        *reinterpret_cast<uint32_t *>(sm + L_BREG + ac * BREG_AC + sw128(di_col(bi) + r, cc >> 3) + cof) =
+                            bf2(kc0 * tb0[bi], kc1 * tb1[bi]);
                     }
                 }
                 if (big > kMaxNegLogDecay) atomicOr(redo + item, 1u);
             }
             fence_proxy_async_smem();
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-            // ---- D_kq = [K; Q] K^T (GDN) or D_i = [KD; QD] B_i^T, i = 0..3 (KDA) -------
+            // ---- D_kq = [K; Q] K^T (GDN) or [KD; QD] [B_0; B_1; B_2; B_3]^T (KDA) -------
             if (issuer) {
                 tc_fence_after();
                 if constexpr (CH) {
+                    const uint64_t db = desc_sw128(sbase + L_BREG, 16, 1024);
 #pragma unroll
-                    for (int bi = 0; bi < 4; ++bi) {
-                        const uint32_t asz = 2048u * (bi + 1);
-                        const uint64_t db = desc_sw128(sbase + L_BREG + bi_off(bi), 16, 1024);
-                        const uint32_t idn = idesc_bf16(128, 16 * (bi + 1), false, false);
-#pragma unroll
-                        for (int k = 0; k < DK / 16; ++k) {
-                            const uint32_t offa = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
-                            const uint32_t offb = ((k >> 2) * asz + (k & 3) * 32) >> 4;
-                            mma_bf16(tmem + TM_KD + di_col(bi), d_raw + offa, db + offb, idn, k > 0);
-                        }
+                    for (int k = 0; k < DK / 16; ++k) {
+                        const uint32_t offa = ((k >> 2) * L_RAW_AC + (k & 3) * 32) >> 4;
+                        const uint32_t offb = ((k >> 2) * BREG_AC + (k & 3) * 32) >> 4;
+                        mma_bf16(tmem + TM_KD, d_raw + offa, db + offb, ID_KD, k > 0);
                     }
                 } else {
 #pragma unroll
@@ -568,7 +584,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 ok = wt.wait(bar_l, bl_wait & 1);
             }
             ++bl_wait;
-            if (!CH && storer && pend) bulk_wait_read();  // the staged tiles are rewritten below
+            if (storer && pend) bulk_wait_read();  // the staged tiles are rewritten below
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
             tc_fence_after();
             // ---- A rows (lanes 0-63) -> fp32;  P rows (lanes 64-127) -> bf16.  GDN
@@ -899,8 +915,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 // during the next chunk (or after the loop)
                 if (m < 2 || wt.wait_peer(bars + LB_SLOTFREE + rs, (uint32_t)(((m >> 1) - 1) & 1))) {
                     const uint8_t *at8 = grp + L_AT;
-                    bulk_store(ring_slot + SG_KT, kxt, 8192);
-                    bulk_store(ring_slot + SG_AC + SG_KT, kxt + 8192, 8192);
+                    bulk_store(ring_slot + SG_KT, kxc, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_KT, kxc + 8192, 8192);
                     bulk_store(ring_slot + SG_MW, at8, 8192);
                     bulk_store(ring_slot + SG_AC + SG_MW, at8 + 8192, 8192);
                     bulk_store(ring_slot + SG_QH, pzt + (CH ? PZ_X3 : PZ_X1), 8192);
