@@ -168,11 +168,15 @@ def test_kda_pair_kernel_and_out_of_range_decay_is_redone_exactly(cuda_ok):
     assert rel_err(s, ref_s.cpu().numpy()) < 1e-2
 
 
+@pytest.mark.parametrize("decay", ["scalar", "channel"])
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 129, 640])
-def test_pair_kernel_chunk_counts(cuda_ok, T):
-    """The two-CTA kernel with 1..10 chunks per sequence: both local groups,
-    odd and even chunk counts, a one-token sequence."""
-    x = prefill_inputs(2, T, 2, 128, 128, dtype=torch.bfloat16, seed=28 + T, init_std=0.05)
+def test_pair_kernel_chunk_counts(cuda_ok, T, decay):
+    """The two-CTA kernel with 1..10 chunks per sequence: both local groups (GDN)
+    or the one group on both ring slots (KDA), odd and even chunk counts, a
+    one-token sequence."""
+    x = prefill_inputs(2, T, 2, 128, 128, dtype=torch.bfloat16, decay=decay,
+                       alpha_shift=2.0 if decay == "scalar" else 3.0, seed=28 + T,
+                       init_std=0.05)
     o, sf = _run(x, pair=True)
     _full_compare(x, o, sf, torch.bfloat16)
 

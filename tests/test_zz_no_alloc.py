@@ -6,8 +6,8 @@ fixed array inside the library as scratch.
 
 This file is named to be collected last, so that a run stopping at the first
 failure has already run every other test; it passes alone in a fresh process
-as well.  The entry point is called through the C ABI (ctypes), twice in a row
-on different problems, and each result is checked against gdn_chunk_fwd's
+as well.  The entry point is called through the C ABI (ctypes), three times in
+a row on different problems, and each result is checked against gdn_chunk_fwd's
 within the parity tolerances."""
 import ctypes
 
@@ -43,7 +43,11 @@ def _problems():
     g = torch.Generator().manual_seed(42)
     b = prefill_inputs(1, 0, 4, 64, 64, dtype=torch.float32, decay="channel", alpha_shift=3.0,
                        init_std=0.02, lengths=[70, 0, 129, 5], gen=g)
-    return [(a, torch.bfloat16), (b, torch.float32)]
+    # KDA bf16 d = 128: the default two-CTA kernel's ring does not fit, so the
+    # entry point runs the CUDA-core kernel; compared with the default path
+    c = prefill_inputs(2, 150, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                       alpha_shift=3.0, seed=43, init_std=0.05)
+    return [(a, torch.bfloat16), (b, torch.float32), (c, torch.bfloat16)]
 
 
 def test_noalloc_matches_chunk_fwd_on_two_calls_in_a_row(cuda_ok):
