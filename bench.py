@@ -116,13 +116,15 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None}
 
 
-def traffic_for(kernel: str, src: str):
-    """DRAM bytes per launch from a committed ncu capture, if the kernel source
-    is unchanged since the counters were taken (else None)."""
+def traffic_for(kernel: str, src: str, workload: str = ""):
+    """DRAM bytes per launch from a committed ncu capture of this kernel on this
+    workload (entry "kernel:workload", else "kernel"), if the kernel source is
+    unchanged since the counters were taken (else None)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
-    rec = json.load(open(p)).get(kernel)
+    recs = json.load(open(p))
+    rec = recs.get(f"{kernel}:{workload}") or recs.get(kernel)
     if not rec:
         return None
     sha = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
@@ -376,7 +378,7 @@ def run_ours(args, rank, world, local):
         pre_src = "gated_delta_rule_140_b200/csrc/" + pre_src
         roof_pre = {"bound": "hbm", "achieved": pbytes / pre_s / 1e9, "peak": hbm,
                     "unit": "GB/s", "frac": pbytes / pre_s / 1e9 / hbm,
-                    "traffic": traffic_for(pre_kernel, pre_src), "kernel": pre_kernel,
+                    "traffic": traffic_for(pre_kernel, pre_src, args.workload), "kernel": pre_kernel,
                     "alg_bytes": pbytes, "peak_source": pk_kind}
         roof_dec = {"bound": "hbm", "achieved": dbytes / dec_s / 1e9, "peak": hbm,
                     "unit": "GB/s", "frac": dbytes / dec_s / 1e9 / hbm,
