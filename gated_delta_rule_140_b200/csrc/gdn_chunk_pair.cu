@@ -104,19 +104,23 @@ static_assert(L_GATES % 1024 == 0 && L_GATES + 2 * GATES_STRIDE <= L_GROUP && L_
 constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
               GR_GAM = 576, GR_DEC = 640;
 constexpr int GR_KB = 512;  // KDA beta (after the scratch)
-// KDA (one local group; the other group's space holds these): the B operand of
-// the decayed [K; Q] products, rows di_col(i) .. of it being, for 16-token row
-// block i, B_i = K[0, 16(i+1)) . e^{G_{m_i} - G} (m_i = 16 i + 7), 160 rows per
-// atom column; afterwards Kg = K . e^{G} (W's operand).  Then the per-block
-// tables and a second Kt buffer.
+// KDA (group 0 runs the products, group 1 the gate pass of the next chunk; the
+// group-1 space holds): the B operand of the decayed [K; Q] products, rows
+// di_col(i) .. of it being, for 16-token row block i, B_i = K[0, 16(i+1)) .
+// e^{G_{m_i} - G} (m_i = 16 i + 7), 160 rows per atom column; then two per-block
+// tables, a second Kt buffer and a second raw tile buffer (raw tiles and tables
+// alternate by chunk parity).  W's operand Kg = K . e^{G} replaces KD in its raw
+// tile once the products are done.
 constexpr uint32_t L_BREG = L_GROUP;  // (group 1's space)
 constexpr uint32_t BREG_AC = 160 * 128;      // atom column stride of the stacked B
 __host__ __device__ constexpr uint32_t di_col(int i) { return 8u * i * (i + 1); }  // 0, 16, 48, 96
-constexpr uint32_t L_KTAB = L_BREG + 2 * BREG_AC;  // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
-constexpr uint32_t L_KX2 = L_KTAB + 6144;          // KDA's second Kt buffer
+constexpr uint32_t KTAB_BYTES = 6144;              // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
+constexpr uint32_t L_KTAB = L_BREG + 2 * BREG_AC;  // two tables
+constexpr uint32_t L_KX2 = L_KTAB + 2 * KTAB_BYTES;  // KDA's second Kt buffer
+constexpr uint32_t L_RAW2 = L_KX2 + 16384;         // KDA's second raw tiles [K0 | Q0 | K1 | Q1]
 constexpr uint32_t TM_KD = 192;                    // D = [D_0 | D_1 | D_2 | D_3], 160 columns
 constexpr uint32_t ID_KD = idesc_bf16(128, 160, false, false);
-static_assert(L_KX2 % 1024 == 0 && L_KX2 + 16384 <= 2 * L_GROUP, "KDA layout");
+static_assert(L_RAW2 % 1024 == 0 && L_RAW2 + 32768 <= 2 * L_GROUP, "KDA layout");
 
 // ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
 constexpr uint32_t OFF_COMMON = 2 * L_GROUP;
@@ -129,7 +133,8 @@ static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr int SB_FULL = 0, SB_READY = 2, SB_VO = 4, SB_DS = 6, SB_OFREE = 8, SB_CONS = 12,
               SB_DRAIN = 14;
 // local-CTA mbarriers
-constexpr int LB_TMA = 0, LB_L = 2, LB_SLOTFREE = 4, LB_DRAIN = 6, LB_OFFSET = 8;
+constexpr int LB_TMA = 0, LB_L = 2, LB_SLOTFREE = 4, LB_DRAIN = 6, LB_OFFSET = 8, LB_GATE = 9,
+              LB_BFREE = 10;
 
 // TMEM columns
 constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_GROUP = 192;  // local: per group
@@ -316,11 +321,15 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         const int BAR_G = 1 + g, BAR_INV = 3 + g;
         uint8_t *grp = sm + g * L_GROUP;
         const uint32_t gbase = sbase + g * L_GROUP;
-        uint8_t *raw = grp + L_RAW;
+        // raw tiles of chunk m: GDN, its group's (group = chunk parity); KDA, by parity
+        auto raw_of = [&](int m) -> uint8_t * {
+            return (m & 1) ? sm + (CH ? L_RAW2 : L_GROUP + L_RAW) : sm + L_RAW;
+        };
+        auto ktab_of = [&](int m) { return reinterpret_cast<float *>(sm + L_KTAB + (m & 1) * KTAB_BYTES); };
         uint8_t *kxt = grp + L_KX;
         uint8_t *pzt = grp + L_PZT;
         float *AT = reinterpret_cast<float *>(grp + L_AT);
-        uint64_t *bar_tma = bars + LB_TMA + g, *bar_l = bars + LB_L + g;
+        uint64_t *bar_tma = bars + LB_TMA + g, *bar_l = bars + LB_L + g;  // (GDN: group = parity)
         // ring slot = chunk parity: GDN's two groups own one slot each, KDA's one
         // group alternates between them
         const uint32_t peer_ready0 = map_peer(smem_u32(bars + SB_READY), peer);
@@ -328,8 +337,6 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         const int mstep = CH ? 1 : 2;  // chunks of this group: g, g + mstep, ...
         const bool active = !CH || g == 0;
         const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
-        const uint64_t d_raw = desc_sw128(gbase + L_RAW, 16, 1024);          // [K;Q], K (K-major)
-        const uint64_t d_kmn = desc_sw128(gbase + L_RAW, L_RAW_AC, 1024);    // K (MN-major)
         const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);    // [P; 0]
         const uint64_t d_x1b = desc_sw128(gbase + L_PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 (| X3)
         const uint64_t d_x1x2 = desc_sw128(gbase + L_PZT + PZ_X1, 16, 1024);  // [X1; X2]
@@ -352,13 +359,15 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
         auto issue_tma = [&](int m) {
             const long long t0 = t_begin + (long long)m * C;
+            uint8_t *dst = raw_of(m);
+            uint64_t *bt = bars + LB_TMA + (m & 1);
             fence_proxy_async_smem();
-            mbar_arrive_expect_tx(bar_tma, 4 * 8192);
-            tma_load_3d(raw + 0, &tm_k, 0, h, (int)t0, bar_tma);
-            tma_load_3d(raw + 8192, &tm_q, 0, h, (int)t0, bar_tma);
-            tma_load_3d(raw + L_RAW_AC, &tm_k, 64, h, (int)t0, bar_tma);
-            tma_load_3d(raw + L_RAW_AC + 8192, &tm_q, 64, h, (int)t0, bar_tma);
-            ++issued[g];
+            mbar_arrive_expect_tx(bt, 4 * 8192);
+            tma_load_3d(dst + 0, &tm_k, 0, h, (int)t0, bt);
+            tma_load_3d(dst + 8192, &tm_q, 0, h, (int)t0, bt);
+            tma_load_3d(dst + L_RAW_AC, &tm_k, 64, h, (int)t0, bt);
+            tma_load_3d(dst + L_RAW_AC + 8192, &tm_q, 64, h, (int)t0, bt);
+            ++issued[m & 1];
         };
         // gate rows of a chunk: two buffers, by the chunk's index within the group
         auto gate_rows = [&](int m) {
@@ -418,6 +427,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         };
 
         if (active && storer && g < nchunks) issue_tma(g);
+        if (CH && active && storer && 1 < nchunks) issue_tma(1);  // KDA: two chunks ahead
         if (!CH && lw == 4 && g < nchunks) {
             load_gates(g);
             compute_gates(g);
@@ -428,51 +438,41 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         if (!CH && g == 1 && issuer && nchunks >= 2) ok0 = wt.wait(bars + LB_OFFSET, 0);
         named_bar_or(BAR_G, 256, !ok0);
 
-        for (int m = g; active && m < nchunks; m += mstep) {
-            const int gi = CH ? m : m >> 1;  // index of the chunk within the group
-            const int rs = m & 1;            // its ring slot
-            uint8_t *ring_slot = ring_pair + (size_t)rs * RING_STRIDE;
-            float *gr = gate_rows(m);
-            uint8_t *kxc = (CH && (gi & 1)) ? sm + L_KX2 : kxt;  // this chunk's Kt
-            const long long t0 = t_begin + (long long)m * C;
-            const int L = chunk_len(m);
-            bool ok = true;
-            // ---- this chunk's tiles (rows past the sequence end read as zero); the
-            //      group's next chunk is fetched into L2 meanwhile.  The previous
-            //      chunk's ring tiles must have been read out of shared memory.
-            if (issuer && m + mstep < nchunks) {
-                const int t2 = (int)(t0 + mstep * C);
-                tma_prefetch_l2_3d(&tm_k, 0, h, t2);
-                tma_prefetch_l2_3d(&tm_k, 64, h, t2);
-                tma_prefetch_l2_3d(&tm_q, 0, h, t2);
-                tma_prefetch_l2_3d(&tm_q, 64, h, t2);
-            }
-            if (CH && m + 1 < nchunks) {  // the next chunk's per-channel gates into L2
-                const int pr = gtid >> 2, pc = gtid & 3;  // 64 rows x 4 lines of 128 B
-                if (t0 + C + pr < t_end)
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + C + pr) * H + h) * DK + 32 * pc));
-            }
-            if (issuer) ok = wt.wait(bar_tma, (uint32_t)(gi & 1));
-            if (L < C) {
+        if (CH && g == 1) {
+            // ===== KDA gate group: chunk m's per-channel gates while group 0 runs
+            //       the products of chunk m - 1 =====
+            for (int m = 0; m < nchunks; ++m) {
+                const long long t0 = t_begin + (long long)m * C;
+                const int L = chunk_len(m);
+                uint8_t *rawp = raw_of(m);
+                float *ktab = ktab_of(m);
+                float *gr = reinterpret_cast<float *>(sm + L_GATES + (m & 1) * GATES_STRIDE);  // group 0's
+                uint8_t *kxc = (m & 1) ? sm + L_KX2 : sm + L_KX;
+                bool ok = true;
+                if (m + 1 < nchunks) {  // the next chunk's per-channel gates into L2
+                    const int pr = gtid >> 2, pc = gtid & 3;  // 64 rows x 4 lines of 128 B
+                    if (t0 + C + pr < t_end)
+                        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + C + pr) * H + h) * DK + 32 * pc));
+                }
+                // chunk m's tiles: group 0 loads them once chunk m - 2 is done with
+                // this parity's raw tiles and table (rows past the sequence end are
+                // zeroed here)
+                if (issuer) ok = wt.wait(bars + LB_TMA + (m & 1), (uint32_t)((m >> 1) & 1));
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
                     const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
                     const uint4 z = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(raw + o) = z;
-                    *reinterpret_cast<uint4 *>(raw + 8192 + o) = z;
-                    *reinterpret_cast<uint4 *>(raw + L_RAW_AC + o) = z;
-                    *reinterpret_cast<uint4 *>(raw + L_RAW_AC + 8192 + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + 8192 + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + 8192 + o) = z;
                 }
-            }
-            if constexpr (CH) {
                 // ---- KDA gates: G_rc by a prefix sum over the rows (thread: two
                 //      channels, the 16 rows of block rq) and the block references
                 //      G at m_i = 16 i + 7; then, with every exponent within 8 tokens'
                 //      decay of zero: KD = K e^{G - G_{m(r)}} and QD likewise in place,
                 //      Kt = K e^{G_C - G} (ring tile), B_i = K[0,16(i+1)) e^{G_{m_i} - G}
-                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
-                float *ktab = reinterpret_cast<float *>(sm + L_KTAB);
                 float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f, p70 = 0.f, p71 = 0.f;
                 const float *lp0 = a.log_alpha + ((t0 + 16 * rq) * H + h) * DK + c0;
 #pragma unroll
@@ -492,7 +492,10 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 *reinterpret_cast<float2 *>(ktab + 128 * rq + c0) = make_float2(acc0, acc1);
                 *reinterpret_cast<float2 *>(ktab + 512 + 128 * rq + c0) = make_float2(p70, p71);
                 if (gtid < 64) gr[GR_KB + gtid] = gtid < L ? a.beta[(t0 + gtid) * H + h] : 0.f;
-                named_bar_sync(BAR_G, 256);
+                // the B region (read by chunk m - 1's products), chunk m - 2's Kt and
+                // e^{G_C} (read by its ring stores) are free once group 0 says so
+                if (issuer && m >= 1) ok = wt.wait(bars + LB_BFREE, (uint32_t)((m - 1) & 1));
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 float gm0[4], gm1[4], off0 = 0.f, off1 = 0.f, run0 = 0.f, run1 = 0.f;
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
@@ -540,8 +543,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     const float f0 = __expf(fminf(x0, kMaxNegLogDecay)), f1 = __expf(fminf(x1, kMaxNegLogDecay));
                     const float h0 = __expf(fminf(-x0, kMaxNegLogDecay)), h1 = __expf(fminf(-x1, kMaxNegLogDecay));
                     const uint32_t o = sw128(r, cc >> 3) + cof;
-                    uint32_t *pk = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + o);
-                    uint32_t *pq = reinterpret_cast<uint32_t *>(raw + ac * L_RAW_AC + 8192 + o);
+                    uint32_t *pk = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + o);
+                    uint32_t *pq = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + 8192 + o);
                     const uint32_t kw = *pk, qw = *pq;
                     const float kx = __uint_as_float(kw << 16), ky = __uint_as_float(kw & 0xffff0000u);
                     const float qx = __uint_as_float(qw << 16), qy = __uint_as_float(qw & 0xffff0000u);
@@ -559,6 +562,50 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 if (big > kMaxNegLogDecay) atomicOr(redo + item, 1u);
+                fence_proxy_async_smem();
+                if (named_bar_or(BAR_G, 256, *abort_flag)) break;
+                if (issuer) mbar_arrive(bars + LB_GATE);
+            }
+        }
+        for (int m = g; active && m < nchunks; m += mstep) {
+            const int gi = CH ? m : m >> 1;  // index of the chunk within the group
+            const int rs = m & 1;            // its ring slot
+            uint8_t *ring_slot = ring_pair + (size_t)rs * RING_STRIDE;
+            float *gr = gate_rows(m);
+            uint8_t *kxc = (CH && (gi & 1)) ? sm + L_KX2 : kxt;  // this chunk's Kt
+            uint8_t *rawp = raw_of(m);
+            const uint32_t raw_s = smem_u32(rawp);
+            const uint64_t d_raw = desc_sw128(raw_s, 16, 1024);        // [K;Q], K (K-major)
+            const uint64_t d_kmn = desc_sw128(raw_s, L_RAW_AC, 1024);  // K (MN-major)
+            const long long t0 = t_begin + (long long)m * C;
+            const int L = chunk_len(m);
+            bool ok = true;
+            // ---- this chunk's tiles (rows past the sequence end read as zero); the
+            //      tiles two chunks ahead are fetched into L2 meanwhile.  The previous
+            //      chunk's ring tiles must have been read out of shared memory.
+            if (issuer && m + 2 < nchunks) {
+                const int t2 = (int)(t0 + 2 * C);
+                tma_prefetch_l2_3d(&tm_k, 0, h, t2);
+                tma_prefetch_l2_3d(&tm_k, 64, h, t2);
+                tma_prefetch_l2_3d(&tm_q, 0, h, t2);
+                tma_prefetch_l2_3d(&tm_q, 64, h, t2);
+            }
+            if constexpr (CH) {
+                // KDA: the gate group has prepared KD, QD, Kt, B and the tables
+                if (issuer) ok = wt.wait(bars + LB_GATE, (uint32_t)(m & 1));
+            } else {
+                if (issuer) ok = wt.wait(bar_tma, (uint32_t)(gi & 1));
+                if (L < C) {
+                    if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                    for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
+                        const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
+                        const uint4 z = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(rawp + o) = z;
+                        *reinterpret_cast<uint4 *>(rawp + 8192 + o) = z;
+                        *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + o) = z;
+                        *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + 8192 + o) = z;
+                    }
+                }
             }
             fence_proxy_async_smem();
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
@@ -586,6 +633,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             ++bl_wait;
             if (storer && pend) bulk_wait_read();  // the staged tiles are rewritten below
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            // KDA: the B region and the previous chunk's ring sources are free for the
+            // gate pass of chunk m + 1
+            if (CH && issuer) mbar_arrive(bars + LB_BFREE);
             tc_fence_after();
             // ---- A rows (lanes 0-63) -> fp32;  P rows (lanes 64-127) -> bf16.  GDN
             //      applies the decay here; KDA's product already carries it.
@@ -653,20 +703,20 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 if constexpr (!CH) {
                     if (lw == 4 && m + 2 < nchunks) compute_gates(m + 2);
                 } else {
-                    // Kg = K e^{G} = KD e^{G_{m(r)}} into the B region (its products are done)
-                    const float *fm = reinterpret_cast<const float *>(sm + L_KTAB) + 1024;
+                    // Kg = K e^{G} = KD e^{G_{m(r)}} in place of KD (its products are done)
+                    const float *fm = ktab_of(m) + 1024;
 #pragma unroll 2
                     for (int q2 = 0; q2 < 8; ++q2) {
                         const int idx = (gtid - 128) + 128 * q2;
                         const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
                         float kv[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(raw + ac * L_RAW_AC + sw128(rr, j)), kv);
+                        unpack8(*reinterpret_cast<const uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)), kv);
                         const float *f = fm + 128 * (rr >> 4) + 64 * ac + 8 * j;
                         const float4 d0 = *reinterpret_cast<const float4 *>(f);
                         const float4 d1 = *reinterpret_cast<const float4 *>(f + 4);
                         kv[0] *= d0.x; kv[1] *= d0.y; kv[2] *= d0.z; kv[3] *= d0.w;
                         kv[4] *= d1.x; kv[5] *= d1.y; kv[6] *= d1.z; kv[7] *= d1.w;
-                        *reinterpret_cast<uint4 *>(sm + L_BREG + ac * 8192 + sw128(rr, j)) = pack8(kv);
+                        *reinterpret_cast<uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)) = pack8(kv);
                     }
                 }
             } else {
@@ -838,7 +888,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             //      rows 0-63 = W, rows 64-127 = P W ---------------------------------------
             if (issuer) {
                 tc_fence_after();
-                const uint64_t dkb = CH ? desc_sw128(sbase + L_BREG, 8192, 1024) : d_kmn;  // Kg : K
+                const uint64_t dkb = d_kmn;  // GDN K, KDA Kg (MN-major)
 #pragma unroll
                 for (int k = 0; k < C / 16; ++k)
                     mma_bf16(tm_ab, d_x1x2 + 2 * k, dkb + 128 * k, ID_N128, k > 0);
@@ -856,7 +906,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const float gam = CH ? 1.f : gr[GR_GAM + r];
                 uint8_t *wst = grp + L_AT + lhalf * 8192;
                 uint8_t *qst = pzt + (CH ? (lhalf ? PZ_P : PZ_X3) : (lhalf ? PZ_X2 : PZ_X1));
-                const uint8_t *qt = raw + lhalf * L_RAW_AC + 8192;
+                const uint8_t *qt = rawp + lhalf * L_RAW_AC + 8192;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float x[32];
@@ -876,7 +926,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                             float qv[8];
                             unpack8(*reinterpret_cast<const uint4 *>(qt + o), qv);
                             if constexpr (CH) {  // QD e^{G_{m(r)}}
-                                const float *f = reinterpret_cast<const float *>(sm + L_KTAB) + 1024 +
+                                const float *f = ktab_of(m) + 1024 +
                                                  128 * (r >> 4) + 64 * lhalf + 8 * (4 * hh + j);
                                 const float4 d0 = *reinterpret_cast<const float4 *>(f);
                                 const float4 d1 = *reinterpret_cast<const float4 *>(f + 4);
@@ -895,7 +945,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         const int idx = gtid + 256 * q2;
                         const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
                         float kv[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(raw + ac * L_RAW_AC + sw128(rr, j)), kv);
+                        unpack8(*reinterpret_cast<const uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)), kv);
                         const float sc = gr[GR_KH + rr];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) kv[e] *= sc;
@@ -909,7 +959,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (storer) {
                 // the raw tiles take the group's next chunk (issued before the ring
                 // stores: the TMA unit serves its requests in order)
-                if (m + mstep < nchunks) issue_tma(m + mstep);
+                if (m + 2 < nchunks) issue_tma(m + 2);
                 // once the state CTA has read the slot's previous chunk, the ring
                 // tiles and e^{G_C} go out by bulk copy; the hand-off follows
                 // during the next chunk (or after the loop)
@@ -936,7 +986,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         if (*abort_flag && issuer) {
             mma_commit(bars + LB_DRAIN + g);
             mbar_wait(bars + LB_DRAIN + g, 0, kWaitLimit);
-            if (issued[g] > 0) mbar_wait(bar_tma, (uint32_t)((issued[g] - 1) & 1), kWaitLimit);
+            for (int p = 0; p < 2; ++p)  // GDN: the group's parity; KDA: group 0 loads both
+                if ((p == g || (CH && g == 0)) && issued[p] > 0)
+                    mbar_wait(bars + LB_TMA + p, (uint32_t)((issued[p] - 1) & 1), kWaitLimit);
         }
     } else if (slot >= 0) {
         // ============================ state CTA ============================
