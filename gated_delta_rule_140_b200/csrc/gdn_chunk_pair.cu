@@ -22,10 +22,11 @@
 //
 // Rank 0 ("local" CTA) computes, per chunk, everything that depends only on
 // the chunk's tokens and writes Kt, Qh, -W, R, T_b (bf16 tiles in the
-// swizzled layout the state CTA's MMAs read) and e^{G_C} into a 2-slot ring in
-// global memory, L2-resident since it is rewritten every other chunk.  Two
-// groups of 8 warps work on two chunks at once (even / odd chunks, ring slot =
-// chunk parity); per group and chunk:
+// swizzled layout the state CTA's MMAs read) and e^{G_C} into a 4-slot ring in
+// global memory (chunk m in slot m % 4), L2-resident since it is rewritten every
+// fourth chunk.  GDN: two groups of 8 warps work on two chunks at once (even / odd
+// chunks); KDA: group 1 runs the next chunk's gate pass while group 0 runs the
+// products of this one.  Per chunk:
 //   GDN: D = [K; Q] K^T, then A and P take the decay e^{g_r-g_s} (block
 //        factored, exact inside the diagonal 32x32 blocks); T_bg = T_b
 //        diag(e^{g}) so that W = T_bg K; [P T_bg | R] = P [T_bg | T_b];
@@ -79,6 +80,7 @@ constexpr uint32_t SG_R = 49152, SG_TB = 57344;  // [R; T_b]  (A of the V produc
 constexpr uint32_t SG_TILES = 65536;             // ring slot: the tiles, then
 constexpr uint32_t SG_DECB = 512;                //   e^{G_C} per key channel
 constexpr uint32_t RING_STRIDE = SG_TILES + 1024;
+constexpr int NRING = 4;                         // ring slots per cluster (chunk m: slot m % 4)
 constexpr uint32_t SG_V = 65536;                 // stage: V tiles, d_v halves at +8K
 constexpr uint32_t SG_DEC = 81920;               //        e^{G_C}
 constexpr uint32_t S_STAGE = 82944;
@@ -86,19 +88,35 @@ constexpr uint32_t S_STAGE_TX = SG_TILES + SG_DECB + 2 * 8192;
 constexpr uint32_t S_OFF_SB = 2 * S_STAGE;       // S_h^T bf16, MN-major [c][i], 16 KB per half
 constexpr uint32_t S_OFF_VP = S_OFF_SB + 2 * 16384;  // V'_h bf16, MN-major [r][i], 8 KB per half
 
-// ---- local-CTA group layout ---------------------------------------------------
-constexpr uint32_t L_RAW = 0;          // [K0 | Q0 | K1 | Q1], 8 KB each (TMA)
-constexpr uint32_t L_RAW_AC = 16384;   //   atom column stride: [K_a; Q_a] is an M=128 tile
-constexpr uint32_t L_KX = 32768;       // 2 x 8 KB: KDA Ki (MMA operand), then Kt; GDN Kt
-constexpr uint32_t L_PZT = 49152;      // [P | 0 | X1 | X2 | X3], 8 KB each
-constexpr uint32_t PZ_P = 0, PZ_Z = 8192, PZ_X1 = 16384, PZ_X2 = 24576, PZ_X3 = 32768;
+// ---- local-CTA layout ------------------------------------------------------------
+// A raw tile buffer is [K0 | Q0 | K1 | Q1], 8 KB each (TMA), atom column stride
+// L_RAW_AC, so that [K_a; Q_a] is an M=128 tile.  A group's space holds
+// [P | X1 | X2 | X3] (8 KB each; [P; X1] is the A operand of the P products,
+// whose rows 64-127 are never read), A and then T in place (fp32 [64][LDA]),
+// and two gate-row buffers.
 //   GDN: X1 = T_bg, X2 = P T_bg, X3 = T_b;  KDA: X1 = T_b, X2 = R, X3 = Qh staging
-constexpr uint32_t L_AT = 90112;                   // A, then T in place: fp32 [64][LDA]
-constexpr uint32_t L_GATES = L_AT + 64 * LDA * 4;  // two gate-row buffers
+// GDN: three raw buffers shared by the two groups (chunk m in buffer m % 3, so
+// that a chunk's tiles are loaded while the chunk three back is still being
+// written out), then the two group spaces; Kt replaces K in its raw buffer.
+// KDA: group 0's space starts with its raw buffer and its Kt buffer; group 1's
+// space holds the gate group's buffers (below).
+constexpr uint32_t L_RAW_AC = 16384;
+constexpr uint32_t RAW_BYTES = 32768;
+constexpr uint32_t PZ_P = 0, PZ_X1 = 8192, PZ_X2 = 16384, PZ_X3 = 24576, PZT_BYTES = 32768;
+constexpr uint32_t AT_BYTES = 64 * LDA * 4;
 constexpr uint32_t GATES_STRIDE = 3072;
-constexpr uint32_t L_GROUP = 113664;
-static_assert(L_GATES % 1024 == 0 && L_GATES + 2 * GATES_STRIDE <= L_GROUP && L_GROUP % 1024 == 0,
-              "local group layout");
+template <bool CH>
+struct Lay {
+    static constexpr uint32_t RAWP = 0;                           // GDN: the 3 raw buffers
+    static constexpr uint32_t G0 = CH ? 0 : 3 * RAW_BYTES;        // group 0's space
+    static constexpr uint32_t RAW = 0, KX = RAW_BYTES;            // KDA, within group 0's space
+    static constexpr uint32_t PZT = CH ? KX + 16384 : 0;
+    static constexpr uint32_t AT = PZT + PZT_BYTES;
+    static constexpr uint32_t GATES = AT + AT_BYTES;
+    static constexpr uint32_t GSZ = GATES + 2 * GATES_STRIDE;     // a group's space
+};
+static_assert(Lay<false>::GATES % 1024 == 0 && Lay<false>::GSZ % 1024 == 0 &&
+              Lay<true>::GATES % 1024 == 0 && Lay<true>::GSZ % 1024 == 0, "local group layout");
 // gate rows (floats).  GDN: g beta beta*gamma colf rowf[4] kh gamma, and dec;
 // KDA: beta and dec (the first 512 floats are the prefix-sum scratch)
 constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
@@ -111,7 +129,7 @@ constexpr int GR_KB = 512;  // KDA beta (after the scratch)
 // tables, a second Kt buffer and a second raw tile buffer (raw tiles and tables
 // alternate by chunk parity).  W's operand Kg = K . e^{G} replaces KD in its raw
 // tile once the products are done.
-constexpr uint32_t L_BREG = L_GROUP;  // (group 1's space)
+constexpr uint32_t L_BREG = Lay<true>::GSZ;  // (group 1's space)
 constexpr uint32_t BREG_AC = 160 * 128;      // atom column stride of the stacked B
 __host__ __device__ constexpr uint32_t di_col(int i) { return 8u * i * (i + 1); }  // 0, 16, 48, 96
 constexpr uint32_t KTAB_BYTES = 6144;              // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
@@ -120,21 +138,23 @@ constexpr uint32_t L_KX2 = L_KTAB + 2 * KTAB_BYTES;  // KDA's second Kt buffer
 constexpr uint32_t L_RAW2 = L_KX2 + 16384;         // KDA's second raw tiles [K0 | Q0 | K1 | Q1]
 constexpr uint32_t TM_KD = 192;                    // D = [D_0 | D_1 | D_2 | D_3], 160 columns
 constexpr uint32_t ID_KD = idesc_bf16(128, 160, false, false);
-static_assert(L_RAW2 % 1024 == 0 && L_RAW2 + 32768 <= 2 * L_GROUP, "KDA layout");
+static_assert(L_RAW2 % 1024 == 0, "KDA layout");
 
 // ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
-constexpr uint32_t OFF_COMMON = 2 * L_GROUP;
-static_assert(S_OFF_VP + 2 * 8192 <= OFF_COMMON, "state layout");
+constexpr uint32_t OFF_COMMON = 215040;
+static_assert(S_OFF_VP + 2 * 8192 <= OFF_COMMON && L_RAW2 + RAW_BYTES <= OFF_COMMON &&
+              Lay<false>::G0 + 2 * Lay<false>::GSZ <= OFF_COMMON, "shared memory layout");
 constexpr uint32_t CM_ABORT = 0, CM_SLOT = 4, CM_TMEM = 8, CM_ISSUED = 32, CM_BARS = 64;
-constexpr uint32_t SMEM_USED = OFF_COMMON + CM_BARS + 16 * 8;
+constexpr int NBARS = 18;
+constexpr uint32_t SMEM_USED = OFF_COMMON + CM_BARS + NBARS * 8;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-// state-CTA mbarriers
-constexpr int SB_FULL = 0, SB_READY = 2, SB_VO = 4, SB_DS = 6, SB_OFREE = 8, SB_CONS = 12,
-              SB_DRAIN = 14;
-// local-CTA mbarriers
-constexpr int LB_TMA = 0, LB_L = 2, LB_SLOTFREE = 4, LB_DRAIN = 6, LB_OFFSET = 8, LB_GATE = 9,
-              LB_BFREE = 10;
+// state-CTA mbarriers (READY: one per ring slot; OFREE: per stage and value half)
+constexpr int SB_FULL = 0, SB_READY = 2, SB_VO = 6, SB_DS = 8, SB_OFREE = 10, SB_CONS = 14,
+              SB_DRAIN = 16;
+// local-CTA mbarriers (TMA: one per raw buffer; SLOTFREE: one per ring slot)
+constexpr int LB_TMA = 0, LB_L = 3, LB_SLOTFREE = 5, LB_DRAIN = 9, LB_OFFSET = 11, LB_GATE = 12,
+              LB_BFREE = 13;
 
 // TMEM columns
 constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_GROUP = 192;  // local: per group
@@ -259,7 +279,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
     volatile int *abort_flag = reinterpret_cast<volatile int *>(cm + CM_ABORT);
     uint64_t *bars = reinterpret_cast<uint64_t *>(cm + CM_BARS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cm + CM_TMEM);
-    int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // [2] loads issued per stage / group
+    int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // [3] loads issued per stage / raw buffer
 
     const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -278,11 +298,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
     if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < NBARS; ++i)
             mbar_init(bars + i, (rank == 1 && (i == SB_CONS || i == SB_CONS + 1)) ? 2 : 1);
         fence_mbar_init();
         *abort_flag = 0;
-        issued[0] = issued[1] = 0;
+        issued[0] = issued[1] = issued[2] = 0;
         if (rank == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -312,34 +332,36 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             *abort_flag = 1;
         }
     }
-    uint8_t *ring_pair = slot >= 0 ? ring + (size_t)slot * 2 * RING_STRIDE : ring;
+    uint8_t *ring_pair = slot >= 0 ? ring + (size_t)slot * NRING * RING_STRIDE : ring;
 
     if (slot >= 0 && rank == 0) {
         // ============================ local CTA ============================
         const int g = warp >> 3, lw = warp & 7, lq = warp & 3, lhalf = lw >> 2;
         const int gtid = tid & 255;
         const int BAR_G = 1 + g, BAR_INV = 3 + g;
-        uint8_t *grp = sm + g * L_GROUP;
-        const uint32_t gbase = sbase + g * L_GROUP;
-        // raw tiles of chunk m: GDN, its group's (group = chunk parity); KDA, by parity
+        using LY = Lay<CH>;
+        uint8_t *grp = sm + LY::G0 + g * LY::GSZ;
+        const uint32_t gbase = sbase + LY::G0 + g * LY::GSZ;
+        // raw tiles of chunk m: GDN, buffer m % 3; KDA, by parity.  Each buffer has
+        // its TMA barrier, the loads into it completing in order.
+        auto rbuf = [&](int m) -> int { return CH ? (m & 1) : (m % 3); };
         auto raw_of = [&](int m) -> uint8_t * {
-            return (m & 1) ? sm + (CH ? L_RAW2 : L_GROUP + L_RAW) : sm + L_RAW;
+            return CH ? ((m & 1) ? sm + L_RAW2 : sm + LY::RAW) : sm + LY::RAWP + rbuf(m) * RAW_BYTES;
         };
+        auto tma_phase = [&](int m) -> uint32_t { return (uint32_t)((CH ? (m >> 1) : (m / 3)) & 1); };
         auto ktab_of = [&](int m) { return reinterpret_cast<float *>(sm + L_KTAB + (m & 1) * KTAB_BYTES); };
-        uint8_t *kxt = grp + L_KX;
-        uint8_t *pzt = grp + L_PZT;
-        float *AT = reinterpret_cast<float *>(grp + L_AT);
-        uint64_t *bar_tma = bars + LB_TMA + g, *bar_l = bars + LB_L + g;  // (GDN: group = parity)
-        // ring slot = chunk parity: GDN's two groups own one slot each, KDA's one
-        // group alternates between them
+        uint8_t *kxt = CH ? sm + LY::KX : nullptr;  // KDA Kt of even chunks
+        uint8_t *pzt = grp + LY::PZT;
+        float *AT = reinterpret_cast<float *>(grp + LY::AT);
+        uint64_t *bar_l = bars + LB_L + g;
         const uint32_t peer_ready0 = map_peer(smem_u32(bars + SB_READY), peer);
         const uint32_t tm_kq = tmem + g * TM_GROUP + TM_KQ, tm_ab = tmem + g * TM_GROUP + TM_AB;
         const int mstep = CH ? 1 : 2;  // chunks of this group: g, g + mstep, ...
         const bool active = !CH || g == 0;
         const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
-        const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);    // [P; 0]
-        const uint64_t d_x1b = desc_sw128(gbase + L_PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 (| X3)
-        const uint64_t d_x1x2 = desc_sw128(gbase + L_PZT + PZ_X1, 16, 1024);  // [X1; X2]
+        const uint64_t d_pz = desc_sw128(gbase + LY::PZT + PZ_P, 16, 1024);    // [P; X1]
+        const uint64_t d_x1b = desc_sw128(gbase + LY::PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 (| X3)
+        const uint64_t d_x1x2 = desc_sw128(gbase + LY::PZT + PZ_X1, 16, 1024);  // [X1; X2]
         uint32_t bl_wait = 0;
         const bool issuer = gtid == 0;       // MMAs
         const bool storer = gtid == 7 * 32;  // tile reloads, ring stores and the hand-off
@@ -353,25 +375,22 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             pend = false;
         };
 
-        for (int i = gtid; i < 512; i += 256)
-            reinterpret_cast<uint4 *>(pzt + PZ_Z)[i] = make_uint4(0, 0, 0, 0);
-        fence_proxy_async_smem();
 
         auto issue_tma = [&](int m) {
             const long long t0 = t_begin + (long long)m * C;
             uint8_t *dst = raw_of(m);
-            uint64_t *bt = bars + LB_TMA + (m & 1);
+            uint64_t *bt = bars + LB_TMA + rbuf(m);
             fence_proxy_async_smem();
             mbar_arrive_expect_tx(bt, 4 * 8192);
             tma_load_3d(dst + 0, &tm_k, 0, h, (int)t0, bt);
             tma_load_3d(dst + 8192, &tm_q, 0, h, (int)t0, bt);
             tma_load_3d(dst + L_RAW_AC, &tm_k, 64, h, (int)t0, bt);
             tma_load_3d(dst + L_RAW_AC + 8192, &tm_q, 64, h, (int)t0, bt);
-            ++issued[m & 1];
+            atomicAdd(issued + rbuf(m), 1);  // (GDN: both groups' storers load)
         };
         // gate rows of a chunk: two buffers, by the chunk's index within the group
         auto gate_rows = [&](int m) {
-            return reinterpret_cast<float *>(grp + L_GATES + (((CH ? m : m >> 1)) & 1) * GATES_STRIDE);
+            return reinterpret_cast<float *>(grp + LY::GATES + (((CH ? m : m >> 1)) & 1) * GATES_STRIDE);
         };
         // GDN gates, prefetched one group chunk ahead in the registers of warp lw 4
         float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
@@ -426,8 +445,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             *reinterpret_cast<float4 *>(gr + GR_DEC + 4 * lane) = make_float4(dC, dC, dC, dC);
         };
 
+        // the first chunks' tiles: GDN, chunks 0-2 (one per raw buffer); KDA, 0 and 1
         if (active && storer && g < nchunks) issue_tma(g);
-        if (CH && active && storer && 1 < nchunks) issue_tma(1);  // KDA: two chunks ahead
+        if (active && storer && g == 0 && (CH ? 1 : 2) < nchunks) issue_tma(CH ? 1 : 2);
         if (!CH && lw == 4 && g < nchunks) {
             load_gates(g);
             compute_gates(g);
@@ -446,8 +466,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const int L = chunk_len(m);
                 uint8_t *rawp = raw_of(m);
                 float *ktab = ktab_of(m);
-                float *gr = reinterpret_cast<float *>(sm + L_GATES + (m & 1) * GATES_STRIDE);  // group 0's
-                uint8_t *kxc = (m & 1) ? sm + L_KX2 : sm + L_KX;
+                float *gr = reinterpret_cast<float *>(sm + LY::GATES + (m & 1) * GATES_STRIDE);  // group 0's
+                uint8_t *kxc = (m & 1) ? sm + L_KX2 : sm + LY::KX;
                 bool ok = true;
                 if (m + 1 < nchunks) {  // the next chunk's per-channel gates into L2
                     const int pr = gtid >> 2, pc = gtid & 3;  // 64 rows x 4 lines of 128 B
@@ -457,7 +477,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 // chunk m's tiles: group 0 loads them once chunk m - 2 is done with
                 // this parity's raw tiles and table (rows past the sequence end are
                 // zeroed here)
-                if (issuer) ok = wt.wait(bars + LB_TMA + (m & 1), (uint32_t)((m >> 1) & 1));
+                if (issuer) ok = wt.wait(bars + LB_TMA + rbuf(m), tma_phase(m));
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
                     const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
@@ -569,7 +589,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         }
         for (int m = g; active && m < nchunks; m += mstep) {
             const int gi = CH ? m : m >> 1;  // index of the chunk within the group
-            const int rs = m & 1;            // its ring slot
+            const int rs = m % NRING;        // its ring slot
             uint8_t *ring_slot = ring_pair + (size_t)rs * RING_STRIDE;
             float *gr = gate_rows(m);
             uint8_t *kxc = (CH && (gi & 1)) ? sm + L_KX2 : kxt;  // this chunk's Kt
@@ -581,10 +601,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             const int L = chunk_len(m);
             bool ok = true;
             // ---- this chunk's tiles (rows past the sequence end read as zero); the
-            //      tiles two chunks ahead are fetched into L2 meanwhile.  The previous
-            //      chunk's ring tiles must have been read out of shared memory.
-            if (issuer && m + 2 < nchunks) {
-                const int t2 = (int)(t0 + 2 * C);
+            //      tiles of the next chunk this group's storer loads are fetched into
+            //      L2 meanwhile (KDA: m + 2; GDN: m + 3).  The previous chunk's ring
+            //      tiles must have been read out of shared memory.
+            if (issuer && m + (CH ? 2 : 3) < nchunks) {
+                const int t2 = (int)(t0 + (CH ? 2 : 3) * C);
                 tma_prefetch_l2_3d(&tm_k, 0, h, t2);
                 tma_prefetch_l2_3d(&tm_k, 64, h, t2);
                 tma_prefetch_l2_3d(&tm_q, 0, h, t2);
@@ -594,7 +615,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 // KDA: the gate group has prepared KD, QD, Kt, B and the tables
                 if (issuer) ok = wt.wait(bars + LB_GATE, (uint32_t)(m & 1));
             } else {
-                if (issuer) ok = wt.wait(bar_tma, (uint32_t)(gi & 1));
+                if (issuer) ok = wt.wait(bars + LB_TMA + rbuf(m), tma_phase(m));
                 if (L < C) {
                     if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                     for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
@@ -632,6 +653,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             }
             ++bl_wait;
             if (storer && pend) bulk_wait_read();  // the staged tiles are rewritten below
+            // GDN: the raw buffer of this group's previous chunk (m - 2, Kt in place of K
+            // read by its ring stores) takes chunk m + 1, the other group's next
+            if (!CH && storer && m >= 2 && m + 1 < nchunks) issue_tma(m + 1);
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
             // KDA: the B region and the previous chunk's ring sources are free for the
             // gate pass of chunk m + 1
@@ -904,7 +928,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             {
                 const int r = 32 * (lq & 1) + lane;
                 const float gam = CH ? 1.f : gr[GR_GAM + r];
-                uint8_t *wst = grp + L_AT + lhalf * 8192;
+                uint8_t *wst = grp + LY::AT + lhalf * 8192;
                 uint8_t *qst = pzt + (CH ? (lhalf ? PZ_P : PZ_X3) : (lhalf ? PZ_X2 : PZ_X1));
                 const uint8_t *qt = rawp + lhalf * L_RAW_AC + 8192;
 #pragma unroll
@@ -949,7 +973,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         const float sc = gr[GR_KH + rr];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) kv[e] *= sc;
-                        *reinterpret_cast<uint4 *>(kxt + ac * 8192 + sw128(rr, j)) = pack8(kv);
+                        *reinterpret_cast<uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)) = pack8(kv);
                     }
                 }
             }
@@ -957,16 +981,17 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             tc_fence_before();
             if (named_bar_or(BAR_G, 256, *abort_flag)) break;
             if (storer) {
-                // the raw tiles take the group's next chunk (issued before the ring
-                // stores: the TMA unit serves its requests in order)
-                if (m + 2 < nchunks) issue_tma(m + 2);
+                // KDA: the raw tiles take chunk m + 2 (issued before the ring stores:
+                // the TMA unit serves its requests in order)
+                if (CH && m + 2 < nchunks) issue_tma(m + 2);
                 // once the state CTA has read the slot's previous chunk, the ring
                 // tiles and e^{G_C} go out by bulk copy; the hand-off follows
                 // during the next chunk (or after the loop)
-                if (m < 2 || wt.wait_peer(bars + LB_SLOTFREE + rs, (uint32_t)(((m >> 1) - 1) & 1))) {
-                    const uint8_t *at8 = grp + L_AT;
-                    bulk_store(ring_slot + SG_KT, kxc, 8192);
-                    bulk_store(ring_slot + SG_AC + SG_KT, kxc + 8192, 8192);
+                if (m < NRING || wt.wait_peer(bars + LB_SLOTFREE + rs, (uint32_t)(((m / NRING) - 1) & 1))) {
+                    const uint8_t *at8 = grp + LY::AT;
+                    const uint8_t *kts = CH ? kxc : rawp;  // GDN: Kt in place of K
+                    bulk_store(ring_slot + SG_KT, kts, 8192);
+                    bulk_store(ring_slot + SG_AC + SG_KT, kts + (CH ? 8192 : L_RAW_AC), 8192);
                     bulk_store(ring_slot + SG_MW, at8, 8192);
                     bulk_store(ring_slot + SG_AC + SG_MW, at8 + 8192, 8192);
                     bulk_store(ring_slot + SG_QH, pzt + (CH ? PZ_X3 : PZ_X1), 8192);
@@ -986,9 +1011,6 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         if (*abort_flag && issuer) {
             mma_commit(bars + LB_DRAIN + g);
             mbar_wait(bars + LB_DRAIN + g, 0, kWaitLimit);
-            for (int p = 0; p < 2; ++p)  // GDN: the group's parity; KDA: group 0 loads both
-                if ((p == g || (CH && g == 0)) && issued[p] > 0)
-                    mbar_wait(bars + LB_TMA + p, (uint32_t)((issued[p] - 1) & 1), kWaitLimit);
         }
     } else if (slot >= 0) {
         // ============================ state CTA ============================
@@ -1160,10 +1182,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 uint8_t *stage = sm + st * S_STAGE;
                 bool ok = true;
                 if (m >= 2) ok = wt.wait(bars + SB_CONS + st, (uint32_t)((it - 1) & 1));
-                if (ok) ok = wt.wait_peer(bars + SB_READY + st, (uint32_t)(it & 1));
+                const int rs = m % NRING;
+                if (ok) ok = wt.wait_peer(bars + SB_READY + rs, (uint32_t)((m / NRING) & 1));
                 if (!ok) break;
                 fence_proxy_async_global();
-                const uint8_t *src = ring_pair + (size_t)st * RING_STRIDE;
+                const uint8_t *src = ring_pair + (size_t)rs * RING_STRIDE;
                 const long long t0 = t_begin + (long long)m * C;
                 mbar_arrive_expect_tx(bars + SB_FULL + st, S_STAGE_TX);
 #pragma unroll
@@ -1175,7 +1198,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 ++issued[st];
                 // the slot is read once the stage has landed: give it back
                 if (!wt.wait(bars + SB_FULL + st, (uint32_t)(it & 1))) break;
-                mbar_arrive_peer(peer_slotfree + 8 * (LB_SLOTFREE + st));
+                mbar_arrive_peer(peer_slotfree + 8 * (LB_SLOTFREE + rs));
             }
             if (*abort_flag)
                 for (int st = 0; st < 2; ++st)
@@ -1186,7 +1209,14 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && *abort_flag && slot >= 0) atomicOr(a.err, kErrTimeout);
+    if (tid == 0 && *abort_flag && slot >= 0) {
+        atomicOr(a.err, kErrTimeout);
+        // local CTA: every raw buffer's last tile load lands before the CTA exits
+        // (both groups' storers load; all have left their loops here)
+        if (rank == 0)
+            for (int p = 0; p < 3; ++p)
+                if (issued[p] > 0) mbar_wait(bars + LB_TMA + p, (uint32_t)((issued[p] - 1) & 1), kWaitLimit);
+    }
     cluster_sync();  // no CTA leaves while its peer may still address its memory
     if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
 }
@@ -1199,7 +1229,7 @@ int ring_slots_for_device() {
     return 2 * nsm;  // SM ids are below this on every part this kernel runs on
 }
 
-size_t ring_bytes(int slots) { return (size_t)slots * 2 * RING_STRIDE; }
+size_t ring_bytes(int slots) { return (size_t)slots * NRING * RING_STRIDE; }
 
 template <bool CH>
 cudaError_t launch_t(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
