@@ -628,10 +628,15 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
             }
-            fence_proxy_async_smem();
-            if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            // GDN with a full chunk: nothing to publish, so the MMA goes out as soon as
+            // the tiles are in (the storer may still be issuing the previous chunk's
+            // ring stores); an abort is seen at the barrier after it
+            if (CH || L < C) {
+                fence_proxy_async_smem();
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+            }
             // ---- D_kq = [K; Q] K^T (GDN) or [KD; QD] [B_0; B_1; B_2; B_3]^T (KDA) -------
-            if (issuer) {
+            if (issuer && ok) {
                 tc_fence_after();
                 if constexpr (CH) {
                     const uint64_t db = desc_sw128(sbase + L_BREG, 16, 1024);
@@ -652,7 +657,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 ok = wt.wait(bar_l, bl_wait & 1);
             }
             ++bl_wait;
-            if (storer && pend) bulk_wait_read();  // the staged tiles are rewritten below
+            // the tiles that the A/P phase below rewrites (and, KDA, the gate group's
+            // Kt and e^{G_C}) went out first, as their own bulk group
+            if (storer && pend) bulk_wait_read_but_last();
             // GDN: the raw buffer of this group's previous chunk (m - 2, Kt in place of K
             // read by its ring stores) takes chunk m + 1, the other group's next
             if (!CH && storer && m >= 2 && m + 1 < nchunks) issue_tma(m + 1);
@@ -988,17 +995,32 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 // tiles and e^{G_C} go out by bulk copy; the hand-off follows
                 // during the next chunk (or after the loop)
                 if (m < NRING || wt.wait_peer(bars + LB_SLOTFREE + rs, (uint32_t)(((m / NRING) - 1) & 1))) {
+                    // two bulk groups: first what the next chunk of this group rewrites
+                    // early (the A/P phase: -W's staging in A's space, the P tile; the
+                    // raw buffer's Kt, GDN; the gate group's Kt and e^{G_C}, KDA), then
+                    // the rest (rewritten from the T_b phase on, after the hand-off
+                    // has waited for every store)
                     const uint8_t *at8 = grp + LY::AT;
                     const uint8_t *kts = CH ? kxc : rawp;  // GDN: Kt in place of K
                     bulk_store(ring_slot + SG_KT, kts, 8192);
                     bulk_store(ring_slot + SG_AC + SG_KT, kts + (CH ? 8192 : L_RAW_AC), 8192);
                     bulk_store(ring_slot + SG_MW, at8, 8192);
                     bulk_store(ring_slot + SG_AC + SG_MW, at8 + 8192, 8192);
-                    bulk_store(ring_slot + SG_QH, pzt + (CH ? PZ_X3 : PZ_X1), 8192);
-                    bulk_store(ring_slot + SG_AC + SG_QH, pzt + (CH ? PZ_P : PZ_X2), 8192);
-                    bulk_store(ring_slot + SG_R, pzt + (CH ? PZ_X2 : PZ_P), 8192);
-                    bulk_store(ring_slot + SG_TB, pzt + (CH ? PZ_X1 : PZ_X3), 8192);
                     bulk_store(ring_slot + SG_TILES, gr + GR_DEC, SG_DECB);
+                    if constexpr (CH) {
+                        bulk_store(ring_slot + SG_AC + SG_QH, pzt + PZ_P, 8192);
+                    } else {
+                        bulk_store(ring_slot + SG_R, pzt + PZ_P, 8192);
+                    }
+                    bulk_commit();
+                    if constexpr (CH) {
+                        bulk_store(ring_slot + SG_QH, pzt + PZ_X3, 8192);
+                        bulk_store(ring_slot + SG_R, pzt + PZ_X2, 8192);
+                    } else {
+                        bulk_store(ring_slot + SG_QH, pzt + PZ_X1, 8192);
+                        bulk_store(ring_slot + SG_AC + SG_QH, pzt + PZ_X2, 8192);
+                    }
+                    bulk_store(ring_slot + SG_TB, pzt + (CH ? PZ_X1 : PZ_X3), 8192);
                     bulk_commit();
                     pend = true;
                     pend_slot = rs;
