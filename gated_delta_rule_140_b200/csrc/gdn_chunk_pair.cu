@@ -474,24 +474,12 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     if (t0 + C + pr < t_end)
                         asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + C + pr) * H + h) * DK + 32 * pc));
                 }
-                // chunk m's tiles: group 0 loads them once chunk m - 2 is done with
-                // this parity's raw tiles and table (rows past the sequence end are
-                // zeroed here)
-                if (issuer) ok = wt.wait(bars + LB_TMA + rbuf(m), tma_phase(m));
-                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-                for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
-                    const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(rawp + o) = z;
-                    *reinterpret_cast<uint4 *>(rawp + 8192 + o) = z;
-                    *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + o) = z;
-                    *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + 8192 + o) = z;
-                }
                 // ---- KDA gates: G_rc by a prefix sum over the rows (thread: two
                 //      channels, the 16 rows of block rq) and the block references
                 //      G at m_i = 16 i + 7; then, with every exponent within 8 tokens'
                 //      decay of zero: KD = K e^{G - G_{m(r)}} and QD likewise in place,
-                //      Kt = K e^{G_C - G} (ring tile), B_i = K[0,16(i+1)) e^{G_{m_i} - G}
+                //      Kt = K e^{G_C - G} (ring tile), B_i = K[0,16(i+1)) e^{G_{m_i} - G}.
+                //      The sums need no tiles, so they run while the tiles load.
                 const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
                 float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f, p70 = 0.f, p71 = 0.f;
                 const float *lp0 = a.log_alpha + ((t0 + 16 * rq) * H + h) * DK + c0;
@@ -511,6 +499,19 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 }
                 *reinterpret_cast<float2 *>(ktab + 128 * rq + c0) = make_float2(acc0, acc1);
                 *reinterpret_cast<float2 *>(ktab + 512 + 128 * rq + c0) = make_float2(p70, p71);
+                // chunk m's tiles: group 0 loads them once chunk m - 2 is done with
+                // this parity's raw tiles, table and gate rows (rows past the sequence
+                // end are zeroed here)
+                if (issuer) ok = wt.wait(bars + LB_TMA + rbuf(m), tma_phase(m));
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
+                    const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(rawp + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + 8192 + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + o) = z;
+                    *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + 8192 + o) = z;
+                }
                 if (gtid < 64) gr[GR_KB + gtid] = gtid < L ? a.beta[(t0 + gtid) * H + h] : 0.f;
                 // the B region (read by chunk m - 1's products), chunk m - 2's Kt and
                 // e^{G_C} (read by its ring stores) are free once group 0 says so
