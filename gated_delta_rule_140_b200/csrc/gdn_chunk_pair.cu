@@ -224,6 +224,33 @@ __device__ __forceinline__ void decay_row(float *x, int r, int rq, int half, con
     }
 }
 
+// Column j of (I + A_d)^{-1} for the 16x16 diagonal block A_d at (o, o) of the
+// fp32 [64][LDA] tile (strictly lower), by left-looking forward substitution:
+// t_i = [i == j] - sum_{k < i} a_ik t_k, row i of the block read with float4
+// loads (t_k = 0 for k < j makes the rows above j come out right).  Called by
+// lanes 0-15 of a warp; the column replaces the block's column j once all 16
+// lanes have read the block.
+__device__ __forceinline__ void invert_diag16(float *AT, int o, int j) {
+    float t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float *row = AT + (o + i) * LDA + o;
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < (i + 3) / 4; ++q) {
+            const float4 av = *reinterpret_cast<const float4 *>(row + 4 * q);
+            const float ak[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (4 * q + e < i) acc[e] = fmaf(ak[e], t[4 * q + e], acc[e]);
+        }
+        t[i] = (i == j ? 1.f : 0.f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+    __syncwarp(0x0000ffffu);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) AT[(o + i) * LDA + o + j] = t[i];
+}
+
 struct Waiter {
     volatile int *abort;
     uint32_t peer_abort;  // shared::cluster address of the peer's abort flag
@@ -483,11 +510,22 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
                 float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f, p70 = 0.f, p71 = 0.f;
                 const float *lp0 = a.log_alpha + ((t0 + 16 * rq) * H + h) * DK + c0;
+                if ((reinterpret_cast<uintptr_t>(a.log_alpha) & 7) == 0) {  // uniform
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {  // all loads first, then the sums
-                    const bool in = 16 * rq + i < L;
-                    gl0[i] = in ? lp0[(size_t)i * H * DK] : 0.f;
-                    gl1[i] = in ? lp0[(size_t)i * H * DK + 1] : 0.f;
+                    for (int i = 0; i < 16; ++i) {  // all loads first, then the sums
+                        const float2 v = 16 * rq + i < L
+                                             ? *reinterpret_cast<const float2 *>(lp0 + (size_t)i * H * DK)
+                                             : make_float2(0.f, 0.f);
+                        gl0[i] = v.x;
+                        gl1[i] = v.y;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const bool in = 16 * rq + i < L;
+                        gl0[i] = in ? lp0[(size_t)i * H * DK] : 0.f;
+                        gl1[i] = in ? lp0[(size_t)i * H * DK + 1] : 0.f;
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
@@ -753,21 +791,26 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 }
             } else {
                 // (1) 16x16 diagonal blocks: warp lw inverts block lw; lane j < 16
-                //     owns column j (right-looking forward substitution), then writes
-                //     it over the block once the warp has read all of A's block.
+                //     owns column j, then writes it over the block once the warp has
+                //     read all of A's block.  GDN: right-looking forward substitution
+                //     (measured faster there); KDA: left-looking with row loads.
                 if (lane < 16) {
-                    const int o = 16 * lw, j = lane;
-                    float t[16];
+                    if constexpr (CH) {
+                        invert_diag16(AT, 16 * lw, lane);
+                    } else {
+                        const int o = 16 * lw, j = lane;
+                        float t[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
+                        for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
 #pragma unroll
-                    for (int mm = 0; mm < 15; ++mm) {
+                        for (int mm = 0; mm < 15; ++mm) {
 #pragma unroll
-                        for (int i = mm + 1; i < 16; ++i) t[i] -= AT[(o + i) * LDA + o + mm] * t[mm];
+                            for (int i = mm + 1; i < 16; ++i) t[i] -= AT[(o + i) * LDA + o + mm] * t[mm];
+                        }
+                        __syncwarp(0x0000ffffu);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) AT[(o + i) * LDA + o + j] = t[i];
                     }
-                    __syncwarp(0x0000ffffu);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) AT[(o + i) * LDA + o + j] = t[i];
                 }
                 named_bar_sync(BAR_INV, 128);
                 // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22);
