@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--decode-workload NAME]
-                    [--prefill-kernel default|pair|cuda_cores]
+                    [--prefill-kernel default|pair|one_cta|cuda_cores]
 
 A step is one pass of the whole hot path on one GPU:
   * prefill leg: gdn_chunk_fwd over one batch of the prefill workload
@@ -281,6 +281,7 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.current_stream()
 
     kflags = {"pair": args.prefill_kernel == "pair",
+              "one_cta": args.prefill_kernel == "one_cta",
               "cuda_cores": args.prefill_kernel == "cuda_cores"}
 
     def prefill():
@@ -426,7 +427,7 @@ def main():
     ap.add_argument("--workload", default="gdn_prefill_bf16")
     ap.add_argument("--decode-workload", default="gdn_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--prefill-kernel", choices=["default", "pair", "cuda_cores"],
+    ap.add_argument("--prefill-kernel", choices=["default", "pair", "one_cta", "cuda_cores"],
                     default="default",
                     help="prefill kernel: the library's choice, the two-CTA tensor-core "
                          "kernel (GDN_FLAG_PAIR) or the fp32 CUDA-core kernel")

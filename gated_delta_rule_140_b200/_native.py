@@ -19,7 +19,7 @@ GDN_OK, GDN_ERR_INVALID, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
     GDN_ERR_DEVICE_INPUT = range(6)
 GDN_BF16, GDN_FP32 = 0, 1
 GDN_DECAY_SCALAR, GDN_DECAY_CHANNEL = 0, 1
-GDN_FLAG_CUDA_CORES, GDN_FLAG_PAIR = 1, 2
+GDN_FLAG_CUDA_CORES, GDN_FLAG_PAIR, GDN_FLAG_ONE_CTA = 1, 2, 4
 
 
 class GdnError(RuntimeError):
@@ -114,13 +114,15 @@ def _check_dev(name, t, dtype=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
-def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False, pair=False) -> Dims:
+def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False, pair=False,
+                 one_cta=False) -> Dims:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     return Dims(B, T, H, dk, dv, (len(cu_seqlens) - 1) if cu_seqlens is not None else B,
                 _dtype_code(q.dtype),
                 GDN_DECAY_CHANNEL if log_alpha.dim() == 4 else GDN_DECAY_SCALAR,
-                (GDN_FLAG_CUDA_CORES if cuda_cores else 0) | (GDN_FLAG_PAIR if pair else 0))
+                (GDN_FLAG_CUDA_CORES if cuda_cores else 0) | (GDN_FLAG_PAIR if pair else 0)
+                | (GDN_FLAG_ONE_CTA if one_cta else 0))
 
 
 def chunk_fwd_path(dims: Dims) -> str:
@@ -170,10 +172,11 @@ def _workspace_for(device, stream) -> Workspace:
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
               output_final_state=True, o=None, final_state=None, workspace: Workspace = None,
-              cuda_cores=False, pair=False, stream=None):
+              cuda_cores=False, pair=False, one_cta=False, stream=None):
     """Chunkwise prefill (gdn_chunk_fwd).  Returns (o, final_state or None).
-    ``cuda_cores`` / ``pair`` select the fp32 CUDA-core or the two-CTA
-    tensor-core kernel instead of the default (GDN_FLAG_*)."""
+    ``cuda_cores`` / ``pair`` / ``one_cta`` select the fp32 CUDA-core, the
+    two-CTA or the single-CTA tensor-core kernel instead of the default
+    (GDN_FLAG_*)."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_dev(name, t, q.dtype)
@@ -181,7 +184,7 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
     _check_dev("beta", beta, torch.float32)
     _check_dev("initial_state", initial_state, torch.float32)
     _check_dev("cu_seqlens", cu_seqlens, torch.int32)
-    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair)
+    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair, one_cta)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:

@@ -21,7 +21,11 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     if (d->d_k <= 0 || d->d_v <= 0) return GDN_ERR_INVALID;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
         return GDN_ERR_UNSUPPORTED;
-    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR)) != 0) return GDN_ERR_INVALID;
+    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA)) != 0)
+        return GDN_ERR_INVALID;
+    if ((d->flags & GDN_FLAG_ONE_CTA) &&
+        ((d->flags & GDN_FLAG_PAIR) || d->decay == GDN_DECAY_CHANNEL))
+        return GDN_ERR_INVALID;
     if (prefill && d->n_seqs < 0) return GDN_ERR_INVALID;
     // every index the kernels form must fit in 63 bits; keep the token axis sane
     if ((long long)d->B * d->T * d->H * (d->d_k > d->d_v ? d->d_k : d->d_v) > (1LL << 40))
@@ -34,10 +38,18 @@ enum class Path { kPair, kOneCta, kCudaCores };
 // The prefill kernel a call runs.  bf16, d_k = d_v = 128: GDN the single-CTA
 // tensor-core kernel (the two-CTA one with GDN_FLAG_PAIR), KDA the two-CTA
 // kernel; every other case, or GDN_FLAG_CUDA_CORES, the fp32 CUDA-core kernel.
+constexpr long long kPairMinMeanTokens = 8192;
+
 Path select_path(const gdn_dims &d) {
     if ((d.flags & GDN_FLAG_CUDA_CORES) || !gdn::chunk_pair_supported(d)) return Path::kCudaCores;
     if (d.decay == GDN_DECAY_CHANNEL || (d.flags & GDN_FLAG_PAIR)) return Path::kPair;
-    return gdn::chunk_tc_supported(d) ? Path::kOneCta : Path::kCudaCores;
+    if (!gdn::chunk_tc_supported(d)) return Path::kCudaCores;
+    if (d.flags & GDN_FLAG_ONE_CTA) return Path::kOneCta;
+    // scalar decay: the two-CTA kernel's steady state is faster per chunk, its
+    // start-up (the first chunk through both SMs) longer; it pays from sequences
+    // of about 128 chunks on
+    const long long seqs = d.n_seqs > 0 ? d.n_seqs : (d.B > 0 ? d.B : 1);
+    return (long long)d.B * d.T >= kPairMinMeanTokens * seqs ? Path::kPair : Path::kOneCta;
 }
 
 int prefill_seqs(const gdn_dims &d, const int32_t *cu_seqlens) {

@@ -45,7 +45,7 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
         // the two-CTA kernel's ring does not fit: GDN runs the single-CTA
         // tensor-core kernel, KDA the CUDA-core kernel
         d.flags &= ~GDN_FLAG_PAIR;
-        if (d.decay == GDN_DECAY_CHANNEL) d.flags |= GDN_FLAG_CUDA_CORES;
+        d.flags |= d.decay == GDN_DECAY_CHANNEL ? GDN_FLAG_CUDA_CORES : GDN_FLAG_ONE_CTA;
         need = gdn_chunk_fwd_workspace_size(&d);
     }
     if (need > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_UNSUPPORTED;

@@ -61,9 +61,13 @@ typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
 
 /* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: for bf16
- * with d_k = d_v = 128 the single-CTA tensor-core kernel (scalar decay) or the
- * two-CTA tensor-core kernel (channel decay), the fp32 CUDA-core kernel
- * otherwise.  GDN_FLAG_PAIR selects the two-CTA kernel for scalar decay too.
+ * with d_k = d_v = 128 the two-CTA tensor-core kernel for channel decay, and for
+ * scalar decay the two-CTA kernel when the sequences hold 8192 tokens or more on
+ * average (B * T / n_seqs; its steady state is faster, its start-up longer) and
+ * the single-CTA tensor-core kernel otherwise; the fp32 CUDA-core kernel for
+ * every other shape.  GDN_FLAG_PAIR selects the two-CTA kernel and
+ * GDN_FLAG_ONE_CTA the single-CTA kernel for scalar decay (the two are
+ * exclusive; GDN_FLAG_ONE_CTA with channel decay is GDN_ERR_INVALID).
  * The two-CTA kernel runs one thread-block cluster per sequence and head: one
  * SM computes the chunk-local matrices, the other runs the sequential state
  * pass; it needs a larger workspace (see below).  For channel decay it covers
@@ -72,7 +76,7 @@ typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
  * recomputed by the CUDA-core kernel (exact for any decay) within the same
  * call.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use
  * the flags to compare the device paths. */
-enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2 };
+enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4 };
 
 typedef struct {
     int32_t B;       /* batch (1 for a packed batch)                           */
@@ -89,7 +93,7 @@ typedef struct {
 /* Bytes of device workspace gdn_chunk_fwd needs for `dims` (always >= 256),
  * on the current device.  The first 256 bytes hold the sticky error word;
  * zero them once before the workspace's first use (gdn_workspace_init).  The
- * two-CTA tensor-core kernel adds a ring of two 64 KiB slots for each SM index
+ * two-CTA tensor-core kernel adds a ring of four 64 KiB slots for each SM index
  * of the device (2 x its SM count), through which the chunk-local SM hands each
  * chunk's matrices to the state SM; it is written before it is read and needs
  * no initialisation.  The other kernels need only the header.  Returns 0 for

@@ -56,6 +56,30 @@ def test_workspace_size(L):
     assert L.gdn_chunk_fwd_workspace_size(None) == 0
 
 
+def test_prefill_kernel_choice(L):
+    """The library's choice for bf16 d = 128: channel decay on the two-CTA
+    kernel; scalar decay on the two-CTA kernel from a mean sequence length of
+    8192 tokens (B * T / n_seqs), on the single-CTA kernel below; the flags
+    override it, GDN_FLAG_ONE_CTA only for scalar decay and not with
+    GDN_FLAG_PAIR; other shapes on CUDA cores."""
+    path = lambda **kw: nat.chunk_fwd_path(_dims(**kw))
+    assert path(B=4, T=4096, n_seqs=4) == "tensor_core"
+    assert path(B=4, T=8192, n_seqs=4) == "tensor_core_pair"
+    assert path(B=1, T=65536, n_seqs=1) == "tensor_core_pair"
+    assert path(B=1, T=65536, n_seqs=16) == "tensor_core"         # packed, mean 4096
+    assert path(B=1, T=65536, n_seqs=8) == "tensor_core_pair"     # packed, mean 8192
+    assert path(B=1, T=65536, n_seqs=1, flags=nat.GDN_FLAG_ONE_CTA) == "tensor_core"
+    assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_PAIR) == "tensor_core_pair"
+    assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_CUDA_CORES) == "cuda_core"
+    assert path(decay=nat.GDN_DECAY_CHANNEL) == "tensor_core_pair"
+    assert path(dtype=nat.GDN_FP32) == "cuda_core"
+    assert path(d_k=64, d_v=64, flags=nat.GDN_FLAG_ONE_CTA) == "cuda_core"
+    for flags, decay in ((nat.GDN_FLAG_ONE_CTA | nat.GDN_FLAG_PAIR, nat.GDN_DECAY_SCALAR),
+                         (nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_CHANNEL), (8, nat.GDN_DECAY_SCALAR)):
+        with pytest.raises(nat.GdnError):
+            path(flags=flags, decay=decay)
+
+
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
 
 

@@ -168,6 +168,24 @@ def test_kda_pair_kernel_and_out_of_range_decay_is_redone_exactly(cuda_ok):
     assert rel_err(s, ref_s.cpu().numpy()) < 1e-2
 
 
+def test_kda_log_alpha_4_byte_aligned_gives_identical_results(cuda_ok):
+    """The ABI asks 4-byte alignment of log alpha; the KDA gate pass loads channel
+    pairs as float2 when the pointer allows and one float at a time otherwise.
+    Both read the same values and sum them in the same order: bit-identical."""
+    x = prefill_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                       alpha_shift=3.0, seed=32, init_std=0.05)
+    d = to_dev(x)
+    o1, s1 = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"])
+    n = d["log_alpha"].numel()
+    buf = torch.empty(n + 1, dtype=torch.float32, device="cuda")
+    la = buf[1:].view(d["log_alpha"].shape)
+    la.copy_(d["log_alpha"])
+    assert la.data_ptr() % 8 == 4
+    o2, s2 = chunk_fwd(d["q"], d["k"], d["v"], la, d["beta"], d["initial_state"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+
+
 @pytest.mark.parametrize("decay", ["scalar", "channel"])
 @pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 129, 640])
 def test_pair_kernel_chunk_counts(cuda_ok, T, decay):
