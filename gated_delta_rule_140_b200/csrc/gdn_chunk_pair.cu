@@ -190,25 +190,38 @@ __device__ __forceinline__ void unpack8(uint4 u, float *x) {
 // Decay of 32 entries (columns 32*half ..) of row r of a C x C product,
 // e^{g_r - g_s} for s < r (strict) or s <= r.  rq = r / 32 is uniform per warp,
 // so each warp takes one of three branches: the diagonal 32x32 block (exact
-// exponentials, g_r - g_s <= 0 wherever kept, masked elsewhere), a block
-// strictly below it (factored at the 16-block boundary: e^{g_r - g_e} e^{g_e - g_s},
-// both factors <= 1), or a block above it (not called: nothing to keep).
+// exponentials inside the row's own 16-block, g_r - g_s <= 0 wherever kept,
+// masked elsewhere; factored across the 16-block boundary), a block strictly
+// below it (factored at the 16-block boundary: e^{g_r - g_e} e^{g_e - g_s}, both
+// factors <= 1), or a block above it (not called: nothing to keep).
 __device__ __forceinline__ void decay_row(float *x, int r, int rq, int half, const float *gr,
                                           bool incl) {
     const float *g = gr + GR_G;
     if (rq == half) {
+        // exact exponentials inside the row's own 16-block only (16 per thread);
+        // the earlier 16-block of the diagonal 32-block is factored like the
+        // blocks below, the later one is masked
+        const int rb = r >> 4;  // 2 half or 2 half + 1: differs between the half-warps
         const float g_r = g[r];
+        float d[16];
 #pragma unroll
-        for (int j4 = 0; j4 < 8; ++j4) {
-            const float4 gs = *reinterpret_cast<const float4 *>(g + 32 * half + 4 * j4);
-            const float gv[4] = {gs.x, gs.y, gs.z, gs.w};
+        for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 gs = *reinterpret_cast<const float4 *>(g + 16 * rb + 4 * e4);
+            d[4 * e4] = __expf(g_r - gs.x);
+            d[4 * e4 + 1] = __expf(g_r - gs.y);
+            d[4 * e4 + 2] = __expf(g_r - gs.z);
+            d[4 * e4 + 3] = __expf(g_r - gs.w);
+        }
+        const bool upper = rb & 1;  // the row's block is the second of the 32-block
+        const float f0 = gr[GR_ROWF + 4 * r + 2 * half];  // to the first block's end
+        const float *colf = gr + GR_COLF + 32 * half;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int j = 4 * j4 + e, s = 32 * half + j;
-                const bool keep = incl ? (s <= r) : (s < r);
-                const float d = __expf(g_r - gv[e]);
-                x[j] = keep ? x[j] * d : 0.f;
-            }
+        for (int j = 0; j < 32; ++j) {
+            const int s = 32 * half + j;
+            const bool keep = incl ? (s <= r) : (s < r);
+            const bool own = (j >> 4) == (upper ? 1 : 0);
+            const float fac = own ? d[j & 15] : f0 * colf[j];
+            x[j] = keep ? x[j] * fac : 0.f;
         }
     } else {
         const float *colf = gr + GR_COLF + 32 * half;
