@@ -62,7 +62,7 @@ typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
 
 /* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: for bf16
  * with d_k = d_v = 128 the two-CTA tensor-core kernel for channel decay, and for
- * scalar decay the two-CTA kernel when the sequences hold 8192 tokens or more on
+ * scalar decay the two-CTA kernel when the sequences hold 2048 tokens or more on
  * average (B * T / n_seqs; its steady state is faster, its start-up longer) and
  * the single-CTA tensor-core kernel otherwise; the fp32 CUDA-core kernel for
  * every other shape.  GDN_FLAG_PAIR selects the two-CTA kernel and

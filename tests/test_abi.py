@@ -59,15 +59,16 @@ def test_workspace_size(L):
 def test_prefill_kernel_choice(L):
     """The library's choice for bf16 d = 128: channel decay on the two-CTA
     kernel; scalar decay on the two-CTA kernel from a mean sequence length of
-    8192 tokens (B * T / n_seqs), on the single-CTA kernel below; the flags
+    2048 tokens (B * T / n_seqs), on the single-CTA kernel below; the flags
     override it, GDN_FLAG_ONE_CTA only for scalar decay and not with
     GDN_FLAG_PAIR; other shapes on CUDA cores."""
     path = lambda **kw: nat.chunk_fwd_path(_dims(**kw))
-    assert path(B=4, T=4096, n_seqs=4) == "tensor_core"
-    assert path(B=4, T=8192, n_seqs=4) == "tensor_core_pair"
+    assert path(B=4, T=1024, n_seqs=4) == "tensor_core"
+    assert path(B=4, T=2048, n_seqs=4) == "tensor_core_pair"
+    assert path(B=4, T=4096, n_seqs=4) == "tensor_core_pair"
     assert path(B=1, T=65536, n_seqs=1) == "tensor_core_pair"
-    assert path(B=1, T=65536, n_seqs=16) == "tensor_core"         # packed, mean 4096
-    assert path(B=1, T=65536, n_seqs=8) == "tensor_core_pair"     # packed, mean 8192
+    assert path(B=1, T=65536, n_seqs=64) == "tensor_core"         # packed, mean 1024
+    assert path(B=1, T=65536, n_seqs=32) == "tensor_core_pair"    # packed, mean 2048
     assert path(B=1, T=65536, n_seqs=1, flags=nat.GDN_FLAG_ONE_CTA) == "tensor_core"
     assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_PAIR) == "tensor_core_pair"
     assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_CUDA_CORES) == "cuda_core"

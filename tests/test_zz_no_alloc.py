@@ -47,9 +47,9 @@ def _problems():
     # entry point runs the CUDA-core kernel; compared with the default path
     c = prefill_inputs(2, 150, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
                        alpha_shift=3.0, seed=43, init_std=0.05)
-    # GDN bf16 d = 128 with a sequence of 8192+ tokens: the default is the two-CTA
+    # GDN bf16 d = 128 with a sequence of 2048+ tokens: the default is the two-CTA
     # kernel, whose ring does not fit; the entry point runs the single-CTA kernel
-    e = prefill_inputs(1, 8192 + 37, 2, 128, 128, dtype=torch.bfloat16, seed=44, init_std=0.05)
+    e = prefill_inputs(1, 2048 + 37, 2, 128, 128, dtype=torch.bfloat16, seed=44, init_std=0.05)
     return [(a, torch.bfloat16), (b, torch.float32), (c, torch.bfloat16), (e, torch.bfloat16)]
 
 
