@@ -271,7 +271,9 @@ struct Waiter {
         *abort = 1;
         st_peer_u32(peer_abort, 1u);
     }
-    // Bounded wait for a phase completed inside this CTA (MMA commits, TMA).
+    // Bounded wait for a phase completed inside this CTA (MMA commits, TMA).  No
+    // sleep between polls: mbarrier.try_wait suspends the thread for a while
+    // itself, and a sleep only delays the waiter (measured: 2.5% of the prefill).
     __device__ __forceinline__ bool wait(uint64_t *bar, uint32_t parity) const {
         if (mbar_try_wait(bar, parity)) return true;
         const long long t0 = clock64();
@@ -281,7 +283,6 @@ struct Waiter {
                 raise();
                 return false;
             }
-            __nanosleep(32);
         }
         return true;
     }
@@ -295,7 +296,6 @@ struct Waiter {
                 raise();
                 return false;
             }
-            __nanosleep(32);
         }
         return true;
     }

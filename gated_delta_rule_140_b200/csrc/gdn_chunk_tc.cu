@@ -133,7 +133,8 @@ __device__ __forceinline__ void decay_row(float *x, int r, int rb, int half, con
 
 // Called by one thread per group; the others sleep on a named barrier, so the
 // polling does not compete with the busy warps for issue slots or the shared
-// memory pipe.
+// memory pipe.  No sleep between polls: mbarrier.try_wait suspends the thread
+// for a while itself, and a sleep only delays the waiter (measured).
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
@@ -143,7 +144,6 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
             *abort = 1;
             return false;
         }
-        __nanosleep(64);
     }
     return true;
 }
