@@ -956,17 +956,25 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
             tc_fence_after();
             // GDN: lw 0,1 P T_bg -> X2, lw 4,5 R -> P's tile (P is consumed);
-            // KDA: lw 0,1 R -> X2
-            if (lq < 2 && (!CH || lhalf == 0)) {
+            // KDA: R -> X2, columns 32 lhalf .. by lw 0,1 and 4,5
+            if (lq < 2) {
                 const int r = 32 * lq + lane;
-                uint8_t *dst = pzt + (lhalf == 0 ? PZ_X2 : PZ_P);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
+                if constexpr (CH) {
                     float x[32];
-                    tmem_load<32>(tm_ab + lane_off + 64 * lhalf + 32 * hh, x);
+                    tmem_load<32>(tm_ab + lane_off + 32 * lhalf, x);
 #pragma unroll
                     for (int j = 0; j < 4; ++j)
-                        *reinterpret_cast<uint4 *>(dst + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
+                        *reinterpret_cast<uint4 *>(pzt + PZ_X2 + sw128(r, 4 * lhalf + j)) = pack8(x + 8 * j);
+                } else {
+                    uint8_t *dst = pzt + (lhalf == 0 ? PZ_X2 : PZ_P);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float x[32];
+                        tmem_load<32>(tm_ab + lane_off + 64 * lhalf + 32 * hh, x);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(dst + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
+                    }
                 }
             }
             fence_proxy_async_smem();
