@@ -27,20 +27,22 @@
 // fourth chunk.  GDN: two groups of 8 warps work on two chunks at once (even / odd
 // chunks); KDA: group 1 runs the next chunk's gate pass while group 0 runs the
 // products of this one.  Per chunk:
-//   GDN: D = [K; Q] K^T, then A and P take the decay e^{g_r-g_s} (block
-//        factored, exact inside the diagonal 32x32 blocks); T_bg = T_b
-//        diag(e^{g}) so that W = T_bg K; [P T_bg | R] = P [T_bg | T_b];
-//        [W; P W] = [T_bg; P T_bg] K.
-//   KDA (one group, the other's shared memory holding its extra operands):
-//        each 16-token row block i takes the reference m_i = 16 i + 7 (its
-//        middle token): K and Q become KD, QD = . e^{G - G_{m(r)}} in place, and
-//        B_i = K[0, 16(i+1)) . e^{G_{m_i} - G}, so that D_i = [KD; QD] B_i^T
-//        (four MMAs, N = 16, 32, 48, 64) holds the decayed A and P of block i
-//        (masks only); every factor is within 8 tokens' decay of 1.  Then
+//   GDN: D = [K; Q] K^T, then A and P take the decay e^{g_r-g_s} (exact inside
+//        each row's own 16-token block, factored at the 16-token block
+//        boundaries elsewhere, both factors <= 1); T_bg = T_b diag(e^{g}) so
+//        that W = T_bg K; [P T_bg | R] = P [T_bg | T_b]; [W; P W] = [T_bg; P T_bg] K.
+//   KDA (group 1, one chunk ahead): each 16-token row block i takes the
+//        reference m_i = 16 i + 7 (its middle token): K and Q become KD, QD =
+//        . e^{G - G_{m(r)}} in place, and B_i = K[0, 16(i+1)) . e^{G_{m_i} - G},
+//        stacked into one 160-row operand, so that one MMA (N = 160) gives
+//        D_i = [KD; QD] B_i^T, the decayed A and P of block i (masks only);
+//        every factor is within 8 tokens' decay of 1.  Then (group 0)
 //        R = P T_b, Kg = KD . e^{G_{m(r)}}, [W; P W] = [T_b; R] Kg, and
 //        Qh = QD . e^{G_{m(r)}} - P W.
 // T comes from blocked forward substitution in fp32 (tf32 MMAs for the
-// off-diagonal blocks), computed in place of A.
+// off-diagonal blocks), computed in place of A.  The ring tiles leave shared
+// memory by bulk copy in two groups (what the group's next chunk rewrites early
+// first), and the state CTA learns of a slot through a cluster mbarrier.
 // Rank 1 ("state" CTA) holds S (fp32, registers) for all 128 value channels as
 // two independent halves of 64, each with its own chain of warps, loads each
 // chunk's ring slot and V tile (bulk copy + TMA), and per chunk and half
