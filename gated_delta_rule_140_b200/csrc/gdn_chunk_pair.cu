@@ -918,7 +918,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             // ---- T_b (and GDN's T_bg) in bf16, K-major rows r, columns s ----------
 #pragma unroll
             for (int q2 = 0; q2 < 2; ++q2) {
-                const int idx = gtid + 256 * q2, r = idx >> 3, j = idx & 7;
+                const int idx = gtid + 256 * q2, r = idx & 63, j = idx >> 6;  // lanes: rows
                 float tv[8], bv[8], tb[8];
                 *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(AT + r * LDA + 8 * j);
                 *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(AT + r * LDA + 8 * j + 4);

@@ -504,7 +504,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             // ---- T diag(beta) and T diag(beta gamma) in bf16 (K-major, s cols) ---
 #pragma unroll
             for (int it = 0; it < 2; ++it) {
-                const int idx = tid + kLocal * it, r = idx >> 3, j = idx & 7;
+                const int idx = tid + kLocal * it, r = idx & 63, j = idx >> 6;  // lanes: rows
                 float tv[8], bv[8], gv[8], tb[8], tg[8];
                 *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j);
                 *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(TF + r * LDA + 8 * j + 4);
