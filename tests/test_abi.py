@@ -65,6 +65,8 @@ def test_prefill_kernel_choice(L):
     path = lambda **kw: nat.chunk_fwd_path(_dims(**kw))
     assert path(B=4, T=1024, n_seqs=4) == "tensor_core"
     assert path(B=4, T=2048, n_seqs=4) == "tensor_core_pair"
+    assert path(B=4, T=2048, n_seqs=0) == "tensor_core_pair"      # n_seqs 0: B sequences
+    assert path(B=4, T=2047, n_seqs=0) == "tensor_core"
     assert path(B=4, T=4096, n_seqs=4) == "tensor_core_pair"
     assert path(B=1, T=65536, n_seqs=1) == "tensor_core_pair"
     assert path(B=1, T=65536, n_seqs=64) == "tensor_core"         # packed, mean 1024
