@@ -19,7 +19,7 @@ GDN_OK, GDN_ERR_INVALID, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
     GDN_ERR_DEVICE_INPUT = range(6)
 GDN_BF16, GDN_FP32 = 0, 1
 GDN_DECAY_SCALAR, GDN_DECAY_CHANNEL = 0, 1
-GDN_FLAG_CUDA_CORES, GDN_FLAG_PAIR, GDN_FLAG_ONE_CTA = 1, 2, 4
+GDN_FLAG_CUDA_CORES, GDN_FLAG_PAIR, GDN_FLAG_ONE_CTA, GDN_FLAG_POOL = 1, 2, 4, 8
 
 
 class GdnError(RuntimeError):
@@ -55,6 +55,8 @@ def lib():
     L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
     L.gdn_recurrent_step.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp]
     L.gdn_recurrent_step.restype = ctypes.c_int
+    L.gdn_noalloc_status.argtypes = [vp]
+    L.gdn_noalloc_status.restype = ctypes.c_int
     L.gdn_workspace_init.argtypes = [vp, sz, vp]
     L.gdn_workspace_init.restype = ctypes.c_int
     L.gdn_workspace_status.argtypes = [vp, vp]
@@ -115,19 +117,19 @@ def _check_dev(name, t, dtype=None):
 
 
 def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False, pair=False,
-                 one_cta=False) -> Dims:
+                 one_cta=False, pool=False) -> Dims:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     return Dims(B, T, H, dk, dv, (len(cu_seqlens) - 1) if cu_seqlens is not None else B,
                 _dtype_code(q.dtype),
                 GDN_DECAY_CHANNEL if log_alpha.dim() == 4 else GDN_DECAY_SCALAR,
                 (GDN_FLAG_CUDA_CORES if cuda_cores else 0) | (GDN_FLAG_PAIR if pair else 0)
-                | (GDN_FLAG_ONE_CTA if one_cta else 0))
+                | (GDN_FLAG_ONE_CTA if one_cta else 0) | (GDN_FLAG_POOL if pool else 0))
 
 
 def chunk_fwd_path(dims: Dims) -> str:
-    """"tensor_core_pair", "tensor_core" or "cuda_core": the prefill kernel
-    gdn_chunk_fwd selects."""
+    """"tensor_core_pool", "tensor_core_pair", "tensor_core" or "cuda_core": the
+    prefill kernel gdn_chunk_fwd selects."""
     r = lib().gdn_chunk_fwd_path(ctypes.byref(dims))
     if r is None:
         raise GdnError(GDN_ERR_INVALID, "gdn_chunk_fwd_path")
@@ -155,9 +157,29 @@ class Workspace:
         return self.buf
 
     def status(self, stream=None) -> int:
+        """Synchronise the stream, read and clear the sticky device error word."""
         if self.buf is None:
             return GDN_OK
         return int(lib().gdn_workspace_status(_ptr(self.buf), _stream(stream)))
+
+    def set_wait_limit(self, cycles: int, stream=None):
+        """Test-only: the second header word replaces the tensor-core kernels'
+        bounded-wait limit on data waits (0 restores the default)."""
+        import torch
+        if self.buf is None:
+            self.get(256, stream)
+        word = torch.tensor([int(cycles)], dtype=torch.int32).view(torch.uint8)
+        self.buf[4:8].copy_(word.to(self.buf.device), non_blocking=False)
+
+
+def noalloc_status(stream=None) -> int:
+    """gdn_noalloc_status: the device errors of the last gdn_chunk_fwd_noalloc call."""
+    return int(lib().gdn_noalloc_status(_stream(stream)))
+
+
+def _raise_on_status(st: int, where: str):
+    if st != GDN_OK:
+        raise GdnError(st, where)
 
 
 _default_ws = {}
@@ -172,11 +194,15 @@ def _workspace_for(device, stream) -> Workspace:
 
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
               output_final_state=True, o=None, final_state=None, workspace: Workspace = None,
-              cuda_cores=False, pair=False, one_cta=False, stream=None):
+              cuda_cores=False, pair=False, one_cta=False, pool=False, check=False,
+              stream=None):
     """Chunkwise prefill (gdn_chunk_fwd).  Returns (o, final_state or None).
-    ``cuda_cores`` / ``pair`` / ``one_cta`` select the fp32 CUDA-core, the
-    two-CTA or the single-CTA tensor-core kernel instead of the default
-    (GDN_FLAG_*)."""
+    ``cuda_cores`` / ``pool`` / ``pair`` / ``one_cta`` select the fp32
+    CUDA-core kernel or one of the tensor-core kernels instead of the default
+    (GDN_FLAG_*).  With ``check`` the call synchronises the stream afterwards
+    and raises GdnError if the device recorded an error (bad cu_seqlens
+    contents, an expired bounded wait, an internal error): without it such
+    errors stay in the workspace's sticky word until ``workspace.status()``."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_dev(name, t, q.dtype)
@@ -184,7 +210,7 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
     _check_dev("beta", beta, torch.float32)
     _check_dev("initial_state", initial_state, torch.float32)
     _check_dev("cu_seqlens", cu_seqlens, torch.int32)
-    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair, one_cta)
+    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair, one_cta, pool)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:
@@ -199,13 +225,17 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
                              _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_chunk_fwd")
+    if check:
+        _raise_on_status(ws.status(stream), "gdn_chunk_fwd (device)")
     return o, final_state
 
 
-def recurrent_step(q, k, v, log_alpha, beta, state, *, o=None, stream=None):
+def recurrent_step(q, k, v, log_alpha, beta, state, *, o=None, check=False, stream=None):
     """One decode step (gdn_recurrent_step); ``state`` [N,H,dv,dk] fp32 is updated
     in place.  q, k [N,H,dk]; v [N,H,dv]; log_alpha [N,H] or [N,H,dk]; beta [N,H].
-    Returns o [N,H,dv]."""
+    Returns o [N,H,dv].  The decode kernel has no device-detected errors (no
+    waits, no offsets); with ``check`` the call synchronises the stream and
+    raises if the launch or the kernel failed."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_dev(name, t, q.dtype)
@@ -223,4 +253,10 @@ def recurrent_step(q, k, v, log_alpha, beta, state, *, o=None, stream=None):
                                   _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_recurrent_step")
+    if check:
+        s = stream if stream is not None else torch.cuda.current_stream()
+        try:
+            s.synchronize()
+        except RuntimeError as e:
+            raise GdnError(GDN_ERR_CUDA, f"gdn_recurrent_step (device): {e}") from e
     return o

@@ -21,10 +21,11 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     if (d->d_k <= 0 || d->d_v <= 0) return GDN_ERR_INVALID;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
         return GDN_ERR_UNSUPPORTED;
-    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA)) != 0)
+    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA | GDN_FLAG_POOL)) != 0)
         return GDN_ERR_INVALID;
-    if ((d->flags & GDN_FLAG_ONE_CTA) &&
-        ((d->flags & GDN_FLAG_PAIR) || d->decay == GDN_DECAY_CHANNEL))
+    const int kernel_flags = d->flags & (GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA | GDN_FLAG_POOL);
+    if (kernel_flags & (kernel_flags - 1)) return GDN_ERR_INVALID;  // at most one
+    if ((d->flags & (GDN_FLAG_ONE_CTA | GDN_FLAG_POOL)) && d->decay == GDN_DECAY_CHANNEL)
         return GDN_ERR_INVALID;
     if (prefill && d->n_seqs < 0) return GDN_ERR_INVALID;
     // every index the kernels form must fit in 63 bits; keep the token axis sane
@@ -33,7 +34,7 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     return GDN_OK;
 }
 
-enum class Path { kPair, kOneCta, kCudaCores };
+enum class Path { kPool, kPair, kOneCta, kCudaCores };
 
 // The prefill kernel a call runs.  bf16, d_k = d_v = 128: GDN the single-CTA
 // tensor-core kernel (the two-CTA one with GDN_FLAG_PAIR), KDA the two-CTA
@@ -45,6 +46,8 @@ Path select_path(const gdn_dims &d) {
     if (d.decay == GDN_DECAY_CHANNEL || (d.flags & GDN_FLAG_PAIR)) return Path::kPair;
     if (!gdn::chunk_tc_supported(d)) return Path::kCudaCores;
     if (d.flags & GDN_FLAG_ONE_CTA) return Path::kOneCta;
+    if ((d.flags & GDN_FLAG_POOL) && gdn::chunk_pool_supported(d))
+        return Path::kPool;
     // scalar decay: the two-CTA kernel's steady state is faster per chunk, its
     // start-up (the first chunk through both SMs) longer; measured, it is ahead
     // from sequences of about 32 chunks on (16 chunks: 3% behind; 64: 3% ahead;
@@ -64,7 +67,8 @@ extern "C" {
 size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims) {
     if (check_dims(dims, true) != GDN_OK) return 0;
     const Path p = select_path(*dims);
-    size_t extra = p == Path::kPair     ? gdn::chunk_pair_scratch_bytes(*dims)
+    size_t extra = p == Path::kPool     ? gdn::chunk_pool_scratch_bytes(*dims)
+                   : p == Path::kPair   ? gdn::chunk_pair_scratch_bytes(*dims)
                    : p == Path::kOneCta ? gdn::chunk_tc_scratch_bytes(*dims)
                                         : 0;
     return gdn::kWorkspaceHeader + ((extra + 255) & ~size_t(255));
@@ -110,7 +114,8 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
     int launches = 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const Path p = select_path(d);
-    cudaError_t e = p == Path::kPair     ? gdn::launch_chunk_pair(a, s, &launches)
+    cudaError_t e = p == Path::kPool     ? gdn::launch_chunk_pool(a, s, &launches)
+                    : p == Path::kPair   ? gdn::launch_chunk_pair(a, s, &launches)
                     : p == Path::kOneCta ? gdn::launch_chunk_tc(a, s, &launches)
                                          : gdn::launch_chunk_simt(a, s, &launches);
     g_launches.fetch_add(launches, std::memory_order_relaxed);
@@ -168,6 +173,7 @@ gdn_status gdn_workspace_status(void *workspace, gdn_stream_t stream) {
 const char *gdn_chunk_fwd_path(const gdn_dims *dims) {
     if (check_dims(dims, true) != GDN_OK) return nullptr;
     switch (select_path(*dims)) {
+        case Path::kPool: return "tensor_core_pool";
         case Path::kPair: return "tensor_core_pair";
         case Path::kOneCta: return "tensor_core";
         default: return "cuda_core";

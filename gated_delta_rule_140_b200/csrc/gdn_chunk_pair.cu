@@ -60,6 +60,8 @@
 // read).  Every wait is bounded: on expiry the CTA records kErrTimeout, raises
 // the abort flag of both CTAs, drains what it issued and leaves through the
 // final cluster barrier.
+#include <mutex>
+
 #include "gdn_internal.cuh"
 #include "sm100.cuh"
 
@@ -71,7 +73,7 @@ using namespace sm100;
 constexpr int C = kChunk;  // 64
 constexpr int DK = 128, DV = 128;
 constexpr int kThreads = 512;
-constexpr long long kWaitLimit = 1LL << 31;  // SM cycles (~1 s)
+constexpr long long kWaitLimit = kDefaultWaitLimit;  // drains after an abort
 constexpr int LDA = 68;                      // fp32 row stride of A / T
 constexpr float kMaxNegLogDecay = 80.f;      // e^{80} < bf16 and fp32 max
 
@@ -269,6 +271,7 @@ __device__ __forceinline__ void invert_diag16(float *AT, int o, int j) {
 struct Waiter {
     volatile int *abort;
     uint32_t peer_abort;  // shared::cluster address of the peer's abort flag
+    long long limit;      // SM cycles before a data wait gives up
     __device__ __forceinline__ void raise() const {
         *abort = 1;
         st_peer_u32(peer_abort, 1u);
@@ -281,7 +284,7 @@ struct Waiter {
         const long long t0 = clock64();
         while (!mbar_try_wait(bar, parity)) {
             if (*abort) return false;
-            if (clock64() - t0 > kWaitLimit) {
+            if (clock64() - t0 > limit) {
                 raise();
                 return false;
             }
@@ -294,7 +297,7 @@ struct Waiter {
         const long long t0 = clock64();
         while (!mbar_try_wait_cluster(bar, parity)) {
             if (*abort) return false;
-            if (clock64() - t0 > kWaitLimit) {
+            if (clock64() - t0 > limit) {
                 raise();
                 return false;
             }
@@ -367,7 +370,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const int slot = *reinterpret_cast<volatile int *>(cm + CM_SLOT);
-    const Waiter wt{abort_flag, map_peer(sbase + OFF_COMMON + CM_ABORT, peer)};
+    const Waiter wt{abort_flag, map_peer(sbase + OFF_COMMON + CM_ABORT, peer), data_wait_limit(a.err)};
     if (slot < 0) {
         if (tid == 0) {
             atomicOr(a.err, kErrInternal);
@@ -1311,11 +1314,33 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 }
 
 // ------------------------------------------------------------------- host --
+// %nsmid: an upper bound of %smid on this device (which need not equal the SM
+// count, nor the SM ids be contiguous).
+__device__ int g_nsmid;
+__global__ void nsmid_probe_kernel() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nsmid;" : "=r"(r));
+    g_nsmid = (int)r;
+}
+
+// Ring slots: one per possible SM id, from %nsmid read once per device (the
+// first call on a device launches a one-thread kernel on the legacy default
+// stream and waits for it, so that call should come before any stream capture).
 int ring_slots_for_device() {
-    int dev = 0, nsm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    return 2 * nsm;  // SM ids are below this on every part this kernel runs on
+    constexpr int kMaxDevices = 64;
+    static std::mutex mu;
+    static int slots[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (slots[dev] == 0) {
+        int n = 0;
+        nsmid_probe_kernel<<<1, 1>>>();
+        if (cudaGetLastError() != cudaSuccess) return 0;
+        if (cudaMemcpyFromSymbol(&n, g_nsmid, sizeof(int)) != cudaSuccess || n <= 0) return 0;
+        slots[dev] = n;
+    }
+    return slots[dev];
 }
 
 size_t ring_bytes(int slots) { return (size_t)slots * NRING * RING_STRIDE; }

@@ -1,0 +1,1397 @@
+// gdn_chunk_pool.cu -- chunkwise gated delta rule prefill on the tensor cores
+// with the chunk-local work spread over a pool of SMs and the sequential state
+// pass on dedicated "chain" SMs: one persistent CTA per SM, bf16 inputs,
+// d_k = d_v = 128, scalar decay (Gated DeltaNet).
+//
+// Chunkwise form (FG2-GDN paper, section 3.6: WY representation, UT
+// transform, inter-chunk state propagation; Gated Delta Networks page,
+// section 3.3, for the cumulative decay g_r inside a chunk), C = 64 tokens,
+// g_r = sum_{t<=r} log alpha_t, gamma_r = e^{g_r}:
+//
+//   A_rs = beta_r e^{g_r-g_s} k_r.k_s (s < r),   T = (I + A)^{-1}
+//   P_rs = e^{g_r-g_s} q_r.k_s (s <= r),          T_b = T diag(beta)
+//   W = T_b diag(gamma) K,  U = T_b V,  Kt_r = e^{g_C-g_r} k_r
+//   V' = U - W S^T,  S <- e^{g_C} S + V'^T Kt,  o = (gamma.Q) S^T + P V'.
+//
+// Regrouped so that the sequential chain is ONE product per chunk:
+//   S <- e^{g_C} S + V^T Z + S G,    Z = T_b^T Kt (C x d_k),  G = -W^T Kt (d_k x d_k)
+//   o^T = S Qh^T + V^T R^T,          Qh = gamma.Q - P W,  R = P T_b
+// (V'^T Kt = U^T Kt - S W^T Kt; o = (gamma.Q - P W) S^T + P T_b V).
+//
+// Roles (blockIdx.x < nch: chain CTA b; otherwise a local CTA of the pool):
+//  * Local CTAs take chunk tasks in a fixed global order (round by round, and
+//    inside a round chunk-major over the round's chains; local CTA c takes
+//    tasks c, c + nloc, c + 2 nloc, ...).  Two groups of 8 warps work on
+//    alternate tasks of the CTA, with three raw K/Q tile buffers between them.
+//    Per task: [K;Q] K^T on the tensor cores; A and P with the decay (exact
+//    exponentials inside each row's own 16-token block, factored at the block
+//    boundaries elsewhere, both factors <= 1); T by blocked forward
+//    substitution (fp32 16x16 diagonal blocks, tf32 MMAs above them);
+//    [P T_bg | R] = P [T_bg | T_b]; [W; P W] = [T_bg; P T_bg] K; then -W, Qh and
+//    Kt.  The tiles T_b, -W, Kt, Qh, R (64 KB, bf16, in the layouts the chain
+//    CTA's MMAs read) and e^{g_C} go by bulk copy into a ring slot in global
+//    memory (chain CTA b, slot m % 4), L2-resident; a release store of the
+//    slot's tag hands it over.
+//  * Chain CTA b owns the chains b, b + nch, ... one after another, S (fp32)
+//    in registers of 8 warps (thread = value row j, 64 key columns).  Per
+//    chunk: a loader thread bulk-loads the slot and TMA-loads the V tile into
+//    one of two stages; X = Kt^T [T_b | -W] (one M=128, N=192 MMA) gives Z^T and
+//    G^T, which 4 warps write back as bf16 operands; D_S = V^T Z (issued ahead)
+//    and then the chain product D_S += S G; the 8 state warps update
+//    S <- e^{g_C} S + D_S and write it back as the bf16 operand of the next
+//    chunk; D_O = V^T R^T + S Qh^T = o^T, which 4 warps write out.
+//
+// The hand-offs through global memory: ready[b][slot] holds the tag of the
+// (round, chunk) written there; cons[b] the chain CTA's progress (round,
+// chunks consumed), which a local CTA waits for before it rewrites a slot.
+// All CTAs are co-resident (cooperative launch, one CTA per SM).  Every wait is
+// bounded: on expiry a CTA records kErrTimeout, raises the grid-wide abort
+// word, drains what it issued and returns.
+#include <algorithm>
+#include <cstdlib>
+#include <mutex>
+
+#include "gdn_internal.cuh"
+#include "sm100.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+
+constexpr int C = kChunk;  // 64
+constexpr int DK = 128, DV = 128;
+constexpr int kThreads = 512;                      // 16 warps
+constexpr long long kWaitLimit = kDefaultWaitLimit;  // drains after an abort
+constexpr int LDA = 68;                            // fp32 row stride of A / T
+constexpr int NR = 6;                              // ring slots per chain CTA
+
+// ---- ring slot (global) and chain-CTA stage (shared) layouts, bytes ----------
+// slot:  [T_b | -W0 | -W1 | Kt0 | Kt1] (5 x 8 KB) [Qh0 | Qh1 | R] (3 x 8 KB) [e^{g_C} x128]
+constexpr uint32_t RG_TB = 0, RG_MW = 8192, RG_KT = 24576, RG_QH = 40960, RG_R = 57344,
+                   RG_DEC = 65536, RG_PART1 = 40960, RG_PART2 = 65536 + 512 - 40960;
+constexpr uint32_t RING_STRIDE = 66560;
+// stage: the slot's first part at 0 (overlaid by Z^T at 0 and G^T = Y at 16 KB once
+// X is formed), its second part at CS_QH, then V (TMA, two 64-wide halves)
+constexpr uint32_t CS_TB = 0, CS_MW = 8192, CS_KT = 24576, CS_ZT = 0, CS_Y = 16384;
+constexpr uint32_t CS_QH = 49152, CS_R = 65536, CS_DEC = 73728, CS_V = 74752;
+constexpr uint32_t CS_STAGE = 91136;
+constexpr uint32_t CS_S = 2 * CS_STAGE;  // S bf16, K-major rows j, 2 atoms of 16 KB
+constexpr uint32_t STAGE_TX = RG_PART1 + RG_PART2 + 2 * 8192;
+static_assert(CS_QH + RG_PART2 == CS_DEC + 512 && CS_DEC + 512 <= CS_V &&
+              CS_V + 16384 <= CS_STAGE && CS_Y + 32768 <= CS_QH, "chain stage layout");
+
+// ---- local-CTA layout (GDN) -------------------------------------------------
+// three raw tile buffers [K0 | Q0 | K1 | Q1] shared by the two groups (task k in
+// buffer k % 3; Kt replaces K in place), then per group [P | X1 | X2 | X3]
+// (X1 = T_bg, X2 = P T_bg, X3 = T_b), A and then T in place (fp32 [64][LDA]),
+// and two gate-row buffers.
+constexpr uint32_t L_RAW_AC = 16384, RAW_BYTES = 32768;
+constexpr uint32_t PZ_P = 0, PZ_X1 = 8192, PZ_X2 = 16384, PZ_X3 = 24576, PZT_BYTES = 32768;
+constexpr uint32_t AT_BYTES = 64 * LDA * 4;
+constexpr uint32_t GATES_STRIDE = 3072;
+constexpr uint32_t L_G0 = 3 * RAW_BYTES;
+constexpr uint32_t L_PZT = 0, L_AT = PZT_BYTES, L_GATES = L_AT + AT_BYTES;
+constexpr uint32_t L_GSZ = L_GATES + 2 * GATES_STRIDE;
+static_assert(L_GATES % 1024 == 0 && L_GSZ % 1024 == 0, "local group layout");
+// gate rows (floats): g beta beta*gamma colf rowf[4] kh gamma, and e^{g_C} x128
+constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
+              GR_GAM = 576, GR_DEC = 640;
+
+// ---- bookkeeping (same offset in both roles) --------------------------------
+constexpr uint32_t OFF_COMMON = CS_S + 32768;  // 215040
+static_assert(L_G0 + 2 * L_GSZ <= OFF_COMMON, "local shared memory layout");
+constexpr uint32_t CM_ABORT = 0, CM_TMEM = 8, CM_ISSUED = 16, CM_BARS = 64;
+constexpr int NBARS = 24;
+// local CTAs of packed batches: the descriptors of their first kDescCache tasks
+constexpr int kDescCache = 512;
+constexpr uint32_t OFF_DESC = OFF_COMMON + 256;
+static_assert(CM_BARS + NBARS * 8 <= 256, "bookkeeping");
+constexpr uint32_t SMEM_USED = OFF_DESC + kDescCache * 16;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+// chain-CTA mbarriers
+constexpr int CB_FULL = 0, CB_SFREE = 2, CB_XFULL = 4, CB_DSFULL = 5, CB_DSFREE = 7,
+              CB_OFULL = 9, CB_OFREE = 10, CB_AISS = 11, CB_DRAIN = 13;
+static_assert(1 + NR <= 8, "flag words per chain CTA");
+// local-CTA mbarriers (TMA: one per raw buffer)
+constexpr int LB_TMA = 0, LB_L = 3, LB_OFFSET = 5, LB_DRAIN = 6;
+
+// TMEM columns.  Chain: D_S (2 x 128), X (192), D_O (64).  Local: per group 192.
+constexpr uint32_t TM_DS = 0, TM_X = 256, TM_O = 448;
+constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_GROUP = 192;
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);    // [K;Q] K^T
+constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, true);  // [P;0][T_bg|T_b], [X1;X2] K
+constexpr uint32_t ID_X = idesc_bf16(128, 192, true, true);      // Kt^T [T_b | -W]
+constexpr uint32_t ID_VZ = idesc_bf16(128, 128, true, false);    // V^T Z
+constexpr uint32_t ID_SG = idesc_bf16(128, 128, false, false);   // S G
+constexpr uint32_t ID_VR = idesc_bf16(128, 64, true, false);     // V^T R^T
+constexpr uint32_t ID_SQ = idesc_bf16(128, 64, false, false);    // S Qh^T
+
+// named barriers
+constexpr int BAR_UPD = 5, BAR_CONV = 6;  // chain: state warps, X warps (local: 1-4)
+
+struct PoolArgs {
+    uint8_t *ring;         // nch x NR slots of RING_STRIDE bytes
+    uint64_t *flags;       // per chain CTA 8 words: cons, ready[NR], pad
+    uint32_t *gabort;      // grid-wide abort word
+    const long long *rbase;  // packed batches: task offset of each round [nrounds + 1]
+    int nrounds;
+    long long ntask;       // task count (fixed rows)
+    int nch;               // chain CTAs
+    int nck;               // chunks per chain (fixed rows)
+};
+
+// One chunk task: token range, head, its chain CTA and ring tag.
+struct Task {
+    long long t0;
+    int L;      // tokens (0: an empty padding task)
+    int h;
+    int b;      // chain CTA
+    int m;      // chunk index in its chain
+    int rho;    // round
+};
+
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ uint64_t ready_tag(int rho, int m) {
+    return ((uint64_t)(rho + 1) << 32) | (uint32_t)(m + 1);
+}
+// cons[b] after chunk m of round rho has been read out of its slot
+__device__ __forceinline__ uint64_t cons_after(int rho, int m, int nck) {
+    return m + 1 == nck ? ((uint64_t)(rho + 1) << 32) : (((uint64_t)rho << 32) | (uint32_t)(m + 1));
+}
+// cons[b] a local CTA needs before it writes chunk m of round rho into its slot
+// (the slot's previous occupant, chunk m - NR or a chunk of an earlier round,
+// has been read)
+__device__ __forceinline__ uint64_t cons_needed(int rho, int m) {
+    return ((uint64_t)rho << 32) | (uint32_t)(m >= NR ? m - NR + 1 : 0);
+}
+
+// Task t of the global order.  Chains are x = rho * nch + b (sequence x / H,
+// head x % H); round rho holds the chains of its nch chain CTAs and lists their
+// chunks chunk-major, every chain padded to the round's longest (padding tasks
+// are empty).  Fixed rows: closed form.  Packed batches: the round offsets
+// (rbase, written by the schedule kernel) are searched.
+__device__ __forceinline__ Task task_of(const PrefillArgs &a, const PoolArgs &p, long long t) {
+    Task k;
+    const long long nchains = (long long)a.n_seqs * a.H;
+    int rho;
+    long long rem;
+    if (p.rbase == nullptr) {
+        const long long per_round = (long long)p.nch * p.nck;
+        rho = (int)(t / per_round);
+        rem = t - (long long)rho * per_round;
+    } else {
+        int lo = 0, hi = p.nrounds - 1;  // last round with rbase <= t
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.rbase[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        rho = lo;
+        rem = t - p.rbase[rho];
+    }
+    const int nround = (int)min((long long)p.nch, nchains - (long long)rho * p.nch);
+    const int m = (int)(rem / nround), i = (int)(rem % nround);
+    const long long x = (long long)rho * p.nch + i;
+    const int n = (int)(x / a.H);
+    long long tb, te;
+    seq_range(a, n, &tb, &te);
+    k.h = (int)(x % a.H);
+    k.t0 = tb + (long long)m * C;
+    const long long rest = te - k.t0;
+    k.L = rest <= 0 ? 0 : (rest < C ? (int)rest : C);
+    k.b = i;
+    k.m = m;
+    k.rho = rho;
+    return k;
+}
+
+__device__ __forceinline__ int4 pack_task(const Task &k) {
+    return make_int4((int)k.t0, k.h | (k.L << 16), k.b | (k.rho << 8), k.m);
+}
+__device__ __forceinline__ Task unpack_task(int4 d) {
+    Task k;
+    k.t0 = (long long)(uint32_t)d.x;
+    k.h = d.y & 0xffff;
+    k.L = d.y >> 16;
+    k.b = d.z & 0xff;
+    k.rho = (int)((uint32_t)d.z >> 8);
+    k.m = d.w;
+    return k;
+}
+
+__device__ __forceinline__ uint4 pack8(const float *x) {
+    uint4 u;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(x[0], x[1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(x[2], x[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(x[4], x[5]);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(x[6], x[7]);
+    u.x = *reinterpret_cast<uint32_t *>(&h0);
+    u.y = *reinterpret_cast<uint32_t *>(&h1);
+    u.z = *reinterpret_cast<uint32_t *>(&h2);
+    u.w = *reinterpret_cast<uint32_t *>(&h3);
+    return u;
+}
+__device__ __forceinline__ void unpack8(uint4 u, float *x) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&t);
+}
+
+// Decay of 32 entries (columns 32*half ..) of row r of a C x C product,
+// e^{g_r - g_s} for s < r (strict) or s <= r.  rq = r / 32 is uniform per warp:
+// the diagonal 32x32 block takes exact exponentials inside the row's own
+// 16-block (g_r - g_s <= 0 wherever kept) and is factored across the 16-block
+// boundary; a block strictly below it is factored at the 16-block boundary:
+// e^{g_r - g_e} e^{g_e - g_s}, both factors <= 1.
+__device__ __forceinline__ void decay_row(float *x, int r, int rq, int half, const float *gr,
+                                          bool incl) {
+    const float *g = gr + GR_G;
+    if (rq == half) {
+        const int rb = r >> 4;
+        const float g_r = g[r];
+        float d[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 gs = *reinterpret_cast<const float4 *>(g + 16 * rb + 4 * e4);
+            d[4 * e4] = __expf(g_r - gs.x);
+            d[4 * e4 + 1] = __expf(g_r - gs.y);
+            d[4 * e4 + 2] = __expf(g_r - gs.z);
+            d[4 * e4 + 3] = __expf(g_r - gs.w);
+        }
+        const bool upper = rb & 1;
+        const float f0 = gr[GR_ROWF + 4 * r + 2 * half];
+        const float *colf = gr + GR_COLF + 32 * half;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int s = 32 * half + j;
+            const bool keep = incl ? (s <= r) : (s < r);
+            const bool own = (j >> 4) == (upper ? 1 : 0);
+            const float fac = own ? d[j & 15] : f0 * colf[j];
+            x[j] = keep ? x[j] * fac : 0.f;
+        }
+    } else {
+        const float *colf = gr + GR_COLF + 32 * half;
+        const float f0 = gr[GR_ROWF + 4 * r + 2 * half], f1 = gr[GR_ROWF + 4 * r + 2 * half + 1];
+#pragma unroll
+        for (int j4 = 0; j4 < 8; ++j4) {
+            const float4 c = *reinterpret_cast<const float4 *>(colf + 4 * j4);
+            const float f = j4 < 4 ? f0 : f1;
+            const float2 lo = __fmul2_rn(make_float2(x[4 * j4], x[4 * j4 + 1]), make_float2(f * c.x, f * c.y));
+            const float2 hi = __fmul2_rn(make_float2(x[4 * j4 + 2], x[4 * j4 + 3]), make_float2(f * c.z, f * c.w));
+            x[4 * j4] = lo.x; x[4 * j4 + 1] = lo.y; x[4 * j4 + 2] = hi.x; x[4 * j4 + 3] = hi.y;
+        }
+    }
+}
+
+// Bounded waits.  `abort` is this CTA's flag, `gabort` the grid's: a wait on
+// another CTA's progress gives up when either is raised or after `limit` cycles.
+struct Waiter {
+    volatile int *abort;
+    volatile uint32_t *gabort;
+    uint32_t *err;
+    long long limit;
+    __device__ __forceinline__ void raise() const {
+        *abort = 1;
+        atomicExch(const_cast<uint32_t *>(gabort), 1u);
+        atomicOr(err, kErrTimeout);
+    }
+    // a phase completed inside this CTA (MMA commits, TMA, other warps)
+    __device__ __forceinline__ bool wait(uint64_t *bar, uint32_t parity) const {
+        if (mbar_try_wait(bar, parity)) return true;
+        const long long t0 = clock64();
+        while (!mbar_try_wait(bar, parity)) {
+            if (*abort) return false;
+            if (clock64() - t0 > limit) {
+                raise();
+                return false;
+            }
+        }
+        return true;
+    }
+    // one lane waits, the warp gets the answer
+    __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int lane) const {
+        bool ok = true;
+        if (lane == 0) ok = wait(bar, parity);
+        return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    // a global word written by another CTA reaches `want` (== or >=)
+    __device__ __forceinline__ bool wait_global(const uint64_t *p, uint64_t want, bool exact) const {
+        uint64_t v = ld_acquire_u64(p);
+        if (exact ? v == want : v >= want) return true;
+        const long long t0 = clock64();
+        for (;;) {
+            __nanosleep(64);
+            v = ld_acquire_u64(p);
+            if (exact ? v == want : v >= want) return true;
+            if (*abort || *gabort) {
+                *abort = 1;
+                return false;
+            }
+            if (clock64() - t0 > limit) {
+                raise();
+                return false;
+            }
+        }
+    }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    uint8_t *cm = sm + OFF_COMMON;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(cm + CM_ABORT);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(cm + CM_BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cm + CM_TMEM);
+    int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // [3] loads issued per buffer / stage
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool chain_role = (int)blockIdx.x < p.nch;
+    const int H = a.H;
+
+    if (warp == 0) tmem_alloc(tmem_slot, TMEM_COLS);
+    if (tid == 0) {
+        for (int i = 0; i < NBARS; ++i) {
+            uint32_t cnt = 1;
+            if (chain_role && (i == CB_DSFREE || i == CB_DSFREE + 1)) cnt = 8;
+            if (chain_role && i == CB_OFREE) cnt = 4;
+            mbar_init(bars + i, cnt);
+        }
+        fence_mbar_init();
+        *abort_flag = 0;
+        issued[0] = issued[1] = issued[2] = 0;
+        if (chain_role) {
+            tma_prefetch_desc(&tm_v);
+        } else {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Waiter wt{abort_flag, p.gabort, a.err, data_wait_limit(a.err)};
+
+    if (!chain_role) {
+        // ============================ local CTA ============================
+        const int c = (int)blockIdx.x - p.nch, nloc = (int)gridDim.x - p.nch;
+        const long long ntask_all = p.rbase ? p.rbase[p.nrounds] : p.ntask;
+        const int ntask = c < ntask_all ? (int)((ntask_all - c + nloc - 1) / nloc) : 0;
+        auto gid = [&](int k) -> long long { return (long long)c + (long long)k * nloc; };
+        // packed batches: this CTA's first task descriptors, looked up once
+        int4 *sdesc = reinterpret_cast<int4 *>(sm + OFF_DESC);
+        if (p.rbase) {
+            for (int k = tid; k < min(ntask, kDescCache); k += kThreads)
+                sdesc[k] = pack_task(task_of(a, p, gid(k)));
+            __syncthreads();
+        }
+        auto task = [&](int k) -> Task {
+            if (p.rbase && k < kDescCache) return unpack_task(sdesc[k]);
+            return task_of(a, p, gid(k));
+        };
+        if (warp < 16) {
+            const int g = warp >> 3, lw = warp & 7, lq = warp & 3, lhalf = lw >> 2;
+            const int gtid = tid & 255;
+            const int BAR_G = 1 + g, BAR_INV = 3 + g;
+            uint8_t *grp = sm + L_G0 + g * L_GSZ;
+            const uint32_t gbase = sbase + L_G0 + g * L_GSZ;
+            auto raw_of = [&](int k) -> uint8_t * { return sm + (k % 3) * RAW_BYTES; };
+            auto tma_phase = [&](int k) -> uint32_t { return (uint32_t)((k / 3) & 1); };
+            uint8_t *pzt = grp + L_PZT;
+            float *AT = reinterpret_cast<float *>(grp + L_AT);
+            uint64_t *bar_l = bars + LB_L + g;
+            const uint32_t tm_kq = tmem + g * TM_GROUP + TM_KQ, tm_ab = tmem + g * TM_GROUP + TM_AB;
+            const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
+            const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);                // [P; X1]
+            const uint64_t d_x1b = desc_sw128(gbase + L_PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 | X3
+            const uint64_t d_x1x2 = desc_sw128(gbase + L_PZT + PZ_X1, 16, 1024);            // [X1; X2]
+            uint32_t bl_wait = 0;
+            const bool issuer = gtid == 0;       // MMAs
+            const bool storer = gtid == 7 * 32;  // tile loads, ring stores and the hand-off
+            bool pend = false;                   // storer: a task's ring stores are in flight
+            uint64_t *pend_flag = nullptr;
+            uint64_t pend_tag = 0;
+            auto hand_over = [&]() {
+                bulk_wait_all();
+                fence_proxy_async_global();
+                st_release_u64(pend_flag, pend_tag);
+                pend = false;
+            };
+            // raw tiles of task k into buffer k % 3 (an empty task completes the
+            // buffer's phase with a plain arrive)
+            auto issue_tma = [&](int k) {
+                const Task tk = task(k);
+                uint8_t *dst = raw_of(k);
+                uint64_t *bt = bars + LB_TMA + (k % 3);
+                if (tk.L == 0) {
+                    mbar_arrive(bt);
+                } else {
+                    fence_proxy_async_smem();
+                    mbar_arrive_expect_tx(bt, 4 * 8192);
+                    tma_load_3d(dst + 0, &tm_k, 0, tk.h, (int)tk.t0, bt);
+                    tma_load_3d(dst + 8192, &tm_q, 0, tk.h, (int)tk.t0, bt);
+                    tma_load_3d(dst + L_RAW_AC, &tm_k, 64, tk.h, (int)tk.t0, bt);
+                    tma_load_3d(dst + L_RAW_AC + 8192, &tm_q, 64, tk.h, (int)tk.t0, bt);
+                }
+                atomicAdd(issued + (k % 3), 1);
+            };
+            auto gate_rows = [&](int k) {
+                return reinterpret_cast<float *>(grp + L_GATES + ((k >> 1) & 1) * GATES_STRIDE);
+            };
+            // gates of the group's task after next, prefetched in warp lw 4's registers
+            float nla0 = 0.f, nla1 = 0.f, nbe0 = 0.f, nbe1 = 0.f;
+            auto load_gates = [&](int k) {
+                const Task tk = task(k);
+                const int r0 = 2 * lane, r1 = 2 * lane + 1;
+                nla0 = r0 < tk.L ? a.log_alpha[(tk.t0 + r0) * H + tk.h] : 0.f;
+                nla1 = r1 < tk.L ? a.log_alpha[(tk.t0 + r1) * H + tk.h] : 0.f;
+                nbe0 = r0 < tk.L ? a.beta[(tk.t0 + r0) * H + tk.h] : 0.f;
+                nbe1 = r1 < tk.L ? a.beta[(tk.t0 + r1) * H + tk.h] : 0.f;
+            };
+            // gate rows of task kk (one warp): cumulative log decay, beta, the
+            // factored block decays, kh and gamma, e^{g_C} for every channel
+            auto compute_gates = [&](int kk) {
+                float *gr = gate_rows(kk);
+                const int r0 = 2 * lane, r1 = 2 * lane + 1;
+                const float la0 = nla0, la1 = nla1, be0 = nbe0, be1 = nbe1;
+                if (kk + 2 < ntask) load_gates(kk + 2);
+                float incl = la0 + la1;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, incl, off);
+                    if (lane >= off) incl += y;
+                }
+                const float g1 = incl, g0 = incl - la1;
+                float gend[4];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) gend[b] = __shfl_sync(0xffffffffu, incl, 8 * b + 7);
+                const float gC = gend[3];
+                const int blk = r0 >> 4;
+                const float e0 = __expf(g0), e1 = __expf(g1);
+                const float c0 = __expf(gend[blk] - g0), c1 = __expf(gend[blk] - g1);
+                const float k0 = __expf(gC - g0), k1 = __expf(gC - g1);
+                float f0[3], f1[3];
+#pragma unroll
+                for (int b = 0; b < 3; ++b) {
+                    f0[b] = __expf(fminf(g0 - gend[b], 0.f));
+                    f1[b] = __expf(fminf(g1 - gend[b], 0.f));
+                }
+                gr[GR_G + r0] = g0; gr[GR_G + r1] = g1;
+                gr[GR_B + r0] = be0; gr[GR_B + r1] = be1;
+                gr[GR_BG + r0] = be0 * e0; gr[GR_BG + r1] = be1 * e1;
+                gr[GR_COLF + r0] = c0; gr[GR_COLF + r1] = c1;
+                gr[GR_KH + r0] = k0; gr[GR_KH + r1] = k1;
+                gr[GR_GAM + r0] = e0; gr[GR_GAM + r1] = e1;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) {
+                    gr[GR_ROWF + 4 * r0 + b] = b < blk ? f0[b < 3 ? b : 0] : 0.f;
+                    gr[GR_ROWF + 4 * r1 + b] = b < blk ? f1[b < 3 ? b : 0] : 0.f;
+                }
+                const float dC = __expf(gC);
+                *reinterpret_cast<float4 *>(gr + GR_DEC + 4 * lane) = make_float4(dC, dC, dC, dC);
+            };
+
+            // the first tasks' tiles (one per raw buffer) and the group's first gates
+            if (storer && g < ntask) issue_tma(g);
+            if (storer && g == 0 && 2 < ntask) issue_tma(2);
+            if (lw == 4 && g < ntask) {
+                load_gates(g);
+                compute_gates(g);
+            }
+            // group 1 starts half a task after group 0, so that the two groups'
+            // CUDA-core phases tend to overlap the other's MMA and load waits
+            bool ok0 = true;
+            if (g == 1 && issuer && ntask >= 2) ok0 = wt.wait(bars + LB_OFFSET, 0);
+            named_bar_or(BAR_G, 256, !ok0);
+
+            for (int k = g; k < ntask; k += 2) {
+                const Task tk = task(k);
+                float *gr = gate_rows(k);
+                uint8_t *rawp = raw_of(k);
+                const uint32_t raw_s = smem_u32(rawp);
+                const uint64_t d_raw = desc_sw128(raw_s, 16, 1024);        // [K;Q], K (K-major)
+                const uint64_t d_kmn = desc_sw128(raw_s, L_RAW_AC, 1024);  // K (MN-major)
+                const int L = tk.L;
+                bool ok = true;
+                // the next-but-two task's tiles into L2 while this one runs
+                if (issuer && k + 3 < ntask) {
+                    const Task t3 = task(k + 3);
+                    if (t3.L > 0) {
+                        tma_prefetch_l2_3d(&tm_k, 0, t3.h, (int)t3.t0);
+                        tma_prefetch_l2_3d(&tm_k, 64, t3.h, (int)t3.t0);
+                        tma_prefetch_l2_3d(&tm_q, 0, t3.h, (int)t3.t0);
+                        tma_prefetch_l2_3d(&tm_q, 64, t3.h, (int)t3.t0);
+                    }
+                }
+                if (issuer) ok = wt.wait(bars + LB_TMA + (k % 3), tma_phase(k));
+                if (L == 0) {
+                    // empty padding task: only the duties other tasks rely on
+                    if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                    if (storer && pend) hand_over();
+                    if (storer && k >= 2 && k + 1 < ntask) issue_tma(k + 1);
+                    if (lw == 4 && k + 2 < ntask) compute_gates(k + 2);
+                    if (g == 0 && k == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
+                    named_bar_sync(BAR_G, 256);
+                    continue;
+                }
+                if (L < C) {
+                    if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                    for (int idx = gtid; idx < (C - L) * 8; idx += 256) {
+                        const uint32_t o = (L + (idx >> 3)) * 128 + (idx & 7) * 16;
+                        const uint4 z = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(rawp + o) = z;
+                        *reinterpret_cast<uint4 *>(rawp + 8192 + o) = z;
+                        *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + o) = z;
+                        *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + 8192 + o) = z;
+                    }
+                    fence_proxy_async_smem();
+                    if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                }
+                // ---- D_kq = [K; Q] K^T (a full task's MMA goes out as soon as its
+                //      tiles are in; an abort is seen at the barrier after it) -------
+                if (issuer && ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t off = ((kk >> 2) * L_RAW_AC + (kk & 3) * 32) >> 4;
+                        mma_bf16(tm_kq, d_raw + off, d_raw + off, ID_KK, kk > 0);
+                    }
+                    mma_commit(bar_l);
+                    ok = wt.wait(bar_l, bl_wait & 1);
+                }
+                ++bl_wait;
+                // the tiles that the A/P phase below rewrites went out first, as
+                // their own bulk group
+                if (storer && pend) bulk_wait_read_but_last();
+                // the raw buffer of this group's previous task (k - 2, read by its
+                // ring stores) takes task k + 1, the other group's next
+                if (storer && k >= 2 && k + 1 < ntask) issue_tma(k + 1);
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                tc_fence_after();
+                // ---- A rows (lanes 0-63) -> fp32 with beta; P rows (lanes 64-127) -> bf16
+                const float *gb = gr + GR_B;
+                if ((lq & 1) >= lhalf) {
+                    float x[32];
+                    tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
+                    if (lq < 2) {
+                        const int r = 32 * lq + lane;
+                        decay_row(x, r, lq, lhalf, gr, false);
+                        const float br = gb[r];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            *reinterpret_cast<float4 *>(AT + r * LDA + 32 * lhalf + j) =
+                                make_float4(br * x[j], br * x[j + 1], br * x[j + 2], br * x[j + 3]);
+                        }
+                    } else {
+                        const int r = 32 * (lq - 2) + lane;
+                        decay_row(x, r, lq - 2, lhalf, gr, true);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(pzt + PZ_P + sw128(r, 4 * lhalf + j)) = pack8(x + 8 * j);
+                    }
+                } else if (lq >= 2) {
+                    // P rows 0-31, columns 32-63 (above the diagonal): zero
+#pragma unroll
+                    for (int j = 4; j < 8; ++j)
+                        *reinterpret_cast<uint4 *>(pzt + PZ_P + sw128(lane, j)) = make_uint4(0, 0, 0, 0);
+                }
+                named_bar_sync(BAR_G, 256);
+                if (g == 0 && k == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
+                // ---- T = (I + A)^{-1} in place of A: lw 0-3; meanwhile lw 4 prepares
+                //      the group's next gates and the storer hands over its last task
+                if (lw >= 4) {
+                    if (storer && pend) hand_over();
+                    if (lw == 4 && k + 2 < ntask) compute_gates(k + 2);
+                } else {
+                    // (1) 16x16 diagonal blocks, right-looking forward substitution;
+                    //     lane j < 16 owns column j
+                    if (lane < 16) {
+                        const int o = 16 * lw, j = lane;
+                        float t[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) t[i] = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                        for (int mm = 0; mm < 15; ++mm) {
+#pragma unroll
+                            for (int i = mm + 1; i < 16; ++i) t[i] -= AT[(o + i) * LDA + o + mm] * t[mm];
+                        }
+                        __syncwarp(0x0000ffffu);
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) AT[(o + i) * LDA + o + j] = t[i];
+                    }
+                    named_bar_sync(BAR_INV, 128);
+                    // (2) 32x32 halves: T_10 = -T_11 (A_10 T_00), T_32 = -T_33 (A_32 T_22)
+                    const int fg = lane >> 2, ft = lane & 3;
+                    const int o = 32 * (lw >> 1), n0 = 8 * (lw & 1);
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t af[4], bf[2];
+                        const int ar = o + 16 + fg, ac = o + 8 * ks + ft;
+                        af[0] = to_tf32(AT[ar * LDA + ac]);
+                        af[1] = to_tf32(AT[(ar + 8) * LDA + ac]);
+                        af[2] = to_tf32(AT[ar * LDA + ac + 4]);
+                        af[3] = to_tf32(AT[(ar + 8) * LDA + ac + 4]);
+                        bf[0] = to_tf32(AT[(o + 8 * ks + ft) * LDA + o + n0 + fg]);
+                        bf[1] = to_tf32(AT[(o + 8 * ks + ft + 4) * LDA + o + n0 + fg]);
+                        mma_tf32_16x8x8(x, af, bf);
+                    }
+                    AT[(o + fg) * LDA + o + 16 + n0 + 2 * ft] = x[0];
+                    AT[(o + fg) * LDA + o + 16 + n0 + 2 * ft + 1] = x[1];
+                    AT[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft] = x[2];
+                    AT[(o + fg + 8) * LDA + o + 16 + n0 + 2 * ft + 1] = x[3];
+                    named_bar_sync(BAR_INV, 128);
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t af[4], bf[2];
+                        const int ar = o + 16 + fg, ac = o + 16 + 8 * ks + ft;
+                        af[0] = to_tf32(AT[ar * LDA + ac]);
+                        af[1] = to_tf32(AT[(ar + 8) * LDA + ac]);
+                        af[2] = to_tf32(AT[ar * LDA + ac + 4]);
+                        af[3] = to_tf32(AT[(ar + 8) * LDA + ac + 4]);
+                        bf[0] = to_tf32(AT[(o + 8 * ks + ft) * LDA + o + 16 + n0 + fg]);
+                        bf[1] = to_tf32(AT[(o + 8 * ks + ft + 4) * LDA + o + 16 + n0 + fg]);
+                        mma_tf32_16x8x8(y, af, bf);
+                    }
+                    AT[(o + 16 + fg) * LDA + o + n0 + 2 * ft] = -y[0];
+                    AT[(o + 16 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[1];
+                    AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
+                    AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
+                }
+                if (named_bar_or(BAR_G, 256, *abort_flag)) break;
+                // (3) T_{H1,H0} = -T_{H1} (A_{H1,H0} T_{H0}), 32x32 blocks; warp lw owns
+                //     output rows 16(lw/4).., columns 8(lw%4)..
+                {
+                    const int fg = lane >> 2, ft = lane & 3;
+                    const int m0 = 16 * (lw >> 2), n0 = 8 * (lw & 3);
+                    float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        uint32_t af[4], bf[2];
+                        const int ar = 32 + m0 + fg, ac = 8 * ks + ft;
+                        af[0] = to_tf32(AT[ar * LDA + ac]);
+                        af[1] = to_tf32(AT[(ar + 8) * LDA + ac]);
+                        af[2] = to_tf32(AT[ar * LDA + ac + 4]);
+                        af[3] = to_tf32(AT[(ar + 8) * LDA + ac + 4]);
+                        const int br = 8 * ks + ft, bc = n0 + fg;
+                        bf[0] = to_tf32(br >= bc ? AT[br * LDA + bc] : 0.f);
+                        bf[1] = to_tf32(br + 4 >= bc ? AT[(br + 4) * LDA + bc] : 0.f);
+                        mma_tf32_16x8x8(x, af, bf);
+                    }
+                    AT[(m0 + fg) * LDA + 32 + n0 + 2 * ft] = x[0];
+                    AT[(m0 + fg) * LDA + 32 + n0 + 2 * ft + 1] = x[1];
+                    AT[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft] = x[2];
+                    AT[(m0 + fg + 8) * LDA + 32 + n0 + 2 * ft + 1] = x[3];
+                    named_bar_sync(BAR_G, 256);
+                    float y[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        uint32_t af[4], bf[2];
+                        const int r = m0 + fg, kc = 8 * ks + ft;
+                        af[0] = to_tf32(kc <= r ? AT[(32 + r) * LDA + 32 + kc] : 0.f);
+                        af[1] = to_tf32(kc <= r + 8 ? AT[(40 + r) * LDA + 32 + kc] : 0.f);
+                        af[2] = to_tf32(kc + 4 <= r ? AT[(32 + r) * LDA + 36 + kc] : 0.f);
+                        af[3] = to_tf32(kc + 4 <= r + 8 ? AT[(40 + r) * LDA + 36 + kc] : 0.f);
+                        bf[0] = to_tf32(AT[(8 * ks + ft) * LDA + 32 + n0 + fg]);
+                        bf[1] = to_tf32(AT[(8 * ks + ft + 4) * LDA + 32 + n0 + fg]);
+                        mma_tf32_16x8x8(y, af, bf);
+                    }
+                    AT[(32 + m0 + fg) * LDA + n0 + 2 * ft] = -y[0];
+                    AT[(32 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[1];
+                    AT[(40 + m0 + fg) * LDA + n0 + 2 * ft] = -y[2];
+                    AT[(40 + m0 + fg) * LDA + n0 + 2 * ft + 1] = -y[3];
+                }
+                named_bar_sync(BAR_G, 256);
+                // ---- T_b and T_bg in bf16, rows r, columns s (consecutive threads on
+                //      consecutive rows: no bank conflict on T's rows, beta broadcast)
+#pragma unroll
+                for (int q2 = 0; q2 < 2; ++q2) {
+                    const int idx = gtid + 256 * q2, r = idx & 63, j = idx >> 6;
+                    float tv[8], bv[8], tb[8], gv[8], tg[8];
+                    *reinterpret_cast<float4 *>(tv) = *reinterpret_cast<const float4 *>(AT + r * LDA + 8 * j);
+                    *reinterpret_cast<float4 *>(tv + 4) = *reinterpret_cast<const float4 *>(AT + r * LDA + 8 * j + 4);
+                    *reinterpret_cast<float4 *>(bv) = *reinterpret_cast<const float4 *>(gb + 8 * j);
+                    *reinterpret_cast<float4 *>(bv + 4) = *reinterpret_cast<const float4 *>(gb + 8 * j + 4);
+                    *reinterpret_cast<float4 *>(gv) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j);
+                    *reinterpret_cast<float4 *>(gv + 4) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j + 4);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int s2 = 8 * j + e;
+                        tv[e] = s2 < r ? tv[e] : (s2 == r ? 1.f : 0.f);
+                        tb[e] = tv[e] * bv[e];
+                        tg[e] = tv[e] * gv[e];
+                    }
+                    *reinterpret_cast<uint4 *>(pzt + PZ_X3 + sw128(r, j)) = pack8(tb);
+                    *reinterpret_cast<uint4 *>(pzt + PZ_X1 + sw128(r, j)) = pack8(tg);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(BAR_G, 256);
+                // ---- D_ab = [P; 0] [T_bg | T_b]: rows 0-63 = [P T_bg | R] ----------
+                if (issuer) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_bf16(tm_ab, d_pz + 2 * kk, d_x1b + 128 * kk, ID_N128, kk > 0);
+                    mma_commit(bar_l);
+                    ok = wt.wait(bar_l, bl_wait & 1);
+                }
+                ++bl_wait;
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                tc_fence_after();
+                // lw 0,1: P T_bg -> X2;  lw 4,5: R -> P's tile (P is consumed)
+                if (lq < 2) {
+                    const int r = 32 * lq + lane;
+                    uint8_t *dst = pzt + (lhalf == 0 ? PZ_X2 : PZ_P);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float x[32];
+                        tmem_load<32>(tm_ab + lane_off + 64 * lhalf + 32 * hh, x);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            *reinterpret_cast<uint4 *>(dst + sw128(r, 4 * hh + j)) = pack8(x + 8 * j);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(BAR_G, 256);
+                // ---- D_ab = [T_bg; P T_bg] K: rows 0-63 = W, rows 64-127 = P W -------
+                if (issuer) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_bf16(tm_ab, d_x1x2 + 2 * kk, d_kmn + 128 * kk, ID_N128, kk > 0);
+                    mma_commit(bar_l);
+                    ok = wt.wait(bar_l, bl_wait & 1);
+                }
+                ++bl_wait;
+                if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                tc_fence_after();
+                // ---- -W (lanes 0-63) staged in A/T's space; Qh = gamma Q - P W (lanes
+                //      64-127) staged in X1/X2; Kt = kh . K in place of K.  The raw
+                //      tiles' Q is then free.
+                {
+                    const int r = 32 * (lq & 1) + lane;
+                    const float gam = gr[GR_GAM + r];
+                    uint8_t *wst = grp + L_AT + lhalf * 8192;
+                    uint8_t *qst = pzt + (lhalf ? PZ_X2 : PZ_X1);
+                    const uint8_t *qt = rawp + lhalf * L_RAW_AC + 8192;
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float x[32];
+                        tmem_load<32>(tm_ab + lane_off + 64 * lhalf + 32 * hh, x);
+                        if (lq < 2) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                float w[8];
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) w[e] = -x[8 * j + e];
+                                *reinterpret_cast<uint4 *>(wst + sw128(r, 4 * hh + j)) = pack8(w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const uint32_t o = sw128(r, 4 * hh + j);
+                                float qv[8];
+                                unpack8(*reinterpret_cast<const uint4 *>(qt + o), qv);
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) qv[e] = gam * qv[e] - x[8 * j + e];
+                                *reinterpret_cast<uint4 *>(qst + o) = pack8(qv);
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const int idx = gtid + 256 * q2;
+                        const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
+                        float kv[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)), kv);
+                        const float sc = gr[GR_KH + rr];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) kv[e] *= sc;
+                        *reinterpret_cast<uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)) = pack8(kv);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (named_bar_or(BAR_G, 256, *abort_flag)) break;
+                if (storer) {
+                    // once chain CTA b has read the slot's previous chunk, the tiles and
+                    // e^{g_C} go out by bulk copy; the hand-off follows during the
+                    // group's next task (or after the loop)
+                    uint64_t *fl = p.flags + (size_t)tk.b * 8;
+                    const uint64_t need = cons_needed(tk.rho, tk.m);
+                    if (need == 0 || wt.wait_global(fl, need, false)) {
+                        uint8_t *slot = p.ring + ((size_t)tk.b * NR + (tk.m % NR)) * RING_STRIDE;
+                        // two bulk groups: first what the group's next task rewrites
+                        // early (-W in A's space and Kt in the raw buffer before the
+                        // A/P phase ... R in P's tile), then the rest
+                        const uint8_t *at8 = grp + L_AT;
+                        bulk_store(slot + RG_KT, rawp, 8192);
+                        bulk_store(slot + RG_KT + 8192, rawp + L_RAW_AC, 8192);
+                        bulk_store(slot + RG_MW, at8, 8192);
+                        bulk_store(slot + RG_MW + 8192, at8 + 8192, 8192);
+                        bulk_store(slot + RG_DEC, gr + GR_DEC, 512);
+                        bulk_store(slot + RG_R, pzt + PZ_P, 8192);
+                        bulk_commit();
+                        bulk_store(slot + RG_QH, pzt + PZ_X1, 8192);
+                        bulk_store(slot + RG_QH + 8192, pzt + PZ_X2, 8192);
+                        bulk_store(slot + RG_TB, pzt + PZ_X3, 8192);
+                        bulk_commit();
+                        pend = true;
+                        pend_flag = fl + 1 + (tk.m % NR);
+                        pend_tag = ready_tag(tk.rho, tk.m);
+                    }
+                }
+            }
+            if (storer && pend && !*abort_flag) hand_over();
+            // drain: every bulk copy and MMA this group issued
+            if (storer) bulk_wait_all();
+            if (*abort_flag && issuer) {
+                mma_commit(bars + LB_DRAIN + g);
+                mbar_wait(bars + LB_DRAIN + g, 0, kWaitLimit);
+            }
+        }
+    } else {
+        // ============================ chain CTA ============================
+        const int b = (int)blockIdx.x;
+        const long long nchains = (long long)a.n_seqs * H;
+        // chain (round) rho of this CTA: sequence, head, token range, chunks
+        struct Chain {
+            int n, h, nck;
+            long long t_begin, t_end;
+        };
+        auto chain_of = [&](int rho, Chain *ch) -> bool {
+            const long long x = (long long)rho * p.nch + b;
+            if (x >= nchains) return false;
+            ch->n = (int)(x / H);
+            ch->h = (int)(x % H);
+            seq_range(a, ch->n, &ch->t_begin, &ch->t_end);
+            ch->nck = (int)((ch->t_end - ch->t_begin + C - 1) / C);
+            return true;
+        };
+        const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
+        if (warp < 8) {
+            // ---- state warps: row j = 32 (warp % 4) + lane, key columns 64 ch .. ------
+            const int ch = warp >> 2, j = 32 * (warp & 3) + lane;
+            const bool leader = tid == 0;  // issues the chain and output products
+            uint8_t *stile = sm + CS_S + ch * 16384;
+            const uint64_t d_s = desc_sw128(sbase + CS_S, 16, 1024);
+            float s_reg[64];
+            auto load_s0 = [&](const Chain &cc) {
+                const size_t base = (((size_t)cc.n * H + cc.h) * DV + j) * DK + 64 * ch;
+#pragma unroll
+                for (int e = 0; e < 64; e += 4) {
+                    const float4 v = a.s0 ? *reinterpret_cast<const float4 *>(a.s0 + base + e)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+                    s_reg[e] = v.x; s_reg[e + 1] = v.y; s_reg[e + 2] = v.z; s_reg[e + 3] = v.w;
+                }
+            };
+            auto store_sf = [&](const Chain &cc) {
+                if (!a.s_final) return;
+                const size_t base = (((size_t)cc.n * H + cc.h) * DV + j) * DK + 64 * ch;
+#pragma unroll
+                for (int e = 0; e < 64; e += 4)
+                    *reinterpret_cast<float4 *>(a.s_final + base + e) =
+                        make_float4(s_reg[e], s_reg[e + 1], s_reg[e + 2], s_reg[e + 3]);
+            };
+            auto write_stile = [&]() {
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                    *reinterpret_cast<uint4 *>(stile + sw128(j, cc)) = pack8(s_reg + 8 * cc);
+            };
+            // the next chain with tokens, from round rho on: empty chains get their
+            // final state (the initial one) here; returns false past the last chain
+            auto open_chain = [&](int *rho, Chain *cc) -> bool {
+                for (;; ++*rho) {
+                    if (!chain_of(*rho, cc)) return false;
+                    load_s0(*cc);
+                    if (cc->nck > 0) return true;
+                    store_sf(*cc);
+                }
+            };
+            int rho = 0;
+            Chain cur;
+            bool have = open_chain(&rho, &cur);
+            if (have) write_stile();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(BAR_UPD, 256);
+            uint32_t u = 0;  // chunk counter over this CTA's chains
+            int m = 0;
+            while (have) {
+                const int s = u & 1;
+                const uint32_t sb = sbase + s * CS_STAGE;
+                bool ok = true;
+                if (leader) {
+                    // D_S += S G (after D_S = V^T Z went out); then D_O = V^T R^T + S Qh^T
+                    ok = wt.wait(bars + CB_AISS + s, (u >> 1) & 1);
+                    if (ok) {
+                        tc_fence_after();
+                        const uint64_t d_y = desc_sw128(sb + CS_Y, 16, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < DK / 16; ++kk) {
+                            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                            mma_bf16(tmem + TM_DS + 128 * s, d_s + off, d_y + off, ID_SG, 1);
+                        }
+                        mma_commit(bars + CB_DSFULL + s);
+                    }
+                    if (ok && u >= 1) ok = wt.wait(bars + CB_OFREE, (u - 1) & 1);
+                    if (ok) {
+                        tc_fence_after();
+                        const uint64_t d_v = desc_sw128(sb + CS_V, 8192, 1024);
+                        const uint64_t d_r = desc_sw128(sb + CS_R, 16, 1024);
+                        const uint64_t d_q = desc_sw128(sb + CS_QH, 16, 1024);
+#pragma unroll
+                        for (int kk = 0; kk < C / 16; ++kk)
+                            mma_bf16(tmem + TM_O, d_v + 128 * kk, d_r + 2 * kk, ID_VR, kk > 0);
+#pragma unroll
+                        for (int kk = 0; kk < DK / 16; ++kk) {
+                            const uint32_t off_s = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+                            const uint32_t off_q = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                            mma_bf16(tmem + TM_O, d_s + off_s, d_q + off_q, ID_SQ, 1);
+                        }
+                        mma_commit(bars + CB_OFULL);
+                        mma_commit(bars + CB_SFREE + s);
+                    }
+                }
+                // S <- e^{g_C} S + D_S (columns of this thread's half)
+                const bool okd = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
+                                 wt.warp_wait(bars + CB_DSFULL + s, (u >> 1) & 1, lane);
+                if (okd) {
+                    tc_fence_after();
+                    const float *dec = reinterpret_cast<const float *>(sm + s * CS_STAGE + CS_DEC) + 64 * ch;
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        float ds[16];
+                        tmem_ld16(tmem + TM_DS + 128 * s + 64 * ch + 16 * q4 + lane_q, ds);
+                        tmem_wait_ld16(ds);
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4) {
+                            const float4 dv = *reinterpret_cast<const float4 *>(dec + 16 * q4 + e);
+                            s_reg[16 * q4 + e] = fmaf(dv.x, s_reg[16 * q4 + e], ds[e]);
+                            s_reg[16 * q4 + e + 1] = fmaf(dv.y, s_reg[16 * q4 + e + 1], ds[e + 1]);
+                            s_reg[16 * q4 + e + 2] = fmaf(dv.z, s_reg[16 * q4 + e + 2], ds[e + 2]);
+                            s_reg[16 * q4 + e + 3] = fmaf(dv.w, s_reg[16 * q4 + e + 3], ds[e + 3]);
+                        }
+                    }
+                }
+                // the output product reads the S tile: it must be done before the rewrite
+                const bool oko = okd && wt.warp_wait(bars + CB_OFULL, u & 1, lane);
+                if (oko) {
+                    if (m + 1 == cur.nck) {
+                        store_sf(cur);
+                        ++rho;
+                        have = open_chain(&rho, &cur);
+                        m = 0;
+                    } else {
+                        ++m;
+                    }
+                    if (have) write_stile();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bars + CB_DSFREE + s);
+                if (named_bar_or(BAR_UPD, 256, !oko || *abort_flag)) break;
+                ++u;
+            }
+            if (*abort_flag && leader) {
+                mma_commit(bars + CB_DRAIN);
+                mbar_wait(bars + CB_DRAIN, 0, kWaitLimit);
+            }
+        } else if (warp < 12) {
+            // ---- X warps: X = Kt^T [T_b | -W] -> Z^T, G^T (bf16, K-major rows n);
+            //      then D_S = V^T Z ---------------------------------------------------
+            const int n = 32 * (warp & 3) + lane;
+            const bool leader = warp == 8 && lane == 0;
+            uint32_t u = 0;
+            bool stop = false;
+            for (int rho = 0; !stop; ++rho) {
+                Chain cc;
+                if (!chain_of(rho, &cc)) break;
+                for (int m = 0; m < cc.nck; ++m, ++u) {
+                    const int s = u & 1;
+                    const uint32_t sb = sbase + s * CS_STAGE;
+                    uint8_t *sp = sm + s * CS_STAGE;
+                    bool ok = true;
+                    if (leader) {
+                        ok = wt.wait(bars + CB_FULL + s, (u >> 1) & 1);
+                        if (ok) {
+                            tc_fence_after();
+                            const uint64_t d_kt = desc_sw128(sb + CS_KT, 8192, 1024);
+                            const uint64_t d_tw = desc_sw128(sb + CS_TB, 8192, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < C / 16; ++kk)
+                                mma_bf16(tmem + TM_X, d_kt + 128 * kk, d_tw + 128 * kk, ID_X, kk > 0);
+                            mma_commit(bars + CB_XFULL);
+                        }
+                    }
+                    const bool okx = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
+                                     wt.warp_wait(bars + CB_XFULL, u & 1, lane);
+                    if (okx) {
+                        tc_fence_after();
+#pragma unroll
+                        for (int q3 = 0; q3 < 3; ++q3) {  // columns 64 q3 .. : Z^T, G^T atom 0, 1
+                            float x[64];
+                            tmem_load<64>(tmem + TM_X + 64 * q3 + lane_q, x);
+                            uint8_t *dst = sp + (q3 == 0 ? CS_ZT : CS_Y + (q3 - 1) * 16384);
+#pragma unroll
+                            for (int cc2 = 0; cc2 < 8; ++cc2)
+                                *reinterpret_cast<uint4 *>(dst + sw128(n, cc2)) = pack8(x + 8 * cc2);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    if (named_bar_or(BAR_CONV, 128, !okx || *abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                    if (leader) {
+                        ok = u < 2 || wt.wait(bars + CB_DSFREE + s, ((u >> 1) - 1) & 1);
+                        if (ok) {
+                            tc_fence_after();
+                            const uint64_t d_v = desc_sw128(sb + CS_V, 8192, 1024);
+                            const uint64_t d_z = desc_sw128(sb + CS_ZT, 16, 1024);
+#pragma unroll
+                            for (int kk = 0; kk < C / 16; ++kk)
+                                mma_bf16(tmem + TM_DS + 128 * s, d_v + 128 * kk, d_z + 2 * kk, ID_VZ, kk > 0);
+                            mbar_arrive(bars + CB_AISS + s);
+                        }
+                    }
+                    if (named_bar_or(BAR_CONV, 128, !ok || *abort_flag)) {
+                        stop = true;
+                        break;
+                    }
+                }
+            }
+            if (*abort_flag && leader) {
+                mma_commit(bars + CB_DRAIN + 1);
+                mbar_wait(bars + CB_DRAIN + 1, 0, kWaitLimit);
+            }
+        } else {
+            // ---- output warps: D_O = o^T (lane j = value channel, columns =
+            //      tokens).  Lane 0 of warp 12 is also the loader: the ring slot and
+            //      the V tile of chunk u + 2 go into stage u % 2 once chunk u is out
+            //      of it; the slot is given back (cons) once its loads have landed,
+            //      checked at the loader's next step.
+            const int j = 32 * (warp & 3) + lane;
+            const bool loader = warp == 12 && lane == 0;
+            uint64_t *fl = p.flags + (size_t)b * 8;
+            // loader state: next chunk to load (lu, of chain lrho, chunk lm), and
+            // the cons value waiting for the stage of chunk pend_u to land
+            uint32_t lu = 0;
+            int lrho = 0, lm = 0;
+            Chain lcc;
+            bool lhave = false;
+            long long pend_u = -1;
+            uint64_t pend_val = 0;
+            bool lok = true;
+            auto flush = [&]() {
+                if (pend_u < 0) return;
+                const int s2 = (int)(pend_u & 1);
+                if (lok) lok = wt.wait(bars + CB_FULL + s2, (uint32_t)((pend_u >> 1) & 1));
+                if (lok) st_release_u64(fl, pend_val);
+                pend_u = -1;
+            };
+            // the next chain with chunks from round lrho on (empty ones are passed
+            // at once: their chain CTA has nothing to read)
+            auto lopen = [&]() {
+                for (;; ++lrho) {
+                    lhave = chain_of(lrho, &lcc);
+                    if (!lhave || lcc.nck > 0) return;
+                    flush();
+                    if (lok) st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
+                }
+            };
+            // issue the loads of chunk lu into its stage (the stage is free)
+            auto load_one = [&]() {
+                const int s2 = lu & 1;
+                uint8_t *stage = sm + s2 * CS_STAGE;
+                if (lok) lok = wt.wait_global(fl + 1 + (lm % NR), ready_tag(lrho, lm), true);
+                if (!lok) return;
+                fence_proxy_async_global();
+                const uint8_t *src = p.ring + ((size_t)b * NR + (lm % NR)) * RING_STRIDE;
+                const long long t0 = lcc.t_begin + (long long)lm * C;
+                mbar_arrive_expect_tx(bars + CB_FULL + s2, STAGE_TX);
+                bulk_load(stage, src, RG_PART1, bars + CB_FULL + s2);
+                bulk_load(stage + CS_QH, src + RG_QH, RG_PART2, bars + CB_FULL + s2);
+                tma_load_3d(stage + CS_V, &tm_v, 0, lcc.h, (int)t0, bars + CB_FULL + s2);
+                tma_load_3d(stage + CS_V + 8192, &tm_v, 64, lcc.h, (int)t0, bars + CB_FULL + s2);
+                ++issued[s2];
+                flush();
+                pend_u = lu;
+                pend_val = cons_after(lrho, lm, lcc.nck);
+                ++lu;
+                if (++lm == lcc.nck) {
+                    lm = 0;
+                    ++lrho;
+                    lopen();
+                }
+            };
+            if (loader) {
+                lopen();
+                for (int q = 0; q < 2 && lhave && lok; ++q) load_one();
+            }
+            uint32_t u = 0;
+            bool stop = false;
+            for (int rho = 0; !stop; ++rho) {
+                Chain cc;
+                if (!chain_of(rho, &cc)) break;
+                for (int m = 0; m < cc.nck; ++m, ++u) {
+                    const bool ok = wt.warp_wait(bars + CB_OFULL, u & 1, lane);
+                    if (!ok) {
+                        stop = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    float x[64];
+                    tmem_load<64>(tmem + TM_O + lane_q, x);
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + CB_OFREE);
+                    const long long t0 = cc.t_begin + (long long)m * C;
+                    const int L = (int)min((long long)C, cc.t_end - t0);
+                    // lane pairs (j even, j + 1) write bf16 pairs: the even lane row r,
+                    // the odd lane row r + 1
+                    __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(a.o);
+                    const bool odd = lane & 1;
+#pragma unroll
+                    for (int r = 0; r < C; r += 2) {
+                        const float mine = odd ? x[r] : x[r + 1];
+                        const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                        const int row = odd ? r + 1 : r;
+                        if (row < L) {
+                            const uint32_t v = odd ? pack2(other, x[r + 1]) : pack2(x[r], other);
+                            *reinterpret_cast<uint32_t *>(ob + ((t0 + row) * H + cc.h) * (long long)DV +
+                                                          (j & ~1)) = v;
+                        }
+                    }
+                    // chunk u is out of stage u % 2 once its products are done (the
+                    // output product was the last) and the state warps have read its
+                    // decay: chunk u + 2 may go in
+                    if (loader && lhave && lok) {
+                        const int s2 = u & 1;
+                        lok = wt.wait(bars + CB_SFREE + s2, (u >> 1) & 1) &&
+                              wt.wait(bars + CB_DSFREE + s2, (u >> 1) & 1);
+                        if (lok) load_one();
+                    }
+                    if (__shfl_sync(0xffffffffu, (loader && !lok) ? 1 : 0, 0)) {
+                        stop = true;
+                        break;
+                    }
+                }
+            }
+            if (loader) {
+                flush();
+                if (*abort_flag)
+                    for (int s2 = 0; s2 < 2; ++s2)
+                        if (issued[s2] > 0)
+                            mbar_wait(bars + CB_FULL + s2, (uint32_t)((issued[s2] - 1) & 1), kWaitLimit);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) {
+        atomicOr(a.err, kErrTimeout);
+        // local CTA: every raw buffer's last tile load lands before the CTA exits
+        if (!chain_role)
+            for (int q = 0; q < 3; ++q)
+                if (issued[q] > 0) mbar_wait(bars + LB_TMA + q, (uint32_t)((issued[q] - 1) & 1), kWaitLimit);
+    }
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// Before each launch: zero the hand-off words (cons, ready, the grid's abort
+// word) and, for a packed batch, write the task offset of every round: round
+// rho has (its chains) x (the chunks of its longest sequence) tasks.
+__global__ void __launch_bounds__(1024)
+pool_schedule_kernel(const PrefillArgs a, int nch, int nrounds, long long *rbase, uint64_t *flags,
+                     int nwords) {
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) flags[i] = 0;
+    if (rbase == nullptr) return;
+    const long long nchains = (long long)a.n_seqs * a.H;
+    auto round_tasks = [&](int rho) -> long long {
+        const long long x0 = (long long)rho * nch, x1 = min(x0 + nch, nchains);
+        long long maxck = 0;
+        for (long long n = x0 / a.H; n <= (x1 - 1) / a.H; ++n) {
+            long long tb, te;
+            seq_range(a, (int)n, &tb, &te);
+            maxck = max(maxck, (te - tb + C - 1) / C);
+        }
+        return (x1 - x0) * maxck;
+    };
+    const int per = (nrounds + (int)blockDim.x - 1) / (int)blockDim.x;
+    const int r0 = (int)threadIdx.x * per, r1 = min(nrounds, r0 + per);
+    long long sum = 0;
+    for (int rho = r0; rho < r1; ++rho) sum += round_tasks(rho);
+    __shared__ long long part[1024];
+    part[threadIdx.x] = sum;
+    __syncthreads();
+    for (int off = 1; off < (int)blockDim.x; off <<= 1) {  // inclusive scan
+        const long long v = threadIdx.x >= (unsigned)off ? part[threadIdx.x - off] : 0;
+        __syncthreads();
+        part[threadIdx.x] += v;
+        __syncthreads();
+    }
+    long long base = part[threadIdx.x] - sum;
+    for (int rho = r0; rho < r1; ++rho) {
+        rbase[rho] = base;
+        base += round_tasks(rho);
+    }
+    if (threadIdx.x == blockDim.x - 1) rbase[nrounds] = part[threadIdx.x];
+}
+
+// ------------------------------------------------------------------- host --
+struct PoolPlan {
+    int nch, nloc;
+};
+
+int device_sms() {
+    int dev = 0, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    return nsm;
+}
+
+// The split of the SMs between chain CTAs and the local pool: the chain CTAs
+// take the chains in rounds of nch, so the state pass takes rounds x chunks
+// steps of ~kChainCost cycles; the pool works through every chunk at
+// ~kLocalCost SM-cycles each.  Pick nch to balance the two.
+constexpr double kChainCost = 2000.0, kLocalCost = 7500.0;
+
+PoolPlan plan_for(const gdn_dims &d, int nsm) {
+    PoolPlan pl{0, 0};
+    const long long nchains = (long long)(d.n_seqs > 0 ? d.n_seqs : d.B) * d.H;
+    const long long seqs = d.n_seqs > 0 ? d.n_seqs : (d.B > 0 ? d.B : 1);
+    const double nck = std::max(1.0, (double)d.B * d.T / (double)seqs / C);
+    if (nchains <= 0 || nsm < 2) return pl;
+    int best = 1;
+    double best_t = 1e300;
+    const int hi = (int)std::min<long long>(nchains, nsm - 1);
+    for (int nch = 1; nch <= hi; ++nch) {
+        const double rounds = (double)((nchains + nch - 1) / nch);
+        const double t_chain = rounds * nck * kChainCost;
+        const double t_local = (double)nchains * nck * kLocalCost / (nsm - nch);
+        const double t = std::max(t_chain, t_local);
+        if (t < best_t * 0.999) {
+            best_t = t;
+            best = nch;
+        }
+    }
+    if (const char *e = getenv("GDN_POOL_CHAIN_CTAS")) {
+        const int v = atoi(e);
+        if (v >= 1 && v <= hi) best = v;
+    }
+    pl.nch = best;
+    pl.nloc = nsm - best;
+    return pl;
+}
+
+constexpr size_t kFlagWordsPerChain = 8;
+
+size_t flags_bytes(int nch) { return (((size_t)nch * kFlagWordsPerChain + 8) * 8 + 255) & ~size_t(255); }
+
+}  // namespace
+
+bool chunk_pool_supported(const gdn_dims &d) {
+    return d.dtype == GDN_BF16 && d.d_k == DK && d.d_v == DV && d.decay == GDN_DECAY_SCALAR &&
+           (long long)d.B * d.T < (1LL << 31) && d.H < 65536;
+}
+
+size_t chunk_pool_scratch_bytes(const gdn_dims &d) {
+    const PoolPlan pl = plan_for(d, device_sms());
+    if (pl.nch <= 0) return 0;
+    const long long nchains = (long long)(d.n_seqs > 0 ? d.n_seqs : d.B) * d.H;
+    const long long nrounds = (nchains + pl.nch - 1) / pl.nch;
+    return flags_bytes(pl.nch) + (size_t)pl.nch * NR * RING_STRIDE +
+           (((size_t)(nrounds + 1) * 8 + 255) & ~size_t(255));
+}
+
+cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launches) {
+    const long long nchains = (long long)a.n_seqs * a.H;
+    const long long ntok = (long long)a.B * a.T;
+    if (nchains == 0) return cudaSuccess;
+    if (ntok == 0) {
+        if (a.s_final && a.s_final != a.s0) {
+            const size_t bytes = (size_t)nchains * a.dv * a.dk * sizeof(float);
+            return a.s0 ? cudaMemcpyAsync(a.s_final, a.s0, bytes, cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(a.s_final, 0, bytes, s);
+        }
+        return cudaSuccess;
+    }
+    gdn_dims d{};
+    d.B = a.B; d.T = a.T; d.H = a.H; d.d_k = a.dk; d.d_v = a.dv; d.n_seqs = a.n_seqs;
+    d.dtype = GDN_BF16; d.decay = GDN_DECAY_SCALAR;
+    const int nsm = device_sms();
+    const PoolPlan pl = plan_for(d, nsm);
+    if (pl.nch <= 0) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv;
+    if (!make_tile_map(&mq, a.q, a.dk, a.H, ntok) || !make_tile_map(&mk, a.k, a.dk, a.H, ntok) ||
+        !make_tile_map(&mv, a.v, a.dv, a.H, ntok))
+        return cudaErrorInvalidValue;
+    PoolArgs p{};
+    uint8_t *ws = reinterpret_cast<uint8_t *>(a.scratch);
+    p.flags = reinterpret_cast<uint64_t *>(ws);
+    p.gabort = reinterpret_cast<uint32_t *>(p.flags + (size_t)pl.nch * kFlagWordsPerChain);
+    p.ring = ws + flags_bytes(pl.nch);
+    p.nch = pl.nch;
+    p.nrounds = (int)((nchains + pl.nch - 1) / pl.nch);
+    p.rbase = a.cu_seqlens ? reinterpret_cast<const long long *>(
+                                 p.ring + (size_t)pl.nch * NR * RING_STRIDE)
+                           : nullptr;
+    p.nck = (int)((a.T + C - 1) / C);
+    p.ntask = nchains * (long long)p.nck;
+    const int nwords = (int)(pl.nch * kFlagWordsPerChain + 8);
+    pool_schedule_kernel<<<1, 1024, 0, s>>>(a, p.nch, p.nrounds, const_cast<long long *>(p.rbase),
+                                             p.flags, nwords);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (launches) ++*launches;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(chunk_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(pl.nch + pl.nloc));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, chunk_pool_kernel, a, p, mq, mk, mv);
+    if (e != cudaSuccess) return e;
+    if (launches) ++*launches;
+    return cudaSuccess;
+}
+
+}  // namespace gdn

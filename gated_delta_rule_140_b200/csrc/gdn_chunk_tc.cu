@@ -46,7 +46,7 @@ constexpr int kLocal = 256;     // threads of the local group
 constexpr int kState = 128;     // threads of the state group
 constexpr int kThreads = kLocal + kState;
 constexpr int BAR_LOCAL = 1, BAR_STATE = 2, BAR_INV = 3;  // named barrier ids
-constexpr long long kWaitLimit = 1LL << 31;   // SM cycles (~1 s)
+constexpr long long kWaitLimit = kDefaultWaitLimit;  // drains after an abort
 constexpr int LDA = 68;         // fp32 row stride of A and T in smem
 
 // shared memory map (bytes from a 1024-aligned base)
@@ -135,12 +135,13 @@ __device__ __forceinline__ void decay_row(float *x, int r, int rb, int half, con
 // polling does not compete with the busy warps for issue slots or the shared
 // memory pipe.  No sleep between polls: mbarrier.try_wait suspends the thread
 // for a while itself, and a sleep only delays the waiter (measured).
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort) {
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                         long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (*abort) return false;
-        if (clock64() - t0 > kWaitLimit) {
+        if (clock64() - t0 > limit) {
             *abort = 1;
             return false;
         }
@@ -175,6 +176,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
     uint64_t *bar_pfree = bars + 7;   // the state pass has consumed P of a chunk
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_BAR + 64);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_BAR + 68);
+    const long long lim = data_wait_limit(a.err);  // data waits (the header can shorten it)
     int *tma_issued = reinterpret_cast<int *>(sm + OFF_BAR + 72);  // [2] loads issued per stage
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -264,7 +266,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         auto start_chunk = [&](int m, int issuer) -> bool {
             const int st = m & 1;
             bool ok = true;
-            if (tid == issuer) ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag);
+            if (tid == issuer) ok = wait_bar(&bar_tma[st], (uint32_t)((st ? tma_seen1 : tma_seen0) & 1), abort_flag, lim);
             if (st) ++tma_seen1; else ++tma_seen0;
             const int L = chunk_len(m);
             if (L < C) {
@@ -363,7 +365,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             bool ok = true;
 
             // ---- D_kq of this chunk ----------------------------------------------
-            if (tid == 0) ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
+            if (tid == 0) ok &= wait_bar(bar_l, bl_wait & 1, abort_flag, lim);
             ++bl_wait;
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
             tc_fence_after();
@@ -528,7 +530,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             // (D_vp of this parity and its handoff slot are free once the state
             // pass of chunk m-2 is over)
             if (tid == 4 * 32) {  // warp 4 is idle during the P stores below
-                if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag);
+                if (m >= 2) ok &= wait_bar(&bar_vpfree[st], (uint32_t)(((m >> 1) - 1) & 1), abort_flag, lim);
                 tc_fence_after();
                 const uint64_t dk = d_kmn0 + st * (RAW_STAGE >> 4);
                 const uint64_t dv = d_vmn0 + st * (RAW_STAGE >> 4);
@@ -543,7 +545,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             ++bl_commit;
             // ---- while those run: store P once the state pass has consumed the
             //      previous chunk's P ------------------------------------------------
-            if (tid == 0 && m >= 1) ok &= wait_bar(bar_pfree, (uint32_t)((m - 1) & 1), abort_flag);
+            if (tid == 0 && m >= 1) ok &= wait_bar(bar_pfree, (uint32_t)((m - 1) & 1), abort_flag, lim);
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
             if (lq >= 2) {
                 const int r = 32 * (lq - 2) + lane;
@@ -556,7 +558,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 hand[2 * lane + 1] = g_s[2 * lane + 1];
                 if (lane == 0) hand[64] = g_s[63];
             }
-            if (tid == 0) ok &= wait_bar(bar_l, bl_wait & 1, abort_flag);
+            if (tid == 0) ok &= wait_bar(bar_l, bl_wait & 1, abort_flag, lim);
             ++bl_wait;
             if (named_bar_or(BAR_LOCAL, kLocal, !ok || *abort_flag)) break;
             tc_fence_after();
@@ -598,7 +600,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             const int L = chunk_len(m);
             const float *hand = reinterpret_cast<const float *>(sm + OFF_HAND + st * HAND_STRIDE);
             bool ok = true;
-            if (tid == kLocal) ok = wait_bar(bar_ready, (uint32_t)(m & 1), abort_flag);
+            if (tid == kLocal) ok = wait_bar(bar_ready, (uint32_t)(m & 1), abort_flag, lim);
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
             tc_fence_after();
             const float gC = hand[64];
@@ -614,7 +616,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 mma_commit(bar_s);
             }
             ++bs_commit;
-            if (tid == kLocal) ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
+            if (tid == kLocal) ok &= wait_bar(bar_s, bs_wait & 1, abort_flag, lim);
             ++bs_wait;
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
             tc_fence_after();
@@ -650,7 +652,7 @@ chunk_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 mma_commit(bar_pfree);
             }
             ++bs_commit;
-            if (tid == kLocal) ok &= wait_bar(bar_s, bs_wait & 1, abort_flag);
+            if (tid == kLocal) ok &= wait_bar(bar_s, bs_wait & 1, abort_flag, lim);
             ++bs_wait;
             if (named_bar_or(BAR_STATE, kState, !ok || *abort_flag)) break;
             tc_fence_after();

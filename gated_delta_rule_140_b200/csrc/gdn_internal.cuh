@@ -16,6 +16,11 @@ constexpr int kChunk = 64;  // chunk size C of the chunkwise form
 // Sticky error bits kept in the first word of the workspace.
 enum : uint32_t { kErrBadSeqlens = 1u, kErrTimeout = 2u, kErrInternal = 4u };
 constexpr size_t kWorkspaceHeader = 256;
+// Bounded waits of the tensor-core kernels (SM clock cycles, ~1 s at 2 GHz).
+// The second word of the workspace header, when nonzero, replaces this limit
+// for the waits on data (tiles, products, hand-offs); the waits that drain a
+// kernel's own copies and MMAs after an abort always use the default.
+constexpr long long kDefaultWaitLimit = 1LL << 31;
 
 // Everything a prefill kernel needs, in device pointers.  Token-major layouts
 // (see gdn.h).  `seq_start` is null for fixed-length rows of T tokens.
@@ -50,6 +55,10 @@ cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t s, int *launche
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches);
+cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launches);
+size_t chunk_pool_scratch_bytes(const gdn_dims &d);
+// bf16 d_k = d_v = 128 scalar-decay shapes the pool kernel takes (fixed rows)
+bool chunk_pool_supported(const gdn_dims &d);
 size_t chunk_tc_scratch_bytes(const gdn_dims &d);
 size_t chunk_pair_scratch_bytes(const gdn_dims &d);
 // bf16 d_k = d_v = 128 shapes (either decay) the two-CTA kernel takes
@@ -59,6 +68,11 @@ bool chunk_tc_supported(const gdn_dims &d);
 // [tokens, H, d] bf16 as a 3-D TMA tensor map (d, H, tokens), box 64 x 1 x 64,
 // 128-byte swizzle (defined with the single-CTA tensor-core kernel).
 bool make_tile_map(CUtensorMap *m, const void *base, int d, int H, long long ntok);
+
+__device__ __forceinline__ long long data_wait_limit(const uint32_t *hdr) {
+    const uint32_t w = hdr[1];
+    return w ? (long long)w : kDefaultWaitLimit;
+}
 
 // Token range of sequence n for fixed rows or packed sequences, validated on
 // the device: a bad range records kErrBadSeqlens and yields an empty range.

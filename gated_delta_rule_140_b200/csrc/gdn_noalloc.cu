@@ -44,7 +44,7 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
     if (need > GDN_NOALLOC_SCRATCH_BYTES) {
         // the two-CTA kernel's ring does not fit: GDN runs the single-CTA
         // tensor-core kernel, KDA the CUDA-core kernel
-        d.flags &= ~GDN_FLAG_PAIR;
+        d.flags &= ~(GDN_FLAG_PAIR | GDN_FLAG_POOL);
         d.flags |= d.decay == GDN_DECAY_CHANNEL ? GDN_FLAG_CUDA_CORES : GDN_FLAG_ONE_CTA;
         need = gdn_chunk_fwd_workspace_size(&d);
     }
@@ -61,4 +61,15 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
         return GDN_ERR_CUDA;
     return gdn_chunk_fwd(&d, q, k, v, log_alpha, beta, initial_state, cu_seqlens, o,
                          final_state, scratch, GDN_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+// The error word of the array's header on the current device, read and
+// cleared like a caller workspace's (gdn_workspace_status).
+extern "C" gdn_status gdn_noalloc_status(gdn_stream_t stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if (scratch_address(dev, &scratch) != cudaSuccess) return GDN_ERR_CUDA;
+    return gdn_workspace_status(scratch, stream);
 }

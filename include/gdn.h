@@ -76,7 +76,7 @@ typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
  * recomputed by the CUDA-core kernel (exact for any decay) within the same
  * call.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use
  * the flags to compare the device paths. */
-enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4 };
+enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4, GDN_FLAG_POOL = 8 };
 
 typedef struct {
     int32_t B;       /* batch (1 for a packed batch)                           */
@@ -91,8 +91,14 @@ typedef struct {
 } gdn_dims;
 
 /* Bytes of device workspace gdn_chunk_fwd needs for `dims` (always >= 256),
- * on the current device.  The first 256 bytes hold the sticky error word;
- * zero them once before the workspace's first use (gdn_workspace_init).  The
+ * on the current device.  The first 256 bytes are a header: word 0 (bytes
+ * 0-3) is the sticky error word; word 1 (bytes 4-7), when nonzero, replaces
+ * the default limit of the tensor-core kernels' bounded waits on data (2^31 SM
+ * clock cycles, about a second) -- a test-only control: set to a few hundred
+ * cycles it makes those waits run out on purpose, and the kernels then record
+ * GDN_ERR_TIMEOUT, drain their own copies and MMAs, free their tensor memory
+ * and return.  Zero the header once before the workspace's first use
+ * (gdn_workspace_init).  The
  * two-CTA tensor-core kernel adds a ring of four 64 KiB slots for each SM index
  * of the device (2 x its SM count), through which the chunk-local SM hands each
  * chunk's matrices to the state SM; it is written before it is read and needs
@@ -167,14 +173,22 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
  *   - Every call on a device shares the one array.  Each call clears its
  *     header on `stream` before the kernels run, so calls that overlap on the
  *     GPU (other streams, other host threads) race: serialise them.
- *   - Device-detected errors are recorded in the array's header and are not
- *     reported back; inconsistent cu_seqlens still never cause an
- *     out-of-bounds access (the affected sequences are skipped).
+ *   - Device-detected errors (inconsistent cu_seqlens contents, whose
+ *     sequences are skipped without any out-of-bounds access; an expired
+ *     bounded wait) are recorded in the array's header: read them with
+ *     gdn_noalloc_status after the call.
  *   - Calls no cudaMalloc, cudaFree or other allocating routine. */
 gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q, const void *k,
                                  const void *v, const float *log_alpha, const float *beta,
                                  const float *initial_state, const int32_t *cu_seqlens,
                                  void *o, float *final_state, gdn_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the error word of the array that
+ * gdn_chunk_fwd_noalloc uses on the current device; the codes are those of
+ * gdn_workspace_status.  Since every gdn_chunk_fwd_noalloc call clears the
+ * word before its kernels run, this reports the errors of the last call on
+ * the device.  The paper has no counterpart either. */
+gdn_status gdn_noalloc_status(gdn_stream_t stream);
 
 /* Zero the workspace header (the sticky error word) on `stream`. */
 gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_stream_t stream);

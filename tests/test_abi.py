@@ -77,8 +77,14 @@ def test_prefill_kernel_choice(L):
     assert path(decay=nat.GDN_DECAY_CHANNEL) == "tensor_core_pair"
     assert path(dtype=nat.GDN_FP32) == "cuda_core"
     assert path(d_k=64, d_v=64, flags=nat.GDN_FLAG_ONE_CTA) == "cuda_core"
+    assert path(B=4, T=4096, n_seqs=4, flags=nat.GDN_FLAG_POOL) == "tensor_core_pool"
+    assert path(B=1, T=65536, n_seqs=40, flags=nat.GDN_FLAG_POOL) == "tensor_core_pool"
+    assert path(dtype=nat.GDN_FP32, flags=nat.GDN_FLAG_POOL) == "cuda_core"
     for flags, decay in ((nat.GDN_FLAG_ONE_CTA | nat.GDN_FLAG_PAIR, nat.GDN_DECAY_SCALAR),
-                         (nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_CHANNEL), (8, nat.GDN_DECAY_SCALAR)):
+                         (nat.GDN_FLAG_POOL | nat.GDN_FLAG_PAIR, nat.GDN_DECAY_SCALAR),
+                         (nat.GDN_FLAG_POOL | nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_SCALAR),
+                         (nat.GDN_FLAG_POOL, nat.GDN_DECAY_CHANNEL),
+                         (nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_CHANNEL), (16, nat.GDN_DECAY_SCALAR)):
         with pytest.raises(nat.GdnError):
             path(flags=flags, decay=decay)
 
@@ -110,7 +116,7 @@ def _call_fwd(L, dims, **kw):
     ("H = 0", {}, dict(H=0), nat.GDN_ERR_INVALID),
     ("bad dtype", {}, dict(dtype=7), nat.GDN_ERR_INVALID),
     ("bad decay", {}, dict(decay=3), nat.GDN_ERR_INVALID),
-    ("bad flags", {}, dict(flags=8), nat.GDN_ERR_INVALID),
+    ("bad flags", {}, dict(flags=16), nat.GDN_ERR_INVALID),
     ("n_seqs != B", {}, dict(n_seqs=3), nat.GDN_ERR_INVALID),
     ("cu_seqlens with B > 1", dict(cu=FAKE), dict(n_seqs=2), nat.GDN_ERR_INVALID),
     ("cu_seqlens with no sequences", dict(cu=FAKE), dict(B=1, n_seqs=0), nat.GDN_ERR_INVALID),

@@ -51,13 +51,15 @@ def test_tiny_fp32_workload(cuda_ok):
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("decay", ["scalar", "channel"])
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("path", ["default", "pair", "cuda_cores"])
+@pytest.mark.parametrize("path", ["default", "pool", "pair", "cuda_cores"])
 def test_reduced_ragged(cuda_ok, dtype, decay, d, path):
     """Several chunks and a ragged tail (T = 3*64 + 37), with an initial state,
-    on each prefill kernel that takes the shape."""
+    on each prefill kernel that takes the shape (the pool kernel is GDN only)."""
+    if path == "pool" and decay == "channel":
+        pytest.skip("the pool kernel takes scalar decay")
     x = prefill_inputs(2, 229, 3, d, d, dtype=dtype, decay=decay, seed=21,
                        alpha_shift=2.0 if decay == "scalar" else 3.0, init_std=0.05)
-    o, sf = _run(x, cuda_cores=path == "cuda_cores", pair=path == "pair")
+    o, sf = _run(x, cuda_cores=path == "cuda_cores", pair=path == "pair", pool=path == "pool")
     _full_compare(x, o, sf, dtype)
 
 
@@ -125,6 +127,50 @@ def test_bad_cu_seqlens_reported_by_workspace_status(cuda_ok):
     cu = torch.tensor([0, 100, 200, 256], dtype=torch.int32, device="cuda")
     chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, cu, workspace=ws)
     assert ws.status() == nat.GDN_OK
+
+
+def test_check_flag_raises_on_bad_cu_seqlens(cuda_ok):
+    """chunk_fwd(check=True) turns the sticky device word into an exception."""
+    x = prefill_inputs(1, 256, 2, 128, 128, dtype=torch.bfloat16, seed=26)
+    d = to_dev(x)
+    bad = torch.tensor([0, 200, 100, 256], dtype=torch.int32, device="cuda")
+    with pytest.raises(nat.GdnError) as ei:
+        chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, bad, check=True)
+    assert ei.value.status == nat.GDN_ERR_DEVICE_INPUT
+    good = torch.tensor([0, 100, 200, 256], dtype=torch.int32, device="cuda")
+    o, sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None, good, check=True)
+    x["cu_seqlens"] = good.cpu()
+    _full_compare(x, o, sf, torch.bfloat16)
+    recurrent_step(d["q"][0, :2], d["k"][0, :2], d["v"][0, :2], d["log_alpha"][0, :2],
+                   d["beta"][0, :2], torch.zeros(2, 2, 128, 128, device="cuda"), check=True)
+
+
+TC_KERNELS = [("one_cta", "scalar"), ("pair", "scalar"), ("pair", "channel"),
+              ("pool", "scalar")]
+
+
+@pytest.mark.parametrize("kind,decay", TC_KERNELS)
+def test_bounded_waits_expire_cleanly(cuda_ok, kind, decay):
+    """The test-only header word shortens every data wait to 200 SM cycles, so
+    the waits run out: the kernel records GDN_ERR_TIMEOUT, drains its own copies
+    and MMAs, frees its tensor memory and returns.  A normal call on the same
+    workspace, process and GPU right after is exact again (nothing left hung or
+    allocated)."""
+    x = prefill_inputs(2, 600, 2, 128, 128, dtype=torch.bfloat16, decay=decay,
+                       alpha_shift=2.0 if decay == "scalar" else 3.0, seed=33, init_std=0.05)
+    d = to_dev(x)
+    kw = {kind: True}
+    ws = nat.Workspace()
+    ws.get(nat.workspace_size(nat.prefill_dims(d["q"], d["v"], d["log_alpha"], **kw)))
+    ws.set_wait_limit(200)
+    chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+              workspace=ws, **kw)
+    assert ws.status() == nat.GDN_ERR_TIMEOUT
+    ws.set_wait_limit(0)
+    for _ in range(2):
+        o, sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                          workspace=ws, check=True, **kw)
+        _full_compare(x, o, sf, torch.bfloat16)
 
 
 def test_tensor_core_and_cuda_core_paths_agree(cuda_ok):
@@ -206,9 +252,64 @@ def test_pair_kernel_strong_and_zero_decay(cuda_ok):
     la = x["log_alpha"]
     la[:, :64] = -20.0
     la[:, 64:128] = 0.0
-    for pair in (False, True):
-        o, sf = _run(x, pair=pair)
+    for kw in ({}, {"pair": True}, {"pool": True}, {"one_cta": True}):
+        o, sf = _run(x, **kw)
         _full_compare(x, o, sf, torch.bfloat16)
+
+
+# --------------------------------------------------------------------------- #
+# the pool kernel: chunk-local work on a pool of SMs, chains on chain SMs     #
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 128, 129, 640, 1000])
+def test_pool_kernel_chunk_counts(cuda_ok, T):
+    """1..16 chunks per sequence: both local groups, every ring slot, partial
+    last chunks, a one-token sequence."""
+    x = prefill_inputs(2, T, 2, 128, 128, dtype=torch.bfloat16, seed=60 + T, init_std=0.05)
+    o, sf = _run(x, pool=True)
+    _full_compare(x, o, sf, torch.bfloat16)
+
+
+@pytest.mark.parametrize("nch", ["1", "3", "7"])
+def test_pool_kernel_chain_rounds(cuda_ok, monkeypatch, nch):
+    """Fewer chain CTAs than chains: each chain CTA runs several chains one after
+    another (rounds), the ring slots are reused across chains."""
+    monkeypatch.setenv("GDN_POOL_CHAIN_CTAS", nch)
+    x = prefill_inputs(3, 300, 4, 128, 128, dtype=torch.bfloat16, seed=70, init_std=0.05)
+    o, sf = _run(x, pool=True)
+    _full_compare(x, o, sf, torch.bfloat16)
+
+
+@pytest.mark.parametrize("nch", ["0", "2", "5"])
+def test_pool_kernel_packed_batch(cuda_ok, monkeypatch, nch):
+    """Packed sequences of 0..700 tokens (empty ones too), initial states; rounds
+    padded to their longest chain (empty padding tasks)."""
+    if nch != "0":
+        monkeypatch.setenv("GDN_POOL_CHAIN_CTAS", nch)
+    lens = [0, 1, 63, 64, 65, 200, 0, 130, 700, 5, 0]
+    g = torch.Generator().manual_seed(71)
+    x = prefill_inputs(1, 0, 3, 128, 128, dtype=torch.bfloat16, init_std=0.02, lengths=lens,
+                       gen=g)
+    d = to_dev(x)
+    assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"], d["cu_seqlens"],
+                                               pool=True)) == "tensor_core_pool"
+    o, sf = _run(x, pool=True, check=True)
+    _full_compare(x, o, sf, torch.bfloat16)
+    for n, L in enumerate(lens):
+        if L == 0:
+            assert torch.equal(sf[n].cpu(), x["initial_state"][n])
+
+
+def test_pool_kernel_matches_pair_kernel_bitwise_in_local_products(cuda_ok):
+    """The pool and two-CTA kernels share the chunk-local arithmetic; their state
+    passes differ (one product per chunk against two), so results agree within
+    rounding, and each run of the pool kernel is deterministic."""
+    x = prefill_inputs(2, 700, 3, 128, 128, dtype=torch.bfloat16, seed=72, init_std=0.05)
+    o1, s1 = _run(x, pool=True)
+    o2, s2 = _run(x, pool=True)
+    assert torch.equal(o1, o2) and torch.equal(s1, s2)
+    o3, s3 = _run(x, pair=True)
+    assert rel_err(o1, o3.float().cpu().numpy()) < 2e-2
+    assert rel_err(s1, s3.cpu().numpy()) < 1e-2
 
 
 # --------------------------------------------------------------------------- #
@@ -222,10 +323,13 @@ FULL = {
 }
 
 
+@pytest.mark.parametrize("kernel", ["default", "pool"])
 @pytest.mark.parametrize("name", list(FULL))
-def test_full_workload_sampled(cuda_ok, name):
+def test_full_workload_sampled(cuda_ok, name, kernel):
+    if kernel == "pool" and WORKLOADS[name].decay == "channel":
+        pytest.skip("the pool kernel takes scalar decay")
     x = workload_inputs(name)
-    o, sf = _run(x)
+    o, sf = _run(x, pool=kernel == "pool", check=True)
     assert torch.isfinite(o).all() and torch.isfinite(sf).all()
     to, ts = TOL[WORKLOADS[name].dtype]
     for n, h, ro, rs in oracle_heads(x, FULL[name]):

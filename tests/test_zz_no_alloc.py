@@ -6,9 +6,10 @@ fixed array inside the library as scratch.
 
 This file is named to be collected last, so that a run stopping at the first
 failure has already run every other test; it passes alone in a fresh process
-as well.  The entry point is called through the C ABI (ctypes), three times in
-a row on different problems, and each result is checked against gdn_chunk_fwd's
-within the parity tolerances."""
+as well.  The entry point is called through the C ABI (ctypes), once per
+problem on four problems in a row, and each result is checked against
+gdn_chunk_fwd's within the parity tolerances; a call with bad cu_seqlens
+contents is then reported by gdn_noalloc_status."""
 import ctypes
 
 import pytest
@@ -53,7 +54,7 @@ def _problems():
     return [(a, torch.bfloat16), (b, torch.float32), (c, torch.bfloat16), (e, torch.bfloat16)]
 
 
-def test_noalloc_matches_chunk_fwd_on_two_calls_in_a_row(cuda_ok):
+def test_noalloc_matches_chunk_fwd_on_calls_in_a_row(cuda_ok):
     for x, dtype in _problems():
         d = to_dev(x)
         o, sf = _noalloc(d)
@@ -78,3 +79,22 @@ def test_noalloc_fits_its_array_or_refuses(cuda_ok):
     # invalid dims are still invalid
     bad = nat.Dims(1, 64, 16, 96, 128, 1, nat.GDN_BF16, nat.GDN_DECAY_SCALAR, 0)
     assert L.gdn_chunk_fwd_noalloc(ctypes.byref(bad), *([None] * 9), None) != nat.GDN_OK
+
+
+def test_noalloc_status_reports_bad_cu_seqlens(cuda_ok):
+    """Errors only the device can see land in the array's header; the caller
+    reads them with gdn_noalloc_status (the next call clears them)."""
+    x = prefill_inputs(1, 256, 2, 128, 128, dtype=torch.bfloat16, seed=45)
+    d = to_dev(x)
+    d["cu_seqlens"] = torch.tensor([0, 200, 100, 256], dtype=torch.int32, device="cuda")
+    _noalloc(d)
+    assert nat.noalloc_status() == nat.GDN_ERR_DEVICE_INPUT
+    assert nat.noalloc_status() == nat.GDN_OK  # cleared by the read
+    d["cu_seqlens"] = torch.tensor([0, 100, 200, 256], dtype=torch.int32, device="cuda")
+    o, sf = _noalloc(d)
+    assert nat.noalloc_status() == nat.GDN_OK
+    o_ref, sf_ref = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], None,
+                              d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert rel_err(o, o_ref.double().cpu().numpy()) <= TOL[torch.bfloat16][0]
+    assert rel_err(sf, sf_ref.cpu().numpy()) <= TOL[torch.bfloat16][1]
