@@ -16,6 +16,9 @@ chunkwise(...)   the chunkwise WY / UT-transform form of FG2-GDN section 3.6,
                  with explicit per-chunk matrices; equal to ``recurrent`` in
                  exact arithmetic.
 chunk_stage(...) one chunk's intermediates (g, A, T, W, U, V', O, S_out).
+prologue(...)    the input prologue of the fused entry point (FG2-GDN section
+                 3.5): L2-normalised q and k, beta = sigmoid(b),
+                 log alpha = -softplus(a + bias).
 """
 from __future__ import annotations
 
@@ -54,6 +57,9 @@ def _bind(path):
     lib.oracle_gdn_chunkwise.restype = ctypes.c_int
     lib.oracle_gdn_chunk_stage.argtypes = [ctypes.c_int] * 3 + [_D] * 14
     lib.oracle_gdn_chunk_stage.restype = None
+    lib.oracle_gdn_prologue.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        _D, _D, _D, _D, _D, _D, _D, _D, _D]
+    lib.oracle_gdn_prologue.restype = ctypes.c_int
     return lib
 
 
@@ -165,3 +171,24 @@ def chunk_stage(q, k, v, log_alpha, beta, S):
                                    _ptr(S), *(_ptr(out[x]) for x in
                                               ("G", "A", "T", "W", "U", "Vp", "O", "S_out")))
     return out
+
+
+def prologue(q_raw, k_raw, a_logit, b_logit, a_bias=None):
+    """The fused entry point's input prologue in fp64.  q_raw, k_raw [...,H,dk];
+    a_logit [...,H] (scalar decay) or [...,H,dk] (channel decay); b_logit
+    [...,H]; a_bias [H] or [H,dk] or None.  Returns (q, k, log_alpha, beta) as
+    float64 arrays of the input shapes."""
+    qr, kr, al, bl = (_f64(x) for x in (q_raw, k_raw, a_logit, b_logit))
+    H, dk = qr.shape[-2], qr.shape[-1]
+    ntok = qr.size // (H * dk)
+    channel = al.shape == qr.shape
+    ab = _f64(a_bias)
+    if ab is not None and ab.size != (H * dk if channel else H):
+        raise ValueError("a_bias must be [H] (scalar decay) or [H, d_k] (channel decay)")
+    q, k = np.zeros_like(qr), np.zeros_like(kr)
+    la, b = np.zeros_like(al), np.zeros_like(bl)
+    r = _load().oracle_gdn_prologue(ntok, H, dk, int(channel), _ptr(qr), _ptr(kr), _ptr(al),
+                                    _ptr(ab), _ptr(bl), _ptr(q), _ptr(k), _ptr(la), _ptr(b))
+    if r != 0:
+        raise ValueError("oracle rejected its arguments")
+    return q, k, la, b

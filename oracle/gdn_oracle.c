@@ -320,3 +320,50 @@ int oracle_gdn_chunkwise(int n_seqs, const int64_t *seq_start, int H, int dk, in
                  S0, o, S_final, chunk};
     return run(&p, 1, nthreads);
 }
+
+/* ------------------------------------------------------------------------ */
+/* The input prologue of the fused entry point (FG2-GDN paper, section 3.5,  */
+/* "Gate Parameterization"): queries and keys are L2-normalised per token    */
+/* and head; the writing rate is a sigmoid of its projection, beta_t =       */
+/* sigmoid(b_t); the decay comes from a negative softplus of its projection  */
+/* plus an optional bias, log alpha_t = -softplus(a_t + bias).  A zero        */
+/* vector is left at zero (its norm is clamped below at 1e-12).              */
+/* ------------------------------------------------------------------------ */
+static double softplus(double x) {
+    /* log(1 + e^x) without overflow: x + log(1 + e^-x) for x > 0 */
+    return x > 0 ? x + log1p(exp(-x)) : log1p(exp(x));
+}
+
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+static void unit_rows(int64_t rows, int d, const double *in, double *out) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double ss = 0.0;
+        for (int c = 0; c < d; ++c) ss += in[r * d + c] * in[r * d + c];
+        double nrm = sqrt(ss);
+        if (nrm < 1e-12) nrm = 1e-12;
+        for (int c = 0; c < d; ++c) out[r * d + c] = in[r * d + c] / nrm;
+    }
+}
+
+/* ntok tokens x H heads.  channel = 0: a_logit [ntok,H], a_bias [H] or NULL;
+ * channel = 1: a_logit [ntok,H,dk], a_bias [H,dk] or NULL.  b_logit [ntok,H]. */
+int oracle_gdn_prologue(int64_t ntok, int H, int dk, int channel, const double *q_raw,
+                        const double *k_raw, const double *a_logit, const double *a_bias,
+                        const double *b_logit, double *q, double *k, double *log_alpha,
+                        double *beta) {
+    if (ntok < 0 || H <= 0 || dk <= 0) return -1;
+    unit_rows(ntok * H, dk, q_raw, q);
+    unit_rows(ntok * H, dk, k_raw, k);
+    const int per = channel ? dk : 1;
+    for (int64_t t = 0; t < ntok; ++t)
+        for (int h = 0; h < H; ++h) {
+            beta[t * H + h] = sigmoid(b_logit[t * H + h]);
+            for (int c = 0; c < per; ++c) {
+                const int64_t i = (t * H + h) * per + c;
+                const double bias = a_bias ? a_bias[h * per + c] : 0.0;
+                log_alpha[i] = -softplus(a_logit[i] + bias);
+            }
+        }
+    return 0;
+}

@@ -44,6 +44,17 @@ MUTATIONS = [
      "acc += Vp[s * dv + i] * k[s * dk + c];"),
     ("chunk end state: state transposed",
      "double acc = S[i * dk + c] * exp(gL);", "double acc = S[c * dk + i] * exp(gL);"),
+    ("prologue: norm not rooted", "double nrm = sqrt(ss);", "double nrm = ss;"),
+    ("prologue: sigmoid of the negated logit",
+     "static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }",
+     "static double sigmoid(double x) { return 1.0 / (1.0 + exp(x)); }"),
+    ("prologue: softplus tail loses x",
+     "return x > 0 ? x + log1p(exp(-x)) : log1p(exp(x));",
+     "return x > 0 ? log1p(exp(-x)) : log1p(exp(x));"),
+    ("prologue: decay bias dropped",
+     "log_alpha[i] = -softplus(a_logit[i] + bias);", "log_alpha[i] = -softplus(a_logit[i]);"),
+    ("prologue: decay sign", "log_alpha[i] = -softplus(a_logit[i] + bias);",
+     "log_alpha[i] = softplus(a_logit[i] + bias);"),
 ]
 
 PIN_TESTS = [
@@ -55,6 +66,9 @@ PIN_TESTS = [
     (pins.test_brute_force_transition_products, [(False,), (True,)]),
     (pins.test_chunkwise_equals_recurrent, [(False, 16), (True, 16)]),
     (pins.test_chunk_stage_ut_factor, [(False,), (True,)]),
+    (pins.test_prologue_gate_closed_forms, [()]),
+    (pins.test_prologue_decay_bias_per_head_and_channel, [()]),
+    (pins.test_prologue_unit_norm_scale_invariance_and_direction, [()]),
 ]
 
 

@@ -367,3 +367,80 @@ def test_threads_do_not_change_results():
     o2, s2 = oracle.recurrent(q, k, v, la, beta, S0, nthreads=8)
     np.testing.assert_array_equal(o1, o2)
     np.testing.assert_array_equal(s1, s2)
+
+
+# --------------------------------------------------------------------------- #
+# the fused entry point's input prologue (FG2-GDN section 3.5, "Gate           #
+# Parameterization": L2-normalised queries and keys, beta from a sigmoid, the   #
+# decay from a negative softplus)                                               #
+# --------------------------------------------------------------------------- #
+def _prologue_gates(a, b, bias=None, H=None):
+    a = np.asarray(a, dtype=np.float64).reshape(-1, H or 1)
+    b = np.asarray(b, dtype=np.float64).reshape(-1, H or 1)
+    H = a.shape[1]
+    z = np.ones((a.shape[0], H, 4))
+    _, _, la, be = oracle.prologue(z, z, a, b, bias)
+    return la, be
+
+
+def test_prologue_gate_closed_forms():
+    """Points where sigmoid and softplus have exact values: sigmoid(0) = 1/2,
+    sigmoid(ln 3) = 3/4, softplus(0) = ln 2, softplus(ln(e^2 - 1)) = 2; the
+    identities sigmoid(x) + sigmoid(-x) = 1 and softplus(x) - softplus(-x) = x;
+    and the tails softplus(40) = 40 + e^-40, softplus(-40) = e^-40 (up to
+    rounding), where a naive log(1 + e^x) would overflow or lose all digits."""
+    x = np.array([0.0, np.log(3.0), np.log(np.e ** 2 - 1.0), 40.0, -40.0, 1.7, -0.3])
+    la, be = _prologue_gates(x, x)
+    la_m, be_m = _prologue_gates(-x, -x)
+    sp, sig = -la[:, 0], be[:, 0]
+    assert sig[0] == 0.5 and abs(sig[1] - 0.75) < 1e-15
+    assert abs(sp[0] - np.log(2.0)) < 1e-15 and abs(sp[1] - np.log(4.0)) < 1e-15
+    assert abs(sp[2] - 2.0) < 1e-14
+    assert abs(sp[3] - 40.0) < 1e-13 and abs(sp[4] - np.exp(-40.0)) < 1e-30
+    assert np.all(np.abs(sig + be_m[:, 0] - 1.0) < 1e-15)
+    assert np.all(np.abs(sp - (-la_m[:, 0]) - x) < 1e-13)
+    assert np.all(la < 0) and np.all((be > 0) & (be <= 1))  # sigmoid(40) rounds to 1
+
+
+def test_prologue_decay_bias_per_head_and_channel():
+    """The bias is added to the decay logit before the softplus, per head
+    (scalar decay) or per head and key channel (channel decay): a bias equal
+    to c gives exactly the unbiased result at logit + c."""
+    rng = np.random.default_rng(80)
+    a = rng.standard_normal((5, 3))
+    bias = np.array([0.5, -1.0, 2.0])
+    la_b, _ = _prologue_gates(a, a, bias, H=3)
+    la_s, _ = _prologue_gates(a + bias[None, :], a, None, H=3)
+    assert np.array_equal(la_b, la_s)
+    z = np.ones((5, 3, 4))
+    ac = rng.standard_normal((5, 3, 4))
+    bc = rng.standard_normal((3, 4))
+    _, _, la1, _ = oracle.prologue(z, z, ac, a, bc)
+    _, _, la2, _ = oracle.prologue(z, z, ac + bc[None], a, None)
+    assert np.array_equal(la1, la2)
+
+
+def test_prologue_unit_norm_scale_invariance_and_direction():
+    """Each (token, head) query and key vector comes out with unit norm, in the
+    direction of the raw vector, unchanged by a positive scale of the raw
+    vector; a zero vector stays zero; heads do not mix."""
+    rng = np.random.default_rng(81)
+    q = rng.standard_normal((7, 3, 16)) * rng.uniform(0.01, 100, (7, 3, 1))
+    k = rng.standard_normal((7, 3, 16))
+    k[2, 1] = 0.0
+    a, b = np.zeros((7, 3)), np.zeros((7, 3))
+    qn, kn, _, _ = oracle.prologue(q, k, a, b)
+    assert np.all(np.abs(np.linalg.norm(qn, axis=-1) - 1) < 1e-14)
+    nz = np.linalg.norm(k, axis=-1) > 0
+    assert np.all(np.abs(np.linalg.norm(kn, axis=-1)[nz] - 1) < 1e-14)
+    assert np.all(kn[2, 1] == 0)
+    # collinear with the raw vector and pointing the same way
+    dots = np.einsum("thd,thd->th", qn, q)
+    assert np.all(dots > 0)
+    assert np.max(np.abs(q - dots[..., None] * qn)) < 1e-12 * np.abs(q).max()
+    qn2, _, _, _ = oracle.prologue(3.5 * q, k, a, b)
+    assert np.max(np.abs(qn2 - qn)) < 1e-15
+    q3 = q.copy()
+    q3[:, 0] *= -7.0
+    qn3, _, _, _ = oracle.prologue(q3, k, a, b)
+    assert np.array_equal(qn3[:, 1:], qn[:, 1:])
