@@ -51,6 +51,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 CHUNK = 64
 PREFILL_LEGS = ("gdn_prefill_bf16", "gdn_varlen_bf16", "kda_prefill_bf16",
                 "gdn_long_prefill_bf16")
+RAW_LEG = "gdn_prefill_bf16_raw"  # the config-2 shapes through the fused input prologue
 DECODE_LEG = "gdn_decode"
 KERNEL_SRC = {
     "tensor_core_pool": ("chunk_pool_kernel", "gdn_chunk_pool.cu"),
@@ -472,6 +473,50 @@ def e2e_decode(xd, state, od, wd, n, stream):
     return go(n), h2d, d2h
 
 
+def raw_leg(head, dev, ws, stream, pk, pk_kind, args, K):
+    """The headline workload's shapes through gdn_chunk_fwd_raw: unnormalised q,
+    k and gate logits in, the L2 norms, sigmoid and -softplus applied inside the
+    kernel.  Beside it, the unfused route a caller would take otherwise: torch
+    element-wise passes (normalise q and k, sigmoid, -softplus) that read the raw
+    inputs and write the prepared ones, then the same call on the pool kernel."""
+    import torch
+    import torch.nn.functional as F
+    from gated_delta_rule_140_b200 import chunk_fwd, chunk_fwd_raw
+    from gated_delta_rule_140_b200.inputs import raw_prefill_inputs
+    w = head.w
+    r = {k: v.to(dev) for k, v in raw_prefill_inputs(w.B, w.T, w.H, w.d, seed=11).items()}
+    o = torch.empty_like(r["v"])
+    sf = torch.empty(w.B, w.H, w.d, w.d, dtype=torch.float32, device=dev)
+
+    def fused():
+        chunk_fwd_raw(r["q_raw"], r["k_raw"], r["v"], r["alpha_logit"], r["beta_logit"],
+                      r["alpha_bias"], o=o, final_state=sf, workspace=ws)
+
+    def unfused():
+        q = (r["q_raw"].float() / r["q_raw"].float().norm(dim=-1, keepdim=True)).to(r["v"].dtype)
+        k = (r["k_raw"].float() / r["k_raw"].float().norm(dim=-1, keepdim=True)).to(r["v"].dtype)
+        la = -F.softplus(r["alpha_logit"] + r["alpha_bias"])
+        be = torch.sigmoid(r["beta_logit"])
+        chunk_fwd(q, k, r["v"], la, be, o=o, final_state=sf, workspace=ws, pool=True)
+
+    for _ in range(3):
+        fused()
+        unfused()
+    t1 = time_loop(fused, 3, stream) / 3 / 1e3
+    reps = max(K, math.ceil(args.leg_seconds / max(t1, 1e-6)))
+    sec = time_loop(fused, reps, stream) / reps / 1e3
+    reps_u = max(K, math.ceil(0.5 * args.leg_seconds / max(t1, 1e-6)))
+    sec_u = time_loop(unfused, reps_u, stream) / reps_u / 1e3
+    fl, by = head.work()
+    th = head.tokens * head.H
+    extra = th * (2 * 2 * 2 * w.d + 4 * 4)  # q, k read + written (bf16), 2 gates read + written
+    return {"value": head.tokens / sec, "unit": "tokens/s", "ms": sec * 1e3, "reps": reps,
+            "roofline": roofline(fl, by, sec, pk, pk_kind, None, "chunk_pool_kernel"),
+            "unfused_ms": sec_u * 1e3, "unfused_extra_hbm_bytes": extra,
+            "config": {"B": w.B, "T": w.T, "H": w.H, "d_k": w.d, "d_v": w.d,
+                       "inputs": "q, k unnormalised; decay and rate logits; bias 2 per head"}}
+
+
 def run_ours(args, rank, world, local):
     import torch
     from gated_delta_rule_140_b200 import _native as nat
@@ -539,13 +584,17 @@ def run_ours(args, rank, world, local):
     pre_s, dec_s = pre_ms / K / 1e3, dec_ms / K / 1e3
 
     # ---- every workload on its own, >= leg_seconds of device time each -------
-    want = PREFILL_LEGS + (DECODE_LEG,) if args.legs == "all" else \
+    want = PREFILL_LEGS + (RAW_LEG, DECODE_LEG) if args.legs == "all" else \
         tuple() if args.legs == "none" else tuple(args.legs.split(","))
     legs = {}
     n_leg_launches = 0
     if rank == 0 or world > 1:
         for name in want:
             rows0 = len(clocks.rows)
+            if name == RAW_LEG:
+                legs[name] = raw_leg(head, dev, ws, stream, pk, pk_kind, args, K)
+                legs[name]["clocks"] = clocks.summary(clocks.rows[rows0:])
+                continue
             if name == DECODE_LEG:
                 dec_reps = max(K, math.ceil(args.leg_seconds / max(dec_s, 1e-6)))
                 l0 = nat.launch_count()

@@ -55,6 +55,8 @@ def lib():
     L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
     L.gdn_recurrent_step.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp]
     L.gdn_recurrent_step.restype = ctypes.c_int
+    L.gdn_chunk_fwd_raw.argtypes = [D, vp, vp, vp, fp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
+    L.gdn_chunk_fwd_raw.restype = ctypes.c_int
     L.gdn_noalloc_status.argtypes = [vp]
     L.gdn_noalloc_status.restype = ctypes.c_int
     L.gdn_workspace_init.argtypes = [vp, sz, vp]
@@ -227,6 +229,44 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
         raise GdnError(st, "gdn_chunk_fwd")
     if check:
         _raise_on_status(ws.status(stream), "gdn_chunk_fwd (device)")
+    return o, final_state
+
+
+def chunk_fwd_raw(q_raw, k_raw, v, alpha_logit, beta_logit, alpha_bias=None,
+                  initial_state=None, cu_seqlens=None, *, output_final_state=True, o=None,
+                  final_state=None, workspace: Workspace = None, check=False, stream=None):
+    """Chunkwise prefill with the input prologue fused in (gdn_chunk_fwd_raw):
+    q_raw, k_raw unnormalised, alpha_logit [B,T,H] and beta_logit [B,T,H]
+    logits, alpha_bias [H] or None.  The kernel L2-normalises q and k, takes
+    beta = sigmoid(beta_logit) and log alpha = -softplus(alpha_logit + bias).
+    Returns (o, final_state or None)."""
+    import torch
+    for name, t in (("q_raw", q_raw), ("k_raw", k_raw), ("v", v)):
+        _check_dev(name, t, q_raw.dtype)
+    _check_dev("alpha_logit", alpha_logit, torch.float32)
+    _check_dev("beta_logit", beta_logit, torch.float32)
+    _check_dev("alpha_bias", alpha_bias, torch.float32)
+    _check_dev("initial_state", initial_state, torch.float32)
+    _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    dims = prefill_dims(q_raw, v, alpha_logit, cu_seqlens, pool=True)
+    if o is None:
+        o = torch.empty(v.shape, dtype=q_raw.dtype, device=q_raw.device)
+    if final_state is None and output_final_state:
+        final_state = torch.empty(dims.n_seqs, dims.H, dims.d_v, dims.d_k, dtype=torch.float32,
+                                  device=q_raw.device)
+    ws = workspace if workspace is not None else _workspace_for(q_raw.device, stream)
+    # (a shape the fused path does not take has no workspace size: the call
+    # itself then returns its status)
+    buf = ws.get(max(256, int(lib().gdn_chunk_fwd_workspace_size(ctypes.byref(dims)))), stream)
+    st = lib().gdn_chunk_fwd_raw(ctypes.byref(dims), _ptr(q_raw), _ptr(k_raw), _ptr(v),
+                                 _ptr(alpha_logit), _ptr(alpha_bias), _ptr(beta_logit),
+                                 _ptr(initial_state), _ptr(cu_seqlens), _ptr(o),
+                                 _ptr(final_state), _ptr(buf), ctypes.c_size_t(buf.numel()),
+                                 _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_chunk_fwd_raw")
+    if check:
+        _raise_on_status(ws.status(stream), "gdn_chunk_fwd_raw (device)")
     return o, final_state
 
 

@@ -74,11 +74,17 @@ size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims) {
     return gdn::kWorkspaceHeader + ((extra + 255) & ~size_t(255));
 }
 
-gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, const void *v,
-                         const float *log_alpha, const float *beta,
-                         const float *initial_state, const int32_t *cu_seqlens,
-                         void *o, float *final_state,
-                         void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// The prefill entry points: validate on the host, fill the device arguments,
+// launch the selected kernel.  raw = 1: the fused input prologue (pool kernel).
+gdn_status chunk_fwd_impl(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta, const float *alpha_bias,
+                          int raw, const float *initial_state, const int32_t *cu_seqlens,
+                          void *o, float *final_state, void *workspace, size_t workspace_bytes,
+                          gdn_stream_t stream) {
     gdn_status st = check_dims(dims, true);
     if (st != GDN_OK) return st;
     const gdn_dims &d = *dims;
@@ -95,8 +101,10 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
                           (const void *)final_state, (const void *)workspace})
         if (p && !aligned16(p)) return GDN_ERR_INVALID;
     if ((reinterpret_cast<uintptr_t>(log_alpha) | reinterpret_cast<uintptr_t>(beta) |
-         reinterpret_cast<uintptr_t>(cu_seqlens)) & 3u)
+         reinterpret_cast<uintptr_t>(alpha_bias) | reinterpret_cast<uintptr_t>(cu_seqlens)) & 3u)
         return GDN_ERR_INVALID;
+    const Path p = select_path(d);
+    if (raw && p != Path::kPool) return GDN_ERR_UNSUPPORTED;
 
     gdn::PrefillArgs a{};
     a.q = q; a.k = k; a.v = v;
@@ -108,18 +116,47 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
     a.B = d.B; a.T = d.T; a.H = d.H; a.dk = d.d_k; a.dv = d.d_v; a.n_seqs = n_seqs;
     a.channel = d.decay == GDN_DECAY_CHANNEL;
     a.bf16 = d.dtype == GDN_BF16;
+    a.raw = raw;
+    a.alpha_bias = alpha_bias;
 
     // Nothing to compute and nothing to write: an empty batch is a no-op.
     if (n_seqs == 0) return GDN_OK;
     int launches = 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const Path p = select_path(d);
     cudaError_t e = p == Path::kPool     ? gdn::launch_chunk_pool(a, s, &launches)
                     : p == Path::kPair   ? gdn::launch_chunk_pair(a, s, &launches)
                     : p == Path::kOneCta ? gdn::launch_chunk_tc(a, s, &launches)
                                          : gdn::launch_chunk_simt(a, s, &launches);
     g_launches.fetch_add(launches, std::memory_order_relaxed);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                         const float *log_alpha, const float *beta,
+                         const float *initial_state, const int32_t *cu_seqlens,
+                         void *o, float *final_state,
+                         void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    return chunk_fwd_impl(dims, q, k, v, log_alpha, beta, nullptr, 0, initial_state, cu_seqlens,
+                          o, final_state, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_fwd_raw(const gdn_dims *dims, const void *q_raw, const void *k_raw,
+                             const void *v, const float *alpha_logit, const float *alpha_bias,
+                             const float *beta_logit, const float *initial_state,
+                             const int32_t *cu_seqlens, void *o, float *final_state,
+                             void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    if (!dims) return GDN_ERR_INVALID;
+    if (dims->decay != GDN_DECAY_SCALAR || (dims->flags & ~GDN_FLAG_POOL) != 0)
+        return dims->decay == GDN_DECAY_CHANNEL ? GDN_ERR_UNSUPPORTED : GDN_ERR_INVALID;
+    gdn_dims d = *dims;
+    d.flags = GDN_FLAG_POOL;
+    return chunk_fwd_impl(&d, q_raw, k_raw, v, alpha_logit, beta_logit, alpha_bias, 1,
+                          initial_state, cu_seqlens, o, final_state, workspace, workspace_bytes,
+                          stream);
 }
 
 gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k, const void *v,

@@ -1168,7 +1168,10 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 // takes this chunk's decay of its key channel; the V' warps (lanes
                 // 64-127) write V' as bf16, MN-major [r][i]
                 float dec = 0.f;
-                const bool okv = ok && wt.warp_wait(bars + SB_VO + hv, (uint32_t)(m & 1), lane);
+                // (the leader's result reaches its whole warp before the warp-wide
+                // wait, so that every lane takes the same branch)
+                const bool okv = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
+                                 wt.warp_wait(bars + SB_VO + hv, (uint32_t)(m & 1), lane);
                 if (okv) {
                     dec = reinterpret_cast<const float *>(sm + st * S_STAGE + SG_DEC)[c];
                     if (q >= 2) {

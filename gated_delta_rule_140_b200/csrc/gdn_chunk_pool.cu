@@ -89,14 +89,15 @@ static_assert(CS_QH + RG_PART2 == CS_DEC + 512 && CS_DEC + 512 <= CS_V &&
 constexpr uint32_t L_RAW_AC = 16384, RAW_BYTES = 32768;
 constexpr uint32_t PZ_P = 0, PZ_X1 = 8192, PZ_X2 = 16384, PZ_X3 = 24576, PZT_BYTES = 32768;
 constexpr uint32_t AT_BYTES = 64 * LDA * 4;
-constexpr uint32_t GATES_STRIDE = 3072;
+constexpr uint32_t GATES_STRIDE = 3584;
 constexpr uint32_t L_G0 = 3 * RAW_BYTES;
 constexpr uint32_t L_PZT = 0, L_AT = PZT_BYTES, L_GATES = L_AT + AT_BYTES;
 constexpr uint32_t L_GSZ = L_GATES + 2 * GATES_STRIDE;
 static_assert(L_GATES % 1024 == 0 && L_GSZ % 1024 == 0, "local group layout");
-// gate rows (floats): g beta beta*gamma colf rowf[4] kh gamma, and e^{g_C} x128
+// gate rows (floats): g beta beta*gamma colf rowf[4] kh gamma, e^{g_C} x128, and
+// (raw inputs) the inverse key and query norms of the task's rows
 constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR_KH = 512,
-              GR_GAM = 576, GR_DEC = 640;
+              GR_GAM = 576, GR_DEC = 640, GR_INVK = 768, GR_INVQ = 832;
 
 // ---- bookkeeping (same offset in both roles) --------------------------------
 constexpr uint32_t OFF_COMMON = CS_S + 32768;  // 215040
@@ -214,6 +215,12 @@ __device__ __forceinline__ Task task_of(const PrefillArgs &a, const PoolArgs &p,
     k.rho = rho;
     return k;
 }
+
+// log(1 + e^x) without overflow, and 1 / (1 + e^-x), in fp32
+__device__ __forceinline__ float softplusf(float x) {
+    return x > 0.f ? x + log1pf(expf(-x)) : log1pf(expf(x));
+}
+__device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + expf(-x)); }
 
 __device__ __forceinline__ int4 pack_task(const Task &k) {
     return make_int4((int)k.t0, k.h | (k.L << 16), k.b | (k.rho << 8), k.m);
@@ -352,6 +359,10 @@ struct Waiter {
     }
 };
 
+// RAW: q, k arrive unnormalised and the gates as logits (the fused input
+// prologue: L2 norms folded into the row and column scales of the products,
+// beta = sigmoid(b), log alpha = -softplus(a + bias)).
+template <bool RAW>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
@@ -467,6 +478,14 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 nla1 = r1 < tk.L ? a.log_alpha[(tk.t0 + r1) * H + tk.h] : 0.f;
                 nbe0 = r0 < tk.L ? a.beta[(tk.t0 + r0) * H + tk.h] : 0.f;
                 nbe1 = r1 < tk.L ? a.beta[(tk.t0 + r1) * H + tk.h] : 0.f;
+                if constexpr (RAW) {
+                    // logits -> gates; rows past the sequence end stay (0, 0)
+                    const float bias = a.alpha_bias ? a.alpha_bias[tk.h] : 0.f;
+                    nla0 = r0 < tk.L ? -softplusf(nla0 + bias) : 0.f;
+                    nla1 = r1 < tk.L ? -softplusf(nla1 + bias) : 0.f;
+                    nbe0 = r0 < tk.L ? sigmoidf(nbe0) : 0.f;
+                    nbe1 = r1 < tk.L ? sigmoidf(nbe1) : 0.f;
+                }
             };
             // gate rows of task kk (one warp): cumulative log decay, beta, the
             // factored block decays, kh and gamma, e^{g_C} for every channel
@@ -567,6 +586,10 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     fence_proxy_async_smem();
                     if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 }
+                // raw inputs: every thread reads the tiles for the norms below
+                if (RAW && L == C) {
+                    if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                }
                 // ---- D_kq = [K; Q] K^T (a full task's MMA goes out as soon as its
                 //      tiles are in; an abort is seen at the barrier after it) -------
                 if (issuer && ok) {
@@ -577,7 +600,24 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                         mma_bf16(tm_kq, d_raw + off, d_raw + off, ID_KK, kk > 0);
                     }
                     mma_commit(bar_l);
-                    ok = wt.wait(bar_l, bl_wait & 1);
+                    if (!RAW) ok = wt.wait(bar_l, bl_wait & 1);
+                }
+                if constexpr (RAW) {
+                    // 1 / ||k_r||, 1 / ||q_r|| of the raw bf16 rows (norm clamped at
+                    // 1e-12) while the product runs: thread pair per (tile, row)
+                    const int tsel = gtid >> 7, r = (gtid & 127) >> 1, at = gtid & 1;
+                    const uint8_t *rowp = rawp + at * L_RAW_AC + tsel * 8192;
+                    float ss = 0.f;
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        float v8[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(rowp + sw128(r, cc)), v8);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) ss = fmaf(v8[e], v8[e], ss);
+                    }
+                    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                    if (at == 0) gr[(tsel ? GR_INVQ : GR_INVK) + r] = rsqrtf(fmaxf(ss, 1e-24f));
+                    if (issuer && ok) ok = wt.wait(bar_l, bl_wait & 1);
                 }
                 ++bl_wait;
                 // the tiles that the A/P phase below rewrites went out first, as
@@ -593,6 +633,17 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 if ((lq & 1) >= lhalf) {
                     float x[32];
                     tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
+                    if constexpr (RAW) {
+                        // normalised rows and columns: x_rs / (||row_r|| ||k_s||)
+                        const int r = 32 * (lq & 1) + lane;
+                        const float rsc = gr[(lq < 2 ? GR_INVK : GR_INVQ) + r];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const float4 cs = *reinterpret_cast<const float4 *>(gr + GR_INVK + 32 * lhalf + j);
+                            x[j] *= rsc * cs.x; x[j + 1] *= rsc * cs.y;
+                            x[j + 2] *= rsc * cs.z; x[j + 3] *= rsc * cs.w;
+                        }
+                    }
                     if (lq < 2) {
                         const int r = 32 * lq + lane;
                         decay_row(x, r, lq, lhalf, gr, false);
@@ -735,6 +786,12 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     *reinterpret_cast<float4 *>(bv + 4) = *reinterpret_cast<const float4 *>(gb + 8 * j + 4);
                     *reinterpret_cast<float4 *>(gv) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j);
                     *reinterpret_cast<float4 *>(gv + 4) = *reinterpret_cast<const float4 *>(gr + GR_BG + 8 * j + 4);
+                    if constexpr (RAW) {  // W = T_b diag(gamma) K_n = T_b diag(gamma / ||k||) K
+                        const float4 i0 = *reinterpret_cast<const float4 *>(gr + GR_INVK + 8 * j);
+                        const float4 i1 = *reinterpret_cast<const float4 *>(gr + GR_INVK + 8 * j + 4);
+                        gv[0] *= i0.x; gv[1] *= i0.y; gv[2] *= i0.z; gv[3] *= i0.w;
+                        gv[4] *= i1.x; gv[5] *= i1.y; gv[6] *= i1.z; gv[7] *= i1.w;
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int s2 = 8 * j + e;
@@ -792,7 +849,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 //      tiles' Q is then free.
                 {
                     const int r = 32 * (lq & 1) + lane;
-                    const float gam = gr[GR_GAM + r];
+                    const float gam = gr[GR_GAM + r] * (RAW ? gr[GR_INVQ + r] : 1.f);
                     uint8_t *wst = grp + L_AT + lhalf * 8192;
                     uint8_t *qst = pzt + (lhalf ? PZ_X2 : PZ_X1);
                     const uint8_t *qt = rawp + lhalf * L_RAW_AC + 8192;
@@ -826,7 +883,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                         const int ac = idx >> 9, rr = (idx >> 3) & 63, j = idx & 7;
                         float kv[8];
                         unpack8(*reinterpret_cast<const uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)), kv);
-                        const float sc = gr[GR_KH + rr];
+                        const float sc = gr[GR_KH + rr] * (RAW ? gr[GR_INVK + rr] : 1.f);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) kv[e] *= sc;
                         *reinterpret_cast<uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)) = pack8(kv);
@@ -1022,9 +1079,61 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             }
         } else if (warp < 12) {
             // ---- X warps: X = Kt^T [T_b | -W] -> Z^T, G^T (bf16, K-major rows n);
-            //      then D_S = V^T Z ---------------------------------------------------
+            //      then D_S = V^T Z.  Lane 0 of warp 8 issues these products and is
+            //      also the loader: the ring slot and the V tile of chunk u + 1 go
+            //      into stage (u + 1) % 2 as soon as chunk u - 1 is out of it, and
+            //      the slot is given back (cons) as soon as they have landed.
             const int n = 32 * (warp & 3) + lane;
             const bool leader = warp == 8 && lane == 0;
+            uint64_t *fl = p.flags + (size_t)b * 8;
+            // loader cursor: the chain and chunk of the next load
+            int lrho = 0, lm = 0;
+            Chain lcc;
+            bool lhave = false;
+            bool lok = true;
+            // the next chain with chunks from round lrho on (an empty chain is
+            // passed at once: its chain CTA has nothing to read)
+            auto lopen = [&]() {
+                for (;; ++lrho) {
+                    lhave = chain_of(lrho, &lcc);
+                    if (!lhave || lcc.nck > 0) return;
+                    st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
+                }
+            };
+            // issue the loads of the cursor's chunk (global index lu) into its stage
+            auto load_one = [&](uint32_t lu) {
+                const int s2 = lu & 1;
+                uint8_t *stage = sm + s2 * CS_STAGE;
+                if (lok) lok = wt.wait_global(fl + 1 + (lm % NR), ready_tag(lrho, lm), true);
+                if (!lok) return;
+                fence_proxy_async_global();
+                const uint8_t *src = p.ring + ((size_t)b * NR + (lm % NR)) * RING_STRIDE;
+                const long long t0 = lcc.t_begin + (long long)lm * C;
+                mbar_arrive_expect_tx(bars + CB_FULL + s2, STAGE_TX);
+                bulk_load(stage, src, RG_PART1, bars + CB_FULL + s2);
+                bulk_load(stage + CS_QH, src + RG_QH, RG_PART2, bars + CB_FULL + s2);
+                tma_load_3d(stage + CS_V, &tm_v, 0, lcc.h, (int)t0, bars + CB_FULL + s2);
+                tma_load_3d(stage + CS_V + 8192, &tm_v, 64, lcc.h, (int)t0, bars + CB_FULL + s2);
+                ++issued[s2];
+                // the V tiles two chunks on, into L2
+                if (lm + 2 < lcc.nck) {
+                    tma_prefetch_l2_3d(&tm_v, 0, lcc.h, (int)(t0 + 2 * C));
+                    tma_prefetch_l2_3d(&tm_v, 64, lcc.h, (int)(t0 + 2 * C));
+                }
+            };
+            // after chunk lu has landed: give its slot back, move the cursor on
+            auto loaded = [&](uint32_t lu) {
+                st_release_u64(fl, cons_after(lrho, lm, lcc.nck));
+                if (++lm == lcc.nck) {
+                    lm = 0;
+                    ++lrho;
+                    lopen();
+                }
+            };
+            if (leader) {
+                lopen();
+                if (lhave) load_one(0);
+            }
             uint32_t u = 0;
             bool stop = false;
             for (int rho = 0; !stop; ++rho) {
@@ -1034,10 +1143,11 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     const int s = u & 1;
                     const uint32_t sb = sbase + s * CS_STAGE;
                     uint8_t *sp = sm + s * CS_STAGE;
-                    bool ok = true;
-                    if (leader) {
+                    bool ok = lok;
+                    if (leader && ok) {
                         ok = wt.wait(bars + CB_FULL + s, (u >> 1) & 1);
                         if (ok) {
+                            loaded(u);
                             tc_fence_after();
                             const uint64_t d_kt = desc_sw128(sb + CS_KT, 8192, 1024);
                             const uint64_t d_tw = desc_sw128(sb + CS_TB, 8192, 1024);
@@ -1078,6 +1188,16 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                                 mma_bf16(tmem + TM_DS + 128 * s, d_v + 128 * kk, d_z + 2 * kk, ID_VZ, kk > 0);
                             mbar_arrive(bars + CB_AISS + s);
                         }
+                        // chunk u + 1 into the other stage once chunk u - 1 has left it
+                        // (its products done, its decay read by the state warps)
+                        if (ok && lhave) {
+                            const int s1 = (u + 1) & 1;
+                            if (u >= 1)
+                                ok = wt.wait(bars + CB_SFREE + s1, ((u - 1) >> 1) & 1) &&
+                                     wt.wait(bars + CB_DSFREE + s1, ((u - 1) >> 1) & 1);
+                            if (ok) load_one(u + 1);
+                            ok = ok && lok;
+                        }
                     }
                     if (named_bar_or(BAR_CONV, 128, !ok || *abort_flag)) {
                         stop = true;
@@ -1088,71 +1208,13 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             if (*abort_flag && leader) {
                 mma_commit(bars + CB_DRAIN + 1);
                 mbar_wait(bars + CB_DRAIN + 1, 0, kWaitLimit);
+                for (int s2 = 0; s2 < 2; ++s2)
+                    if (issued[s2] > 0)
+                        mbar_wait(bars + CB_FULL + s2, (uint32_t)((issued[s2] - 1) & 1), kWaitLimit);
             }
         } else {
-            // ---- output warps: D_O = o^T (lane j = value channel, columns =
-            //      tokens).  Lane 0 of warp 12 is also the loader: the ring slot and
-            //      the V tile of chunk u + 2 go into stage u % 2 once chunk u is out
-            //      of it; the slot is given back (cons) once its loads have landed,
-            //      checked at the loader's next step.
+            // ---- output warps: D_O = o^T (lane j = value channel, columns = tokens)
             const int j = 32 * (warp & 3) + lane;
-            const bool loader = warp == 12 && lane == 0;
-            uint64_t *fl = p.flags + (size_t)b * 8;
-            // loader state: next chunk to load (lu, of chain lrho, chunk lm), and
-            // the cons value waiting for the stage of chunk pend_u to land
-            uint32_t lu = 0;
-            int lrho = 0, lm = 0;
-            Chain lcc;
-            bool lhave = false;
-            long long pend_u = -1;
-            uint64_t pend_val = 0;
-            bool lok = true;
-            auto flush = [&]() {
-                if (pend_u < 0) return;
-                const int s2 = (int)(pend_u & 1);
-                if (lok) lok = wt.wait(bars + CB_FULL + s2, (uint32_t)((pend_u >> 1) & 1));
-                if (lok) st_release_u64(fl, pend_val);
-                pend_u = -1;
-            };
-            // the next chain with chunks from round lrho on (empty ones are passed
-            // at once: their chain CTA has nothing to read)
-            auto lopen = [&]() {
-                for (;; ++lrho) {
-                    lhave = chain_of(lrho, &lcc);
-                    if (!lhave || lcc.nck > 0) return;
-                    flush();
-                    if (lok) st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
-                }
-            };
-            // issue the loads of chunk lu into its stage (the stage is free)
-            auto load_one = [&]() {
-                const int s2 = lu & 1;
-                uint8_t *stage = sm + s2 * CS_STAGE;
-                if (lok) lok = wt.wait_global(fl + 1 + (lm % NR), ready_tag(lrho, lm), true);
-                if (!lok) return;
-                fence_proxy_async_global();
-                const uint8_t *src = p.ring + ((size_t)b * NR + (lm % NR)) * RING_STRIDE;
-                const long long t0 = lcc.t_begin + (long long)lm * C;
-                mbar_arrive_expect_tx(bars + CB_FULL + s2, STAGE_TX);
-                bulk_load(stage, src, RG_PART1, bars + CB_FULL + s2);
-                bulk_load(stage + CS_QH, src + RG_QH, RG_PART2, bars + CB_FULL + s2);
-                tma_load_3d(stage + CS_V, &tm_v, 0, lcc.h, (int)t0, bars + CB_FULL + s2);
-                tma_load_3d(stage + CS_V + 8192, &tm_v, 64, lcc.h, (int)t0, bars + CB_FULL + s2);
-                ++issued[s2];
-                flush();
-                pend_u = lu;
-                pend_val = cons_after(lrho, lm, lcc.nck);
-                ++lu;
-                if (++lm == lcc.nck) {
-                    lm = 0;
-                    ++lrho;
-                    lopen();
-                }
-            };
-            if (loader) {
-                lopen();
-                for (int q = 0; q < 2 && lhave && lok; ++q) load_one();
-            }
             uint32_t u = 0;
             bool stop = false;
             for (int rho = 0; !stop; ++rho) {
@@ -1187,27 +1249,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                                                           (j & ~1)) = v;
                         }
                     }
-                    // chunk u is out of stage u % 2 once its products are done (the
-                    // output product was the last) and the state warps have read its
-                    // decay: chunk u + 2 may go in
-                    if (loader && lhave && lok) {
-                        const int s2 = u & 1;
-                        lok = wt.wait(bars + CB_SFREE + s2, (u >> 1) & 1) &&
-                              wt.wait(bars + CB_DSFREE + s2, (u >> 1) & 1);
-                        if (lok) load_one();
-                    }
-                    if (__shfl_sync(0xffffffffu, (loader && !lok) ? 1 : 0, 0)) {
-                        stop = true;
-                        break;
-                    }
                 }
-            }
-            if (loader) {
-                flush();
-                if (*abort_flag)
-                    for (int s2 = 0; s2 < 2; ++s2)
-                        if (issued[s2] > 0)
-                            mbar_wait(bars + CB_FULL + s2, (uint32_t)((issued[s2] - 1) & 1), kWaitLimit);
             }
         }
     }
@@ -1374,8 +1416,11 @@ cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launche
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(chunk_pool_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        SMEM_BYTES);
+        attr_err = cudaFuncSetAttribute(chunk_pool_kernel<false>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(chunk_pool_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return attr_err;
     cudaLaunchConfig_t cfg{};
@@ -1388,7 +1433,8 @@ cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launche
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, chunk_pool_kernel, a, p, mq, mk, mv);
+    e = a.raw ? cudaLaunchKernelEx(&cfg, chunk_pool_kernel<true>, a, p, mq, mk, mv)
+              : cudaLaunchKernelEx(&cfg, chunk_pool_kernel<false>, a, p, mq, mk, mv);
     if (e != cudaSuccess) return e;
     if (launches) ++*launches;
     return cudaSuccess;

@@ -39,6 +39,11 @@ struct PrefillArgs {
     // CUDA-core kernel only: if set, process only the (sequence, head) items
     // with redo[n * H + h] != 0 (the re-run of items another kernel flagged)
     const uint32_t *redo;
+    // fused input prologue (pool kernel): q, k unnormalised, log_alpha and beta
+    // hold the decay and writing-rate logits, alpha_bias [H] (or null) is added
+    // to the decay logit
+    int raw;
+    const float *alpha_bias;
 };
 
 struct DecodeArgs {

@@ -19,7 +19,8 @@ from dataclasses import dataclass, field
 import torch
 import torch.nn.functional as F
 
-__all__ = ["WORKLOADS", "Workload", "prefill_inputs", "decode_inputs", "varlen_lengths"]
+__all__ = ["WORKLOADS", "Workload", "prefill_inputs", "decode_inputs", "varlen_lengths",
+           "raw_prefill_inputs"]
 
 
 @dataclass(frozen=True)
@@ -132,3 +133,22 @@ def workload_inputs(name: str, **overrides) -> dict:
     return prefill_inputs(overrides.get("B", w.B), overrides.get("T", w.T), H, d, d,
                           dtype=w.dtype, decay=w.decay, alpha_shift=w.alpha_shift,
                           init_std=w.init_std, lengths=lengths, gen=g)
+
+
+def raw_prefill_inputs(B: int, T: int, H: int, d: int, *, seed: int = 0, bias: float = 2.0,
+                       dtype=torch.bfloat16) -> dict:
+    """Inputs of the fused entry point (gdn_chunk_fwd_raw) before any
+    normalisation: q_raw, k_raw ~ N(0,1) times a per-token scale in [0.5, 3.5];
+    v ~ N(0,1); decay and writing-rate logits ~ N(0,1); a per-head decay bias
+    (``bias``, so that the decay has the distribution of the prefill workloads).
+    Draw order: q scale, q, k scale, k, v, decay logits, rate logits."""
+    g = torch.Generator().manual_seed(seed)
+    qs = 0.5 + 3.0 * torch.rand(B, T, H, 1, generator=g)
+    q = (torch.randn(B, T, H, d, generator=g) * qs).to(dtype)
+    ks = 0.5 + 3.0 * torch.rand(B, T, H, 1, generator=g)
+    k = (torch.randn(B, T, H, d, generator=g) * ks).to(dtype)
+    v = torch.randn(B, T, H, d, generator=g).to(dtype)
+    a = torch.randn(B, T, H, generator=g)
+    b = torch.randn(B, T, H, generator=g)
+    return dict(q_raw=q, k_raw=k, v=v, alpha_logit=a, beta_logit=b,
+                alpha_bias=torch.full((H,), float(bias)))

@@ -131,6 +131,31 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
                          void *o, float *final_state,
                          void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
+/* gdn_chunk_fwd with the input prologue fused into the kernel: the queries
+ * and keys arrive unnormalised and the gates as logits, and the kernel applies
+ * (FG2-GDN section 3.5, "Gate Parameterization")
+ *   q_t <- q_t / ||q_t||,  k_t <- k_t / ||k_t||   (per token and head, norms in
+ *                                                  fp32, clamped below at 1e-12)
+ *   beta_t = sigmoid(beta_logit_t)
+ *   log alpha_t = -softplus(alpha_logit_t + alpha_bias[h])
+ * before the chunkwise pass, without writing the normalised inputs or the
+ * gates anywhere: the norms become row and column scales of the chunk
+ * products.  The result equals gdn_chunk_fwd on the prologue's outputs up to
+ * rounding (the normalised vectors are never rounded to bf16 here).
+ *   q_raw, k_raw     [B,T,H,d_k] bf16, unnormalised
+ *   alpha_logit      [B,T,H] fp32;  alpha_bias [H] fp32 or NULL (zero)
+ *   beta_logit       [B,T,H] fp32
+ *   everything else  as for gdn_chunk_fwd; the workspace is that of
+ *                    gdn_chunk_fwd_workspace_size for the same dims with
+ *                    flags = GDN_FLAG_POOL
+ * Scalar decay, bf16, d_k = d_v = 128 only (the pool kernel); other shapes
+ * return GDN_ERR_UNSUPPORTED.  dims->flags must be 0 or GDN_FLAG_POOL. */
+gdn_status gdn_chunk_fwd_raw(const gdn_dims *dims, const void *q_raw, const void *k_raw,
+                             const void *v, const float *alpha_logit, const float *alpha_bias,
+                             const float *beta_logit, const float *initial_state,
+                             const int32_t *cu_seqlens, void *o, float *final_state,
+                             void *workspace, size_t workspace_bytes, gdn_stream_t stream);
+
 /* One recurrent decode step for N = dims->B sequences (dims->T is ignored,
  * one token each): for every (sequence, head), with the state updated in place,
  *   S <- S Diag(alpha) (I - beta k k^T) + beta v k^T   (scalar alpha for GDN)

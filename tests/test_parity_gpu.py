@@ -391,3 +391,72 @@ def test_decode_matches_prefill(cuda_ok):
     torch.cuda.synchronize()
     assert rel_err(torch.stack(outs).transpose(0, 1), o.float().cpu().numpy()) < 2e-2
     assert rel_err(state, sf.cpu().numpy()) < 1e-2
+
+
+# --------------------------------------------------------------------------- #
+# the fused input prologue (gdn_chunk_fwd_raw)                                #
+# --------------------------------------------------------------------------- #
+def _raw_problem(B, T, H, seed, lengths=None, zero_key=False):
+    """Unnormalised q, k (per-token scales 0.5..3.5), v, decay and writing-rate
+    logits ~ N(0,1), a per-head decay bias, an initial state."""
+    g = torch.Generator().manual_seed(seed)
+    cu = None
+    if lengths is not None:
+        B, T = 1, int(sum(lengths))
+        cu = torch.zeros(len(lengths) + 1, dtype=torch.int32)
+        cu[1:] = torch.cumsum(torch.tensor(lengths), 0).to(torch.int32)
+    n = B if cu is None else len(lengths)
+    scale = lambda: 0.5 + 3.0 * torch.rand(B, T, H, 1, generator=g)
+    q = (torch.randn(B, T, H, 128, generator=g) * scale()).to(torch.bfloat16)
+    k = (torch.randn(B, T, H, 128, generator=g) * scale()).to(torch.bfloat16)
+    if zero_key:
+        k[0, min(5, T - 1), 0] = 0
+    v = torch.randn(B, T, H, 128, generator=g).to(torch.bfloat16)
+    a = torch.randn(B, T, H, generator=g)
+    b = torch.randn(B, T, H, generator=g)
+    bias = torch.linspace(1.0, 3.0, H)
+    s0 = torch.randn(n, H, 128, 128, generator=g) * 0.05
+    return dict(q_raw=q, k_raw=k, v=v, a=a, b=b, bias=bias, s0=s0, cu=cu)
+
+
+@pytest.mark.parametrize("case", ["ragged", "packed", "zero_key", "no_bias"])
+def test_fused_prologue_matches_oracle(cuda_ok, case):
+    """chunk_fwd_raw against the oracle's prologue (FG2-GDN section 3.5: unit
+    q and k, sigmoid beta, -softplus decay with a bias) followed by its
+    recurrence; and against gdn_chunk_fwd on the prologue's outputs."""
+    from gated_delta_rule_140_b200 import chunk_fwd_raw
+    if case == "packed":
+        r = _raw_problem(0, 0, 3, 91, lengths=[0, 1, 63, 64, 65, 200, 0, 130, 700])
+    else:
+        r = _raw_problem(2, 229 if case != "no_bias" else 700, 3, 90, zero_key=case == "zero_key")
+    bias = None if case == "no_bias" else r["bias"]
+    q, k, la, beta = oracle.prologue(r["q_raw"], r["k_raw"], r["a"], r["b"], bias)
+    ro, rs = oracle.recurrent(q, k, r["v"], la, beta, r["s0"], r["cu"])
+    dv = lambda t: None if t is None else t.cuda()
+    o, sf = chunk_fwd_raw(dv(r["q_raw"]), dv(r["k_raw"]), dv(r["v"]), dv(r["a"]), dv(r["b"]),
+                          dv(bias), dv(r["s0"]), dv(r["cu"]), check=True)
+    torch.cuda.synchronize()
+    to, ts = TOL[torch.bfloat16]
+    eo, es = rel_err(o, ro), rel_err(sf, rs)
+    assert eo <= to and es <= ts, (eo, es)
+    # the unfused path on the prologue's outputs (q, k rounded to bf16 there)
+    t = lambda x, dt: torch.from_numpy(x).to(dt).cuda()
+    o2, sf2 = chunk_fwd(t(q, torch.bfloat16), t(k, torch.bfloat16), dv(r["v"]),
+                        t(la, torch.float32), t(beta, torch.float32), dv(r["s0"]), dv(r["cu"]),
+                        pool=True)
+    torch.cuda.synchronize()
+    assert rel_err(o, o2.double().cpu().numpy()) < 2e-2
+    assert rel_err(sf, sf2.cpu().numpy()) < 1e-2
+
+
+def test_fused_prologue_rejects_other_shapes(cuda_ok):
+    from gated_delta_rule_140_b200 import chunk_fwd_raw
+    r = _raw_problem(1, 64, 2, 92)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in r.items()}
+    with pytest.raises(nat.GdnError) as ei:  # channel decay
+        chunk_fwd_raw(d["q_raw"], d["k_raw"], d["v"], d["a"][..., None].expand(1, 64, 2, 128)
+                      .contiguous(), d["b"])
+    assert ei.value.status == nat.GDN_ERR_UNSUPPORTED
+    with pytest.raises(nat.GdnError) as ei:  # fp32
+        chunk_fwd_raw(d["q_raw"].float(), d["k_raw"].float(), d["v"].float(), d["a"], d["b"])
+    assert ei.value.status == nat.GDN_ERR_UNSUPPORTED
