@@ -64,22 +64,28 @@ constexpr int DK = 128, DV = 128;
 constexpr int kThreads = 512;                      // 16 warps
 constexpr long long kWaitLimit = kDefaultWaitLimit;  // drains after an abort
 constexpr int LDA = 68;                            // fp32 row stride of A / T
-constexpr int NR = 6;                              // ring slots per chain CTA
+constexpr int NR = 8;                              // ring slots per chain CTA
+constexpr int kFlagWords = 16;                     // per chain CTA: cons, ready[NR], pad
 
-// ---- ring slot (global) and chain-CTA stage (shared) layouts, bytes ----------
-// slot:  [T_b | -W0 | -W1 | Kt0 | Kt1] (5 x 8 KB) [Qh0 | Qh1 | R] (3 x 8 KB) [e^{g_C} x128]
-constexpr uint32_t RG_TB = 0, RG_MW = 8192, RG_KT = 24576, RG_QH = 40960, RG_R = 57344,
-                   RG_DEC = 65536, RG_PART1 = 40960, RG_PART2 = 65536 + 512 - 40960;
-constexpr uint32_t RING_STRIDE = 66560;
-// stage: the slot's first part at 0 (overlaid by Z^T at 0 and G^T = Y at 16 KB once
-// X is formed), its second part at CS_QH, then V (TMA, two 64-wide halves)
-constexpr uint32_t CS_TB = 0, CS_MW = 8192, CS_KT = 24576, CS_ZT = 0, CS_Y = 16384;
-constexpr uint32_t CS_QH = 49152, CS_R = 65536, CS_DEC = 73728, CS_V = 74752;
-constexpr uint32_t CS_STAGE = 91136;
-constexpr uint32_t CS_S = 2 * CS_STAGE;  // S bf16, K-major rows j, 2 atoms of 16 KB
-constexpr uint32_t STAGE_TX = RG_PART1 + RG_PART2 + 2 * 8192;
-static_assert(CS_QH + RG_PART2 == CS_DEC + 512 && CS_DEC + 512 <= CS_V &&
-              CS_V + 16384 <= CS_STAGE && CS_Y + 32768 <= CS_QH, "chain stage layout");
+// ---- ring slot (global) and chain-CTA buffers (shared), bytes ----------------
+// slot: the early part [e^{g_C} x128 (1 KB) | Z^T | Y0 | Y1] (16 KB tiles: 128 rows;
+// Y = G^T in two 64-wide atoms), read by V^T Z and S G; the late part [R | Qh0 |
+// Qh1] (8 KB tiles: 64 rows), read by the output product.  Every tile bf16,
+// K-major, 128-byte swizzled.  The chain CTA loads the early part into one of two
+// early buffers and the late part, with V (one TMA load of both 64-wide halves),
+// into one of three late buffers: the output product of a chunk runs after the
+// state product of the next one, so its operands live longer.
+constexpr uint32_t RG_DEC = 0, RG_ZT = 1024, RG_Y = 17408, RG_EARLY = 50176;
+constexpr uint32_t RG_R = RG_EARLY, RG_QH = RG_EARLY + 8192, RG_LATE = 24576;
+constexpr uint32_t RG_BYTES = RG_EARLY + RG_LATE;
+constexpr uint32_t RING_STRIDE = RG_BYTES;
+constexpr uint32_t CE_DEC = RG_DEC, CE_ZT = RG_ZT, CE_Y = RG_Y, CE_BYTES = RG_EARLY;
+constexpr uint32_t CL_R = 0, CL_QH = 8192, CL_V = RG_LATE, CL_BYTES = RG_LATE + 16384;
+constexpr int NE = 2, NL = 3;  // early / late buffers
+constexpr uint32_t OFF_EARLY = 0, OFF_LATE = NE * CE_BYTES;
+constexpr uint32_t LATE_TX = RG_LATE + 2 * 8192;
+static_assert((CE_ZT | CE_Y | CE_BYTES | CL_QH | CL_V | CL_BYTES) % 1024 == 0 &&
+              CE_Y + 32768 == CE_BYTES, "chain buffer layout");
 
 // ---- local-CTA layout (GDN) -------------------------------------------------
 // three raw tile buffers [K0 | Q0 | K1 | Q1] shared by the two groups (task k in
@@ -100,39 +106,44 @@ constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR
               GR_GAM = 576, GR_DEC = 640, GR_INVK = 768, GR_INVQ = 832;
 
 // ---- bookkeeping (same offset in both roles) --------------------------------
-constexpr uint32_t OFF_COMMON = CS_S + 32768;  // 215040
+constexpr uint32_t OFF_COMMON = OFF_LATE + NL * CL_BYTES;  // 223232
 static_assert(L_G0 + 2 * L_GSZ <= OFF_COMMON, "local shared memory layout");
-constexpr uint32_t CM_ABORT = 0, CM_TMEM = 8, CM_ISSUED = 16, CM_BARS = 64;
+constexpr uint32_t CM_ABORT = 0, CM_TMEM = 8, CM_ISSUED = 16, CM_BARS = 64;  // issued: 8 ints
 constexpr int NBARS = 24;
 // local CTAs of packed batches: the descriptors of their first kDescCache tasks
-constexpr int kDescCache = 512;
+constexpr int kDescCache = 256;
 constexpr uint32_t OFF_DESC = OFF_COMMON + 256;
 static_assert(CM_BARS + NBARS * 8 <= 256, "bookkeeping");
 constexpr uint32_t SMEM_USED = OFF_DESC + kDescCache * 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 // chain-CTA mbarriers
-constexpr int CB_FULL = 0, CB_SFREE = 2, CB_XFULL = 4, CB_DSFULL = 5, CB_DSFREE = 7,
-              CB_OFULL = 9, CB_OFREE = 10, CB_AISS = 11, CB_DRAIN = 13;
-static_assert(1 + NR <= 8, "flag words per chain CTA");
+constexpr int CB_EFULL = 0, CB_LFULL = 2, CB_LFREE = 5, CB_DSFULL = 8, CB_DSFREE = 10,
+              CB_OFULL = 12, CB_OFREE = 13, CB_AISS = 14, CB_DRAIN = 16;
+static_assert(1 + NR <= kFlagWords, "flag words per chain CTA");
 // local-CTA mbarriers (TMA: one per raw buffer)
-constexpr int LB_TMA = 0, LB_L = 3, LB_OFFSET = 5, LB_DRAIN = 6;
+constexpr int LB_TMA = 0, LB_L = 3, LB_OFFSET = 5, LB_DRAIN = 6, LB_X = 8;
 
-// TMEM columns.  Chain: D_S (2 x 128), X (192), D_O (64).  Local: per group 192.
-constexpr uint32_t TM_DS = 0, TM_X = 256, TM_O = 448;
-constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_GROUP = 192;
+// TMEM columns.  Chain: D_S (2 x 128), D_O (64), S as the bf16 A operand of the
+// state and output products (three buffers of 64 columns, two values per column:
+// the output product of chunk u - 1 still reads S_{u-1} while S_{u+1} is written).
+// Local: per group 256 (D_kq; D_ab, and X over D_ab and the 64 columns after it:
+// X of task k stays until task k + 2's inversion phase has converted it).
+constexpr uint32_t TM_DS = 0, TM_O = 256, TM_S = 320;
+constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_X = 64, TM_GROUP = 256;
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);    // [K;Q] K^T
 constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, true);  // [P;0][T_bg|T_b], [X1;X2] K
-constexpr uint32_t ID_X = idesc_bf16(128, 192, true, true);      // Kt^T [T_b | -W]
+constexpr uint32_t ID_X = idesc_bf16(128, 192, true, true);      // Kt^T [T_b | -W] (local)
 constexpr uint32_t ID_VZ = idesc_bf16(128, 128, true, false);    // V^T Z
 constexpr uint32_t ID_SG = idesc_bf16(128, 128, false, false);   // S G
 constexpr uint32_t ID_VR = idesc_bf16(128, 64, true, false);     // V^T R^T
 constexpr uint32_t ID_SQ = idesc_bf16(128, 64, false, false);    // S Qh^T
 
 // named barriers
-constexpr int BAR_UPD = 5, BAR_CONV = 6;  // chain: state warps, X warps (local: 1-4)
+constexpr int BAR_UPD = 5;  // chain: the state warps (local: 1-4 groups, 5-6 X conversion)
+constexpr int BAR_X = 5;
 
 struct PoolArgs {
     uint8_t *ring;         // nch x NR slots of RING_STRIDE bytes
@@ -365,7 +376,7 @@ struct Waiter {
 template <bool RAW>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v2) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -373,7 +384,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
     volatile int *abort_flag = reinterpret_cast<volatile int *>(cm + CM_ABORT);
     uint64_t *bars = reinterpret_cast<uint64_t *>(cm + CM_BARS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cm + CM_TMEM);
-    int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // [3] loads issued per buffer / stage
+    int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // loads issued per buffer
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool chain_role = (int)blockIdx.x < p.nch;
@@ -383,15 +394,15 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) {
             uint32_t cnt = 1;
-            if (chain_role && (i == CB_DSFREE || i == CB_DSFREE + 1)) cnt = 8;
+            if (chain_role && (i == CB_DSFREE || i == CB_DSFREE + 1)) cnt = 8;  // state warps
             if (chain_role && i == CB_OFREE) cnt = 4;
             mbar_init(bars + i, cnt);
         }
         fence_mbar_init();
         *abort_flag = 0;
-        issued[0] = issued[1] = issued[2] = 0;
+        for (int i = 0; i < 8; ++i) issued[i] = 0;
         if (chain_role) {
-            tma_prefetch_desc(&tm_v);
+            tma_prefetch_desc(&tm_v2);
         } else {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
@@ -431,22 +442,55 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             uint8_t *pzt = grp + L_PZT;
             float *AT = reinterpret_cast<float *>(grp + L_AT);
             uint64_t *bar_l = bars + LB_L + g;
+            // the X product completes on a barrier of its own: it and the next task's
+            // first product are both in flight before either is waited for, and two
+            // phases of one barrier completing before a wait would look like none
+            uint64_t *bar_x = bars + LB_X + g;
             const uint32_t tm_kq = tmem + g * TM_GROUP + TM_KQ, tm_ab = tmem + g * TM_GROUP + TM_AB;
+            const uint32_t tm_x = tmem + g * TM_GROUP + TM_X;
+            // the group's task whose X product is issued but not yet converted (-1: none)
+            int xk = -1;
             const uint32_t lane_off = (uint32_t)(32 * lq) << 16;
             const uint64_t d_pz = desc_sw128(gbase + L_PZT + PZ_P, 16, 1024);                // [P; X1]
             const uint64_t d_x1b = desc_sw128(gbase + L_PZT + PZ_X1, PZ_X3 - PZ_X1, 1024);  // X1 | X3
             const uint64_t d_x1x2 = desc_sw128(gbase + L_PZT + PZ_X1, 16, 1024);            // [X1; X2]
-            uint32_t bl_wait = 0;
+            uint32_t bl_wait = 0, bx_wait = 0;
             const bool issuer = gtid == 0;       // MMAs
-            const bool storer = gtid == 7 * 32;  // tile loads, ring stores and the hand-off
-            bool pend = false;                   // storer: a task's ring stores are in flight
-            uint64_t *pend_flag = nullptr;
-            uint64_t pend_tag = 0;
-            auto hand_over = [&]() {
-                bulk_wait_all();
-                fence_proxy_async_global();
-                st_release_u64(pend_flag, pend_tag);
-                pend = false;
+            const bool storer = gtid == 7 * 32;  // tile loads, the slot wait and the hand-off
+            // X of task xk -> Z^T (columns 0-63) and G^T = Y (64-191) of row n = 32 lq +
+            // lane, bf16, to the task's ring slot (K-major, 128-byte swizzled), by
+            // the 4 warps lw 4-7; then the storer hands the task over (its fence
+            // waits for the group's ring stores to reach L2)
+            auto convert_x = [&]() {
+                const Task tx = task(xk);
+                uint8_t *xs = p.ring + ((size_t)tx.b * NR + (tx.m % NR)) * RING_STRIDE;
+                const int n = 32 * lq + lane;
+                tc_fence_after();
+#pragma unroll 1
+                for (int hh = 0; hh < 4; ++hh) {
+                    float x[48];
+                    tmem_ld16(tm_x + lane_off + 48 * hh, x);
+                    tmem_ld16(tm_x + lane_off + 48 * hh + 16, x + 16);
+                    tmem_ld16(tm_x + lane_off + 48 * hh + 32, x + 32);
+                    tmem_wait_ld16(x);
+                    reg_fence16(x + 16);
+                    reg_fence16(x + 32);
+#pragma unroll
+                    for (int q6 = 0; q6 < 6; ++q6) {
+                        const int c0 = 48 * hh + 8 * q6;
+                        const uint32_t off = c0 < 64 ? RG_ZT + sw128(n, c0 >> 3)
+                                                     : RG_Y + ((c0 - 64) >> 6) * 16384 +
+                                                           sw128(n, ((c0 - 64) & 63) >> 3);
+                        *reinterpret_cast<uint4 *>(xs + off) = pack8(x + 8 * q6);
+                    }
+                }
+                tc_fence_before();
+                named_bar_sync(BAR_X + g, 128);
+                if (storer) {
+                    __threadfence();
+                    st_release_u64(p.flags + (size_t)tx.b * kFlagWords + 1 + (tx.m % NR),
+                                   ready_tag(tx.rho, tx.m));
+                }
             };
             // raw tiles of task k into buffer k % 3 (an empty task completes the
             // buffer's phase with a plain arrive)
@@ -545,6 +589,10 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
 
             for (int k = g; k < ntask; k += 2) {
                 const Task tk = task(k);
+                // this task's ring slot (chain CTA tk.b, slot tk.m % NR): every thread
+                // writes its part of the tiles there with plain 16-byte stores
+                uint8_t *slot = p.ring + ((size_t)tk.b * NR + (tk.m % NR)) * RING_STRIDE;
+                uint64_t *fl = p.flags + (size_t)tk.b * kFlagWords;
                 float *gr = gate_rows(k);
                 uint8_t *rawp = raw_of(k);
                 const uint32_t raw_s = smem_u32(rawp);
@@ -565,8 +613,11 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 if (issuer) ok = wt.wait(bars + LB_TMA + (k % 3), tma_phase(k));
                 if (L == 0) {
                     // empty padding task: only the duties other tasks rely on
+                    if (issuer && ok && xk >= 0) ok = wt.wait(bar_x, bx_wait & 1);
+                    if (xk >= 0) ++bx_wait;
                     if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-                    if (storer && pend) hand_over();
+                    if (xk >= 0 && lw >= 4) convert_x();
+                    xk = -1;
                     if (storer && k >= 2 && k + 1 < ntask) issue_tma(k + 1);
                     if (lw == 4 && k + 2 < ntask) compute_gates(k + 2);
                     if (g == 0 && k == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
@@ -600,8 +651,11 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                         mma_bf16(tm_kq, d_raw + off, d_raw + off, ID_KK, kk > 0);
                     }
                     mma_commit(bar_l);
-                    if (!RAW) ok = wt.wait(bar_l, bl_wait & 1);
                 }
+                // (this group's previous task's X product completes first, then D_kq)
+                if (!RAW && issuer && ok && xk >= 0) ok = wt.wait(bar_x, bx_wait & 1);
+                if (!RAW && xk >= 0) ++bx_wait;
+                if (!RAW && issuer && ok) ok = wt.wait(bar_l, bl_wait & 1);
                 if constexpr (RAW) {
                     // 1 / ||k_r||, 1 / ||q_r|| of the raw bf16 rows (norm clamped at
                     // 1e-12) while the product runs: thread pair per (tile, row)
@@ -617,16 +671,15 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     }
                     ss += __shfl_xor_sync(0xffffffffu, ss, 1);
                     if (at == 0) gr[(tsel ? GR_INVQ : GR_INVK) + r] = rsqrtf(fmaxf(ss, 1e-24f));
+                    if (issuer && ok && xk >= 0) ok = wt.wait(bar_x, bx_wait & 1);
+                    if (xk >= 0) ++bx_wait;
                     if (issuer && ok) ok = wt.wait(bar_l, bl_wait & 1);
                 }
                 ++bl_wait;
-                // the tiles that the A/P phase below rewrites went out first, as
-                // their own bulk group
-                if (storer && pend) bulk_wait_read_but_last();
-                // the raw buffer of this group's previous task (k - 2, read by its
-                // ring stores) takes task k + 1, the other group's next
-                if (storer && k >= 2 && k + 1 < ntask) issue_tma(k + 1);
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
+                // the raw buffer of this group's previous task (k - 2, an operand of its
+                // X product, complete now) takes task k + 1, the other group's next
+                if (storer && k >= 2 && k + 1 < ntask) issue_tma(k + 1);
                 tc_fence_after();
                 // ---- A rows (lanes 0-63) -> fp32 with beta; P rows (lanes 64-127) -> bf16
                 const float *gb = gr + GR_B;
@@ -671,7 +724,14 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 // ---- T = (I + A)^{-1} in place of A: lw 0-3; meanwhile lw 4 prepares
                 //      the group's next gates and the storer hands over its last task
                 if (lw >= 4) {
-                    if (storer && pend) hand_over();
+                    // the group's previous task's X product -> its ring slot, handed over
+                    if (xk >= 0) convert_x();
+                    // the slot's previous chunk must have been read by chain CTA b
+                    // before this task's first tile goes out (R, below)
+                    if (storer) {
+                        const uint64_t need = cons_needed(tk.rho, tk.m);
+                        if (need != 0) wt.wait_global(fl, need, false);
+                    }
                     if (lw == 4 && k + 2 < ntask) compute_gates(k + 2);
                 } else {
                     // (1) 16x16 diagonal blocks, right-looking forward substitution;
@@ -730,6 +790,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
                     AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
                 }
+                xk = -1;
                 if (named_bar_or(BAR_G, 256, *abort_flag)) break;
                 // (3) T_{H1,H0} = -T_{H1} (A_{H1,H0} T_{H0}), 32x32 blocks; warp lw owns
                 //     output rows 16(lw/4).., columns 8(lw%4)..
@@ -816,10 +877,10 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 ++bl_wait;
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 tc_fence_after();
-                // lw 0,1: P T_bg -> X2;  lw 4,5: R -> P's tile (P is consumed)
+                // lw 0,1: P T_bg -> X2;  lw 4,5: R -> the ring slot
                 if (lq < 2) {
                     const int r = 32 * lq + lane;
-                    uint8_t *dst = pzt + (lhalf == 0 ? PZ_X2 : PZ_P);
+                    uint8_t *dst = lhalf == 0 ? pzt + PZ_X2 : slot + RG_R;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         float x[32];
@@ -844,14 +905,14 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 ++bl_wait;
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
                 tc_fence_after();
-                // ---- -W (lanes 0-63) staged in A/T's space; Qh = gamma Q - P W (lanes
-                //      64-127) staged in X1/X2; Kt = kh . K in place of K.  The raw
-                //      tiles' Q is then free.
+                // ---- -W (lanes 0-63) into A/T's space and Kt = kh . K in place of K: the
+                //      operands of X below; Qh = gamma Q - P W (lanes 64-127) and e^{g_C}
+                //      straight to the ring slot
                 {
                     const int r = 32 * (lq & 1) + lane;
                     const float gam = gr[GR_GAM + r] * (RAW ? gr[GR_INVQ + r] : 1.f);
                     uint8_t *wst = grp + L_AT + lhalf * 8192;
-                    uint8_t *qst = pzt + (lhalf ? PZ_X2 : PZ_X1);
+                    uint8_t *qst = slot + RG_QH + lhalf * 8192;
                     const uint8_t *qt = rawp + lhalf * L_RAW_AC + 8192;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
@@ -888,42 +949,35 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                         for (int e = 0; e < 8; ++e) kv[e] *= sc;
                         *reinterpret_cast<uint4 *>(rawp + ac * L_RAW_AC + sw128(rr, j)) = pack8(kv);
                     }
+                    if (lw == 5)
+                        *reinterpret_cast<uint4 *>(slot + RG_DEC + 16 * lane) =
+                            *reinterpret_cast<const uint4 *>(gr + GR_DEC + 4 * lane);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
                 if (named_bar_or(BAR_G, 256, *abort_flag)) break;
-                if (storer) {
-                    // once chain CTA b has read the slot's previous chunk, the tiles and
-                    // e^{g_C} go out by bulk copy; the hand-off follows during the
-                    // group's next task (or after the loop)
-                    uint64_t *fl = p.flags + (size_t)tk.b * 8;
-                    const uint64_t need = cons_needed(tk.rho, tk.m);
-                    if (need == 0 || wt.wait_global(fl, need, false)) {
-                        uint8_t *slot = p.ring + ((size_t)tk.b * NR + (tk.m % NR)) * RING_STRIDE;
-                        // two bulk groups: first what the group's next task rewrites
-                        // early (-W in A's space and Kt in the raw buffer before the
-                        // A/P phase ... R in P's tile), then the rest
-                        const uint8_t *at8 = grp + L_AT;
-                        bulk_store(slot + RG_KT, rawp, 8192);
-                        bulk_store(slot + RG_KT + 8192, rawp + L_RAW_AC, 8192);
-                        bulk_store(slot + RG_MW, at8, 8192);
-                        bulk_store(slot + RG_MW + 8192, at8 + 8192, 8192);
-                        bulk_store(slot + RG_DEC, gr + GR_DEC, 512);
-                        bulk_store(slot + RG_R, pzt + PZ_P, 8192);
-                        bulk_commit();
-                        bulk_store(slot + RG_QH, pzt + PZ_X1, 8192);
-                        bulk_store(slot + RG_QH + 8192, pzt + PZ_X2, 8192);
-                        bulk_store(slot + RG_TB, pzt + PZ_X3, 8192);
-                        bulk_commit();
-                        pend = true;
-                        pend_flag = fl + 1 + (tk.m % NR);
-                        pend_tag = ready_tag(tk.rho, tk.m);
-                    }
+                // ---- X = Kt^T [T_b | -W] (M = d_k, N = 64 + 128) over D_ab and the 64
+                //      columns after it: row n holds Z^T (columns 0-63, Z = T_b^T Kt) and
+                //      G^T (64-191, G = -W^T Kt), the chain CTA's operands of V^T Z and
+                //      S G.  Issued here, converted during the group's next task --------
+                if (issuer) {
+                    tc_fence_after();
+                    const uint64_t d_tw = desc_sw128(gbase + L_PZT + PZ_X3, 8192, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < C / 16; ++kk)
+                        mma_bf16(tm_x, d_kmn + 128 * kk, d_tw + 128 * kk, ID_X, kk > 0);
+                    mma_commit(bar_x);
                 }
+                xk = k;
             }
-            if (storer && pend && !*abort_flag) hand_over();
-            // drain: every bulk copy and MMA this group issued
-            if (storer) bulk_wait_all();
+            // the last task's X product
+            if (xk >= 0 && !*abort_flag) {
+                bool ok = true;
+                if (issuer) ok = wt.wait(bar_x, bx_wait & 1);
+                ++bx_wait;
+                if (!named_bar_or(BAR_G, 256, !ok || *abort_flag) && lw >= 4) convert_x();
+            }
+            // drain: every MMA this group issued
             if (*abort_flag && issuer) {
                 mma_commit(bars + LB_DRAIN + g);
                 mbar_wait(bars + LB_DRAIN + g, 0, kWaitLimit);
@@ -950,10 +1004,10 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
         const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
         if (warp < 8) {
             // ---- state warps: row j = 32 (warp % 4) + lane, key columns 64 ch .. ------
+            //      S lives in fp32 registers and, as the bf16 A operand of S G and
+            //      S Qh^T, in tensor memory (this thread: packed columns 32 ch ..)
             const int ch = warp >> 2, j = 32 * (warp & 3) + lane;
             const bool leader = tid == 0;  // issues the chain and output products
-            uint8_t *stile = sm + CS_S + ch * 16384;
-            const uint64_t d_s = desc_sw128(sbase + CS_S, 16, 1024);
             float s_reg[64];
             auto load_s0 = [&](const Chain &cc) {
                 const size_t base = (((size_t)cc.n * H + cc.h) * DV + j) * DK + 64 * ch;
@@ -972,10 +1026,12 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     *reinterpret_cast<float4 *>(a.s_final + base + e) =
                         make_float4(s_reg[e], s_reg[e + 1], s_reg[e + 2], s_reg[e + 3]);
             };
-            auto write_stile = [&]() {
+            auto write_s_tmem = [&](uint32_t buf) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    *reinterpret_cast<uint4 *>(stile + sw128(j, cc)) = pack8(s_reg + 8 * cc);
+                for (int e = 0; e < 32; ++e) pk[e] = pack2(s_reg[2 * e], s_reg[2 * e + 1]);
+                tmem_st32(tmem + TM_S + 64 * buf + 32 * ch + lane_q, pk);
+                tmem_wait_st();
             };
             // the next chain with tokens, from round rho on: empty chains get their
             // final state (the initial one) here; returns false past the last chain
@@ -990,54 +1046,59 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             int rho = 0;
             Chain cur;
             bool have = open_chain(&rho, &cur);
-            if (have) write_stile();
-            fence_proxy_async_smem();
+            uint32_t u = 0;  // chunk counter over this CTA's chains
+            if (have) write_s_tmem(0);
             tc_fence_before();
             named_bar_sync(BAR_UPD, 256);
-            uint32_t u = 0;  // chunk counter over this CTA's chains
+            // D_O = V^T R^T + S Qh^T of chunk uc (late buffer uc % 3, S buffer uc % 3),
+            // once the output warps have read chunk uc - 1's
+            auto issue_output = [&](uint32_t uc) -> bool {
+                if (uc >= 1 && !wt.wait(bars + CB_OFREE, (uc - 1) & 1)) return false;
+                tc_fence_after();
+                const uint32_t lb = sbase + OFF_LATE + (uc % NL) * CL_BYTES;
+                const uint64_t d_v = desc_sw128(lb + CL_V, 8192, 1024);
+                const uint64_t d_r = desc_sw128(lb + CL_R, 16, 1024);
+                const uint64_t d_q = desc_sw128(lb + CL_QH, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < C / 16; ++kk)
+                    mma_bf16(tmem + TM_O, d_v + 128 * kk, d_r + 2 * kk, ID_VR, kk > 0);
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t off_q = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_S + 64 * (uc % 3) + 8 * kk, d_q + off_q, ID_SQ, 1);
+                }
+                mma_commit(bars + CB_OFULL);
+                mma_commit(bars + CB_LFREE + uc % NL);
+                return true;
+            };
             int m = 0;
             while (have) {
                 const int s = u & 1;
-                const uint32_t sb = sbase + s * CS_STAGE;
                 bool ok = true;
                 if (leader) {
-                    // D_S += S G (after D_S = V^T Z went out); then D_O = V^T R^T + S Qh^T
+                    // D_S += S G (after D_S = V^T Z went out); then the output product of
+                    // the previous chunk, behind it in the tensor pipe
                     ok = wt.wait(bars + CB_AISS + s, (u >> 1) & 1);
                     if (ok) {
                         tc_fence_after();
-                        const uint64_t d_y = desc_sw128(sb + CS_Y, 16, 1024);
+                        const uint64_t d_y = desc_sw128(sbase + OFF_EARLY + s * CE_BYTES + CE_Y, 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < DK / 16; ++kk) {
                             const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                            mma_bf16(tmem + TM_DS + 128 * s, d_s + off, d_y + off, ID_SG, 1);
+                            mma_bf16_ts(tmem + TM_DS + 128 * s, tmem + TM_S + 64 * (u % 3) + 8 * kk,
+                                        d_y + off, ID_SG, 1);
                         }
                         mma_commit(bars + CB_DSFULL + s);
                     }
-                    if (ok && u >= 1) ok = wt.wait(bars + CB_OFREE, (u - 1) & 1);
-                    if (ok) {
-                        tc_fence_after();
-                        const uint64_t d_v = desc_sw128(sb + CS_V, 8192, 1024);
-                        const uint64_t d_r = desc_sw128(sb + CS_R, 16, 1024);
-                        const uint64_t d_q = desc_sw128(sb + CS_QH, 16, 1024);
-#pragma unroll
-                        for (int kk = 0; kk < C / 16; ++kk)
-                            mma_bf16(tmem + TM_O, d_v + 128 * kk, d_r + 2 * kk, ID_VR, kk > 0);
-#pragma unroll
-                        for (int kk = 0; kk < DK / 16; ++kk) {
-                            const uint32_t off_s = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                            const uint32_t off_q = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                            mma_bf16(tmem + TM_O, d_s + off_s, d_q + off_q, ID_SQ, 1);
-                        }
-                        mma_commit(bars + CB_OFULL);
-                        mma_commit(bars + CB_SFREE + s);
-                    }
+                    if (ok && u >= 1) ok = issue_output(u - 1);
                 }
                 // S <- e^{g_C} S + D_S (columns of this thread's half)
                 const bool okd = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
                                  wt.warp_wait(bars + CB_DSFULL + s, (u >> 1) & 1, lane);
                 if (okd) {
                     tc_fence_after();
-                    const float *dec = reinterpret_cast<const float *>(sm + s * CS_STAGE + CS_DEC) + 64 * ch;
+                    const float *dec =
+                        reinterpret_cast<const float *>(sm + OFF_EARLY + s * CE_BYTES + CE_DEC) + 64 * ch;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         float ds[16];
@@ -1052,10 +1113,8 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                             s_reg[16 * q4 + e + 3] = fmaf(dv.w, s_reg[16 * q4 + e + 3], ds[e + 3]);
                         }
                     }
-                }
-                // the output product reads the S tile: it must be done before the rewrite
-                const bool oko = okd && wt.warp_wait(bars + CB_OFULL, u & 1, lane);
-                if (oko) {
+                    // S_{u+1} into S buffer (u + 1) % 3: its last readers, the products of
+                    // chunk u - 2, are done (they precede S G of chunk u in the pipe)
                     if (m + 1 == cur.nck) {
                         store_sf(cur);
                         ++rho;
@@ -1064,153 +1123,121 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     } else {
                         ++m;
                     }
-                    if (have) write_stile();
+                    if (have) write_s_tmem((u + 1) % 3);
                 }
-                fence_proxy_async_smem();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bars + CB_DSFREE + s);
-                if (named_bar_or(BAR_UPD, 256, !oko || *abort_flag)) break;
+                if (named_bar_or(BAR_UPD, 256, !okd || *abort_flag)) break;
                 ++u;
+            }
+            // the output product of the last chunk
+            if (leader && u >= 1 && !*abort_flag && !have) {
+                if (!issue_output(u - 1)) {
+                    // (an expired wait: the abort below drains)
+                }
             }
             if (*abort_flag && leader) {
                 mma_commit(bars + CB_DRAIN);
                 mbar_wait(bars + CB_DRAIN, 0, kWaitLimit);
             }
         } else if (warp < 12) {
-            // ---- X warps: X = Kt^T [T_b | -W] -> Z^T, G^T (bf16, K-major rows n);
-            //      then D_S = V^T Z.  Lane 0 of warp 8 issues these products and is
-            //      also the loader: the ring slot and the V tile of chunk u + 1 go
-            //      into stage (u + 1) % 2 as soon as chunk u - 1 is out of it, and
-            //      the slot is given back (cons) as soon as they have landed.
-            const int n = 32 * (warp & 3) + lane;
-            const bool leader = warp == 8 && lane == 0;
-            uint64_t *fl = p.flags + (size_t)b * 8;
-            // loader cursor: the chain and chunk of the next load
-            int lrho = 0, lm = 0;
-            Chain lcc;
-            bool lhave = false;
-            bool lok = true;
-            // the next chain with chunks from round lrho on (an empty chain is
-            // passed at once: its chain CTA has nothing to read)
-            auto lopen = [&]() {
-                for (;; ++lrho) {
-                    lhave = chain_of(lrho, &lcc);
-                    if (!lhave || lcc.nck > 0) return;
-                    st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
-                }
-            };
-            // issue the loads of the cursor's chunk (global index lu) into its stage
-            auto load_one = [&](uint32_t lu) {
-                const int s2 = lu & 1;
-                uint8_t *stage = sm + s2 * CS_STAGE;
-                if (lok) lok = wt.wait_global(fl + 1 + (lm % NR), ready_tag(lrho, lm), true);
-                if (!lok) return;
-                fence_proxy_async_global();
-                const uint8_t *src = p.ring + ((size_t)b * NR + (lm % NR)) * RING_STRIDE;
-                const long long t0 = lcc.t_begin + (long long)lm * C;
-                mbar_arrive_expect_tx(bars + CB_FULL + s2, STAGE_TX);
-                bulk_load(stage, src, RG_PART1, bars + CB_FULL + s2);
-                bulk_load(stage + CS_QH, src + RG_QH, RG_PART2, bars + CB_FULL + s2);
-                tma_load_3d(stage + CS_V, &tm_v, 0, lcc.h, (int)t0, bars + CB_FULL + s2);
-                tma_load_3d(stage + CS_V + 8192, &tm_v, 64, lcc.h, (int)t0, bars + CB_FULL + s2);
-                ++issued[s2];
-                // the V tiles two chunks on, into L2
-                if (lm + 2 < lcc.nck) {
-                    tma_prefetch_l2_3d(&tm_v, 0, lcc.h, (int)(t0 + 2 * C));
-                    tma_prefetch_l2_3d(&tm_v, 64, lcc.h, (int)(t0 + 2 * C));
-                }
-            };
-            // after chunk lu has landed: give its slot back, move the cursor on
-            auto loaded = [&](uint32_t lu) {
-                st_release_u64(fl, cons_after(lrho, lm, lcc.nck));
-                if (++lm == lcc.nck) {
-                    lm = 0;
-                    ++lrho;
-                    lopen();
-                }
-            };
-            if (leader) {
+            // ---- lane 0 of warp 8: D_S = V^T Z for each chunk once its parts have
+            //      landed, and the loader: chunk u + 1's early part goes into early
+            //      buffer (u + 1) % 2 once chunk u - 1's state update is done, its late
+            //      part and V into late buffer (u + 1) % 3 once chunk u - 2's output
+            //      product is done; the ring slot is given back (cons) as soon as both
+            //      parts of a chunk have landed
+            if (warp == 8 && lane == 0) {
+                uint64_t *fl = p.flags + (size_t)b * kFlagWords;
+                int lrho = 0, lm = 0;  // loader cursor: the chain and chunk of the next load
+                Chain lcc;
+                bool lhave = false;
+                bool ok = true;
+                int *iss_e = issued, *iss_l = issued + NE;
+                // the next chain with chunks from round lrho on (an empty chain is
+                // passed at once: its chain CTA has nothing to read)
+                auto lopen = [&]() {
+                    for (;; ++lrho) {
+                        lhave = chain_of(lrho, &lcc);
+                        if (!lhave || lcc.nck > 0) return;
+                        st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
+                    }
+                };
+                // the loads of the cursor's chunk (global index lu); the buffers are free
+                auto load_one = [&](uint32_t lu) {
+                    if (ok) ok = wt.wait_global(fl + 1 + (lm % NR), ready_tag(lrho, lm), true);
+                    if (!ok) return;
+                    fence_proxy_async_global();
+                    const uint8_t *src = p.ring + ((size_t)b * NR + (lm % NR)) * RING_STRIDE;
+                    const long long t0 = lcc.t_begin + (long long)lm * C;
+                    const int e = lu % NE, l = lu % NL;
+                    uint8_t *eb = sm + OFF_EARLY + e * CE_BYTES, *lb = sm + OFF_LATE + l * CL_BYTES;
+                    mbar_arrive_expect_tx(bars + CB_EFULL + e, CE_BYTES);
+                    bulk_load(eb, src, CE_BYTES, bars + CB_EFULL + e);
+                    ++iss_e[e];
+                    // (late buffer lu % 3 last held chunk lu - 3: its output product done)
+                    if (lu >= NL && !wt.wait(bars + CB_LFREE + (lu - NL) % NL, ((lu - NL) / NL) & 1)) {
+                        ok = false;
+                        return;
+                    }
+                    mbar_arrive_expect_tx(bars + CB_LFULL + l, LATE_TX);
+                    bulk_load(lb, src + RG_EARLY, RG_LATE, bars + CB_LFULL + l);
+                    tma_load_4d(lb + CL_V, &tm_v2, 0, (int)t0, 0, lcc.h, bars + CB_LFULL + l);
+                    ++iss_l[l];
+                    // the V tile two chunks on, into L2
+                    if (lm + 2 < lcc.nck) tma_prefetch_l2_4d(&tm_v2, 0, (int)(t0 + 2 * C), 0, lcc.h);
+                };
+                // after both parts of the chunk have landed: give its slot back, move on
+                auto loaded = [&]() {
+                    st_release_u64(fl, cons_after(lrho, lm, lcc.nck));
+                    if (++lm == lcc.nck) {
+                        lm = 0;
+                        ++lrho;
+                        lopen();
+                    }
+                };
                 lopen();
                 if (lhave) load_one(0);
-            }
-            uint32_t u = 0;
-            bool stop = false;
-            for (int rho = 0; !stop; ++rho) {
-                Chain cc;
-                if (!chain_of(rho, &cc)) break;
-                for (int m = 0; m < cc.nck; ++m, ++u) {
-                    const int s = u & 1;
-                    const uint32_t sb = sbase + s * CS_STAGE;
-                    uint8_t *sp = sm + s * CS_STAGE;
-                    bool ok = lok;
-                    if (leader && ok) {
-                        ok = wt.wait(bars + CB_FULL + s, (u >> 1) & 1);
-                        if (ok) {
-                            loaded(u);
-                            tc_fence_after();
-                            const uint64_t d_kt = desc_sw128(sb + CS_KT, 8192, 1024);
-                            const uint64_t d_tw = desc_sw128(sb + CS_TB, 8192, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < C / 16; ++kk)
-                                mma_bf16(tmem + TM_X, d_kt + 128 * kk, d_tw + 128 * kk, ID_X, kk > 0);
-                            mma_commit(bars + CB_XFULL);
-                        }
-                    }
-                    const bool okx = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
-                                     wt.warp_wait(bars + CB_XFULL, u & 1, lane);
-                    if (okx) {
+                uint32_t u = 0;
+                for (int rho = 0; ok; ++rho) {
+                    Chain cc;
+                    if (!chain_of(rho, &cc)) break;
+                    for (int m = 0; m < cc.nck && ok; ++m, ++u) {
+                        const int s = u & 1;
+                        ok = wt.wait(bars + CB_EFULL + u % NE, (u / NE) & 1) &&
+                             wt.wait(bars + CB_LFULL + u % NL, (u / NL) & 1);
+                        if (!ok) break;
+                        loaded();
+                        if (u >= 2) ok = wt.wait(bars + CB_DSFREE + s, ((u >> 1) - 1) & 1);
+                        if (!ok) break;
                         tc_fence_after();
+                        const uint32_t lb = sbase + OFF_LATE + (u % NL) * CL_BYTES;
+                        const uint64_t d_v = desc_sw128(lb + CL_V, 8192, 1024);
+                        const uint64_t d_z = desc_sw128(sbase + OFF_EARLY + (u % NE) * CE_BYTES + CE_ZT, 16, 1024);
 #pragma unroll
-                        for (int q3 = 0; q3 < 3; ++q3) {  // columns 64 q3 .. : Z^T, G^T atom 0, 1
-                            float x[64];
-                            tmem_load<64>(tmem + TM_X + 64 * q3 + lane_q, x);
-                            uint8_t *dst = sp + (q3 == 0 ? CS_ZT : CS_Y + (q3 - 1) * 16384);
-#pragma unroll
-                            for (int cc2 = 0; cc2 < 8; ++cc2)
-                                *reinterpret_cast<uint4 *>(dst + sw128(n, cc2)) = pack8(x + 8 * cc2);
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    tc_fence_before();
-                    if (named_bar_or(BAR_CONV, 128, !okx || *abort_flag)) {
-                        stop = true;
-                        break;
-                    }
-                    if (leader) {
-                        ok = u < 2 || wt.wait(bars + CB_DSFREE + s, ((u >> 1) - 1) & 1);
-                        if (ok) {
-                            tc_fence_after();
-                            const uint64_t d_v = desc_sw128(sb + CS_V, 8192, 1024);
-                            const uint64_t d_z = desc_sw128(sb + CS_ZT, 16, 1024);
-#pragma unroll
-                            for (int kk = 0; kk < C / 16; ++kk)
-                                mma_bf16(tmem + TM_DS + 128 * s, d_v + 128 * kk, d_z + 2 * kk, ID_VZ, kk > 0);
-                            mbar_arrive(bars + CB_AISS + s);
-                        }
-                        // chunk u + 1 into the other stage once chunk u - 1 has left it
-                        // (its products done, its decay read by the state warps)
-                        if (ok && lhave) {
-                            const int s1 = (u + 1) & 1;
+                        for (int kk = 0; kk < C / 16; ++kk)
+                            mma_bf16(tmem + TM_DS + 128 * s, d_v + 128 * kk, d_z + 2 * kk, ID_VZ, kk > 0);
+                        mbar_arrive(bars + CB_AISS + s);
+                        // chunk u + 1: its early buffer is free once chunk u - 1's state
+                        // update is done (which follows its S G)
+                        if (lhave) {
                             if (u >= 1)
-                                ok = wt.wait(bars + CB_SFREE + s1, ((u - 1) >> 1) & 1) &&
-                                     wt.wait(bars + CB_DSFREE + s1, ((u - 1) >> 1) & 1);
+                                ok = wt.wait(bars + CB_DSFREE + ((u - 1) & 1), ((u - 1) >> 1) & 1);
                             if (ok) load_one(u + 1);
-                            ok = ok && lok;
                         }
-                    }
-                    if (named_bar_or(BAR_CONV, 128, !ok || *abort_flag)) {
-                        stop = true;
-                        break;
                     }
                 }
-            }
-            if (*abort_flag && leader) {
-                mma_commit(bars + CB_DRAIN + 1);
-                mbar_wait(bars + CB_DRAIN + 1, 0, kWaitLimit);
-                for (int s2 = 0; s2 < 2; ++s2)
-                    if (issued[s2] > 0)
-                        mbar_wait(bars + CB_FULL + s2, (uint32_t)((issued[s2] - 1) & 1), kWaitLimit);
+                if (*abort_flag) {
+                    mma_commit(bars + CB_DRAIN + 1);
+                    mbar_wait(bars + CB_DRAIN + 1, 0, kWaitLimit);
+                    for (int i = 0; i < NE; ++i)
+                        if (iss_e[i] > 0)
+                            mbar_wait(bars + CB_EFULL + i, (uint32_t)((iss_e[i] - 1) & 1), kWaitLimit);
+                    for (int i = 0; i < NL; ++i)
+                        if (iss_l[i] > 0)
+                            mbar_wait(bars + CB_LFULL + i, (uint32_t)((iss_l[i] - 1) & 1), kWaitLimit);
+                }
             }
         } else {
             // ---- output warps: D_O = o^T (lane j = value channel, columns = tokens)
@@ -1353,7 +1380,7 @@ PoolPlan plan_for(const gdn_dims &d, int nsm) {
     return pl;
 }
 
-constexpr size_t kFlagWordsPerChain = 8;
+constexpr size_t kFlagWordsPerChain = kFlagWords;
 
 size_t flags_bytes(int nch) { return (((size_t)nch * kFlagWordsPerChain + 8) * 8 + 255) & ~size_t(255); }
 
@@ -1393,7 +1420,7 @@ cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launche
     if (pl.nch <= 0) return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv;
     if (!make_tile_map(&mq, a.q, a.dk, a.H, ntok) || !make_tile_map(&mk, a.k, a.dk, a.H, ntok) ||
-        !make_tile_map(&mv, a.v, a.dv, a.H, ntok))
+        !make_halves_map(&mv, a.v, a.H, ntok))
         return cudaErrorInvalidValue;
     PoolArgs p{};
     uint8_t *ws = reinterpret_cast<uint8_t *>(a.scratch);

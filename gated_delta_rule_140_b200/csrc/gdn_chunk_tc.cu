@@ -750,6 +750,22 @@ bool make_tile_map(CUtensorMap *m, const void *base, int d, int H, long long nto
            CUDA_SUCCESS;
 }
 
+// [tokens, H, 128] bf16 viewed as a 4-D tensor (64, tokens, 2, H): one box
+// (64, 64, 2, 1) brings both 64-wide halves of a 64-token tile as two
+// consecutive 8 KB tiles, 128-byte swizzled (coordinates {0, t0, 0, h}).
+bool make_halves_map(CUtensorMap *m, const void *base, int H, long long ntok) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {64, (cuuint64_t)ntok, 2, (cuuint64_t)H};
+    cuuint64_t strides[3] = {(cuuint64_t)H * 256, 128, 256};
+    cuuint32_t box[4] = {64, 64, 2, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
 bool chunk_tc_supported(const gdn_dims &d) {
     return d.dtype == GDN_BF16 && d.d_k == DK && d.d_v == 128 && d.decay == GDN_DECAY_SCALAR &&
            (long long)d.B * d.T < (1LL << 31);

@@ -73,6 +73,9 @@ bool chunk_tc_supported(const gdn_dims &d);
 // [tokens, H, d] bf16 as a 3-D TMA tensor map (d, H, tokens), box 64 x 1 x 64,
 // 128-byte swizzle (defined with the single-CTA tensor-core kernel).
 bool make_tile_map(CUtensorMap *m, const void *base, int d, int H, long long ntok);
+// [tokens, H, 128] bf16 as a 4-D tensor map (64, tokens, 2, H), box 64 x 64 x 2 x 1:
+// both 64-wide halves of a 64-token tile in one load, two consecutive 8 KB tiles.
+bool make_halves_map(CUtensorMap *m, const void *base, int H, long long ntok);
 
 __device__ __forceinline__ long long data_wait_limit(const uint32_t *hdr) {
     const uint32_t w = hdr[1];
