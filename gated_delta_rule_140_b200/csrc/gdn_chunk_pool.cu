@@ -68,24 +68,21 @@ constexpr int NR = 8;                              // ring slots per chain CTA
 constexpr int kFlagWords = 16;                     // per chain CTA: cons, ready[NR], pad
 
 // ---- ring slot (global) and chain-CTA buffers (shared), bytes ----------------
-// slot: the early part [e^{g_C} x128 (1 KB) | Z^T | Y0 | Y1] (16 KB tiles: 128 rows;
-// Y = G^T in two 64-wide atoms), read by V^T Z and S G; the late part [R | Qh0 |
-// Qh1] (8 KB tiles: 64 rows), read by the output product.  Every tile bf16,
-// K-major, 128-byte swizzled.  The chain CTA loads the early part into one of two
-// early buffers and the late part, with V (one TMA load of both 64-wide halves),
-// into one of three late buffers: the output product of a chunk runs after the
-// state product of the next one, so its operands live longer.
-constexpr uint32_t RG_DEC = 0, RG_ZT = 1024, RG_Y = 17408, RG_EARLY = 50176;
-constexpr uint32_t RG_R = RG_EARLY, RG_QH = RG_EARLY + 8192, RG_LATE = 24576;
-constexpr uint32_t RG_BYTES = RG_EARLY + RG_LATE;
+// slot: [e^{g_C} x128 (1 KB) | Z^T | R] then two 64-wide atoms [Y_h | Qh_h] of
+// the key dimension (Y = G^T).  Z^T and Y have 128 rows (16 KB per atom), R and
+// Qh 64 rows (8 KB); every tile bf16, K-major, 128-byte swizzled, so that
+// [Z^T; R] (N = 192, K = 64 tokens) and [Y; Qh] (N = 192, K = d_k) are the B
+// operands of the chain CTA's two products V^T [Z | R^T] and S [Y^T | Qh^T]:
+// one accumulator holds the state increment (columns 0-127) and o^T (128-191).
+// The chain CTA loads a slot, and V (one TMA load of both 64-wide halves), into
+// one of two stages.
+constexpr uint32_t RG_DEC = 0, RG_ZT = 1024, RG_R = RG_ZT + 16384, RG_YQ = RG_R + 8192;
+constexpr uint32_t YQ_HALF = 24576, YQ_QH = 16384;  // atom stride; Qh inside an atom
+constexpr uint32_t RG_BYTES = RG_YQ + 2 * YQ_HALF;
 constexpr uint32_t RING_STRIDE = RG_BYTES;
-constexpr uint32_t CE_DEC = RG_DEC, CE_ZT = RG_ZT, CE_Y = RG_Y, CE_BYTES = RG_EARLY;
-constexpr uint32_t CL_R = 0, CL_QH = 8192, CL_V = RG_LATE, CL_BYTES = RG_LATE + 16384;
-constexpr int NE = 2, NL = 3;  // early / late buffers
-constexpr uint32_t OFF_EARLY = 0, OFF_LATE = NE * CE_BYTES;
-constexpr uint32_t LATE_TX = RG_LATE + 2 * 8192;
-static_assert((CE_ZT | CE_Y | CE_BYTES | CL_QH | CL_V | CL_BYTES) % 1024 == 0 &&
-              CE_Y + 32768 == CE_BYTES, "chain buffer layout");
+constexpr uint32_t CS_V = RG_BYTES, CS_BYTES = RG_BYTES + 16384;
+constexpr uint32_t STAGE_TX = CS_BYTES;
+static_assert((RG_ZT | RG_R | RG_YQ | YQ_HALF | YQ_QH | CS_V | CS_BYTES) % 1024 == 0, "chain buffer layout");
 
 // ---- local-CTA layout (GDN) -------------------------------------------------
 // three raw tile buffers [K0 | Q0 | K1 | Q1] shared by the two groups (task k in
@@ -106,40 +103,40 @@ constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR
               GR_GAM = 576, GR_DEC = 640, GR_INVK = 768, GR_INVQ = 832;
 
 // ---- bookkeeping (same offset in both roles) --------------------------------
-constexpr uint32_t OFF_COMMON = OFF_LATE + NL * CL_BYTES;  // 223232
-static_assert(L_G0 + 2 * L_GSZ <= OFF_COMMON, "local shared memory layout");
+constexpr uint32_t OFF_COMMON = L_G0 + 2 * L_GSZ;  // 212992
+static_assert(2 * CS_BYTES <= OFF_COMMON, "chain shared memory layout");
 constexpr uint32_t CM_ABORT = 0, CM_TMEM = 8, CM_ISSUED = 16, CM_BARS = 64;  // issued: 8 ints
 constexpr int NBARS = 24;
-// local CTAs of packed batches: the descriptors of their first kDescCache tasks
-constexpr int kDescCache = 256;
+// local CTAs: the descriptors of their first kDescCache tasks
+constexpr int kDescCache = 1024;
 constexpr uint32_t OFF_DESC = OFF_COMMON + 256;
 static_assert(CM_BARS + NBARS * 8 <= 256, "bookkeeping");
 constexpr uint32_t SMEM_USED = OFF_DESC + kDescCache * 16;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 // chain-CTA mbarriers
-constexpr int CB_EFULL = 0, CB_LFULL = 2, CB_LFREE = 5, CB_DSFULL = 8, CB_DSFREE = 10,
-              CB_OFULL = 12, CB_OFREE = 13, CB_AISS = 14, CB_DRAIN = 16;
+// (FULL: a stage's loads landed; DSFULL: a chunk's products done; DFREE: its
+// accumulator read by the 8 state and 4 output warps; AISS: V^T [Z | R^T] issued)
+constexpr int CB_FULL = 0, CB_DSFULL = 2, CB_DFREE = 4, CB_AISS = 6, CB_DRAIN = 8;
+constexpr uint32_t kDfreeCount = 12;
 static_assert(1 + NR <= kFlagWords, "flag words per chain CTA");
 // local-CTA mbarriers (TMA: one per raw buffer)
 constexpr int LB_TMA = 0, LB_L = 3, LB_OFFSET = 5, LB_DRAIN = 6, LB_X = 8;
 
-// TMEM columns.  Chain: D_S (2 x 128), D_O (64), S as the bf16 A operand of the
-// state and output products (three buffers of 64 columns, two values per column:
-// the output product of chunk u - 1 still reads S_{u-1} while S_{u+1} is written).
+// TMEM columns.  Chain: two accumulators D = [D_S | D_O] of 192 columns, and S
+// as the bf16 A operand of S [Y^T | Qh^T] (two buffers of 64 columns, two values
+// per column: S_{u+1} is written while chunk u's product may still read S_u).
 // Local: per group 256 (D_kq; D_ab, and X over D_ab and the 64 columns after it:
 // X of task k stays until task k + 2's inversion phase has converted it).
-constexpr uint32_t TM_DS = 0, TM_O = 256, TM_S = 320;
+constexpr uint32_t TM_D = 0, TM_DSTRIDE = 192, TM_O = 128, TM_S = 384;
 constexpr uint32_t TM_KQ = 0, TM_AB = 64, TM_X = 64, TM_GROUP = 256;
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t ID_KK = idesc_bf16(128, 64, false, false);    // [K;Q] K^T
 constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, true);  // [P;0][T_bg|T_b], [X1;X2] K
 constexpr uint32_t ID_X = idesc_bf16(128, 192, true, true);      // Kt^T [T_b | -W] (local)
-constexpr uint32_t ID_VZ = idesc_bf16(128, 128, true, false);    // V^T Z
-constexpr uint32_t ID_SG = idesc_bf16(128, 128, false, false);   // S G
-constexpr uint32_t ID_VR = idesc_bf16(128, 64, true, false);     // V^T R^T
-constexpr uint32_t ID_SQ = idesc_bf16(128, 64, false, false);    // S Qh^T
+constexpr uint32_t ID_VZR = idesc_bf16(128, 192, true, false);   // V^T [Z | R^T]
+constexpr uint32_t ID_SYQ = idesc_bf16(128, 192, false, false);  // S [Y^T | Qh^T]
 
 // named barriers
 constexpr int BAR_UPD = 5;  // chain: the state warps (local: 1-4 groups, 5-6 X conversion)
@@ -394,8 +391,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
     if (tid == 0) {
         for (int i = 0; i < NBARS; ++i) {
             uint32_t cnt = 1;
-            if (chain_role && (i == CB_DSFREE || i == CB_DSFREE + 1)) cnt = 8;  // state warps
-            if (chain_role && i == CB_OFREE) cnt = 4;
+            if (chain_role && (i == CB_DFREE || i == CB_DFREE + 1)) cnt = kDfreeCount;
             mbar_init(bars + i, cnt);
         }
         fence_mbar_init();
@@ -420,15 +416,14 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
         const long long ntask_all = p.rbase ? p.rbase[p.nrounds] : p.ntask;
         const int ntask = c < ntask_all ? (int)((ntask_all - c + nloc - 1) / nloc) : 0;
         auto gid = [&](int k) -> long long { return (long long)c + (long long)k * nloc; };
-        // packed batches: this CTA's first task descriptors, looked up once
+        // this CTA's first kDescCache task descriptors, decoded once by all threads
+        // (the decode takes several 64-bit divisions, or a search of the rounds)
         int4 *sdesc = reinterpret_cast<int4 *>(sm + OFF_DESC);
-        if (p.rbase) {
-            for (int k = tid; k < min(ntask, kDescCache); k += kThreads)
-                sdesc[k] = pack_task(task_of(a, p, gid(k)));
-            __syncthreads();
-        }
+        for (int k = tid; k < min(ntask, kDescCache); k += kThreads)
+            sdesc[k] = pack_task(task_of(a, p, gid(k)));
+        __syncthreads();
         auto task = [&](int k) -> Task {
-            if (p.rbase && k < kDescCache) return unpack_task(sdesc[k]);
+            if (k < kDescCache) return unpack_task(sdesc[k]);
             return task_of(a, p, gid(k));
         };
         if (warp < 16) {
@@ -458,39 +453,62 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             const bool issuer = gtid == 0;       // MMAs
             const bool storer = gtid == 7 * 32;  // tile loads, the slot wait and the hand-off
             // X of task xk -> Z^T (columns 0-63) and G^T = Y (64-191) of row n = 32 lq +
-            // lane, bf16, to the task's ring slot (K-major, 128-byte swizzled), by
-            // the 4 warps lw 4-7; then the storer hands the task over (its fence
-            // waits for the group's ring stores to reach L2)
+            // lane, bf16, to the task's ring slot (K-major, 128-byte swizzled), by the
+            // 4 warps lw 4-7, 64 columns (one 128-byte row segment) at a time: each
+            // 8-lane group transposes its 8 rows x 8 16-byte chunks with three
+            // xor-shuffle stages, so that every store instruction writes whole
+            // 128-byte rows; then the storer hands the task over (the barrier
+            // orders the group's ring stores before its release)
             auto convert_x = [&]() {
                 const Task tx = task(xk);
                 uint8_t *xs = p.ring + ((size_t)tx.b * NR + (tx.m % NR)) * RING_STRIDE;
-                const int n = 32 * lq + lane;
+                const int j8 = lane & 7;
+                const int n0 = 32 * lq + (lane & ~7);
                 tc_fence_after();
 #pragma unroll 1
-                for (int hh = 0; hh < 4; ++hh) {
-                    float x[48];
-                    tmem_ld16(tm_x + lane_off + 48 * hh, x);
-                    tmem_ld16(tm_x + lane_off + 48 * hh + 16, x + 16);
-                    tmem_ld16(tm_x + lane_off + 48 * hh + 32, x + 32);
-                    tmem_wait_ld16(x);
-                    reg_fence16(x + 16);
-                    reg_fence16(x + 32);
+                for (int pass = 0; pass < 3; ++pass) {
+                    uint32_t w[32];
 #pragma unroll
-                    for (int q6 = 0; q6 < 6; ++q6) {
-                        const int c0 = 48 * hh + 8 * q6;
-                        const uint32_t off = c0 < 64 ? RG_ZT + sw128(n, c0 >> 3)
-                                                     : RG_Y + ((c0 - 64) >> 6) * 16384 +
-                                                           sw128(n, ((c0 - 64) & 63) >> 3);
-                        *reinterpret_cast<uint4 *>(xs + off) = pack8(x + 8 * q6);
+                    for (int hq = 0; hq < 2; ++hq) {
+                        float x[32];
+                        tmem_ld16(tm_x + lane_off + 64 * pass + 32 * hq, x);
+                        tmem_ld16(tm_x + lane_off + 64 * pass + 32 * hq + 16, x + 16);
+                        tmem_wait_ld16(x);
+                        reg_fence16(x + 16);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const uint4 v = pack8(x + 8 * c);
+                            w[16 * hq + 4 * c] = v.x; w[16 * hq + 4 * c + 1] = v.y;
+                            w[16 * hq + 4 * c + 2] = v.z; w[16 * hq + 4 * c + 3] = v.w;
+                        }
                     }
+                    // w[4c..] = chunk c of row n0 + j8  ->  w[4t..] = chunk j8 of row n0 + t
+#pragma unroll
+                    for (int bb = 1; bb < 8; bb <<= 1) {
+                        const bool hi = (lane & bb) != 0;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            if (c & bb) continue;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const uint32_t send = hi ? w[4 * c + e] : w[4 * (c | bb) + e];
+                                const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, bb);
+                                if (hi) w[4 * c + e] = recv;
+                                else w[4 * (c | bb) + e] = recv;
+                            }
+                        }
+                    }
+                    uint8_t *dst = xs + (pass == 0 ? RG_ZT : RG_YQ + (pass - 1) * YQ_HALF);
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        *reinterpret_cast<uint4 *>(dst + (n0 + t) * 128 + ((j8 ^ t) << 4)) =
+                            make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
                 }
                 tc_fence_before();
                 named_bar_sync(BAR_X + g, 128);
-                if (storer) {
-                    __threadfence();
+                if (storer)
                     st_release_u64(p.flags + (size_t)tx.b * kFlagWords + 1 + (tx.m % NR),
                                    ready_tag(tx.rho, tx.m));
-                }
             };
             // raw tiles of task k into buffer k % 3 (an empty task completes the
             // buffer's phase with a plain arrive)
@@ -912,7 +930,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     const int r = 32 * (lq & 1) + lane;
                     const float gam = gr[GR_GAM + r] * (RAW ? gr[GR_INVQ + r] : 1.f);
                     uint8_t *wst = grp + L_AT + lhalf * 8192;
-                    uint8_t *qst = slot + RG_QH + lhalf * 8192;
+                    uint8_t *qst = slot + RG_YQ + lhalf * YQ_HALF + YQ_QH;
                     const uint8_t *qt = rawp + lhalf * L_RAW_AC + 8192;
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
@@ -1002,12 +1020,13 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             return true;
         };
         const uint32_t lane_q = (uint32_t)(32 * (warp & 3)) << 16;
+        auto stage_of = [&](uint32_t u) -> uint8_t * { return sm + (u & 1) * CS_BYTES; };
         if (warp < 8) {
             // ---- state warps: row j = 32 (warp % 4) + lane, key columns 64 ch .. ------
-            //      S lives in fp32 registers and, as the bf16 A operand of S G and
-            //      S Qh^T, in tensor memory (this thread: packed columns 32 ch ..)
+            //      S lives in fp32 registers and, as the bf16 A operand of
+            //      S [Y^T | Qh^T], in tensor memory (this thread: packed columns 32 ch ..)
             const int ch = warp >> 2, j = 32 * (warp & 3) + lane;
-            const bool leader = tid == 0;  // issues the chain and output products
+            const bool leader = tid == 0;  // issues S [Y^T | Qh^T]
             float s_reg[64];
             auto load_s0 = [&](const Chain &cc) {
                 const size_t base = (((size_t)cc.n * H + cc.h) * DV + j) * DK + 64 * ch;
@@ -1033,6 +1052,13 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 tmem_st32(tmem + TM_S + 64 * buf + 32 * ch + lane_q, pk);
                 tmem_wait_st();
             };
+            // e^{g_C} of chunk u (scalar decay: every entry of the slot's row is the
+            // same), read once the stage has landed
+            auto read_dec = [&](uint32_t u, float *dC) -> bool {
+                if (!wt.warp_wait(bars + CB_FULL + (u & 1), (u >> 1) & 1, lane)) return false;
+                *dC = *reinterpret_cast<const volatile float *>(stage_of(u) + RG_DEC);
+                return true;
+            };
             // the next chain with tokens, from round rho on: empty chains get their
             // final state (the initial one) here; returns false past the last chain
             auto open_chain = [&](int *rho, Chain *cc) -> bool {
@@ -1047,74 +1073,51 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             Chain cur;
             bool have = open_chain(&rho, &cur);
             uint32_t u = 0;  // chunk counter over this CTA's chains
-            if (have) write_s_tmem(0);
+            float dC = 0.f;
+            bool okr = true;
+            if (have) {
+                write_s_tmem(0);
+                okr = read_dec(0, &dC);
+            }
             tc_fence_before();
-            named_bar_sync(BAR_UPD, 256);
-            // D_O = V^T R^T + S Qh^T of chunk uc (late buffer uc % 3, S buffer uc % 3),
-            // once the output warps have read chunk uc - 1's
-            auto issue_output = [&](uint32_t uc) -> bool {
-                if (uc >= 1 && !wt.wait(bars + CB_OFREE, (uc - 1) & 1)) return false;
-                tc_fence_after();
-                const uint32_t lb = sbase + OFF_LATE + (uc % NL) * CL_BYTES;
-                const uint64_t d_v = desc_sw128(lb + CL_V, 8192, 1024);
-                const uint64_t d_r = desc_sw128(lb + CL_R, 16, 1024);
-                const uint64_t d_q = desc_sw128(lb + CL_QH, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < C / 16; ++kk)
-                    mma_bf16(tmem + TM_O, d_v + 128 * kk, d_r + 2 * kk, ID_VR, kk > 0);
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t off_q = ((kk >> 2) * 8192 + (kk & 3) * 32) >> 4;
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_S + 64 * (uc % 3) + 8 * kk, d_q + off_q, ID_SQ, 1);
-                }
-                mma_commit(bars + CB_OFULL);
-                mma_commit(bars + CB_LFREE + uc % NL);
-                return true;
-            };
+            const bool bad0 = named_bar_or(BAR_UPD, 256, !okr);
             int m = 0;
-            while (have) {
+            while (have && !bad0) {
                 const int s = u & 1;
                 bool ok = true;
                 if (leader) {
-                    // D_S += S G (after D_S = V^T Z went out); then the output product of
-                    // the previous chunk, behind it in the tensor pipe
+                    // D[s] += S_u [Y^T | Qh^T] (after D[s] = V^T [Z | R^T] went out)
                     ok = wt.wait(bars + CB_AISS + s, (u >> 1) & 1);
                     if (ok) {
                         tc_fence_after();
-                        const uint64_t d_y = desc_sw128(sbase + OFF_EARLY + s * CE_BYTES + CE_Y, 16, 1024);
+                        const uint64_t d_yq = desc_sw128(smem_u32(stage_of(u) + RG_YQ), 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < DK / 16; ++kk) {
-                            const uint32_t off = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
-                            mma_bf16_ts(tmem + TM_DS + 128 * s, tmem + TM_S + 64 * (u % 3) + 8 * kk,
-                                        d_y + off, ID_SG, 1);
+                            const uint32_t off = ((kk >> 2) * YQ_HALF + (kk & 3) * 32) >> 4;
+                            mma_bf16_ts(tmem + TM_D + TM_DSTRIDE * s, tmem + TM_S + 64 * s + 8 * kk,
+                                        d_yq + off, ID_SYQ, 1);
                         }
                         mma_commit(bars + CB_DSFULL + s);
                     }
-                    if (ok && u >= 1) ok = issue_output(u - 1);
                 }
                 // S <- e^{g_C} S + D_S (columns of this thread's half)
-                const bool okd = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
-                                 wt.warp_wait(bars + CB_DSFULL + s, (u >> 1) & 1, lane);
+                bool okd = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 &&
+                           wt.warp_wait(bars + CB_DSFULL + s, (u >> 1) & 1, lane);
                 if (okd) {
                     tc_fence_after();
-                    const float *dec =
-                        reinterpret_cast<const float *>(sm + OFF_EARLY + s * CE_BYTES + CE_DEC) + 64 * ch;
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         float ds[16];
-                        tmem_ld16(tmem + TM_DS + 128 * s + 64 * ch + 16 * q4 + lane_q, ds);
+                        tmem_ld16(tmem + TM_D + TM_DSTRIDE * s + 64 * ch + 16 * q4 + lane_q, ds);
                         tmem_wait_ld16(ds);
 #pragma unroll
-                        for (int e = 0; e < 16; e += 4) {
-                            const float4 dv = *reinterpret_cast<const float4 *>(dec + 16 * q4 + e);
-                            s_reg[16 * q4 + e] = fmaf(dv.x, s_reg[16 * q4 + e], ds[e]);
-                            s_reg[16 * q4 + e + 1] = fmaf(dv.y, s_reg[16 * q4 + e + 1], ds[e + 1]);
-                            s_reg[16 * q4 + e + 2] = fmaf(dv.z, s_reg[16 * q4 + e + 2], ds[e + 2]);
-                            s_reg[16 * q4 + e + 3] = fmaf(dv.w, s_reg[16 * q4 + e + 3], ds[e + 3]);
-                        }
+                        for (int e = 0; e < 16; ++e) s_reg[16 * q4 + e] = fmaf(dC, s_reg[16 * q4 + e], ds[e]);
                     }
-                    // S_{u+1} into S buffer (u + 1) % 3: its last readers, the products of
-                    // chunk u - 2, are done (they precede S G of chunk u in the pipe)
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bars + CB_DFREE + s);
+                    // S_{u+1} into S buffer (u + 1) & 1: its last reader, chunk u - 1's
+                    // product, is done (this warp waited for it before chunk u - 1's update)
                     if (m + 1 == cur.nck) {
                         store_sf(cur);
                         ++rho;
@@ -1123,38 +1126,35 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     } else {
                         ++m;
                     }
-                    if (have) write_s_tmem((u + 1) % 3);
+                    if (have) {
+                        write_s_tmem((u + 1) & 1);
+                        // the next chunk's decay, read before the barrier below: the
+                        // stage is reloaded only after the next chunk's product, which
+                        // the leader issues after it
+                        okd = read_dec(u + 1, &dC);
+                    }
                 }
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bars + CB_DSFREE + s);
                 if (named_bar_or(BAR_UPD, 256, !okd || *abort_flag)) break;
                 ++u;
-            }
-            // the output product of the last chunk
-            if (leader && u >= 1 && !*abort_flag && !have) {
-                if (!issue_output(u - 1)) {
-                    // (an expired wait: the abort below drains)
-                }
             }
             if (*abort_flag && leader) {
                 mma_commit(bars + CB_DRAIN);
                 mbar_wait(bars + CB_DRAIN, 0, kWaitLimit);
             }
         } else if (warp < 12) {
-            // ---- lane 0 of warp 8: D_S = V^T Z for each chunk once its parts have
-            //      landed, and the loader: chunk u + 1's early part goes into early
-            //      buffer (u + 1) % 2 once chunk u - 1's state update is done, its late
-            //      part and V into late buffer (u + 1) % 3 once chunk u - 2's output
-            //      product is done; the ring slot is given back (cons) as soon as both
-            //      parts of a chunk have landed
+            // ---- lane 0 of warp 8: D[s] = V^T [Z | R^T] for each chunk once its
+            //      stage has landed and chunk u - 2's accumulator has been read, and
+            //      the loader: chunk u + 1 goes into stage (u + 1) & 1 once chunk
+            //      u - 1's products are done; the ring slot is given back (cons) as
+            //      soon as a chunk has landed
             if (warp == 8 && lane == 0) {
                 uint64_t *fl = p.flags + (size_t)b * kFlagWords;
                 int lrho = 0, lm = 0;  // loader cursor: the chain and chunk of the next load
                 Chain lcc;
                 bool lhave = false;
                 bool ok = true;
-                int *iss_e = issued, *iss_l = issued + NE;
+                int *iss = issued;
                 // the next chain with chunks from round lrho on (an empty chain is
                 // passed at once: its chain CTA has nothing to read)
                 auto lopen = [&]() {
@@ -1164,31 +1164,25 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                         st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
                     }
                 };
-                // the loads of the cursor's chunk (global index lu); the buffers are free
+                // the loads of the cursor's chunk (global index lu) into its stage (free)
                 auto load_one = [&](uint32_t lu) {
                     if (ok) ok = wt.wait_global(fl + 1 + (lm % NR), ready_tag(lrho, lm), true);
                     if (!ok) return;
                     fence_proxy_async_global();
                     const uint8_t *src = p.ring + ((size_t)b * NR + (lm % NR)) * RING_STRIDE;
                     const long long t0 = lcc.t_begin + (long long)lm * C;
-                    const int e = lu % NE, l = lu % NL;
-                    uint8_t *eb = sm + OFF_EARLY + e * CE_BYTES, *lb = sm + OFF_LATE + l * CL_BYTES;
-                    mbar_arrive_expect_tx(bars + CB_EFULL + e, CE_BYTES);
-                    bulk_load(eb, src, CE_BYTES, bars + CB_EFULL + e);
-                    ++iss_e[e];
-                    // (late buffer lu % 3 last held chunk lu - 3: its output product done)
-                    if (lu >= NL && !wt.wait(bars + CB_LFREE + (lu - NL) % NL, ((lu - NL) / NL) & 1)) {
-                        ok = false;
-                        return;
-                    }
-                    mbar_arrive_expect_tx(bars + CB_LFULL + l, LATE_TX);
-                    bulk_load(lb, src + RG_EARLY, RG_LATE, bars + CB_LFULL + l);
-                    tma_load_4d(lb + CL_V, &tm_v2, 0, (int)t0, 0, lcc.h, bars + CB_LFULL + l);
-                    ++iss_l[l];
+                    uint8_t *st = stage_of(lu);
+                    uint64_t *bf = bars + CB_FULL + (lu & 1);
+                    mbar_arrive_expect_tx(bf, STAGE_TX);
+                    bulk_load(st, src, RG_YQ, bf);
+                    bulk_load(st + RG_YQ, src + RG_YQ, YQ_HALF, bf);
+                    bulk_load(st + RG_YQ + YQ_HALF, src + RG_YQ + YQ_HALF, YQ_HALF, bf);
+                    tma_load_4d(st + CS_V, &tm_v2, 0, (int)t0, 0, lcc.h, bf);
+                    ++iss[lu & 1];
                     // the V tile two chunks on, into L2
                     if (lm + 2 < lcc.nck) tma_prefetch_l2_4d(&tm_v2, 0, (int)(t0 + 2 * C), 0, lcc.h);
                 };
-                // after both parts of the chunk have landed: give its slot back, move on
+                // after the chunk has landed: give its slot back, move on
                 auto loaded = [&]() {
                     st_release_u64(fl, cons_after(lrho, lm, lcc.nck));
                     if (++lm == lcc.nck) {
@@ -1205,25 +1199,24 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     if (!chain_of(rho, &cc)) break;
                     for (int m = 0; m < cc.nck && ok; ++m, ++u) {
                         const int s = u & 1;
-                        ok = wt.wait(bars + CB_EFULL + u % NE, (u / NE) & 1) &&
-                             wt.wait(bars + CB_LFULL + u % NL, (u / NL) & 1);
+                        ok = wt.wait(bars + CB_FULL + s, (u >> 1) & 1);
                         if (!ok) break;
                         loaded();
-                        if (u >= 2) ok = wt.wait(bars + CB_DSFREE + s, ((u >> 1) - 1) & 1);
+                        if (u >= 2) ok = wt.wait(bars + CB_DFREE + s, ((u >> 1) - 1) & 1);
                         if (!ok) break;
                         tc_fence_after();
-                        const uint32_t lb = sbase + OFF_LATE + (u % NL) * CL_BYTES;
-                        const uint64_t d_v = desc_sw128(lb + CL_V, 8192, 1024);
-                        const uint64_t d_z = desc_sw128(sbase + OFF_EARLY + (u % NE) * CE_BYTES + CE_ZT, 16, 1024);
+                        const uint32_t sb = smem_u32(stage_of(u));
+                        const uint64_t d_v = desc_sw128(sb + CS_V, 8192, 1024);
+                        const uint64_t d_zr = desc_sw128(sb + RG_ZT, 16, 1024);
 #pragma unroll
                         for (int kk = 0; kk < C / 16; ++kk)
-                            mma_bf16(tmem + TM_DS + 128 * s, d_v + 128 * kk, d_z + 2 * kk, ID_VZ, kk > 0);
+                            mma_bf16(tmem + TM_D + TM_DSTRIDE * s, d_v + 128 * kk, d_zr + 2 * kk, ID_VZR, kk > 0);
                         mbar_arrive(bars + CB_AISS + s);
-                        // chunk u + 1: its early buffer is free once chunk u - 1's state
-                        // update is done (which follows its S G)
+                        // chunk u + 1's stage held chunk u - 1: free once its products are
+                        // done (its decay was read before chunk u's product went out)
                         if (lhave) {
                             if (u >= 1)
-                                ok = wt.wait(bars + CB_DSFREE + ((u - 1) & 1), ((u - 1) >> 1) & 1);
+                                ok = wt.wait(bars + CB_DSFULL + ((u - 1) & 1), ((u - 1) >> 1) & 1);
                             if (ok) load_one(u + 1);
                         }
                     }
@@ -1231,12 +1224,9 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 if (*abort_flag) {
                     mma_commit(bars + CB_DRAIN + 1);
                     mbar_wait(bars + CB_DRAIN + 1, 0, kWaitLimit);
-                    for (int i = 0; i < NE; ++i)
-                        if (iss_e[i] > 0)
-                            mbar_wait(bars + CB_EFULL + i, (uint32_t)((iss_e[i] - 1) & 1), kWaitLimit);
-                    for (int i = 0; i < NL; ++i)
-                        if (iss_l[i] > 0)
-                            mbar_wait(bars + CB_LFULL + i, (uint32_t)((iss_l[i] - 1) & 1), kWaitLimit);
+                    for (int i = 0; i < 2; ++i)
+                        if (iss[i] > 0)
+                            mbar_wait(bars + CB_FULL + i, (uint32_t)((iss[i] - 1) & 1), kWaitLimit);
                 }
             }
         } else {
@@ -1248,17 +1238,18 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 Chain cc;
                 if (!chain_of(rho, &cc)) break;
                 for (int m = 0; m < cc.nck; ++m, ++u) {
-                    const bool ok = wt.warp_wait(bars + CB_OFULL, u & 1, lane);
+                    const int s = u & 1;
+                    const bool ok = wt.warp_wait(bars + CB_DSFULL + s, (u >> 1) & 1, lane);
                     if (!ok) {
                         stop = true;
                         break;
                     }
                     tc_fence_after();
                     float x[64];
-                    tmem_load<64>(tmem + TM_O + lane_q, x);
+                    tmem_load<64>(tmem + TM_D + TM_DSTRIDE * s + TM_O + lane_q, x);
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(bars + CB_OFREE);
+                    if (lane == 0) mbar_arrive(bars + CB_DFREE + s);
                     const long long t0 = cc.t_begin + (long long)m * C;
                     const int L = (int)min((long long)C, cc.t_end - t0);
                     // lane pairs (j even, j + 1) write bf16 pairs: the even lane row r,
