@@ -60,6 +60,9 @@ def _bind(path):
     lib.oracle_gdn_prologue.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         _D, _D, _D, _D, _D, _D, _D, _D, _D]
     lib.oracle_gdn_prologue.restype = ctypes.c_int
+    lib.oracle_fg2_recurrent.argtypes = [ctypes.c_int, _I64, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int] + [_D] * 9 + [ctypes.c_int]
+    lib.oracle_fg2_recurrent.restype = ctypes.c_int
     return lib
 
 
@@ -150,6 +153,36 @@ def chunkwise(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, chu
     used = _load().oracle_gdn_chunkwise(n, starts.ctypes.data_as(_I64), H, dk, dv, int(channel),
                                         _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(s0),
                                         _ptr(o), _ptr(sf), int(chunk), int(nthreads))
+    if used < 0:
+        raise ValueError("oracle rejected its arguments")
+    return o, sf
+
+
+def fg2_recurrent(q, k, v, log_alpha, beta_k, beta_v=None, initial_state=None, cu_seqlens=None,
+                  nthreads=0):
+    """FG2-GDN (FG2-GDN paper, sections 3.2, 3.4, 3.6; the update's equations are
+    lost from the page): channel decay log_alpha [B,T,H,dk], key-side writing rate
+    beta_k [B,T,H,dk] and, for FG2-GDN+, a value-side rate beta_v [B,T,H,dv]
+    (None: FG2-GDN, no value gate).  Keys and values are scaled by the square
+    roots of their rates, k~ = sqrt(beta_k) . k and v~ = sqrt(beta_v) . v, and
+    S_t = S_{t-1} Diag(alpha_t) (I - k~ k~^T) + v~ k~^T,  o_t = S_t q_t, token by
+    token in fp64.  Returns (o, S_final) like ``recurrent``."""
+    bk = _f64(beta_k)
+    bv = _f64(beta_v)
+    dummy_beta = np.zeros(np.asarray(bk).shape[:3], np.float64)
+    q, k, v, la, _, s0, starts, (B, T, H, dk, dv, n, channel) = _problem(
+        q, k, v, log_alpha, dummy_beta, initial_state, cu_seqlens)
+    if not channel:
+        raise ValueError("FG2-GDN takes channel decay (log_alpha [B,T,H,dk])")
+    if bk.shape != (B, T, H, dk):
+        raise ValueError(f"beta_k must be {(B, T, H, dk)}, got {bk.shape}")
+    if bv is not None and bv.shape != (B, T, H, dv):
+        raise ValueError(f"beta_v must be {(B, T, H, dv)}, got {bv.shape}")
+    o = np.zeros((B, T, H, dv), np.float64)
+    sf = np.zeros((n, H, dv, dk), np.float64)
+    used = _load().oracle_fg2_recurrent(n, starts.ctypes.data_as(_I64), H, dk, dv, _ptr(q),
+                                        _ptr(k), _ptr(v), _ptr(la), _ptr(bk), _ptr(bv),
+                                        _ptr(s0), _ptr(o), _ptr(sf), int(nthreads))
     if used < 0:
         raise ValueError("oracle rejected its arguments")
     return o, sf

@@ -33,6 +33,18 @@
  * oracle_gdn_chunk_stage exposes one chunk's intermediates (g, A, T, W, U, V',
  * O, S_out) so the steps can be pinned one by one.
  *
+ * oracle_fg2_recurrent is FG2-GDN's channel-wise writing rate (FG2-GDN paper,
+ * section 3.2 "FG2-GDN Update Rule", section 3.4 "FG2-GDN+ Variant", section
+ * 3.6 "Chunkwise Parallel Training"; the update's equations are lost from the
+ * page, and this is the reading the text supports): the key is scaled by the
+ * square root of the per-channel rate, k~ = sqrt(beta^k) . k, which keeps KDA's
+ * tied (symmetric) transition; the FG2-GDN+ value gate scales the value the
+ * same way, v~ = sqrt(beta^v) . v (FG2-GDN: no value gate, v~ = v); then
+ *       S_t = S_{t-1} Diag(alpha_t) (I - k~_t k~_t^T) + v~_t k~_t^T
+ *       o_t = S_t q_t
+ * which is KDA's update with unit rate on (k~, v~): uniform beta^k = beta^v = b
+ * gives KDA with beta = b.
+ *
  * Everything is fp64; inputs are passed in already rounded to the precision
  * the GPU path reads (bf16 or fp32), upcast to double.  Independent (sequence,
  * head) chains run on POSIX threads; the arithmetic inside one chain is
@@ -61,6 +73,8 @@ typedef struct {
     double *o;                  /* [tok, H, dv]                                 */
     double *S_final;            /* [n_seqs, H, dv, dk] or NULL                  */
     int chunk;                  /* chunk size (chunkwise driver only)           */
+    const double *beta_k;       /* FG2: [tok, H, dk] key-side rate (else NULL)   */
+    const double *beta_v;       /* FG2+: [tok, H, dv] value-side rate, or NULL   */
 } problem;
 
 /* log decay of channel c for token t of head h */
@@ -78,6 +92,32 @@ static void recurrent_chain(const problem *p, int n, int h, double *S, double *r
         const double *q = p->q + (t * H + h) * dk;
         const double *k = p->k + (t * H + h) * dk;
         const double *v = p->v + (t * H + h) * dv;
+        if (p->beta_k) {
+            /* FG2: S <- S Diag(alpha) (I - k~ k~^T) + v~ k~^T with
+             * k~ = sqrt(beta^k) . k and v~ = sqrt(beta^v) . v (or v)          */
+            double *kt = r + dv, *vt = r + dv + dk;
+            for (int c = 0; c < dk; ++c) kt[c] = sqrt(p->beta_k[(t * H + h) * dk + c]) * k[c];
+            for (int i = 0; i < dv; ++i)
+                vt[i] = p->beta_v ? sqrt(p->beta_v[(t * H + h) * dv + i]) * v[i] : v[i];
+            for (int c = 0; c < dk; ++c) {
+                const double ac = exp(log_decay(p, t, h, c));   /* column c decays */
+                for (int i = 0; i < dv; ++i) S[i * dk + c] = ac * S[i * dk + c];
+            }
+            for (int i = 0; i < dv; ++i) {
+                double e = 0.0;
+                for (int c = 0; c < dk; ++c) e += kt[c] * S[i * dk + c];
+                r[i] = e;                         /* (S_{t-1} Diag(alpha) k~)_i */
+            }
+            for (int i = 0; i < dv; ++i)
+                for (int c = 0; c < dk; ++c) S[i * dk + c] += (vt[i] - r[i]) * kt[c];
+            double *ot = p->o + (t * H + h) * dv;
+            for (int i = 0; i < dv; ++i) {
+                double e = 0.0;
+                for (int c = 0; c < dk; ++c) e += q[c] * S[i * dk + c];
+                ot[i] = e;                                      /* o_t = S_t q_t */
+            }
+            continue;
+        }
         const double b = p->beta[t * H + h];
         if (!p->channel_decay) {
             /* S <- alpha S (I - b k k^T) + b v k^T
@@ -266,7 +306,7 @@ static void *worker(void *arg) {
     const problem *p = pl->p;
     const int64_t items = (int64_t)p->n_seqs * p->H;
     double *S = (double *)malloc(sizeof(double) * p->dv * p->dk);
-    double *r = (double *)malloc(sizeof(double) * p->dv);
+    double *r = (double *)malloc(sizeof(double) * (2 * p->dv + p->dk));
     for (;;) {
         pthread_mutex_lock(&pl->mu);
         const int64_t it = pl->next++;
@@ -307,7 +347,19 @@ int oracle_gdn_recurrent(int n_seqs, const int64_t *seq_start, int H, int dk, in
                          double *o, double *S_final, int nthreads) {
     if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || !seq_start) return -1;
     problem p = {n_seqs, seq_start, H, dk, dv, channel_decay, q, k, v, log_alpha, beta,
-                 S0, o, S_final, 0};
+                 S0, o, S_final, 0, NULL, NULL};
+    return run(&p, 0, nthreads);
+}
+
+/* FG2-GDN / FG2-GDN+ (channel decay): beta_k [tok, H, dk]; beta_v [tok, H, dv]
+ * or NULL for FG2-GDN.  Returns the number of threads used, or -1. */
+int oracle_fg2_recurrent(int n_seqs, const int64_t *seq_start, int H, int dk, int dv,
+                         const double *q, const double *k, const double *v,
+                         const double *log_alpha, const double *beta_k, const double *beta_v,
+                         const double *S0, double *o, double *S_final, int nthreads) {
+    if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || !seq_start || !beta_k) return -1;
+    problem p = {n_seqs, seq_start, H, dk, dv, 1, q, k, v, log_alpha, NULL,
+                 S0, o, S_final, 0, beta_k, beta_v};
     return run(&p, 0, nthreads);
 }
 
@@ -317,7 +369,7 @@ int oracle_gdn_chunkwise(int n_seqs, const int64_t *seq_start, int H, int dk, in
                          double *o, double *S_final, int chunk, int nthreads) {
     if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || chunk <= 0 || !seq_start) return -1;
     problem p = {n_seqs, seq_start, H, dk, dv, channel_decay, q, k, v, log_alpha, beta,
-                 S0, o, S_final, chunk};
+                 S0, o, S_final, chunk, NULL, NULL};
     return run(&p, 1, nthreads);
 }
 

@@ -44,6 +44,21 @@ MUTATIONS = [
      "acc += Vp[s * dv + i] * k[s * dk + c];"),
     ("chunk end state: state transposed",
      "double acc = S[i * dk + c] * exp(gL);", "double acc = S[c * dk + i] * exp(gL);"),
+    ("fg2: key rate not rooted",
+     "kt[c] = sqrt(p->beta_k[(t * H + h) * dk + c]) * k[c];",
+     "kt[c] = p->beta_k[(t * H + h) * dk + c] * k[c];"),
+    ("fg2: value gate ignored",
+     "vt[i] = p->beta_v ? sqrt(p->beta_v[(t * H + h) * dv + i]) * v[i] : v[i];",
+     "vt[i] = v[i];"),
+    ("fg2: erase along the unscaled key",
+     "for (int c = 0; c < dk; ++c) e += kt[c] * S[i * dk + c];",
+     "for (int c = 0; c < dk; ++c) e += k[c] * S[i * dk + c];"),
+    ("fg2: decay dropped",
+     "const double ac = exp(log_decay(p, t, h, c));   /* column c decays */",
+     "const double ac = 1.0;"),
+    ("fg2: write along the unscaled key",
+     "S[i * dk + c] += (vt[i] - r[i]) * kt[c];",
+     "S[i * dk + c] += vt[i] * k[c] - r[i] * kt[c];"),
     ("prologue: norm not rooted", "double nrm = sqrt(ss);", "double nrm = ss;"),
     ("prologue: sigmoid of the negated logit",
      "static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }",
@@ -67,6 +82,9 @@ PIN_TESTS = [
     (pins.test_chunkwise_equals_recurrent, [(False, 16), (True, 16)]),
     (pins.test_chunk_stage_ut_factor, [(False,), (True,)]),
     (pins.test_prologue_gate_closed_forms, [()]),
+    (pins.test_fg2_uniform_rates_equal_kda, [()]),
+    (pins.test_fg2_is_kda_on_scaled_keys_and_values_chunkwise_too, [()]),
+    (pins.test_fg2_erase_is_exact_along_a_unit_scaled_key, [()]),
     (pins.test_prologue_decay_bias_per_head_and_channel, [()]),
     (pins.test_prologue_unit_norm_scale_invariance_and_direction, [()]),
 ]

@@ -14,6 +14,10 @@ Citations name the page and section each fact comes from:
     section 3.6.
   * A state impulse is forgotten within hundreds of steps: the NVFP4 (Minima)
     abstract on the DeltaNet papers page.
+  * FG2-GDN's channel-wise writing rate keeps KDA's tied transition through
+    square-root-scaled keys (FG2-GDN sections 3.2, 3.4, 3.6): uniform rates give
+    KDA; the update is KDA's with unit rate on the scaled keys and values, so
+    KDA's chunkwise form computes it.
 """
 import os
 
@@ -444,3 +448,71 @@ def test_prologue_unit_norm_scale_invariance_and_direction():
     q3[:, 0] *= -7.0
     qn3, _, _, _ = oracle.prologue(q3, k, a, b)
     assert np.array_equal(qn3[:, 1:], qn[:, 1:])
+
+
+# --------------------------------------------------------------------------- #
+# FG2-GDN: channel-wise writing rate through square-root-scaled keys          #
+# --------------------------------------------------------------------------- #
+def _fg2_problem(rng, B=1, T=41, H=2, dk=8, dv=6):
+    q, k, v, la, _, S0 = _rand_problem(rng, B=B, T=T, H=H, dk=dk, dv=dv, channel=True)
+    bk = rng.uniform(0.05, 1.0, size=(B, T, H, dk))
+    bv = rng.uniform(0.05, 1.0, size=(B, T, H, dv))
+    return q, k, v, la, bk, bv, S0
+
+
+def test_fg2_uniform_rates_equal_kda():
+    """beta^k = beta^v = b on every channel: FG2-GDN+ is KDA with beta = b (the
+    page's claim that FG2-GDN extends KDA's scalar rate to a vector)."""
+    rng = np.random.default_rng(91)
+    q, k, v, la, _, _, S0 = _fg2_problem(rng)
+    b = rng.uniform(0.05, 1.0, size=q.shape[:3])
+    bk = np.repeat(b[..., None], q.shape[-1], axis=-1)
+    bv = np.repeat(b[..., None], v.shape[-1], axis=-1)
+    o1, s1 = oracle.fg2_recurrent(q, k, v, la, bk, bv, S0)
+    o2, s2 = oracle.recurrent(q, k, v, la, b, S0)
+    assert np.allclose(o1, o2, rtol=0, atol=1e-12) and np.allclose(s1, s2, rtol=0, atol=1e-12)
+    # FG2-GDN (no value gate) is FG2-GDN+ with a unit value rate, exactly
+    o3, s3 = oracle.fg2_recurrent(q, k, v, la, bk)
+    o4, s4 = oracle.fg2_recurrent(q, k, v, la, bk, np.ones_like(bv))
+    assert np.array_equal(o3, o4) and np.array_equal(s3, s4)
+
+
+def test_fg2_is_kda_on_scaled_keys_and_values_chunkwise_too():
+    """The update is KDA's with unit rate on k~ = sqrt(beta^k) k, v~ = sqrt(beta^v) v
+    (the page's 'identical in form'): the KDA recurrence and KDA's chunkwise WY/UT
+    form (chunks of 16 over 41 tokens, packed sequences) fed the scaled keys and
+    values give FG2's result."""
+    rng = np.random.default_rng(92)
+    q, k, v, la, bk, bv, _ = _fg2_problem(rng, T=41)
+    cu = np.array([0, 7, 7, 41])
+    S0 = rng.standard_normal((3, 2, 6, 8)) * 0.3
+    kt, vt = np.sqrt(bk) * k, np.sqrt(bv) * v
+    ones = np.ones(q.shape[:3])
+    o1, s1 = oracle.fg2_recurrent(q, k, v, la, bk, bv, S0, cu)
+    o2, s2 = oracle.recurrent(q, kt, vt, la, ones, S0, cu)
+    o3, s3 = oracle.chunkwise(q, kt, vt, la, ones, S0, cu, chunk=16)
+    for o, st in ((o2, s2), (o3, s3)):
+        assert np.allclose(o1, o, rtol=0, atol=1e-11) and np.allclose(s1, st, rtol=0, atol=1e-11)
+
+
+def test_fg2_erase_is_exact_along_a_unit_scaled_key():
+    """No decay, one token whose scaled key k~ = sqrt(beta^k) . k has unit norm:
+    the delta rule overwrites the memory along k~, S_1 k~ = v~ exactly, and leaves
+    every direction orthogonal to k~ as it was."""
+    rng = np.random.default_rng(93)
+    dk, dv = 8, 5
+    u = rng.standard_normal(dk)
+    u /= np.linalg.norm(u)
+    bk = rng.uniform(0.1, 1.0, size=dk)
+    k = u / np.sqrt(bk)                   # so that sqrt(bk) * k = u
+    v = rng.standard_normal(dv)
+    bv = rng.uniform(0.1, 1.0, size=dv)
+    S0 = rng.standard_normal((1, 1, dv, dk))
+    q = rng.standard_normal(dk)
+    sh = lambda x: x.reshape(1, 1, 1, -1)
+    _, s1 = oracle.fg2_recurrent(sh(q), sh(k), sh(v), np.zeros((1, 1, 1, dk)), sh(bk), sh(bv), S0)
+    S1 = s1[0, 0]
+    assert np.allclose(S1 @ u, np.sqrt(bv) * v, rtol=0, atol=1e-13)
+    w = rng.standard_normal(dk)
+    w -= (w @ u) * u
+    assert np.allclose(S1 @ w, S0[0, 0] @ w, rtol=0, atol=1e-13)
