@@ -20,9 +20,11 @@ with no data-path collective): weak scaling.  Inputs are larger than L2
 (prefill 275 MB, decode state 537 MB), so no flush is needed between steps.
 
 ``legs`` (rank 0 of a 1-GPU run, or every rank with --legs on N GPUs) times
-each workload on its own for at least --leg-seconds of device time: the four
+each workload on its own for at least --leg-seconds of device time: the six
 bf16 prefill workloads (GDN B4 H16 T4096; packed varlen, 32 sequences of
-256-4096 tokens with initial states; KDA B2 H32 T8192; GDN B1 H32 T65536)
+256-4096 tokens with initial states; KDA B2 H32 T8192, the same with 8 key
+channels per head forgetting at log alpha = -30 per token, and with FG2-GDN's
+writing rate per key channel; GDN B1 H32 T65536)
 and the decode step (N256 H32, fp32 state in place).  Each leg carries its own
 roofline (max of FLOPs / bf16 peak and algorithmic bytes / HBM bandwidth, the
 measured peaks), end-to-end rate through host buffers, and a bounded CPU
@@ -50,7 +52,7 @@ METRIC = "gated-delta-rule prefill tokens/s and decode steps/s; % of roofline on
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CHUNK = 64
 PREFILL_LEGS = ("gdn_prefill_bf16", "gdn_varlen_bf16", "kda_prefill_bf16",
-                "gdn_long_prefill_bf16")
+                "kda_fast8_prefill_bf16", "fg2_prefill_bf16", "gdn_long_prefill_bf16")
 RAW_LEG = "gdn_prefill_bf16_raw"  # the config-2 shapes through the fused input prologue
 DECODE_LEG = "gdn_decode"
 KERNEL_SRC = {
@@ -72,11 +74,12 @@ def peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
-def prefill_bytes(es, channel, tok_heads, dk, dv, n_states):
+def prefill_bytes(es, channel, tok_heads, dk, dv, n_states, beta_channel=False):
     """Algorithmic HBM bytes of one prefill: q, k, v read and o written once
-    (element size ``es``), fp32 log alpha (per key channel for KDA) and beta read
-    once, and ``n_states`` fp32 states of d_v x d_k read or written once."""
-    per_tok = es * (2 * dk + 2 * dv) + 4 * (dk if channel else 1) + 4
+    (element size ``es``), fp32 log alpha (per key channel for KDA) and beta (per
+    key channel for FG2-GDN) read once, and ``n_states`` fp32 states of d_v x d_k
+    read or written once."""
+    per_tok = es * (2 * dk + 2 * dv) + 4 * (dk if channel else 1) + 4 * (dk if beta_channel else 1)
     return tok_heads * per_tok + n_states * dv * dk * 4
 
 
@@ -262,6 +265,10 @@ def oracle_sample(workload, budget_token_heads=SAMPLE_TOKEN_HEADS):
 
 def _oracle_pass(s, s0, cu, nthreads=0):
     import oracle
+    if s["beta"].dim() == 4:  # FG2-GDN's rate per key channel
+        oracle.fg2_recurrent(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], None, s0, cu,
+                             nthreads=nthreads)
+        return nthreads if nthreads > 0 else (os.cpu_count() or 1)
     _, _, used = oracle.recurrent(s["q"], s["k"], s["v"], s["log_alpha"], s["beta"], s0, cu,
                                   nthreads=nthreads, return_threads=True)
     return used
@@ -338,6 +345,8 @@ class PrefillLeg:
         import torch
         from gated_delta_rule_140_b200.inputs import WORKLOADS, workload_inputs
         self.name, self.w, self.kflags, self.ws = name, WORKLOADS[name], kflags, ws
+        if self.w.decay == "channel":  # the pool and single-CTA kernels take scalar decay
+            self.kflags = {k: (v and k not in ("pool", "one_cta")) for k, v in kflags.items()}
         self.cpu = workload_inputs(name)
         self.x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.cpu.items()}
         x = self.x
@@ -363,7 +372,7 @@ class PrefillLeg:
         n_states = self.n_seqs * (int(self.x["initial_state"] is not None) + 1)
         return (prefill_flops(th, self.dk, self.dv),
                 prefill_bytes(es, self.w.decay == "channel", th, self.dk, self.dv,
-                              n_states * self.H))
+                              n_states * self.H, self.w.beta_channel))
 
     def kernel(self):
         from gated_delta_rule_140_b200 import _native as nat

@@ -20,6 +20,7 @@ GDN_OK, GDN_ERR_INVALID, GDN_ERR_UNSUPPORTED, GDN_ERR_CUDA, GDN_ERR_TIMEOUT, \
 GDN_BF16, GDN_FP32 = 0, 1
 GDN_DECAY_SCALAR, GDN_DECAY_CHANNEL = 0, 1
 GDN_FLAG_CUDA_CORES, GDN_FLAG_PAIR, GDN_FLAG_ONE_CTA, GDN_FLAG_POOL = 1, 2, 4, 8
+GDN_FLAG_BETA_CHANNEL = 16
 
 
 class GdnError(RuntimeError):
@@ -119,14 +120,15 @@ def _check_dev(name, t, dtype=None):
 
 
 def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False, pair=False,
-                 one_cta=False, pool=False) -> Dims:
+                 one_cta=False, pool=False, beta_channel=False) -> Dims:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     return Dims(B, T, H, dk, dv, (len(cu_seqlens) - 1) if cu_seqlens is not None else B,
                 _dtype_code(q.dtype),
                 GDN_DECAY_CHANNEL if log_alpha.dim() == 4 else GDN_DECAY_SCALAR,
                 (GDN_FLAG_CUDA_CORES if cuda_cores else 0) | (GDN_FLAG_PAIR if pair else 0)
-                | (GDN_FLAG_ONE_CTA if one_cta else 0) | (GDN_FLAG_POOL if pool else 0))
+                | (GDN_FLAG_ONE_CTA if one_cta else 0) | (GDN_FLAG_POOL if pool else 0)
+                | (GDN_FLAG_BETA_CHANNEL if beta_channel else 0))
 
 
 def chunk_fwd_path(dims: Dims) -> str:
@@ -199,6 +201,8 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
               cuda_cores=False, pair=False, one_cta=False, pool=False, check=False,
               stream=None):
     """Chunkwise prefill (gdn_chunk_fwd).  Returns (o, final_state or None).
+    A ``beta`` of shape [B,T,H,d_k] (with channel decay) is FG2-GDN's writing rate
+    per key channel (GDN_FLAG_BETA_CHANNEL); [B,T,H] is the usual scalar rate.
     ``cuda_cores`` / ``pool`` / ``pair`` / ``one_cta`` select the fp32
     CUDA-core kernel or one of the tensor-core kernels instead of the default
     (GDN_FLAG_*).  With ``check`` the call synchronises the stream afterwards
@@ -212,7 +216,9 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
     _check_dev("beta", beta, torch.float32)
     _check_dev("initial_state", initial_state, torch.float32)
     _check_dev("cu_seqlens", cu_seqlens, torch.int32)
-    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair, one_cta, pool)
+    beta_channel = beta is not None and beta.dim() == 4
+    dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair, one_cta, pool,
+                        beta_channel)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:

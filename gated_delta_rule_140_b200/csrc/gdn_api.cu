@@ -21,8 +21,17 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     if (d->d_k <= 0 || d->d_v <= 0) return GDN_ERR_INVALID;
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
         return GDN_ERR_UNSUPPORTED;
-    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA | GDN_FLAG_POOL)) != 0)
+    if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA | GDN_FLAG_POOL |
+                      GDN_FLAG_BETA_CHANNEL)) != 0)
         return GDN_ERR_INVALID;
+    if (d->flags & GDN_FLAG_BETA_CHANNEL) {
+        // FG2-GDN: a writing rate per key channel rides on KDA's decay, prefill only,
+        // on the two-CTA tensor-core kernel
+        if (d->decay != GDN_DECAY_CHANNEL || (d->flags & (GDN_FLAG_ONE_CTA | GDN_FLAG_POOL)))
+            return GDN_ERR_INVALID;
+        if (!prefill || (d->flags & GDN_FLAG_CUDA_CORES) || !gdn::chunk_pair_supported(*d))
+            return GDN_ERR_UNSUPPORTED;
+    }
     const int kernel_flags = d->flags & (GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA | GDN_FLAG_POOL);
     if (kernel_flags & (kernel_flags - 1)) return GDN_ERR_INVALID;  // at most one
     if ((d->flags & (GDN_FLAG_ONE_CTA | GDN_FLAG_POOL)) && d->decay == GDN_DECAY_CHANNEL)
@@ -117,6 +126,7 @@ gdn_status chunk_fwd_impl(const gdn_dims *dims, const void *q, const void *k, co
     a.channel = d.decay == GDN_DECAY_CHANNEL;
     a.bf16 = d.dtype == GDN_BF16;
     a.raw = raw;
+    a.beta_channel = (d.flags & GDN_FLAG_BETA_CHANNEL) != 0;
     a.alpha_bias = alpha_bias;
 
     // Nothing to compute and nothing to write: an empty batch is a no-op.

@@ -31,14 +31,20 @@
 //        each row's own 16-token block, factored at the 16-token block
 //        boundaries elsewhere, both factors <= 1); T_bg = T_b diag(e^{g}) so
 //        that W = T_bg K; [P T_bg | R] = P [T_bg | T_b]; [W; P W] = [T_bg; P T_bg] K.
-//   KDA (group 1, one chunk ahead): each 16-token row block i takes the
-//        reference m_i = 16 i + 7 (its middle token): K and Q become KD, QD =
-//        . e^{G - G_{m(r)}} in place, and B_i = K[0, 16(i+1)) . e^{G_{m_i} - G},
-//        stacked into one 160-row operand, so that one MMA (N = 160) gives
-//        D_i = [KD; QD] B_i^T, the decayed A and P of block i (masks only);
-//        every factor is within 8 tokens' decay of 1.  Then (group 0)
-//        R = P T_b, Kg = KD . e^{G_{m(r)}}, [W; P W] = [T_b; R] Kg, and
-//        Qh = QD . e^{G_{m(r)}} - P W.
+//   KDA (group 1, one chunk ahead): each 16-token row block i takes its start
+//        as the reference (off_i = G at the end of block i - 1, off_0 = 0): K and
+//        Q become KD, QD = . e^{G - off_{i(r)}} in place (<= 1), and B_i =
+//        K[0, 16(i+1)) . e^{off_i - G}, stacked into one 160-row operand, so that
+//        one MMA (N = 160) gives D_i = [KD; QD] B_i^T, the decayed A and P of
+//        block i (masks only).  Off the diagonal block both factors are <= 1 (they
+//        can only underflow, where the exact term is as small); inside it B_i's
+//        factor is e^{off_i - G} <= e^{block decay}.  A channel whose decay over
+//        the block passes e^{-kMaxNegLogDecay} is zeroed in B_i's diagonal rows,
+//        and its exact diagonal-block terms k_r k_s e^{G_r - G_s}, q_r k_s e^{G_r
+//        - G_s} (exponent <= 0, taken directly) are summed into a correction
+//        table that the A/P phase adds.  Exact for any decay.  Then (group 0)
+//        R = P T_b, Kg = KD . e^{off}, [W; P W] = [T_b; R] Kg, and
+//        Qh = QD . e^{off} - P W.
 // T comes from blocked forward substitution in fp32 (tf32 MMAs for the
 // off-diagonal blocks), computed in place of A.  The ring tiles leave shared
 // memory by bulk copy in two groups (what the group's next chunk rewrites early
@@ -48,13 +54,6 @@
 // chunk's ring slot and V tile (bulk copy + TMA), and per chunk and half
 // issues D = [R;T_b] V_h + [Qh;-W] S_h^T, writes o, converts V' to bf16 and
 // issues dS = Kt^T V'.
-//
-// KDA range: the factors are finite while the decay over any 8 consecutive
-// tokens stays above e^{-kMaxNegLogDecay} on every channel (log alpha > -10 per
-// token on average; the KDA workload's -3 is far inside).  A chunk past that is
-// computed with the exponents clamped and its (sequence, head) is flagged in the
-// workspace; the host re-runs the flagged items on the CUDA-core kernel, which
-// is exact for any decay, and this kernel leaves their final state to it.
 //
 // The CTAs signal each other with mbarriers (ring slot written / ring slot
 // read).  Every wait is bounded: on expiry the CTA records kErrTimeout, raises
@@ -75,7 +74,7 @@ constexpr int DK = 128, DV = 128;
 constexpr int kThreads = 512;
 constexpr long long kWaitLimit = kDefaultWaitLimit;  // drains after an abort
 constexpr int LDA = 68;                      // fp32 row stride of A / T
-constexpr float kMaxNegLogDecay = 80.f;      // e^{80} < bf16 and fp32 max
+constexpr float kMaxNegLogDecay = 80.f;      // e^{80} < bf16 and fp32 max; e^{-80} normal
 
 // ---- ring slot / state-CTA stage layout (bytes, 1024-aligned tiles) --------
 // per atom column a (d_k 64a .. 64a+63):  [Kt rows 0-63 | Qh rows | -W rows]
@@ -129,24 +128,36 @@ constexpr int GR_KB = 512;  // KDA beta (after the scratch)
 // KDA (group 0 runs the products, group 1 the gate pass of the next chunk; the
 // group-1 space holds): the B operand of the decayed [K; Q] products, rows
 // di_col(i) .. of it being, for 16-token row block i, B_i = K[0, 16(i+1)) .
-// e^{G_{m_i} - G} (m_i = 16 i + 7), 160 rows per atom column; then two per-block
-// tables, a second Kt buffer and a second raw tile buffer (raw tiles and tables
-// alternate by chunk parity).  W's operand Kg = K . e^{G} replaces KD in its raw
-// tile once the products are done.
+// e^{off_i - G} (off_i: G at the block's start), 160 rows per atom column; then
+// two per-block tables, a second Kt buffer, a second raw tile buffer (raw tiles
+// and tables alternate by chunk parity) and the two correction tables.  W's
+// operand Kg = K . e^{G} replaces KD in its raw tile once the products are done.
 constexpr uint32_t L_BREG = Lay<true>::GSZ;  // (group 1's space)
 constexpr uint32_t BREG_AC = 160 * 128;      // atom column stride of the stacked B
 __host__ __device__ constexpr uint32_t di_col(int i) { return 8u * i * (i + 1); }  // 0, 16, 48, 96
-constexpr uint32_t KTAB_BYTES = 6144;              // fp32 [4][128] x 3: block totals, G at m_i, e^{G_{m_i}}
+constexpr uint32_t KTAB_BYTES = 4096;              // fp32 [4][128] x 2: block totals, e^{off_i}
 constexpr uint32_t L_KTAB = L_BREG + 2 * BREG_AC;  // two tables
 constexpr uint32_t L_KX2 = L_KTAB + 2 * KTAB_BYTES;  // KDA's second Kt buffer
 constexpr uint32_t L_RAW2 = L_KX2 + 16384;         // KDA's second raw tiles [K0 | Q0 | K1 | Q1]
+// the exact diagonal-block terms of the channels whose decay over a 16-token
+// block passes e^{-kMaxNegLogDecay}: fp32 [block][A, P][lower triangle incl. the
+// diagonal], and a word "the table holds this chunk's terms", two tables by chunk
+// parity; then the gate group's staging of such (block, channel) pairs: a count,
+// the pairs (block << 8 | channel) and their 16 cumulative log decays, KSTG_CAP
+// pairs at a time
+constexpr int KCOR_TRI = 136, KCOR_FLAG = 8 * KCOR_TRI;
+constexpr uint32_t KCOR_BYTES = (KCOR_FLAG + 4) * 4;
+constexpr uint32_t L_KCOR = L_RAW2 + RAW_BYTES;
+constexpr int KSTG_CAP = 32;
+constexpr uint32_t L_KSTG = L_KCOR + 2 * KCOR_BYTES;  // count | pairs at +16 | G at +256
+constexpr uint32_t KSTG_BYTES = 256 + KSTG_CAP * 16 * 4;
 constexpr uint32_t TM_KD = 192;                    // D = [D_0 | D_1 | D_2 | D_3], 160 columns
 constexpr uint32_t ID_KD = idesc_bf16(128, 160, false, false);
 static_assert(L_RAW2 % 1024 == 0, "KDA layout");
 
 // ---- shared bookkeeping (same offset in both CTAs, so peers can address it) --
 constexpr uint32_t OFF_COMMON = 215040;
-static_assert(S_OFF_VP + 2 * 8192 <= OFF_COMMON && L_RAW2 + RAW_BYTES <= OFF_COMMON &&
+static_assert(S_OFF_VP + 2 * 8192 <= OFF_COMMON && L_KSTG + KSTG_BYTES <= OFF_COMMON &&
               Lay<false>::G0 + 2 * Lay<false>::GSZ <= OFF_COMMON, "shared memory layout");
 constexpr uint32_t CM_ABORT = 0, CM_SLOT = 4, CM_TMEM = 8, CM_ISSUED = 32, CM_BARS = 64;
 constexpr int NBARS = 18;
@@ -316,7 +327,7 @@ template <bool CH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  uint8_t *ring, int ring_slots, uint32_t *redo) {
+                  uint8_t *ring, int ring_slots) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -353,9 +364,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             tma_prefetch_desc(&tm_k);
         } else {
             tma_prefetch_desc(&tm_v);
-            if (CH) redo[item] = 0u;
         }
     }
+    if (CH && rank == 0)
+        for (int i = tid; i < 2 * (int)(KCOR_BYTES / 4); i += kThreads)
+            reinterpret_cast<float *>(sm + L_KCOR)[i] = 0.f;
     cluster_sync();  // both CTAs' barriers and flags are initialised
     if (rank == 1 && tid == 0) {
         // the ring slot pair of this cluster: indexed by the state CTA's SM,
@@ -395,6 +408,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
         };
         auto tma_phase = [&](int m) -> uint32_t { return (uint32_t)((CH ? (m >> 1) : (m / 3)) & 1); };
         auto ktab_of = [&](int m) { return reinterpret_cast<float *>(sm + L_KTAB + (m & 1) * KTAB_BYTES); };
+        auto kcor_of = [&](int m) { return reinterpret_cast<float *>(sm + L_KCOR + (m & 1) * KCOR_BYTES); };
         uint8_t *kxt = CH ? sm + LY::KX : nullptr;  // KDA Kt of even chunks
         uint8_t *pzt = grp + LY::PZT;
         float *AT = reinterpret_cast<float *>(grp + LY::AT);
@@ -520,13 +534,13 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + C + pr) * H + h) * DK + 32 * pc));
                 }
                 // ---- KDA gates: G_rc by a prefix sum over the rows (thread: two
-                //      channels, the 16 rows of block rq) and the block references
-                //      G at m_i = 16 i + 7; then, with every exponent within 8 tokens'
-                //      decay of zero: KD = K e^{G - G_{m(r)}} and QD likewise in place,
-                //      Kt = K e^{G_C - G} (ring tile), B_i = K[0,16(i+1)) e^{G_{m_i} - G}.
-                //      The sums need no tiles, so they run while the tiles load.
+                //      channels, the 16 rows of block rq) and the block totals; then
+                //      KD = K e^{G - off_{i(r)}} and QD likewise in place, Kt = K
+                //      e^{G_C - G} (ring tile), B_i = K[0,16(i+1)) e^{off_i - G}, and the
+                //      exact diagonal-block terms of fast-decaying channels.  The sums
+                //      need no tiles, so they run while the tiles load.
                 const int cp = gtid & 63, rq = gtid >> 6, c0 = 2 * cp;
-                float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f, p70 = 0.f, p71 = 0.f;
+                float gl0[16], gl1[16], acc0 = 0.f, acc1 = 0.f;
                 const float *lp0 = a.log_alpha + ((t0 + 16 * rq) * H + h) * DK + c0;
                 if ((reinterpret_cast<uintptr_t>(a.log_alpha) & 7) == 0) {  // uniform
 #pragma unroll
@@ -551,10 +565,10 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     acc1 += gl1[i];
                     gl0[i] = acc0;
                     gl1[i] = acc1;
-                    if (i == 7) { p70 = acc0; p71 = acc1; }
                 }
                 *reinterpret_cast<float2 *>(ktab + 128 * rq + c0) = make_float2(acc0, acc1);
-                *reinterpret_cast<float2 *>(ktab + 512 + 128 * rq + c0) = make_float2(p70, p71);
+                // (the staging count, read last in chunk m - 1 before its final barrier)
+                if (gtid == 0) *reinterpret_cast<volatile uint32_t *>(sm + L_KSTG) = 0u;
                 // chunk m's tiles: group 0 loads them once chunk m - 2 is done with
                 // this parity's raw tiles, table and gate rows (rows past the sequence
                 // end are zeroed here)
@@ -568,77 +582,157 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + o) = z;
                     *reinterpret_cast<uint4 *>(rawp + L_RAW_AC + 8192 + o) = z;
                 }
-                if (gtid < 64) gr[GR_KB + gtid] = gtid < L ? a.beta[(t0 + gtid) * H + h] : 0.f;
+                // (FG2-GDN: unit rate; the per-channel rate scales the keys below)
+                if (gtid < 64)
+                    gr[GR_KB + gtid] = gtid < L ? (a.beta_channel ? 1.f : a.beta[(t0 + gtid) * H + h]) : 0.f;
                 // the B region (read by chunk m - 1's products), chunk m - 2's Kt and
                 // e^{G_C} (read by its ring stores) are free once group 0 says so
                 if (issuer && m >= 1) ok = wt.wait(bars + LB_BFREE, (uint32_t)((m - 1) & 1));
                 if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-                float gm0[4], gm1[4], off0 = 0.f, off1 = 0.f, run0 = 0.f, run1 = 0.f;
+                // block starts off_b (G at the end of block b - 1; off_0 = 0) and the
+                // chunk total G_C, from the block totals
+                float ob0[4], ob1[4], run0 = 0.f, run1 = 0.f;
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
                     const float2 tt = *reinterpret_cast<const float2 *>(ktab + 128 * q2 + c0);
-                    const float2 pp = *reinterpret_cast<const float2 *>(ktab + 512 + 128 * q2 + c0);
-                    gm0[q2] = run0 + pp.x;
-                    gm1[q2] = run1 + pp.y;
-                    if (q2 == rq) { off0 = run0; off1 = run1; }
+                    ob0[q2] = run0;
+                    ob1[q2] = run1;
                     run0 += tt.x;
                     run1 += tt.y;
                 }
+                float off0 = ob0[0], off1 = ob1[0];
+#pragma unroll
+                for (int q2 = 1; q2 < 4; ++q2)
+                    if (q2 == rq) { off0 = ob0[q2]; off1 = ob1[q2]; }
                 if (rq == 0) {
                     *reinterpret_cast<float2 *>(gr + GR_DEC + c0) = make_float2(__expf(run0), __expf(run1));
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2)
-                        *reinterpret_cast<float2 *>(ktab + 1024 + 128 * q2 + c0) =
-                            make_float2(__expf(gm0[q2]), __expf(gm1[q2]));
+                        *reinterpret_cast<float2 *>(ktab + 512 + 128 * q2 + c0) =
+                            make_float2(__expf(ob0[q2]), __expf(ob1[q2]));
                 }
                 const int ac = c0 >> 6, cc = c0 & 63;
                 const uint32_t cof = (uint32_t)((cc & 7) * 2);
-                float big = 0.f;  // largest exponent met (range check)
                 auto bf2 = [](float x, float y) {
                     __nv_bfloat162 t = __floats2bfloat162_rn(x, y);
                     return *reinterpret_cast<uint32_t *>(&t);
                 };
-                // this block's reference, and the factors from it to the later blocks'
-                // references and to the chunk end (all <= 1)
-                float gr0 = gm0[0], gr1 = gm1[0];
-#pragma unroll
-                for (int q2 = 1; q2 < 4; ++q2)
-                    if (q2 == rq) { gr0 = gm0[q2]; gr1 = gm1[q2]; }
+                if (a.beta_channel) {
+                    // FG2-GDN: K <- sqrt(beta) . K in place, this thread's rows and channels
+                    const float *bp = a.beta + ((t0 + 16 * rq) * H + h) * DK + c0;
+#pragma unroll 4
+                    for (int i = 0; i < 16; ++i) {
+                        if (16 * rq + i >= L) break;  // (rows past the end are zero)
+                        const float b0 = bp[(size_t)i * H * DK], b1 = bp[(size_t)i * H * DK + 1];
+                        uint32_t *pk = reinterpret_cast<uint32_t *>(
+                            rawp + ac * L_RAW_AC + sw128(16 * rq + i, cc >> 3) + cof);
+                        const uint32_t kw = *pk;
+                        *pk = bf2(__uint_as_float(kw << 16) * sqrtf(b0),
+                                  __uint_as_float(kw & 0xffff0000u) * sqrtf(b1));
+                    }
+                }
+                // this block's end end_rq = off_rq + acc; the factors from it to the later
+                // blocks' starts and to the chunk end (all <= 1)
+                const float end0 = off0 + acc0, end1 = off1 + acc1;
                 float tb0[4], tb1[4];
 #pragma unroll
                 for (int bi = 0; bi < 4; ++bi) {
-                    tb0[bi] = bi > rq ? __expf(gm0[bi] - gr0) : 1.f;
-                    tb1[bi] = bi > rq ? __expf(gm1[bi] - gr1) : 1.f;
+                    tb0[bi] = bi > rq ? __expf(ob0[bi] - end0) : 0.f;
+                    tb1[bi] = bi > rq ? __expf(ob1[bi] - end1) : 0.f;
                 }
-                const float tc0 = __expf(run0 - gr0), tc1 = __expf(run1 - gr1);
+                const float tc0 = __expf(run0 - end0), tc1 = __expf(run1 - end1);
+                // a channel whose decay over this block passes e^{-kMaxNegLogDecay} leaves
+                // the factored diagonal block; its exact terms k_r k_s e^{G_r - G_s} and
+                // q_r k_s e^{G_r - G_s} (s <= r in the block, exponent <= 0) go to the
+                // correction table, every thread taking a few entries over all such
+                // (block, channel) pairs, which their owners stage
+                const bool fl0 = -acc0 > kMaxNegLogDecay, fl1 = -acc1 > kMaxNegLogDecay;
+                float *cor = kcor_of(m);
+                uint32_t *kst_cnt = reinterpret_cast<uint32_t *>(sm + L_KSTG);
+                int *kst_pair = reinterpret_cast<int *>(sm + L_KSTG + 16);
+                float *kst_g = reinterpret_cast<float *>(sm + L_KSTG + 256);
+                const int my0 = fl0 ? (int)atomicAdd(kst_cnt, 1u) : -1;
+                const int my1 = fl1 ? (int)atomicAdd(kst_cnt, 1u) : -1;
+                const bool anyfl = named_bar_or(BAR_G, 256, fl0 || fl1);
+                if (anyfl) {
+                    const int npairs = (int)*reinterpret_cast<volatile uint32_t *>(kst_cnt);
+                    for (int p0 = 0; p0 < npairs; p0 += KSTG_CAP) {
+#pragma unroll
+                        for (int hc = 0; hc < 2; ++hc) {
+                            const int my = hc ? my1 : my0;
+                            if (my < p0 || my >= p0 + KSTG_CAP) continue;
+                            kst_pair[my - p0] = (rq << 8) | (c0 + hc);
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) kst_g[(my - p0) * 16 + i] = hc ? gl1[i] : gl0[i];
+                        }
+                        named_bar_sync(BAR_G, 256);
+                        const int np = min(KSTG_CAP, npairs - p0);
+                        for (int e = gtid; e < KCOR_FLAG; e += 256) {
+                            const int blk = e / (2 * KCOR_TRI), ap = (e / KCOR_TRI) & 1, tri = e % KCOR_TRI;
+                            int i = 0;
+                            while ((i + 1) * (i + 2) / 2 <= tri) ++i;
+                            const int s2 = tri - i * (i + 1) / 2;
+                            float accv = p0 == 0 ? 0.f : cor[e];
+                            if (ap == 1 || s2 < i) {
+                                for (int pp = 0; pp < np; ++pp) {
+                                    const int pr = kst_pair[pp];
+                                    if ((pr >> 8) != blk) continue;
+                                    const int c = pr & 255;
+                                    const uint8_t *tile = rawp + (c >> 6) * L_RAW_AC;
+                                    const uint32_t co = (uint32_t)((c & 7) * 2);
+                                    auto ld = [&](uint32_t off) {
+                                        return __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(tile + off) << 16);
+                                    };
+                                    const float ks = ld(sw128(16 * blk + s2, (c & 63) >> 3) + co);
+                                    const float li = ld((ap ? 8192u : 0u) + sw128(16 * blk + i, (c & 63) >> 3) + co);
+                                    accv += li * ks * __expf(kst_g[pp * 16 + i] - kst_g[pp * 16 + s2]);
+                                }
+                            }
+                            cor[e] = accv;
+                        }
+                        named_bar_sync(BAR_G, 256);
+                    }
+                }
+                if (gtid == 0) *reinterpret_cast<volatile int *>(cor + KCOR_FLAG) = anyfl ? 1 : 0;
+                const float eacc0 = __expf(acc0), eacc1 = __expf(acc1);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int r = 16 * rq + i;
-                    const float x0 = off0 + gl0[i] - gr0, x1 = off1 + gl1[i] - gr1;
-                    big = fmaxf(big, fmaxf(fabsf(x0), fabsf(x1)));
-                    // KD, QD = . e^{G - G_m};  KC = K e^{G_m - G} (B_rq's row)
-                    const float f0 = __expf(fminf(x0, kMaxNegLogDecay)), f1 = __expf(fminf(x1, kMaxNegLogDecay));
-                    const float h0 = __expf(fminf(-x0, kMaxNegLogDecay)), h1 = __expf(fminf(-x1, kMaxNegLogDecay));
+                    // x = G_r - off_rq in [acc, 0]
+                    const float x0 = gl0[i], x1 = gl1[i];
+                    const float e0 = __expf(x0), e1 = __expf(x1);  // KD, QD
+                    // de = e^{-x} (<= e^{kMaxNegLogDecay} unless flagged: then 0) and
+                    // ee = e^{acc - x} <= 1, to the block end
+                    float de0, ee0, de1, ee1;
+                    {
+                        // one exponential per channel: e^{-x} unless flagged, e^{acc - x} if
+                        const float t0 = __expf(fl0 ? acc0 - x0 : -x0), t1 = __expf(fl1 ? acc1 - x1 : -x1);
+                        de0 = fl0 ? 0.f : t0; ee0 = fl0 ? t0 : eacc0 * t0;
+                        de1 = fl1 ? 0.f : t1; ee1 = fl1 ? t1 : eacc1 * t1;
+                    }
                     const uint32_t o = sw128(r, cc >> 3) + cof;
                     uint32_t *pk = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + o);
                     uint32_t *pq = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + 8192 + o);
                     const uint32_t kw = *pk, qw = *pq;
                     const float kx = __uint_as_float(kw << 16), ky = __uint_as_float(kw & 0xffff0000u);
                     const float qx = __uint_as_float(qw << 16), qy = __uint_as_float(qw & 0xffff0000u);
-                    *pk = bf2(kx * f0, ky * f1);
-                    *pq = bf2(qx * f0, qy * f1);
-                    const float kc0 = kx * h0, kc1 = ky * h1;
-                    // Kt = K e^{G_C - G} = KC e^{G_C - G_m}
-                    *reinterpret_cast<uint32_t *>(kxc + ac * 8192 + o) = bf2(kc0 * tc0, kc1 * tc1);
-                    // B_i = K e^{G_{m_i} - G} = KC e^{G_{m_i} - G_m}, i >= rq
+                    // KD, QD = . e^{G - off}
+                    *pk = bf2(kx * e0, ky * e1);
+                    *pq = bf2(qx * e0, qy * e1);
+                    // KE = K e^{end - G};  Kt = K e^{G_C - G} = KE e^{G_C - end}
+                    const float ke0 = kx * ee0, ke1 = ky * ee1;
+                    *reinterpret_cast<uint32_t *>(kxc + ac * 8192 + o) = bf2(ke0 * tc0, ke1 * tc1);
+                    // B_rq = K e^{off_rq - G} (<= e^{kMaxNegLogDecay}; flagged channels 0),
+                    // B_i = K e^{off_i - G} = KE e^{off_i - end} for the later blocks i
+                    *reinterpret_cast<uint32_t *>(sm + L_BREG + ac * BREG_AC + sw128(di_col(rq) + r, cc >> 3) + cof) =
+                        bf2(kx * de0, ky * de1);
 #pragma unroll
-                    for (int bi = 0; bi < 4; ++bi) {
-                        if (bi < rq) continue;  // rq is uniform per warp
+                    for (int bi = 1; bi < 4; ++bi) {
+                        if (bi <= rq) continue;  // rq is uniform per warp
                         *reinterpret_cast<uint32_t *>(sm + L_BREG + ac * BREG_AC + sw128(di_col(bi) + r, cc >> 3) + cof) =
-                            bf2(kc0 * tb0[bi], kc1 * tb1[bi]);
+                            bf2(ke0 * tb0[bi], ke1 * tb1[bi]);
                     }
                 }
-                if (big > kMaxNegLogDecay) atomicOr(redo + item, 1u);
                 fence_proxy_async_smem();
                 if (named_bar_or(BAR_G, 256, *abort_flag)) break;
                 if (issuer) mbar_arrive(bars + LB_GATE);
@@ -744,6 +838,17 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         const int s2 = 32 * lhalf + j;
                         x[j] = s2 < nb ? (hi ? x1[j] : x[j]) : 0.f;
                     }
+                    // the exact diagonal-block terms of the fast-decaying channels
+                    const float *cor = kcor_of(m);
+                    if (*reinterpret_cast<const volatile int *>(cor + KCOR_FLAG)) {
+                        const int rr = 32 * (lq & 1) + lane, bb = rr >> 4, il = rr & 15;
+                        const float *ct = cor + (2 * bb + (lq >= 2 ? 1 : 0)) * KCOR_TRI + il * (il + 1) / 2;
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const int s2 = 32 * lhalf + j;
+                            if ((s2 >> 4) == bb && (s2 & 15) <= il) x[j] += ct[s2 & 15];
+                        }
+                    }
                 } else {
                     tmem_load<32>(tm_kq + lane_off + 32 * lhalf, x);
                 }
@@ -792,7 +897,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     if (lw == 4 && m + 2 < nchunks) compute_gates(m + 2);
                 } else {
                     // Kg = K e^{G} = KD e^{G_{m(r)}} in place of KD (its products are done)
-                    const float *fm = ktab_of(m) + 1024;
+                    const float *fm = ktab_of(m) + 512;
 #pragma unroll 2
                     for (int q2 = 0; q2 < 8; ++q2) {
                         const int idx = (gtid - 128) + 128 * q2;
@@ -1027,7 +1132,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                             float qv[8];
                             unpack8(*reinterpret_cast<const uint4 *>(qt + o), qv);
                             if constexpr (CH) {  // QD e^{G_{m(r)}}
-                                const float *f = ktab_of(m) + 1024 +
+                                const float *f = ktab_of(m) + 512 +
                                                  128 * (r >> 4) + 64 * lhalf + 8 * (4 * hh + j);
                                 const float4 d0 = *reinterpret_cast<const float4 *>(f);
                                 const float4 d1 = *reinterpret_cast<const float4 *>(f + 4);
@@ -1234,8 +1339,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     mma_commit(bars + SB_DRAIN + hv);
                     mbar_wait(bars + SB_DRAIN + hv, 0, kWaitLimit);
                 }
-            } else if (a.s_final && !(CH && *reinterpret_cast<volatile uint32_t *>(redo + item))) {
-                // (a flagged KDA item gets its final state from the exact re-run)
+            } else if (a.s_final) {
 #pragma unroll
                 for (int i = 0; i < 64; ++i) a.s_final[st_base + (size_t)(64 * hv + i) * DK + c] = s_reg[i];
             }
@@ -1350,13 +1454,13 @@ size_t ring_bytes(int slots) { return (size_t)slots * NRING * RING_STRIDE; }
 
 template <bool CH>
 cudaError_t launch_t(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
-                     const CUtensorMap &mv, int slots, uint32_t *redo, cudaStream_t s) {
+                     const CUtensorMap &mv, int slots, cudaStream_t s) {
     auto kern = chunk_pair_kernel<CH>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const long long items = (long long)a.n_seqs * a.H;
     kern<<<(unsigned)(2 * items), kThreads, SMEM_BYTES, s>>>(
-        a, mq, mk, mv, reinterpret_cast<uint8_t *>(a.scratch), slots, redo);
+        a, mq, mk, mv, reinterpret_cast<uint8_t *>(a.scratch), slots);
     return cudaGetLastError();
 }
 
@@ -1366,10 +1470,7 @@ bool chunk_pair_supported(const gdn_dims &d) {
     return d.dtype == GDN_BF16 && d.d_k == DK && d.d_v == DV && (long long)d.B * d.T < (1LL << 31);
 }
 
-size_t chunk_pair_scratch_bytes(const gdn_dims &d) {
-    const long long items = (long long)(d.n_seqs > 0 ? d.n_seqs : d.B) * d.H;
-    return ring_bytes(ring_slots_for_device()) + (size_t)((items * 4 + 255) & ~255LL);
-}
+size_t chunk_pair_scratch_bytes(const gdn_dims &) { return ring_bytes(ring_slots_for_device()); }
 
 cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches) {
     const long long items = (long long)a.n_seqs * a.H;
@@ -1389,17 +1490,10 @@ cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launche
         return cudaErrorInvalidValue;
     const int slots = ring_slots_for_device();
     if (slots <= 0) return cudaErrorInvalidValue;
-    uint32_t *redo = reinterpret_cast<uint32_t *>(reinterpret_cast<uint8_t *>(a.scratch) + ring_bytes(slots));
-    cudaError_t e = a.channel ? launch_t<true>(a, mq, mk, mv, slots, redo, s)
-                              : launch_t<false>(a, mq, mk, mv, slots, redo, s);
+    cudaError_t e = a.channel ? launch_t<true>(a, mq, mk, mv, slots, s)
+                              : launch_t<false>(a, mq, mk, mv, slots, s);
     if (e != cudaSuccess) return e;
     if (launches) ++*launches;
-    if (a.channel) {
-        // the items whose decay left the fast path's range, exactly on CUDA cores
-        PrefillArgs r = a;
-        r.redo = redo;
-        e = launch_chunk_simt(r, s, launches);
-    }
     return e;
 }
 

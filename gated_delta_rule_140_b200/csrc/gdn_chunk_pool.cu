@@ -82,6 +82,9 @@ constexpr uint32_t RG_BYTES = RG_YQ + 2 * YQ_HALF;
 constexpr uint32_t RING_STRIDE = RG_BYTES;
 constexpr uint32_t CS_V = RG_BYTES, CS_BYTES = RG_BYTES + 16384;
 constexpr uint32_t STAGE_TX = CS_BYTES;
+// o tiles of the output warps: two buffers of two 64 x 64 halves (bf16, 128-byte
+// swizzled), written back by TMA tensor stores
+constexpr uint32_t OFF_OBUF = 2 * CS_BYTES, OBUF_BYTES = 16384;
 static_assert((RG_ZT | RG_R | RG_YQ | YQ_HALF | YQ_QH | CS_V | CS_BYTES) % 1024 == 0, "chain buffer layout");
 
 // ---- local-CTA layout (GDN) -------------------------------------------------
@@ -103,12 +106,12 @@ constexpr int GR_G = 0, GR_B = 64, GR_BG = 128, GR_COLF = 192, GR_ROWF = 256, GR
               GR_GAM = 576, GR_DEC = 640, GR_INVK = 768, GR_INVQ = 832;
 
 // ---- bookkeeping (same offset in both roles) --------------------------------
-constexpr uint32_t OFF_COMMON = L_G0 + 2 * L_GSZ;  // 212992
-static_assert(2 * CS_BYTES <= OFF_COMMON, "chain shared memory layout");
-constexpr uint32_t CM_ABORT = 0, CM_TMEM = 8, CM_ISSUED = 16, CM_BARS = 64;  // issued: 8 ints
+constexpr uint32_t OFF_COMMON = OFF_OBUF + 2 * OBUF_BYTES;  // 215040
+static_assert(L_G0 + 2 * L_GSZ <= OFF_COMMON, "local shared memory layout");
+constexpr uint32_t CM_ABORT = 0, CM_TMEM = 8, CM_ISSUED = 16, CM_LANDED = 48, CM_BARS = 64;  // issued: 8 ints
 constexpr int NBARS = 24;
 // local CTAs: the descriptors of their first kDescCache tasks
-constexpr int kDescCache = 1024;
+constexpr int kDescCache = 960;
 constexpr uint32_t OFF_DESC = OFF_COMMON + 256;
 static_assert(CM_BARS + NBARS * 8 <= 256, "bookkeeping");
 constexpr uint32_t SMEM_USED = OFF_DESC + kDescCache * 16;
@@ -139,8 +142,8 @@ constexpr uint32_t ID_VZR = idesc_bf16(128, 192, true, false);   // V^T [Z | R^T
 constexpr uint32_t ID_SYQ = idesc_bf16(128, 192, false, false);  // S [Y^T | Qh^T]
 
 // named barriers
-constexpr int BAR_UPD = 5;  // chain: the state warps (local: 1-4 groups, 5-6 X conversion)
-constexpr int BAR_X = 5;
+constexpr int BAR_UPD = 5;  // chain: the state warps (local: 1-2 groups, 3-4 inversion warps)
+constexpr int BAR_OUT = 6;  // chain: the output warps
 
 struct PoolArgs {
     uint8_t *ring;         // nch x NR slots of RING_STRIDE bytes
@@ -170,6 +173,14 @@ __device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t *p) {
 }
 __device__ __forceinline__ void st_release_u64(uint64_t *p, uint64_t v) {
     asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_release_cta_u32(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_cta_u32(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
 }
 __device__ __forceinline__ uint64_t ready_tag(int rho, int m) {
     return ((uint64_t)(rho + 1) << 32) | (uint32_t)(m + 1);
@@ -346,6 +357,19 @@ struct Waiter {
         if (lane == 0) ok = wait(bar, parity);
         return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
     }
+    // a shared counter written by another warp of this CTA reaches `want`
+    __device__ __forceinline__ bool wait_count(const uint32_t *c, uint32_t want) const {
+        if (ld_acquire_cta_u32(c) >= want) return true;
+        const long long t0 = clock64();
+        while (ld_acquire_cta_u32(c) < want) {
+            if (*abort) return false;
+            if (clock64() - t0 > limit) {
+                raise();
+                return false;
+            }
+        }
+        return true;
+    }
     // a global word written by another CTA reaches `want` (== or >=)
     __device__ __forceinline__ bool wait_global(const uint64_t *p, uint64_t want, bool exact) const {
         uint64_t v = ld_acquire_u64(p);
@@ -373,7 +397,8 @@ struct Waiter {
 template <bool RAW>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v2) {
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v2,
+                  const __grid_constant__ CUtensorMap tm_o) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -382,6 +407,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
     uint64_t *bars = reinterpret_cast<uint64_t *>(cm + CM_BARS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(cm + CM_TMEM);
     int *issued = reinterpret_cast<int *>(cm + CM_ISSUED);  // loads issued per buffer
+    uint32_t *landed = reinterpret_cast<uint32_t *>(cm + CM_LANDED);  // chain: chunks landed
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool chain_role = (int)blockIdx.x < p.nch;
@@ -396,6 +422,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
         }
         fence_mbar_init();
         *abort_flag = 0;
+        *landed = 0;
         for (int i = 0; i < 8; ++i) issued[i] = 0;
         if (chain_role) {
             tma_prefetch_desc(&tm_v2);
@@ -452,21 +479,21 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             uint32_t bl_wait = 0, bx_wait = 0;
             const bool issuer = gtid == 0;       // MMAs
             const bool storer = gtid == 7 * 32;  // tile loads, the slot wait and the hand-off
-            // X of task xk -> Z^T (columns 0-63) and G^T = Y (64-191) of row n = 32 lq +
-            // lane, bf16, to the task's ring slot (K-major, 128-byte swizzled), by the
-            // 4 warps lw 4-7, 64 columns (one 128-byte row segment) at a time: each
-            // 8-lane group transposes its 8 rows x 8 16-byte chunks with three
-            // xor-shuffle stages, so that every store instruction writes whole
-            // 128-byte rows; then the storer hands the task over (the barrier
-            // orders the group's ring stores before its release)
-            auto convert_x = [&]() {
-                const Task tx = task(xk);
+            // X of task kx -> Z^T (columns 0-63) and G^T = Y (64-191) of row n = 32 lq +
+            // lane, bf16, to the task's ring slot (K-major, 128-byte swizzled), 64
+            // columns (one 128-byte row segment) per pass: lw 4-7 take passes 0-1 while
+            // lw 0-3 invert, lw 0-3 pass 2 after.  Each 8-lane group transposes its 8
+            // rows x 8 16-byte chunks with three xor-shuffle stages, so that every store
+            // instruction writes whole 128-byte rows.  The storer hands the task over
+            // (publish_x) two barriers later, once the stores have drained.
+            auto convert_x = [&](int kx, int p0, int p1) {
+                const Task tx = task(kx);
                 uint8_t *xs = p.ring + ((size_t)tx.b * NR + (tx.m % NR)) * RING_STRIDE;
                 const int j8 = lane & 7;
                 const int n0 = 32 * lq + (lane & ~7);
                 tc_fence_after();
 #pragma unroll 1
-                for (int pass = 0; pass < 3; ++pass) {
+                for (int pass = p0; pass < p1; ++pass) {
                     uint32_t w[32];
 #pragma unroll
                     for (int hq = 0; hq < 2; ++hq) {
@@ -505,11 +532,14 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                             make_uint4(w[4 * t], w[4 * t + 1], w[4 * t + 2], w[4 * t + 3]);
                 }
                 tc_fence_before();
-                named_bar_sync(BAR_X + g, 128);
-                if (storer)
-                    st_release_u64(p.flags + (size_t)tx.b * kFlagWords + 1 + (tx.m % NR),
-                                   ready_tag(tx.rho, tx.m));
             };
+            // (storer) task kx's tiles are all in its slot: the group barriers since its
+            // stores order them before this release
+            auto publish_x = [&](int kx) {
+                const Task tx = task(kx);
+                st_release_u64(p.flags + (size_t)tx.b * kFlagWords + 1 + (tx.m % NR), ready_tag(tx.rho, tx.m));
+            };
+            auto convert_part = [&](int kx) { convert_x(kx, lw >= 4 ? 0 : 2, lw >= 4 ? 2 : 3); };
             // raw tiles of task k into buffer k % 3 (an empty task completes the
             // buffer's phase with a plain arrive)
             auto issue_tma = [&](int k) {
@@ -634,12 +664,13 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     if (issuer && ok && xk >= 0) ok = wt.wait(bar_x, bx_wait & 1);
                     if (xk >= 0) ++bx_wait;
                     if (named_bar_or(BAR_G, 256, !ok || *abort_flag)) break;
-                    if (xk >= 0 && lw >= 4) convert_x();
-                    xk = -1;
+                    if (xk >= 0) convert_part(xk);
                     if (storer && k >= 2 && k + 1 < ntask) issue_tma(k + 1);
                     if (lw == 4 && k + 2 < ntask) compute_gates(k + 2);
                     if (g == 0 && k == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
                     named_bar_sync(BAR_G, 256);
+                    if (storer && xk >= 0) publish_x(xk);
+                    xk = -1;
                     continue;
                 }
                 if (L < C) {
@@ -741,15 +772,12 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 if (g == 0 && k == 0 && issuer) mbar_arrive(bars + LB_OFFSET);
                 // ---- T = (I + A)^{-1} in place of A: lw 0-3; meanwhile lw 4 prepares
                 //      the group's next gates and the storer hands over its last task
+                // (the X product converted here is handed over below, before this task's
+                // slot wait)
+                const int xpub = xk;
                 if (lw >= 4) {
-                    // the group's previous task's X product -> its ring slot, handed over
-                    if (xk >= 0) convert_x();
-                    // the slot's previous chunk must have been read by chain CTA b
-                    // before this task's first tile goes out (R, below)
-                    if (storer) {
-                        const uint64_t need = cons_needed(tk.rho, tk.m);
-                        if (need != 0) wt.wait_global(fl, need, false);
-                    }
+                    // the group's previous task's X product -> its ring slot
+                    if (xk >= 0) convert_part(xk);
                     if (lw == 4 && k + 2 < ntask) compute_gates(k + 2);
                 } else {
                     // (1) 16x16 diagonal blocks, right-looking forward substitution;
@@ -807,6 +835,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     AT[(o + 16 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[1];
                     AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft] = -y[2];
                     AT[(o + 24 + fg) * LDA + o + n0 + 2 * ft + 1] = -y[3];
+                    if (xk >= 0) convert_part(xk);
                 }
                 xk = -1;
                 if (named_bar_or(BAR_G, 256, *abort_flag)) break;
@@ -883,6 +912,13 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 }
                 fence_proxy_async_smem();
                 named_bar_sync(BAR_G, 256);
+                // the previous task handed over; then this task's slot: its previous chunk
+                // must have been read by chain CTA b before R goes out (below)
+                if (storer) {
+                    if (xpub >= 0) publish_x(xpub);
+                    const uint64_t need = cons_needed(tk.rho, tk.m);
+                    if (need != 0) ok = wt.wait_global(fl, need, false);
+                }
                 // ---- D_ab = [P; 0] [T_bg | T_b]: rows 0-63 = [P T_bg | R] ----------
                 if (issuer) {
                     tc_fence_after();
@@ -993,7 +1029,10 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 bool ok = true;
                 if (issuer) ok = wt.wait(bar_x, bx_wait & 1);
                 ++bx_wait;
-                if (!named_bar_or(BAR_G, 256, !ok || *abort_flag) && lw >= 4) convert_x();
+                if (!named_bar_or(BAR_G, 256, !ok || *abort_flag)) {
+                    convert_part(xk);
+                    if (!named_bar_or(BAR_G, 256, *abort_flag) && storer) publish_x(xk);
+                }
             }
             // drain: every MMA this group issued
             if (*abort_flag && issuer) {
@@ -1146,8 +1185,24 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
             // ---- lane 0 of warp 8: D[s] = V^T [Z | R^T] for each chunk once its
             //      stage has landed and chunk u - 2's accumulator has been read, and
             //      the loader: chunk u + 1 goes into stage (u + 1) & 1 once chunk
-            //      u - 1's products are done; the ring slot is given back (cons) as
-            //      soon as a chunk has landed
+            //      u - 1's products are done.  Lane 0 of warp 9 gives each ring slot
+            //      back (cons) once its chunk has landed: a gpu-scope release takes
+            //      about a thousand cycles, which the loader's loop cannot carry.
+            if (warp == 9 && lane == 0) {
+                uint64_t *fl = p.flags + (size_t)b * kFlagWords;
+                uint32_t u = 0;
+                bool ok = true;
+                for (int rho = 0; ok; ++rho) {
+                    Chain cc;
+                    if (!chain_of(rho, &cc)) break;
+                    // (an empty chain is passed at once: nothing of it is read)
+                    if (cc.nck == 0) st_release_u64(fl, (uint64_t)(rho + 1) << 32);
+                    for (int m = 0; m < cc.nck && ok; ++m, ++u) {
+                        ok = wt.wait_count(landed, u + 1);
+                        if (ok) st_release_u64(fl, cons_after(rho, m, cc.nck));
+                    }
+                }
+            }
             if (warp == 8 && lane == 0) {
                 uint64_t *fl = p.flags + (size_t)b * kFlagWords;
                 int lrho = 0, lm = 0;  // loader cursor: the chain and chunk of the next load
@@ -1155,13 +1210,11 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 bool lhave = false;
                 bool ok = true;
                 int *iss = issued;
-                // the next chain with chunks from round lrho on (an empty chain is
-                // passed at once: its chain CTA has nothing to read)
+                // the next chain with chunks from round lrho on
                 auto lopen = [&]() {
                     for (;; ++lrho) {
                         lhave = chain_of(lrho, &lcc);
                         if (!lhave || lcc.nck > 0) return;
-                        st_release_u64(fl, (uint64_t)(lrho + 1) << 32);
                     }
                 };
                 // the loads of the cursor's chunk (global index lu) into its stage (free)
@@ -1182,9 +1235,10 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     // the V tile two chunks on, into L2
                     if (lm + 2 < lcc.nck) tma_prefetch_l2_4d(&tm_v2, 0, (int)(t0 + 2 * C), 0, lcc.h);
                 };
-                // after the chunk has landed: give its slot back, move on
-                auto loaded = [&]() {
-                    st_release_u64(fl, cons_after(lrho, lm, lcc.nck));
+                // after the chunk has landed: count it (warp 9 gives the slot back),
+                // move the cursor on
+                auto loaded = [&](uint32_t uu) {
+                    st_release_cta_u32(landed, uu + 1);
                     if (++lm == lcc.nck) {
                         lm = 0;
                         ++lrho;
@@ -1201,7 +1255,7 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                         const int s = u & 1;
                         ok = wt.wait(bars + CB_FULL + s, (u >> 1) & 1);
                         if (!ok) break;
-                        loaded();
+                        loaded(u);
                         if (u >= 2) ok = wt.wait(bars + CB_DFREE + s, ((u >> 1) - 1) & 1);
                         if (!ok) break;
                         tc_fence_after();
@@ -1230,17 +1284,31 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                 }
             }
         } else {
-            // ---- output warps: D_O = o^T (lane j = value channel, columns = tokens)
+            // ---- output warps: D_O = o^T (lane j = value channel, columns = tokens).
+            //      A full chunk goes through an o tile in shared memory (two buffers)
+            //      and two TMA tensor stores issued by lane 0 of warp 12; a partial
+            //      one (a sequence's last) is stored row by row, so that nothing past
+            //      the sequence end is written.
             const int j = 32 * (warp & 3) + lane;
+            const bool ostorer = warp == 12 && lane == 0;
             uint32_t u = 0;
-            bool stop = false;
+            bool stop = false, prev_full = false;
             for (int rho = 0; !stop; ++rho) {
                 Chain cc;
                 if (!chain_of(rho, &cc)) break;
                 for (int m = 0; m < cc.nck; ++m, ++u) {
                     const int s = u & 1;
+                    const long long t0 = cc.t_begin + (long long)m * C;
+                    const int L = (int)min((long long)C, cc.t_end - t0);
+                    const bool full = L == C;
+                    // buffer s last held chunk u - 2: its stores have read it (all stores,
+                    // when chunk u - 1 was partial and committed none)
+                    if (ostorer && full) {
+                        if (prev_full) bulk_wait_read_but_last();
+                        else bulk_wait_read();
+                    }
                     const bool ok = wt.warp_wait(bars + CB_DSFULL + s, (u >> 1) & 1, lane);
-                    if (!ok) {
+                    if (named_bar_or(BAR_OUT, 128, !ok)) {
                         stop = true;
                         break;
                     }
@@ -1250,25 +1318,48 @@ chunk_pool_kernel(const PrefillArgs a, const PoolArgs p, const __grid_constant__
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bars + CB_DFREE + s);
-                    const long long t0 = cc.t_begin + (long long)m * C;
-                    const int L = (int)min((long long)C, cc.t_end - t0);
-                    // lane pairs (j even, j + 1) write bf16 pairs: the even lane row r,
+                    // lane pairs (j even, j + 1) hold bf16 pairs: the even lane row r,
                     // the odd lane row r + 1
-                    __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(a.o);
                     const bool odd = lane & 1;
+                    if (full) {
+                        uint8_t *ob = sm + OFF_OBUF + s * OBUF_BYTES + (j >> 6) * 8192;
+                        const int col = (j & 63) & ~1;
 #pragma unroll
-                    for (int r = 0; r < C; r += 2) {
-                        const float mine = odd ? x[r] : x[r + 1];
-                        const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                        const int row = odd ? r + 1 : r;
-                        if (row < L) {
+                        for (int r = 0; r < C; r += 2) {
+                            const float mine = odd ? x[r] : x[r + 1];
+                            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                            const int row = odd ? r + 1 : r;
                             const uint32_t v = odd ? pack2(other, x[r + 1]) : pack2(x[r], other);
-                            *reinterpret_cast<uint32_t *>(ob + ((t0 + row) * H + cc.h) * (long long)DV +
-                                                          (j & ~1)) = v;
+                            *reinterpret_cast<uint32_t *>(ob + row * 128 + (((col >> 3) ^ (row & 7)) << 4) +
+                                                          (col & 7) * 2) = v;
+                        }
+                        fence_proxy_async_smem();
+                        named_bar_sync(BAR_OUT, 128);
+                        if (ostorer) {
+                            const uint8_t *ot = sm + OFF_OBUF + s * OBUF_BYTES;
+                            tma_store_3d(&tm_o, ot, 0, cc.h, (int)t0);
+                            tma_store_3d(&tm_o, ot + 8192, 64, cc.h, (int)t0);
+                            bulk_commit();
+                        }
+                    } else {
+                        __nv_bfloat16 *ob = reinterpret_cast<__nv_bfloat16 *>(a.o);
+#pragma unroll
+                        for (int r = 0; r < C; r += 2) {
+                            const float mine = odd ? x[r] : x[r + 1];
+                            const float other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                            const int row = odd ? r + 1 : r;
+                            if (row < L) {
+                                const uint32_t v = odd ? pack2(other, x[r + 1]) : pack2(x[r], other);
+                                *reinterpret_cast<uint32_t *>(ob + ((t0 + row) * H + cc.h) * (long long)DV +
+                                                              (j & ~1)) = v;
+                            }
                         }
                     }
+                    prev_full = full;
                 }
             }
+            // every tile store complete before the CTA's shared memory goes away
+            if (ostorer) bulk_wait_all();
         }
     }
 
@@ -1338,10 +1429,12 @@ int device_sms() {
 }
 
 // The split of the SMs between chain CTAs and the local pool: the chain CTAs
-// take the chains in rounds of nch, so the state pass takes rounds x chunks
-// steps of ~kChainCost cycles; the pool works through every chunk at
-// ~kLocalCost SM-cycles each.  Pick nch to balance the two.
-constexpr double kChainCost = 2000.0, kLocalCost = 7500.0;
+// take the chains in rounds of nch, so the state pass takes rounds x (chunks
+// steps of ~kChainCost cycles + a fill and drain of ~kRoundCost); the pool works
+// through every chunk at ~kLocalCost SM-cycles each.  Pick nch to balance the
+// two.  (Measured on B200: ~4.0k cycles per chunk on a chain CTA running alone,
+// ~10.7k SM-cycles per task when the pool is the bound.)
+constexpr double kChainCost = 4000.0, kLocalCost = 10700.0, kRoundCost = 30000.0;
 
 PoolPlan plan_for(const gdn_dims &d, int nsm) {
     PoolPlan pl{0, 0};
@@ -1354,7 +1447,7 @@ PoolPlan plan_for(const gdn_dims &d, int nsm) {
     const int hi = (int)std::min<long long>(nchains, nsm - 1);
     for (int nch = 1; nch <= hi; ++nch) {
         const double rounds = (double)((nchains + nch - 1) / nch);
-        const double t_chain = rounds * nck * kChainCost;
+        const double t_chain = rounds * (nck * kChainCost + kRoundCost);
         const double t_local = (double)nchains * nck * kLocalCost / (nsm - nch);
         const double t = std::max(t_chain, t_local);
         if (t < best_t * 0.999) {
@@ -1409,9 +1502,9 @@ cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launche
     const int nsm = device_sms();
     const PoolPlan pl = plan_for(d, nsm);
     if (pl.nch <= 0) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, mo;
     if (!make_tile_map(&mq, a.q, a.dk, a.H, ntok) || !make_tile_map(&mk, a.k, a.dk, a.H, ntok) ||
-        !make_halves_map(&mv, a.v, a.H, ntok))
+        !make_halves_map(&mv, a.v, a.H, ntok) || !make_tile_map(&mo, a.o, a.dv, a.H, ntok))
         return cudaErrorInvalidValue;
     PoolArgs p{};
     uint8_t *ws = reinterpret_cast<uint8_t *>(a.scratch);
@@ -1451,8 +1544,8 @@ cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launche
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = a.raw ? cudaLaunchKernelEx(&cfg, chunk_pool_kernel<true>, a, p, mq, mk, mv)
-              : cudaLaunchKernelEx(&cfg, chunk_pool_kernel<false>, a, p, mq, mk, mv);
+    e = a.raw ? cudaLaunchKernelEx(&cfg, chunk_pool_kernel<true>, a, p, mq, mk, mv, mo)
+              : cudaLaunchKernelEx(&cfg, chunk_pool_kernel<false>, a, p, mq, mk, mv, mo);
     if (e != cudaSuccess) return e;
     if (launches) ++*launches;
     return cudaSuccess;

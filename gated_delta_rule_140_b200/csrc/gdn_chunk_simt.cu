@@ -115,7 +115,6 @@ chunk_simt_kernel(PrefillArgs a) {
     const int v0 = slice * kDvs;
     const int H = a.H, dv = a.dv;
 
-    if (a.redo && a.redo[(size_t)n * H + h] == 0u) return;
     long long t_begin, t_end;
     seq_range(a, n, &t_begin, &t_end);
 

@@ -36,14 +36,15 @@ struct PrefillArgs {
     int B, T, H, dk, dv, n_seqs;
     int channel;              // 1 = KDA channel-wise decay
     int bf16;                 // 1 = bf16 q/k/v/o, 0 = fp32
-    // CUDA-core kernel only: if set, process only the (sequence, head) items
-    // with redo[n * H + h] != 0 (the re-run of items another kernel flagged)
-    const uint32_t *redo;
     // fused input prologue (pool kernel): q, k unnormalised, log_alpha and beta
     // hold the decay and writing-rate logits, alpha_bias [H] (or null) is added
     // to the decay logit
     int raw;
     const float *alpha_bias;
+    // FG2-GDN (two-CTA kernel, channel decay): beta is [tokens, H, d_k], the
+    // writing rate per key channel; keys are scaled by its square root and the
+    // rate is 1 in the delta-rule step
+    int beta_channel;
 };
 
 struct DecodeArgs {

@@ -40,6 +40,9 @@ class Workload:
     n_seqs: int = 0           # > 0: variable-length packed batch
     len_range: tuple = field(default=(0, 0))
     steps: int = 0            # decode steps
+    beta_channel: bool = False  # FG2-GDN: beta per key channel [B,T,H,dk]
+    fast_channels: int = 0    # KDA: the first n key channels of every head decay at
+    fast_log_alpha: float = -30.0  # this log alpha per token (fast-forgetting channels)
 
 
 WORKLOADS = {
@@ -55,6 +58,10 @@ WORKLOADS = {
                  init_std=0.02, seed=4),
         Workload("gdn_long_prefill_bf16", "prefill", H=32, d=128, dtype=torch.bfloat16, B=1,
                  T=65536, seed=5),
+        Workload("kda_fast8_prefill_bf16", "prefill", H=32, d=128, dtype=torch.bfloat16, B=2,
+                 T=8192, decay="channel", alpha_shift=3.0, seed=3, fast_channels=8),
+        Workload("fg2_prefill_bf16", "prefill", H=32, d=128, dtype=torch.bfloat16, B=2,
+                 T=8192, decay="channel", alpha_shift=3.0, seed=6, beta_channel=True),
     )
 }
 
@@ -71,12 +78,14 @@ def _unit(x: torch.Tensor) -> torch.Tensor:
 
 def prefill_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype=torch.bfloat16,
                    decay: str = "scalar", seed: int = 0, alpha_shift: float = 2.0,
-                   init_std: float | None = None, lengths=None, gen=None) -> dict:
+                   init_std: float | None = None, lengths=None, gen=None,
+                   beta_channel: bool = False) -> dict:
     """Draw one prefill problem on the CPU.
 
     Returns a dict with q, k [B,T,H,dk] and v [B,T,H,dv] in ``dtype``;
     log_alpha [B,T,H] (scalar decay) or [B,T,H,dk] (channel decay) and beta
-    [B,T,H] in fp32; initial_state [N,H,dv,dk] fp32 or None; cu_seqlens int32
+    [B,T,H] (or [B,T,H,dk] with ``beta_channel``: FG2-GDN's rate per key
+    channel) in fp32; initial_state [N,H,dv,dk] fp32 or None; cu_seqlens int32
     [N+1] or None.  With ``lengths`` the batch is packed (B = 1, T = sum).
     """
     g = gen if gen is not None else torch.Generator().manual_seed(seed)
@@ -90,7 +99,7 @@ def prefill_inputs(B: int, T: int, H: int, dk: int, dv: int, *, dtype=torch.bflo
     q = _unit(torch.randn(B, T, H, dk, generator=g)).to(dtype)
     k = _unit(torch.randn(B, T, H, dk, generator=g)).to(dtype)
     v = torch.randn(B, T, H, dv, generator=g).to(dtype)
-    beta = torch.sigmoid(torch.randn(B, T, H, generator=g))
+    beta = torch.sigmoid(torch.randn(*((B, T, H, dk) if beta_channel else (B, T, H)), generator=g))
     la_shape = (B, T, H) if decay == "scalar" else (B, T, H, dk)
     log_alpha = -F.softplus(torch.randn(*la_shape, generator=g) + alpha_shift)
     s0 = None
@@ -130,9 +139,12 @@ def workload_inputs(name: str, **overrides) -> dict:
         n = overrides.get("n_seqs", w.n_seqs)
         lo, hi = overrides.get("len_range", w.len_range)
         lengths = varlen_lengths(n, lo, hi, g)
-    return prefill_inputs(overrides.get("B", w.B), overrides.get("T", w.T), H, d, d,
-                          dtype=w.dtype, decay=w.decay, alpha_shift=w.alpha_shift,
-                          init_std=w.init_std, lengths=lengths, gen=g)
+    x = prefill_inputs(overrides.get("B", w.B), overrides.get("T", w.T), H, d, d,
+                       dtype=w.dtype, decay=w.decay, alpha_shift=w.alpha_shift,
+                       init_std=w.init_std, lengths=lengths, gen=g, beta_channel=w.beta_channel)
+    if w.fast_channels:
+        x["log_alpha"][..., :w.fast_channels] = w.fast_log_alpha
+    return x
 
 
 def raw_prefill_inputs(B: int, T: int, H: int, d: int, *, seed: int = 0, bias: float = 2.0,

@@ -76,7 +76,18 @@ typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
  * recomputed by the CUDA-core kernel (exact for any decay) within the same
  * call.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use
  * the flags to compare the device paths. */
-enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4, GDN_FLAG_POOL = 8 };
+enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4, GDN_FLAG_POOL = 8,
+       GDN_FLAG_BETA_CHANNEL = 16 };
+/* GDN_FLAG_BETA_CHANNEL (prefill, channel decay): FG2-GDN's writing rate per key
+ * channel (FG2-GDN paper, section 3.2 "FG2-GDN Update Rule" and 3.6 "Chunkwise
+ * Parallel Training").  beta is then [B, T, H, d_k] fp32 (per-channel rates in
+ * (0, 1]) and the update is
+ *     S_t = S_{t-1} Diag(alpha_t) (I - k~_t k~_t^T) + v_t k~_t^T,  k~_t = sqrt(beta_t) . k_t,
+ * KDA's update with unit rate on the square-root-scaled keys.  It runs on the
+ * two-CTA kernel (bf16, d_k = d_v = 128): GDN_ERR_UNSUPPORTED for every other
+ * shape, with GDN_FLAG_CUDA_CORES, for gdn_recurrent_step and on the
+ * no-allocation entry point; GDN_ERR_INVALID with scalar decay,
+ * GDN_FLAG_ONE_CTA or GDN_FLAG_POOL. */
 
 typedef struct {
     int32_t B;       /* batch (1 for a packed batch)                           */

@@ -39,7 +39,10 @@ def oracle_heads(x: dict, picks, nthreads=0):
             sl = (slice(0, 1), slice(s, e), slice(h, h + 1))
         args = [x[name][sl] for name in ("q", "k", "v", "log_alpha", "beta")]
         s0 = None if x.get("initial_state") is None else x["initial_state"][n:n + 1, h:h + 1]
-        o, sf = oracle.recurrent(*args, s0, nthreads=nthreads)
+        if x["beta"].dim() == 4:  # FG2-GDN: rate per key channel
+            o, sf = oracle.fg2_recurrent(*args, None, s0, nthreads=nthreads)
+        else:
+            o, sf = oracle.recurrent(*args, s0, nthreads=nthreads)
         out.append((n, h, o[0, :, 0], sf[0, 0]))
     return out
 

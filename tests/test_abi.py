@@ -84,9 +84,28 @@ def test_prefill_kernel_choice(L):
                          (nat.GDN_FLAG_POOL | nat.GDN_FLAG_PAIR, nat.GDN_DECAY_SCALAR),
                          (nat.GDN_FLAG_POOL | nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_SCALAR),
                          (nat.GDN_FLAG_POOL, nat.GDN_DECAY_CHANNEL),
-                         (nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_CHANNEL), (16, nat.GDN_DECAY_SCALAR)):
+                         (nat.GDN_FLAG_ONE_CTA, nat.GDN_DECAY_CHANNEL), (32, nat.GDN_DECAY_SCALAR)):
         with pytest.raises(nat.GdnError):
             path(flags=flags, decay=decay)
+
+
+def test_fg2_rate_per_key_channel_runs_on_the_two_cta_kernel_only(L):
+    """GDN_FLAG_BETA_CHANNEL (FG2-GDN's writing rate per key channel) needs channel
+    decay and the two-CTA kernel's shapes; it is a prefill-only option."""
+    fg2 = nat.GDN_FLAG_BETA_CHANNEL
+    ch = nat.GDN_DECAY_CHANNEL
+    assert nat.chunk_fwd_path(_dims(decay=ch, flags=fg2)) == "tensor_core_pair"
+    assert nat.chunk_fwd_path(_dims(decay=ch, flags=fg2 | nat.GDN_FLAG_PAIR)) == "tensor_core_pair"
+    assert _call_fwd(L, _dims(flags=fg2)) == nat.GDN_ERR_INVALID                       # scalar decay
+    assert _call_fwd(L, _dims(decay=ch, flags=fg2 | nat.GDN_FLAG_POOL)) == nat.GDN_ERR_INVALID
+    assert _call_fwd(L, _dims(decay=ch, flags=fg2 | nat.GDN_FLAG_ONE_CTA)) == nat.GDN_ERR_INVALID
+    assert _call_fwd(L, _dims(decay=ch, flags=fg2 | nat.GDN_FLAG_CUDA_CORES)) == \
+        nat.GDN_ERR_UNSUPPORTED
+    assert _call_fwd(L, _dims(decay=ch, flags=fg2, dtype=nat.GDN_FP32)) == nat.GDN_ERR_UNSUPPORTED
+    assert _call_fwd(L, _dims(decay=ch, flags=fg2, d_k=64, d_v=64)) == nat.GDN_ERR_UNSUPPORTED
+    d = _dims(B=8, T=1, n_seqs=8, decay=ch, flags=fg2)
+    v = ctypes.c_void_p(FAKE)
+    assert L.gdn_recurrent_step(ctypes.byref(d), v, v, v, v, v, v, v, None) == nat.GDN_ERR_UNSUPPORTED
 
 
 FAKE = 0x10000  # 16-byte aligned, never dereferenced: every call below fails validation
@@ -116,7 +135,8 @@ def _call_fwd(L, dims, **kw):
     ("H = 0", {}, dict(H=0), nat.GDN_ERR_INVALID),
     ("bad dtype", {}, dict(dtype=7), nat.GDN_ERR_INVALID),
     ("bad decay", {}, dict(decay=3), nat.GDN_ERR_INVALID),
-    ("bad flags", {}, dict(flags=16), nat.GDN_ERR_INVALID),
+    ("bad flags", {}, dict(flags=32), nat.GDN_ERR_INVALID),
+    ("FG2 rate with scalar decay", {}, dict(flags=16), nat.GDN_ERR_INVALID),
     ("n_seqs != B", {}, dict(n_seqs=3), nat.GDN_ERR_INVALID),
     ("cu_seqlens with B > 1", dict(cu=FAKE), dict(n_seqs=2), nat.GDN_ERR_INVALID),
     ("cu_seqlens with no sequences", dict(cu=FAKE), dict(B=1, n_seqs=0), nat.GDN_ERR_INVALID),

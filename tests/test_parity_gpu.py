@@ -186,24 +186,41 @@ def test_tensor_core_and_cuda_core_paths_agree(cuda_ok):
         assert rel_err(s1, s2.cpu().numpy()) < 1e-2
 
 
-def test_kda_pair_kernel_and_out_of_range_decay_is_redone_exactly(cuda_ok):
-    """KDA's default path is the two-CTA kernel (16-token block references).
-    Decays inside its range: mild, and the KDA workload's (log alpha ~ -3).
-    Out of range (log alpha = -30 per token on 8 channels of head 0: e^-240 over
-    8 tokens): that (sequence, head) is recomputed by the CUDA-core kernel,
-    which is exact for any decay; head 1 stays on the fast path."""
-    for shift, seed in ((-2.0, 31), (3.0, 30)):
+def test_kda_pair_kernel_is_exact_for_any_decay_in_one_launch(cuda_ok):
+    """KDA runs on the two-CTA tensor-core kernel for every decay, in one launch.
+    Off the diagonal 16-token blocks the products are referenced at the row
+    block's start (both factors <= 1); inside a diagonal block a channel whose
+    decay over the block passes e^-80 is left out of the factored product and its
+    exact terms are added from a correction table.  Cases: mild decay; the KDA
+    workload's (log alpha ~ -3); -30 per token on 8 channels of head 0 (e^-480
+    over a block); -30 on every channel of head 0; channels straddling the
+    block-decay limit (-4.9 and -5.1 per token: 16 tokens give -78 and -82)."""
+    cases = [((-2.0, 31), None), ((3.0, 30), None), ((3.0, 30), ("ch8", -30.0)),
+             ((3.0, 34), ("all", -30.0)), ((3.0, 35), ("edge", None))]
+    for (shift, seed), strong in cases:
         x = prefill_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
                            alpha_shift=shift, seed=seed, init_std=0.05)
+        if strong is not None:
+            kind, val = strong
+            if kind == "ch8":
+                x["log_alpha"][:, :, 0, :8] = val
+            elif kind == "all":
+                x["log_alpha"][:, :, 0, :] = val
+            else:
+                x["log_alpha"][:, :, 0, 0:4] = -4.9
+                x["log_alpha"][:, :, 0, 4:8] = -5.1
+                x["log_alpha"][:, :, 1, 8:12] = -100.0
         d = to_dev(x)
         assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"])) == \
             "tensor_core_pair"
+        n0 = nat.launch_count()
         o, sf = _run(x)
+        assert nat.launch_count() - n0 == 1, "one launch, no re-run"
         _full_compare(x, o, sf, torch.bfloat16)
+    # final state aliasing the initial state, with fast-decaying channels
+    x = prefill_inputs(2, 200, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                       alpha_shift=3.0, seed=30, init_std=0.05)
     x["log_alpha"][:, :, 0, :8] = -30.0
-    o, sf = _run(x)
-    _full_compare(x, o, sf, torch.bfloat16)
-    # final state aliasing the initial state: the re-run must see the original S0
     d = to_dev(x)
     ref_o, ref_s = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"],
                              d["initial_state"].clone(), cuda_cores=True)
@@ -212,6 +229,38 @@ def test_kda_pair_kernel_and_out_of_range_decay_is_redone_exactly(cuda_ok):
     torch.cuda.synchronize()
     assert rel_err(o2, ref_o.float().cpu().numpy()) < 2e-2
     assert rel_err(s, ref_s.cpu().numpy()) < 1e-2
+
+
+def _fg2_compare(x, o, sf):
+    ro, rs = oracle.fg2_recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None,
+                                  x["initial_state"], x["cu_seqlens"])
+    to, ts = TOL[torch.bfloat16]
+    eo, es = rel_err(o, ro), rel_err(sf, rs)
+    assert eo <= to, f"o error {eo:.3g} > {to}"
+    assert es <= ts, f"final-state error {es:.3g} > {ts}"
+
+
+@pytest.mark.parametrize("case", ["ragged", "packed", "fast_channels"])
+def test_fg2_rate_per_key_channel_matches_oracle(cuda_ok, case):
+    """FG2-GDN: beta [B,T,H,d_k], keys scaled by sqrt(beta) in the two-CTA
+    kernel's gate pass, unit rate in the delta-rule step; against the oracle's
+    FG2 recurrence (which its pins tie to KDA and to KDA's chunkwise form).
+    Ragged sequences, a packed batch with empty ones, and fast-forgetting
+    channels (the exact diagonal-block correction with scaled keys)."""
+    if case == "packed":
+        x = prefill_inputs(1, 0, 3, 128, 128, dtype=torch.bfloat16, decay="channel",
+                           alpha_shift=3.0, init_std=0.05, lengths=[0, 1, 65, 200, 0, 130],
+                           gen=torch.Generator().manual_seed(81), beta_channel=True)
+    else:
+        x = prefill_inputs(2, 229, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                           alpha_shift=3.0, seed=82, init_std=0.05, beta_channel=True)
+        if case == "fast_channels":
+            x["log_alpha"][:, :, 0, :8] = -30.0
+    d = to_dev(x)
+    assert nat.chunk_fwd_path(nat.prefill_dims(d["q"], d["v"], d["log_alpha"],
+                                               beta_channel=True)) == "tensor_core_pair"
+    o, sf = _run(x, check=True)
+    _fg2_compare(x, o, sf)
 
 
 def test_kda_log_alpha_4_byte_aligned_gives_identical_results(cuda_ok):
@@ -319,6 +368,8 @@ FULL = {
     "gdn_prefill_bf16": [(0, 0), (3, 15), (1, 7)],
     "gdn_varlen_bf16": [(0, 0), (31, 15), (17, 5)],
     "kda_prefill_bf16": [(0, 0), (1, 31)],
+    "kda_fast8_prefill_bf16": [(0, 0), (1, 17)],
+    "fg2_prefill_bf16": [(0, 0), (1, 29)],
     "gdn_long_prefill_bf16": [(0, 0), (0, 31)],
 }
 
