@@ -55,6 +55,7 @@ PREFILL_LEGS = ("gdn_prefill_bf16", "gdn_varlen_bf16", "kda_prefill_bf16",
                 "kda_fast8_prefill_bf16", "fg2_prefill_bf16", "gdn_long_prefill_bf16")
 RAW_LEG = "gdn_prefill_bf16_raw"  # the config-2 shapes through the fused input prologue
 DECODE_LEG = "gdn_decode"
+DECODE_LEGS = (DECODE_LEG, "kda_decode")  # the scalar- and channel-decay decode steps
 KERNEL_SRC = {
     "tensor_core_pool": ("chunk_pool_kernel", "gdn_chunk_pool.cu"),
     "tensor_core_pair": ("chunk_pair_kernel", "gdn_chunk_pair.cu"),
@@ -593,7 +594,7 @@ def run_ours(args, rank, world, local):
     pre_s, dec_s = pre_ms / K / 1e3, dec_ms / K / 1e3
 
     # ---- every workload on its own, >= leg_seconds of device time each -------
-    want = PREFILL_LEGS + (RAW_LEG, DECODE_LEG) if args.legs == "all" else \
+    want = PREFILL_LEGS + (RAW_LEG,) + DECODE_LEGS if args.legs == "all" else \
         tuple() if args.legs == "none" else tuple(args.legs.split(","))
     legs = {}
     n_leg_launches = 0
@@ -604,32 +605,49 @@ def run_ours(args, rank, world, local):
                 legs[name] = raw_leg(head, dev, ws, stream, pk, pk_kind, args, K)
                 legs[name]["clocks"] = clocks.summary(clocks.rows[rows0:])
                 continue
-            if name == DECODE_LEG:
-                dec_reps = max(K, math.ceil(args.leg_seconds / max(dec_s, 1e-6)))
+            if name in DECODE_LEGS:
+                if name == args.decode_workload:
+                    wl, xl_cpu, xl, st_l, od_l, dec_fn, dl_s = wd, xd_cpu, xd, state, od, decode, dec_s
+                else:
+                    wl = WORKLOADS[name]
+                    xl_cpu = workload_inputs(name)
+                    xl = {k: v.to(dev) for k, v in xl_cpu.items()}
+                    st_l = xl["state"].clone()
+                    od_l = torch.empty(wl.B, wl.H, wl.d, dtype=wl.dtype, device=dev)
+
+                    def dec_fn(t, xl=xl, st_l=st_l, od_l=od_l, n=xl["q"].shape[0]):
+                        i = t % n
+                        recurrent_step(xl["q"][i], xl["k"][i], xl["v"][i], xl["log_alpha"][i],
+                                       xl["beta"][i], st_l, o=od_l)
+                    for t in range(3):
+                        dec_fn(t)
+                    dl_s = time_loop(lambda it=iter(range(10 ** 9)): dec_fn(next(it)), 3, stream) / 3 / 1e3
+                dec_reps = max(K, math.ceil(args.leg_seconds / max(dl_s, 1e-6)))
                 l0 = nat.launch_count()
-                ms = time_loop(lambda it=iter(range(10 ** 9)): decode(next(it)), dec_reps, stream)
+                ms = time_loop(lambda it=iter(range(10 ** 9)): dec_fn(next(it)), dec_reps, stream)
                 n_leg_launches += nat.launch_count() - l0
                 sec = ms / dec_reps / 1e3
-                fl = decode_flops(wd.B, wd.H, wd.d, wd.d)
-                by = decode_bytes(wd.B, wd.H, wd.d, wd.d, 2 if wd.dtype == torch.bfloat16 else 4,
-                                  wd.decay == "channel")
-                e2e_ms, h2d, d2h = e2e_decode(xd, state, od, wd, max(64, min(dec_reps, 2000)),
+                fl = decode_flops(wl.B, wl.H, wl.d, wl.d)
+                by = decode_bytes(wl.B, wl.H, wl.d, wl.d, 2 if wl.dtype == torch.bfloat16 else 4,
+                                  wl.decay == "channel")
+                e2e_ms, h2d, d2h = e2e_decode(xl, st_l, od_l, wl, max(64, min(dec_reps, 2000)),
                                               stream)
                 n_e2e = max(64, min(dec_reps, 2000))
                 legs[name] = {
                     "value": 1.0 / sec, "unit": "steps/s", "ms": sec * 1e3, "reps": dec_reps,
-                    "tokens_per_s": wd.B / sec,
+                    "tokens_per_s": wl.B / sec,
                     "roofline": roofline(fl, by, sec, pk, pk_kind,
                                          traffic_for("decode_kernel",
-                                                     "gated_delta_rule_140_b200/csrc/gdn_decode.cu"),
+                                                     "gated_delta_rule_140_b200/csrc/gdn_decode.cu",
+                                                     name),
                                          "decode_kernel"),
                     "e2e": {"value": n_e2e / (e2e_ms / 1e3), "unit": "steps/s",
                             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-                    "config": {"N": wd.B, "H": wd.H, "d_k": wd.d, "d_v": wd.d,
-                               "decay": wd.decay, "state": "fp32, in place"},
+                    "config": {"N": wl.B, "H": wl.H, "d_k": wl.d, "d_v": wl.d,
+                               "decay": wl.decay, "state": "fp32, in place"},
                 }
                 if world == 1 and not args.no_cpu_baseline:
-                    legs[name]["cpu_baseline"] = cpu_baseline_decode(xd_cpu)
+                    legs[name]["cpu_baseline"] = cpu_baseline_decode(xl_cpu)
             else:
                 leg = head if name == args.workload else PrefillLeg(name, dev, kflags, ws)
                 for _ in range(3):
@@ -719,6 +737,30 @@ def run_ours(args, rank, world, local):
     return 0
 
 
+def profile_once(args):
+    """Run one prefill workload ``warmup + steps`` times (no timing, one GPU): the
+    command the committed ncu captures profile, with -s/-c picking one launch."""
+    import torch
+    from gated_delta_rule_140_b200 import _native as nat
+    from gated_delta_rule_140_b200 import chunk_fwd
+    from gated_delta_rule_140_b200.inputs import workload_inputs
+    name, _, tok = args.profile_once.partition(":")
+    ov = {"T": int(tok)} if tok else {}
+    x = {k: (v.cuda() if isinstance(v, torch.Tensor) else v)
+         for k, v in workload_inputs(name, **ov).items()}
+    kw = {k: v for k, v in _kflags(args.prefill_kernel).items() if v}
+    ws = nat.Workspace()
+    for _ in range(args.warmup + args.steps):
+        chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"],
+                  x["cu_seqlens"], workspace=ws, **kw)
+    torch.cuda.synchronize()
+    st = ws.status()
+    path = nat.chunk_fwd_path(nat.prefill_dims(x["q"], x["v"], x["log_alpha"], x["cu_seqlens"],
+                                               beta_channel=x["beta"].dim() == 4, **kw))
+    print(f"{name} {ov} [{path}] x{args.warmup + args.steps}: status {st}")
+    return 0 if st == nat.GDN_OK else 1
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -737,7 +779,13 @@ def main():
                     default="default",
                     help="prefill kernel: the library's choice, or force one of the "
                          "tensor-core kernels or the fp32 CUDA-core kernel")
+    ap.add_argument("--profile-once", default=None, metavar="WORKLOAD[:T]",
+                    help="no timing: run one prefill workload (optionally with T tokens per "
+                         "sequence) warmup + steps times through the library and exit, for a "
+                         "profiler capture of one launch")
     args = ap.parse_args()
+    if args.profile_once:
+        return profile_once(args)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     rank, world, local = dist_setup(args.gpus)

@@ -45,9 +45,11 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
 
 enum class Path { kPool, kPair, kOneCta, kCudaCores };
 
-// The prefill kernel a call runs.  bf16, d_k = d_v = 128: GDN the single-CTA
-// tensor-core kernel (the two-CTA one with GDN_FLAG_PAIR), KDA the two-CTA
-// kernel; every other case, or GDN_FLAG_CUDA_CORES, the fp32 CUDA-core kernel.
+// The prefill kernel a call runs.  bf16, d_k = d_v = 128: KDA (and FG2-GDN) the
+// two-CTA kernel; GDN the pool kernel for few long sequences, else the two-CTA
+// kernel from 2048 tokens per sequence on average and the single-CTA kernel below
+// (the flags choose one); every other case, or GDN_FLAG_CUDA_CORES, the fp32
+// CUDA-core kernel.
 constexpr long long kPairMinMeanTokens = 2048;
 
 Path select_path(const gdn_dims &d) {
@@ -57,6 +59,7 @@ Path select_path(const gdn_dims &d) {
     if (d.flags & GDN_FLAG_ONE_CTA) return Path::kOneCta;
     if ((d.flags & GDN_FLAG_POOL) && gdn::chunk_pool_supported(d))
         return Path::kPool;
+    if (gdn::chunk_pool_preferred(d)) return Path::kPool;
     // scalar decay: the two-CTA kernel's steady state is faster per chunk, its
     // start-up (the first chunk through both SMs) longer; measured, it is ahead
     // from sequences of about 32 chunks on (16 chunks: 3% behind; 64: 3% ahead;

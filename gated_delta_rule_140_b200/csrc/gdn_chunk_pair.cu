@@ -142,15 +142,17 @@ constexpr uint32_t L_RAW2 = L_KX2 + 16384;         // KDA's second raw tiles [K0
 // the exact diagonal-block terms of the channels whose decay over a 16-token
 // block passes e^{-kMaxNegLogDecay}: fp32 [block][A, P][lower triangle incl. the
 // diagonal], and a word "the table holds this chunk's terms", two tables by chunk
-// parity; then the gate group's staging of such (block, channel) pairs: a count,
-// the pairs (block << 8 | channel) and their 16 cumulative log decays, KSTG_CAP
-// pairs at a time
+// parity; then the gate group's count of such channels per block.  The channels'
+// k, q and cumulative log decays (fp32 [16] each) are staged, up to KSTG_CAP per
+// block at a time, in the B region (free between the gate pass's B_FREE wait and
+// its rewrite of B).
 constexpr int KCOR_TRI = 136, KCOR_FLAG = 8 * KCOR_TRI;
 constexpr uint32_t KCOR_BYTES = (KCOR_FLAG + 4) * 4;
 constexpr uint32_t L_KCOR = L_RAW2 + RAW_BYTES;
-constexpr int KSTG_CAP = 32;
-constexpr uint32_t L_KSTG = L_KCOR + 2 * KCOR_BYTES;  // count | pairs at +16 | G at +256
-constexpr uint32_t KSTG_BYTES = 256 + KSTG_CAP * 16 * 4;
+constexpr uint32_t L_KSTG = L_KCOR + 2 * KCOR_BYTES;  // 4 counts (one per block)
+constexpr uint32_t KSTG_BYTES = 16;
+constexpr int KSTG_CAP = 48;                          // channels per block and batch
+static_assert(4 * KSTG_CAP * 48 * 4 <= 2 * 160 * 128, "staging in the B region");
 constexpr uint32_t TM_KD = 192;                    // D = [D_0 | D_1 | D_2 | D_3], 160 columns
 constexpr uint32_t ID_KD = idesc_bf16(128, 160, false, false);
 static_assert(L_RAW2 % 1024 == 0, "KDA layout");
@@ -209,6 +211,62 @@ __device__ __forceinline__ void unpack8(uint4 u, float *x) {
 // masked elsewhere; factored across the 16-block boundary), a block strictly
 // below it (factored at the 16-block boundary: e^{g_r - g_e} e^{g_e - g_s}, both
 // factors <= 1), or a block above it (not called: nothing to keep).
+// KDA's correction table for one batch of staged fast-decaying channels: the
+// 128 threads gtid < 128 each take one row i of one block's A (ap = 0, s < i)
+// or P (ap = 1, s <= i) part and sum, over the block's staged channels, left_i
+// k_s e^{G_i - G_s} (left = k for A, q for P).  An exponent below -88 gives 0 in
+// fp32 and is skipped.  Out of line: it runs only when a channel decays that
+// fast, and keeps the gate loop's code small.
+__device__ __noinline__ void kda_correction_rows(float *cor, const float *stg, int n0, int n1, int n2,
+                                                 int n3, int p0, int cap, int gtid) {
+    if (gtid >= 128) return;
+    const int blk = gtid >> 5, ap = (gtid >> 4) & 1, i = gtid & 15;
+    const int nb = blk == 0 ? n0 : blk == 1 ? n1 : blk == 2 ? n2 : n3;
+    const int np = min(cap, nb - p0);
+    float *row = cor + (2 * blk + ap) * 136 + i * (i + 1) / 2;
+    float acc[16];
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) acc[s2] = (p0 > 0 && s2 <= i) ? row[s2] : 0.f;
+    const float *d = stg + blk * cap * 48;
+    for (int pp = 0; pp < np; ++pp, d += 48) {
+        const float gi = d[32 + i], li = d[16 * ap + i];
+#pragma unroll
+        for (int s2 = 0; s2 < 16; ++s2) {
+            const float ex = gi - d[32 + s2];
+            if (s2 < i + ap && ex > -88.f) acc[s2] = fmaf(li * d[s2], __expf(ex), acc[s2]);
+        }
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2)
+        if (s2 <= i) row[s2] = acc[s2];
+}
+
+// FG2-GDN: K <- sqrt(beta) . K in place for one gate thread's 16 rows (block rq)
+// and two key channels (c0, c0 + 1 = column cc of atom ac); rows past the
+// sequence end (>= L) are zero and stay so.  Out of line like the correction.
+__device__ __noinline__ void fg2_scale_keys(uint8_t *rawp, const float *bp, size_t row_stride, int rq,
+                                            int L, int ac, int cc) {
+    const uint32_t cof = (uint32_t)((cc & 7) * 2);
+#pragma unroll
+    for (int i0 = 0; i0 < 16; i0 += 8) {
+        float b0[8], b1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const bool in = 16 * rq + i0 + i < L;
+            b0[i] = in ? __ldg(bp + (i0 + i) * row_stride) : 0.f;
+            b1[i] = in ? __ldg(bp + (i0 + i) * row_stride + 1) : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t *pk = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + sw128(16 * rq + i0 + i, cc >> 3) + cof);
+            const uint32_t kw = *pk;
+            __nv_bfloat162 t = __floats2bfloat162_rn(__uint_as_float(kw << 16) * sqrtf(b0[i]),
+                                                     __uint_as_float(kw & 0xffff0000u) * sqrtf(b1[i]));
+            *pk = *reinterpret_cast<uint32_t *>(&t);
+        }
+    }
+}
+
 __device__ __forceinline__ void decay_row(float *x, int r, int rq, int half, const float *gr,
                                           bool incl) {
     const float *g = gr + GR_G;
@@ -366,8 +424,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
             tma_prefetch_desc(&tm_v);
         }
     }
-    if (CH && rank == 0)
-        for (int i = tid; i < 2 * (int)(KCOR_BYTES / 4); i += kThreads)
+    if (CH && rank == 0)  // the correction tables and the staging count
+        for (int i = tid; i < (int)((2 * KCOR_BYTES + 16) / 4); i += kThreads)
             reinterpret_cast<float *>(sm + L_KCOR)[i] = 0.f;
     cluster_sync();  // both CTAs' barriers and flags are initialised
     if (rank == 1 && tid == 0) {
@@ -530,8 +588,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                 bool ok = true;
                 if (m + 1 < nchunks) {  // the next chunk's per-channel gates into L2
                     const int pr = gtid >> 2, pc = gtid & 3;  // 64 rows x 4 lines of 128 B
-                    if (t0 + C + pr < t_end)
+                    if (t0 + C + pr < t_end) {
                         asm volatile("prefetch.global.L2 [%0];" ::"l"(a.log_alpha + ((t0 + C + pr) * H + h) * DK + 32 * pc));
+                        if (a.beta_channel)  // FG2-GDN: the rates per key channel likewise
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.beta + ((t0 + C + pr) * H + h) * DK + 32 * pc));
+                    }
                 }
                 // ---- KDA gates: G_rc by a prefix sum over the rows (thread: two
                 //      channels, the 16 rows of block rq) and the block totals; then
@@ -567,8 +628,13 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     gl1[i] = acc1;
                 }
                 *reinterpret_cast<float2 *>(ktab + 128 * rq + c0) = make_float2(acc0, acc1);
-                // (the staging count, read last in chunk m - 1 before its final barrier)
-                if (gtid == 0) *reinterpret_cast<volatile uint32_t *>(sm + L_KSTG) = 0u;
+                // a channel whose decay over this block passes e^{-kMaxNegLogDecay} leaves
+                // the factored diagonal block (below): registered here, counted after the
+                // next barrier (the count was reset before chunk m - 1's last barrier)
+                const bool fl0 = -acc0 > kMaxNegLogDecay, fl1 = -acc1 > kMaxNegLogDecay;
+                uint32_t *kst_cnt = reinterpret_cast<uint32_t *>(sm + L_KSTG);
+                const int my0 = fl0 ? (int)atomicAdd(kst_cnt + rq, 1u) : -1;
+                const int my1 = fl1 ? (int)atomicAdd(kst_cnt + rq, 1u) : -1;
                 // chunk m's tiles: group 0 loads them once chunk m - 2 is done with
                 // this parity's raw tiles, table and gate rows (rows past the sequence
                 // end are zeroed here)
@@ -617,20 +683,9 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     __nv_bfloat162 t = __floats2bfloat162_rn(x, y);
                     return *reinterpret_cast<uint32_t *>(&t);
                 };
-                if (a.beta_channel) {
-                    // FG2-GDN: K <- sqrt(beta) . K in place, this thread's rows and channels
-                    const float *bp = a.beta + ((t0 + 16 * rq) * H + h) * DK + c0;
-#pragma unroll 4
-                    for (int i = 0; i < 16; ++i) {
-                        if (16 * rq + i >= L) break;  // (rows past the end are zero)
-                        const float b0 = bp[(size_t)i * H * DK], b1 = bp[(size_t)i * H * DK + 1];
-                        uint32_t *pk = reinterpret_cast<uint32_t *>(
-                            rawp + ac * L_RAW_AC + sw128(16 * rq + i, cc >> 3) + cof);
-                        const uint32_t kw = *pk;
-                        *pk = bf2(__uint_as_float(kw << 16) * sqrtf(b0),
-                                  __uint_as_float(kw & 0xffff0000u) * sqrtf(b1));
-                    }
-                }
+                // FG2-GDN: K <- sqrt(beta) . K in place, this thread's rows and channels
+                if (a.beta_channel)
+                    fg2_scale_keys(rawp, a.beta + ((t0 + 16 * rq) * H + h) * DK + c0, (size_t)H * DK, rq, L, ac, cc);
                 // this block's end end_rq = off_rq + acc; the factors from it to the later
                 // blocks' starts and to the chunk end (all <= 1)
                 const float end0 = off0 + acc0, end1 = off1 + acc1;
@@ -641,55 +696,38 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     tb1[bi] = bi > rq ? __expf(ob1[bi] - end1) : 0.f;
                 }
                 const float tc0 = __expf(run0 - end0), tc1 = __expf(run1 - end1);
-                // a channel whose decay over this block passes e^{-kMaxNegLogDecay} leaves
-                // the factored diagonal block; its exact terms k_r k_s e^{G_r - G_s} and
-                // q_r k_s e^{G_r - G_s} (s <= r in the block, exponent <= 0) go to the
-                // correction table, every thread taking a few entries over all such
-                // (block, channel) pairs, which their owners stage
-                const bool fl0 = -acc0 > kMaxNegLogDecay, fl1 = -acc1 > kMaxNegLogDecay;
+                // the exact diagonal-block terms of the flagged channels, k_r k_s e^{G_r -
+                // G_s} and q_r k_s e^{G_r - G_s} (s <= r in the block, exponent <= 0), go
+                // to the correction table, every thread taking a few entries over all
+                // flagged (block, channel) pairs, which their owners stage
                 float *cor = kcor_of(m);
-                uint32_t *kst_cnt = reinterpret_cast<uint32_t *>(sm + L_KSTG);
-                int *kst_pair = reinterpret_cast<int *>(sm + L_KSTG + 16);
-                float *kst_g = reinterpret_cast<float *>(sm + L_KSTG + 256);
-                const int my0 = fl0 ? (int)atomicAdd(kst_cnt, 1u) : -1;
-                const int my1 = fl1 ? (int)atomicAdd(kst_cnt, 1u) : -1;
-                const bool anyfl = named_bar_or(BAR_G, 256, fl0 || fl1);
+                const int nc0 = (int)reinterpret_cast<volatile uint32_t *>(kst_cnt)[0];
+                const int nc1 = (int)reinterpret_cast<volatile uint32_t *>(kst_cnt)[1];
+                const int nc2 = (int)reinterpret_cast<volatile uint32_t *>(kst_cnt)[2];
+                const int nc3 = (int)reinterpret_cast<volatile uint32_t *>(kst_cnt)[3];
+                const int maxcnt = max(max(nc0, nc1), max(nc2, nc3));
+                const bool anyfl = maxcnt > 0;
                 if (anyfl) {
-                    const int npairs = (int)*reinterpret_cast<volatile uint32_t *>(kst_cnt);
-                    for (int p0 = 0; p0 < npairs; p0 += KSTG_CAP) {
-#pragma unroll
+                    // [block][slot][k | q | G][16] fp32
+                    float *stg = reinterpret_cast<float *>(sm + L_BREG);
+                    for (int p0 = 0; p0 < maxcnt; p0 += KSTG_CAP) {
+#pragma unroll 1
                         for (int hc = 0; hc < 2; ++hc) {
                             const int my = hc ? my1 : my0;
                             if (my < p0 || my >= p0 + KSTG_CAP) continue;
-                            kst_pair[my - p0] = (rq << 8) | (c0 + hc);
+                            float *d = stg + (rq * KSTG_CAP + (my - p0)) * 48;
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) kst_g[(my - p0) * 16 + i] = hc ? gl1[i] : gl0[i];
+                            for (int i = 0; i < 16; ++i) {
+                                const uint32_t o = sw128(16 * rq + i, cc >> 3) + cof;
+                                const uint32_t kw = *reinterpret_cast<const uint32_t *>(rawp + ac * L_RAW_AC + o);
+                                const uint32_t qw = *reinterpret_cast<const uint32_t *>(rawp + ac * L_RAW_AC + 8192 + o);
+                                d[i] = hc ? __uint_as_float(kw & 0xffff0000u) : __uint_as_float(kw << 16);
+                                d[16 + i] = hc ? __uint_as_float(qw & 0xffff0000u) : __uint_as_float(qw << 16);
+                                d[32 + i] = hc ? gl1[i] : gl0[i];
+                            }
                         }
                         named_bar_sync(BAR_G, 256);
-                        const int np = min(KSTG_CAP, npairs - p0);
-                        for (int e = gtid; e < KCOR_FLAG; e += 256) {
-                            const int blk = e / (2 * KCOR_TRI), ap = (e / KCOR_TRI) & 1, tri = e % KCOR_TRI;
-                            int i = 0;
-                            while ((i + 1) * (i + 2) / 2 <= tri) ++i;
-                            const int s2 = tri - i * (i + 1) / 2;
-                            float accv = p0 == 0 ? 0.f : cor[e];
-                            if (ap == 1 || s2 < i) {
-                                for (int pp = 0; pp < np; ++pp) {
-                                    const int pr = kst_pair[pp];
-                                    if ((pr >> 8) != blk) continue;
-                                    const int c = pr & 255;
-                                    const uint8_t *tile = rawp + (c >> 6) * L_RAW_AC;
-                                    const uint32_t co = (uint32_t)((c & 7) * 2);
-                                    auto ld = [&](uint32_t off) {
-                                        return __uint_as_float((uint32_t)*reinterpret_cast<const uint16_t *>(tile + off) << 16);
-                                    };
-                                    const float ks = ld(sw128(16 * blk + s2, (c & 63) >> 3) + co);
-                                    const float li = ld((ap ? 8192u : 0u) + sw128(16 * blk + i, (c & 63) >> 3) + co);
-                                    accv += li * ks * __expf(kst_g[pp * 16 + i] - kst_g[pp * 16 + s2]);
-                                }
-                            }
-                            cor[e] = accv;
-                        }
+                        kda_correction_rows(cor, stg, nc0, nc1, nc2, nc3, p0, KSTG_CAP, gtid);
                         named_bar_sync(BAR_G, 256);
                     }
                 }
@@ -734,6 +772,8 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                     }
                 }
                 fence_proxy_async_smem();
+                // (every read of the staging count is behind a barrier by now)
+                if (gtid < 4) reinterpret_cast<volatile uint32_t *>(kst_cnt)[gtid] = 0u;
                 if (named_bar_or(BAR_G, 256, *abort_flag)) break;
                 if (issuer) mbar_arrive(bars + LB_GATE);
             }

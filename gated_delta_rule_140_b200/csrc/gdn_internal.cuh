@@ -65,6 +65,7 @@ cudaError_t launch_chunk_pool(const PrefillArgs &a, cudaStream_t s, int *launche
 size_t chunk_pool_scratch_bytes(const gdn_dims &d);
 // bf16 d_k = d_v = 128 scalar-decay shapes the pool kernel takes (fixed rows)
 bool chunk_pool_supported(const gdn_dims &d);
+bool chunk_pool_preferred(const gdn_dims &d);
 size_t chunk_tc_scratch_bytes(const gdn_dims &d);
 size_t chunk_pair_scratch_bytes(const gdn_dims &d);
 // bf16 d_k = d_v = 128 shapes (either decay) the two-CTA kernel takes

@@ -56,6 +56,8 @@ WORKLOADS = {
                  decay="channel", alpha_shift=3.0, seed=3),
         Workload("gdn_decode", "decode", H=32, d=128, dtype=torch.bfloat16, B=256, steps=64,
                  init_std=0.02, seed=4),
+        Workload("kda_decode", "decode", H=32, d=128, dtype=torch.bfloat16, B=256, steps=64,
+                 decay="channel", alpha_shift=3.0, init_std=0.02, seed=7),
         Workload("gdn_long_prefill_bf16", "prefill", H=32, d=128, dtype=torch.bfloat16, B=1,
                  T=65536, seed=5),
         Workload("kda_fast8_prefill_bf16", "prefill", H=32, d=128, dtype=torch.bfloat16, B=2,

@@ -61,21 +61,22 @@ typedef enum { GDN_BF16 = 0, GDN_FP32 = 1 } gdn_dtype;
 typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
 
 /* Kernel selection flags (gdn_dims.flags).  0 = the library's choice: for bf16
- * with d_k = d_v = 128 the two-CTA tensor-core kernel for channel decay, and for
- * scalar decay the two-CTA kernel when the sequences hold 2048 tokens or more on
- * average (B * T / n_seqs; its steady state is faster, its start-up longer) and
- * the single-CTA tensor-core kernel otherwise; the fp32 CUDA-core kernel for
- * every other shape.  GDN_FLAG_PAIR selects the two-CTA kernel and
- * GDN_FLAG_ONE_CTA the single-CTA kernel for scalar decay (the two are
- * exclusive; GDN_FLAG_ONE_CTA with channel decay is GDN_ERR_INVALID).
- * The two-CTA kernel runs one thread-block cluster per sequence and head: one
- * SM computes the chunk-local matrices, the other runs the sequential state
- * pass; it needs a larger workspace (see below).  For channel decay it covers
- * chunks whose decay over any 8 consecutive tokens stays above e^-80 on every
- * key channel; the (sequence, head) pairs with a chunk beyond that are
- * recomputed by the CUDA-core kernel (exact for any decay) within the same
- * call.  GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use
- * the flags to compare the device paths. */
+ * with d_k = d_v = 128, channel decay on the two-CTA tensor-core kernel; scalar
+ * decay on the pool kernel when the sequences hold 2048 tokens or more on average
+ * (B * T / n_seqs) and there are at most SMs / 4 (sequence, head) chains, else on
+ * the two-CTA kernel from 2048 tokens on average and on the single-CTA kernel
+ * below; the fp32 CUDA-core kernel for every other shape.  GDN_FLAG_POOL,
+ * GDN_FLAG_PAIR and GDN_FLAG_ONE_CTA select one of the three tensor-core kernels
+ * (at most one of them; GDN_FLAG_POOL and GDN_FLAG_ONE_CTA take scalar decay only,
+ * else GDN_ERR_INVALID).  The pool kernel is one persistent grid over all SMs:
+ * a few CTAs run the sequential state pass of all chains while the others work
+ * through the chunk-local steps of every chunk, so one long sequence uses the
+ * whole GPU.  The two-CTA kernel runs one thread-block cluster per sequence and
+ * head (one SM for the chunk-local steps, one for the state pass); it is exact
+ * for any decay (a channel that decays by more than e^-80 over 16 tokens has its
+ * within-block terms taken directly).  Both need a larger workspace (see below).
+ * GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use the flags
+ * to compare the device paths. */
 enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4, GDN_FLAG_POOL = 8,
        GDN_FLAG_BETA_CHANNEL = 16 };
 /* GDN_FLAG_BETA_CHANNEL (prefill, channel decay): FG2-GDN's writing rate per key
@@ -113,7 +114,9 @@ typedef struct {
  * two-CTA tensor-core kernel adds a ring of four 64 KiB slots for each SM index
  * of the device (2 x its SM count), through which the chunk-local SM hands each
  * chunk's matrices to the state SM; it is written before it is read and needs
- * no initialisation.  The other kernels need only the header.  Returns 0 for
+ * no initialisation.  The pool kernel adds eight 73 KiB ring slots per chain
+ * CTA, its hand-off flags and (packed batches) a table of round offsets, which
+ * a small kernel before it writes.  The other kernels need only the header.  Returns 0 for
  * invalid dims. */
 size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims);
 
@@ -197,9 +200,9 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
  * Instead of a caller workspace it uses one fixed device array of
  * GDN_NOALLOC_SCRATCH_BYTES compiled into the library.  Where the selected
  * kernel's workspace (gdn_chunk_fwd_workspace_size) does not fit in it -- the
- * two-CTA tensor-core kernel's ring never does -- the call runs the single-CTA
- * tensor-core kernel (scalar decay) or the CUDA-core kernel (channel decay)
- * instead, whose workspace is the header alone.
+ * rings of the pool and two-CTA tensor-core kernels never do -- the call runs
+ * the single-CTA tensor-core kernel (scalar decay) or the CUDA-core kernel
+ * (channel decay) instead, whose workspace is the header alone.
  * Problems whose workspace exceeds the array even then return
  * GDN_ERR_UNSUPPORTED before anything is launched.  All other arguments,
  * layouts and results are those of gdn_chunk_fwd.
@@ -236,9 +239,9 @@ gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_strea
 gdn_status gdn_workspace_status(void *workspace, gdn_stream_t stream);
 
 /* Name of the prefill kernel gdn_chunk_fwd selects for `dims` (static
- * storage): "tensor_core_pair" (two-CTA tcgen05 kernel), "tensor_core"
- * (single-CTA tcgen05 kernel) or "cuda_core" (fp32 CUDA cores); NULL for
- * invalid dims. */
+ * storage): "tensor_core_pool" (pool tcgen05 kernel), "tensor_core_pair"
+ * (two-CTA tcgen05 kernel), "tensor_core" (single-CTA tcgen05 kernel) or
+ * "cuda_core" (fp32 CUDA cores); NULL for invalid dims. */
 const char *gdn_chunk_fwd_path(const gdn_dims *dims);
 
 /* Human-readable name of a status code (static storage). */

@@ -58,27 +58,34 @@ def test_workspace_size(L):
 
 def test_prefill_kernel_choice(L):
     """The library's choice for bf16 d = 128: channel decay on the two-CTA
-    kernel; scalar decay on the two-CTA kernel from a mean sequence length of
-    2048 tokens (B * T / n_seqs), on the single-CTA kernel below; the flags
+    kernel; scalar decay on the pool kernel when the sequences average 2048
+    tokens or more and the (sequence, head) chains number at most a quarter of
+    the SMs (148 without a device), else on the two-CTA kernel from a mean of
+    2048 tokens (B * T / n_seqs) and on the single-CTA kernel below; the flags
     override it, GDN_FLAG_ONE_CTA only for scalar decay and not with
     GDN_FLAG_PAIR; other shapes on CUDA cores."""
     path = lambda **kw: nat.chunk_fwd_path(_dims(**kw))
-    assert path(B=4, T=1024, n_seqs=4) == "tensor_core"
-    assert path(B=4, T=2048, n_seqs=4) == "tensor_core_pair"
-    assert path(B=4, T=2048, n_seqs=0) == "tensor_core_pair"      # n_seqs 0: B sequences
+    # few long sequences: the pool kernel (chains <= 37)
+    assert path(B=4, T=2048, n_seqs=4) == "tensor_core_pool"        # 16 chains
+    assert path(B=4, T=2048, n_seqs=0) == "tensor_core_pool"        # n_seqs 0: B sequences
+    assert path(B=1, T=65536, n_seqs=1, H=32) == "tensor_core_pool"  # 32 chains
+    assert path(B=1, T=65536, n_seqs=9) == "tensor_core_pool"       # 36 chains
+    # many: the two-CTA kernel from 2048 tokens, the single-CTA one below
+    assert path(B=4, T=4096, n_seqs=4, H=16) == "tensor_core_pair"   # 64 chains
+    assert path(B=1, T=65536, n_seqs=10) == "tensor_core_pair"      # 40 chains
+    assert path(B=1, T=65536, n_seqs=32, H=16) == "tensor_core_pair"
     assert path(B=4, T=2047, n_seqs=0) == "tensor_core"
-    assert path(B=4, T=4096, n_seqs=4) == "tensor_core_pair"
-    assert path(B=1, T=65536, n_seqs=1) == "tensor_core_pair"
-    assert path(B=1, T=65536, n_seqs=64) == "tensor_core"         # packed, mean 1024
-    assert path(B=1, T=65536, n_seqs=32) == "tensor_core_pair"    # packed, mean 2048
+    assert path(B=1, T=65536, n_seqs=64) == "tensor_core"           # packed, mean 1024
     assert path(B=1, T=65536, n_seqs=1, flags=nat.GDN_FLAG_ONE_CTA) == "tensor_core"
+    assert path(B=1, T=65536, n_seqs=1, flags=nat.GDN_FLAG_PAIR) == "tensor_core_pair"
     assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_PAIR) == "tensor_core_pair"
     assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_CUDA_CORES) == "cuda_core"
     assert path(decay=nat.GDN_DECAY_CHANNEL) == "tensor_core_pair"
+    assert path(decay=nat.GDN_DECAY_CHANNEL, B=1, T=65536, n_seqs=1) == "tensor_core_pair"
     assert path(dtype=nat.GDN_FP32) == "cuda_core"
     assert path(d_k=64, d_v=64, flags=nat.GDN_FLAG_ONE_CTA) == "cuda_core"
     assert path(B=4, T=4096, n_seqs=4, flags=nat.GDN_FLAG_POOL) == "tensor_core_pool"
-    assert path(B=1, T=65536, n_seqs=40, flags=nat.GDN_FLAG_POOL) == "tensor_core_pool"
+    assert path(B=4, T=128, n_seqs=4, flags=nat.GDN_FLAG_POOL) == "tensor_core_pool"
     assert path(dtype=nat.GDN_FP32, flags=nat.GDN_FLAG_POOL) == "cuda_core"
     for flags, decay in ((nat.GDN_FLAG_ONE_CTA | nat.GDN_FLAG_PAIR, nat.GDN_DECAY_SCALAR),
                          (nat.GDN_FLAG_POOL | nat.GDN_FLAG_PAIR, nat.GDN_DECAY_SCALAR),
