@@ -212,33 +212,46 @@ __device__ __forceinline__ void unpack8(uint4 u, float *x) {
 // below it (factored at the 16-block boundary: e^{g_r - g_e} e^{g_e - g_s}, both
 // factors <= 1), or a block above it (not called: nothing to keep).
 // KDA's correction table for one batch of staged fast-decaying channels: the
-// 128 threads gtid < 128 each take one row i of one block's A (ap = 0, s < i)
-// or P (ap = 1, s <= i) part and sum, over the block's staged channels, left_i
-// k_s e^{G_i - G_s} (left = k for A, q for P).  An exponent below -88 gives 0 in
-// fp32 and is skipped.  Out of line: it runs only when a channel decays that
-// fast, and keeps the gate loop's code small.
-__device__ __noinline__ void kda_correction_rows(float *cor, const float *stg, int n0, int n1, int n2,
-                                                 int n3, int p0, int cap, int gtid) {
-    if (gtid >= 128) return;
-    const int blk = gtid >> 5, ap = (gtid >> 4) & 1, i = gtid & 15;
-    const int nb = blk == 0 ? n0 : blk == 1 ? n1 : blk == 2 ? n2 : n3;
-    const int np = min(cap, nb - p0);
-    float *row = cor + (2 * blk + ap) * 136 + i * (i + 1) / 2;
-    float acc[16];
+// 256 gate threads each take entries e = gtid + 256 j of the table [block][A, P]
+// [lower triangle (i, s)] and sum, over the block's staged channels, left_i k_s
+// e^{G_i - G_s} (left = k for A, s < i; q for P, s <= i).  An exponent below -88
+// gives 0 in fp32 and is skipped.  Out of line: it runs only when a channel decays
+// that fast, and keeps the gate loop's code small.
+__device__ __noinline__ void kda_correction_entries(float *cor, const float *stg, int n0, int n1,
+                                                    int n2, int n3, int p0, int cap, int gtid) {
+    for (int e = gtid; e < 8 * 136; e += 256) {
+        const int blk = e / 272, ap = (e / 136) & 1, tri = e % 136;
+        int i = (int)((sqrtf(8.f * (float)tri + 1.f) - 1.f) * 0.5f);
+        if ((i + 1) * (i + 2) / 2 <= tri) ++i;
+        if (i * (i + 1) / 2 > tri) --i;
+        const int s2 = tri - i * (i + 1) / 2;
+        float accv = p0 == 0 ? 0.f : cor[e];
+        if (ap == 1 || s2 < i) {
+            const int nb = blk == 0 ? n0 : blk == 1 ? n1 : blk == 2 ? n2 : n3;
+            const int np = min(cap, nb - p0);
+            const float *d = stg + blk * cap * 48;
+            // four channels at a time, four partial sums: the loads and exponentials
+            // of one group overlap instead of chaining through one accumulator
+            float a4[4] = {0.f, 0.f, 0.f, 0.f};
+            int pp = 0;
+            for (; pp + 4 <= np; pp += 4) {
 #pragma unroll
-    for (int s2 = 0; s2 < 16; ++s2) acc[s2] = (p0 > 0 && s2 <= i) ? row[s2] : 0.f;
-    const float *d = stg + blk * cap * 48;
-    for (int pp = 0; pp < np; ++pp, d += 48) {
-        const float gi = d[32 + i], li = d[16 * ap + i];
-#pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2) {
-            const float ex = gi - d[32 + s2];
-            if (s2 < i + ap && ex > -88.f) acc[s2] = fmaf(li * d[s2], __expf(ex), acc[s2]);
+                for (int q = 0; q < 4; ++q) {
+                    const float *dq = d + (pp + q) * 48;
+                    const float ex = dq[32 + i] - dq[32 + s2];
+                    const float w = ex > -88.f ? __expf(ex) : 0.f;
+                    a4[q] = fmaf(dq[16 * ap + i] * dq[s2], w, a4[q]);
+                }
+            }
+            for (; pp < np; ++pp) {
+                const float *dq = d + pp * 48;
+                const float ex = dq[32 + i] - dq[32 + s2];
+                if (ex > -88.f) a4[0] = fmaf(dq[16 * ap + i] * dq[s2], __expf(ex), a4[0]);
+            }
+            accv += (a4[0] + a4[1]) + (a4[2] + a4[3]);
         }
+        cor[e] = accv;
     }
-#pragma unroll
-    for (int s2 = 0; s2 < 16; ++s2)
-        if (s2 <= i) row[s2] = acc[s2];
 }
 
 // FG2-GDN: K <- sqrt(beta) . K in place for one gate thread's 16 rows (block rq)
@@ -247,23 +260,23 @@ __device__ __noinline__ void kda_correction_rows(float *cor, const float *stg, i
 __device__ __noinline__ void fg2_scale_keys(uint8_t *rawp, const float *bp, size_t row_stride, int rq,
                                             int L, int ac, int cc) {
     const uint32_t cof = (uint32_t)((cc & 7) * 2);
+    // all 16 rows' rate pairs in flight at once (one 8-byte load each when aligned)
+    const bool al8 = ((reinterpret_cast<uintptr_t>(bp) | (row_stride * sizeof(float))) & 7) == 0;
+    float2 bb[16];
 #pragma unroll
-    for (int i0 = 0; i0 < 16; i0 += 8) {
-        float b0[8], b1[8];
+    for (int i = 0; i < 16; ++i) {
+        const float *pi = bp + i * row_stride;
+        bb[i] = 16 * rq + i >= L ? make_float2(0.f, 0.f)
+                : al8            ? __ldg(reinterpret_cast<const float2 *>(pi))
+                                 : make_float2(__ldg(pi), __ldg(pi + 1));
+    }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const bool in = 16 * rq + i0 + i < L;
-            b0[i] = in ? __ldg(bp + (i0 + i) * row_stride) : 0.f;
-            b1[i] = in ? __ldg(bp + (i0 + i) * row_stride + 1) : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            uint32_t *pk = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + sw128(16 * rq + i0 + i, cc >> 3) + cof);
-            const uint32_t kw = *pk;
-            __nv_bfloat162 t = __floats2bfloat162_rn(__uint_as_float(kw << 16) * sqrtf(b0[i]),
-                                                     __uint_as_float(kw & 0xffff0000u) * sqrtf(b1[i]));
-            *pk = *reinterpret_cast<uint32_t *>(&t);
-        }
+    for (int i = 0; i < 16; ++i) {
+        uint32_t *pk = reinterpret_cast<uint32_t *>(rawp + ac * L_RAW_AC + sw128(16 * rq + i, cc >> 3) + cof);
+        const uint32_t kw = *pk;
+        __nv_bfloat162 t = __floats2bfloat162_rn(__uint_as_float(kw << 16) * sqrtf(bb[i].x),
+                                                 __uint_as_float(kw & 0xffff0000u) * sqrtf(bb[i].y));
+        *pk = *reinterpret_cast<uint32_t *>(&t);
     }
 }
 
@@ -727,7 +740,7 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                             }
                         }
                         named_bar_sync(BAR_G, 256);
-                        kda_correction_rows(cor, stg, nc0, nc1, nc2, nc3, p0, KSTG_CAP, gtid);
+                        kda_correction_entries(cor, stg, nc0, nc1, nc2, nc3, p0, KSTG_CAP, gtid);
                         named_bar_sync(BAR_G, 256);
                     }
                 }
