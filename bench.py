@@ -56,6 +56,7 @@ PREFILL_LEGS = ("gdn_prefill_bf16", "gdn_varlen_bf16", "kda_prefill_bf16",
 RAW_LEG = "gdn_prefill_bf16_raw"  # the config-2 shapes through the fused input prologue
 DECODE_LEG = "gdn_decode"
 DECODE_LEGS = (DECODE_LEG, "kda_decode")  # the scalar- and channel-decay decode steps
+FIG3_LEGS = tuple(f"fig3_{T // 1024}kx{32768 // T}" for T in (2048, 4096, 8192, 16384, 32768))
 KERNEL_SRC = {
     "tensor_core_pool": ("chunk_pool_kernel", "gdn_chunk_pool.cu"),
     "tensor_core_pair": ("chunk_pair_kernel", "gdn_chunk_pair.cu"),
@@ -596,6 +597,8 @@ def run_ours(args, rank, world, local):
     # ---- every workload on its own, >= leg_seconds of device time each -------
     want = PREFILL_LEGS + (RAW_LEG,) + DECODE_LEGS if args.legs == "all" else \
         tuple() if args.legs == "none" else tuple(args.legs.split(","))
+    if args.fig3:
+        want = want + FIG3_LEGS
     legs = {}
     n_leg_launches = 0
     if rank == 0 or world > 1:
@@ -722,6 +725,9 @@ def run_ours(args, rank, world, local):
             "clocks": clocks.summary(),
             "legs": legs,
         }
+        if all(n in legs for n in FIG3_LEGS):
+            # FG2-GDN Fig. 3's comparison: throughput of 32k x 1 over 2k x 16
+            line["fig3_ratio_32kx1_over_2kx16"] = legs["fig3_32kx1"]["value"] / legs["fig3_2kx16"]["value"]
         if world == 1 and not args.no_cpu_baseline:
             if args.workload in legs and "cpu_baseline" in legs[args.workload]:
                 line["cpu_baseline"] = legs[args.workload]["cpu_baseline"]
@@ -779,6 +785,9 @@ def main():
                     default="default",
                     help="prefill kernel: the library's choice, or force one of the "
                          "tensor-core kernels or the fp32 CUDA-core kernel")
+    ap.add_argument("--fig3", action="store_true",
+                    help="add the FG2-GDN Fig. 3 shape sweep to the legs: 32k tokens as 2k x 16, "
+                         "4k x 8, 8k x 4, 16k x 2 and 32k x 1 (GDN, 16 heads, d = 128)")
     ap.add_argument("--profile-once", default=None, metavar="WORKLOAD[:T]",
                     help="no timing: run one prefill workload (optionally with T tokens per "
                          "sequence) warmup + steps times through the library and exit, for a "

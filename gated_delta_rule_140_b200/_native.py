@@ -56,6 +56,8 @@ def lib():
     L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
     L.gdn_recurrent_step.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp]
     L.gdn_recurrent_step.restype = ctypes.c_int
+    L.gdn_recurrent_verify.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, vp]
+    L.gdn_recurrent_verify.restype = ctypes.c_int
     L.gdn_chunk_fwd_raw.argtypes = [D, vp, vp, vp, fp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
     L.gdn_chunk_fwd_raw.restype = ctypes.c_int
     L.gdn_noalloc_status.argtypes = [vp]
@@ -274,6 +276,43 @@ def chunk_fwd_raw(q_raw, k_raw, v, alpha_logit, beta_logit, alpha_bias=None,
     if check:
         _raise_on_status(ws.status(stream), "gdn_chunk_fwd_raw (device)")
     return o, final_state
+
+
+def recurrent_verify(q, k, v, log_alpha, beta, state, n_commit=None, *, outputs=True, o=None,
+                     check=False, stream=None):
+    """Multi-token verification (gdn_recurrent_verify): K draft tokens per sequence
+    from ``state`` [N,H,dv,dk] fp32.  q, k [N,K,H,dk]; v [N,K,H,dv]; log_alpha
+    [N,K,H] or [N,K,H,dk]; beta [N,K,H]; ``n_commit`` int32 [N] on the device or
+    None.  Returns o [N,K,H,dv] (None with ``outputs=False``); the state becomes
+    the state after the first n_commit[n] tokens of each sequence (untouched for
+    None or 0)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_dev(name, t, q.dtype)
+    _check_dev("log_alpha", log_alpha, torch.float32)
+    _check_dev("beta", beta, torch.float32)
+    _check_dev("state", state, torch.float32)
+    _check_dev("n_commit", n_commit, torch.int32)
+    N, K, H, dk = q.shape
+    dv = v.shape[-1]
+    dims = Dims(N, K, H, dk, dv, N, _dtype_code(q.dtype),
+                GDN_DECAY_CHANNEL if log_alpha.dim() == 4 else GDN_DECAY_SCALAR, 0)
+    if outputs and o is None:
+        o = torch.empty(N, K, H, dv, dtype=q.dtype, device=q.device)
+    if not outputs:
+        o = None
+    st = lib().gdn_recurrent_verify(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(n_commit),
+                                    _ptr(o), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_recurrent_verify")
+    if check:
+        s = stream if stream is not None else torch.cuda.current_stream()
+        try:
+            s.synchronize()
+        except RuntimeError as e:
+            raise GdnError(GDN_ERR_CUDA, f"gdn_recurrent_verify (device): {e}") from e
+    return o
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, *, o=None, check=False, stream=None):

@@ -198,6 +198,32 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta, float *state_inout,
+                                const int32_t *n_commit, void *o, gdn_stream_t stream) {
+    gdn_status st = check_dims(dims, false);
+    if (st != GDN_OK) return st;
+    const gdn_dims &d = *dims;
+    if (d.B == 0 || d.T == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !state_inout) return GDN_ERR_INVALID;
+    if (!aligned16(state_inout)) return GDN_ERR_INVALID;
+    for (const void *p : {q, k, (const void *)o})
+        if (p && (reinterpret_cast<uintptr_t>(p) & (d.dtype == GDN_BF16 ? 7u : 15u))) return GDN_ERR_INVALID;
+    if ((reinterpret_cast<uintptr_t>(v) | reinterpret_cast<uintptr_t>(log_alpha) |
+         reinterpret_cast<uintptr_t>(beta) | reinterpret_cast<uintptr_t>(n_commit)) & 3u)
+        return GDN_ERR_INVALID;
+    gdn::VerifyArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.state = state_inout; a.n_commit = n_commit; a.o = o;
+    a.N = d.B; a.K = d.T; a.H = d.H; a.dk = d.d_k; a.dv = d.d_v;
+    a.channel = d.decay == GDN_DECAY_CHANNEL;
+    a.bf16 = d.dtype == GDN_BF16;
+    int launches = 0;
+    cudaError_t e = gdn::launch_verify(a, reinterpret_cast<cudaStream_t>(stream), &launches);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
     if (!workspace || workspace_bytes < gdn::kWorkspaceHeader || !aligned16(workspace))
         return GDN_ERR_INVALID;

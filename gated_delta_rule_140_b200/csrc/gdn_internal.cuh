@@ -56,7 +56,19 @@ struct DecodeArgs {
     int channel, bf16;
 };
 
+// Multi-token verification: K draft tokens per sequence, token-major [N, K, H].
+struct VerifyArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    float *state;
+    const int32_t *n_commit;  // device [N] or null (no commit)
+    void *o;                  // [N, K, H, dv] or null (no outputs)
+    int N, K, H, dk, dv;
+    int channel, bf16;
+};
+
 // Host launchers (each returns cudaGetLastError() of its launches).
+cudaError_t launch_verify(const VerifyArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_chunk_simt(const PrefillArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s, int *launches);
 cudaError_t launch_chunk_tc(const PrefillArgs &a, cudaStream_t s, int *launches);

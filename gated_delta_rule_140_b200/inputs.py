@@ -64,6 +64,11 @@ WORKLOADS = {
                  T=8192, decay="channel", alpha_shift=3.0, seed=3, fast_channels=8),
         Workload("fg2_prefill_bf16", "prefill", H=32, d=128, dtype=torch.bfloat16, B=2,
                  T=8192, decay="channel", alpha_shift=3.0, seed=6, beta_channel=True),
+        # FG2-GDN section 4.5, Fig. 3: prefill shapes of 32k tokens, sequence length x batch
+        # from 2k x 16 to 32k x 1 (GDN layers of the 1.3B models: 16 heads of d = 128)
+        *(Workload(f"fig3_{T // 1024}kx{32768 // T}", "prefill", H=16, d=128,
+                   dtype=torch.bfloat16, B=32768 // T, T=T, seed=8)
+          for T in (2048, 4096, 8192, 16384, 32768)),
     )
 }
 

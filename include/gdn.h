@@ -183,6 +183,24 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
                               const float *log_alpha, const float *beta,
                               float *state_inout, void *o, gdn_stream_t stream);
 
+/* Multi-token verification for speculative decoding (a chain of K drafts; the
+ * TreeWY finding on the Gated DeltaNet-2 page: no per-node state snapshots).
+ * For N = dims->B sequences of K = dims->T draft tokens each, the recurrence of
+ * gdn_recurrent_step runs through the K tokens from state_inout:
+ *   o_t = S_t q_t for t = 0..K-1 (if o is not null);
+ *   state_inout <- S_c, the state after the first c = n_commit[n] tokens of
+ *   sequence n (n_commit: device int32 [N], values clamped to [0, K]; c = 0, or a
+ *   null n_commit, leaves the state untouched).
+ * Speculative decoding peeks at a draft (o, n_commit = null), picks the accepted
+ * length j per sequence, then commits it (o = null, n_commit = j): the state after
+ * j tokens is recomputed from the state before them, so nothing per position is
+ * kept.  Layouts are token-major: q, k [N,K,H,d_k]; v, o [N,K,H,d_v]; log_alpha
+ * [N,K,H] or [N,K,H,d_k]; beta [N,K,H]; state_inout fp32 [N,H,d_v,d_k].  No
+ * workspace.  GDN_FLAG_BETA_CHANNEL is GDN_ERR_UNSUPPORTED. */
+gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                                const float *log_alpha, const float *beta, float *state_inout,
+                                const int32_t *n_commit, void *o, gdn_stream_t stream);
+
 /* Size of the device array that gdn_chunk_fwd_noalloc uses in place of a
  * caller workspace: 256 KiB, held by every GPU that loads the library until
  * the process exits. */

@@ -172,6 +172,30 @@ def test_recurrent_step_rejects_bad_arguments(L, kw, expect):
                                 v(p["beta"]), v(p["state"]), v(p["o"]), None) == expect
 
 
+@pytest.mark.parametrize("kw,dims_kw,expect", [
+    (dict(q=None), {}, nat.GDN_ERR_INVALID),
+    (dict(state=FAKE + 8), {}, nat.GDN_ERR_INVALID),
+    (dict(k=FAKE + 2), {}, nat.GDN_ERR_INVALID),
+    (dict(n_commit=FAKE + 2), {}, nat.GDN_ERR_INVALID),
+    ({}, dict(flags=nat.GDN_FLAG_BETA_CHANNEL, decay=nat.GDN_DECAY_CHANNEL), nat.GDN_ERR_UNSUPPORTED),
+    ({}, dict(d_k=96), nat.GDN_ERR_UNSUPPORTED),
+])
+def test_recurrent_verify_rejects_bad_arguments(L, kw, dims_kw, expect):
+    p = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, state=FAKE, n_commit=FAKE, o=FAKE)
+    p.update(kw)
+    v = lambda x: None if x is None else ctypes.c_void_p(x)
+    d = _dims(**{**dict(B=8, T=5, n_seqs=8), **dims_kw})
+    assert L.gdn_recurrent_verify(ctypes.byref(d), v(p["q"]), v(p["k"]), v(p["v"]), v(p["la"]),
+                                  v(p["beta"]), v(p["state"]), v(p["n_commit"]), v(p["o"]),
+                                  None) == expect
+
+
+def test_recurrent_verify_without_tokens_is_a_noop_without_device(L):
+    for dims_kw in (dict(B=0, T=5, n_seqs=0), dict(B=8, T=0, n_seqs=8)):
+        d = _dims(**dims_kw)
+        assert L.gdn_recurrent_verify(ctypes.byref(d), *([None] * 8), None) == nat.GDN_OK
+
+
 def test_empty_batch_is_a_noop_without_device(L):
     # B = 0: nothing to launch, nothing touched -- succeeds even without a GPU
     d = _dims(B=0, n_seqs=0)

@@ -393,6 +393,70 @@ def test_full_workload_sampled(cuda_ok, name, kernel):
 # --------------------------------------------------------------------------- #
 # decode                                                                      #
 # --------------------------------------------------------------------------- #
+def _verify_inputs(N, K, H, d, dtype, decay, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = prefill_inputs(N, K, H, d, d, dtype=dtype, decay=decay, init_std=0.3, gen=g,
+                       alpha_shift=2.0 if decay == "scalar" else 3.0)
+    return x
+
+
+@pytest.mark.parametrize("decay,dtype,d", [("scalar", torch.bfloat16, 128),
+                                           ("channel", torch.bfloat16, 128),
+                                           ("scalar", torch.float32, 64)])
+def test_recurrent_verify_outputs_and_commit_match_oracle(cuda_ok, decay, dtype, d):
+    """Multi-token verification: the outputs of all K drafts equal the oracle's
+    recurrence over the K tokens from the state; the committed state equals the
+    oracle's state after each sequence's first n_commit tokens (0 .. K, 0 leaves it
+    as it was); a peek (no commit) leaves the state bit for bit untouched."""
+    from gated_delta_rule_140_b200 import recurrent_verify
+    N, K, H = 6, 7, 3
+    x = _verify_inputs(N, K, H, d, dtype, decay, 91)
+    d_ = to_dev(x)
+    s0 = d_["initial_state"].contiguous()
+    commit = torch.tensor([0, 1, 3, 7, 5, 2], dtype=torch.int32)
+    to, ts = TOL[dtype]
+    ro, _ = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+    # peek
+    st = s0.clone()
+    o = recurrent_verify(d_["q"], d_["k"], d_["v"], d_["log_alpha"], d_["beta"], st, check=True)
+    assert torch.equal(st, s0)
+    assert rel_err(o, ro) <= to
+    # commit with and without outputs
+    for outputs in (True, False):
+        st = s0.clone()
+        o2 = recurrent_verify(d_["q"], d_["k"], d_["v"], d_["log_alpha"], d_["beta"], st,
+                              commit.cuda(), outputs=outputs, check=True)
+        if outputs:
+            assert torch.equal(o2, o)
+        for n in range(N):
+            j = int(commit[n])
+            if j == 0:
+                assert torch.equal(st[n], s0[n])
+                continue
+            sl = lambda t: t[n:n + 1, :j]
+            _, rs = oracle.recurrent(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["log_alpha"]),
+                                     sl(x["beta"]), x["initial_state"][n:n + 1])
+            assert rel_err(st[n], rs[0]) <= ts, (n, j)
+
+
+def test_recurrent_verify_commit_all_equals_decode_steps_bitwise(cuda_ok):
+    """Committing all K tokens is K decode steps in the same arithmetic order:
+    states and outputs are bit-identical to gdn_recurrent_step called K times."""
+    from gated_delta_rule_140_b200 import recurrent_verify
+    N, K, H = 5, 4, 2
+    for decay in ("scalar", "channel"):
+        x = to_dev(_verify_inputs(N, K, H, 128, torch.bfloat16, decay, 92))
+        st = x["initial_state"].clone()
+        o = recurrent_verify(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], st,
+                             torch.full((N,), K, dtype=torch.int32, device="cuda"), check=True)
+        st2 = x["initial_state"].clone()
+        outs = [recurrent_step(x["q"][:, t].contiguous(), x["k"][:, t].contiguous(),
+                               x["v"][:, t].contiguous(), x["log_alpha"][:, t].contiguous(),
+                               x["beta"][:, t].contiguous(), st2) for t in range(K)]
+        torch.cuda.synchronize()
+        assert torch.equal(st, st2)
+        assert torch.equal(o, torch.stack(outs, 1))
+
 def _decode_check(x, picks, dtype):
     steps = x["q"].shape[0]
     d = to_dev(x)
