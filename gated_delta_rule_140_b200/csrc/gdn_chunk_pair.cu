@@ -143,16 +143,17 @@ constexpr uint32_t L_RAW2 = L_KX2 + 16384;         // KDA's second raw tiles [K0
 // block passes e^{-kMaxNegLogDecay}: fp32 [block][A, P][lower triangle incl. the
 // diagonal], and a word "the table holds this chunk's terms", two tables by chunk
 // parity; then the gate group's count of such channels per block.  The channels'
-// k, q and cumulative log decays (fp32 [16] each) are staged, up to KSTG_CAP per
-// block at a time, in the B region (free between the gate pass's B_FREE wait and
-// its rewrite of B).
+// k, q, cumulative log decays G and per-token decays alpha_s = e^{G_s - G_{s-1}}
+// (fp32 [16] each) are staged, up to KSTG_CAP per block at a time, in the B region
+// (free between the gate pass's B_FREE wait and its rewrite of B).
 constexpr int KCOR_TRI = 136, KCOR_FLAG = 8 * KCOR_TRI;
 constexpr uint32_t KCOR_BYTES = (KCOR_FLAG + 4) * 4;
 constexpr uint32_t L_KCOR = L_RAW2 + RAW_BYTES;
 constexpr uint32_t L_KSTG = L_KCOR + 2 * KCOR_BYTES;  // 4 counts (one per block)
 constexpr uint32_t KSTG_BYTES = 16;
-constexpr int KSTG_CAP = 48;                          // channels per block and batch
-static_assert(4 * KSTG_CAP * 48 * 4 <= 2 * 160 * 128, "staging in the B region");
+constexpr int KSTG_CAP = 40;                          // channels per block and batch
+constexpr int KSTG_REC = 64;                          // floats per staged channel
+static_assert(4 * KSTG_CAP * KSTG_REC * 4 <= 2 * 160 * 128, "staging in the B region");
 constexpr uint32_t TM_KD = 192;                    // D = [D_0 | D_1 | D_2 | D_3], 160 columns
 constexpr uint32_t ID_KD = idesc_bf16(128, 160, false, false);
 static_assert(L_RAW2 % 1024 == 0, "KDA layout");
@@ -212,46 +213,48 @@ __device__ __forceinline__ void unpack8(uint4 u, float *x) {
 // below it (factored at the 16-block boundary: e^{g_r - g_e} e^{g_e - g_s}, both
 // factors <= 1), or a block above it (not called: nothing to keep).
 // KDA's correction table for one batch of staged fast-decaying channels: the
-// 256 gate threads each take entries e = gtid + 256 j of the table [block][A, P]
-// [lower triangle (i, s)] and sum, over the block's staged channels, left_i k_s
-// e^{G_i - G_s} (left = k for A, s < i; q for P, s <= i).  An exponent below -88
-// gives 0 in fp32 and is skipped.  Out of line: it runs only when a channel decays
-// that fast, and keeps the gate loop's code small.
-__device__ __noinline__ void kda_correction_entries(float *cor, const float *stg, int n0, int n1,
+// 256 gate threads each take one row i of one block's A or P terms and one half
+// of its columns s (8 of them), and sum, over the block's staged channels,
+// left_i k_s e^{G_i - G_s} (left = k for A, s < i; q for P, s <= i).  Along the
+// row the factor is a running product, e^{G_i - G_{s-1}} = e^{G_i - G_s} alpha_s,
+// every factor <= 1 (it can only underflow, where the exact term is as small), so
+// a channel costs one exponential per thread.  Inlined, with the channel loop
+// rolled: as a call its code was fetched cold at every chunk, which measured
+// slower.
+__device__ __forceinline__ void kda_correction_entries(float *cor, const float *stg, int n0, int n1,
                                                     int n2, int n3, int p0, int cap, int gtid) {
-    for (int e = gtid; e < 8 * 136; e += 256) {
-        const int blk = e / 272, ap = (e / 136) & 1, tri = e % 136;
-        int i = (int)((sqrtf(8.f * (float)tri + 1.f) - 1.f) * 0.5f);
-        if ((i + 1) * (i + 2) / 2 <= tri) ++i;
-        if (i * (i + 1) / 2 > tri) --i;
-        const int s2 = tri - i * (i + 1) / 2;
-        float accv = p0 == 0 ? 0.f : cor[e];
-        if (ap == 1 || s2 < i) {
-            const int nb = blk == 0 ? n0 : blk == 1 ? n1 : blk == 2 ? n2 : n3;
-            const int np = min(cap, nb - p0);
-            const float *d = stg + blk * cap * 48;
-            // four channels at a time, four partial sums: the loads and exponentials
-            // of one group overlap instead of chaining through one accumulator
-            float a4[4] = {0.f, 0.f, 0.f, 0.f};
-            int pp = 0;
-            for (; pp + 4 <= np; pp += 4) {
+    const int blk = gtid >> 6, ap = (gtid >> 5) & 1, i = (gtid >> 1) & 15, hf = gtid & 1;
+    const int s0 = 8 * hf, top = s0 + 7;
+    if (s0 > i) return;  // the row's terms all lie left of this half
+    const int nb = blk == 0 ? n0 : blk == 1 ? n1 : blk == 2 ? n2 : n3;
+    const int np = min(cap, nb - p0);
+    float *ct = cor + (2 * blk + ap) * 136 + i * (i + 1) / 2;  // row i: entries s = 0 .. i
+    float acc[8];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float *dq = d + (pp + q) * 48;
-                    const float ex = dq[32 + i] - dq[32 + s2];
-                    const float w = ex > -88.f ? __expf(ex) : 0.f;
-                    a4[q] = fmaf(dq[16 * ap + i] * dq[s2], w, a4[q]);
-                }
-            }
-            for (; pp < np; ++pp) {
-                const float *dq = d + pp * 48;
-                const float ex = dq[32 + i] - dq[32 + s2];
-                if (ex > -88.f) a4[0] = fmaf(dq[16 * ap + i] * dq[s2], __expf(ex), a4[0]);
-            }
-            accv += (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    for (int j = 0; j < 8; ++j) acc[j] = (p0 > 0 && s0 + j <= i) ? ct[s0 + j] : 0.f;
+    const float *d = stg + blk * cap * KSTG_REC;
+#pragma unroll 1
+    for (int pp = 0; pp < np; ++pp) {
+        const float *dq = d + pp * KSTG_REC;
+        const float li = dq[16 * ap + i], gi = dq[32 + i];
+        float k8[8], a8[8];
+        *reinterpret_cast<float4 *>(k8) = *reinterpret_cast<const float4 *>(dq + s0);
+        *reinterpret_cast<float4 *>(k8 + 4) = *reinterpret_cast<const float4 *>(dq + s0 + 4);
+        *reinterpret_cast<float4 *>(a8) = *reinterpret_cast<const float4 *>(dq + 48 + s0);
+        *reinterpret_cast<float4 *>(a8 + 4) = *reinterpret_cast<const float4 *>(dq + 48 + s0 + 4);
+        // e^{G_i - G_top} when the row reaches past this half (exponent <= 0)
+        float w = i > top ? __expf(gi - dq[32 + top]) : 0.f;
+#pragma unroll
+        for (int j = 7; j >= 0; --j) {
+            if (s0 + j == i) w = 1.f;
+            const float wt = (s0 + j == i && ap == 0) ? 0.f : w;  // A: no diagonal term
+            acc[j] = fmaf(li * k8[j], wt, acc[j]);
+            w *= a8[j];
         }
-        cor[e] = accv;
     }
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        if (s0 + j <= i) ct[s0 + j] = acc[j];
 }
 
 // FG2-GDN: K <- sqrt(beta) . K in place for one gate thread's 16 rows (block rq)
@@ -728,15 +731,18 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                         for (int hc = 0; hc < 2; ++hc) {
                             const int my = hc ? my1 : my0;
                             if (my < p0 || my >= p0 + KSTG_CAP) continue;
-                            float *d = stg + (rq * KSTG_CAP + (my - p0)) * 48;
+                            float *d = stg + (rq * KSTG_CAP + (my - p0)) * KSTG_REC;
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 const uint32_t o = sw128(16 * rq + i, cc >> 3) + cof;
                                 const uint32_t kw = *reinterpret_cast<const uint32_t *>(rawp + ac * L_RAW_AC + o);
                                 const uint32_t qw = *reinterpret_cast<const uint32_t *>(rawp + ac * L_RAW_AC + 8192 + o);
+                                const float gi = hc ? gl1[i] : gl0[i];
                                 d[i] = hc ? __uint_as_float(kw & 0xffff0000u) : __uint_as_float(kw << 16);
                                 d[16 + i] = hc ? __uint_as_float(qw & 0xffff0000u) : __uint_as_float(qw << 16);
-                                d[32 + i] = hc ? gl1[i] : gl0[i];
+                                d[32 + i] = gi;
+                                // alpha_i = e^{G_i - G_{i-1}} (alpha_0 is never read)
+                                d[48 + i] = i == 0 ? 1.f : __expf(gi - (hc ? gl1[i - 1] : gl0[i - 1]));
                             }
                         }
                         named_bar_sync(BAR_G, 256);
