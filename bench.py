@@ -696,7 +696,8 @@ def run_ours(args, rank, world, local):
                               wd.decay == "channel")
         roof_dec = roofline(decode_flops(wd.B, wd.H, wd.d, wd.d), dbytes, dec_s, pk, pk_kind,
                             traffic_for("decode_kernel",
-                                        "gated_delta_rule_140_b200/csrc/gdn_decode.cu"),
+                                        "gated_delta_rule_140_b200/csrc/gdn_decode.cu",
+                                        args.decode_workload),
                             "decode_kernel")
         dominant = roof_pre if pre_s >= dec_s else roof_dec
         hl = legs.get(args.workload)
