@@ -153,6 +153,7 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
                          const float *initial_state, const int32_t *cu_seqlens,
                          void *o, float *final_state,
                          void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_chunk_fwd");
     return chunk_fwd_impl(dims, q, k, v, log_alpha, beta, nullptr, 0, initial_state, cu_seqlens,
                           o, final_state, workspace, workspace_bytes, stream);
 }
@@ -162,6 +163,7 @@ gdn_status gdn_chunk_fwd_raw(const gdn_dims *dims, const void *q_raw, const void
                              const float *beta_logit, const float *initial_state,
                              const int32_t *cu_seqlens, void *o, float *final_state,
                              void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_chunk_fwd_raw");
     if (!dims) return GDN_ERR_INVALID;
     if (dims->decay != GDN_DECAY_SCALAR || (dims->flags & ~GDN_FLAG_POOL) != 0)
         return dims->decay == GDN_DECAY_CHANNEL ? GDN_ERR_UNSUPPORTED : GDN_ERR_INVALID;
@@ -175,6 +177,7 @@ gdn_status gdn_chunk_fwd_raw(const gdn_dims *dims, const void *q_raw, const void
 gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k, const void *v,
                               const float *log_alpha, const float *beta,
                               float *state_inout, void *o, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_recurrent_step");
     gdn_status st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     const gdn_dims &d = *dims;
@@ -201,6 +204,7 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
 gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta, float *state_inout,
                                 const int32_t *n_commit, void *o, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_recurrent_verify");
     gdn_status st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     const gdn_dims &d = *dims;

@@ -5,11 +5,21 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "gdn.h"
 
 namespace gdn {
+
+// A named NVTX range over one C-ABI call (host side; a few instructions unless a
+// profiler is attached), so that timelines show which entry point issued a launch.
+struct ApiRange {
+    explicit ApiRange(const char *name) { nvtxRangePushA(name); }
+    ~ApiRange() { nvtxRangePop(); }
+    ApiRange(const ApiRange &) = delete;
+    ApiRange &operator=(const ApiRange &) = delete;
+};
 
 constexpr int kChunk = 64;  // chunk size C of the chunkwise form
 

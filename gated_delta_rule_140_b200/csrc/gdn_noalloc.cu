@@ -38,6 +38,7 @@ extern "C" gdn_status gdn_chunk_fwd_noalloc(const gdn_dims *dims, const void *q,
                                             const float *beta, const float *initial_state,
                                             const int32_t *cu_seqlens, void *o,
                                             float *final_state, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_chunk_fwd_noalloc");
     size_t need = gdn_chunk_fwd_workspace_size(dims);
     if (need == 0) return GDN_ERR_INVALID;
     gdn_dims d = *dims;

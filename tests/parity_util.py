@@ -4,6 +4,9 @@ Error measure (the stated tolerance): max |gpu - oracle| divided by the max
 |oracle| of the same tensor.  Bounds: 2e-2 on o and 1e-2 on the final state
 for bf16 inputs with fp32 accumulation; 1e-4 on both for fp32 inputs.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -19,6 +22,18 @@ def rel_err(gpu, ref) -> float:
     assert np.all(np.isfinite(g)), "non-finite values in the GPU result"
     scale = np.abs(r).max()
     return float(np.abs(g - r).max() / (scale if scale > 0 else 1.0))
+
+
+def record_margin(case: str, err_o: float, tol_o: float, err_s: float, tol_s: float) -> None:
+    """Append one case's achieved worst errors and its bounds as a JSON line to the
+    file named by GDN_PARITY_MARGINS (nothing is written when it is unset), so that
+    a run can report how much of each tolerance a configuration uses."""
+    path = os.environ.get("GDN_PARITY_MARGINS")
+    if not path:
+        return
+    with open(path, "a") as f:
+        f.write(json.dumps({"case": case, "o_err": err_o, "o_tol": tol_o, "state_err": err_s,
+                            "state_tol": tol_s}) + "\n")
 
 
 def to_dev(x: dict, device="cuda") -> dict:

@@ -15,7 +15,7 @@ from gated_delta_rule_140_b200 import _native as nat
 from gated_delta_rule_140_b200 import chunk_fwd, recurrent_step
 from gated_delta_rule_140_b200.inputs import (WORKLOADS, decode_inputs, prefill_inputs,
                                               workload_inputs)
-from tests.parity_util import TOL, gpu_head, oracle_heads, rel_err, to_dev
+from tests.parity_util import TOL, gpu_head, oracle_heads, record_margin, rel_err, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -383,11 +383,14 @@ def test_full_workload_sampled(cuda_ok, name, kernel):
     o, sf = _run(x, pool=kernel == "pool", check=True)
     assert torch.isfinite(o).all() and torch.isfinite(sf).all()
     to, ts = TOL[WORKLOADS[name].dtype]
+    worst_o = worst_s = 0.0
     for n, h, ro, rs in oracle_heads(x, FULL[name]):
         go, gs = gpu_head(x, o, sf, n, h)
         eo, es = rel_err(go, ro), rel_err(gs, rs)
+        worst_o, worst_s = max(worst_o, eo), max(worst_s, es)
         assert eo <= to, f"{name} (n={n}, h={h}) o error {eo:.3g}"
         assert es <= ts, f"{name} (n={n}, h={h}) final-state error {es:.3g}"
+    record_margin(f"{name} [{kernel}]", worst_o, to, worst_s, ts)
 
 
 # --------------------------------------------------------------------------- #
@@ -468,14 +471,18 @@ def _decode_check(x, picks, dtype):
     torch.cuda.synchronize()
     o = torch.stack(outs)  # [S,N,H,dv]
     to, ts = TOL[dtype]
+    worst_o = worst_s = 0.0
     for n, h in picks:
         # the oracle sees the same tokens as one sequence of `steps` tokens
         seq = lambda t: t[:, n:n + 1, h:h + 1].transpose(0, 1)  # [1,S,1,...]
         ro, rs = oracle.recurrent(seq(x["q"]), seq(x["k"]), seq(x["v"]),
                                   seq(x["log_alpha"]), seq(x["beta"]),
                                   x["state"][n:n + 1, h:h + 1])
-        assert rel_err(o[:, n, h], ro[0, :, 0]) <= to
-        assert rel_err(state[n, h], rs[0, 0]) <= ts
+        eo, es = rel_err(o[:, n, h], ro[0, :, 0]), rel_err(state[n, h], rs[0, 0])
+        worst_o, worst_s = max(worst_o, eo), max(worst_s, es)
+        assert eo <= to
+        assert es <= ts
+    return worst_o, worst_s
 
 
 @pytest.mark.parametrize("decay", ["scalar", "channel"])
@@ -490,7 +497,9 @@ def test_decode_reduced(cuda_ok, decay, d, dtype):
 def test_decode_full_workload_sampled(cuda_ok):
     """N=256, H=32, d=128, fp32 state in place, 64 steps."""
     x = workload_inputs("gdn_decode")
-    _decode_check(x, [(0, 0), (255, 31), (100, 17)], torch.bfloat16)
+    eo, es = _decode_check(x, [(0, 0), (255, 31), (100, 17)], torch.bfloat16)
+    record_margin("gdn_decode [decode, 64 steps]", eo, TOL[torch.bfloat16][0], es,
+                  TOL[torch.bfloat16][1])
 
 
 def test_decode_matches_prefill(cuda_ok):
