@@ -401,7 +401,7 @@ template <bool CH>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  uint8_t *ring, int ring_slots) {
+                  uint8_t *ring, int ring_slots, const int32_t *order) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
@@ -413,9 +413,11 @@ chunk_pair_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap tm_q,
 
     const uint32_t rank = cluster_rank(), peer = rank ^ 1u;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // cluster i takes (sequence, head) item i; a packed batch's sequences are taken
+    // longest first (order), so that the last clusters to start are short ones
     const int item = blockIdx.x >> 1;
     const int h = item % a.H;
-    const int n = item / a.H;
+    const int n = order ? order[item / a.H] : item / a.H;
     const int H = a.H;
     long long t_begin, t_end;
     seq_range(a, n, &t_begin, &t_end);
@@ -1511,6 +1513,28 @@ int ring_slots_for_device() {
 
 size_t ring_bytes(int slots) { return (size_t)slots * NRING * RING_STRIDE; }
 
+// Longest-first order of a packed batch's sequences (by chunk count; ties by
+// index), for list scheduling of the clusters: thread i ranks sequence i among
+// all of them from a shared-memory copy of the chunk counts.
+constexpr int kOrderMax = 4096;  // larger batches keep the index order
+__global__ void __launch_bounds__(1024) pair_order_kernel(const int32_t *cu, int n, int32_t *order) {
+    __shared__ int nck[kOrderMax];
+    for (int i = threadIdx.x; i < n; i += blockDim.x) nck[i] = (cu[i + 1] - cu[i] + C - 1) / C;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int ki = nck[i];
+        int r = 0;
+        for (int j = 0; j < n; ++j) {
+            const int kj = nck[j];
+            r += (kj > ki) | ((kj == ki) & (j < i));
+        }
+        order[r] = i;
+    }
+}
+
+bool use_order(const PrefillArgs &a) { return a.cu_seqlens && a.n_seqs > 1 && a.n_seqs <= kOrderMax; }
+size_t order_bytes(int n_seqs) { return ((size_t)n_seqs * sizeof(int32_t) + 255) & ~(size_t)255; }
+
 template <bool CH>
 cudaError_t launch_t(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk,
                      const CUtensorMap &mv, int slots, cudaStream_t s) {
@@ -1518,8 +1542,9 @@ cudaError_t launch_t(const PrefillArgs &a, const CUtensorMap &mq, const CUtensor
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const long long items = (long long)a.n_seqs * a.H;
-    kern<<<(unsigned)(2 * items), kThreads, SMEM_BYTES, s>>>(
-        a, mq, mk, mv, reinterpret_cast<uint8_t *>(a.scratch), slots);
+    uint8_t *ring = reinterpret_cast<uint8_t *>(a.scratch);
+    const int32_t *order = use_order(a) ? reinterpret_cast<const int32_t *>(ring + ring_bytes(slots)) : nullptr;
+    kern<<<(unsigned)(2 * items), kThreads, SMEM_BYTES, s>>>(a, mq, mk, mv, ring, slots, order);
     return cudaGetLastError();
 }
 
@@ -1529,7 +1554,10 @@ bool chunk_pair_supported(const gdn_dims &d) {
     return d.dtype == GDN_BF16 && d.d_k == DK && d.d_v == DV && (long long)d.B * d.T < (1LL << 31);
 }
 
-size_t chunk_pair_scratch_bytes(const gdn_dims &) { return ring_bytes(ring_slots_for_device()); }
+size_t chunk_pair_scratch_bytes(const gdn_dims &d) {
+    // the ring, then (packed batches) the sequences' longest-first order
+    return ring_bytes(ring_slots_for_device()) + (d.n_seqs > 1 ? order_bytes(d.n_seqs) : 0);
+}
 
 cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launches) {
     const long long items = (long long)a.n_seqs * a.H;
@@ -1549,6 +1577,14 @@ cudaError_t launch_chunk_pair(const PrefillArgs &a, cudaStream_t s, int *launche
         return cudaErrorInvalidValue;
     const int slots = ring_slots_for_device();
     if (slots <= 0) return cudaErrorInvalidValue;
+    if (use_order(a)) {
+        pair_order_kernel<<<1, 1024, 0, s>>>(
+            a.cu_seqlens, a.n_seqs,
+            reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(a.scratch) + ring_bytes(slots)));
+        const cudaError_t eo = cudaGetLastError();
+        if (eo != cudaSuccess) return eo;
+        if (launches) ++*launches;
+    }
     cudaError_t e = a.channel ? launch_t<true>(a, mq, mk, mv, slots, s)
                               : launch_t<false>(a, mq, mk, mv, slots, s);
     if (e != cudaSuccess) return e;

@@ -113,8 +113,10 @@ typedef struct {
  * (gdn_workspace_init).  The
  * two-CTA tensor-core kernel adds a ring of four 64 KiB slots for each SM index
  * of the device (2 x its SM count), through which the chunk-local SM hands each
- * chunk's matrices to the state SM; it is written before it is read and needs
- * no initialisation.  The pool kernel adds eight 73 KiB ring slots per chain
+ * chunk's matrices to the state SM, and (packed batches of up to 4096
+ * sequences) the sequences' longest-first order, 4 bytes each, which a small
+ * kernel before it writes; both are written before they are read and need no
+ * initialisation.  The pool kernel adds eight 73 KiB ring slots per chain
  * CTA, its hand-off flags and (packed batches) a table of round offsets, which
  * a small kernel before it writes.  The other kernels need only the header.  Returns 0 for
  * invalid dims. */
