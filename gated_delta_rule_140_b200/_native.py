@@ -58,6 +58,10 @@ def lib():
     L.gdn_recurrent_step.restype = ctypes.c_int
     L.gdn_recurrent_verify.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, vp]
     L.gdn_recurrent_verify.restype = ctypes.c_int
+    L.gdn_state_compose.argtypes = [D, fp, fp, fp, fp, vp]
+    L.gdn_state_compose.restype = ctypes.c_int
+    L.gdn_state_identity.argtypes = [D, fp, vp]
+    L.gdn_state_identity.restype = ctypes.c_int
     L.gdn_chunk_fwd_raw.argtypes = [D, vp, vp, vp, fp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
     L.gdn_chunk_fwd_raw.restype = ctypes.c_int
     L.gdn_noalloc_status.argtypes = [vp]
@@ -313,6 +317,43 @@ def recurrent_verify(q, k, v, log_alpha, beta, state, n_commit=None, *, outputs=
         except RuntimeError as e:
             raise GdnError(GDN_ERR_CUDA, f"gdn_recurrent_verify (device): {e}") from e
     return o
+
+
+def _state_dims(N, H, dk, dv):
+    return Dims(N, 0, H, dk, dv, N, GDN_FP32, GDN_DECAY_SCALAR, 0)
+
+
+def state_compose(s, m, b=None, *, out=None, stream=None):
+    """out = s m (+ b) per (sequence, head) through gdn_state_compose: s, b
+    [N,H,dv,dk] and m [N,H,dk,dk] fp32 on the device.  Composes segment state
+    maps (S_start M + B); ``out`` may be ``b``, not ``s`` or ``m``."""
+    import torch
+    for name, t in (("s", s), ("m", m), ("b", b), ("out", out)):
+        _check_dev(name, t, torch.float32)
+    N, H, dv, dk = s.shape
+    if tuple(m.shape) != (N, H, dk, dk) or (b is not None and tuple(b.shape) != tuple(s.shape)):
+        raise ValueError("state_compose: s [N,H,dv,dk], m [N,H,dk,dk], b like s")
+    if out is None:
+        out = torch.empty_like(s)
+    st = lib().gdn_state_compose(ctypes.byref(_state_dims(N, H, dk, dv)), _ptr(s), _ptr(m),
+                                 _ptr(b), _ptr(out), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_state_compose")
+    return out
+
+
+def state_identity(N, H, d, device, *, out=None, stream=None):
+    """An identity state per (sequence, head), fp32 [N,H,d,d] (gdn_state_identity):
+    the initial state from which a prefill with v = 0 returns a segment's
+    transition matrix."""
+    import torch
+    if out is None:
+        out = torch.empty(N, H, d, d, dtype=torch.float32, device=device)
+    _check_dev("out", out, torch.float32)
+    st = lib().gdn_state_identity(ctypes.byref(_state_dims(N, H, d, d)), _ptr(out), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_state_identity")
+    return out
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, *, o=None, check=False, stream=None):

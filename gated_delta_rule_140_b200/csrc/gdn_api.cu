@@ -228,6 +228,38 @@ gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void 
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+gdn_status gdn_state_compose(const gdn_dims *dims, const float *s, const float *m, const float *b,
+                             float *out, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_state_compose");
+    if (!dims || dims->B < 0 || dims->H <= 0) return GDN_ERR_INVALID;
+    const int dk = dims->d_k, dv = dims->d_v;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GDN_ERR_UNSUPPORTED;
+    if (dims->B == 0) return GDN_OK;
+    if (!s || !m || !out) return GDN_ERR_INVALID;
+    for (const void *p : {(const void *)s, (const void *)m, (const void *)out})
+        if (!aligned16(p)) return GDN_ERR_INVALID;
+    if (b && !aligned16(b)) return GDN_ERR_INVALID;
+    if (out == s || out == m) return GDN_ERR_INVALID;
+    int launches = 0;
+    cudaError_t e = gdn::launch_state_compose(s, m, b, out, (long long)dims->B * dims->H, dv, dk,
+                                              reinterpret_cast<cudaStream_t>(stream), &launches);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_state_identity(const gdn_dims *dims, float *out, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_state_identity");
+    if (!dims || dims->B < 0 || dims->H <= 0) return GDN_ERR_INVALID;
+    if (dims->d_k != dims->d_v || (dims->d_k != 64 && dims->d_k != 128)) return GDN_ERR_UNSUPPORTED;
+    if (dims->B == 0) return GDN_OK;
+    if (!out || !aligned16(out)) return GDN_ERR_INVALID;
+    int launches = 0;
+    cudaError_t e = gdn::launch_state_identity(out, (long long)dims->B * dims->H, dims->d_k,
+                                               reinterpret_cast<cudaStream_t>(stream), &launches);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
 gdn_status gdn_workspace_init(void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
     if (!workspace || workspace_bytes < gdn::kWorkspaceHeader || !aligned16(workspace))
         return GDN_ERR_INVALID;

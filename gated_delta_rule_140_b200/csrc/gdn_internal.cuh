@@ -90,6 +90,10 @@ bool chunk_pool_supported(const gdn_dims &d);
 bool chunk_pool_preferred(const gdn_dims &d);
 size_t chunk_tc_scratch_bytes(const gdn_dims &d);
 size_t chunk_pair_scratch_bytes(const gdn_dims &d);
+// state maps of sequence segments (gdn_state.cu): out = s m (+ b), out = I
+cudaError_t launch_state_compose(const float *s, const float *m, const float *b, float *out,
+                                 long long nh, int dv, int dk, cudaStream_t st, int *launches);
+cudaError_t launch_state_identity(float *out, long long nh, int d, cudaStream_t st, int *launches);
 // bf16 d_k = d_v = 128 shapes (either decay) the two-CTA kernel takes
 bool chunk_pair_supported(const gdn_dims &d);
 // bf16 d_k = d_v = 128 scalar-decay shapes the tensor-core kernels take

@@ -203,6 +203,25 @@ gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void 
                                 const float *log_alpha, const float *beta, float *state_inout,
                                 const int32_t *n_commit, void *o, gdn_stream_t stream);
 
+/* Segment state maps, for sharding one long sequence over GPUs (the exchange of
+ * per-segment affine maps).  Over a segment the recurrence is affine in the state
+ * it starts from (FG2-GDN section 1: S_t = S_{t-1} A_t + beta_t v_t k_t^T with
+ * A_t = Diag(alpha_t)(I - beta_t k_t k_t^T)):
+ *   S_end = S_start M + B,   M = A_1 ... A_n,   B = S_end when S_start = 0.
+ * B is gdn_chunk_fwd's final state from a null initial state; M is its final
+ * state from the identity (gdn_state_identity) with v = 0.  Consecutive segments
+ * compose: S_start(r + 1) = S_start(r) M_r + B_r, after which each segment is
+ * rerun from its true start.
+ *
+ * gdn_state_compose: out = s m + b for every (sequence, head), fp32:
+ *   s, b, out [N,H,d_v,d_k]; m [N,H,d_k,d_k]; N = dims->B, H = dims->H.
+ *   b may be null (out = s m).  out may alias b, not s or m.  d_v and d_k are
+ *   64 or 128; all pointers 16-byte aligned device memory.
+ * gdn_state_identity: out [N,H,d_k,d_k] = I (requires d_v == d_k). */
+gdn_status gdn_state_compose(const gdn_dims *dims, const float *s, const float *m, const float *b,
+                             float *out, gdn_stream_t stream);
+gdn_status gdn_state_identity(const gdn_dims *dims, float *out, gdn_stream_t stream);
+
 /* Size of the device array that gdn_chunk_fwd_noalloc uses in place of a
  * caller workspace: 256 KiB, held by every GPU that loads the library until
  * the process exits. */

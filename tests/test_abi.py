@@ -204,6 +204,26 @@ def test_empty_batch_is_a_noop_without_device(L):
     assert L.gdn_recurrent_step(ctypes.byref(d), *([None] * 8)) == nat.GDN_OK
 
 
+def test_state_maps_reject_bad_arguments(L):
+    f = ctypes.c_void_p(FAKE)
+    d = _dims(dtype=nat.GDN_FP32)
+    # null operands, an output that aliases s or m, misalignment, unsupported sizes
+    assert L.gdn_state_compose(ctypes.byref(d), None, f, None, f, None) == nat.GDN_ERR_INVALID
+    assert L.gdn_state_compose(ctypes.byref(d), f, f, None, f, None) == nat.GDN_ERR_INVALID
+    odd = ctypes.c_void_p(FAKE + 4)
+    assert L.gdn_state_compose(ctypes.byref(d), f, ctypes.c_void_p(FAKE + 4096), None, odd,
+                               None) == nat.GDN_ERR_INVALID
+    assert L.gdn_state_compose(ctypes.byref(_dims(d_k=96)), f, f, None, f, None) == \
+        nat.GDN_ERR_UNSUPPORTED
+    assert L.gdn_state_compose(None, f, f, None, f, None) == nat.GDN_ERR_INVALID
+    assert L.gdn_state_identity(ctypes.byref(_dims(d_v=64)), f, None) == nat.GDN_ERR_UNSUPPORTED
+    assert L.gdn_state_identity(ctypes.byref(d), None, None) == nat.GDN_ERR_INVALID
+    # no sequences: nothing to launch, succeeds without a device
+    d0 = _dims(B=0, n_seqs=0)
+    assert L.gdn_state_compose(ctypes.byref(d0), None, None, None, None, None) == nat.GDN_OK
+    assert L.gdn_state_identity(ctypes.byref(d0), None, None) == nat.GDN_OK
+
+
 def test_workspace_init_rejects_bad_arguments(L):
     assert L.gdn_workspace_init(None, 256, None) == nat.GDN_ERR_INVALID
     assert L.gdn_workspace_init(ctypes.c_void_p(FAKE), 16, None) == nat.GDN_ERR_INVALID
