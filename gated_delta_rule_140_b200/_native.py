@@ -21,6 +21,7 @@ GDN_BF16, GDN_FP32 = 0, 1
 GDN_DECAY_SCALAR, GDN_DECAY_CHANNEL = 0, 1
 GDN_FLAG_CUDA_CORES, GDN_FLAG_PAIR, GDN_FLAG_ONE_CTA, GDN_FLAG_POOL = 1, 2, 4, 8
 GDN_FLAG_BETA_CHANNEL = 16
+GDN_FLAG_VALUE_RATE = 32
 
 
 class GdnError(RuntimeError):
@@ -52,6 +53,8 @@ def lib():
     L.gdn_chunk_fwd_workspace_size.restype = sz
     L.gdn_chunk_fwd.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
     L.gdn_chunk_fwd.restype = ctypes.c_int
+    L.gdn_chunk_fwd_value_rate.argtypes = [D, vp, vp, vp, fp, fp, fp, fp, vp, vp, fp, vp, sz, vp]
+    L.gdn_chunk_fwd_value_rate.restype = ctypes.c_int
     L.gdn_chunk_fwd_noalloc.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, fp, vp]
     L.gdn_chunk_fwd_noalloc.restype = ctypes.c_int
     L.gdn_recurrent_step.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp]
@@ -126,7 +129,7 @@ def _check_dev(name, t, dtype=None):
 
 
 def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False, pair=False,
-                 one_cta=False, pool=False, beta_channel=False) -> Dims:
+                 one_cta=False, pool=False, beta_channel=False, value_rate=False) -> Dims:
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     return Dims(B, T, H, dk, dv, (len(cu_seqlens) - 1) if cu_seqlens is not None else B,
@@ -134,7 +137,8 @@ def prefill_dims(q, v, log_alpha, cu_seqlens=None, cuda_cores=False, pair=False,
                 GDN_DECAY_CHANNEL if log_alpha.dim() == 4 else GDN_DECAY_SCALAR,
                 (GDN_FLAG_CUDA_CORES if cuda_cores else 0) | (GDN_FLAG_PAIR if pair else 0)
                 | (GDN_FLAG_ONE_CTA if one_cta else 0) | (GDN_FLAG_POOL if pool else 0)
-                | (GDN_FLAG_BETA_CHANNEL if beta_channel else 0))
+                | (GDN_FLAG_BETA_CHANNEL if beta_channel else 0)
+                | (GDN_FLAG_VALUE_RATE if value_rate else 0))
 
 
 def chunk_fwd_path(dims: Dims) -> str:
@@ -205,10 +209,12 @@ def _workspace_for(device, stream) -> Workspace:
 def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
               output_final_state=True, o=None, final_state=None, workspace: Workspace = None,
               cuda_cores=False, pair=False, one_cta=False, pool=False, check=False,
-              stream=None):
+              stream=None, beta_v=None):
     """Chunkwise prefill (gdn_chunk_fwd).  Returns (o, final_state or None).
     A ``beta`` of shape [B,T,H,d_k] (with channel decay) is FG2-GDN's writing rate
     per key channel (GDN_FLAG_BETA_CHANNEL); [B,T,H] is the usual scalar rate.
+    ``beta_v`` [B,T,H,d_v] adds FG2-GDN+'s value-side rate (with a per-channel
+    ``beta``; gdn_chunk_fwd_value_rate).
     ``cuda_cores`` / ``pool`` / ``pair`` / ``one_cta`` select the fp32
     CUDA-core kernel or one of the tensor-core kernels instead of the default
     (GDN_FLAG_*).  With ``check`` the call synchronises the stream afterwards
@@ -222,9 +228,10 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
     _check_dev("beta", beta, torch.float32)
     _check_dev("initial_state", initial_state, torch.float32)
     _check_dev("cu_seqlens", cu_seqlens, torch.int32)
+    _check_dev("beta_v", beta_v, torch.float32)
     beta_channel = beta is not None and beta.dim() == 4
     dims = prefill_dims(q, v, log_alpha, cu_seqlens, cuda_cores, pair, one_cta, pool,
-                        beta_channel)
+                        beta_channel, beta_v is not None)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     if final_state is None and output_final_state:
@@ -233,12 +240,19 @@ def chunk_fwd(q, k, v, log_alpha, beta, initial_state=None, cu_seqlens=None, *,
     ws = workspace if workspace is not None else _workspace_for(q.device, stream)
     nbytes = workspace_size(dims)
     buf = ws.get(nbytes, stream)
-    st = lib().gdn_chunk_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
-                             _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(o),
-                             _ptr(final_state), _ptr(buf), ctypes.c_size_t(buf.numel()),
-                             _stream(stream))
+    if beta_v is not None:
+        st = lib().gdn_chunk_fwd_value_rate(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(log_alpha), _ptr(beta), _ptr(beta_v),
+                                            _ptr(initial_state), _ptr(cu_seqlens), _ptr(o),
+                                            _ptr(final_state), _ptr(buf),
+                                            ctypes.c_size_t(buf.numel()), _stream(stream))
+    else:
+        st = lib().gdn_chunk_fwd(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                 _ptr(beta), _ptr(initial_state), _ptr(cu_seqlens), _ptr(o),
+                                 _ptr(final_state), _ptr(buf), ctypes.c_size_t(buf.numel()),
+                                 _stream(stream))
     if st != GDN_OK:
-        raise GdnError(st, "gdn_chunk_fwd")
+        raise GdnError(st, "gdn_chunk_fwd_value_rate" if beta_v is not None else "gdn_chunk_fwd")
     if check:
         _raise_on_status(ws.status(stream), "gdn_chunk_fwd (device)")
     return o, final_state

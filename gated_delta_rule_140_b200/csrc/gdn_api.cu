@@ -22,7 +22,10 @@ gdn_status check_dims(const gdn_dims *d, bool prefill) {
     if ((d->d_k != 64 && d->d_k != 128) || (d->d_v != 64 && d->d_v != 128))
         return GDN_ERR_UNSUPPORTED;
     if ((d->flags & ~(GDN_FLAG_CUDA_CORES | GDN_FLAG_PAIR | GDN_FLAG_ONE_CTA | GDN_FLAG_POOL |
-                      GDN_FLAG_BETA_CHANNEL)) != 0)
+                      GDN_FLAG_BETA_CHANNEL | GDN_FLAG_VALUE_RATE)) != 0)
+        return GDN_ERR_INVALID;
+    // FG2-GDN+: the value-side rate comes with the key-side one
+    if ((d->flags & GDN_FLAG_VALUE_RATE) && !(d->flags & GDN_FLAG_BETA_CHANNEL))
         return GDN_ERR_INVALID;
     if (d->flags & GDN_FLAG_BETA_CHANNEL) {
         // FG2-GDN: a writing rate per key channel rides on KDA's decay, prefill only,
@@ -68,6 +71,22 @@ Path select_path(const gdn_dims &d) {
     return (long long)d.B * d.T >= kPairMinMeanTokens * seqs ? Path::kPair : Path::kOneCta;
 }
 
+// the selected prefill kernel's scratch after the header (256-byte multiple)
+size_t kernel_scratch_bytes(const gdn_dims &d) {
+    const Path p = select_path(d);
+    const size_t extra = p == Path::kPool     ? gdn::chunk_pool_scratch_bytes(d)
+                         : p == Path::kPair   ? gdn::chunk_pair_scratch_bytes(d)
+                         : p == Path::kOneCta ? gdn::chunk_tc_scratch_bytes(d)
+                                              : 0;
+    return (extra + 255) & ~size_t(255);
+}
+
+// FG2-GDN+: v~ (bf16, the layout of v) after the kernel scratch
+size_t value_rate_bytes(const gdn_dims &d) {
+    if (!(d.flags & GDN_FLAG_VALUE_RATE)) return 0;
+    return ((size_t)d.B * d.T * d.H * d.d_v * 2 + 255) & ~size_t(255);
+}
+
 int prefill_seqs(const gdn_dims &d, const int32_t *cu_seqlens) {
     return cu_seqlens ? d.n_seqs : d.B;
 }
@@ -78,12 +97,7 @@ extern "C" {
 
 size_t gdn_chunk_fwd_workspace_size(const gdn_dims *dims) {
     if (check_dims(dims, true) != GDN_OK) return 0;
-    const Path p = select_path(*dims);
-    size_t extra = p == Path::kPool     ? gdn::chunk_pool_scratch_bytes(*dims)
-                   : p == Path::kPair   ? gdn::chunk_pair_scratch_bytes(*dims)
-                   : p == Path::kOneCta ? gdn::chunk_tc_scratch_bytes(*dims)
-                                        : 0;
-    return gdn::kWorkspaceHeader + ((extra + 255) & ~size_t(255));
+    return gdn::kWorkspaceHeader + kernel_scratch_bytes(*dims) + value_rate_bytes(*dims);
 }
 
 }  // extern "C"
@@ -154,7 +168,33 @@ gdn_status gdn_chunk_fwd(const gdn_dims *dims, const void *q, const void *k, con
                          void *o, float *final_state,
                          void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
     gdn::ApiRange range("gdn_chunk_fwd");
+    if (dims && (dims->flags & GDN_FLAG_VALUE_RATE)) return GDN_ERR_INVALID;
     return chunk_fwd_impl(dims, q, k, v, log_alpha, beta, nullptr, 0, initial_state, cu_seqlens,
+                          o, final_state, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_chunk_fwd_value_rate(const gdn_dims *dims, const void *q, const void *k,
+                                    const void *v, const float *log_alpha, const float *beta,
+                                    const float *beta_v, const float *initial_state,
+                                    const int32_t *cu_seqlens, void *o, float *final_state,
+                                    void *workspace, size_t workspace_bytes, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_chunk_fwd_value_rate");
+    if (!dims) return GDN_ERR_INVALID;
+    const int both = GDN_FLAG_BETA_CHANNEL | GDN_FLAG_VALUE_RATE;
+    if ((dims->flags & both) != both) return GDN_ERR_INVALID;
+    gdn_status st = check_dims(dims, true);
+    if (st != GDN_OK) return st;
+    const long long n = (long long)dims->B * dims->T * dims->H * dims->d_v;
+    if (n > 0 && (!v || !beta_v || !aligned16(v) || !aligned16(beta_v))) return GDN_ERR_INVALID;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < gdn_chunk_fwd_workspace_size(dims))
+        return GDN_ERR_INVALID;
+    void *vt = reinterpret_cast<char *>(workspace) + gdn::kWorkspaceHeader + kernel_scratch_bytes(*dims);
+    int launches = 0;
+    cudaError_t e = gdn::launch_value_rate(v, beta_v, vt, n, reinterpret_cast<cudaStream_t>(stream),
+                                           &launches);
+    g_launches.fetch_add(launches, std::memory_order_relaxed);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    return chunk_fwd_impl(dims, q, k, vt, log_alpha, beta, nullptr, 0, initial_state, cu_seqlens,
                           o, final_state, workspace, workspace_bytes, stream);
 }
 

@@ -94,6 +94,9 @@ size_t chunk_pair_scratch_bytes(const gdn_dims &d);
 cudaError_t launch_state_compose(const float *s, const float *m, const float *b, float *out,
                                  long long nh, int dv, int dk, cudaStream_t st, int *launches);
 cudaError_t launch_state_identity(float *out, long long nh, int d, cudaStream_t st, int *launches);
+// FG2-GDN+ (gdn_state.cu): out = sqrt(beta_v) . v, bf16, n elements (a multiple of 8)
+cudaError_t launch_value_rate(const void *v, const float *beta_v, void *out, long long n,
+                              cudaStream_t st, int *launches);
 // bf16 d_k = d_v = 128 shapes (either decay) the two-CTA kernel takes
 bool chunk_pair_supported(const gdn_dims &d);
 // bf16 d_k = d_v = 128 scalar-decay shapes the tensor-core kernels take

@@ -11,6 +11,8 @@
 // maps.  This file holds the two small kernels of that exchange:
 //   compose:  out = s m + b   per (sequence, head), fp32, d_v x d_k times d_k x d_k;
 //   identity: out = I         per (sequence, head) (d_v = d_k).
+// It also holds FG2-GDN+'s value scaling, v~ = sqrt(beta^v) . v (section 3.4 of
+// the FG2-GDN page), written once before the prefill reads v~ in place of v.
 #include <algorithm>
 
 #include "gdn_internal.cuh"
@@ -59,6 +61,26 @@ compose_kernel(const float *s, const float *m, const float *b, float *out, int d
     }
 }
 
+// FG2-GDN+'s scaled values, 8 elements per step: 16 bytes of v, 32 of rates.
+__global__ void value_rate_kernel(const uint4 *v, const float4 *bv, uint4 *out, long long n8) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n8;
+         i += (long long)gridDim.x * blockDim.x) {
+        const uint4 x = v[i];
+        const float4 b0 = bv[2 * i], b1 = bv[2 * i + 1];
+        const float r[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t y[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float lo = __uint_as_float(w[j] << 16) * sqrtf(r[2 * j]);
+            const float hi = __uint_as_float(w[j] & 0xffff0000u) * sqrtf(r[2 * j + 1]);
+            __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+            y[j] = *reinterpret_cast<uint32_t *>(&t);
+        }
+        out[i] = make_uint4(y[0], y[1], y[2], y[3]);
+    }
+}
+
 __global__ void identity_kernel(float *out, int d, long long total) {
     for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
          i += (long long)gridDim.x * blockDim.x) {
@@ -75,6 +97,19 @@ cudaError_t launch_state_compose(const float *s, const float *m, const float *b,
     const long long blocks = nh * (dk / kTile) * (dv / kTile);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
     compose_kernel<<<(unsigned)blocks, dim3(kTile, 8), 0, st>>>(s, m, b, out, dv, dk);
+    if (launches) ++*launches;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_value_rate(const void *v, const float *beta_v, void *out, long long n,
+                              cudaStream_t st, int *launches) {
+    if (n == 0) return cudaSuccess;
+    if (n % 8) return cudaErrorInvalidValue;
+    const long long n8 = n / 8;
+    const long long blocks = std::min<long long>((n8 + 255) / 256, 148LL * 32);
+    value_rate_kernel<<<(unsigned)blocks, 256, 0, st>>>(reinterpret_cast<const uint4 *>(v),
+                                                         reinterpret_cast<const float4 *>(beta_v),
+                                                         reinterpret_cast<uint4 *>(out), n8);
     if (launches) ++*launches;
     return cudaGetLastError();
 }

@@ -78,7 +78,7 @@ typedef enum { GDN_DECAY_SCALAR = 0, GDN_DECAY_CHANNEL = 1 } gdn_decay;
  * GDN_FLAG_CUDA_CORES forces the fp32 CUDA-core kernel.  The tests use the flags
  * to compare the device paths. */
 enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4, GDN_FLAG_POOL = 8,
-       GDN_FLAG_BETA_CHANNEL = 16 };
+       GDN_FLAG_BETA_CHANNEL = 16, GDN_FLAG_VALUE_RATE = 32 };
 /* GDN_FLAG_BETA_CHANNEL (prefill, channel decay): FG2-GDN's writing rate per key
  * channel (FG2-GDN paper, section 3.2 "FG2-GDN Update Rule" and 3.6 "Chunkwise
  * Parallel Training").  beta is then [B, T, H, d_k] fp32 (per-channel rates in
@@ -88,7 +88,11 @@ enum { GDN_FLAG_CUDA_CORES = 1, GDN_FLAG_PAIR = 2, GDN_FLAG_ONE_CTA = 4, GDN_FLA
  * two-CTA kernel (bf16, d_k = d_v = 128): GDN_ERR_UNSUPPORTED for every other
  * shape, with GDN_FLAG_CUDA_CORES, for gdn_recurrent_step and on the
  * no-allocation entry point; GDN_ERR_INVALID with scalar decay,
- * GDN_FLAG_ONE_CTA or GDN_FLAG_POOL. */
+ * GDN_FLAG_ONE_CTA or GDN_FLAG_POOL.
+ * GDN_FLAG_VALUE_RATE (with GDN_FLAG_BETA_CHANNEL): FG2-GDN+'s value-side rate
+ * (section 3.4 "FG2-GDN+ Variant"), v~_t = sqrt(beta^v_t) . v_t in place of v_t
+ * in the update above; the call is gdn_chunk_fwd_value_rate, whose workspace
+ * (gdn_chunk_fwd_workspace_size with this flag) also holds v~. */
 
 typedef struct {
     int32_t B;       /* batch (1 for a packed batch)                           */
@@ -202,6 +206,17 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
 gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta, float *state_inout,
                                 const int32_t *n_commit, void *o, gdn_stream_t stream);
+
+/* FG2-GDN+ prefill: gdn_chunk_fwd with dims->flags holding GDN_FLAG_BETA_CHANNEL
+ * and GDN_FLAG_VALUE_RATE, and the value-side rate beta_v [B,T,H,d_v] fp32 (16-byte
+ * aligned), rates in (0, 1].  A small kernel first writes v~ = sqrt(beta_v) . v
+ * (bf16) into the workspace; the prefill then runs on (k~, v~) with unit rate.
+ * Without both flags: GDN_ERR_INVALID; gdn_chunk_fwd refuses GDN_FLAG_VALUE_RATE. */
+gdn_status gdn_chunk_fwd_value_rate(const gdn_dims *dims, const void *q, const void *k,
+                                    const void *v, const float *log_alpha, const float *beta,
+                                    const float *beta_v, const float *initial_state,
+                                    const int32_t *cu_seqlens, void *o, float *final_state,
+                                    void *workspace, size_t workspace_bytes, gdn_stream_t stream);
 
 /* Segment state maps, for sharding one long sequence over GPUs (the exchange of
  * per-segment affine maps).  Over a segment the recurrence is affine in the state

@@ -204,6 +204,27 @@ def test_empty_batch_is_a_noop_without_device(L):
     assert L.gdn_recurrent_step(ctypes.byref(d), *([None] * 8)) == nat.GDN_OK
 
 
+def test_value_rate_flags_and_workspace(L):
+    f = ctypes.c_void_p(FAKE)
+    fg2 = dict(decay=nat.GDN_DECAY_CHANNEL, flags=nat.GDN_FLAG_BETA_CHANNEL)
+    both = dict(decay=nat.GDN_DECAY_CHANNEL,
+                flags=nat.GDN_FLAG_BETA_CHANNEL | nat.GDN_FLAG_VALUE_RATE)
+    # the value rate needs the key-side rate; gdn_chunk_fwd refuses it
+    assert L.gdn_chunk_fwd_workspace_size(ctypes.byref(_dims(flags=nat.GDN_FLAG_VALUE_RATE))) == 0
+    n_fg2 = L.gdn_chunk_fwd_workspace_size(ctypes.byref(_dims(**fg2)))
+    n_both = L.gdn_chunk_fwd_workspace_size(ctypes.byref(_dims(**both)))
+    assert n_both - n_fg2 == 2 * 128 * 4 * 128 * 2  # v~: B T H d_v bf16
+    d = _dims(**both)
+    assert _call_fwd(L, d) == nat.GDN_ERR_INVALID
+    args = [f, f, f, f, f]  # q k v log_alpha beta
+    assert L.gdn_chunk_fwd_value_rate(ctypes.byref(_dims(**fg2)), *args, f, None, None, f, None, f,
+                                      n_both, None) == nat.GDN_ERR_INVALID
+    assert L.gdn_chunk_fwd_value_rate(ctypes.byref(d), *args, None, None, None, f, None, f,
+                                      n_both, None) == nat.GDN_ERR_INVALID
+    assert L.gdn_chunk_fwd_value_rate(ctypes.byref(d), *args, f, None, None, f, None, f,
+                                      n_fg2, None) == nat.GDN_ERR_INVALID
+
+
 def test_state_maps_reject_bad_arguments(L):
     f = ctypes.c_void_p(FAKE)
     d = _dims(dtype=nat.GDN_FP32)

@@ -263,6 +263,39 @@ def test_fg2_rate_per_key_channel_matches_oracle(cuda_ok, case):
     _fg2_compare(x, o, sf)
 
 
+@pytest.mark.parametrize("case", ["ragged", "packed"])
+def test_fg2plus_value_rate_matches_oracle(cuda_ok, case):
+    """FG2-GDN+: a value-side rate beta_v [B,T,H,d_v] with FG2-GDN's key-side one;
+    v is scaled by sqrt(beta_v) into the workspace (gdn_chunk_fwd_value_rate) and
+    the FG2-GDN prefill runs on it.  Against the oracle's FG2 recurrence with the
+    value gate; rates of exactly 1 leave the FG2-GDN result unchanged."""
+    g = torch.Generator().manual_seed(84)
+    if case == "packed":
+        x = prefill_inputs(1, 0, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                           alpha_shift=3.0, init_std=0.05, lengths=[0, 70, 200, 1, 129],
+                           gen=g, beta_channel=True)
+    else:
+        x = prefill_inputs(2, 229, 2, 128, 128, dtype=torch.bfloat16, decay="channel",
+                           alpha_shift=3.0, init_std=0.05, gen=g, beta_channel=True)
+    bv = torch.sigmoid(torch.randn(x["v"].shape, generator=g) + 1.0)
+    d = to_dev(x)
+    o, sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                      d["cu_seqlens"], beta_v=bv.cuda(), check=True)
+    torch.cuda.synchronize()
+    ro, rs = oracle.fg2_recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], bv,
+                                  x["initial_state"], x["cu_seqlens"])
+    to, ts = TOL[torch.bfloat16]
+    eo, es = rel_err(o, ro), rel_err(sf, rs)
+    assert eo <= to and es <= ts, (eo, es)
+    # unit value rates: FG2-GDN bit for bit (sqrt(1) = 1, the same bf16 values)
+    o1, s1 = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                       d["cu_seqlens"], beta_v=torch.ones_like(bv).cuda(), check=True)
+    o0, s0 = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["initial_state"],
+                       d["cu_seqlens"], check=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o0) and torch.equal(s1, s0)
+
+
 def test_kda_log_alpha_4_byte_aligned_gives_identical_results(cuda_ok):
     """The ABI asks 4-byte alignment of log alpha; the KDA gate pass loads channel
     pairs as float2 when the pointer allows and one float at a time otherwise.
