@@ -61,6 +61,8 @@ def lib():
     L.gdn_recurrent_step.restype = ctypes.c_int
     L.gdn_recurrent_verify.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, vp]
     L.gdn_recurrent_verify.restype = ctypes.c_int
+    L.gdn_recurrent_verify_tree.argtypes = [D, vp, vp, vp, fp, fp, fp, vp, vp, vp, vp]
+    L.gdn_recurrent_verify_tree.restype = ctypes.c_int
     L.gdn_state_compose.argtypes = [D, fp, fp, fp, fp, vp]
     L.gdn_state_compose.restype = ctypes.c_int
     L.gdn_state_identity.argtypes = [D, fp, vp]
@@ -297,13 +299,16 @@ def chunk_fwd_raw(q_raw, k_raw, v, alpha_logit, beta_logit, alpha_bias=None,
 
 
 def recurrent_verify(q, k, v, log_alpha, beta, state, n_commit=None, *, outputs=True, o=None,
-                     check=False, stream=None):
+                     check=False, stream=None, parent=None):
     """Multi-token verification (gdn_recurrent_verify): K draft tokens per sequence
     from ``state`` [N,H,dv,dk] fp32.  q, k [N,K,H,dk]; v [N,K,H,dv]; log_alpha
     [N,K,H] or [N,K,H,dk]; beta [N,K,H]; ``n_commit`` int32 [N] on the device or
     None.  Returns o [N,K,H,dv] (None with ``outputs=False``); the state becomes
     the state after the first n_commit[n] tokens of each sequence (untouched for
-    None or 0)."""
+    None or 0).  With ``parent`` int32 [N,K] on the device the drafts form a tree
+    (gdn_recurrent_verify_tree): node j follows node parent[n][j] (-1: the state),
+    its output is read after the path to it, and n_commit[n] = c commits the state
+    after node c - 1's path."""
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_dev(name, t, q.dtype)
@@ -311,6 +316,7 @@ def recurrent_verify(q, k, v, log_alpha, beta, state, n_commit=None, *, outputs=
     _check_dev("beta", beta, torch.float32)
     _check_dev("state", state, torch.float32)
     _check_dev("n_commit", n_commit, torch.int32)
+    _check_dev("parent", parent, torch.int32)
     N, K, H, dk = q.shape
     dv = v.shape[-1]
     dims = Dims(N, K, H, dk, dv, N, _dtype_code(q.dtype),
@@ -319,11 +325,18 @@ def recurrent_verify(q, k, v, log_alpha, beta, state, n_commit=None, *, outputs=
         o = torch.empty(N, K, H, dv, dtype=q.dtype, device=q.device)
     if not outputs:
         o = None
-    st = lib().gdn_recurrent_verify(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
-                                    _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(n_commit),
-                                    _ptr(o), _stream(stream))
+    if parent is not None:
+        st = lib().gdn_recurrent_verify_tree(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(log_alpha), _ptr(beta), _ptr(state),
+                                             _ptr(parent), _ptr(n_commit), _ptr(o),
+                                             _stream(stream))
+    else:
+        st = lib().gdn_recurrent_verify(ctypes.byref(dims), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(log_alpha), _ptr(beta), _ptr(state), _ptr(n_commit),
+                                        _ptr(o), _stream(stream))
     if st != GDN_OK:
-        raise GdnError(st, "gdn_recurrent_verify")
+        raise GdnError(st, "gdn_recurrent_verify_tree" if parent is not None else
+                       "gdn_recurrent_verify")
     if check:
         s = stream if stream is not None else torch.cuda.current_stream()
         try:

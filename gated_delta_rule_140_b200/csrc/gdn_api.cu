@@ -241,10 +241,39 @@ gdn_status gdn_recurrent_step(const gdn_dims *dims, const void *q, const void *k
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
+namespace {
+gdn_status verify_impl(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta, float *state_inout,
+                       const int32_t *parent, const int32_t *n_commit, void *o,
+                       gdn_stream_t stream);
+}  // namespace
+
 gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void *k, const void *v,
                                 const float *log_alpha, const float *beta, float *state_inout,
                                 const int32_t *n_commit, void *o, gdn_stream_t stream) {
     gdn::ApiRange range("gdn_recurrent_verify");
+    return verify_impl(dims, q, k, v, log_alpha, beta, state_inout, nullptr, n_commit, o, stream);
+}
+
+gdn_status gdn_recurrent_verify_tree(const gdn_dims *dims, const void *q, const void *k,
+                                     const void *v, const float *log_alpha, const float *beta,
+                                     float *state_inout, const int32_t *parent,
+                                     const int32_t *n_commit, void *o, gdn_stream_t stream) {
+    gdn::ApiRange range("gdn_recurrent_verify_tree");
+    if (!dims) return GDN_ERR_INVALID;
+    if (dims->T > gdn::kMaxTreeNodes) return GDN_ERR_UNSUPPORTED;
+    if ((long long)dims->B * dims->T > 0 && (!parent || (reinterpret_cast<uintptr_t>(parent) & 3u)))
+        return GDN_ERR_INVALID;
+    return verify_impl(dims, q, k, v, log_alpha, beta, state_inout, parent, n_commit, o, stream);
+}
+
+}  // extern "C"
+
+namespace {
+gdn_status verify_impl(const gdn_dims *dims, const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta, float *state_inout,
+                       const int32_t *parent, const int32_t *n_commit, void *o,
+                       gdn_stream_t stream) {
     gdn_status st = check_dims(dims, false);
     if (st != GDN_OK) return st;
     const gdn_dims &d = *dims;
@@ -258,7 +287,7 @@ gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void 
         return GDN_ERR_INVALID;
     gdn::VerifyArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
-    a.state = state_inout; a.n_commit = n_commit; a.o = o;
+    a.state = state_inout; a.n_commit = n_commit; a.o = o; a.parent = parent;
     a.N = d.B; a.K = d.T; a.H = d.H; a.dk = d.d_k; a.dv = d.d_v;
     a.channel = d.decay == GDN_DECAY_CHANNEL;
     a.bf16 = d.dtype == GDN_BF16;
@@ -267,6 +296,9 @@ gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void 
     g_launches.fetch_add(launches, std::memory_order_relaxed);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
+}  // namespace
+
+extern "C" {
 
 gdn_status gdn_state_compose(const gdn_dims *dims, const float *s, const float *m, const float *b,
                              float *out, gdn_stream_t stream) {

@@ -67,11 +67,14 @@ struct DecodeArgs {
 };
 
 // Multi-token verification: K draft tokens per sequence, token-major [N, K, H].
+constexpr int kMaxTreeNodes = 64;  // tree-shaped drafts per sequence (gdn_recurrent_verify_tree)
+
 struct VerifyArgs {
     const void *q, *k, *v;
     const float *log_alpha, *beta;
     float *state;
     const int32_t *n_commit;  // device [N] or null (no commit)
+    const int32_t *parent;    // device [N, K] (tree-shaped drafts) or null (a chain)
     void *o;                  // [N, K, H, dv] or null (no outputs)
     int N, K, H, dk, dv;
     int channel, bf16;

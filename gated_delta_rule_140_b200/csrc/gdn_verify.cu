@@ -55,6 +55,59 @@ __device__ __forceinline__ void load_vec(const void *p, long long i, int bf16, f
     }
 }
 
+// One token of the recurrence on kRows state rows of this warp (rows i0 ..),
+// lane's columns; writes the outputs of the rows when o is not null.
+template <int DK, bool CH>
+__device__ __forceinline__ void token_step(const VerifyArgs &a, long long tok, int i0, int lane,
+                                           float (&s)[kRows][DK / 32], bool out) {
+    constexpr int VEC = DK / 32;
+    const int dv = a.dv;
+    float kk[VEC], qq[VEC], al[VEC];
+    load_vec(a.k, tok * DK + lane * VEC, a.bf16, kk, VEC);
+    load_vec(a.q, tok * DK + lane * VEC, a.bf16, qq, VEC);
+    const float beta = a.beta[tok];
+    if (CH) {
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) al[j] = expf(a.log_alpha[tok * DK + lane * VEC + j]);
+    } else {
+        const float alpha = expf(a.log_alpha[tok]);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) al[j] = alpha;
+    }
+    float kq = 0.f;
+#pragma unroll
+    for (int j = 0; j < VEC; ++j) kq += kk[j] * qq[j];
+    float r[kRows], o[kRows];
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+        r[u] = 0.f; o[u] = 0.f;
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) {
+            s[u][j] *= al[j];  // S~ = S Diag(alpha)
+            r[u] += s[u][j] * kk[j];
+            o[u] += s[u][j] * qq[j];
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        kq += __shfl_xor_sync(0xffffffffu, kq, off);
+#pragma unroll
+        for (int u = 0; u < kRows; ++u) {
+            r[u] += __shfl_xor_sync(0xffffffffu, r[u], off);
+            o[u] += __shfl_xor_sync(0xffffffffu, o[u], off);
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kRows; ++u) {
+        const int i = i0 + u;
+        const float vi = load_elem(a.v, tok * dv + i, a.bf16);
+        const float delta = beta * (vi - r[u]);
+#pragma unroll
+        for (int j = 0; j < VEC; ++j) s[u][j] += delta * kk[j];
+        if (out && lane == 0) store_elem(a.o, tok * dv + i, o[u] + delta * kq, a.bf16);
+    }
+}
+
 template <int DK, bool CH>
 __global__ void __launch_bounds__(kWarps * 32)
 verify_kernel(VerifyArgs a) {
@@ -82,50 +135,7 @@ verify_kernel(VerifyArgs a) {
         }
         for (int t = 0; t < steps; ++t) {
             const long long tok = ((long long)n * K + t) * a.H + h;  // token-major [N, K, H]
-            float kk[VEC], qq[VEC], al[VEC];
-            load_vec(a.k, tok * DK + lane * VEC, a.bf16, kk, VEC);
-            load_vec(a.q, tok * DK + lane * VEC, a.bf16, qq, VEC);
-            const float beta = a.beta[tok];
-            if (CH) {
-#pragma unroll
-                for (int j = 0; j < VEC; ++j) al[j] = expf(a.log_alpha[tok * DK + lane * VEC + j]);
-            } else {
-                const float alpha = expf(a.log_alpha[tok]);
-#pragma unroll
-                for (int j = 0; j < VEC; ++j) al[j] = alpha;
-            }
-            float kq = 0.f;
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) kq += kk[j] * qq[j];
-            float r[kRows], o[kRows];
-#pragma unroll
-            for (int u = 0; u < kRows; ++u) {
-                r[u] = 0.f; o[u] = 0.f;
-#pragma unroll
-                for (int j = 0; j < VEC; ++j) {
-                    s[u][j] *= al[j];  // S~ = S Diag(alpha)
-                    r[u] += s[u][j] * kk[j];
-                    o[u] += s[u][j] * qq[j];
-                }
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                kq += __shfl_xor_sync(0xffffffffu, kq, off);
-#pragma unroll
-                for (int u = 0; u < kRows; ++u) {
-                    r[u] += __shfl_xor_sync(0xffffffffu, r[u], off);
-                    o[u] += __shfl_xor_sync(0xffffffffu, o[u], off);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kRows; ++u) {
-                const int i = i0 + u;
-                const float vi = load_elem(a.v, tok * dv + i, a.bf16);
-                const float delta = beta * (vi - r[u]);
-#pragma unroll
-                for (int j = 0; j < VEC; ++j) s[u][j] += delta * kk[j];
-                if (a.o && lane == 0) store_elem(a.o, tok * dv + i, o[u] + delta * kq, a.bf16);
-            }
+            token_step<DK, CH>(a, tok, i0, lane, s, a.o != nullptr);
             if (t + 1 == commit) {
 #pragma unroll
                 for (int u = 0; u < kRows; ++u) {
@@ -140,11 +150,97 @@ verify_kernel(VerifyArgs a) {
     }
 }
 
+// Tree-shaped drafts: node j's token follows its parent's (parent[n][j] in
+// [-1, j - 1]; -1: the current state; anything else is taken as -1).  Node j's
+// output is S_j q_j, S_j the state after the path from the current state to j;
+// n_commit[n] = c >= 1 commits the state after node c - 1's path.  Each node's
+// root-first path is tabulated in shared memory; a warp keeps the current state
+// of its rows in registers and walks a node's path from it, except that a node
+// whose parent is the node just done continues from that state (a chain of
+// drafts costs one step per node).
+constexpr int kMaxTree = kMaxTreeNodes;
+
+template <int DK, bool CH>
+__global__ void __launch_bounds__(kWarps * 32)
+verify_tree_kernel(VerifyArgs a) {
+    constexpr int VEC = DK / 32;
+    using V = typename VecF<VEC>::T;
+    __shared__ int anc[kMaxTree][kMaxTree];
+    __shared__ int depth[kMaxTree];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nh = blockIdx.x;  // n * H + h
+    const int n = nh / a.H, h = nh % a.H;
+    const int dv = a.dv, K = a.K;
+    const int commit = a.n_commit ? min(max(a.n_commit[n], 0), K) : 0;
+    if (!a.o && commit == 0) return;
+    const int32_t *par = a.parent + (size_t)n * K;
+    auto parent_of = [&](int x) {
+        const int p = par[x];
+        return (p >= 0 && p < x) ? p : -1;
+    };
+    for (int j = threadIdx.x; j < K; j += blockDim.x) {
+        int d = 0;
+        for (int x = j; x >= 0; x = parent_of(x)) ++d;
+        depth[j] = d;
+        int i = d - 1;
+        for (int x = j; x >= 0; x = parent_of(x)) anc[j][i--] = x;
+    }
+    __syncthreads();
+
+    float *state = a.state + (size_t)nh * dv * DK;
+    auto tok_of = [&](int x) { return ((long long)n * K + x) * a.H + h; };
+    for (int i0 = warp * kRows; i0 < dv; i0 += kWarps * kRows) {
+        float s0[kRows][VEC], s[kRows][VEC];
+#pragma unroll
+        for (int u = 0; u < kRows; ++u) {
+            const V x = *reinterpret_cast<const V *>(state + (size_t)(i0 + u) * DK + lane * VEC);
+            const float *xf = reinterpret_cast<const float *>(&x);
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) s0[u][j] = s[u][j] = xf[j];
+        }
+        int cur = -1;  // the node whose state s holds (-1: the current state)
+        // the state after node x's path, continuing from s when x's parent is cur
+        auto reach = [&](int x, bool out_last) {
+            const int d = depth[x];
+            const int px = d >= 2 ? anc[x][d - 2] : -1;
+            if (px != cur) {
+                // restart from the current state and walk the whole path
+#pragma unroll
+                for (int u = 0; u < kRows; ++u)
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) s[u][j] = s0[u][j];
+                for (int i = 0; i < d; ++i)
+                    token_step<DK, CH>(a, tok_of(anc[x][i]), i0, lane, s, out_last && i == d - 1);
+            } else {
+                token_step<DK, CH>(a, tok_of(x), i0, lane, s, out_last);
+            }
+            cur = x;
+        };
+        if (a.o)
+            for (int j = 0; j < K; ++j) reach(j, true);
+        if (commit > 0) {
+            const int x = commit - 1;
+            if (cur != x) reach(x, false);
+#pragma unroll
+            for (int u = 0; u < kRows; ++u) {
+                V y;
+                float *yf = reinterpret_cast<float *>(&y);
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) yf[j] = s[u][j];
+                *reinterpret_cast<V *>(state + (size_t)(i0 + u) * DK + lane * VEC) = y;
+            }
+        }
+    }
+}
+
 template <int DK, bool CH>
 cudaError_t launch_t(const VerifyArgs &a, cudaStream_t s) {
     const long long blocks = (long long)a.N * a.H;
     if (blocks == 0 || a.K == 0) return cudaSuccess;
-    verify_kernel<DK, CH><<<(unsigned)blocks, kWarps * 32, 0, s>>>(a);
+    if (a.parent)
+        verify_tree_kernel<DK, CH><<<(unsigned)blocks, kWarps * 32, 0, s>>>(a);
+    else
+        verify_kernel<DK, CH><<<(unsigned)blocks, kWarps * 32, 0, s>>>(a);
     return cudaGetLastError();
 }
 

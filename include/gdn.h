@@ -207,6 +207,19 @@ gdn_status gdn_recurrent_verify(const gdn_dims *dims, const void *q, const void 
                                 const float *log_alpha, const float *beta, float *state_inout,
                                 const int32_t *n_commit, void *o, gdn_stream_t stream);
 
+/* Tree-shaped drafts (the TreeWY setting on the Gated DeltaNet-2 page): the K =
+ * dims->T draft tokens of sequence n form a tree through parent [N,K] int32
+ * (device): node j follows node parent[n][j] in [0, j - 1], or the current state
+ * when parent[n][j] = -1 (any other value is taken as -1).  o_j = S_j q_j, S_j the
+ * state after the path from the current state to node j; n_commit[n] = c >= 1
+ * commits the state after node c - 1's path (0 or a null n_commit: untouched), so
+ * a chain (parent[n][j] = j - 1) behaves as gdn_recurrent_verify.  K <= 64
+ * (GDN_ERR_UNSUPPORTED above).  Layouts and the rest as gdn_recurrent_verify. */
+gdn_status gdn_recurrent_verify_tree(const gdn_dims *dims, const void *q, const void *k,
+                                     const void *v, const float *log_alpha, const float *beta,
+                                     float *state_inout, const int32_t *parent,
+                                     const int32_t *n_commit, void *o, gdn_stream_t stream);
+
 /* FG2-GDN+ prefill: gdn_chunk_fwd with dims->flags holding GDN_FLAG_BETA_CHANNEL
  * and GDN_FLAG_VALUE_RATE, and the value-side rate beta_v [B,T,H,d_v] fp32 (16-byte
  * aligned), rates in (0, 1].  A small kernel first writes v~ = sqrt(beta_v) . v

@@ -225,6 +225,20 @@ def test_value_rate_flags_and_workspace(L):
                                       n_fg2, None) == nat.GDN_ERR_INVALID
 
 
+def test_recurrent_verify_tree_rejects_bad_arguments(L):
+    f = ctypes.c_void_p(FAKE)
+    args = [f, f, f, f, f, f]  # q k v log_alpha beta state
+    d = _dims(T=8)
+    assert L.gdn_recurrent_verify_tree(ctypes.byref(d), *args, None, None, f, None) == \
+        nat.GDN_ERR_INVALID  # no parent
+    assert L.gdn_recurrent_verify_tree(ctypes.byref(_dims(T=65)), *args, f, None, f, None) == \
+        nat.GDN_ERR_UNSUPPORTED  # more than 64 nodes
+    assert L.gdn_recurrent_verify_tree(None, *args, f, None, f, None) == nat.GDN_ERR_INVALID
+    # no drafts: nothing to do, succeeds without a device
+    assert L.gdn_recurrent_verify_tree(ctypes.byref(_dims(T=0)), *([None] * 6), None, None, None,
+                                       None) == nat.GDN_OK
+
+
 def test_state_maps_reject_bad_arguments(L):
     f = ctypes.c_void_p(FAKE)
     d = _dims(dtype=nat.GDN_FP32)

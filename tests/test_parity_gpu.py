@@ -475,6 +475,58 @@ def test_recurrent_verify_outputs_and_commit_match_oracle(cuda_ok, decay, dtype,
             assert rel_err(st[n], rs[0]) <= ts, (n, j)
 
 
+@pytest.mark.parametrize("decay,dtype,d", [("scalar", torch.bfloat16, 128),
+                                           ("channel", torch.bfloat16, 128),
+                                           ("scalar", torch.float32, 64)])
+def test_recurrent_verify_tree_matches_oracle_paths(cuda_ok, decay, dtype, d):
+    """Tree-shaped drafts: node j's output equals the oracle's recurrence over the
+    tokens on the path from the state to j; committing node c - 1 leaves the
+    oracle's state after that path.  Sequence 0 is a chain (its outputs equal the
+    chain verification's bit for bit), sequence 1 branches, sequence 2 has
+    out-of-range parents, which count as -1 (children of the state)."""
+    from gated_delta_rule_140_b200 import recurrent_verify
+    N, K, H = 3, 10, 2
+    x = _verify_inputs(N, K, H, d, dtype, decay, 93)
+    dd = to_dev(x)
+    s0 = dd["initial_state"].contiguous()
+    parent = torch.tensor([[-1, 0, 1, 2, 3, 4, 5, 6, 7, 8],
+                           [-1, 0, 0, 1, 1, 2, -1, 6, 7, 3],
+                           [-1, 5, 0, 9, 2, -7, 4, 6, 6, 12]], dtype=torch.int32)
+    commit = torch.tensor([7, 10, 9], dtype=torch.int32)  # nodes 6, 9, 8
+
+    def path(n, j):
+        p = []
+        while j >= 0:
+            p.append(j)
+            q_ = int(parent[n, j])
+            j = q_ if 0 <= q_ < j else -1
+        return p[::-1]
+
+    to, ts = TOL[dtype]
+    st = s0.clone()
+    o = recurrent_verify(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], st,
+                         commit.cuda(), parent=parent.cuda(), check=True)
+    for n in range(N):
+        for j in range(K):
+            pj = path(n, j)
+            sl = lambda t: t[n:n + 1, pj]
+            ro, rs = oracle.recurrent(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["log_alpha"]),
+                                      sl(x["beta"]), x["initial_state"][n:n + 1])
+            assert rel_err(o[n, j], ro[0, -1]) <= to, (n, j)
+            if j == int(commit[n]) - 1:
+                assert rel_err(st[n], rs[0]) <= ts, (n, j)
+    # the chain-shaped sequence: the chain kernel's outputs bit for bit
+    s_chain = s0.clone()
+    o_chain = recurrent_verify(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], s_chain,
+                               check=True)
+    assert torch.equal(o[0], o_chain[0])
+    # a peek leaves the state untouched
+    st2 = s0.clone()
+    recurrent_verify(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], st2,
+                     parent=parent.cuda(), check=True)
+    assert torch.equal(st2, s0)
+
+
 def test_recurrent_verify_commit_all_equals_decode_steps_bitwise(cuda_ok):
     """Committing all K tokens is K decode steps in the same arithmetic order:
     states and outputs are bit-identical to gdn_recurrent_step called K times."""
