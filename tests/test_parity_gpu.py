@@ -527,6 +527,42 @@ def test_recurrent_verify_tree_matches_oracle_paths(cuda_ok, decay, dtype, d):
     assert torch.equal(st2, s0)
 
 
+def test_recurrent_verify_tree_of_64_nodes(cuda_ok):
+    """The largest tree (64 nodes, random parents, bf16 KDA): every node's output and
+    the commit of the deepest node against the oracle's recurrence over its path."""
+    from gated_delta_rule_140_b200 import recurrent_verify
+    N, K, H, d = 2, 64, 2, 128
+    x = _verify_inputs(N, K, H, d, torch.bfloat16, "channel", 95)
+    dd = to_dev(x)
+    g = torch.Generator().manual_seed(96)
+    parent = torch.stack([torch.tensor([-1] + [int(torch.randint(-1, j, (1,), generator=g))
+                                               for j in range(1, K)], dtype=torch.int32)
+                          for _ in range(N)])
+
+    def path(n, j):
+        p = []
+        while j >= 0:
+            p.append(j)
+            j = int(parent[n, j])
+        return p[::-1]
+
+    deepest = [max(range(K), key=lambda j: len(path(n, j))) for n in range(N)]
+    commit = torch.tensor([c + 1 for c in deepest], dtype=torch.int32)
+    st = dd["initial_state"].clone()
+    o = recurrent_verify(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], st,
+                         commit.cuda(), parent=parent.cuda(), check=True)
+    to, ts = TOL[torch.bfloat16]
+    for n in range(N):
+        for j in range(K):
+            pj = path(n, j)
+            sl = lambda t: t[n:n + 1, pj]
+            ro, rs = oracle.recurrent(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["log_alpha"]),
+                                      sl(x["beta"]), x["initial_state"][n:n + 1])
+            assert rel_err(o[n, j], ro[0, -1]) <= to, (n, j)
+            if j == deepest[n]:
+                assert rel_err(st[n], rs[0]) <= ts, n
+
+
 def test_recurrent_verify_commit_all_equals_decode_steps_bitwise(cuda_ok):
     """Committing all K tokens is K decode steps in the same arithmetic order:
     states and outputs are bit-identical to gdn_recurrent_step called K times."""
