@@ -237,7 +237,8 @@ gdn_status gdn_chunk_fwd_value_rate(const gdn_dims *dims, const void *q, const v
  * A_t = Diag(alpha_t)(I - beta_t k_t k_t^T)):
  *   S_end = S_start M + B,   M = A_1 ... A_n,   B = S_end when S_start = 0.
  * B is gdn_chunk_fwd's final state from a null initial state; M is its final
- * state from the identity (gdn_state_identity) with v = 0.  Consecutive segments
+ * state from the identity (gdn_state_identity) with v = 0 of width d_k (every
+ * state row a probe vector, so the state is d_k x d_k).  Consecutive segments
  * compose: S_start(r + 1) = S_start(r) M_r + B_r, after which each segment is
  * rerun from its true start.
  *
