@@ -15,7 +15,7 @@
 // for a chain of drafts).
 //
 // Layout as the decode step's: a warp owns whole state rows, each lane DK/32
-// consecutive columns; kRows rows are in flight per warp and stay in registers
+// consecutive columns; kRows (8) rows are in flight per warp and stay in registers
 // across the K tokens, so the state is read once and written at most once.
 #include "gdn_internal.cuh"
 
@@ -23,7 +23,7 @@ namespace gdn {
 namespace {
 
 constexpr int kWarps = 4;
-constexpr int kRows = 4;
+constexpr int kRows = 8;
 
 template <int VEC>
 struct VecF;
@@ -56,10 +56,17 @@ __device__ __forceinline__ void load_vec(const void *p, long long i, int bf16, f
 }
 
 // One token of the recurrence on kRows state rows of this warp (rows i0 ..),
-// lane's columns; writes the outputs of the rows when o is not null.
+// lane's columns; writes the outputs of the rows when `out`.  The 2 kRows row
+// sums (r_u = S~_u . k, o_u = S~_u . q) are reduced across the warp by a
+// transposed butterfly: at each of the first four levels a lane keeps half of its
+// values and adds its partner's copy of them, so 16 values take 8 + 4 + 2 + 1 + 1
+// shuffles and lane l ends with value 8 b4 + 4 b3 + 2 b2 + b1 (l's bits): r_u in
+// lanes 2u, 2u + 1 and o_u in lanes 16 + 2u, 16 + 2u + 1.  Each r_u then goes to
+// every lane for the update, and lane 16 + 2u writes row u's output.
 template <int DK, bool CH>
 __device__ __forceinline__ void token_step(const VerifyArgs &a, long long tok, int i0, int lane,
                                            float (&s)[kRows][DK / 32], bool out) {
+    static_assert(kRows == 8, "the butterfly below reduces 2 x 8 values");
     constexpr int VEC = DK / 32;
     const int dv = a.dv;
     float kk[VEC], qq[VEC], al[VEC];
@@ -77,34 +84,57 @@ __device__ __forceinline__ void token_step(const VerifyArgs &a, long long tok, i
     float kq = 0.f;
 #pragma unroll
     for (int j = 0; j < VEC; ++j) kq += kk[j] * qq[j];
-    float r[kRows], o[kRows];
+    float p[16];  // r_0 .. r_7, o_0 .. o_7 (this lane's columns)
 #pragma unroll
     for (int u = 0; u < kRows; ++u) {
-        r[u] = 0.f; o[u] = 0.f;
+        p[u] = 0.f; p[8 + u] = 0.f;
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
             s[u][j] *= al[j];  // S~ = S Diag(alpha)
-            r[u] += s[u][j] * kk[j];
-            o[u] += s[u][j] * qq[j];
+            p[u] += s[u][j] * kk[j];
+            p[8 + u] += s[u][j] * qq[j];
         }
     }
+    float p8[8], p4[4], p2[2];
+    const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        kq += __shfl_xor_sync(0xffffffffu, kq, off);
-#pragma unroll
-        for (int u = 0; u < kRows; ++u) {
-            r[u] += __shfl_xor_sync(0xffffffffu, r[u], off);
-            o[u] += __shfl_xor_sync(0xffffffffu, o[u], off);
-        }
+    for (int j = 0; j < 8; ++j) {
+        const float keep = b4 ? p[8 + j] : p[j], give = b4 ? p[j] : p[8 + j];
+        p8[j] = keep + __shfl_xor_sync(0xffffffffu, give, 16);
     }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float keep = b3 ? p8[4 + j] : p8[j], give = b3 ? p8[j] : p8[4 + j];
+        p4[j] = keep + __shfl_xor_sync(0xffffffffu, give, 8);
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float keep = b2 ? p4[2 + j] : p4[j], give = b2 ? p4[j] : p4[2 + j];
+        p2[j] = keep + __shfl_xor_sync(0xffffffffu, give, 4);
+    }
+    float v1;
+    {
+        const float keep = b1 ? p2[1] : p2[0], give = b1 ? p2[0] : p2[1];
+        v1 = keep + __shfl_xor_sync(0xffffffffu, give, 2);
+    }
+    v1 += __shfl_xor_sync(0xffffffffu, v1, 1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    // this lane's output row (lanes 16 + 2u) and its r
+    const int uo = (lane >> 1) & 7;
+    const float r_o = __shfl_sync(0xffffffffu, v1, 2 * uo);
 #pragma unroll
     for (int u = 0; u < kRows; ++u) {
-        const int i = i0 + u;
-        const float vi = load_elem(a.v, tok * dv + i, a.bf16);
-        const float delta = beta * (vi - r[u]);
+        const float r = __shfl_sync(0xffffffffu, v1, 2 * u);
+        const float vi = load_elem(a.v, tok * dv + i0 + u, a.bf16);
+        const float delta = beta * (vi - r);
 #pragma unroll
         for (int j = 0; j < VEC; ++j) s[u][j] += delta * kk[j];
-        if (out && lane == 0) store_elem(a.o, tok * dv + i, o[u] + delta * kq, a.bf16);
+    }
+    if (out && lane >= 16 && !(lane & 1)) {
+        const int i = i0 + uo;
+        const float delta = beta * (load_elem(a.v, tok * dv + i, a.bf16) - r_o);
+        store_elem(a.o, tok * dv + i, v1 + delta * kq, a.bf16);
     }
 }
 
@@ -154,8 +184,8 @@ verify_kernel(VerifyArgs a) {
 // [-1, j - 1]; -1: the current state; anything else is taken as -1).  Node j's
 // output is S_j q_j, S_j the state after the path from the current state to j;
 // n_commit[n] = c >= 1 commits the state after node c - 1's path.  Each node's
-// root-first path is tabulated in shared memory; a warp keeps the current state
-// of its rows in registers and walks a node's path from it, except that a node
+// root-first path is tabulated in shared memory; a warp walks a node's path from
+// the current state of its rows (read from the state buffer), except that a node
 // whose parent is the node just done continues from that state (a chain of
 // drafts costs one step per node).
 constexpr int kMaxTree = kMaxTreeNodes;
@@ -190,44 +220,54 @@ verify_tree_kernel(VerifyArgs a) {
     float *state = a.state + (size_t)nh * dv * DK;
     auto tok_of = [&](int x) { return ((long long)n * K + x) * a.H + h; };
     for (int i0 = warp * kRows; i0 < dv; i0 += kWarps * kRows) {
-        float s0[kRows][VEC], s[kRows][VEC];
-#pragma unroll
-        for (int u = 0; u < kRows; ++u) {
-            const V x = *reinterpret_cast<const V *>(state + (size_t)(i0 + u) * DK + lane * VEC);
-            const float *xf = reinterpret_cast<const float *>(&x);
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) s0[u][j] = s[u][j] = xf[j];
-        }
-        int cur = -1;  // the node whose state s holds (-1: the current state)
-        // the state after node x's path, continuing from s when x's parent is cur
-        auto reach = [&](int x, bool out_last) {
-            const int d = depth[x];
-            const int px = d >= 2 ? anc[x][d - 2] : -1;
-            if (px != cur) {
-                // restart from the current state and walk the whole path
-#pragma unroll
-                for (int u = 0; u < kRows; ++u)
-#pragma unroll
-                    for (int j = 0; j < VEC; ++j) s[u][j] = s0[u][j];
-                for (int i = 0; i < d; ++i)
-                    token_step<DK, CH>(a, tok_of(anc[x][i]), i0, lane, s, out_last && i == d - 1);
+        float s[kRows][VEC];
+        // s holds the state after node `cur`'s path (-2: nothing yet).  Targets: the
+        // K nodes when the outputs are wanted, then the committed node.
+        int cur = -2;
+        for (int it = 0; it <= K; ++it) {
+            int x;
+            bool out_last;
+            if (it < K) {
+                if (!a.o) continue;
+                x = it;
+                out_last = true;
             } else {
-                token_step<DK, CH>(a, tok_of(x), i0, lane, s, out_last);
+                if (commit == 0) break;
+                x = commit - 1;
+                out_last = false;
             }
-            cur = x;
-        };
-        if (a.o)
-            for (int j = 0; j < K; ++j) reach(j, true);
-        if (commit > 0) {
-            const int x = commit - 1;
-            if (cur != x) reach(x, false);
+            if (x != cur) {
+                const int d = depth[x];
+                const int px = d >= 2 ? anc[x][d - 2] : -1;
+                int i = d - 1;  // continue from cur when it is x's parent
+                if (px != cur) {
+                    // restart from the current state of these rows (the state
+                    // buffer: the commit below writes it only after its last read)
 #pragma unroll
-            for (int u = 0; u < kRows; ++u) {
-                V y;
-                float *yf = reinterpret_cast<float *>(&y);
+                    for (int u = 0; u < kRows; ++u) {
+                        const V y = *reinterpret_cast<const V *>(state + (size_t)(i0 + u) * DK + lane * VEC);
+                        const float *yf = reinterpret_cast<const float *>(&y);
 #pragma unroll
-                for (int j = 0; j < VEC; ++j) yf[j] = s[u][j];
-                *reinterpret_cast<V *>(state + (size_t)(i0 + u) * DK + lane * VEC) = y;
+                        for (int j = 0; j < VEC; ++j) s[u][j] = yf[j];
+                    }
+                    i = 0;
+                }
+                for (; i < d; ++i) {
+                    const int t = anc[x][i];
+                    token_step<DK, CH>(a, ((long long)n * K + t) * a.H + h, i0, lane, s,
+                                       out_last && i == d - 1);
+                }
+                cur = x;
+            }
+            if (it == K) {
+#pragma unroll
+                for (int u = 0; u < kRows; ++u) {
+                    V y;
+                    float *yf = reinterpret_cast<float *>(&y);
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) yf[j] = s[u][j];
+                    *reinterpret_cast<V *>(state + (size_t)(i0 + u) * DK + lane * VEC) = y;
+                }
             }
         }
     }

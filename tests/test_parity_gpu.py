@@ -563,9 +563,10 @@ def test_recurrent_verify_tree_of_64_nodes(cuda_ok):
                 assert rel_err(st[n], rs[0]) <= ts, n
 
 
-def test_recurrent_verify_commit_all_equals_decode_steps_bitwise(cuda_ok):
-    """Committing all K tokens is K decode steps in the same arithmetic order:
-    states and outputs are bit-identical to gdn_recurrent_step called K times."""
+def test_recurrent_verify_commit_all_equals_decode_steps(cuda_ok):
+    """Committing all K tokens is K decode steps: the same recurrence in fp32, with
+    the row sums reduced in another order (a transposed butterfly over eight rows
+    against the decode kernel's per-row reduction), so equal to rounding."""
     from gated_delta_rule_140_b200 import recurrent_verify
     N, K, H = 5, 4, 2
     for decay in ("scalar", "channel"):
@@ -578,8 +579,8 @@ def test_recurrent_verify_commit_all_equals_decode_steps_bitwise(cuda_ok):
                                x["v"][:, t].contiguous(), x["log_alpha"][:, t].contiguous(),
                                x["beta"][:, t].contiguous(), st2) for t in range(K)]
         torch.cuda.synchronize()
-        assert torch.equal(st, st2)
-        assert torch.equal(o, torch.stack(outs, 1))
+        assert rel_err(st, st2.double().cpu().numpy()) <= 1e-5
+        assert rel_err(o, torch.stack(outs, 1).double().cpu().numpy()) <= 1e-2 / 4  # bf16 o
 
 def _decode_check(x, picks, dtype):
     steps = x["q"].shape[0]
