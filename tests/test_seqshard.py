@@ -47,11 +47,12 @@ def _seg(x, a, b):
     return {k: x[k][:, a:b] for k in ("q", "k", "v", "log_alpha", "beta")}
 
 
-@pytest.mark.parametrize("decay", ["scalar", "channel"])
-def test_segment_maps_compose_to_the_whole_sequence(decay):
+@pytest.mark.parametrize("decay,bounds", [("scalar", [0, 37, 64, 121, 150]),
+                                          ("channel", [0, 37, 64, 121, 150]),
+                                          ("scalar", [0, 50, 50, 150])])  # an empty segment
+def test_segment_maps_compose_to_the_whole_sequence(decay, bounds):
     x = _problem(decay)
     ro, rs = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
-    bounds = [0, 37, 64, 121, 150]  # four ragged segments
     prefill, compose, identity = _ops()
     maps, outs = [], []
     for r in range(len(bounds) - 1):
@@ -115,7 +116,7 @@ def _worker(rank, world, port, decay, result_dir):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,decay", [(2, "scalar"), (3, "channel")])
+@pytest.mark.parametrize("world,decay", [(1, "scalar"), (2, "scalar"), (3, "channel")])
 def test_sequence_sharded_prefill_on_gloo_ranks(tmp_path, world, decay):
     mp.start_processes(_worker, args=(world, _free_port(), decay, str(tmp_path)), nprocs=world,
                        join=True, start_method="spawn")
