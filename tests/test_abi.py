@@ -265,6 +265,24 @@ def test_workspace_init_rejects_bad_arguments(L):
     assert L.gdn_workspace_status(None, None) == nat.GDN_ERR_INVALID
 
 
+def test_python_api_refuses_host_tensors():
+    """No CPU fallback: every entry of the binding refuses host tensors before any call."""
+    import torch
+    from gated_delta_rule_140_b200 import (chunk_fwd, recurrent_step, recurrent_verify,
+                                           state_compose)
+    q = torch.zeros(1, 4, 2, 64)
+    la, b = torch.zeros(1, 4, 2), torch.zeros(1, 4, 2)
+    for call in (lambda: chunk_fwd(q, q, q, la, b),
+                 lambda: chunk_fwd(q, q, q, la, b, beta_v=torch.zeros(1, 4, 2, 64)),
+                 lambda: recurrent_step(q[:, 0], q[:, 0], q[:, 0], la[:, 0], b[:, 0],
+                                        torch.zeros(1, 2, 64, 64)),
+                 lambda: recurrent_verify(q, q, q, la, b, torch.zeros(1, 2, 64, 64),
+                                          parent=torch.zeros(1, 4, dtype=torch.int32)),
+                 lambda: state_compose(torch.zeros(1, 2, 64, 64), torch.zeros(1, 2, 64, 64))):
+        with pytest.raises(ValueError, match="CUDA tensor"):
+            call()
+
+
 def test_python_api_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(nat, "_lib", None)
     monkeypatch.setattr(nat, "LIB_PATH", str(tmp_path / "missing.so"))
