@@ -15,8 +15,9 @@ runs its segment directly and publishes (M, B) = (0, its final state).  One
 all-gather shares the maps (2 x H x d_k x d_k fp32 per sequence and rank); each
 rank composes its true start S_start(r) = S_start(r - 1) M_{r-1} + B_{r-1} with
 the compose kernel and reruns its segment from it, which gives its outputs and
-its final state.  Ranks >= 1 do three passes over their segment, rank 0 one: a
-caller can give rank 0 the longer segment.
+its final state.  Ranks >= 1 do three passes over their segment, rank 0 one:
+``balanced_bounds`` splits a sequence so that rank 0 takes three times the tokens of
+each other rank, which balances the passes.
 
 Every step runs in libgdn.so's kernels (gdn_chunk_fwd, gdn_state_identity,
 gdn_state_compose); the collective is torch.distributed's all-gather (NCCL over
@@ -24,6 +25,26 @@ NVLink between GPUs).  The ``prefill``, ``compose`` and ``identity`` arguments
 exist so that the exchange can be run on CPU ranks with other implementations of
 the same three operations; their defaults are the library's.
 """
+
+
+def balanced_bounds(T, world, chunk=64):
+    """Token boundaries [0, b_1, ..., T] of ``world`` segments that balance the
+    passes: rank 0 runs its segment once, the others three times (two map passes
+    and the rerun), so rank 0 takes about three times the tokens of each other
+    rank, T / (world + 2) per pass.  Boundaries fall on multiples of ``chunk``
+    where the lengths allow, so that no segment but the last ends in a partial
+    chunk.  With one rank the whole sequence is rank 0's."""
+    if world < 1 or T < 0:
+        raise ValueError("world >= 1 and T >= 0")
+    if world == 1:
+        return [0, T]
+    unit = T / (world + 2)
+    bounds = [0]
+    for r in range(1, world):
+        b = int(round((3 + (r - 1)) * unit / chunk)) * chunk
+        bounds.append(min(max(b, bounds[-1]), T))
+    bounds.append(T)
+    return bounds
 
 
 def _default_ops():

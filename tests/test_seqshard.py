@@ -82,6 +82,22 @@ def test_segment_maps_compose_to_the_whole_sequence(decay, bounds):
     assert not torch.allclose(se, m_map @ s_any + b_map, atol=1e-6)
 
 
+def test_balanced_bounds():
+    # rank 0 takes three shares (one pass), every other rank one share (three passes)
+    b = seqshard.balanced_bounds(65536, 8)
+    assert b[0] == 0 and b[-1] == 65536 and len(b) == 9
+    lens = np.diff(b)
+    assert all(x % 64 == 0 for x in b[:-1])
+    assert abs(lens[0] - 3 * 65536 / 10) <= 64 and all(abs(x - 65536 / 10) <= 128 for x in lens[1:])
+    # per-rank passes x tokens are balanced: max / min close to 1
+    work = [lens[0]] + [3 * x for x in lens[1:]]
+    assert max(work) / min(work) < 1.05
+    assert seqshard.balanced_bounds(100, 1) == [0, 100]
+    assert seqshard.balanced_bounds(0, 3) == [0, 0, 0, 0]
+    small = seqshard.balanced_bounds(130, 3)
+    assert small[0] == 0 and small[-1] == 130 and list(small) == sorted(small)
+
+
 def _free_port():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
